@@ -1,0 +1,410 @@
+"""Checks that tie the CPU oracle to facts other than itself.
+
+Each ``pin_*`` function takes a loaded oracle and raises AssertionError when
+the oracle disagrees with what the pages or the mathematics fix:
+
+* exact widening of fp16/bf16 (NumPy's and PyTorch's own conversions);
+* brute force in 50-digit arithmetic on tiny inputs (mpmath);
+* closed forms: a context of one token returns that token's V row, identical
+  keys return the mean of V, one dominant logit returns its V row, logits
+  near 1000 stay finite, a context of zero returns zeros;
+* the block-mapping examples in tests/golden (logical block 0 -> physical
+  block 7, 5688vip.com section 2.2) whose outputs follow by hand;
+* non-contiguous storage (zingnex.cn section 3.2 item 2): relabelling the
+  physical blocks leaves the output bit-identical, and the paged result equals
+  dense attention over the static [batch, heads, max_len, head_dim] layout of
+  the same page's section 3.1;
+* block sharing (section 3.2 item 3): shared blocks give the same output as
+  private copies;
+* grouped queries equal full multi-head attention with repeated kv heads;
+* the partitioned (split-K) form equals the direct one;
+* append and copy-on-write equal a NumPy scatter/copy over the whole pool.
+
+The pins are plain functions so that tests/test_oracle_mutations.py can run
+them against oracle builds with planted mistakes.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from paged_kv_cache_458_b200 import gen
+import golden_cases
+
+
+def _case(seed, **kw):
+    return gen.random_decode_case(np.random.default_rng(seed), **kw)
+
+
+def _decode(orc, dtype, c, scale=None):
+    return orc.decode(dtype, c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
+                      c["context_lens"], c["scale"] if scale is None else scale)
+
+
+def _widen(bits, dtype):
+    return gen.bits_to_f32(bits, dtype).astype(np.float64)
+
+
+# ---------------------------------------------------------------- conversions
+
+def pin_f16_widening(orc):
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = np.array([orc.f16_to_f64(b) for b in bits.tolist()])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan), "fp16 NaN patterns differ"
+    assert np.array_equal(got[~nan], ref[~nan]), "fp16 widening differs from NumPy"
+
+
+def pin_bf16_widening(orc):
+    import torch
+
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    got = np.array([orc.bf16_to_f64(b) for b in bits.tolist()])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan), "bf16 NaN patterns differ"
+    assert np.array_equal(got[~nan], ref[~nan]), "bf16 widening differs from PyTorch"
+
+
+# ---------------------------------------------------------------- brute force
+
+def _mp_decode(q, kc, vc, bt, cl, scale, dtype):
+    import mpmath
+
+    mpmath.mp.dps = 50
+    S, Hq, D = q.shape
+    NB, bs, Hkv, _ = kc.shape
+    g = Hq // Hkv
+    out = np.zeros((S, Hq, D))
+    qf, kf, vf = _widen(q, dtype), _widen(kc, dtype), _widen(vc, dtype)
+    for s in range(S):
+        for h in range(Hq):
+            L = int(cl[s])
+            if L == 0:
+                continue
+            rows = []
+            for j in range(L):
+                blk = int(bt[s, j // bs])
+                rows.append((blk, j % bs))
+            x = []
+            for blk, off in rows:
+                acc = mpmath.mpf(0)
+                for d in range(D):
+                    acc += mpmath.mpf(qf[s, h, d]) * mpmath.mpf(kf[blk, off, h // g, d])
+                x.append(mpmath.mpf(scale) * acc)
+            m = max(x)
+            p = [mpmath.exp(xi - m) for xi in x]
+            den = mpmath.fsum(p)
+            for d in range(D):
+                num = mpmath.fsum(pi * mpmath.mpf(vf[blk, off, h // g, d])
+                                  for pi, (blk, off) in zip(p, rows))
+                out[s, h, d] = float(num / den)
+    return out
+
+
+def pin_brute_force_tiny(orc):
+    rng = np.random.default_rng(20240458)
+    for trial in range(24):
+        dtype = gen.F16 if trial % 2 == 0 else gen.BF16
+        D = int(rng.integers(1, 5))
+        bs = int(rng.integers(1, 4))
+        Hkv = int(rng.integers(1, 3))
+        g = int(rng.integers(1, 3))
+        S = int(rng.integers(1, 3))
+        ctx = rng.integers(0, 6, size=S)
+        c = gen.random_decode_case(rng, num_seqs=S, num_q_heads=Hkv * g, num_kv_heads=Hkv,
+                                   head_dim=D, block_size=bs, dtype=dtype, context_lens=ctx)
+        scale = float(rng.uniform(0.2, 2.0))
+        got = _decode(orc, dtype, c, scale)
+        ref = _mp_decode(c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
+                         c["context_lens"], scale, dtype)
+        err = np.abs(got - ref) / np.maximum(1.0, np.abs(ref))
+        assert np.all(np.isfinite(got)), f"trial {trial}: non-finite oracle output"
+        assert err.max() <= 1e-14, f"trial {trial}: brute-force mismatch {err.max():.3e}"
+
+
+# ---------------------------------------------------------------- closed forms
+
+def pin_context_one_returns_v0(orc):
+    for dtype in (gen.F16, gen.BF16):
+        c = _case(11, num_seqs=3, num_q_heads=4, num_kv_heads=2, head_dim=64, block_size=16,
+                  dtype=dtype, context_lens=[1, 1, 1])
+        out = _decode(orc, dtype, c)
+        v = _widen(c["v_cache"], dtype)
+        for s in range(3):
+            blk = c["block_tables"][s, 0]
+            for h in range(4):
+                assert np.array_equal(out[s, h], v[blk, 0, h // 2]), "ctx=1 must return V_0"
+
+
+def pin_identical_keys_give_mean_of_v(orc):
+    for dtype in (gen.F16, gen.BF16):
+        c = _case(12, num_seqs=2, num_q_heads=2, num_kv_heads=1, head_dim=32, block_size=16,
+                  dtype=dtype, context_lens=[37, 5])
+        kc = c["k_cache"]
+        key = kc[c["block_tables"][0, 0], 0, 0].copy()
+        for s in range(2):
+            L = int(c["context_lens"][s])
+            for j in range(L):
+                kc[c["block_tables"][s, j // 16], j % 16, 0] = key
+        out = _decode(orc, dtype, c)
+        v = _widen(c["v_cache"], dtype)
+        for s in range(2):
+            L = int(c["context_lens"][s])
+            rows = np.stack([v[c["block_tables"][s, j // 16], j % 16, 0] for j in range(L)])
+            ref = rows.mean(axis=0)
+            for h in range(2):
+                assert np.allclose(out[s, h], ref, rtol=1e-13, atol=1e-13), \
+                    "identical keys must give the mean of V"
+
+
+def pin_dominant_logit_selects_its_row(orc):
+    dtype = gen.F16
+    c = _case(13, num_seqs=1, num_q_heads=1, num_kv_heads=1, head_dim=16, block_size=16,
+              dtype=dtype, context_lens=[23])
+    D = 16
+    q = np.zeros(D, dtype=np.float32)
+    q[3] = 1.0
+    c["q"] = gen.f32_to_f16_bits(q).reshape(1, 1, D)
+    kc = c["k_cache"]
+    rng = np.random.default_rng(5)
+    target = 17
+    for j in range(23):
+        k = rng.uniform(-0.5, 0.5, size=D).astype(np.float32)
+        k[3] = 60.0 if j == target else float(rng.uniform(-1.0, 1.0))
+        kc[c["block_tables"][0, j // 16], j % 16, 0] = gen.f32_to_f16_bits(k)
+    out = _decode(orc, dtype, c, scale=1.0)
+    v = _widen(c["v_cache"], dtype)[c["block_tables"][0, target // 16], target % 16, 0]
+    # every other logit is at least 59 below: total weight elsewhere < 23 e^-59
+    assert np.allclose(out[0, 0], v, rtol=1e-15, atol=1e-20 + 23 * math.exp(-59) * 8), \
+        "a dominant logit must select its own V row"
+
+
+def pin_large_logits_stay_finite(orc):
+    """Softmax is shift invariant; logits near 1000 must not overflow."""
+    D = 8
+    dtype = gen.F16
+    c = _case(14, num_seqs=1, num_q_heads=1, num_kv_heads=1, head_dim=D, block_size=16,
+              dtype=dtype, context_lens=[2])
+    q = np.zeros(D, dtype=np.float32)
+    q[0] = 1.0
+    c["q"] = gen.f32_to_f16_bits(q).reshape(1, 1, D)
+    k0 = np.zeros(D, dtype=np.float32)
+    k0[0] = 1.0
+    k1 = np.zeros(D, dtype=np.float32)
+    k1[0] = 1.0 + 2.0 ** -10
+    blk = c["block_tables"][0, 0]
+    c["k_cache"][blk, 0, 0] = gen.f32_to_f16_bits(k0)
+    c["k_cache"][blk, 1, 0] = gen.f32_to_f16_bits(k1)
+    scale = 1000.0
+    out = _decode(orc, dtype, c, scale=scale)
+    v = _widen(c["v_cache"], dtype)
+    w = math.exp(scale * 2.0 ** -10)
+    ref = (v[blk, 0, 0] + w * v[blk, 1, 0]) / (1.0 + w)
+    assert np.all(np.isfinite(out)), "logits near 1000 overflowed"
+    assert np.allclose(out[0, 0], ref, rtol=1e-13, atol=1e-13)
+
+
+def pin_context_zero_gives_zeros(orc):
+    c = _case(15, num_seqs=3, num_q_heads=2, num_kv_heads=2, head_dim=64, block_size=16,
+              dtype=gen.F16, context_lens=[0, 5, 0])
+    out = _decode(orc, gen.F16, c)
+    assert np.array_equal(out[0], np.zeros_like(out[0])) and np.array_equal(out[2], np.zeros_like(out[2]))
+    assert np.all(np.isfinite(out[1]))
+
+
+def pin_golden_block_mapping(orc):
+    for case in golden_cases.load_cases():
+        c = golden_cases.build(case)
+        out = orc.decode(c["dtype"], c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
+                         c["context_lens"], c["scale"])
+        assert np.allclose(out, c["expected"], rtol=1e-14, atol=1e-14), \
+            f"{case['name']}: oracle differs from the hand-derived output"
+
+
+# ---------------------------------------------------------------- structure
+
+def pin_permutation_invariance(orc):
+    """Relabel physical blocks by a random permutation and move their contents."""
+    for dtype, bs in ((gen.F16, 16), (gen.BF16, 256), (gen.F16, 3)):
+        rng = np.random.default_rng(16 + bs)
+        c = gen.random_decode_case(rng, num_seqs=4, num_q_heads=8, num_kv_heads=2, head_dim=32,
+                                   block_size=bs, dtype=dtype, context_lens=[1, 40, 300, 17])
+        base = _decode(orc, dtype, c)
+        NB = c["num_blocks"]
+        pi = rng.permutation(NB)
+        kc = np.empty_like(c["k_cache"])
+        vc = np.empty_like(c["v_cache"])
+        kc[pi] = c["k_cache"]
+        vc[pi] = c["v_cache"]
+        bt = c["block_tables"].copy()
+        m = bt >= 0
+        bt[m] = pi[bt[m]]
+        perm = orc.decode(dtype, c["q"], kc, vc, bt, c["context_lens"], c["scale"])
+        assert np.array_equal(base, perm), "output changed under a relabelling of physical blocks"
+
+
+def _dense_attention(c, dtype):
+    """Static contiguous layout [S, Hkv, max_len, D] + library softmax."""
+    from scipy.special import softmax
+
+    q = _widen(c["q"], dtype)
+    kc, vc = _widen(c["k_cache"], dtype), _widen(c["v_cache"], dtype)
+    bt, cl = c["block_tables"], c["context_lens"]
+    S, Hq, D = q.shape
+    NB, bs, Hkv, _ = kc.shape
+    g = Hq // Hkv
+    Lmax = int(cl.max())
+    Kd = np.zeros((S, Hkv, Lmax, D))
+    Vd = np.zeros((S, Hkv, Lmax, D))
+    for s in range(S):
+        L = int(cl[s])
+        j = np.arange(L)
+        blocks = bt[s, j // bs]
+        Kd[s, :, :L] = np.transpose(kc[blocks, j % bs], (1, 0, 2))
+        Vd[s, :, :L] = np.transpose(vc[blocks, j % bs], (1, 0, 2))
+    out = np.zeros((S, Hq, D))
+    for s in range(S):
+        L = int(cl[s])
+        if L == 0:
+            continue
+        Kg = np.repeat(Kd[s, :, :L], g, axis=0)          # [Hq, L, D]
+        Vg = np.repeat(Vd[s, :, :L], g, axis=0)
+        logits = c["scale"] * np.einsum("hd,hld->hl", q[s], Kg)
+        p = softmax(logits, axis=-1)
+        out[s] = np.einsum("hl,hld->hd", p, Vg)
+    return out
+
+
+def pin_dense_equality(orc):
+    for dtype, bs, g in ((gen.F16, 16, 1), (gen.BF16, 16, 4), (gen.F16, 256, 8)):
+        rng = np.random.default_rng(17 + g)
+        c = gen.random_decode_case(rng, num_seqs=5, num_q_heads=2 * g, num_kv_heads=2,
+                                   head_dim=64, block_size=bs, dtype=dtype,
+                                   context_lens=[1, 16, 17, 300, 600])
+        got = _decode(orc, dtype, c)
+        ref = _dense_attention(c, dtype)
+        err = np.abs(got - ref) / np.maximum(1e-3, np.abs(ref))
+        assert err.max() <= 1e-12, f"paged vs dense mismatch {err.max():.3e}"
+
+
+def pin_gqa_equals_repeated_mha(orc):
+    dtype = gen.BF16
+    g, Hkv = 4, 2
+    c = _case(18, num_seqs=3, num_q_heads=g * Hkv, num_kv_heads=Hkv, head_dim=32, block_size=16,
+              dtype=dtype, context_lens=[5, 33, 64])
+    gqa = _decode(orc, dtype, c)
+    mha = orc.decode(dtype, c["q"], np.ascontiguousarray(np.repeat(c["k_cache"], g, axis=2)),
+                     np.ascontiguousarray(np.repeat(c["v_cache"], g, axis=2)),
+                     c["block_tables"], c["context_lens"], c["scale"])
+    assert np.array_equal(gqa, mha), "grouped-query output differs from repeated-head MHA"
+    # and the groups are contiguous: q heads 0..g-1 share kv head 0
+    solo = orc.decode(dtype, np.ascontiguousarray(c["q"][:, :g]),
+                      np.ascontiguousarray(c["k_cache"][:, :, :1]),
+                      np.ascontiguousarray(c["v_cache"][:, :, :1]),
+                      c["block_tables"], c["context_lens"], c["scale"])
+    assert np.array_equal(gqa[:, :g], solo), "q heads 0..g-1 must read kv head 0"
+
+
+def pin_sharing_equals_private_copies(orc):
+    dtype = gen.F16
+    rng = np.random.default_rng(19)
+    c = gen.random_decode_case(rng, num_seqs=4, num_q_heads=2, num_kv_heads=2, head_dim=32,
+                               block_size=16, dtype=dtype, context_lens=[40, 50, 33, 64],
+                               shared_prefix_blocks=2)
+    assert len({tuple(c["block_tables"][s, :2]) for s in range(4)}) == 1
+    shared = _decode(orc, dtype, c)
+    # give every sequence private copies of the shared blocks
+    NB = c["num_blocks"]
+    extra = 4 * 2
+    kc = np.concatenate([c["k_cache"], np.zeros((extra,) + c["k_cache"].shape[1:], np.uint16)])
+    vc = np.concatenate([c["v_cache"], np.zeros((extra,) + c["v_cache"].shape[1:], np.uint16)])
+    bt = c["block_tables"].copy()
+    nxt = NB
+    for s in range(4):
+        for i in range(2):
+            src = bt[s, i]
+            kc[nxt] = kc[src]
+            vc[nxt] = vc[src]
+            bt[s, i] = nxt
+            nxt += 1
+    private = orc.decode(dtype, c["q"], kc, vc, bt, c["context_lens"], c["scale"])
+    assert np.array_equal(shared, private), "shared blocks must read like private copies"
+
+
+def pin_split_identity(orc):
+    dtype = gen.BF16
+    rng = np.random.default_rng(20)
+    c = gen.random_decode_case(rng, num_seqs=4, num_q_heads=4, num_kv_heads=2, head_dim=64,
+                               block_size=16, dtype=dtype, context_lens=[1, 511, 513, 1500])
+    direct = _decode(orc, dtype, c)
+    for pt in (1, 7, 16, 512, 4096):
+        part = orc.decode_partitioned(dtype, c["q"], c["k_cache"], c["v_cache"],
+                                      c["block_tables"], c["context_lens"], c["scale"], pt)
+        err = np.abs(part - direct).max()     # outputs are O(1): absolute bound
+        assert err <= 1e-13, f"partition {pt}: split-K merge differs by {err:.3e}"
+
+
+def pin_stale_entries_are_not_read(orc):
+    dtype = gen.F16
+    c = _case(21, num_seqs=2, num_q_heads=2, num_kv_heads=1, head_dim=32, block_size=16,
+              dtype=dtype, context_lens=[17, 3])
+    bt = np.full((2, 6), 1 << 30, dtype=np.int32)
+    bt[:, :c["block_tables"].shape[1]] = c["block_tables"]
+    bt[0, 2:] = -1
+    bt[1, 1:] = 123456789
+    c["block_tables"] = bt
+    out = _decode(orc, dtype, c)
+    assert np.all(np.isfinite(out)), "a stale slot or table entry was read"
+
+
+def pin_refuses_out_of_pool_entry(orc):
+    import oracle
+
+    c = _case(22, num_seqs=1, num_q_heads=1, num_kv_heads=1, head_dim=16, block_size=16,
+              dtype=gen.F16, context_lens=[20])
+    c["block_tables"][0, 1] = c["num_blocks"]
+    try:
+        _decode(orc, gen.F16, c)
+    except oracle.OracleError:
+        return
+    raise AssertionError("an out-of-pool table entry below the context must be refused")
+
+
+# ---------------------------------------------------------------- append / copy
+
+def pin_append_matches_scatter(orc):
+    rng = np.random.default_rng(23)
+    NB, bs, Hkv, D = 9, 16, 3, 64
+    kc = rng.integers(0, 1 << 16, size=(NB, bs, Hkv, D), dtype=np.uint16)
+    vc = rng.integers(0, 1 << 16, size=(NB, bs, Hkv, D), dtype=np.uint16)
+    T = 7
+    slots = rng.choice(NB * bs, size=T, replace=False).astype(np.int32)
+    slots[2] = -1
+    k = rng.integers(0, 1 << 16, size=(T, Hkv, D), dtype=np.uint16)
+    v = rng.integers(0, 1 << 16, size=(T, Hkv, D), dtype=np.uint16)
+    ek, ev = kc.copy(), vc.copy()
+    keep = slots >= 0
+    ek.reshape(NB * bs, Hkv, D)[slots[keep]] = k[keep]
+    ev.reshape(NB * bs, Hkv, D)[slots[keep]] = v[keep]
+    orc.cache_append(k, v, slots, kc, vc)
+    assert np.array_equal(kc, ek) and np.array_equal(vc, ev), "append differs from a scatter"
+
+
+def pin_copy_matches_block_copy(orc):
+    rng = np.random.default_rng(24)
+    NB, bs, Hkv, D = 12, 16, 2, 64
+    kc = rng.integers(0, 1 << 16, size=(NB, bs, Hkv, D), dtype=np.uint16)
+    vc = rng.integers(0, 1 << 16, size=(NB, bs, Hkv, D), dtype=np.uint16)
+    pairs = np.array([[3, 7], [3, 9], [0, 11], [5, 1]], dtype=np.int32)
+    ek, ev = kc.copy(), vc.copy()
+    for s, d in pairs:
+        ek[d] = ek[s]
+        ev[d] = ev[s]
+    orc.copy_blocks(pairs, kc, vc)
+    assert np.array_equal(kc, ek) and np.array_equal(vc, ev), "copy differs from a block copy"
+
+
+PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

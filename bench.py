@@ -1,0 +1,511 @@
+"""Benchmark: paged decode attention on B200 through the C ABI of libpa.so.
+
+One *step* is one pass of the whole hot path over one decode batch of the
+workload: copy-on-write of shared blocks (pa_copy_blocks), append of each
+sequence's new token (pa_cache_append), then decode attention over every
+context (pa_decode).  Inputs are seeded synthetic data with the workload's
+shapes (paged_kv_cache_458_b200.gen); the K/V pool and every step's inputs are
+resident in HBM before the timed region starts.
+
+The reported metric is the decode's K/V-read bandwidth: algorithmic bytes of
+the decode (K and V rows of every context, q, out, block-table entries and
+context lengths) divided by the device time of the whole step, plus decode
+tokens/s per layer.  The `roofline` object is the decode kernels alone,
+timed with CUDA events on their stream.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--impl ours|reference]
+
+With N > 1 (torchrun) every rank runs its own replica of the workload (its
+own seed); there is no data exchange, only a max-over-ranks of the device
+time.  `--impl reference` times the CPU oracle (fp64, all host cores) on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_458_b200 import gen  # noqa: E402
+
+METRIC = ("paged decode-attn KV-read GB/s (% of B200 HBM peak); decode tokens/s per layer")
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=3000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--workload", default="llama2_7b", choices=sorted(gen.WORKLOADS))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--partition-tokens", type=int, default=0)
+    p.add_argument("--cycle", type=int, default=64,
+                   help="distinct precomputed steps; longer runs replay them in order")
+    p.add_argument("--e2e-steps", type=int, default=500)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=15.0)
+    return p.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas only)
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world: int, backend: str):
+    import datetime
+
+    import torch.distributed as dist
+
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def max_over_ranks(x: float, dist, device=None) -> float:
+    """Largest value of `x` over all ranks (a timing reduction, not data)."""
+    if dist is None:
+        return x
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, dist, device=None) -> float:
+    if dist is None:
+        return x
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# byte and flop accounting (per decode)
+
+
+def decode_bytes(ctx: np.ndarray, num_q_heads, num_kv_heads, head_dim, block_size, elem=2) -> int:
+    """Algorithmic bytes of one decode: K+V rows, q+out, table entries, lengths."""
+    ctx = np.asarray(ctx, dtype=np.int64)
+    S = ctx.shape[0]
+    kv = int(2 * ctx.sum() * num_kv_heads * head_dim * elem)
+    qo = 2 * S * num_q_heads * head_dim * elem
+    tables = int(4 * np.ceil(ctx / block_size).sum())
+    return kv + qo + tables + 4 * S
+
+
+def unique_kv_bytes(tables: np.ndarray, ctx: np.ndarray, block_size, num_kv_heads, head_dim,
+                    elem=2) -> int:
+    """K+V bytes of the distinct slots a decode reads (shared blocks once)."""
+    slots = set()
+    for s in range(len(ctx)):
+        L = int(ctx[s])
+        nb = -(-L // block_size)
+        for i in range(nb):
+            n = min(block_size, L - i * block_size)
+            slots.update(int(tables[s, i]) * block_size + j for j in range(n))
+    return 2 * len(slots) * num_kv_heads * head_dim * elem
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML, read-only)
+
+
+class ClockSampler:
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, uuid: str | None, period_s: float = 0.005):
+        self.uuid, self.period = uuid, period_s
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.error = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            # CUDA and NVML may number devices differently: match by UUID.
+            self._h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid.encode())
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        except Exception as e:  # noqa: BLE001 - clocks are reported, never required
+            self.error = repr(e)
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            except Exception as e:  # noqa: BLE001
+                self.error = repr(e)
+                return
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples),
+                **({"error": self.error} if self.error else {})}
+
+
+def device_uuid(torch) -> str:
+    u = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+    return u if u.startswith("GPU-") else "GPU-" + u
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the kernel source as it is now (else None)."""
+    path = os.path.join(ROOT, "profiles", f"pa_decode_{workload}.json")
+    try:
+        with open(path) as f:
+            prof = json.load(f)
+    except (OSError, ValueError):
+        return None
+    src = os.path.join(ROOT, "paged_kv_cache_458_b200", "csrc", "pa_decode.cu")
+    with open(src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()[:16]
+    if prof.get("source_sha256_16") != digest:
+        return None
+    return prof.get("dram_bytes_per_launch_full_size")
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+
+
+class DeviceWorkload:
+    """The pool and a cycle of precomputed steps, resident on the device."""
+
+    def __init__(self, case, torch, pa, partition_tokens: int):
+        self.case = case
+        self.torch, self.pa = torch, pa
+        dt = pa.torch_dtype(case.dtype)
+        self.dt = dt
+
+        def dev16(a):
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(dt).cuda()
+
+        def dev32(a):
+            return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
+
+        self.k_cache, self.v_cache = dev16(case.k_cache), dev16(case.v_cache)
+        self.steps = []
+        for st in case.steps:
+            self.steps.append(dict(
+                pairs=dev32(st.pairs.reshape(-1, 2)) if len(st.pairs) else None,
+                n_pairs=len(st.pairs), slots=dev32(st.slot_mapping), k_new=dev16(st.k_new),
+                v_new=dev16(st.v_new), q=dev16(st.q), tables=dev32(st.block_tables),
+                lens=dev32(st.context_lens), max_len=int(st.context_lens.max())))
+        self.max_len = max(s["max_len"] for s in self.steps)
+        self.shape = pa.make_shape(
+            num_seqs=case.num_seqs, num_q_heads=case.num_q_heads, num_kv_heads=case.num_kv_heads,
+            head_dim=case.head_dim, block_size=case.block_size, num_blocks=case.num_blocks,
+            max_blocks_per_seq=case.max_blocks_per_seq, partition_tokens=partition_tokens,
+            dtype=case.dtype)
+        self.ws_bytes = pa.pa_decode_workspace_bytes(self.shape, self.max_len)
+        self.ws = torch.empty(max(16, self.ws_bytes), dtype=torch.uint8, device="cuda")
+        self.out = torch.empty((case.num_seqs, case.num_q_heads, case.head_dim), dtype=dt,
+                               device="cuda")
+
+    def step(self, i: int, stream, ev=None):
+        """Enqueue step i (mod the cycle); ev = (start, mid, end) events or None."""
+        self.enqueue(self.steps[i % len(self.steps)], stream, ev)
+
+    def enqueue(self, st: dict, stream, ev=None):
+        pa = self.pa
+        if ev:
+            ev[0].record(stream)
+        if st["n_pairs"]:
+            pa.pa_copy_blocks(st["pairs"], st["n_pairs"], self.k_cache, self.v_cache, self.shape,
+                              stream.cuda_stream)
+        pa.pa_cache_append(st["k_new"], st["v_new"], st["slots"], self.case.num_seqs,
+                           self.k_cache, self.v_cache, self.shape, stream.cuda_stream)
+        if ev:
+            ev[1].record(stream)
+        pa.pa_decode(st["q"], self.k_cache, self.v_cache, st["tables"], st["lens"],
+                     self.case.scale, self.out, self.shape, st["max_len"], self.ws, self.ws_bytes,
+                     stream.cuda_stream)
+        if ev:
+            ev[2].record(stream)
+
+
+def run_ours(args, rank, world, local, dist):
+    import torch
+
+    from paged_kv_cache_458_b200 import pa
+
+    torch.cuda.set_device(local)
+    stream = torch.cuda.Stream()
+    n_cycle = max(1, min(args.cycle, args.steps + args.warmup))
+    case = gen.make_case(args.workload, n_steps=n_cycle, poison=False,
+                         seed=gen.SEED_BASE + gen.WORKLOADS[args.workload].number + 1000 * rank)
+    w = DeviceWorkload(case, torch, pa, args.partition_tokens)
+    bytes_per = [decode_bytes(s.context_lens, case.num_q_heads, case.num_kv_heads, case.head_dim,
+                              case.block_size) for s in case.steps]
+    pool_bytes = 2 * case.k_cache.nbytes
+    kv_step0 = 2 * int(case.steps[0].context_lens.sum()) * case.num_kv_heads * case.head_dim * 2
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            w.step(i, stream)
+        torch.cuda.synchronize()
+        st0, bits = pa.pa_last_device_error(stream.cuda_stream)
+        if st0 != pa.PA_OK:
+            raise RuntimeError(f"device check during warm-up: {bits:#x}")
+
+        evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
+               for _ in range(args.steps)]
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        launches0 = pa.pa_kernel_launches()
+        with ClockSampler(device_uuid(torch)) as clocks:
+            for i in range(args.steps):
+                w.step(args.warmup + i, stream, evs[i])
+            torch.cuda.synchronize()
+        launches = pa.pa_kernel_launches() - launches0
+        if dist is not None:
+            dist.barrier()
+        st1, bits = pa.pa_last_device_error(stream.cuda_stream)
+        if st1 != pa.PA_OK:
+            raise RuntimeError(f"device check during the timed steps: {bits:#x}")
+
+    step_ms = [evs[i][0].elapsed_time(evs[i][2]) for i in range(args.steps)]
+    dec_ms = [evs[i][1].elapsed_time(evs[i][2]) for i in range(args.steps)]
+    total_ms = sum(step_ms)
+    dec_total_ms = sum(dec_ms)
+    step_bytes = sum(bytes_per[(args.warmup + i) % n_cycle] for i in range(args.steps))
+    max_ms = max_over_ranks(total_ms, dist, "cuda")
+    all_bytes = sum_over_ranks(float(step_bytes), dist, "cuda")
+    value = all_bytes / (max_ms * 1e-3) / 1e9
+
+    peak, peak_kind = measured_peak()
+    achieved = step_bytes / (dec_total_ms * 1e-3) / 1e9
+    traffic = profiled_traffic(args.workload)
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(max_ms / args.steps, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded N(0,1) values, shapes and block structure of the workload)",
+        "config": {
+            "workload": f"{args.workload}: {case.workload.description}",
+            "num_seqs": case.num_seqs, "num_q_heads": case.num_q_heads,
+            "num_kv_heads": case.num_kv_heads, "head_dim": case.head_dim,
+            "block_size": case.block_size, "storage_dtype": gen.DTYPE_NAMES[case.dtype],
+            "partition_tokens": args.partition_tokens or 512,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "steps_cycle": n_cycle,
+            "l2": (f"inputs larger than L2: {kv_step0 / 1e6:.0f} MB of K/V read per decode, "
+                   f"{pool_bytes / 1e6:.0f} MB pool, L2 126 MB; no flush"),
+        },
+        "tokens_per_s_per_layer": round(case.num_seqs * args.steps * world / (max_ms * 1e-3), 1),
+        "decode_ms_per_step": round(dec_total_ms / args.steps, 5),
+        "decode_bytes_per_step": int(step_bytes / args.steps),
+        "pct_of_8tbps": round(100 * value / 8000.0, 2),
+        "roofline": {
+            "bound": "hbm", "kernel": "pa_decode (partition kernel + split-K merge kernel)",
+            "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": traffic,
+        },
+        "gpu_launches": int(launches),
+        "clocks": clocks.summary(),
+    }
+    if case.workload.name in ("qwen_7b_prefix", "llama2_70b_beam"):
+        st = case.steps[0]
+        result["unique_kv_bytes_step0"] = unique_kv_bytes(
+            st.block_tables, st.context_lens, case.block_size, case.num_kv_heads, case.head_dim)
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(args, w, stream, bytes_per, n_cycle, dist)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(case, args.cpu_seconds, case.steps[0])
+    return result
+
+
+def run_e2e(args, w, stream, bytes_per, n_cycle, dist):
+    """Same metric through the public calls with host buffers: every step
+    copies its inputs from pinned host memory and reads its output back."""
+    import torch
+
+    case = w.case
+    host = []
+    for st in case.steps:
+        def pin16(a):
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(w.dt).pin_memory()
+
+        def pin32(a):
+            return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).pin_memory()
+
+        host.append(dict(pairs=pin32(st.pairs.reshape(-1, 2)) if len(st.pairs) else None,
+                         n_pairs=len(st.pairs), slots=pin32(st.slot_mapping), k_new=pin16(st.k_new),
+                         v_new=pin16(st.v_new), q=pin16(st.q), tables=pin32(st.block_tables),
+                         lens=pin32(st.context_lens), max_len=int(st.context_lens.max())))
+    out_host = torch.empty(w.out.shape, dtype=w.dt).pin_memory()
+    dev = [dict((k, (torch.empty_like(v, device="cuda") if isinstance(v, torch.Tensor) else v))
+                for k, v in h.items()) for h in host]
+    h2d = 0
+    steps = min(args.e2e_steps, args.steps)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for i in range(steps):
+            j = (args.warmup + i) % n_cycle
+            h, d = host[j], dev[j]
+            for k, v in h.items():
+                if isinstance(v, torch.Tensor):
+                    d[k].copy_(v, non_blocking=True)
+                    h2d += v.numel() * v.element_size()
+            w.enqueue(d, stream)
+            out_host.copy_(w.out, non_blocking=True)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dist, "cuda")
+    all_bytes = sum_over_ranks(float(sum(bytes_per[(args.warmup + i) % n_cycle]
+                                         for i in range(steps))), dist, "cuda")
+    return {"value": round(all_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "steps": steps, "ms_per_step": round(ms / steps, 5),
+            "h2d_bytes_per_step": int(h2d // steps),
+            "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size())}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (baseline leg and reference arm)
+
+
+def _oracle_sample(case, st, n_seqs, orc, threads):
+    sl = slice(0, n_seqs)
+    t0 = time.perf_counter()
+    orc.decode(case.dtype, st.q[sl], case.k_cache, case.v_cache, st.block_tables[sl],
+               st.context_lens[sl], case.scale, num_threads=threads)
+    dt = time.perf_counter() - t0
+    nbytes = decode_bytes(st.context_lens[sl], case.num_q_heads, case.num_kv_heads, case.head_dim,
+                          case.block_size)
+    return dt, nbytes
+
+
+def cpu_baseline(case, seconds: float, st):
+    """The fp64 oracle on the host cores, on the first sequences of the batch
+    (sized to about `seconds` of work); reported as GB/s of algorithmic bytes."""
+    import oracle
+
+    orc = oracle.load()
+    cores = len(os.sched_getaffinity(0))
+    threads = orc.num_threads(cores)
+    dt1, _ = _oracle_sample(case, st, 1, orc, threads)
+    n = int(max(1, min(case.num_seqs, seconds / max(dt1, 1e-6))))
+    dt, nbytes = _oracle_sample(case, st, n, orc, threads)
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"fp64 C oracle, decode of the first {n} of {case.num_seqs} sequences of step 0 "
+                      f"({nbytes / 1e6:.1f} MB algorithmic), {dt:.2f} s wall, {threads} threads"}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: each step decodes a bounded sample."""
+    import oracle
+
+    case = gen.make_case(args.workload, n_steps=1, poison=False)
+    st = case.steps[0]
+    orc = oracle.load()
+    cores = len(os.sched_getaffinity(0))
+    threads = orc.num_threads(cores)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    dt1, _ = _oracle_sample(case, st, 1, orc, threads)
+    n = int(max(1, min(case.num_seqs, budget / max(dt1, 1e-6))))
+    for _ in range(args.warmup):
+        _oracle_sample(case, st, n, orc, threads)
+    tot_t, tot_b = 0.0, 0
+    for _ in range(args.steps):
+        dt, nb = _oracle_sample(case, st, n, orc, threads)
+        tot_t += dt
+        tot_b += nb
+    value = tot_b / tot_t / 1e9
+    sample = (f"fp64 C oracle, each step decodes the first {n} of {case.num_seqs} sequences "
+              f"of step 0 on {threads} threads")
+    return {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * tot_t / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{args.workload}: {case.workload.description}"},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return 0
+    dist = init_dist(world, "nccl")
+    try:
+        res = run_ours(args, rank, world, local, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

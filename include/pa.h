@@ -1,0 +1,224 @@
+/*
+ * pa.h -- C ABI of libpa.so: paged decode attention on B200 (sm_100a).
+ *
+ * The method (PagedAttention) keeps each sequence's key/value cache in
+ * fixed-size physical blocks of `block_size` tokens inside one pool tensor,
+ * and reaches them through a per-sequence block table that maps logical block
+ * j / block_size to a physical block (zingnex.cn, "vLLM与PagedAttention深度剖析",
+ * section 3.2: the block tensor, items 1-4; 5688vip.com vLLM notes, section
+ * 2.2: "logical block 0 -> physical block 7").  Blocks may be shared by
+ * several sequences (common prefixes, beam candidates) and are copied before
+ * a shared block is written (section 3.2 item 3).  Decode is bandwidth-bound
+ * (5688vip.com section 2.1), so the kernels are built around the K/V read.
+ *
+ * Conventions for every call:
+ *  - Every pointer named "device" is a CUDA device pointer on the current
+ *    device, 16-byte aligned, owned by the caller; the library allocates
+ *    nothing per call and keeps no pointer after the call returns.
+ *  - All device work is enqueued asynchronously on `stream` (a cudaStream_t;
+ *    NULL is the legacy default stream).  No call reads device memory on the
+ *    host or synchronises, except pa_last_device_error().
+ *  - Shapes and host-side arguments are validated before anything is
+ *    launched; a refusal returns PA_ERR_INVALID_ARG or PA_ERR_UNSUPPORTED and
+ *    launches nothing.  A failed launch returns PA_ERR_CUDA.
+ *  - Values that only the device can see (block ids, slots, context lengths,
+ *    copy pairs) are range-checked by the kernels.  A bad value never faults:
+ *    the access is skipped (a K/V row outside the pool reads as zeros), a bit
+ *    is recorded in a per-device error word, and pa_last_device_error()
+ *    returns PA_ERR_DEVICE_CHECK until it is read.
+ *  - No kernel waits on anything but its own TMA copies, and every such wait
+ *    has a wall-clock limit (2 s) after which the kernel records
+ *    PA_DEVERR_WAIT_TIMEOUT and returns.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so this header needs no CUDA
+ * headers. */
+typedef struct CUstream_st *pa_stream_t;
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, misaligned pointer, bad shape */
+  PA_ERR_UNSUPPORTED = 2,  /* valid but not built: head_dim, group size, block size, dtype */
+  PA_ERR_CUDA = 3,         /* a CUDA runtime call or a launch failed */
+  PA_ERR_OOM = 4,          /* the host block allocator has no free block */
+  PA_ERR_DEVICE_CHECK = 5  /* a kernel found a bad device-side value (see pa_last_device_error) */
+} pa_status;
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Bits of the device error word returned by pa_last_device_error(). */
+#define PA_DEVERR_BLOCK_ID 0x1u     /* block-table entry of a token below the context is outside [0, num_blocks) */
+#define PA_DEVERR_CONTEXT_LEN 0x2u  /* context length < 0, > max_context_len or > max_blocks_per_seq * block_size */
+#define PA_DEVERR_SLOT 0x4u         /* append slot >= num_blocks * block_size */
+#define PA_DEVERR_PAIR 0x8u         /* copy pair names a block outside [0, num_blocks) */
+#define PA_DEVERR_WAIT_TIMEOUT 0x10u
+
+/*
+ * Shape of one paged KV cache and of the batch that reads it.
+ *
+ * Layouts (all contiguous, row-major, elements of `dtype`):
+ *   q, out                  [num_seqs][num_q_heads][head_dim]
+ *   k_cache, v_cache        [num_blocks][block_size][num_kv_heads][head_dim]
+ *                           (the pages' [num_blocks, block_size, num_heads,
+ *                           head_dim] block tensor, one for K and one for V)
+ *   block_tables (int32)    [num_seqs][max_blocks_per_seq]
+ *   context_lens (int32)    [num_seqs]
+ *   k, v for append         [num_tokens][num_kv_heads][head_dim]
+ *
+ * Query head h reads kv head h / (num_q_heads / num_kv_heads): grouped-query
+ * heads are contiguous.
+ *
+ * Built values: head_dim in {64, 128}; num_q_heads / num_kv_heads in
+ * {1, 2, 4, 8, 16}; block_size a multiple of 16 (16 and 256 are the measured
+ * ones); num_blocks * block_size < 2^31; partition_tokens a multiple of 16 in
+ * [16, 2048], or 0 for the default 512.
+ */
+typedef struct {
+  int32_t num_seqs;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t block_size;
+  int32_t num_blocks;
+  int32_t max_blocks_per_seq;
+  int32_t partition_tokens;
+  int32_t dtype; /* pa_dtype */
+} pa_shape;
+
+/* Bytes of device workspace pa_decode() needs for `shape` when no context is
+ * longer than `max_context_len` tokens (0 when one partition covers every
+ * context).  The workspace holds, per (sequence, query head, partition), the
+ * running max, the softmax sum and the unnormalised output row in fp32; it
+ * needs no initialisation and is dead after the call's kernels finish. */
+size_t pa_decode_workspace_bytes(const pa_shape *shape, int32_t max_context_len);
+
+/*
+ * Single-token decode attention over the paged cache.
+ *
+ * For every sequence s and query head h, with kv head h / g and
+ * ctx = context_lens[s]:
+ *   x_j  = scale * <q[s][h], K_j>,  K_j = k_cache[block_tables[s][j / bs]][j % bs][h / g]
+ *   out[s][h] = sum_j softmax(x)_j * V_j      (j = 0 .. ctx - 1; V_j likewise)
+ * computed in fp32 and rounded to nearest-even into `dtype`.  ctx == 0 gives a
+ * zero row.  Table entries at or beyond ceil(ctx / bs) and cache slots at or
+ * beyond ctx are never read, so they may hold anything (including NaN).
+ *
+ * Contexts are cut into partitions of shape->partition_tokens tokens; each
+ * (sequence, kv head, partition) is one CTA, and sequences with more than
+ * one partition are merged by a second kernel (log-sum-exp rule).
+ *
+ * q, k_cache, v_cache, block_tables, context_lens, out: device, layouts above.
+ * max_context_len: host-side upper bound on every context_lens[s]; it sizes the
+ *   grid.  A larger device value is clamped and reported (PA_DEVERR_CONTEXT_LEN).
+ * workspace: device, at least pa_decode_workspace_bytes(shape, max_context_len)
+ *   bytes (may be NULL when that is 0).  It must not be shared with a decode
+ *   that runs concurrently.
+ */
+pa_status pa_decode(const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_tables, const int32_t *context_lens, float scale,
+                    void *out, const pa_shape *shape, int32_t max_context_len,
+                    void *workspace, size_t workspace_bytes, pa_stream_t stream);
+
+/*
+ * Append one new token per entry into the cache (the "update KV cache" step of
+ * each decode iteration, 5688vip.com section 2.1): for t < num_tokens with
+ * slot = slot_mapping[t] >= 0,
+ *   k_cache viewed as [num_blocks * block_size][num_kv_heads][head_dim] gets
+ *   row `slot` = k[t], and likewise v_cache = v[t].
+ * slot = physical_block * block_size + offset.  Negative slots are skipped
+ * (padding).  Slots must be distinct.  A bit-exact copy (no conversion).
+ * Uses shape->num_kv_heads, head_dim, block_size, num_blocks, dtype.
+ * k, v, slot_mapping (int32 [num_tokens]), k_cache, v_cache: device.
+ */
+pa_status pa_cache_append(const void *k, const void *v, const int32_t *slot_mapping,
+                          int32_t num_tokens, void *k_cache, void *v_cache,
+                          const pa_shape *shape, pa_stream_t stream);
+
+/*
+ * Copy-on-write of whole blocks (zingnex.cn section 3.2 item 3): for each
+ * pair i, block src_dst_pairs[2i+1] of k_cache and of v_cache becomes a
+ * byte copy of block src_dst_pairs[2i].  Destinations must be distinct and no
+ * destination may also be a source in the same call.
+ * src_dst_pairs: device int32 [num_pairs][2].  num_pairs == 0 launches nothing.
+ */
+pa_status pa_copy_blocks(const int32_t *src_dst_pairs, int32_t num_pairs, void *k_cache,
+                         void *v_cache, const pa_shape *shape, pa_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears this device's error word.
+ * Returns PA_OK when it was zero, PA_ERR_DEVICE_CHECK otherwise (bits in
+ * *bits_out if non-NULL), PA_ERR_CUDA if the synchronisation failed. */
+pa_status pa_last_device_error(pa_stream_t stream, uint32_t *bits_out);
+
+/* Static description of a status code (never NULL). */
+const char *pa_status_string(pa_status status);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t pa_kernel_launches(void);
+
+/* Build description: target architecture and library version. */
+const char *pa_build_info(void);
+
+/* ------------------------------------------------------------------------
+ * Host block allocator (zingnex.cn section 3.2 items 1-4; jsqmd.com
+ * "vLLM-v0.11.0性能实测" section 4.2): a free list of physical blocks, a
+ * reference count per block and a block table per sequence.  It builds the
+ * block tables, slot mappings and copy-on-write pairs the kernels consume.
+ *
+ * The free list is a stack: `order` (a permutation of 0..num_blocks-1, or
+ * NULL for 0, 1, 2, ...) gives the allocation order, and a block whose count
+ * drops to zero goes back on top, so it is the next one handed out.  Freeing a
+ * sequence releases its blocks last-to-first.  Sequence ids are arbitrary
+ * int32 values.  Not thread-safe; all memory is host memory.
+ */
+typedef struct pa_alloc pa_alloc;
+
+/* Returns NULL on bad arguments (order not a permutation, sizes <= 0). */
+pa_alloc *pa_alloc_create(int32_t num_blocks, int32_t block_size, const int32_t *order);
+void pa_alloc_destroy(pa_alloc *a);
+
+/* New sequence with `num_tokens` tokens (blocks allocated on demand). */
+pa_status pa_alloc_add_seq(pa_alloc *a, int32_t seq, int32_t num_tokens);
+/* Grow a sequence by `num_tokens` tokens without copy-on-write (prefill). */
+pa_status pa_alloc_extend(pa_alloc *a, int32_t seq, int32_t num_tokens);
+/* `child` (new) shares every block of `parent`; each block's count + 1. */
+pa_status pa_alloc_fork(pa_alloc *a, int32_t parent, int32_t child);
+/* Drop a sequence; blocks whose count reaches zero return to the free list. */
+pa_status pa_alloc_free_seq(pa_alloc *a, int32_t seq);
+
+/*
+ * Reserve the slot of one new token for each of seqs[0..n-1], in order.
+ * A sequence whose next token starts a block gets a fresh block.  One whose
+ * last block is shared gets a fresh block and a copy pair (src, dst) is
+ * appended to pairs_out (capacity n pairs); the shared block's count drops
+ * by one.  slot_out[i] = block * block_size + offset.
+ * All-or-nothing: PA_ERR_OOM (nothing changed) when the free list cannot
+ * cover the whole batch.
+ */
+pa_status pa_alloc_append_slots(pa_alloc *a, const int32_t *seqs, int32_t n, int32_t *slot_out,
+                                int32_t *pairs_out, int32_t *num_pairs_out);
+
+/* Write the block tables ([n][max_blocks_per_seq], padded with -1) and
+ * context lengths of seqs[0..n-1].  PA_ERR_INVALID_ARG if a table is longer
+ * than max_blocks_per_seq or a sequence is unknown. */
+pa_status pa_alloc_block_tables(const pa_alloc *a, const int32_t *seqs, int32_t n,
+                                int32_t max_blocks_per_seq, int32_t *tables_out,
+                                int32_t *lens_out);
+
+int32_t pa_alloc_num_free(const pa_alloc *a);
+/* Reference count of `block`, or -1 if out of range. */
+int32_t pa_alloc_refcount(const pa_alloc *a, int32_t block);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

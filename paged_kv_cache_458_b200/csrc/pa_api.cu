@@ -1,0 +1,260 @@
+// pa_api.cu -- the C ABI of libpa.so: host-side validation, TMA descriptor
+// set-up and dispatch to the kernels.  See include/pa.h for the contract.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "pa.h"
+#include "pa_internal.h"
+
+namespace {
+
+// The per-device error word the kernels report into (see pa.h).
+__device__ unsigned int g_device_error = 0;
+
+// Device address of g_device_error on the current device, looked up once per
+// device (a host-side symbol name is not a device address).
+unsigned int* error_word() {
+  static std::mutex mu;
+  static unsigned int* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<unsigned int*>(p);
+  }
+  return addr[dev];
+}
+
+std::atomic<uint64_t> g_launches{0};
+
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int effective_partition(const pa_shape* s) {
+  return s->partition_tokens == 0 ? 512 : s->partition_tokens;
+}
+
+// Shape checks common to every call that touches the pool.
+pa_status check_pool_shape(const pa_shape* s) {
+  if (!s) return PA_ERR_INVALID_ARG;
+  if (s->num_kv_heads <= 0 || s->head_dim <= 0 || s->block_size <= 0 || s->num_blocks < 0)
+    return PA_ERR_INVALID_ARG;
+  if (s->dtype != PA_F16 && s->dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (s->head_dim != 64 && s->head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (s->block_size % 16 != 0) return PA_ERR_UNSUPPORTED;
+  if ((long long)s->num_blocks * s->block_size >= (1LL << 31)) return PA_ERR_UNSUPPORTED;
+  return PA_OK;
+}
+
+pa_status check_decode_shape(const pa_shape* s, int32_t max_context_len) {
+  pa_status st = check_pool_shape(s);
+  if (st != PA_OK) return st;
+  if (s->num_seqs < 0 || s->num_q_heads <= 0 || s->max_blocks_per_seq < 0 || max_context_len < 0)
+    return PA_ERR_INVALID_ARG;
+  if (s->num_q_heads % s->num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  const int g = s->num_q_heads / s->num_kv_heads;
+  if (g != 1 && g != 2 && g != 4 && g != 8 && g != 16) return PA_ERR_UNSUPPORTED;
+  const int pt = effective_partition(s);
+  if (pt < 16 || pt % 16 != 0 || pt > pa::decode_max_partition_tokens()) return PA_ERR_UNSUPPORTED;
+  if ((long long)s->num_seqs * s->num_q_heads * s->head_dim >= (1LL << 40)) return PA_ERR_INVALID_ARG;
+  return PA_OK;
+}
+
+int num_partitions(const pa_shape* s, int32_t max_context_len) {
+  const int pt = effective_partition(s);
+  return (max_context_len + pt - 1) / pt;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library does not link libcuda directly.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D map over one pool viewed as [num_blocks * block_size][Hkv][D]; a box
+// is `rows` consecutive token rows of one kv head.
+bool make_pool_map(CUtensorMap* map, const void* pool, const pa_shape* s, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)s->head_dim, (cuuint64_t)s->num_kv_heads,
+                              (cuuint64_t)s->num_blocks * s->block_size};
+  const cuuint64_t strides[2] = {(cuuint64_t)s->head_dim * 2,
+                                 (cuuint64_t)s->num_kv_heads * s->head_dim * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)s->head_dim, 1, (cuuint32_t)rows};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(pool), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t pa_decode_workspace_bytes(const pa_shape* shape, int32_t max_context_len) {
+  if (check_decode_shape(shape, max_context_len) != PA_OK) return 0;
+  const long long P = num_partitions(shape, max_context_len);
+  if (P <= 1) return 0;
+  const long long rows = (long long)shape->num_seqs * shape->num_q_heads * P;
+  const long long acc = rows * shape->head_dim * 4;
+  const long long ml = rows * 2 * 4;
+  return (size_t)(((acc + 255) / 256) * 256 + ml);
+}
+
+pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, const int32_t* context_lens, float scale,
+                    void* out, const pa_shape* shape, int32_t max_context_len, void* workspace,
+                    size_t workspace_bytes, pa_stream_t stream) {
+  pa_status st = check_decode_shape(shape, max_context_len);
+  if (st != PA_OK) return st;
+  if (shape->num_seqs == 0) return PA_OK;
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out) return PA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return PA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+    return PA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  const size_t need = pa_decode_workspace_bytes(shape, max_context_len);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return PA_ERR_INVALID_ARG;
+  if (max_context_len > (long long)shape->max_blocks_per_seq * shape->block_size)
+    return PA_ERR_INVALID_ARG;
+
+  const int P = num_partitions(shape, max_context_len);
+  pa::DecodeArgs a{};
+  a.q = static_cast<const uint16_t*>(q);
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.out = static_cast<uint16_t*>(out);
+  if (need > 0) {
+    const long long rows = (long long)shape->num_seqs * shape->num_q_heads * P;
+    a.ws_acc = static_cast<float*>(workspace);
+    a.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                       ((rows * shape->head_dim * 4 + 255) / 256) * 256);
+  }
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.num_seqs = shape->num_seqs;
+  a.num_q_heads = shape->num_q_heads;
+  a.num_kv_heads = shape->num_kv_heads;
+  a.block_size = shape->block_size;
+  a.num_blocks = shape->num_blocks;
+  a.max_blocks_per_seq = shape->max_blocks_per_seq;
+  a.partition_tokens = effective_partition(shape);
+  a.num_parts = P > 0 ? P : 1;
+  a.max_context_len = max_context_len;
+  a.err = error_word();
+  if (!a.err) return PA_ERR_CUDA;
+
+  CUtensorMap tk, tv;
+  if (shape->num_blocks > 0) {
+    if (!make_pool_map(&tk, k_cache, shape, pa::decode_chunk_tokens()) ||
+        !make_pool_map(&tv, v_cache, shape, pa::decode_chunk_tokens()))
+      return PA_ERR_CUDA;
+  } else {
+    // An empty pool can only serve empty contexts; the kernels issue no load.
+    if (max_context_len > 0) return PA_ERR_INVALID_ARG;
+    memset(&tk, 0, sizeof tk);
+    memset(&tv, 0, sizeof tv);
+  }
+  int launched = 0;
+  cudaError_t e = pa::launch_decode(a, shape->dtype, shape->head_dim,
+                                    shape->num_q_heads / shape->num_kv_heads, tk, tv,
+                                    reinterpret_cast<cudaStream_t>(stream), &launched);
+  count_launches(launched);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_cache_append(const void* k, const void* v, const int32_t* slot_mapping,
+                          int32_t num_tokens, void* k_cache, void* v_cache, const pa_shape* shape,
+                          pa_stream_t stream) {
+  pa_status st = check_pool_shape(shape);
+  if (st != PA_OK) return st;
+  if (num_tokens < 0) return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (reinterpret_cast<uintptr_t>(slot_mapping) & 3u))
+    return PA_ERR_INVALID_ARG;
+  const int row_bytes = shape->num_kv_heads * shape->head_dim * 2;
+  unsigned int* err = error_word();
+  if (!err) return PA_ERR_CUDA;
+  int launched = 0;
+  cudaError_t e = pa::launch_cache_append(k, v, slot_mapping, num_tokens, k_cache, v_cache,
+                                          (long long)shape->num_blocks * shape->block_size,
+                                          row_bytes, err, reinterpret_cast<cudaStream_t>(stream),
+                                          &launched);
+  count_launches(launched);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_copy_blocks(const int32_t* src_dst_pairs, int32_t num_pairs, void* k_cache,
+                         void* v_cache, const pa_shape* shape, pa_stream_t stream) {
+  pa_status st = check_pool_shape(shape);
+  if (st != PA_OK) return st;
+  if (num_pairs < 0) return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PA_OK;
+  if (num_pairs > 65535) return PA_ERR_UNSUPPORTED;
+  if (!src_dst_pairs || !k_cache || !v_cache) return PA_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(src_dst_pairs) & 3u))
+    return PA_ERR_INVALID_ARG;
+  const long long block_bytes =
+      (long long)shape->block_size * shape->num_kv_heads * shape->head_dim * 2;
+  unsigned int* err = error_word();
+  if (!err) return PA_ERR_CUDA;
+  int launched = 0;
+  cudaError_t e = pa::launch_copy_blocks(src_dst_pairs, num_pairs, k_cache, v_cache,
+                                         shape->num_blocks, block_bytes, err,
+                                         reinterpret_cast<cudaStream_t>(stream), &launched);
+  count_launches(launched);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_last_device_error(pa_stream_t stream, uint32_t* bits_out) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return PA_ERR_CUDA;
+  unsigned int bits = 0;
+  const unsigned int zero = 0;
+  if (cudaMemcpyFromSymbol(&bits, g_device_error, sizeof bits) != cudaSuccess) return PA_ERR_CUDA;
+  if (bits && cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (bits_out) *bits_out = bits;
+  return bits ? PA_ERR_DEVICE_CHECK : PA_OK;
+}
+
+const char* pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case PA_ERR_CUDA: return "CUDA error";
+    case PA_ERR_OOM: return "out of blocks";
+    case PA_ERR_DEVICE_CHECK: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+uint64_t pa_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+#define PA_STR2(x) #x
+#define PA_STR(x) PA_STR2(x)
+const char* pa_build_info(void) { return "libpa 0.1 for sm_100a, CUDA runtime " PA_STR(CUDART_VERSION); }
+
+}  // extern "C"

@@ -1,0 +1,106 @@
+// pa_cache.cu -- the two cache-maintenance kernels of the paged KV cache.
+//
+// append: the "update KV cache" step of each decode iteration (5688vip.com
+//   vLLM notes, section 2.1) writes the new token's K and V rows into the slot
+//   the block table reserved for it (zingnex.cn, "vLLM与PagedAttention深度剖析",
+//   section 3.2 item 1: a block is taken only when a token crosses into it).
+// copy:   copy-on-write of a shared block before one of its sharers writes
+//   into it (same page, section 3.2 item 3).
+//
+// Both are byte copies in 16-byte vectors; pools are [NB][bs][Hkv][D], so one
+// token's K row over all kv heads is one contiguous run of Hkv * D elements
+// and one block is a contiguous run of bs * Hkv * D elements.
+#include <cuda_runtime.h>
+
+#include "pa_common.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+// One CTA per token: copies row_bytes of K and of V.
+__global__ void __launch_bounds__(256)
+cache_append_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                    const int32_t* __restrict__ slot_mapping, uint4* __restrict__ k_cache,
+                    uint4* __restrict__ v_cache, long long num_slots, int row_vecs,
+                    unsigned int* err) {
+  const int t = blockIdx.x;
+  const long long slot = __ldg(slot_mapping + t);
+  if (slot < 0) return;
+  if (slot >= num_slots) {
+    if (threadIdx.x == 0) report(err, kErrSlot);
+    return;
+  }
+  const uint4* ks = k + (size_t)t * row_vecs;
+  const uint4* vs = v + (size_t)t * row_vecs;
+  uint4* kd = k_cache + slot * row_vecs;
+  uint4* vd = v_cache + slot * row_vecs;
+  for (int i = threadIdx.x; i < row_vecs; i += blockDim.x) {
+    kd[i] = __ldg(ks + i);
+    vd[i] = __ldg(vs + i);
+  }
+}
+
+// grid.x = pieces of a block, grid.y = pair.  Each CTA copies kPiece vectors
+// of the K block and of the V block.
+constexpr int kCopyThreads = 256;
+constexpr int kCopyUnroll = 4;
+constexpr int kPiece = kCopyThreads * kCopyUnroll;
+
+__global__ void __launch_bounds__(kCopyThreads)
+copy_blocks_kernel(const int32_t* __restrict__ pairs, uint4* __restrict__ k_cache,
+                   uint4* __restrict__ v_cache, int num_blocks, long long block_vecs,
+                   unsigned int* err) {
+  const int i = blockIdx.y;
+  const int src = __ldg(pairs + 2 * i), dst = __ldg(pairs + 2 * i + 1);
+  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) report(err, kErrPair);
+    return;
+  }
+  const long long base = (long long)blockIdx.x * kPiece;
+  const uint4* ks = k_cache + src * block_vecs;
+  const uint4* vs = v_cache + src * block_vecs;
+  uint4* kd = k_cache + dst * block_vecs;
+  uint4* vd = v_cache + dst * block_vecs;
+  uint4 rk[kCopyUnroll], rv[kCopyUnroll];
+#pragma unroll
+  for (int u = 0; u < kCopyUnroll; ++u) {
+    const long long e = base + u * kCopyThreads + threadIdx.x;
+    if (e < block_vecs) { rk[u] = ks[e]; rv[u] = vs[e]; }
+  }
+#pragma unroll
+  for (int u = 0; u < kCopyUnroll; ++u) {
+    const long long e = base + u * kCopyThreads + threadIdx.x;
+    if (e < block_vecs) { kd[e] = rk[u]; vd[e] = rv[u]; }
+  }
+}
+
+cudaError_t launch_cache_append(const void* k, const void* v, const int32_t* slot_mapping,
+                                int num_tokens, void* k_cache, void* v_cache, long long num_slots,
+                                int row_bytes, unsigned int* err, cudaStream_t stream,
+                                int* launches) {
+  if (num_tokens == 0) return cudaSuccess;
+  const int row_vecs = row_bytes / 16;
+  const int threads = row_vecs >= 256 ? 256 : ((row_vecs + 31) / 32) * 32;
+  cache_append_kernel<<<num_tokens, threads, 0, stream>>>(
+      static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), num_slots, row_vecs, err);
+  ++*launches;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_copy_blocks(const int32_t* pairs, int num_pairs, void* k_cache, void* v_cache,
+                               int num_blocks, long long block_bytes, unsigned int* err,
+                               cudaStream_t stream, int* launches) {
+  if (num_pairs == 0) return cudaSuccess;
+  const long long block_vecs = block_bytes / 16;
+  const long long pieces = (block_vecs + kPiece - 1) / kPiece;
+  if (num_pairs > 65535 || pieces > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  dim3 grid((unsigned)pieces, (unsigned)num_pairs);
+  copy_blocks_kernel<<<grid, kCopyThreads, 0, stream>>>(pairs, static_cast<uint4*>(k_cache),
+                                                        static_cast<uint4*>(v_cache), num_blocks,
+                                                        block_vecs, err);
+  ++*launches;
+  return cudaGetLastError();
+}
+
+}  // namespace pa

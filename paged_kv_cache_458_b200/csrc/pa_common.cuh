@@ -1,0 +1,135 @@
+// pa_common.cuh -- device-side helpers shared by the libpa kernels (sm_100a).
+//
+// * element traits for fp16 / bf16 storage with fp32 arithmetic;
+// * the device error word the kernels report bad indices and expired waits in
+//   (no kernel ever traps: a failed check records a bit and skips the access);
+// * thin inline-PTX wrappers for mbarrier and the tiled TMA load
+//   (cp.async.bulk.tensor), all waits bounded by a wall-clock limit.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace pa {
+
+// Bits of the device error word.
+enum DeviceErrorBits : unsigned int {
+  kErrBlockId = 1u << 0,      // a block-table entry below the context is outside the pool
+  kErrContextLen = 1u << 1,   // a context length is negative or above the host's bound
+  kErrSlot = 1u << 2,         // an append slot is outside the pool
+  kErrPair = 1u << 3,         // a copy pair names a block outside the pool
+  kErrWaitTimeout = 1u << 4,  // an mbarrier wait ran past its time limit
+};
+
+// Kernels receive the address of the per-device error word (read and
+// cleared by pa_last_device_error()) and OR bits into it.
+__device__ __forceinline__ void report(unsigned int* err, unsigned int bits) { atomicOr(err, bits); }
+
+// ---------------------------------------------------------------------------
+// element traits
+
+template <typename T> struct Elem;
+
+template <> struct Elem<__half> {
+  // two packed elements -> two floats
+  static __device__ __forceinline__ float2 to_f2(uint32_t u) {
+    __half2 h = *reinterpret_cast<__half2*>(&u);
+    return __half22float2(h);
+  }
+  static __device__ __forceinline__ uint16_t from_f(float x) {
+    __half h = __float2half_rn(x);
+    return *reinterpret_cast<uint16_t*>(&h);
+  }
+};
+
+template <> struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float2 to_f2(uint32_t u) {
+    // bf16 is the top half of an fp32: widening is a shift / mask
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+  }
+  static __device__ __forceinline__ uint16_t from_f(float x) {
+    __nv_bfloat16 b = __float2bfloat16_rn(x);
+    return *reinterpret_cast<uint16_t*>(&b);
+  }
+};
+
+// ---------------------------------------------------------------------------
+// time and shared-memory addressing
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+// Make barrier initialisation visible to the async (TMA) proxy.
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t phase) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(phase)
+      : "memory");
+  return ok != 0;
+}
+
+// Wall-clock limit of any single wait.  A TMA load of a few KB completes in
+// microseconds; two seconds means the copy will never land.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Wait for the barrier's phase `phase` to complete.  Returns false (after
+// recording kErrWaitTimeout) if it has not completed within kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, unsigned int* err) {
+  if (mbar_try_wait(bar, phase)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t spins = 0;
+  while (!mbar_try_wait(bar, phase)) {
+    if ((++spins & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+      report(err, kErrWaitTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// TMA: tiled 3-D load global -> shared, completion counted on an mbarrier.
+// The tensor map lives in kernel parameter space (__grid_constant__).
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint32_t bar, int c0,
+                                            int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const void* tmap) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
+}  // namespace pa

@@ -1,0 +1,451 @@
+// pa_decode.cu -- single-token decode attention over a paged KV cache (sm_100a).
+//
+// Method: PagedAttention keeps K and V in fixed-size physical blocks reached
+// through a per-sequence block table (zingnex.cn, "vLLM与PagedAttention深度剖析",
+// section 3.2; 5688vip.com vLLM notes, section 2.2).  Decode reads every
+// cached K/V row of the sequence once per generated token and does little
+// arithmetic per byte, so this kernel is organised around the HBM read
+// (5688vip.com section 2.1: decode is bandwidth-bound).
+//
+// Work decomposition
+//   One CTA per (partition, sequence, kv head).  A partition is a run of
+//   partition_tokens tokens (512 by default); the CTA holds the whole grouped
+//   query (g = Hq / Hkv heads) in registers.  Inside the CTA each warp owns
+//   every NW-th chunk of 16 tokens and runs its own TMA pipeline of NST
+//   stages: lane 0 issues two tiled TMA loads per chunk (a 16-row box of K
+//   and of V of one kv head inside one physical block) on an mbarrier, so the
+//   gather through the block table costs one table read per chunk and no
+//   address arithmetic per byte.  Warps never wait on each other until the
+//   end, where their (max, sum, output) states are merged in shared memory.
+//
+// Arithmetic per chunk (fp32 throughout)
+//   QK^T: lane l holds D/32 consecutive dims of every query head; per token it
+//   multiplies its slice of the K row, and one transposed butterfly
+//   (reduce-scatter over 32 values) leaves each lane with one complete logit.
+//   Online softmax (log2 domain, scale * log2 e folded into q): running max m
+//   and sum l per head; the output accumulators are rescaled by 2^(m_old-m_new).
+//   PV: p is staged through shared memory and every lane accumulates its dims
+//   of all heads.  Tokens past the context are masked to p = 0 and their V rows
+//   are never touched, so stale slots may hold NaN.
+//
+// Split-K: a sequence with more than one partition stores, per (head,
+//   partition), m, l and the unnormalised output row in fp32; the merge
+//   kernel combines them with M = max m_p, out = sum 2^(m_p-M) acc_p /
+//   sum 2^(m_p-M) l_p.  A sequence with a single partition is written directly.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "pa_common.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+constexpr int kChunk = 16;  // tokens per TMA box (a block is a multiple of this)
+
+template <int D, int G, int NW, int NST>
+struct DecodeSmem {
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kStageBytes = 2 * kChunk * kRowBytes;  // K box then V box
+  static constexpr int kStagesBytes = NW * NST * kStageBytes;
+  static constexpr int kPBytes = NW * (kChunk * G + G) * 4;   // p[16][G] + alpha[G] per warp
+  static constexpr int kBarBytes = NW * NST * 8;
+  static constexpr int kMergeBytes = NW * (G * D + 2 * G) * 4;
+  static_assert(kMergeBytes <= kStagesBytes, "merge area reuses the stage buffers");
+  static constexpr int kTotal = kStagesBytes + kPBytes + kBarBytes;
+};
+
+__device__ __forceinline__ float warp_max_xor(float v, int lo, int hi) {
+  for (int o = lo; o <= hi; o <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum_xor(float v, int lo, int hi) {
+  for (int o = lo; o <= hi; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// One halving step of the transposed reduction: lanes with bit O set keep the
+// upper half of v[0..N), the others the lower half; each adds the partner's
+// copy of the half it keeps.
+template <int O, int N>
+__device__ __forceinline__ void rs_step(float (&v)[32], int lane) {
+  const bool upper = (lane & O) != 0;
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) {
+    const float send = upper ? v[i] : v[i + N / 2];
+    const float keep = upper ? v[i + N / 2] : v[i];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+  }
+}
+
+// Sum N in {16, 32} per-lane partial values over the warp.
+// N == 32: lane l returns the total of value l.
+// N == 16: lane l returns the total of value l >> 1.
+template <int N>
+__device__ __forceinline__ float reduce_scatter(float (&v)[32], int lane) {
+  if constexpr (N == 32) {
+    rs_step<16, 32>(v, lane);
+    rs_step<8, 16>(v, lane);
+    rs_step<4, 8>(v, lane);
+    rs_step<2, 4>(v, lane);
+    rs_step<1, 2>(v, lane);
+    return v[0];
+  } else {
+    rs_step<16, 16>(v, lane);
+    rs_step<8, 8>(v, lane);
+    rs_step<4, 4>(v, lane);
+    rs_step<2, 2>(v, lane);
+    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+  }
+}
+
+// Load this lane's D/32 elements of a row and widen them.
+template <typename T, int D>
+__device__ __forceinline__ void load_row_slice(const unsigned char* row, int lane, float* out) {
+  if constexpr (D == 128) {
+    const uint2 u = *reinterpret_cast<const uint2*>(row + lane * 8);
+    const float2 a = Elem<T>::to_f2(u.x), b = Elem<T>::to_f2(u.y);
+    out[0] = a.x; out[1] = a.y; out[2] = b.x; out[3] = b.y;
+  } else {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(row + lane * 4);
+    const float2 a = Elem<T>::to_f2(u);
+    out[0] = a.x; out[1] = a.y;
+  }
+}
+
+template <typename T, int D, int G, int NW, int NST>
+__global__ void __launch_bounds__(NW * 32)
+decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v) {
+  using L = DecodeSmem<D, G, NW, NST>;
+  constexpr int VEC = D / 32;
+  constexpr int TPP = (G == 1) ? 16 : 32 / G;  // tokens per reduce-scatter pass
+  constexpr int NPASS = kChunk / TPP;          // passes per chunk
+  constexpr int LPH = (G == 1) ? 32 : 32 / G;  // lanes holding one head's logits
+  extern __shared__ __align__(1024) unsigned char smem[];
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+
+  int bid = blockIdx.x;
+  const int kvh = bid % a.num_kv_heads;
+  bid /= a.num_kv_heads;
+  const int s = bid % a.num_seqs;
+  const int part = bid / a.num_seqs;
+
+  int ctx = __ldg(a.context_lens + s);
+  const int ctx_cap = a.max_context_len;
+  if (ctx < 0 || ctx > ctx_cap) {
+    if (part == 0 && kvh == 0 && threadIdx.x == 0) report(a.err, kErrContextLen);
+    ctx = max(0, min(ctx, ctx_cap));
+  }
+  const int PT = a.partition_tokens;
+  const int q_head0 = kvh * G;
+  if (ctx == 0) {
+    if (part == 0) {
+      uint16_t* o = a.out + ((size_t)s * a.num_q_heads + q_head0) * D;
+      for (int i = threadIdx.x; i < G * D; i += NW * 32) o[i] = 0;
+    }
+    return;
+  }
+  const int t_begin = part * PT;
+  if (t_begin >= ctx) return;
+  const int t_end = min(ctx, t_begin + PT);
+  const int n_parts_seq = (ctx + PT - 1) / PT;
+  const int n_chunks = (t_end - t_begin + kChunk - 1) / kChunk;
+  const int n_mine = warp < n_chunks ? (n_chunks - warp + NW - 1) / NW : 0;
+
+  unsigned char* stages = smem;
+  float* p_all = reinterpret_cast<float*>(smem + L::kStagesBytes);
+  float* p_sm = p_all + warp * (kChunk * G + G);  // [16][G]
+  float* alpha_sm = p_sm + kChunk * G;             // [G]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kStagesBytes + L::kPBytes);
+  const uint32_t bar0 = smem_addr(bars + warp * NST);
+  const uint32_t stage0 = smem_addr(stages + warp * NST * L::kStageBytes);
+
+  if (lane == 0) {
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+#pragma unroll
+    for (int st = 0; st < NST; ++st) mbar_init(bar0 + st * 8, 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
+
+  // Lane k resolves the physical row of this warp's k-th chunk through the
+  // block table (one read per chunk, all issued up front).
+  int my_row = 0;
+  if (lane < n_mine) {
+    const int tok = t_begin + (warp + lane * NW) * kChunk;
+    const int blk = __ldg(a.block_tables + (size_t)s * a.max_blocks_per_seq + tok / a.block_size);
+    if (blk < 0 || blk >= a.num_blocks) {
+      report(a.err, kErrBlockId);
+      my_row = a.num_blocks * a.block_size;  // outside the map: TMA fills zeros
+    } else {
+      my_row = blk * a.block_size + tok % a.block_size;
+    }
+  }
+
+  auto issue = [&](int k) {
+    const int row = __shfl_sync(0xffffffffu, my_row, k);
+    if (lane == 0) {
+      const int st = k % NST;
+      const uint32_t bar = bar0 + st * 8;
+      const uint32_t dst = stage0 + st * L::kStageBytes;
+      mbar_arrive_expect_tx(bar, L::kStageBytes);
+      tma_load_3d(dst, &tm_k, bar, 0, kvh, row);
+      tma_load_3d(dst + kChunk * L::kRowBytes, &tm_v, bar, 0, kvh, row);
+    }
+  };
+
+  // Query group in registers, pre-scaled into the log2 domain.
+  float qr[G][VEC];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const unsigned char* qrow = reinterpret_cast<const unsigned char*>(
+        a.q + ((size_t)s * a.num_q_heads + q_head0 + h) * D);
+    load_row_slice<T, D>(qrow, lane, qr[h]);
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) qr[h][v] *= a.scale_log2;
+  }
+
+  float acc[G][VEC];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) acc[h][v] = 0.f;
+  // Running max / sum of the head this lane's logits belong to.
+  float m_run = -INFINITY, l_run = 0.f;
+  const int my_head = (G == 1) ? 0 : lane / LPH;
+
+  const int n_pro = min(NST, n_mine);
+  for (int k = 0; k < n_pro; ++k) issue(k);
+
+  bool ok = true;
+  int k = 0;
+  for (; k < n_mine; ++k) {
+    const int st = k % NST;
+    if (!mbar_wait(bar0 + st * 8, (k / NST) & 1, a.err)) { ok = false; break; }
+    const unsigned char* Ks = stages + (warp * NST + st) * L::kStageBytes;
+    const unsigned char* Vs = Ks + kChunk * L::kRowBytes;
+    const int tok0 = t_begin + (warp + k * NW) * kChunk;
+    const int n_valid = min(kChunk, t_end - tok0);
+
+    // ---- logits: one complete logit per lane per pass
+    float x[NPASS];
+#pragma unroll
+    for (int ps = 0; ps < NPASS; ++ps) {
+      float part_v[32];
+#pragma unroll
+      for (int jj = 0; jj < TPP; ++jj) {
+        float kf[VEC];
+        load_row_slice<T, D>(Ks + (ps * TPP + jj) * L::kRowBytes, lane, kf);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float d = 0.f;
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) d = fmaf(qr[h][v], kf[v], d);
+          part_v[h * TPP + jj] = d;
+        }
+      }
+      float r = reduce_scatter<(G == 1) ? 16 : 32>(part_v, lane);
+      const int jj = (G == 1) ? (lane >> 1) : (lane % TPP);
+      x[ps] = (ps * TPP + jj < n_valid) ? r : -INFINITY;
+    }
+
+    // ---- online softmax for this lane's head
+    float mx = x[0];
+#pragma unroll
+    for (int ps = 1; ps < NPASS; ++ps) mx = fmaxf(mx, x[ps]);
+    mx = (G == 1) ? warp_max_xor(mx, 2, 16) : warp_max_xor(mx, 1, LPH / 2);
+    const float m_new = fmaxf(m_run, mx);
+    const float alpha = exp2f(m_run - m_new);
+    float ls = 0.f;
+#pragma unroll
+    for (int ps = 0; ps < NPASS; ++ps) {
+      const float p = exp2f(x[ps] - m_new);
+      ls += p;
+      const int jj = (G == 1) ? (lane >> 1) : (lane % TPP);
+      if (G > 1 || (lane & 1) == 0) p_sm[(ps * TPP + jj) * G + my_head] = p;
+    }
+    ls = (G == 1) ? warp_sum_xor(ls, 2, 16) : warp_sum_xor(ls, 1, LPH / 2);
+    l_run = l_run * alpha + ls;
+    m_run = m_new;
+    if (lane % LPH == 0) alpha_sm[my_head] = alpha;
+    __syncwarp();
+
+    // ---- rescale and accumulate P V
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float al = alpha_sm[h];
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc[h][v] *= al;
+    }
+    for (int j = 0; j < n_valid; ++j) {
+      float vf[VEC];
+      load_row_slice<T, D>(Vs + j * L::kRowBytes, lane, vf);
+      float pj[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) pj[h] = p_sm[j * G + h];
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) acc[h][v] = fmaf(pj[h], vf[v], acc[h][v]);
+    }
+    __syncwarp();
+    // Stage `st` is free again: refill it with chunk k + NST.
+    if (k + NST < n_mine) {
+      if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue(k + NST);
+    }
+  }
+  if (!ok) {
+    // Let every copy this warp still has in flight land before the CTA exits.
+    for (int kk = k; kk < min(n_mine, k + NST); ++kk) mbar_wait(bar0 + (kk % NST) * 8, (kk / NST) & 1, a.err);
+  }
+
+  // ---- merge the warps' states
+  // All stages consumed (or drained): the stage area becomes the merge area.
+  const int any_failed = __syncthreads_or(!ok);
+  float* mg = reinterpret_cast<float*>(smem);  // [NW][G] m, [NW][G] l, [NW][G][D] acc
+  float* mg_m = mg;
+  float* mg_l = mg + NW * G;
+  float* mg_acc = mg + 2 * NW * G;
+  if (lane % LPH == 0) {
+    mg_m[warp * G + my_head] = m_run;
+    mg_l[warp * G + my_head] = l_run;
+  }
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) mg_acc[(warp * G + h) * D + lane * VEC + v] = acc[h][v];
+  __syncthreads();
+
+  const bool direct = (n_parts_seq == 1);
+  for (int i = threadIdx.x; i < G * D; i += NW * 32) {
+    const int h = i / D, d = i % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, mg_m[w * G + h]);
+    float num = 0.f, den = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float wt = exp2f(mg_m[w * G + h] - M);  // 0 for a warp without tokens
+      num = fmaf(wt, mg_acc[(w * G + h) * D + d], num);
+      den = fmaf(wt, mg_l[w * G + h], den);
+    }
+    if (any_failed) num = __int_as_float(0x7fc00000), den = 1.f;
+    const size_t qh = (size_t)s * a.num_q_heads + q_head0 + h;
+    if (direct) {
+      a.out[qh * D + d] = Elem<T>::from_f(num / den);
+    } else {
+      const size_t slot = qh * a.num_parts + part;
+      a.ws_acc[slot * D + d] = num;
+      if (d == 0) {
+        a.ws_ml[2 * slot] = M;
+        a.ws_ml[2 * slot + 1] = den;
+      }
+    }
+  }
+}
+
+// Merge of the partitions of every (sequence, query head) that has more than
+// one.  One warp per (sequence, query head); lane l owns dims [l*VEC, l*VEC+VEC).
+template <typename T, int D>
+__global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a) {
+  constexpr int VEC = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int pair = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (pair >= a.num_seqs * a.num_q_heads) return;
+  const int s = pair / a.num_q_heads;
+  int ctx = __ldg(a.context_lens + s);
+  ctx = max(0, min(ctx, a.max_context_len));
+  const int P = (ctx + a.partition_tokens - 1) / a.partition_tokens;
+  if (P <= 1) return;
+  const size_t base = (size_t)pair * a.num_parts;
+  float M = -INFINITY;
+  for (int p = 0; p < P; ++p) M = fmaxf(M, a.ws_ml[2 * (base + p)]);
+  float num[VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) num[v] = 0.f;
+  float den = 0.f;
+  for (int p = 0; p < P; ++p) {
+    const float wt = exp2f(a.ws_ml[2 * (base + p)] - M);
+    den = fmaf(wt, a.ws_ml[2 * (base + p) + 1], den);
+    const float* row = a.ws_acc + (base + p) * D + lane * VEC;
+    if constexpr (VEC == 4) {
+      const float4 r = *reinterpret_cast<const float4*>(row);
+      num[0] = fmaf(wt, r.x, num[0]); num[1] = fmaf(wt, r.y, num[1]);
+      num[2] = fmaf(wt, r.z, num[2]); num[3] = fmaf(wt, r.w, num[3]);
+    } else {
+      const float2 r = *reinterpret_cast<const float2*>(row);
+      num[0] = fmaf(wt, r.x, num[0]); num[1] = fmaf(wt, r.y, num[1]);
+    }
+  }
+  const float inv = 1.f / den;
+  uint16_t* o = a.out + (size_t)pair * D + lane * VEC;
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) o[v] = Elem<T>::from_f(num[v] * inv);
+}
+
+// ---------------------------------------------------------------------------
+// host side
+
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kStages = 3;
+
+template <typename T, int D, int G>
+cudaError_t launch_typed(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                         int grid, cudaStream_t stream, int* launches) {
+  using L = DecodeSmem<D, G, kWarps, kStages>;
+  auto* kern = decode_partition_kernel<T, D, G, kWarps, kStages>;
+  static bool configured = false;  // per instantiation; idempotent if raced
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  kern<<<grid, kWarps * 32, L::kTotal, stream>>>(a, tk, tv);
+  ++*launches;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || a.num_parts <= 1) return e;
+  const int pairs = a.num_seqs * a.num_q_heads;
+  decode_merge_kernel<T, D><<<(pairs + 3) / 4, 128, 0, stream>>>(a);
+  ++*launches;
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_group(const DecodeArgs& a, int G, const CUtensorMap& tk, const CUtensorMap& tv,
+                         int grid, cudaStream_t st, int* n) {
+  switch (G) {
+    case 1: return launch_typed<T, D, 1>(a, tk, tv, grid, st, n);
+    case 2: return launch_typed<T, D, 2>(a, tk, tv, grid, st, n);
+    case 4: return launch_typed<T, D, 4>(a, tk, tv, grid, st, n);
+    case 8: return launch_typed<T, D, 8>(a, tk, tv, grid, st, n);
+    case 16: return launch_typed<T, D, 16>(a, tk, tv, grid, st, n);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeArgs& a, int dtype, int head_dim, int group,
+                          const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream,
+                          int* launches) {
+  const long long grid = (long long)a.num_parts * a.num_seqs * a.num_kv_heads;
+  if (grid <= 0) return cudaSuccess;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  if (dtype == 0) {
+    if (head_dim == 128) return launch_group<__half, 128>(a, group, tk, tv, (int)grid, stream, launches);
+    return launch_group<__half, 64>(a, group, tk, tv, (int)grid, stream, launches);
+  }
+  if (head_dim == 128) return launch_group<__nv_bfloat16, 128>(a, group, tk, tv, (int)grid, stream, launches);
+  return launch_group<__nv_bfloat16, 64>(a, group, tk, tv, (int)grid, stream, launches);
+}
+
+int decode_chunk_tokens() { return kChunk; }
+int decode_max_partition_tokens() { return kChunk * kWarps * 32; }
+
+}  // namespace pa

@@ -1,0 +1,42 @@
+// pa_internal.h -- declarations shared by the libpa host code and its kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pa {
+
+// Arguments of the decode kernels (device pointers, host-validated sizes).
+struct DecodeArgs {
+  const uint16_t* q;             // [S][Hq][D]
+  const int32_t* block_tables;   // [S][MBS]
+  const int32_t* context_lens;   // [S]
+  uint16_t* out;                 // [S][Hq][D]
+  float* ws_acc;                 // [S][Hq][num_parts][D] (split-K only)
+  float* ws_ml;                  // [S][Hq][num_parts][2] (split-K only)
+  float scale_log2;              // scale * log2(e)
+  int num_seqs, num_q_heads, num_kv_heads;
+  int block_size, num_blocks, max_blocks_per_seq;
+  int partition_tokens, num_parts;
+  int max_context_len;           // host bound on context_lens, <= max_blocks_per_seq * block_size
+  unsigned int* err;             // device error word
+};
+
+// Launch the partition kernel (+ the merge kernel when num_parts > 1).
+// `launches` is incremented once per kernel launched.
+cudaError_t launch_decode(const DecodeArgs& a, int dtype, int head_dim, int group,
+                          const CUtensorMap& tm_k, const CUtensorMap& tm_v, cudaStream_t stream,
+                          int* launches);
+int decode_chunk_tokens();
+int decode_max_partition_tokens();
+
+cudaError_t launch_cache_append(const void* k, const void* v, const int32_t* slot_mapping,
+                                int num_tokens, void* k_cache, void* v_cache, long long num_slots,
+                                int row_bytes, unsigned int* err, cudaStream_t stream,
+                                int* launches);
+cudaError_t launch_copy_blocks(const int32_t* pairs, int num_pairs, void* k_cache, void* v_cache,
+                               int num_blocks, long long block_bytes, unsigned int* err,
+                               cudaStream_t stream, int* launches);
+
+}  // namespace pa

@@ -1,0 +1,233 @@
+"""The C ABI without a GPU: symbols, host-side validation, host allocator."""
+import ctypes
+
+import numpy as np
+import pytest
+
+from paged_kv_cache_458_b200 import gen, pa
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_458_b200 import build
+
+    build.build()
+    return pa.lib()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = pa.header_functions()
+    assert {"pa_decode", "pa_cache_append", "pa_copy_blocks", "pa_decode_workspace_bytes"} <= set(names)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, f"declared in include/pa.h but not exported: {missing}"
+
+
+def test_status_strings(lib):
+    for st in range(6):
+        assert pa.status_string(st) and pa.status_string(st) != "unknown status"
+    assert lib.pa_status_string(99) == b"unknown status"
+    assert "sm_100a" in pa.pa_build_info()
+
+
+def _shape(**kw):
+    base = dict(num_seqs=4, num_q_heads=8, num_kv_heads=2, head_dim=128, block_size=16,
+                num_blocks=64, max_blocks_per_seq=8, partition_tokens=0, dtype=pa.PA_F16)
+    base.update(kw)
+    return pa.make_shape(**base)
+
+
+FAKE = 1 << 20  # a 16-byte-aligned non-null address; validation fails before any use
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(head_dim=96), pa.PA_ERR_UNSUPPORTED),
+    (dict(head_dim=0), pa.PA_ERR_INVALID_ARG),
+    (dict(num_q_heads=8, num_kv_heads=3), pa.PA_ERR_INVALID_ARG),
+    (dict(num_q_heads=64, num_kv_heads=2), pa.PA_ERR_UNSUPPORTED),  # group 32
+    (dict(block_size=8), pa.PA_ERR_UNSUPPORTED),
+    (dict(dtype=7), pa.PA_ERR_UNSUPPORTED),
+    (dict(partition_tokens=24), pa.PA_ERR_UNSUPPORTED),
+    (dict(partition_tokens=4096), pa.PA_ERR_UNSUPPORTED),
+    (dict(num_blocks=1 << 27), pa.PA_ERR_UNSUPPORTED),      # num_blocks * block_size >= 2^31
+    (dict(num_seqs=-1), pa.PA_ERR_INVALID_ARG),
+])
+def test_decode_rejects_bad_shapes(lib, kw, expect):
+    s = _shape(**kw)
+    st = lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s), 100, FAKE, 1 << 20, None)
+    assert st == expect
+
+
+def test_decode_rejects_bad_pointers_and_sizes(lib):
+    s = _shape()
+    call = lambda **o: lib.pa_decode(  # noqa: E731
+        o.get("q", FAKE), FAKE, FAKE, o.get("bt", FAKE), FAKE, o.get("scale", 0.1), FAKE,
+        ctypes.byref(s), o.get("maxlen", 100), o.get("ws", FAKE), o.get("wsb", 1 << 20), None)
+    assert call(q=None) == pa.PA_ERR_INVALID_ARG
+    assert call(q=FAKE + 8) == pa.PA_ERR_INVALID_ARG            # misaligned
+    assert call(bt=FAKE + 2) == pa.PA_ERR_INVALID_ARG
+    assert call(scale=float("nan")) == pa.PA_ERR_INVALID_ARG
+    assert call(maxlen=8 * 16 + 1) == pa.PA_ERR_INVALID_ARG     # beyond max_blocks_per_seq * bs
+    assert call(maxlen=-1) == pa.PA_ERR_INVALID_ARG
+    # 100 tokens fit one 512-token partition: no workspace needed ...
+    assert lib.pa_decode_workspace_bytes(ctypes.byref(s), 100) == 0
+    # ... 1000 tokens need two partitions and a workspace
+    s2 = _shape(max_blocks_per_seq=64)
+    need = lib.pa_decode_workspace_bytes(ctypes.byref(s2), 1000)
+    assert need >= 4 * 8 * 2 * (128 + 2) * 4
+    st = lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s2), 1000, FAKE, need - 1, None)
+    assert st == pa.PA_ERR_INVALID_ARG
+    st = lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s2), 1000, None, 0, None)
+    assert st == pa.PA_ERR_INVALID_ARG
+
+
+def test_empty_batches_launch_nothing(lib):
+    before = pa.pa_kernel_launches()
+    s = _shape(num_seqs=0)
+    assert lib.pa_decode(None, None, None, None, None, 0.1, None, ctypes.byref(s), 0, None, 0, None) == 0
+    assert lib.pa_cache_append(None, None, None, 0, None, None, ctypes.byref(_shape()), None) == 0
+    assert lib.pa_copy_blocks(None, 0, None, None, ctypes.byref(_shape()), None) == 0
+    assert pa.pa_kernel_launches() == before
+
+
+def test_append_and_copy_reject_bad_arguments(lib):
+    s = _shape()
+    assert lib.pa_cache_append(FAKE, FAKE, FAKE, -1, FAKE, FAKE, ctypes.byref(s), None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_cache_append(None, FAKE, FAKE, 3, FAKE, FAKE, ctypes.byref(s), None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_cache_append(FAKE, FAKE, FAKE, 3, FAKE + 4, FAKE, ctypes.byref(s), None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_copy_blocks(FAKE, -2, FAKE, FAKE, ctypes.byref(s), None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_copy_blocks(None, 2, FAKE, FAKE, ctypes.byref(s), None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_copy_blocks(FAKE, 70000, FAKE, FAKE, ctypes.byref(s), None) == pa.PA_ERR_UNSUPPORTED
+    bad = _shape(head_dim=80)
+    assert lib.pa_copy_blocks(FAKE, 1, FAKE, FAKE, ctypes.byref(bad), None) == pa.PA_ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------- allocator
+
+
+def _apply(ops, mgr_py, mgr_c, max_blocks):
+    """Run the same operation list on both managers and compare state."""
+    for op in ops:
+        kind = op[0]
+        if kind == "add":
+            mgr_py.add_seq(op[1], op[2])
+            mgr_c.add_seq(op[1], op[2])
+        elif kind == "fork":
+            mgr_py.fork(op[1], op[2])
+            mgr_c.fork(op[1], op[2])
+        elif kind == "free":
+            mgr_py.free_seq(op[1])
+            mgr_c.free_seq(op[1])
+        elif kind == "append":
+            seqs = op[1]
+            exp_slots, exp_pairs = [], []
+            for s in seqs:
+                slot, pair = mgr_py.append_slot(s)
+                exp_slots.append(slot)
+                if pair is not None:
+                    exp_pairs.append(pair)
+            slots, pairs = mgr_c.append_slots(seqs)
+            assert slots.tolist() == exp_slots
+            assert [tuple(p) for p in pairs.tolist()] == exp_pairs
+        seqs = sorted(mgr_py.tables)
+        if seqs:
+            t, lens = mgr_c.block_tables(seqs, max_blocks)
+            assert np.array_equal(t, mgr_py.table_array(seqs, max_blocks))
+            assert lens.tolist() == [mgr_py.lens[s] for s in seqs]
+        assert mgr_c.num_free() == len(mgr_py.free)
+        for b in range(mgr_py.num_blocks):
+            assert mgr_c.refcount(b) == mgr_py.ref[b]
+
+
+def test_allocator_matches_generator_block_manager(lib):
+    rng = np.random.default_rng(7)
+    NB, bs = 96, 16
+    order = rng.permutation(NB)
+    py = gen.BlockManager(NB, bs, order)
+    c = pa.Allocator(NB, bs, order)
+    ops, live, nxt = [], [], 0
+    for _ in range(300):
+        r = rng.random()
+        if r < 0.25 or not live:
+            ops.append(("add", nxt, int(rng.integers(0, 40))))
+            live.append(nxt)
+            nxt += 1
+        elif r < 0.4:
+            ops.append(("fork", int(rng.choice(live)), nxt))
+            live.append(nxt)
+            nxt += 1
+        elif r < 0.5 and len(live) > 1:
+            s = int(rng.choice(live))
+            ops.append(("free", s))
+            live.remove(s)
+        else:
+            k = int(rng.integers(1, min(6, len(live)) + 1))
+            ops.append(("append", [int(x) for x in rng.choice(live, size=k, replace=False)]))
+        try:
+            _apply(ops[-1:], py, c, 64)
+        except MemoryError:
+            break  # the Python side ran out first; the C side is checked below
+    c.close()
+
+
+def test_allocator_beam_workload_matches_generator(lib):
+    """The beam workload's per-step host operations through the C allocator."""
+    case = gen.make_case("llama2_70b_beam", n_steps=3, with_pool=False, num_seqs=32)
+    c = pa.Allocator(case.num_blocks, case.block_size, case.structure["pool_order"])
+    ctx = case.structure["initial_context_lens"]
+    bs = case.block_size
+    for g in range(8):
+        L = int(ctx[4 * g])
+        shared = ((L - 1) // bs) * bs
+        c.add_seq(4 * g, shared)
+        for k in range(1, 4):
+            c.fork(4 * g, 4 * g + k)
+        for k in range(4):
+            c.extend(4 * g + k, L - shared)
+    seqs = list(range(32))
+    t, lens = c.block_tables(seqs, case.max_blocks_per_seq)
+    assert np.array_equal(t, case.block_tables) and np.array_equal(lens, case.context_lens)
+    for st in case.steps:
+        for g in range(8):
+            for k in range(1, 4):
+                c.free_seq(4 * g + k)
+                c.fork(4 * g, 4 * g + k)
+        slots, pairs = c.append_slots(seqs)
+        assert np.array_equal(slots, st.slot_mapping)
+        assert np.array_equal(pairs, st.pairs)
+        t, lens = c.block_tables(seqs, case.max_blocks_per_seq)
+        assert np.array_equal(t, st.block_tables) and np.array_equal(lens, st.context_lens)
+    c.close()
+
+
+def test_allocator_out_of_blocks_changes_nothing(lib):
+    c = pa.Allocator(3, 16)
+    c.add_seq(0, 16)
+    c.add_seq(1, 16)
+    c.add_seq(2, 5)
+    before = c.block_tables([0, 1, 2], 4)
+    with pytest.raises(pa.PaError) as e:
+        c.append_slots([2, 0, 1])       # 0 and 1 each need a new block; only 0 free
+    assert e.value.status == pa.PA_ERR_OOM
+    after = c.block_tables([0, 1, 2], 4)
+    assert all(np.array_equal(x, y) for x, y in zip(before, after))
+    assert c.num_free() == 0
+    with pytest.raises(pa.PaError):
+        c.add_seq(3, 1)
+    c.close()
+
+
+def test_allocator_rejects_bad_input(lib):
+    assert not lib.pa_alloc_create(4, 16, (ctypes.c_int32 * 4)(0, 1, 1, 3))
+    assert not lib.pa_alloc_create(0, 16, None)
+    c = pa.Allocator(4, 16)
+    with pytest.raises(pa.PaError):
+        c.fork(5, 6)
+    c.add_seq(1, 3)
+    with pytest.raises(pa.PaError):
+        c.add_seq(1, 3)
+    with pytest.raises(pa.PaError):
+        c.append_slots([1, 1])
+    with pytest.raises(pa.PaError):
+        c.block_tables([1, 9], 4)
+    assert c.refcount(-1) == -1 and c.refcount(4) == -1
+    c.close()

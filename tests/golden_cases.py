@@ -44,14 +44,14 @@ def build(case):
         expected = (V0 + 3 * V1) / 4
     elif case["name"] == "crossing_into_second_block":
         for j in range(16):
-            put(7, j, np.zeros(D), j + d / 64)
-        put(2, 0, e0, 16 + d / 64)
-        expected = 168.0 / 19.0 + d / 64
+            put(7, j, np.zeros(D), (j + d / 64) / 8)
+        put(2, 0, e0, (16 + d / 64) / 8)
+        expected = 47.0 / 32.0 + d / 512
     else:  # pragma: no cover
         raise KeyError(case["name"])
     table = np.array([case["block_table"]], dtype=np.int32)
     ctx = np.array([case["context_len"]], dtype=np.int32)
     q = gen.f32_to_f16_bits(e0.astype(np.float32)).reshape(1, 1, D)
-    assert case["scale"] == "ln(3)"
+    scale = {"ln(3)": math.log(3.0), "ln(16)": math.log(16.0)}[case["scale"]]
     return dict(dtype=dtype, q=q, k_cache=kc, v_cache=vc, block_tables=table,
-                context_lens=ctx, scale=math.log(3.0), expected=expected.reshape(1, 1, D))
+                context_lens=ctx, scale=scale, expected=expected.reshape(1, 1, D))

@@ -129,6 +129,42 @@ pa_status pa_decode(const void *q, const void *k_cache, const void *v_cache,
                     void *workspace, size_t workspace_bytes, pa_stream_t stream);
 
 /*
+ * pa_decode for callers that cannot allocate device memory.
+ *
+ * The paper has no counterpart to this call (it is not part of the method);
+ * it exists for callers of this library that have no way to allocate the
+ * split-K workspace pa_decode needs:
+ * a plug-in running inside a host runtime that owns all device memory and
+ * gives its plug-ins no allocator, or a decode loop that must not call
+ * cudaMalloc (which can synchronise the whole device) once it is running.
+ *
+ * Same arguments and result as pa_decode, minus the workspace: the split-K
+ * scratch comes from one fixed array compiled into the library.  Nothing here
+ * calls cudaMalloc, cudaFree or any allocating routine.
+ *  - Limit: PA_NOALLOC_SCRATCH_BYTES per device.  Every GPU that loads the
+ *    library holds that much device memory for the array until the process
+ *    exits.  A call whose workspace (pa_decode_workspace_bytes for the same
+ *    shape and max_context_len: num_seqs * num_q_heads * partitions *
+ *    (head_dim + 2) * 4 bytes, rounded) exceeds the limit returns
+ *    PA_ERR_UNSUPPORTED and launches nothing; pa_decode with a caller-owned
+ *    workspace has no such limit.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) and caches it; make that first call before any
+ *    stream capture on that device.  It returns PA_ERR_CUDA if the lookup
+ *    fails.
+ *  - Every call on a device shares the one array and finds the previous
+ *    call's contents in it; nothing in it has to start at zero, because each
+ *    call writes every scratch slot it later reads.  Calls whose kernels can
+ *    overlap on the GPU (different streams without ordering between them)
+ *    race on the array: order them, or use pa_decode with separate workspaces.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+pa_status pa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *block_tables, const int32_t *context_lens, float scale,
+                            void *out, const pa_shape *shape, int32_t max_context_len,
+                            pa_stream_t stream);
+
+/*
  * Append one new token per entry into the cache (the "update KV cache" step of
  * each decode iteration, 5688vip.com section 2.1): for t < num_tokens with
  * slot = slot_mapping[t] >= 0,

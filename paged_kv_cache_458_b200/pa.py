@@ -57,6 +57,8 @@ def _declare(lib):
     lib.pa_decode_workspace_bytes.argtypes = [SP, I32]
     lib.pa_decode.restype = c.c_int
     lib.pa_decode.argtypes = [P, P, P, P, P, c.c_float, P, SP, I32, P, SZ, P]
+    lib.pa_decode_noalloc.restype = c.c_int
+    lib.pa_decode_noalloc.argtypes = [P, P, P, P, P, c.c_float, P, SP, I32, P]
     lib.pa_cache_append.restype = c.c_int
     lib.pa_cache_append.argtypes = [P, P, P, I32, P, P, SP, P]
     lib.pa_copy_blocks.restype = c.c_int
@@ -171,6 +173,18 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale: float, out
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
         float(scale), _ptr(out), ctypes.byref(shape), int(max_context_len), _ptr(workspace),
         int(workspace_bytes), _stream(stream)))
+
+
+def pa_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale: float, out,
+                      shape: pa_shape, max_context_len: int, stream=None) -> None:
+    """pa_decode with its split-K scratch taken from a fixed array inside the
+    library, for callers that cannot allocate device memory (see pa.h)."""
+    _check("pa_decode_noalloc", lib().pa_decode_noalloc(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+        float(scale), _ptr(out), ctypes.byref(shape), int(max_context_len), _stream(stream)))
+
+
+PA_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 def pa_cache_append(k, v, slot_mapping, num_tokens: int, k_cache, v_cache, shape: pa_shape,

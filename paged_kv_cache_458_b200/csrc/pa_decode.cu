@@ -392,8 +392,16 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a) {
 
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kStages = 3;
+// Warps per CTA and TMA stages per warp (build-time choices; 4 x 2 keeps
+// three CTAs resident per SM, which measured fastest on every workload).
+#ifndef PA_DECODE_WARPS
+#define PA_DECODE_WARPS 4
+#endif
+#ifndef PA_DECODE_STAGES
+#define PA_DECODE_STAGES 2
+#endif
+constexpr int kWarps = PA_DECODE_WARPS;
+constexpr int kStages = PA_DECODE_STAGES;
 
 template <typename T, int D, int G>
 cudaError_t launch_typed(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,

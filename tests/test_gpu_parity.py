@@ -120,7 +120,7 @@ def test_edge_contexts(orc, dtype, head_dim, group):
 
 
 @pytest.mark.parametrize("block_size", [16, 32, 256])
-@pytest.mark.parametrize("partition_tokens", [16, 48, 256, 512, 2048])
+@pytest.mark.parametrize("partition_tokens", [16, 48, 128, 512, 2048])
 def test_block_and_partition_sizes(orc, block_size, partition_tokens):
     rng = np.random.default_rng(block_size * 7 + partition_tokens)
     ctx = [1, 47, 48, 49, 255, 256, 257, 700, 2048, 2100]
@@ -255,13 +255,36 @@ def test_device_checks_report_and_skip():
 
 def test_launch_counter_counts_kernels():
     rng = np.random.default_rng(9)
-    c = gen.random_decode_case(rng, num_seqs=2, num_q_heads=2, num_kv_heads=2, head_dim=64,
-                               block_size=16, dtype=gen.F16, context_lens=[600, 10])
-    n0 = pa.pa_kernel_launches()
-    gpu_decode(gen.F16, c["q"], c["k_cache"], c["v_cache"], c["block_tables"], c["context_lens"],
-               c["scale"])
-    assert pa.pa_kernel_launches() - n0 == 2   # partition kernel + merge kernel
-    n1 = pa.pa_kernel_launches()
-    gpu_decode(gen.F16, c["q"], c["k_cache"], c["v_cache"], c["block_tables"], c["context_lens"],
-               c["scale"], partition_tokens=1024)
-    assert pa.pa_kernel_launches() - n1 == 1   # one partition: no merge
+    for ctx, pt, kernels in (([600, 10], 256, 2), ([200, 10], 256, 1)):
+        c = gen.random_decode_case(rng, num_seqs=2, num_q_heads=2, num_kv_heads=2, head_dim=64,
+                                   block_size=16, dtype=gen.F16, context_lens=ctx)
+        n0 = pa.pa_kernel_launches()
+        gpu_decode(gen.F16, c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
+                   c["context_lens"], c["scale"], partition_tokens=pt)
+        # partition kernel, plus the split-K merge kernel when a context spans partitions
+        assert pa.pa_kernel_launches() - n0 == kernels
+
+
+def test_workspace_needs_no_initialisation(orc):
+    """Split-K counters carry a per-call tag: garbage or a previous call's
+    values in the workspace must not change the result."""
+    rng = np.random.default_rng(10)
+    ws = torch.full((8 << 20,), 0xFF, dtype=torch.uint8, device="cuda")
+    for trial, (ctx, g) in enumerate((([1500, 700, 33, 2600], 4), ([513, 1024, 4000], 8),
+                                      ([1500, 700, 33, 2600], 4))):
+        c = gen.random_decode_case(rng, num_seqs=len(ctx), num_q_heads=2 * g, num_kv_heads=2,
+                                   head_dim=128, block_size=16, dtype=gen.BF16, context_lens=ctx)
+        shape = shape_of(gen.BF16, c["q"], c["k_cache"], c["block_tables"])
+        maxlen = int(max(ctx))
+        wsb = pa.pa_decode_workspace_bytes(shape, maxlen)
+        assert 0 < wsb <= ws.numel()
+        if trial == 2:
+            ws[:wsb].random_(0, 256)
+        out = torch.empty(c["q"].shape, dtype=torch.bfloat16, device="cuda")
+        pa.pa_decode(dev(c["q"], gen.BF16), dev(c["k_cache"], gen.BF16), dev(c["v_cache"], gen.BF16),
+                     dev_i32(c["block_tables"]), dev_i32(c["context_lens"]), c["scale"], out, shape,
+                     maxlen, ws, wsb)
+        assert pa.pa_last_device_error()[0] == pa.PA_OK
+        ref = orc.decode(gen.BF16, c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
+                         c["context_lens"], c["scale"])
+        assert_decode_close(host_bits(out), ref, gen.BF16, f"trial {trial}")

@@ -91,14 +91,32 @@ typedef struct {
   int32_t num_blocks;
   int32_t max_blocks_per_seq;
   int32_t partition_tokens;
-  int32_t dtype; /* pa_dtype */
+  int32_t dtype;   /* pa_dtype */
+  int32_t variant; /* pa_decode_variant (pa_decode only; 0 = automatic) */
 } pa_shape;
 
+/* How pa_decode computes QK^T and PV.  Both variants read K/V with tiled TMA
+ * loads through the block table and keep the softmax in fp32.
+ *  PA_DECODE_AUTO          tensor cores when head_dim == 128, the group
+ *                          g = Hq / Hkv is at least 8 and partition_tokens is
+ *                          a multiple of 128 up to 512; CUDA cores otherwise.
+ *  PA_DECODE_CUDA_CORES    fp32 FMA on the CUDA cores (any built shape).
+ *  PA_DECODE_TENSOR_CORES  tcgen05 MMA with the g heads padded to 16: fp16/bf16
+ *                          operands (the probabilities are rounded to the
+ *                          input type before the PV product), fp32
+ *                          accumulators in tensor memory.  Needs head_dim 128
+ *                          and partition_tokens a multiple of 128 (else
+ *                          PA_ERR_UNSUPPORTED). */
+typedef enum { PA_DECODE_AUTO = 0, PA_DECODE_CUDA_CORES = 1, PA_DECODE_TENSOR_CORES = 2 } pa_decode_variant;
+
 /* Bytes of device workspace pa_decode() needs for `shape` when no context is
- * longer than `max_context_len` tokens (0 when one partition covers every
- * context).  The workspace holds, per (sequence, query head, partition), the
- * running max, the softmax sum and the unnormalised output row in fp32; it
- * needs no initialisation and is dead after the call's kernels finish. */
+ * longer than `max_context_len` tokens: 256 bytes for the work counter the
+ * tensor-core variant's persistent CTAs take items from, plus, when a context
+ * spans more than one partition, per (sequence, query head, partition) the
+ * running max, the softmax sum and the unnormalised output row in fp32.  The
+ * workspace needs no initialisation (the counter carries a per-call tag, so a
+ * value left by an earlier call is recognised and replaced) and is dead after
+ * the call's kernels finish.  Returns 0 for an invalid shape. */
 size_t pa_decode_workspace_bytes(const pa_shape *shape, int32_t max_context_len);
 
 /*
@@ -113,14 +131,16 @@ size_t pa_decode_workspace_bytes(const pa_shape *shape, int32_t max_context_len)
  * beyond ctx are never read, so they may hold anything (including NaN).
  *
  * Contexts are cut into partitions of shape->partition_tokens tokens; each
- * (sequence, kv head, partition) is one CTA, and sequences with more than
- * one partition are merged by a second kernel (log-sum-exp rule).
+ * (sequence, kv head, partition) is one work item (one CTA on the CUDA-core
+ * variant; items taken by one persistent CTA per SM on the tensor-core
+ * variant), and sequences with more than one partition are merged by a
+ * second kernel (log-sum-exp rule).  shape->variant picks the arithmetic.
  *
  * q, k_cache, v_cache, block_tables, context_lens, out: device, layouts above.
  * max_context_len: host-side upper bound on every context_lens[s]; it sizes the
  *   grid.  A larger device value is clamped and reported (PA_DEVERR_CONTEXT_LEN).
  * workspace: device, at least pa_decode_workspace_bytes(shape, max_context_len)
- *   bytes (may be NULL when that is 0).  It must not be shared with a decode
+ *   bytes, 16-byte aligned, never NULL.  It must not be shared with a decode
  *   that runs concurrently.
  */
 pa_status pa_decode(const void *q, const void *k_cache, const void *v_cache,
@@ -144,7 +164,7 @@ pa_status pa_decode(const void *q, const void *k_cache, const void *v_cache,
  *  - Limit: PA_NOALLOC_SCRATCH_BYTES per device.  Every GPU that loads the
  *    library holds that much device memory for the array until the process
  *    exits.  A call whose workspace (pa_decode_workspace_bytes for the same
- *    shape and max_context_len: num_seqs * num_q_heads * partitions *
+ *    shape and max_context_len: 256 + num_seqs * num_q_heads * partitions *
  *    (head_dim + 2) * 4 bytes, rounded) exceeds the limit returns
  *    PA_ERR_UNSUPPORTED and launches nothing; pa_decode with a caller-owned
  *    workspace has no such limit.

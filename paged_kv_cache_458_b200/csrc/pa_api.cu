@@ -66,7 +66,38 @@ pa_status check_decode_shape(const pa_shape* s, int32_t max_context_len) {
   const int pt = effective_partition(s);
   if (pt < 16 || pt % 16 != 0 || pt > pa::decode_max_partition_tokens()) return PA_ERR_UNSUPPORTED;
   if ((long long)s->num_seqs * s->num_q_heads * s->head_dim >= (1LL << 40)) return PA_ERR_INVALID_ARG;
+  if (s->variant < PA_DECODE_AUTO || s->variant > PA_DECODE_TENSOR_CORES) return PA_ERR_INVALID_ARG;
+  if (s->variant == PA_DECODE_TENSOR_CORES &&
+      (s->head_dim != 128 || pt % pa::decode_tc_tile_tokens() != 0 || pt > 512))
+    return PA_ERR_UNSUPPORTED;
+  // work items of one launch (<= 512 sequences) must fit the 24-bit counter
+  const long long parts = ((long long)max_context_len + pt - 1) / pt;
+  if (512LL * s->num_kv_heads * (parts > 0 ? parts : 1) >= (1LL << 23)) return PA_ERR_UNSUPPORTED;
   return PA_OK;
+}
+
+// Whether pa_decode runs the tensor-core variant for this (valid) shape.
+bool use_tensor_cores(const pa_shape* s) {
+  if (s->variant == PA_DECODE_TENSOR_CORES) return true;
+  if (s->variant == PA_DECODE_CUDA_CORES) return false;
+  const int pt = effective_partition(s);
+  // measured: tensor cores win from group 8 up; at group 4 the CUDA-core
+  // kernel still keeps up with HBM
+  return s->head_dim == 128 && s->num_q_heads / s->num_kv_heads >= 8 &&
+         pt % pa::decode_tc_tile_tokens() == 0 && pt <= 512;
+}
+
+// Workspace: the work counter (8 bytes used of 256), then, for split-K,
+// partial outputs [S][Hq][P][D] and (max, sum) pairs [S][Hq][P][2] in fp32.
+constexpr long long kCounterBytes = 256;
+
+// Tags of decode launches (see the work counter in pa_decode_tc.cu): unique
+// per launch, never 0, below 2^40.
+std::atomic<uint64_t> g_epoch{1};
+uint64_t next_epochs(int n) {
+  uint64_t e = g_epoch.fetch_add((uint64_t)n, std::memory_order_relaxed) & ((1ull << 40) - 1);
+  if (e == 0 || e + (uint64_t)n >= (1ull << 40)) e = 1;
+  return e;
 }
 
 int num_partitions(const pa_shape* s, int32_t max_context_len) {
@@ -106,6 +137,32 @@ bool make_pool_map(CUtensorMap* map, const void* pool, const pa_shape* s, int ro
   return r == CUDA_SUCCESS;
 }
 
+// Maps of the tensor-core variant: pools viewed as [NB * bs][Hkv][128] with
+// 128B-swizzled boxes of 64 elements x 16 token rows; q viewed as
+// [S * Hq][128] with 128B-swizzled boxes of 64 elements x `group` rows.
+bool make_tc_maps(CUtensorMap* tk, CUtensorMap* tv, CUtensorMap* tq, const void* k, const void* v,
+                  const void* q, const pa_shape* s) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {128, (cuuint64_t)s->num_kv_heads, (cuuint64_t)s->num_blocks * s->block_size};
+  const cuuint64_t strides[2] = {256, (cuuint64_t)s->num_kv_heads * 256};
+  const cuuint32_t box[3] = {64, 1, 16};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  for (int i = 0; i < 2; ++i) {
+    CUresult r = fn(i ? tv : tk, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(i ? v : k), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+  }
+  const cuuint64_t qdims[2] = {128, (cuuint64_t)s->num_seqs * s->num_q_heads};
+  const cuuint64_t qstrides[1] = {256};
+  const cuuint32_t qbox[2] = {64, (cuuint32_t)(s->num_q_heads / s->num_kv_heads)};
+  const cuuint32_t qestr[2] = {1, 1};
+  return fn(tq, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(q), qdims, qstrides, qbox, qestr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 extern "C" {
@@ -113,11 +170,11 @@ extern "C" {
 size_t pa_decode_workspace_bytes(const pa_shape* shape, int32_t max_context_len) {
   if (check_decode_shape(shape, max_context_len) != PA_OK) return 0;
   const long long P = num_partitions(shape, max_context_len);
-  if (P <= 1) return 0;
+  if (P <= 1) return (size_t)kCounterBytes;
   const long long rows = (long long)shape->num_seqs * shape->num_q_heads * P;
   const long long acc = rows * shape->head_dim * 4;
   const long long ml = rows * 2 * 4;
-  return (size_t)(((acc + 255) / 256) * 256 + ml);
+  return (size_t)(kCounterBytes + ((acc + 255) / 256) * 256 + ml);
 }
 
 pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
@@ -134,8 +191,7 @@ pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
     return PA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
   const size_t need = pa_decode_workspace_bytes(shape, max_context_len);
-  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
-    return PA_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_INVALID_ARG;
   if (max_context_len > (long long)shape->max_blocks_per_seq * shape->block_size)
     return PA_ERR_INVALID_ARG;
 
@@ -145,11 +201,12 @@ pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.out = static_cast<uint16_t*>(out);
-  if (need > 0) {
+  a.work_counter = static_cast<unsigned long long*>(workspace);
+  if (P > 1) {
     const long long rows = (long long)shape->num_seqs * shape->num_q_heads * P;
-    a.ws_acc = static_cast<float*>(workspace);
-    a.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                       ((rows * shape->head_dim * 4 + 255) / 256) * 256);
+    char* base = static_cast<char*>(workspace) + kCounterBytes;
+    a.ws_acc = reinterpret_cast<float*>(base);
+    a.ws_ml = reinterpret_cast<float*>(base + ((rows * shape->head_dim * 4 + 255) / 256) * 256);
   }
   a.scale_log2 = scale * 1.4426950408889634f;
   a.num_seqs = shape->num_seqs;
@@ -164,21 +221,30 @@ pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
   a.err = error_word();
   if (!a.err) return PA_ERR_CUDA;
 
-  CUtensorMap tk, tv;
-  if (shape->num_blocks > 0) {
-    if (!make_pool_map(&tk, k_cache, shape, pa::decode_chunk_tokens()) ||
-        !make_pool_map(&tv, v_cache, shape, pa::decode_chunk_tokens()))
-      return PA_ERR_CUDA;
-  } else {
-    // An empty pool can only serve empty contexts; the kernels issue no load.
-    if (max_context_len > 0) return PA_ERR_INVALID_ARG;
-    memset(&tk, 0, sizeof tk);
-    memset(&tv, 0, sizeof tv);
-  }
+  if (shape->num_blocks == 0 && max_context_len > 0) return PA_ERR_INVALID_ARG;
+  const int group = shape->num_q_heads / shape->num_kv_heads;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   int launched = 0;
-  cudaError_t e = pa::launch_decode(a, shape->dtype, shape->head_dim,
-                                    shape->num_q_heads / shape->num_kv_heads, tk, tv,
-                                    reinterpret_cast<cudaStream_t>(stream), &launched);
+  cudaError_t e;
+  if (use_tensor_cores(shape) && shape->num_blocks > 0) {
+    CUtensorMap tk, tv, tq;
+    if (!make_tc_maps(&tk, &tv, &tq, k_cache, v_cache, q, shape)) return PA_ERR_CUDA;
+    a.epoch = next_epochs((shape->num_seqs + 511) / 512);
+    e = pa::launch_decode_tc(a, shape->dtype, group, tk, tv, tq, cs, &launched);
+    if (e == cudaSuccess) e = pa::launch_decode_merge(a, shape->dtype, shape->head_dim, cs, &launched);
+  } else {
+    CUtensorMap tk, tv;
+    if (shape->num_blocks > 0) {
+      if (!make_pool_map(&tk, k_cache, shape, pa::decode_chunk_tokens()) ||
+          !make_pool_map(&tv, v_cache, shape, pa::decode_chunk_tokens()))
+        return PA_ERR_CUDA;
+    } else {
+      // An empty pool can only serve empty contexts; the kernels issue no load.
+      memset(&tk, 0, sizeof tk);
+      memset(&tv, 0, sizeof tv);
+    }
+    e = pa::launch_decode(a, shape->dtype, shape->head_dim, group, tk, tv, cs, &launched);
+  }
   count_launches(launched);
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

@@ -96,6 +96,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t phase) {
   return ok != 0;
 }
 
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 // Wall-clock limit of any single wait.  A TMA load of a few KB completes in
 // microseconds; two seconds means the copy will never land.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -113,6 +117,46 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, unsigned
     }
   }
   return true;
+}
+
+// As mbar_wait, but also gives up (returning false) once *abort has been set
+// by another warp of the CTA; a timeout sets *abort itself.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint32_t bar, uint32_t phase, unsigned int* err,
+                                                   volatile int* abort) {
+  if (mbar_try_wait(bar, phase)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t spins = 0;
+  while (!mbar_try_wait(bar, phase)) {
+    if ((++spins & 63u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        report(err, kErrWaitTimeout);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+  return true;
+}
+
+// Named barrier `id` (> 0) over `threads` threads (a multiple of 32).
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Named barrier that also ORs `flag` over its threads: every participant gets
+// the same answer, whatever other warps write to shared memory meanwhile.
+__device__ __forceinline__ bool named_barrier_or(int id, int threads, bool flag) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pin, pout;\n\t"
+      "setp.ne.u32 pin, %1, 0;\n\t"
+      "barrier.red.or.pred pout, %2, %3, pin;\n\t"
+      "selp.u32 %0, 1, 0, pout;\n\t}"
+      : "=r"(out)
+      : "r"((uint32_t)flag), "r"(id), "r"(threads)
+      : "memory");
+  return out != 0;
 }
 
 // ---------------------------------------------------------------------------

@@ -453,6 +453,22 @@ cudaError_t launch_decode(const DecodeArgs& a, int dtype, int head_dim, int grou
   return launch_group<__nv_bfloat16, 64>(a, group, tk, tv, (int)grid, stream, launches);
 }
 
+cudaError_t launch_decode_merge(const DecodeArgs& a, int dtype, int head_dim, cudaStream_t stream,
+                                int* launches) {
+  if (a.num_parts <= 1 || a.num_seqs <= 0) return cudaSuccess;
+  const int pairs = a.num_seqs * a.num_q_heads;
+  const int grid = (pairs + 3) / 4;
+  if (dtype == 0) {
+    if (head_dim == 128) decode_merge_kernel<__half, 128><<<grid, 128, 0, stream>>>(a);
+    else decode_merge_kernel<__half, 64><<<grid, 128, 0, stream>>>(a);
+  } else {
+    if (head_dim == 128) decode_merge_kernel<__nv_bfloat16, 128><<<grid, 128, 0, stream>>>(a);
+    else decode_merge_kernel<__nv_bfloat16, 64><<<grid, 128, 0, stream>>>(a);
+  }
+  ++*launches;
+  return cudaGetLastError();
+}
+
 int decode_chunk_tokens() { return kChunk; }
 int decode_max_partition_tokens() { return kChunk * kWarps * 32; }
 

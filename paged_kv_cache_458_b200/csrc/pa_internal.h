@@ -21,6 +21,9 @@ struct DecodeArgs {
   int partition_tokens, num_parts;
   int max_context_len;           // host bound on context_lens, <= max_blocks_per_seq * block_size
   unsigned int* err;             // device error word
+  unsigned long long* work_counter;  // first 8 bytes of the workspace (tensor-core path)
+  unsigned long long epoch;      // tag of this call's launches (< 2^40, never 0)
+  int seq_offset;                // first sequence of this launch in the whole batch
 };
 
 // Launch the partition kernel (+ the merge kernel when num_parts > 1).
@@ -30,6 +33,16 @@ cudaError_t launch_decode(const DecodeArgs& a, int dtype, int head_dim, int grou
                           int* launches);
 int decode_chunk_tokens();
 int decode_max_partition_tokens();
+// The split-K merge alone (after a partition kernel that wrote partials).
+cudaError_t launch_decode_merge(const DecodeArgs& a, int dtype, int head_dim, cudaStream_t stream,
+                                int* launches);
+
+// The tensor-core path (head_dim 128): maps are 128B-swizzled, boxes of 64
+// elements; tq views q as [S * Hq][128] with boxes of (64 x group) elements.
+cudaError_t launch_decode_tc(const DecodeArgs& a, int dtype, int group, const CUtensorMap& tm_k,
+                             const CUtensorMap& tm_v, const CUtensorMap& tm_q, cudaStream_t stream,
+                             int* launches);
+int decode_tc_tile_tokens();
 
 cudaError_t launch_cache_append(const void* k, const void* v, const int32_t* slot_mapping,
                                 int num_tokens, void* k_cache, void* v_cache, long long num_slots,

@@ -18,18 +18,18 @@ def host_bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-def shape_of(dtype, q, k_cache, block_tables, partition_tokens=0):
+def shape_of(dtype, q, k_cache, block_tables, partition_tokens=0, variant=0):
     S, Hq, D = q.shape
     NB, bs, Hkv, _ = k_cache.shape
     return pa.make_shape(num_seqs=S, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D, block_size=bs,
                          num_blocks=NB, max_blocks_per_seq=block_tables.shape[1],
-                         partition_tokens=partition_tokens, dtype=dtype)
+                         partition_tokens=partition_tokens, dtype=dtype, variant=variant)
 
 
 def gpu_decode(dtype, q, k_cache, v_cache, block_tables, context_lens, scale, partition_tokens=0,
-               max_context_len=None, expect_ok=True):
+               max_context_len=None, expect_ok=True, variant=0):
     """Run pa_decode on host arrays; returns (out bits, device error status, bits)."""
-    shape = shape_of(dtype, q, k_cache, block_tables, partition_tokens)
+    shape = shape_of(dtype, q, k_cache, block_tables, partition_tokens, variant)
     if max_context_len is None:
         max_context_len = int(np.max(context_lens, initial=0))
     kc, vc = dev(k_cache, dtype), dev(v_cache, dtype)

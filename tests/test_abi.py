@@ -50,6 +50,10 @@ FAKE = 1 << 20  # a 16-byte-aligned non-null address; validation fails before an
     (dict(partition_tokens=4096), pa.PA_ERR_UNSUPPORTED),
     (dict(num_blocks=1 << 27), pa.PA_ERR_UNSUPPORTED),      # num_blocks * block_size >= 2^31
     (dict(num_seqs=-1), pa.PA_ERR_INVALID_ARG),
+    (dict(variant=3), pa.PA_ERR_INVALID_ARG),
+    (dict(variant=2, head_dim=64), pa.PA_ERR_UNSUPPORTED),
+    (dict(variant=2, partition_tokens=64), pa.PA_ERR_UNSUPPORTED),
+    (dict(variant=2, partition_tokens=1024), pa.PA_ERR_UNSUPPORTED),
 ])
 def test_decode_rejects_bad_shapes(lib, kw, expect):
     s = _shape(**kw)
@@ -68,12 +72,14 @@ def test_decode_rejects_bad_pointers_and_sizes(lib):
     assert call(scale=float("nan")) == pa.PA_ERR_INVALID_ARG
     assert call(maxlen=8 * 16 + 1) == pa.PA_ERR_INVALID_ARG     # beyond max_blocks_per_seq * bs
     assert call(maxlen=-1) == pa.PA_ERR_INVALID_ARG
-    # 100 tokens fit one 512-token partition: no workspace needed ...
-    assert lib.pa_decode_workspace_bytes(ctypes.byref(s), 100) == 0
-    # ... 1000 tokens need two partitions and a workspace
+    # 100 tokens fit one 512-token partition: only the work counter ...
+    assert lib.pa_decode_workspace_bytes(ctypes.byref(s), 100) == 256
+    st = lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s), 100, None, 0, None)
+    assert st == pa.PA_ERR_INVALID_ARG
+    # ... 1000 tokens need two partitions and split-K space
     s2 = _shape(max_blocks_per_seq=64)
     need = lib.pa_decode_workspace_bytes(ctypes.byref(s2), 1000)
-    assert need >= 4 * 8 * 2 * (128 + 2) * 4
+    assert need >= 256 + 4 * 8 * 2 * (128 + 2) * 4
     st = lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s2), 1000, FAKE, need - 1, None)
     assert st == pa.PA_ERR_INVALID_ARG
     st = lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s2), 1000, None, 0, None)

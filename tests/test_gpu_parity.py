@@ -48,12 +48,37 @@ def test_golden_block_mapping(case):
 # ---------------------------------------------------------------- full workloads
 
 
-def _run_workload(orc, name):
-    case = gen.make_case(name, n_steps=1, poison=True)
+VARIANTS = {0: "auto", 1: "cuda_cores", 2: "tensor_cores"}
+
+
+@pytest.fixture(scope="module")
+def workload_refs(orc):
+    """Each workload's inputs and oracle results, built once per module."""
+    cache = {}
+
+    def get(name):
+        if name not in cache:
+            case = gen.make_case(name, n_steps=1, poison=True)
+            st = case.steps[0]
+            ref0 = orc.decode(case.dtype, case.q, case.k_cache, case.v_cache, case.block_tables,
+                              case.context_lens, case.scale)
+            hk, hv = case.k_cache.copy(), case.v_cache.copy()
+            orc.copy_blocks(st.pairs, hk, hv)
+            orc.cache_append(st.k_new, st.v_new, st.slot_mapping, hk, hv)
+            ref1 = orc.decode(case.dtype, st.q, hk, hv, st.block_tables, st.context_lens, case.scale)
+            cache.clear()  # keep one workload's pools in host memory at a time
+            cache[name] = (case, ref0, hk, hv, ref1)
+        return cache[name]
+
+    return get
+
+
+def _run_workload(workload_refs, name, variant=0):
+    case, ref0, hk, hv, ref1 = workload_refs(name)
     dtype, S = case.dtype, case.num_seqs
     st = case.steps[0]
     maxlen = int(st.context_lens.max())
-    shape = shape_of(dtype, case.q, case.k_cache, case.block_tables)
+    shape = shape_of(dtype, case.q, case.k_cache, case.block_tables, variant=variant)
     kc, vc = dev(case.k_cache, dtype), dev(case.v_cache, dtype)
     ws = torch.empty(max(16, pa.pa_decode_workspace_bytes(shape, maxlen)), dtype=torch.uint8,
                      device="cuda")
@@ -70,31 +95,25 @@ def _run_workload(orc, name):
                  case.scale, out1, shape, maxlen, ws)
     status, bits = pa.pa_last_device_error()
     assert status == pa.PA_OK, f"device check fired: {bits:#x}"
-
-    ref0 = orc.decode(dtype, case.q, case.k_cache, case.v_cache, case.block_tables,
-                      case.context_lens, case.scale)
-    hk, hv = case.k_cache.copy(), case.v_cache.copy()
-    orc.copy_blocks(st.pairs, hk, hv)
-    orc.cache_append(st.k_new, st.v_new, st.slot_mapping, hk, hv)
     assert np.array_equal(host_bits(kc).reshape(hk.shape), hk), "K pool differs after copy+append"
     assert np.array_equal(host_bits(vc).reshape(hv.shape), hv), "V pool differs after copy+append"
-    ref1 = orc.decode(dtype, st.q, hk, hv, st.block_tables, st.context_lens, case.scale)
     s0 = assert_decode_close(host_bits(out0), ref0, dtype, f"{name} initial decode")
     s1 = assert_decode_close(host_bits(out1), ref1, dtype, f"{name} step decode")
     return case, s0, s1
 
 
-def test_tiny_workload(orc):
-    case, s0, s1 = _run_workload(orc, "tiny")
+def test_tiny_workload(workload_refs):
+    case, s0, s1 = _run_workload(workload_refs, "tiny")
     assert case.steps[0].context_lens.tolist() == [2, 16, 17, 38]
 
 
 @pytest.mark.parametrize("name", ["llama2_7b", "mistral_7b_gqa", "qwen_7b_prefix", "llama2_70b_beam"])
-def test_full_workload(orc, name):
-    case, s0, s1 = _run_workload(orc, name)
+@pytest.mark.parametrize("variant", [0, 1, 2], ids=lambda v: VARIANTS[v])
+def test_full_workload(workload_refs, name, variant):
+    case, s0, s1 = _run_workload(workload_refs, name, variant)
     if name == "llama2_70b_beam":
         assert len(case.steps[0].pairs) > 0, "the beam step must exercise copy-on-write"
-    print(f"{name}: initial {s0}  step {s1}")
+    print(f"{name} [{VARIANTS[variant]}]: initial {s0}  step {s1}")
 
 
 # ---------------------------------------------------------------- edge cases
@@ -102,39 +121,47 @@ def test_full_workload(orc, name):
 EDGE_CTX = [0, 1, 15, 16, 17, 31, 33, 511, 512, 513, 1023, 1024, 1025, 2047, 2049]
 
 
+@pytest.mark.parametrize("variant", [1, 2], ids=lambda v: VARIANTS[v])
 @pytest.mark.parametrize("dtype", [gen.F16, gen.BF16], ids=["f16", "bf16"])
 @pytest.mark.parametrize("head_dim", [64, 128])
 @pytest.mark.parametrize("group", [1, 2, 4, 8, 16])
-def test_edge_contexts(orc, dtype, head_dim, group):
+def test_edge_contexts(orc, dtype, head_dim, group, variant):
+    if variant == 2 and head_dim != 128:
+        pytest.skip("the tensor-core variant is built for head_dim 128")
     rng = np.random.default_rng(1000 * group + head_dim + dtype)
     Hkv = 2
     c = gen.random_decode_case(rng, num_seqs=len(EDGE_CTX), num_q_heads=Hkv * group,
                                num_kv_heads=Hkv, head_dim=head_dim, block_size=16, dtype=dtype,
                                context_lens=EDGE_CTX)
     out, _, _ = gpu_decode(dtype, c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
-                           c["context_lens"], c["scale"])
+                           c["context_lens"], c["scale"], variant=variant)
     ref = orc.decode(dtype, c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
                      c["context_lens"], c["scale"])
-    assert_decode_close(out, ref, dtype, f"g{group} D{head_dim}")
+    assert_decode_close(out, ref, dtype, f"g{group} D{head_dim} {VARIANTS[variant]}")
     assert np.all(out[0] == 0), "an empty context must give a zero row"
 
 
+@pytest.mark.parametrize("variant", [1, 2], ids=lambda v: VARIANTS[v])
 @pytest.mark.parametrize("block_size", [16, 32, 256])
-@pytest.mark.parametrize("partition_tokens", [16, 48, 128, 512, 2048])
-def test_block_and_partition_sizes(orc, block_size, partition_tokens):
+@pytest.mark.parametrize("partition_tokens", [16, 48, 128, 256, 512, 2048])
+def test_block_and_partition_sizes(orc, block_size, partition_tokens, variant):
+    if variant == 2 and (partition_tokens % 128 or partition_tokens > 512):
+        pytest.skip("the tensor-core variant takes partitions of 128, 256, 384 or 512 tokens")
     rng = np.random.default_rng(block_size * 7 + partition_tokens)
     ctx = [1, 47, 48, 49, 255, 256, 257, 700, 2048, 2100]
     c = gen.random_decode_case(rng, num_seqs=len(ctx), num_q_heads=8, num_kv_heads=2,
                                head_dim=128, block_size=block_size, dtype=gen.BF16,
                                context_lens=ctx, shared_prefix_blocks=1)
     out, _, _ = gpu_decode(gen.BF16, c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
-                           c["context_lens"], c["scale"], partition_tokens=partition_tokens)
+                           c["context_lens"], c["scale"], partition_tokens=partition_tokens,
+                           variant=variant)
     ref = orc.decode(gen.BF16, c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
                      c["context_lens"], c["scale"])
     assert_decode_close(out, ref, gen.BF16, f"bs{block_size} pt{partition_tokens}")
 
 
-def test_last_physical_block_and_stale_entries(orc):
+@pytest.mark.parametrize("variant", [1, 2], ids=lambda v: VARIANTS[v])
+def test_last_physical_block_and_stale_entries(orc, variant):
     rng = np.random.default_rng(3)
     c = gen.random_decode_case(rng, num_seqs=3, num_q_heads=4, num_kv_heads=4, head_dim=128,
                                block_size=16, dtype=gen.F16, context_lens=[20, 5, 33])
@@ -154,7 +181,7 @@ def test_last_physical_block_and_stale_entries(orc):
     bt[1, 1:] = 1 << 30      # stale entries past the context: never read
     bt[2, 3:] = -7
     out, _, _ = gpu_decode(gen.F16, c["q"], kc, vc, bt, c["context_lens"], c["scale"],
-                           max_context_len=64)
+                           max_context_len=64, variant=variant)
     ref = orc.decode(gen.F16, c["q"], kc, vc, bt, c["context_lens"], c["scale"])
     assert_decode_close(out, ref, gen.F16, "last block / stale entries")
 
@@ -167,13 +194,14 @@ def test_all_contexts_empty():
     assert np.all(out == 0)
 
 
-def test_permutation_invariance_and_determinism():
+@pytest.mark.parametrize("variant", [1, 2], ids=lambda v: VARIANTS[v])
+def test_permutation_invariance_and_determinism(variant):
     rng = np.random.default_rng(5)
     c = gen.random_decode_case(rng, num_seqs=6, num_q_heads=16, num_kv_heads=2, head_dim=128,
                                block_size=16, dtype=gen.BF16, context_lens=[3, 100, 513, 1500, 64, 900])
     args = (c["q"], c["k_cache"], c["v_cache"], c["block_tables"], c["context_lens"], c["scale"])
-    a, _, _ = gpu_decode(gen.BF16, *args)
-    b, _, _ = gpu_decode(gen.BF16, *args)
+    a, _, _ = gpu_decode(gen.BF16, *args, variant=variant)
+    b, _, _ = gpu_decode(gen.BF16, *args, variant=variant)
     assert np.array_equal(a, b), "decode is not deterministic"
     pi = rng.permutation(c["num_blocks"])
     kc = np.empty_like(c["k_cache"])
@@ -181,7 +209,8 @@ def test_permutation_invariance_and_determinism():
     kc[pi], vc[pi] = c["k_cache"], c["v_cache"]
     bt = c["block_tables"].copy()
     bt[bt >= 0] = pi[bt[bt >= 0]]
-    p, _, _ = gpu_decode(gen.BF16, c["q"], kc, vc, bt, c["context_lens"], c["scale"])
+    p, _, _ = gpu_decode(gen.BF16, c["q"], kc, vc, bt, c["context_lens"], c["scale"],
+                         variant=variant)
     assert np.array_equal(a, p), "output depends on where the blocks sit"
 
 
@@ -288,3 +317,35 @@ def test_workspace_needs_no_initialisation(orc):
         ref = orc.decode(gen.BF16, c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
                          c["context_lens"], c["scale"])
         assert_decode_close(host_bits(out), ref, gen.BF16, f"trial {trial}")
+
+
+def test_tensor_core_device_checks_and_launches():
+    """Bad block ids read as zeros on the tensor-core path too, with the error
+    word set; one persistent launch (+ merge) per decode."""
+    rng = np.random.default_rng(11)
+    c = gen.random_decode_case(rng, num_seqs=3, num_q_heads=16, num_kv_heads=2, head_dim=128,
+                               block_size=16, dtype=gen.BF16, context_lens=[700, 40, 300],
+                               poison=False)
+    bt = c["block_tables"].copy()
+    bt[0, 3] = c["num_blocks"] + 1
+    n0 = pa.pa_kernel_launches()
+    out, st, bits = gpu_decode(gen.BF16, c["q"], c["k_cache"], c["v_cache"], bt, c["context_lens"],
+                               c["scale"], variant=2, expect_ok=False)
+    assert pa.pa_kernel_launches() - n0 == 2
+    assert st == pa.PA_ERR_DEVICE_CHECK and bits & pa.PA_DEVERR_BLOCK_ID
+    assert np.all(np.isfinite(gen.bits_to_f32(out, gen.BF16)))
+
+
+def test_tensor_core_batches_beyond_one_launch(orc):
+    """More than 512 sequences run as several persistent launches."""
+    rng = np.random.default_rng(12)
+    ctx = rng.integers(0, 300, size=600)
+    c = gen.random_decode_case(rng, num_seqs=600, num_q_heads=8, num_kv_heads=1, head_dim=128,
+                               block_size=16, dtype=gen.F16, context_lens=ctx)
+    n0 = pa.pa_kernel_launches()
+    out, _, _ = gpu_decode(gen.F16, c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
+                           c["context_lens"], c["scale"], variant=2)
+    assert pa.pa_kernel_launches() - n0 == 2
+    ref = orc.decode(gen.F16, c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
+                     c["context_lens"], c["scale"])
+    assert_decode_close(out, ref, gen.F16, "600 sequences")

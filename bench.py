@@ -43,6 +43,7 @@ from paged_kv_cache_458_b200 import gen  # noqa: E402
 METRIC = ("paged decode-attn KV-read GB/s (% of B200 HBM peak); decode tokens/s per layer")
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+VARIANTS = {"auto": 0, "cuda_cores": 1, "tensor_cores": 2}
 
 
 def parse_args(argv=None):
@@ -53,6 +54,8 @@ def parse_args(argv=None):
     p.add_argument("--workload", default="llama2_7b", choices=sorted(gen.WORKLOADS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--partition-tokens", type=int, default=0)
+    p.add_argument("--variant", default="auto", choices=sorted(VARIANTS),
+                   help="decode kernel: auto, cuda_cores or tensor_cores")
     p.add_argument("--cycle", type=int, default=64,
                    help="distinct precomputed steps; longer runs replay them in order")
     p.add_argument("--e2e-steps", type=int, default=500)
@@ -227,7 +230,7 @@ def profiled_traffic(workload: str):
 class DeviceWorkload:
     """The pool and a cycle of precomputed steps, resident on the device."""
 
-    def __init__(self, case, torch, pa, partition_tokens: int):
+    def __init__(self, case, torch, pa, partition_tokens: int, variant: int = 0):
         self.case = case
         self.torch, self.pa = torch, pa
         dt = pa.torch_dtype(case.dtype)
@@ -252,7 +255,7 @@ class DeviceWorkload:
             num_seqs=case.num_seqs, num_q_heads=case.num_q_heads, num_kv_heads=case.num_kv_heads,
             head_dim=case.head_dim, block_size=case.block_size, num_blocks=case.num_blocks,
             max_blocks_per_seq=case.max_blocks_per_seq, partition_tokens=partition_tokens,
-            dtype=case.dtype)
+            dtype=case.dtype, variant=variant)
         self.ws_bytes = pa.pa_decode_workspace_bytes(self.shape, self.max_len)
         self.ws = torch.empty(max(16, self.ws_bytes), dtype=torch.uint8, device="cuda")
         self.out = torch.empty((case.num_seqs, case.num_q_heads, case.head_dim), dtype=dt,
@@ -290,7 +293,7 @@ def run_ours(args, rank, world, local, dist):
     n_cycle = max(1, min(args.cycle, args.steps + args.warmup))
     case = gen.make_case(args.workload, n_steps=n_cycle, poison=False,
                          seed=gen.SEED_BASE + gen.WORKLOADS[args.workload].number + 1000 * rank)
-    w = DeviceWorkload(case, torch, pa, args.partition_tokens)
+    w = DeviceWorkload(case, torch, pa, args.partition_tokens, VARIANTS[args.variant])
     bytes_per = [decode_bytes(s.context_lens, case.num_q_heads, case.num_kv_heads, case.head_dim,
                               case.block_size) for s in case.steps]
     pool_bytes = 2 * case.k_cache.nbytes
@@ -345,6 +348,7 @@ def run_ours(args, rank, world, local, dist):
             "num_kv_heads": case.num_kv_heads, "head_dim": case.head_dim,
             "block_size": case.block_size, "storage_dtype": gen.DTYPE_NAMES[case.dtype],
             "partition_tokens": args.partition_tokens or 512,
+            "decode_variant": args.variant,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "steps_cycle": n_cycle,
             "l2": (f"inputs larger than L2: {kv_step0 / 1e6:.0f} MB of K/V read per decode, "

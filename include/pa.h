@@ -217,6 +217,13 @@ pa_status pa_last_device_error(pa_stream_t stream, uint32_t *bits_out);
 /* Static description of a status code (never NULL). */
 const char *pa_status_string(pa_status status);
 
+/* Text of the CUDA error behind the calling thread's most recent
+ * PA_ERR_CUDA from pa_decode, pa_cache_append, pa_copy_blocks or
+ * pa_last_device_error ("no CUDA error" before the first one).  The string is
+ * static; the caller does not free it.  Not part of the method: a diagnostic
+ * of this library. */
+const char *pa_last_cuda_error(void);
+
 /* Number of kernels this library has launched in this process. */
 uint64_t pa_kernel_launches(void);
 

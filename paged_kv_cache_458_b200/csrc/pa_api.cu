@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <chrono>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -34,6 +35,19 @@ unsigned int* error_word() {
 }
 
 std::atomic<uint64_t> g_launches{0};
+
+// What the calling thread's last PA_ERR_CUDA came from.
+thread_local const char* t_last_cuda_error = "no CUDA error";
+
+pa_status cuda_failed(cudaError_t e) {
+  t_last_cuda_error = cudaGetErrorString(e);
+  return PA_ERR_CUDA;
+}
+
+pa_status cuda_failed(const char* what) {
+  t_last_cuda_error = what;
+  return PA_ERR_CUDA;
+}
 
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
@@ -93,7 +107,12 @@ constexpr long long kCounterBytes = 256;
 
 // Tags of decode launches (see the work counter in pa_decode_tc.cu): unique
 // per launch, never 0, below 2^40.
-std::atomic<uint64_t> g_epoch{1};
+// Epochs start at a per-process value so that a workspace last used by another
+// library instance or process is unlikely to carry a live epoch.
+std::atomic<uint64_t> g_epoch{
+    1 + ((reinterpret_cast<uintptr_t>(&g_launches) ^
+          (uint64_t)std::chrono::steady_clock::now().time_since_epoch().count() * 0x9E3779B97F4A7C15ull) &
+         ((1ull << 39) - 1))};
 uint64_t next_epochs(int n) {
   uint64_t e = g_epoch.fetch_add((uint64_t)n, std::memory_order_relaxed) & ((1ull << 40) - 1);
   if (e == 0 || e + (uint64_t)n >= (1ull << 40)) e = 1;
@@ -219,7 +238,7 @@ pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
   a.num_parts = P > 0 ? P : 1;
   a.max_context_len = max_context_len;
   a.err = error_word();
-  if (!a.err) return PA_ERR_CUDA;
+  if (!a.err) return cuda_failed("device error word lookup failed");
 
   if (shape->num_blocks == 0 && max_context_len > 0) return PA_ERR_INVALID_ARG;
   const int group = shape->num_q_heads / shape->num_kv_heads;
@@ -228,7 +247,8 @@ pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
   cudaError_t e;
   if (use_tensor_cores(shape) && shape->num_blocks > 0) {
     CUtensorMap tk, tv, tq;
-    if (!make_tc_maps(&tk, &tv, &tq, k_cache, v_cache, q, shape)) return PA_ERR_CUDA;
+    if (!make_tc_maps(&tk, &tv, &tq, k_cache, v_cache, q, shape))
+      return cuda_failed("cuTensorMapEncodeTiled failed");
     a.epoch = next_epochs((shape->num_seqs + 511) / 512);
     e = pa::launch_decode_tc(a, shape->dtype, group, tk, tv, tq, cs, &launched);
     if (e == cudaSuccess) e = pa::launch_decode_merge(a, shape->dtype, shape->head_dim, cs, &launched);
@@ -237,7 +257,7 @@ pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
     if (shape->num_blocks > 0) {
       if (!make_pool_map(&tk, k_cache, shape, pa::decode_chunk_tokens()) ||
           !make_pool_map(&tv, v_cache, shape, pa::decode_chunk_tokens()))
-        return PA_ERR_CUDA;
+        return cuda_failed("cuTensorMapEncodeTiled failed");
     } else {
       // An empty pool can only serve empty contexts; the kernels issue no load.
       memset(&tk, 0, sizeof tk);
@@ -246,7 +266,7 @@ pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
     e = pa::launch_decode(a, shape->dtype, shape->head_dim, group, tk, tv, cs, &launched);
   }
   count_launches(launched);
-  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return e == cudaSuccess ? PA_OK : cuda_failed(e);
 }
 
 pa_status pa_cache_append(const void* k, const void* v, const int32_t* slot_mapping,
@@ -262,14 +282,14 @@ pa_status pa_cache_append(const void* k, const void* v, const int32_t* slot_mapp
     return PA_ERR_INVALID_ARG;
   const int row_bytes = shape->num_kv_heads * shape->head_dim * 2;
   unsigned int* err = error_word();
-  if (!err) return PA_ERR_CUDA;
+  if (!err) return cuda_failed("device error word lookup failed");
   int launched = 0;
   cudaError_t e = pa::launch_cache_append(k, v, slot_mapping, num_tokens, k_cache, v_cache,
                                           (long long)shape->num_blocks * shape->block_size,
                                           row_bytes, err, reinterpret_cast<cudaStream_t>(stream),
                                           &launched);
   count_launches(launched);
-  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return e == cudaSuccess ? PA_OK : cuda_failed(e);
 }
 
 pa_status pa_copy_blocks(const int32_t* src_dst_pairs, int32_t num_pairs, void* k_cache,
@@ -285,22 +305,23 @@ pa_status pa_copy_blocks(const int32_t* src_dst_pairs, int32_t num_pairs, void* 
   const long long block_bytes =
       (long long)shape->block_size * shape->num_kv_heads * shape->head_dim * 2;
   unsigned int* err = error_word();
-  if (!err) return PA_ERR_CUDA;
+  if (!err) return cuda_failed("device error word lookup failed");
   int launched = 0;
   cudaError_t e = pa::launch_copy_blocks(src_dst_pairs, num_pairs, k_cache, v_cache,
                                          shape->num_blocks, block_bytes, err,
                                          reinterpret_cast<cudaStream_t>(stream), &launched);
   count_launches(launched);
-  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return e == cudaSuccess ? PA_OK : cuda_failed(e);
 }
 
 pa_status pa_last_device_error(pa_stream_t stream, uint32_t* bits_out) {
-  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return PA_ERR_CUDA;
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_failed(e);
   unsigned int bits = 0;
   const unsigned int zero = 0;
-  if (cudaMemcpyFromSymbol(&bits, g_device_error, sizeof bits) != cudaSuccess) return PA_ERR_CUDA;
-  if (bits && cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero) != cudaSuccess)
-    return PA_ERR_CUDA;
+  if ((e = cudaMemcpyFromSymbol(&bits, g_device_error, sizeof bits)) != cudaSuccess) return cuda_failed(e);
+  if (bits && (e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero)) != cudaSuccess)
+    return cuda_failed(e);
   if (bits_out) *bits_out = bits;
   return bits ? PA_ERR_DEVICE_CHECK : PA_OK;
 }
@@ -316,6 +337,8 @@ const char* pa_status_string(pa_status s) {
   }
   return "unknown status";
 }
+
+const char* pa_last_cuda_error(void) { return t_last_cuda_error; }
 
 uint64_t pa_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 

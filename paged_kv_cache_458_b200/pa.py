@@ -34,7 +34,10 @@ class LibraryMissing(ImportError):
 class PaError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn} failed: {status_string(status)} (status {status})")
+        msg = f"{fn} failed: {status_string(status)} (status {status})"
+        if status == PA_ERR_CUDA:
+            msg += f": {pa_last_cuda_error()}"
+        super().__init__(msg)
 
 
 class pa_shape(ctypes.Structure):
@@ -72,6 +75,8 @@ def _declare(lib):
     lib.pa_kernel_launches.argtypes = []
     lib.pa_build_info.restype = c.c_char_p
     lib.pa_build_info.argtypes = []
+    lib.pa_last_cuda_error.restype = c.c_char_p
+    lib.pa_last_cuda_error.argtypes = []
     lib.pa_alloc_create.restype = P
     lib.pa_alloc_create.argtypes = [I32, I32, P]
     lib.pa_alloc_destroy.restype = None
@@ -211,6 +216,10 @@ def pa_last_device_error(stream=None) -> tuple[int, int]:
 
 def pa_kernel_launches() -> int:
     return int(lib().pa_kernel_launches())
+
+
+def pa_last_cuda_error() -> str:
+    return lib().pa_last_cuda_error().decode()
 
 
 def pa_build_info() -> str:

@@ -27,6 +27,7 @@ def test_status_strings(lib):
         assert pa.status_string(st) and pa.status_string(st) != "unknown status"
     assert lib.pa_status_string(99) == b"unknown status"
     assert "sm_100a" in pa.pa_build_info()
+    assert pa.pa_last_cuda_error()  # a static string, set by the last PA_ERR_CUDA
 
 
 def _shape(**kw):

@@ -206,21 +206,22 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the kernel source as it is now (else None)."""
+def profiled_traffic(workload: str, variant: str, step_bytes: float):
+    """DRAM bytes per decode launch from the committed ncu summary of this
+    workload, if it was taken on the kernel that runs (same variant, same
+    source digest); else None.  The capture is of one seeded step; its
+    DRAM/algorithmic ratio is applied to this run's average step bytes."""
     path = os.path.join(ROOT, "profiles", f"pa_decode_{workload}.json")
     try:
         with open(path) as f:
             prof = json.load(f)
-    except (OSError, ValueError):
+        with open(os.path.join(ROOT, prof["source"]), "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()[:16]
+    except (OSError, ValueError, KeyError):
         return None
-    src = os.path.join(ROOT, "paged_kv_cache_458_b200", "csrc", "pa_decode.cu")
-    with open(src, "rb") as f:
-        digest = hashlib.sha256(f.read()).hexdigest()[:16]
-    if prof.get("source_sha256_16") != digest:
+    if prof.get("variant") != variant or prof.get("source_sha256_16") != digest:
         return None
-    return prof.get("dram_bytes_per_launch_full_size")
+    return int(round(prof["traffic_over_algorithmic"] * step_bytes))
 
 
 # ---------------------------------------------------------------------------
@@ -335,7 +336,8 @@ def run_ours(args, rank, world, local, dist):
 
     peak, peak_kind = measured_peak()
     achieved = step_bytes / (dec_total_ms * 1e-3) / 1e9
-    traffic = profiled_traffic(args.workload)
+    resolved = {1: "cuda_cores", 2: "tensor_cores"}[pa.pa_decode_resolved_variant(w.shape)]
+    traffic = profiled_traffic(args.workload, resolved, step_bytes / args.steps)
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -348,7 +350,7 @@ def run_ours(args, rank, world, local, dist):
             "num_kv_heads": case.num_kv_heads, "head_dim": case.head_dim,
             "block_size": case.block_size, "storage_dtype": gen.DTYPE_NAMES[case.dtype],
             "partition_tokens": args.partition_tokens or 512,
-            "decode_variant": args.variant,
+            "decode_variant": f"{args.variant} -> {resolved}",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "steps_cycle": n_cycle,
             "l2": (f"inputs larger than L2: {kv_step0 / 1e6:.0f} MB of K/V read per decode, "
@@ -359,7 +361,8 @@ def run_ours(args, rank, world, local, dist):
         "decode_bytes_per_step": int(step_bytes / args.steps),
         "pct_of_8tbps": round(100 * value / 8000.0, 2),
         "roofline": {
-            "bound": "hbm", "kernel": "pa_decode (partition kernel + split-K merge kernel)",
+            "bound": "hbm",
+            "kernel": f"pa_decode ({resolved} partition kernel + split-K merge kernel)",
             "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
             "frac": round(achieved / peak, 4),
             "traffic": traffic,

@@ -109,6 +109,11 @@ typedef struct {
  *                          PA_ERR_UNSUPPORTED). */
 typedef enum { PA_DECODE_AUTO = 0, PA_DECODE_CUDA_CORES = 1, PA_DECODE_TENSOR_CORES = 2 } pa_decode_variant;
 
+/* The kernel pa_decode() runs for `shape`: PA_DECODE_CUDA_CORES or
+ * PA_DECODE_TENSOR_CORES (PA_DECODE_AUTO resolved), or minus the status
+ * pa_decode() would refuse the shape with.  Host only; launches nothing. */
+int pa_decode_resolved_variant(const pa_shape *shape);
+
 /* Bytes of device workspace pa_decode() needs for `shape` when no context is
  * longer than `max_context_len` tokens: 256 bytes for the work counter the
  * tensor-core variant's persistent CTAs take items from, plus, when a context

@@ -314,6 +314,12 @@ pa_status pa_copy_blocks(const int32_t* src_dst_pairs, int32_t num_pairs, void* 
   return e == cudaSuccess ? PA_OK : cuda_failed(e);
 }
 
+int pa_decode_resolved_variant(const pa_shape* shape) {
+  const pa_status st = check_decode_shape(shape, 0);
+  if (st != PA_OK) return -(int)st;
+  return use_tensor_cores(shape) ? PA_DECODE_TENSOR_CORES : PA_DECODE_CUDA_CORES;
+}
+
 pa_status pa_last_device_error(pa_stream_t stream, uint32_t* bits_out) {
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_failed(e);

@@ -75,6 +75,8 @@ def _declare(lib):
     lib.pa_kernel_launches.argtypes = []
     lib.pa_build_info.restype = c.c_char_p
     lib.pa_build_info.argtypes = []
+    lib.pa_decode_resolved_variant.restype = c.c_int
+    lib.pa_decode_resolved_variant.argtypes = [SP]
     lib.pa_last_cuda_error.restype = c.c_char_p
     lib.pa_last_cuda_error.argtypes = []
     lib.pa_alloc_create.restype = P
@@ -216,6 +218,13 @@ def pa_last_device_error(stream=None) -> tuple[int, int]:
 
 def pa_kernel_launches() -> int:
     return int(lib().pa_kernel_launches())
+
+
+def pa_decode_resolved_variant(shape: pa_shape) -> int:
+    v = lib().pa_decode_resolved_variant(ctypes.byref(shape))
+    if v < 0:
+        raise PaError("pa_decode_resolved_variant", -v)
+    return v
 
 
 def pa_last_cuda_error() -> str:

@@ -62,6 +62,17 @@ def test_decode_rejects_bad_shapes(lib, kw, expect):
     assert st == expect
 
 
+def test_resolved_variant(lib):
+    assert pa.pa_decode_resolved_variant(_shape()) == pa.PA_DECODE_CUDA_CORES          # group 4
+    assert pa.pa_decode_resolved_variant(_shape(num_q_heads=16)) == pa.PA_DECODE_TENSOR_CORES
+    assert pa.pa_decode_resolved_variant(_shape(num_q_heads=16, head_dim=64)) == pa.PA_DECODE_CUDA_CORES
+    assert pa.pa_decode_resolved_variant(_shape(num_q_heads=16, partition_tokens=1024)) == pa.PA_DECODE_CUDA_CORES
+    assert pa.pa_decode_resolved_variant(_shape(variant=2)) == pa.PA_DECODE_TENSOR_CORES
+    with pytest.raises(pa.PaError) as e:
+        pa.pa_decode_resolved_variant(_shape(head_dim=96))
+    assert e.value.status == pa.PA_ERR_UNSUPPORTED
+
+
 def test_decode_rejects_bad_pointers_and_sizes(lib):
     s = _shape()
     call = lambda **o: lib.pa_decode(  # noqa: E731

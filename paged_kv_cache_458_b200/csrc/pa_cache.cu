@@ -23,6 +23,8 @@ cache_append_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                     const int32_t* __restrict__ slot_mapping, uint4* __restrict__ k_cache,
                     uint4* __restrict__ v_cache, long long num_slots, int row_vecs,
                     unsigned int* err) {
+  pdl_wait();  // a copy-on-write of this slot's block must land first
+  pdl_launch_dependents();
   const int t = blockIdx.x;
   const long long slot = __ldg(slot_mapping + t);
   if (slot < 0) return;
@@ -50,6 +52,8 @@ __global__ void __launch_bounds__(kCopyThreads)
 copy_blocks_kernel(const int32_t* __restrict__ pairs, uint4* __restrict__ k_cache,
                    uint4* __restrict__ v_cache, int num_blocks, long long block_vecs,
                    unsigned int* err) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int i = blockIdx.y;
   const int src = __ldg(pairs + 2 * i), dst = __ldg(pairs + 2 * i + 1);
   if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
@@ -81,11 +85,12 @@ cudaError_t launch_cache_append(const void* k, const void* v, const int32_t* slo
   if (num_tokens == 0) return cudaSuccess;
   const int row_vecs = row_bytes / 16;
   const int threads = row_vecs >= 256 ? 256 : ((row_vecs + 31) / 32) * 32;
-  cache_append_kernel<<<num_tokens, threads, 0, stream>>>(
-      static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
-      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), num_slots, row_vecs, err);
-  ++*launches;
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(cache_append_kernel, dim3(num_tokens), dim3(threads), 0, stream,
+                             static_cast<const uint4*>(k), static_cast<const uint4*>(v),
+                             slot_mapping, static_cast<uint4*>(k_cache),
+                             static_cast<uint4*>(v_cache), num_slots, row_vecs, err);
+  if (e == cudaSuccess) ++*launches;
+  return e;
 }
 
 cudaError_t launch_copy_blocks(const int32_t* pairs, int num_pairs, void* k_cache, void* v_cache,
@@ -96,11 +101,11 @@ cudaError_t launch_copy_blocks(const int32_t* pairs, int num_pairs, void* k_cach
   const long long pieces = (block_vecs + kPiece - 1) / kPiece;
   if (num_pairs > 65535 || pieces > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   dim3 grid((unsigned)pieces, (unsigned)num_pairs);
-  copy_blocks_kernel<<<grid, kCopyThreads, 0, stream>>>(pairs, static_cast<uint4*>(k_cache),
-                                                        static_cast<uint4*>(v_cache), num_blocks,
-                                                        block_vecs, err);
-  ++*launches;
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(copy_blocks_kernel, grid, dim3(kCopyThreads), 0, stream, pairs,
+                             static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+                             num_blocks, block_vecs, err);
+  if (e == cudaSuccess) ++*launches;
+  return e;
 }
 
 }  // namespace pa

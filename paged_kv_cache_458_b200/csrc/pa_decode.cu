@@ -125,6 +125,8 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  pdl_wait();  // the append before this decode must have landed
+  pdl_launch_dependents();
 
   int bid = blockIdx.x;
   const int kvh = bid % a.num_kv_heads;
@@ -353,6 +355,8 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
 template <typename T, int D>
 __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a) {
   constexpr int VEC = D / 32;
+  pdl_wait();  // every partition's partial is written
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int pair = blockIdx.x * 4 + (threadIdx.x >> 5);
   if (pair >= a.num_seqs * a.num_q_heads) return;
@@ -414,14 +418,14 @@ cudaError_t launch_typed(const DecodeArgs& a, const CUtensorMap& tk, const CUten
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  kern<<<grid, kWarps * 32, L::kTotal, stream>>>(a, tk, tv);
+  cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kWarps * 32), L::kTotal, stream, a, tk, tv);
+  if (e != cudaSuccess) return e;
   ++*launches;
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || a.num_parts <= 1) return e;
+  if (a.num_parts <= 1) return cudaSuccess;
   const int pairs = a.num_seqs * a.num_q_heads;
-  decode_merge_kernel<T, D><<<(pairs + 3) / 4, 128, 0, stream>>>(a);
-  ++*launches;
-  return cudaGetLastError();
+  e = launch_pdl(decode_merge_kernel<T, D>, dim3((pairs + 3) / 4), dim3(128), 0, stream, a);
+  if (e == cudaSuccess) ++*launches;
+  return e;
 }
 
 template <typename T, int D>
@@ -457,16 +461,18 @@ cudaError_t launch_decode_merge(const DecodeArgs& a, int dtype, int head_dim, cu
                                 int* launches) {
   if (a.num_parts <= 1 || a.num_seqs <= 0) return cudaSuccess;
   const int pairs = a.num_seqs * a.num_q_heads;
-  const int grid = (pairs + 3) / 4;
+  const dim3 grid((pairs + 3) / 4), block(128);
+  cudaError_t e;
   if (dtype == 0) {
-    if (head_dim == 128) decode_merge_kernel<__half, 128><<<grid, 128, 0, stream>>>(a);
-    else decode_merge_kernel<__half, 64><<<grid, 128, 0, stream>>>(a);
+    e = head_dim == 128 ? launch_pdl(decode_merge_kernel<__half, 128>, grid, block, 0, stream, a)
+                        : launch_pdl(decode_merge_kernel<__half, 64>, grid, block, 0, stream, a);
   } else {
-    if (head_dim == 128) decode_merge_kernel<__nv_bfloat16, 128><<<grid, 128, 0, stream>>>(a);
-    else decode_merge_kernel<__nv_bfloat16, 64><<<grid, 128, 0, stream>>>(a);
+    e = head_dim == 128
+            ? launch_pdl(decode_merge_kernel<__nv_bfloat16, 128>, grid, block, 0, stream, a)
+            : launch_pdl(decode_merge_kernel<__nv_bfloat16, 64>, grid, block, 0, stream, a);
   }
-  ++*launches;
-  return cudaGetLastError();
+  if (e == cudaSuccess) ++*launches;
+  return e;
 }
 
 int decode_chunk_tokens() { return kChunk; }

@@ -204,6 +204,8 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
+  pdl_wait();  // the append before this decode must have landed
+  pdl_launch_dependents();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = a.num_seqs, Hkv = a.num_kv_heads, PT = a.partition_tokens;
   int* desc_all = reinterpret_cast<int*>(smem + L::kDesc);
@@ -618,10 +620,9 @@ cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUte
     a.epoch = a0.epoch + (unsigned long long)(s0 / kMaxSeqs);
     const int items0 = a.num_seqs * a.num_kv_heads;
     const int grid = items0 < sms ? items0 : sms;
-    kern<<<grid, kThreads, L::kAlloc, stream>>>(a, tk, tv, tq);
-    ++*launches;
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kThreads), L::kAlloc, stream, a, tk, tv, tq);
     if (e != cudaSuccess) return e;
+    ++*launches;
   }
   return cudaSuccess;
 }

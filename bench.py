@@ -56,6 +56,9 @@ def parse_args(argv=None):
     p.add_argument("--partition-tokens", type=int, default=0)
     p.add_argument("--variant", default="auto", choices=sorted(VARIANTS),
                    help="decode kernel: auto, cuda_cores or tensor_cores")
+    p.add_argument("--shared-prefix", default="auto", choices=["auto", "on", "off"],
+                   help="read blocks shared by consecutive sequences once per group; auto: on "
+                        "when the workload's tables share their first block")
     p.add_argument("--cycle", type=int, default=64,
                    help="distinct precomputed steps; longer runs replay them in order")
     p.add_argument("--e2e-steps", type=int, default=500)
@@ -119,6 +122,13 @@ def decode_bytes(ctx: np.ndarray, num_q_heads, num_kv_heads, head_dim, block_siz
     qo = 2 * S * num_q_heads * head_dim * elem
     tables = int(4 * np.ceil(ctx / block_size).sum())
     return kv + qo + tables + 4 * S
+
+
+def tables_share_blocks(tables: np.ndarray, ctx: np.ndarray) -> bool:
+    """Whether two consecutive sequences start with the same physical block."""
+    live = np.asarray(ctx) > 0
+    first = np.asarray(tables)[:, 0]
+    return bool(np.any(live[1:] & live[:-1] & (first[1:] == first[:-1])))
 
 
 def unique_kv_bytes(tables: np.ndarray, ctx: np.ndarray, block_size, num_kv_heads, head_dim,
@@ -231,7 +241,8 @@ def profiled_traffic(workload: str, variant: str, step_bytes: float):
 class DeviceWorkload:
     """The pool and a cycle of precomputed steps, resident on the device."""
 
-    def __init__(self, case, torch, pa, partition_tokens: int, variant: int = 0):
+    def __init__(self, case, torch, pa, partition_tokens: int, variant: int = 0,
+                 shared_prefix: int = 0):
         self.case = case
         self.torch, self.pa = torch, pa
         dt = pa.torch_dtype(case.dtype)
@@ -256,7 +267,7 @@ class DeviceWorkload:
             num_seqs=case.num_seqs, num_q_heads=case.num_q_heads, num_kv_heads=case.num_kv_heads,
             head_dim=case.head_dim, block_size=case.block_size, num_blocks=case.num_blocks,
             max_blocks_per_seq=case.max_blocks_per_seq, partition_tokens=partition_tokens,
-            dtype=case.dtype, variant=variant)
+            dtype=case.dtype, variant=variant, shared_prefix=shared_prefix)
         self.ws_bytes = pa.pa_decode_workspace_bytes(self.shape, self.max_len)
         self.ws = torch.empty(max(16, self.ws_bytes), dtype=torch.uint8, device="cuda")
         self.out = torch.empty((case.num_seqs, case.num_q_heads, case.head_dim), dtype=dt,
@@ -294,7 +305,11 @@ def run_ours(args, rank, world, local, dist):
     n_cycle = max(1, min(args.cycle, args.steps + args.warmup))
     case = gen.make_case(args.workload, n_steps=n_cycle, poison=False,
                          seed=gen.SEED_BASE + gen.WORKLOADS[args.workload].number + 1000 * rank)
-    w = DeviceWorkload(case, torch, pa, args.partition_tokens, VARIANTS[args.variant])
+    shared = {"on": 1, "off": 0}.get(args.shared_prefix)
+    if shared is None:
+        shared = int(args.variant == "auto" and
+                     tables_share_blocks(case.steps[0].block_tables, case.steps[0].context_lens))
+    w = DeviceWorkload(case, torch, pa, args.partition_tokens, VARIANTS[args.variant], shared)
     bytes_per = [decode_bytes(s.context_lens, case.num_q_heads, case.num_kv_heads, case.head_dim,
                               case.block_size) for s in case.steps]
     pool_bytes = 2 * case.k_cache.nbytes
@@ -336,7 +351,8 @@ def run_ours(args, rank, world, local, dist):
 
     peak, peak_kind = measured_peak()
     achieved = step_bytes / (dec_total_ms * 1e-3) / 1e9
-    resolved = {1: "cuda_cores", 2: "tensor_cores"}[pa.pa_decode_resolved_variant(w.shape)]
+    resolved = {1: "cuda_cores", 2: "tensor_cores",
+                3: "shared_prefix"}[pa.pa_decode_resolved_variant(w.shape)]
     traffic = profiled_traffic(args.workload, resolved, step_bytes / args.steps)
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -351,6 +367,7 @@ def run_ours(args, rank, world, local, dist):
             "block_size": case.block_size, "storage_dtype": gen.DTYPE_NAMES[case.dtype],
             "partition_tokens": args.partition_tokens or 512,
             "decode_variant": f"{args.variant} -> {resolved}",
+            "shared_prefix": bool(shared),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "steps_cycle": n_cycle,
             "l2": (f"inputs larger than L2: {kv_step0 / 1e6:.0f} MB of K/V read per decode, "
@@ -362,7 +379,10 @@ def run_ours(args, rank, world, local, dist):
         "pct_of_8tbps": round(100 * value / 8000.0, 2),
         "roofline": {
             "bound": "hbm",
-            "kernel": f"pa_decode ({resolved} partition kernel + split-K merge kernel)",
+            "kernel": (f"pa_decode ({resolved} partition kernel + split-K merge kernel)"
+                       if resolved != "shared_prefix" else
+                       "pa_decode (plan + shared-prefix tensor-core kernel + CUDA-core kernel "
+                       "+ split-K merge)"),
             "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
             "frac": round(achieved / peak, 4),
             "traffic": traffic,
@@ -374,6 +394,9 @@ def run_ours(args, rank, world, local, dist):
         st = case.steps[0]
         result["unique_kv_bytes_step0"] = unique_kv_bytes(
             st.block_tables, st.context_lens, case.block_size, case.num_kv_heads, case.head_dim)
+        # the same decode counted in distinct K/V slots (shared blocks once)
+        result["unique_kv_gbs_step0_est"] = round(
+            result["unique_kv_bytes_step0"] / (dec_total_ms / args.steps * 1e-3) / 1e9, 2)
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, w, stream, bytes_per, n_cycle, dist)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -456,10 +479,15 @@ def cpu_baseline(case, seconds: float, st):
     dt1, _ = _oracle_sample(case, st, 1, orc, threads)
     n = int(max(1, min(case.num_seqs, seconds / max(dt1, 1e-6))))
     dt, nbytes = _oracle_sample(case, st, n, orc, threads)
+    reps = 1
+    while dt < 0.5 * seconds:  # the whole batch took less: decode it again
+        d, b = _oracle_sample(case, st, n, orc, threads)
+        dt, nbytes, reps = dt + d, nbytes + b, reps + 1
     return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": threads,
             "kind": "oracle",
-            "sample": f"fp64 C oracle, decode of the first {n} of {case.num_seqs} sequences of step 0 "
-                      f"({nbytes / 1e6:.1f} MB algorithmic), {dt:.2f} s wall, {threads} threads"}
+            "sample": f"fp64 C oracle, decode of the first {n} of {case.num_seqs} sequences of step 0, "
+                      f"{reps} time(s) ({nbytes / 1e6:.1f} MB algorithmic), {dt:.2f} s wall, "
+                      f"{threads} threads"}
 
 
 def run_reference(args, rank, world):

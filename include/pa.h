@@ -93,6 +93,8 @@ typedef struct {
   int32_t partition_tokens;
   int32_t dtype;   /* pa_dtype */
   int32_t variant; /* pa_decode_variant (pa_decode only; 0 = automatic) */
+  int32_t shared_prefix; /* pa_decode only: 1 = read blocks shared by consecutive
+                            sequences once per group (see pa_decode); 0 = off */
 } pa_shape;
 
 /* How pa_decode computes QK^T and PV.  Both variants read K/V with tiled TMA
@@ -110,15 +112,21 @@ typedef struct {
 typedef enum { PA_DECODE_AUTO = 0, PA_DECODE_CUDA_CORES = 1, PA_DECODE_TENSOR_CORES = 2 } pa_decode_variant;
 
 /* The kernel pa_decode() runs for `shape`: PA_DECODE_CUDA_CORES or
- * PA_DECODE_TENSOR_CORES (PA_DECODE_AUTO resolved), or minus the status
- * pa_decode() would refuse the shape with.  Host only; launches nothing. */
+ * PA_DECODE_TENSOR_CORES (PA_DECODE_AUTO resolved), or
+ * PA_DECODE_RESOLVED_SHARED_PREFIX with shape->shared_prefix (tensor cores for
+ * the shared tokens, CUDA cores for the rest), or minus the status pa_decode()
+ * would refuse the shape with.  Host only; launches nothing. */
+#define PA_DECODE_RESOLVED_SHARED_PREFIX 3
 int pa_decode_resolved_variant(const pa_shape *shape);
 
 /* Bytes of device workspace pa_decode() needs for `shape` when no context is
  * longer than `max_context_len` tokens: 256 bytes for the work counter the
- * tensor-core variant's persistent CTAs take items from, plus, when a context
- * spans more than one partition, per (sequence, query head, partition) the
- * running max, the softmax sum and the unnormalised output row in fp32.  The
+ * tensor-core variant's persistent CTAs take items from; with shared_prefix,
+ * 16 bytes per sequence (rounded up to 256) for the group plan; plus, when a
+ * context spans more than one partition (always with shared_prefix), per
+ * (sequence, query head, partition) the running max, the softmax sum and the
+ * unnormalised output row in fp32, for ceil(max_context_len /
+ * partition_tokens) partitions, one more with shared_prefix.  The
  * workspace needs no initialisation (the counter carries a per-call tag, so a
  * value left by an earlier call is recognised and replaced) and is dead after
  * the call's kernels finish.  Returns 0 for an invalid shape. */
@@ -140,6 +148,24 @@ size_t pa_decode_workspace_bytes(const pa_shape *shape, int32_t max_context_len)
  * variant; items taken by one persistent CTA per SM on the tensor-core
  * variant), and sequences with more than one partition are merged by a
  * second kernel (log-sum-exp rule).  shape->variant picks the arithmetic.
+ *
+ * Shared prefixes (shape->shared_prefix = 1; needs variant PA_DECODE_AUTO,
+ * head_dim 128 and partition_tokens a multiple of 128 up to 512, else
+ * PA_ERR_UNSUPPORTED).  Blocks shared between sequences (zingnex.cn,
+ * "vLLM与PagedAttention深度剖析", section 3.2 item 3: beam candidates forked
+ * from one parent, prompts with a common prefix) are then read once per group
+ * of sequences instead of once per sequence.  A first kernel finds the groups
+ * on the device from the tables alone: runs of consecutive sequences (within
+ * aligned windows of 256) whose tables start with the same physical block, cut
+ * into groups of at most 32 / g members; a group shares its first T tokens,
+ * where T counts the leading table entries equal in all members (below each
+ * member's own block count), capped at the shortest member context and
+ * rounded down to a multiple of 16; groups with T < 128 are dropped.  A
+ * tensor-core kernel computes every group's shared tokens for all members x g
+ * query rows at once, the CUDA-core kernel each sequence's remaining tokens,
+ * and the merge kernel combines the two (log-sum-exp rule).  The result is the
+ * same attention, up to fp32 rounding order; only the order in which the sums
+ * are formed differs.
  *
  * q, k_cache, v_cache, block_tables, context_lens, out: device, layouts above.
  * max_context_len: host-side upper bound on every context_lens[s]; it sizes the

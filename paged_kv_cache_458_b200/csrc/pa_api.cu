@@ -84,6 +84,11 @@ pa_status check_decode_shape(const pa_shape* s, int32_t max_context_len) {
   if (s->variant == PA_DECODE_TENSOR_CORES &&
       (s->head_dim != 128 || pt % pa::decode_tc_tile_tokens() != 0 || pt > 512))
     return PA_ERR_UNSUPPORTED;
+  if (s->shared_prefix != 0 && s->shared_prefix != 1) return PA_ERR_INVALID_ARG;
+  if (s->shared_prefix &&
+      (s->variant != PA_DECODE_AUTO || s->head_dim != 128 || pt % pa::decode_tc_tile_tokens() != 0 ||
+       pt > 512))
+    return PA_ERR_UNSUPPORTED;
   // work items of one launch (<= 512 sequences) must fit the 24-bit counter
   const long long parts = ((long long)max_context_len + pt - 1) / pt;
   if (512LL * s->num_kv_heads * (parts > 0 ? parts : 1) >= (1LL << 23)) return PA_ERR_UNSUPPORTED;
@@ -101,9 +106,26 @@ bool use_tensor_cores(const pa_shape* s) {
          pt % pa::decode_tc_tile_tokens() == 0 && pt <= 512;
 }
 
-// Workspace: the work counter (8 bytes used of 256), then, for split-K,
-// partial outputs [S][Hq][P][D] and (max, sum) pairs [S][Hq][P][2] in fp32.
+// Workspace: the work counter (8 bytes used of 256); with shared_prefix the
+// plan, int4 [S] (rounded up to 256 bytes); then, for split-K, partial
+// outputs [S][Hq][P][D] and (max, sum) pairs [S][Hq][P][2] in fp32.  P is
+// ceil(max_context_len / partition_tokens), plus one with shared_prefix (a
+// sequence's shared tokens and its own ones may each end in a partial
+// partition).
 constexpr long long kCounterBytes = 256;
+
+long long round256(long long x) { return (x + 255) / 256 * 256; }
+
+int num_partitions(const pa_shape* s, int32_t max_context_len);
+
+long long plan_bytes(const pa_shape* s) { return s->shared_prefix ? round256(16LL * s->num_seqs) : 0; }
+
+// Partitions per (sequence, query head) in the workspace (0: no split-K space).
+long long workspace_parts(const pa_shape* s, int32_t max_context_len) {
+  const long long P = num_partitions(s, max_context_len);
+  if (s->shared_prefix) return P + 1;
+  return P > 1 ? P : 0;
+}
 
 // Tags of decode launches (see the work counter in pa_decode_tc.cu): unique
 // per launch, never 0, below 2^40.
@@ -188,12 +210,13 @@ extern "C" {
 
 size_t pa_decode_workspace_bytes(const pa_shape* shape, int32_t max_context_len) {
   if (check_decode_shape(shape, max_context_len) != PA_OK) return 0;
-  const long long P = num_partitions(shape, max_context_len);
-  if (P <= 1) return (size_t)kCounterBytes;
+  const long long head = kCounterBytes + plan_bytes(shape);
+  const long long P = workspace_parts(shape, max_context_len);
+  if (P == 0) return (size_t)head;
   const long long rows = (long long)shape->num_seqs * shape->num_q_heads * P;
   const long long acc = rows * shape->head_dim * 4;
   const long long ml = rows * 2 * 4;
-  return (size_t)(kCounterBytes + ((acc + 255) / 256) * 256 + ml);
+  return (size_t)(head + round256(acc) + ml);
 }
 
 pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
@@ -215,17 +238,23 @@ pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
     return PA_ERR_INVALID_ARG;
 
   const int P = num_partitions(shape, max_context_len);
+  const int P_ws = (int)workspace_parts(shape, max_context_len);
   pa::DecodeArgs a{};
   a.q = static_cast<const uint16_t*>(q);
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.out = static_cast<uint16_t*>(out);
   a.work_counter = static_cast<unsigned long long*>(workspace);
-  if (P > 1) {
-    const long long rows = (long long)shape->num_seqs * shape->num_q_heads * P;
-    char* base = static_cast<char*>(workspace) + kCounterBytes;
-    a.ws_acc = reinterpret_cast<float*>(base);
-    a.ws_ml = reinterpret_cast<float*>(base + ((rows * shape->head_dim * 4 + 255) / 256) * 256);
+  char* ws = static_cast<char*>(workspace) + kCounterBytes;
+  int4* plan = nullptr;
+  if (shape->shared_prefix) {
+    plan = reinterpret_cast<int4*>(ws);
+    ws += plan_bytes(shape);
+  }
+  if (P_ws > 0) {
+    const long long rows = (long long)shape->num_seqs * shape->num_q_heads * P_ws;
+    a.ws_acc = reinterpret_cast<float*>(ws);
+    a.ws_ml = reinterpret_cast<float*>(ws + round256(rows * shape->head_dim * 4));
   }
   a.scale_log2 = scale * 1.4426950408889634f;
   a.num_seqs = shape->num_seqs;
@@ -235,7 +264,8 @@ pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
   a.num_blocks = shape->num_blocks;
   a.max_blocks_per_seq = shape->max_blocks_per_seq;
   a.partition_tokens = effective_partition(shape);
-  a.num_parts = P > 0 ? P : 1;
+  a.num_parts = P_ws > 0 ? P_ws : 1;
+  a.grid_parts = P > 0 ? P : 1;
   a.max_context_len = max_context_len;
   a.err = error_word();
   if (!a.err) return cuda_failed("device error word lookup failed");
@@ -245,7 +275,35 @@ pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   int launched = 0;
   cudaError_t e;
-  if (use_tensor_cores(shape) && shape->num_blocks > 0) {
+  if (shape->shared_prefix && shape->num_blocks > 0) {
+    // plan the groups, then their shared tokens on tensor cores, then every
+    // sequence's own tokens on CUDA cores, then the merge
+    CUtensorMap tk, tv, tq, pk, pv;
+    if (!make_tc_maps(&tk, &tv, &tq, k_cache, v_cache, q, shape) ||
+        !make_pool_map(&pk, k_cache, shape, pa::decode_chunk_tokens()) ||
+        !make_pool_map(&pv, v_cache, shape, pa::decode_chunk_tokens()))
+      return cuda_failed("cuTensorMapEncodeTiled failed");
+    pa::PlanArgs pl{};
+    pl.block_tables = block_tables;
+    pl.context_lens = context_lens;
+    pl.plan = plan;
+    pl.num_seqs = shape->num_seqs;
+    pl.max_blocks_per_seq = shape->max_blocks_per_seq;
+    pl.block_size = shape->block_size;
+    pl.num_blocks = shape->num_blocks;
+    pl.max_context_len = max_context_len;
+    pl.partition_tokens = a.partition_tokens;
+    pl.max_members = 32 / group;
+    pl.min_shared = pa::decode_tc_tile_tokens();
+    pl.chunk = pa::kSharedPrefixSeqsPerLaunch;
+    a.plan = plan;
+    a.epoch = next_epochs((shape->num_seqs + pa::kSharedPrefixSeqsPerLaunch - 1) /
+                          pa::kSharedPrefixSeqsPerLaunch);
+    e = pa::launch_plan(pl, cs, &launched);
+    if (e == cudaSuccess) e = pa::launch_decode_shared_tc(a, shape->dtype, group, tk, tv, cs, &launched);
+    if (e == cudaSuccess)
+      e = pa::launch_decode(a, shape->dtype, shape->head_dim, group, pk, pv, cs, &launched);
+  } else if (use_tensor_cores(shape) && shape->num_blocks > 0) {
     CUtensorMap tk, tv, tq;
     if (!make_tc_maps(&tk, &tv, &tq, k_cache, v_cache, q, shape))
       return cuda_failed("cuTensorMapEncodeTiled failed");
@@ -317,6 +375,7 @@ pa_status pa_copy_blocks(const int32_t* src_dst_pairs, int32_t num_pairs, void* 
 int pa_decode_resolved_variant(const pa_shape* shape) {
   const pa_status st = check_decode_shape(shape, 0);
   if (st != PA_OK) return -(int)st;
+  if (shape->shared_prefix) return PA_DECODE_RESOLVED_SHARED_PREFIX;
   return use_tensor_cores(shape) ? PA_DECODE_TENSOR_CORES : PA_DECODE_CUDA_CORES;
 }
 

@@ -149,10 +149,12 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
     }
     return;
   }
-  const int t_begin = part * PT;
+  // With a shared-prefix plan this CTA covers part of [T, ctx) only.
+  const SeqSplit split = seq_split(a.plan, s, ctx, PT);
+  const int t_begin = split.base + part * PT;
   if (t_begin >= ctx) return;
   const int t_end = min(ctx, t_begin + PT);
-  const int n_parts_seq = (ctx + PT - 1) / PT;
+  const int n_parts_seq = split.total;
   const int n_chunks = (t_end - t_begin + kChunk - 1) / kChunk;
   const int n_mine = warp < n_chunks ? (n_chunks - warp + NW - 1) / NW : 0;
 
@@ -340,7 +342,7 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
     if (direct) {
       a.out[qh * D + d] = Elem<T>::from_f(num / den);
     } else {
-      const size_t slot = qh * a.num_parts + part;
+      const size_t slot = qh * a.num_parts + split.slot0 + part;
       a.ws_acc[slot * D + d] = num;
       if (d == 0) {
         a.ws_ml[2 * slot] = M;
@@ -363,7 +365,7 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a) {
   const int s = pair / a.num_q_heads;
   int ctx = __ldg(a.context_lens + s);
   ctx = max(0, min(ctx, a.max_context_len));
-  const int P = (ctx + a.partition_tokens - 1) / a.partition_tokens;
+  const int P = seq_split(a.plan, s, ctx, a.partition_tokens).total;
   if (P <= 1) return;
   const size_t base = (size_t)pair * a.num_parts;
   float M = -INFINITY;
@@ -446,7 +448,7 @@ cudaError_t launch_group(const DecodeArgs& a, int G, const CUtensorMap& tk, cons
 cudaError_t launch_decode(const DecodeArgs& a, int dtype, int head_dim, int group,
                           const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream,
                           int* launches) {
-  const long long grid = (long long)a.num_parts * a.num_seqs * a.num_kv_heads;
+  const long long grid = (long long)a.grid_parts * a.num_seqs * a.num_kv_heads;
   if (grid <= 0) return cudaSuccess;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   if (dtype == 0) {

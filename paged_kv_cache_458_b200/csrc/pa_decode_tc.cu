@@ -6,32 +6,45 @@
 // that costs CUDA cores about as much time as the HBM read once g >= 4.  This
 // kernel moves both products onto tcgen05.mma and keeps the read on TMA:
 //
-//   S^T[128 tok x 16]  = K_tile[128 tok x 128 d] . Q^T[128 d x 16]   (A K-major, B K-major)
-//   O^T[128 d x 16]    = V_tile^T[128 d x 128 tok] . P^T[128 tok x 16] (A MN-major, B MN-major)
+//   S^T[128 tok x N]  = K_tile[128 tok x 128 d] . Q^T[128 d x N]     (A K-major, B K-major)
+//   O^T[128 d x N]    = V_tile^T[128 d x 128 tok] . P^T[128 tok x N] (A MN-major, B MN-major)
 //
-// with the g heads padded to N = 16 (zero rows of Q), fp16/bf16 operands and
-// fp32 accumulators in tensor memory (TMEM).  The softmax stays in fp32 on the
-// CUDA cores: tcgen05.ld gives thread t (of 128) the 16 logits of token t, the
-// per-head tile maximum is a warp + shared-memory reduction, and thread t writes
-// its row of P.  After the PV product thread d reads row d of O^T and folds it
-// into its running output (rescaled by 2^(m_old - m_new) per head).  The
-// probabilities enter the PV product as two terms of the input type, hi =
+// with fp16/bf16 operands and fp32 accumulators in tensor memory (TMEM).  The
+// N columns are query rows:
+//   - one sequence (the plain kernel): its g query heads, padded to N = 16;
+//   - a group of sequences whose block tables begin with the same physical
+//     blocks (the shared-prefix kernel): members x g query rows, N = 32.  The
+//     blocks every member reads are then read once for all of them, which is
+//     what sharing blocks between sequences (a common prompt prefix, beam
+//     candidates forked from one parent) is for (zingnex.cn,
+//     "vLLM与PagedAttention深度剖析", section 3.2 item 3; jsqmd.com,
+//     "vLLM-v0.11.0性能实测", section 4.2: requests with the same prefix
+//     share pages).
+//
+// The softmax stays in fp32 on the CUDA cores: tcgen05.ld gives thread t (of
+// 128) the N logits of token t; the per-column tile maximum is a transposed
+// warp reduction (lane c ends with column c) plus shared memory, and thread t
+// writes its row of P.  After the PV product thread d reads row d of O^T and
+// folds it into its running output (rescaled by 2^(m_old - m_new) per column).
+// The probabilities enter the PV product as two terms of the input type, hi =
 // round(p) and lo = round(p - hi), so they carry about 16 significant bits (a
 // bf16 P alone, 8 bits, can move a short context's output by more than 2e-3);
 // the tensor cores have ample room for the second set of MMAs.
 //
-// Work: items (sequence, kv head, partition of partition_tokens tokens, a
-// multiple of 128) are numbered as in the CUDA-core kernel (partition 0 of
-// every (sequence, kv head) first, then the further partitions of longer
-// sequences).  One persistent CTA per SM: a producer warp takes items (its
-// first one by number, then from a counter in the workspace whose value
-// carries the call's epoch), resolves each 16-token group of an item through
-// the block table and issues per 128-token tile 32 tiled TMA loads (8 groups x
-// {K, V} x two 64-element halves, 128B-swizzled) into one of NST stages, plus
-// the item's query rows into an item slot.  Four compute warps consume tiles
-// in order; thread 0 issues the MMAs and commits them to mbarriers.  Tokens at
-// or past the context are masked in P and their V rows are zeroed in shared
-// memory before the PV product, so stale or NaN rows never reach the result.
+// Work, plain kernel: items (sequence, kv head, partition of partition_tokens
+// tokens, a multiple of 128) are numbered as in the CUDA-core kernel (partition
+// 0 of every (sequence, kv head) first, then the further partitions of longer
+// sequences).  Shared-prefix kernel: items (group leader, kv head, partition of
+// the shared tokens), numbered over the leaders of the launch.  One persistent
+// CTA per SM: a producer warp takes items (its first one by number, then from a
+// counter in the workspace whose value carries the call's epoch), resolves each
+// 16-token group of an item through the block table and issues per 128-token
+// tile 32 tiled TMA loads (8 groups x {K, V} x two 64-element halves,
+// 128B-swizzled) into one of NST stages, plus the item's query rows into an
+// item slot.  Four compute warps consume tiles in order; thread 0 issues the
+// MMAs and commits them to mbarriers.  Tokens at or past the end of the item
+// are masked in P and their V rows are zeroed in shared memory before the PV
+// product, so stale or NaN rows never reach the result.
 //
 // Split-K partials and the merge kernel are shared with the CUDA-core path.
 //
@@ -51,37 +64,48 @@ namespace pa {
 namespace tc {
 
 constexpr int kTile = 128;          // tokens per MMA tile (M)
-constexpr int kN = 16;              // padded query heads (N)
 constexpr int kD = 128;             // head_dim of this path
 constexpr int kGroupRows = 16;      // token rows per TMA box (a block is a multiple)
 constexpr int kSlots = 2;           // item slots (descriptor + query rows)
-constexpr int kMaxSeqs = 512;       // sequences per launch (prefix in shared memory)
 constexpr int kComputeThreads = 128;
 constexpr int kThreads = kComputeThreads + 32;
-constexpr uint32_t kTmemCols = 32;  // S^T in columns [0,16), O^T in [16,32)
 
-template <int NST>
+// Per kernel kind: N columns, sequences per launch (their prefix sums live in
+// shared memory) and TMEM columns (S^T in [0, N), O^T in [N, 2N)).
+template <bool GROUP>
+struct Cfg {
+  static constexpr int kN = GROUP ? 32 : 16;
+  static constexpr int kMaxSeqs = GROUP ? kSharedPrefixSeqsPerLaunch : 512;
+  static constexpr uint32_t kTmemCols = GROUP ? 64 : 32;
+};
+
+template <int NST, int N, int MAXSEQS>
 struct Layout {
   // offsets from a 1024-byte aligned base
   static constexpr int kStageBytes = 2 * kTile * kD * 2;      // K tile then V tile (64 KB)
   static constexpr int kHalf = kTile * 128;                    // one 64-element half of a tile (16 KB)
   static constexpr int kStages = 0;
-  static constexpr int kQ = kStages + NST * kStageBytes;       // [slots][2 halves][16 rows][128 B]
-  static constexpr int kQBytes = 2 * kN * 128;
-  static constexpr int kP = kQ + kSlots * kQBytes;             // P hi, then P lo: [128 tok][16] 32-B rows
-  static constexpr int kPBytes = kTile * kN * 2;
-  static constexpr int kRed = kP + 2 * kPBytes;                // [4 warps][16] f32
-  static constexpr int kDesc = kRed + 4 * kN * 4;              // [slots][8] int
-  static constexpr int kPrefix = kDesc + kSlots * 8 * 4;       // [kMaxSeqs + 1] int
-  static constexpr int kBars = (kPrefix + (kMaxSeqs + 1) * 4 + 7) / 8 * 8;
+  static constexpr int kQ = kStages + NST * kStageBytes;       // [slots][2 halves][N rows][128 B]
+  static constexpr int kQBytes = 2 * N * 128;
+  static constexpr int kP = kQ + kSlots * kQBytes;             // P hi, then P lo
+  static constexpr int kPBytes = kTile * N * 2;                // [N/16 atoms][128 tok][32 B]
+  static constexpr int kPAtom = kTile * 32;                    // bytes of one 16-column atom
+  static constexpr int kRed = kP + 2 * kPBytes;                // [4 warps][N] f32
+  static constexpr int kStat = kRed + 4 * N * 4;               // m[N], then alpha[N] or l[N], f32
+  static constexpr int kDesc = kStat + 2 * N * 4;              // [slots][8] int
+  static constexpr int kPrefix = kDesc + kSlots * 8 * 4;       // [MAXSEQS + 1] int
+  static constexpr int kBars = (kPrefix + (MAXSEQS + 1) * 4 + 7) / 8 * 8;
   // full[NST], empty[NST], ready[slots], free[slots], qk, pv
   static constexpr int kNumBars = 2 * NST + 2 * kSlots + 2;
   static constexpr int kMisc = kBars + kNumBars * 8;           // tmem address, abort flag
   static constexpr int kUsed = kMisc + 16;
   static constexpr int kAlloc = kUsed + 1024;                  // room to align the base
   static_assert(kQ % 1024 == 0 && kQBytes % 1024 == 0 && kP % 256 == 0, "swizzle atoms");
+  static_assert(kAlloc <= 232448, "shared memory per CTA");
 };
 
+// Item descriptor fields (kDCtx: the context of a plain item, the number of
+// member sequences of a shared-prefix item).
 enum { kDS = 0, kDKvh, kDPart, kDBegin, kDEnd, kDTiles, kDParts, kDCtx };
 
 // ---------------------------------------------------------------------------
@@ -125,19 +149,34 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-// 16 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-      "%12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
+// N (16 or 32) consecutive fp32 columns of this thread's TMEM lane.
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[N]) {
+  uint32_t r[N];
+  if constexpr (N == 16) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+        "%12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+  } else {
+    static_assert(N == 32, "16 or 32 columns");
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+        "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+        "%30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+  }
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < N; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int c0, int c1) {
@@ -157,9 +196,40 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi, bool bf16) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Item number -> (sequence, kv head, partition); see the file comment.
-__device__ __forceinline__ void locate(int f, int n_first, int Hkv, int S, const int* prefix, int& s,
-                                       int& kvh, int& part) {
+// Column-wise reduction of a warp's 32 rows of NC values: on return lane l
+// holds the maximum (or sum) of column l % NC over the warp.  Lanes first
+// combine with the partners that will end up holding the same column; then
+// each step of width w hands half of a lane's columns to the partner lane^w.
+// NC - 1 + NC * (5 - log2 NC) shuffles instead of 5 * NC.  `v` is consumed.
+template <int NC, bool MAX>
+__device__ __forceinline__ float column_reduce(float (&v)[NC], int lane) {
+#pragma unroll
+  for (int w = 16; w >= NC; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+      const float o = __shfl_xor_sync(0xffffffffu, v[i], w);
+      v[i] = MAX ? fmaxf(v[i], o) : v[i] + o;
+    }
+#pragma unroll
+  for (int w = NC / 2; w >= 1; w >>= 1) {
+    const bool upper = (lane & w) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const float send = upper ? v[i] : v[i + w];
+      const float keep = upper ? v[i + w] : v[i];
+      const float got = __shfl_xor_sync(0xffffffffu, send, w);
+      v[i] = MAX ? fmaxf(keep, got) : keep + got;
+    }
+  }
+  return v[0];
+}
+
+// Item number -> (sequence, kv head, partition); see the file comment.  The
+// first n_first numbers are partition 0 of every (sequence, kv head); the
+// rest are counted by prefix[] (prefix[s] = items of sequences before s, per
+// kv head), numbered from `part0` within a sequence.
+__device__ __forceinline__ void locate(int f, int n_first, int Hkv, int S, const int* prefix, int part0,
+                                       int& s, int& kvh, int& part) {
   if (f < n_first) {
     s = f / Hkv;
     kvh = f % Hkv;
@@ -175,7 +245,7 @@ __device__ __forceinline__ void locate(int f, int n_first, int Hkv, int S, const
     if (prefix[mid] <= r) lo = mid; else hi = mid;
   }
   s = lo;
-  part = 1 + r - prefix[lo];
+  part = part0 + r - prefix[lo];
 }
 
 // Work counter tagged with the call's epoch in bits 24..63 (see pa_decode.cu).
@@ -192,25 +262,30 @@ __device__ __forceinline__ int take_item(unsigned long long* ctr, unsigned long 
   return -1;
 }
 
-template <typename T, int G, int NST>
+template <typename T, int G, int NST, bool GROUP>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q) {
-  using L = Layout<NST>;
+  using C = Cfg<GROUP>;
+  constexpr int N = C::kN;
+  constexpr int NC = GROUP ? N : G;  // columns that carry query rows
+  using L = Layout<NST, N, C::kMaxSeqs>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
-  constexpr uint32_t kIdescQK = instr_desc(kBf16 ? 1 : 0, 0, 0, kTile, kN);
-  constexpr uint32_t kIdescPV = instr_desc(kBf16 ? 1 : 0, 1, 1, kTile, kN);
+  constexpr uint32_t kIdescQK = instr_desc(kBf16 ? 1 : 0, 0, 0, kTile, N);
+  constexpr uint32_t kIdescPV = instr_desc(kBf16 ? 1 : 0, 1, 1, kTile, N);
+  static_assert(GROUP || G <= N, "query heads per tile");
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-  pdl_wait();  // the append before this decode must have landed
+  pdl_wait();  // the kernels before this decode (append, plan) must have landed
   pdl_launch_dependents();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = a.num_seqs, Hkv = a.num_kv_heads, PT = a.partition_tokens;
   int* desc_all = reinterpret_cast<int*>(smem + L::kDesc);
   int* prefix = reinterpret_cast<int*>(smem + L::kPrefix);
   float* red = reinterpret_cast<float*>(smem + L::kRed);
+  float* stat = reinterpret_cast<float*>(smem + L::kStat);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   const uint32_t bars = smem_addr(smem + L::kBars);
@@ -227,7 +302,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(tmem_holder)),
-                 "r"(kTmemCols)
+                 "r"(C::kTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -245,13 +320,15 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     *abort_flag = 0;
     mbar_init_fence();
   }
-  // Query rows G..15 of both slots are zero for good (the padded heads).
-  if constexpr (G < kN) {
-    constexpr int kPad = kN - G;
+  // Query rows that no item fills stay zero (padded heads); a shared-prefix
+  // item fills members x g rows, so the slots start all zero.
+  constexpr int kRow0 = GROUP ? 0 : G;
+  constexpr int kPad = N - kRow0;
+  if constexpr (kPad > 0) {
     for (int i = tid; i < kSlots * 2 * kPad * 8; i += kThreads) {
-      const int chunk = i % 8, row = G + (i / 8) % kPad, half = (i / 8 / kPad) % 2,
+      const int chunk = i % 8, row = kRow0 + (i / 8) % kPad, half = (i / 8 / kPad) % 2,
                 slot = i / 8 / kPad / 2;
-      *reinterpret_cast<uint4*>(smem + L::kQ + slot * L::kQBytes + half * kN * 128 + row * 128 +
+      *reinterpret_cast<uint4*>(smem + L::kQ + slot * L::kQBytes + half * N * 128 + row * 128 +
                                 chunk * 16) = make_uint4(0, 0, 0, 0);
     }
   }
@@ -263,22 +340,29 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
 
   if (warp == 4) {
     // =====================================================================
-    // producer warp: items, table entries, TMA loads
+    // producer warp: items, table entries, query rows, TMA loads
     // =====================================================================
+    // Per sequence, the items numbered through prefix[]: further partitions
+    // (plain) or the shared partitions of a group leader (shared-prefix).
     int carry = 0;
     if (lane == 0) prefix[0] = 0;
     for (int base = 0; base < S; base += 32) {
       const int s = base + lane;
-      int extra = 0;
+      int cnt = 0;
       if (s < S) {
-        int ctx = __ldg(a.context_lens + s);
-        if (ctx < 0 || ctx > a.max_context_len) {
-          if (blockIdx.x == 0) report(a.err, kErrContextLen);
-          ctx = max(0, min(ctx, a.max_context_len));
+        if constexpr (GROUP) {
+          const int4 pl = __ldg(a.plan + s);
+          cnt = (pl.x == 0 && pl.y >= 2) ? pl.w : 0;
+        } else {
+          int ctx = __ldg(a.context_lens + s);
+          if (ctx < 0 || ctx > a.max_context_len) {
+            if (blockIdx.x == 0) report(a.err, kErrContextLen);
+            ctx = max(0, min(ctx, a.max_context_len));
+          }
+          cnt = max((ctx + PT - 1) / PT - 1, 0);
         }
-        extra = max((ctx + PT - 1) / PT - 1, 0);
       }
-      int incl = extra;
+      int incl = cnt;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int t = __shfl_up_sync(0xffffffffu, incl, o);
@@ -288,7 +372,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
     __syncwarp();
-    const int n_first = S * Hkv;
+    const int n_first = GROUP ? 0 : S * Hkv;
     const int total = n_first + Hkv * carry;
 
     int issued = 0;  // tiles armed so far (stage ring position)
@@ -310,10 +394,18 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         break;
       }
       int s, kvh, part;
-      locate(f, n_first, Hkv, S, prefix, s, kvh, part);
-      const int ctx = max(0, min(__ldg(a.context_lens + s), a.max_context_len));
+      locate(f, n_first, Hkv, S, prefix, GROUP ? 0 : 1, s, kvh, part);
+      int t_end, ctx_or_members;
       const int t_begin = part * PT;
-      const int t_end = min(ctx, t_begin + PT);
+      if constexpr (GROUP) {
+        const int4 pl = __ldg(a.plan + s);
+        t_end = min(pl.z, t_begin + PT);
+        ctx_or_members = pl.y;
+      } else {
+        const int ctx = max(0, min(__ldg(a.context_lens + s), a.max_context_len));
+        t_end = min(ctx, t_begin + PT);
+        ctx_or_members = ctx;
+      }
       const int n_tok = max(0, t_end - t_begin);
       const int n_tiles = (n_tok + kTile - 1) / kTile;
       const int n_groups = (n_tok + kGroupRows - 1) / kGroupRows;  // <= 32
@@ -328,6 +420,24 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           my_row = blk * a.block_size + tok % a.block_size;
         }
       }
+      if constexpr (GROUP) {
+        // members x g query rows, 16-byte pieces stored in the 128B-swizzled
+        // K-major layout the QK descriptor reads (piece c of row r at c ^ (r & 7))
+        const int rows = ctx_or_members * G;
+        const uint32_t qs = sm_q + slot * L::kQBytes;
+        for (int i = lane; i < rows * 16; i += 32) {
+          const int r = i >> 4, cc = i & 15;
+          const int m = r / G, h = r % G;
+          const size_t qrow = (size_t)(a.seq_offset + s + m) * a.num_q_heads + kvh * G + h;
+          const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.q + qrow * kD) + cc);
+          const uint32_t dst = qs + (cc >> 3) * N * 128 + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y),
+                       "r"(v.z), "r"(v.w)
+                       : "memory");
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+      }
       if (lane == 0) {
         desc[kDS] = s;
         desc[kDKvh] = kvh;
@@ -335,13 +445,17 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         desc[kDBegin] = t_begin;
         desc[kDEnd] = t_end;
         desc[kDTiles] = n_tiles;
-        desc[kDParts] = (ctx + PT - 1) / PT;
-        desc[kDCtx] = ctx;
+        desc[kDParts] = GROUP ? 0 : (ctx_or_members + PT - 1) / PT;
+        desc[kDCtx] = ctx_or_members;
         const uint32_t rb = ready_bar(slot);
-        mbar_arrive_expect_tx(rb, 2 * G * 128);
-        const int qrow = (a.seq_offset + s) * a.num_q_heads + kvh * G;
-        tma_load_2d(sm_q + slot * L::kQBytes, &tm_q, rb, 0, qrow);
-        tma_load_2d(sm_q + slot * L::kQBytes + kN * 128, &tm_q, rb, 64, qrow);
+        if constexpr (GROUP) {
+          mbar_arrive(rb);
+        } else {
+          mbar_arrive_expect_tx(rb, 2 * G * 128);
+          const int qrow = (a.seq_offset + s) * a.num_q_heads + kvh * G;
+          tma_load_2d(sm_q + slot * L::kQBytes, &tm_q, rb, 0, qrow);
+          tma_load_2d(sm_q + slot * L::kQBytes + N * 128, &tm_q, rb, 64, qrow);
+        }
       }
       for (int j = 0; j < n_tiles && ok; ++j) {
         const int st = issued % NST;
@@ -397,12 +511,13 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       if (n_tiles < 0) break;  // end of work
       const int s = desc[kDS], kvh = desc[kDKvh], part = desc[kDPart];
       const int t_begin = desc[kDBegin], t_end = desc[kDEnd], n_parts = desc[kDParts];
-      const int ctx = desc[kDCtx];
+      const int ctx_or_members = desc[kDCtx];
       const uint32_t q_addr = sm_q + slot * L::kQBytes;
 
-      float acc[G], l_tok[G], m_run[G];
+      float acc[NC], l_tok[NC];
 #pragma unroll
-      for (int h = 0; h < G; ++h) acc[h] = 0.f, l_tok[h] = 0.f, m_run[h] = -INFINITY;
+      for (int c = 0; c < NC; ++c) acc[c] = 0.f, l_tok[c] = 0.f;
+      float m_col = -INFINITY;  // warp 0, lane c < NC: running max of column c
 
       for (int j = 0; j < n_tiles; ++j, ++n_used) {
         const int st = n_used % NST;
@@ -417,7 +532,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
             for (int kk = 0; kk < kD / 16; ++kk) {
               const uint32_t ko = (kk / 4) * L::kHalf + (kk % 4) * 32;
-              const uint32_t qo = (kk / 4) * kN * 128 + (kk % 4) * 32;
+              const uint32_t qo = (kk / 4) * N * 128 + (kk % 4) * 32;
               mma_f16(tmem, smem_desc(kt + ko, 16, 1024, kSw128),
                       smem_desc(q_addr + qo, 16, 1024, kSw128), kIdescQK, kk > 0);
             }
@@ -428,67 +543,66 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         }
         if (named_barrier_or(1, kComputeThreads, !ok || *abort_flag)) { ok = false; break; }
         tc_fence_after();
-        float sv[16];
-        tmem_ld16(tmem + t_lane, sv);
+        float sv[N];
+        tmem_ld<N>(tmem + t_lane, sv);
 
         // ---- softmax over this tile (log2 domain)
         const bool valid = tid < n_valid;
-        float tile_max[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          sv[h] = valid ? sv[h] * a.scale_log2 : -INFINITY;
-          float mx = sv[h];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          tile_max[h] = mx;
-        }
-        if (lane == 0)
-#pragma unroll
-          for (int h = 0; h < G; ++h) red[warp * kN + h] = tile_max[h];
-        named_barrier(1, kComputeThreads);
-        float alpha[G], p[kN];
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float mt = fmaxf(fmaxf(red[h], red[kN + h]), fmaxf(red[2 * kN + h], red[3 * kN + h]));
-          const float m_new = fmaxf(m_run[h], mt);
-          alpha[h] = exp2f(m_run[h] - m_new);
-          m_run[h] = m_new;
-          p[h] = valid ? exp2f(sv[h] - m_new) : 0.f;
-        }
-#pragma unroll
-        for (int h = G; h < kN; ++h) p[h] = 0.f;
-        // P^T rows (MN-major, 32-byte rows, 32-byte swizzle: 16-byte half c of
-        // row t sits at c ^ bit 2 of t), once for hi = round(p) and once for
-        // lo = round(p - hi).
         {
-          float plo[kN];
-          uint4 lo, hi;
-          lo.x = pack2(p[0], p[1], kBf16);  lo.y = pack2(p[2], p[3], kBf16);
-          lo.z = pack2(p[4], p[5], kBf16);  lo.w = pack2(p[6], p[7], kBf16);
-          hi.x = pack2(p[8], p[9], kBf16);  hi.y = pack2(p[10], p[11], kBf16);
-          hi.z = pack2(p[12], p[13], kBf16); hi.w = pack2(p[14], p[15], kBf16);
-          {
-            const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+          float t[NC];
+#pragma unroll
+          for (int c = 0; c < NC; ++c) {
+            sv[c] = valid ? sv[c] * a.scale_log2 : -INFINITY;
+            t[c] = sv[c];
+          }
+          const float wmax = column_reduce<NC, true>(t, lane);
+          if (lane < NC) red[warp * N + lane] = wmax;
+        }
+        named_barrier(1, kComputeThreads);
+        if (warp == 0 && lane < NC) {
+          const float mt = fmaxf(fmaxf(red[lane], red[N + lane]), fmaxf(red[2 * N + lane], red[3 * N + lane]));
+          const float m_new = fmaxf(m_col, mt);
+          stat[N + lane] = exp2f(m_col - m_new);  // alpha
+          stat[lane] = m_new;
+          m_col = m_new;
+        }
+        named_barrier(1, kComputeThreads);
+        float alpha[NC], p[N];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+          alpha[c] = stat[N + c];
+          p[c] = valid ? exp2f(sv[c] - stat[c]) : 0.f;
+          l_tok[c] = l_tok[c] * alpha[c] + p[c];
+        }
+#pragma unroll
+        for (int c = NC; c < N; ++c) p[c] = 0.f;
+        // P^T rows: per 16-column atom, a 32-byte row per token (MN-major,
+        // 32-byte swizzle: 16-byte piece c of row t sits at c ^ bit 2 of t),
+        // once for hi = round(p) and once for lo = round(p - hi).
+        {
+          const int sw = (tid >> 2) & 1;
+#pragma unroll
+          for (int at = 0; at < N / 16; ++at) {
+            const float* pa = p + at * 16;
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[i] = pack2(pa[2 * i], pa[2 * i + 1], kBf16);
+            float r[16];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              const float2 r = Elem<T>::to_f2(w[i]);
-              plo[2 * i] = p[2 * i] - r.x;
-              plo[2 * i + 1] = p[2 * i + 1] - r.y;
+              const float2 x = Elem<T>::to_f2(w[i]);
+              r[2 * i] = pa[2 * i] - x.x;
+              r[2 * i + 1] = pa[2 * i + 1] - x.y;
             }
-          }
-          const int sw = (tid >> 2) & 1;
-          unsigned char* prow = smem + L::kP + tid * 32;
-          *reinterpret_cast<uint4*>(prow + 16 * sw) = lo;
-          *reinterpret_cast<uint4*>(prow + 16 * (sw ^ 1)) = hi;
-          uint4 lo2, hi2;
-          lo2.x = pack2(plo[0], plo[1], kBf16);   lo2.y = pack2(plo[2], plo[3], kBf16);
-          lo2.z = pack2(plo[4], plo[5], kBf16);   lo2.w = pack2(plo[6], plo[7], kBf16);
-          hi2.x = pack2(plo[8], plo[9], kBf16);   hi2.y = pack2(plo[10], plo[11], kBf16);
-          hi2.z = pack2(plo[12], plo[13], kBf16); hi2.w = pack2(plo[14], plo[15], kBf16);
-          *reinterpret_cast<uint4*>(prow + L::kPBytes + 16 * sw) = lo2;
-          *reinterpret_cast<uint4*>(prow + L::kPBytes + 16 * (sw ^ 1)) = hi2;
+            unsigned char* prow = smem + L::kP + at * L::kPAtom + tid * 32;
+            *reinterpret_cast<uint4*>(prow + 16 * sw) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(prow + 16 * (sw ^ 1)) = make_uint4(w[4], w[5], w[6], w[7]);
 #pragma unroll
-          for (int h = 0; h < G; ++h) l_tok[h] = l_tok[h] * alpha[h] + p[h];
+            for (int i = 0; i < 8; ++i) w[i] = pack2(r[2 * i], r[2 * i + 1], kBf16);
+            *reinterpret_cast<uint4*>(prow + L::kPBytes + 16 * sw) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(prow + L::kPBytes + 16 * (sw ^ 1)) =
+                make_uint4(w[4], w[5], w[6], w[7]);
+          }
         }
         if (!valid) {
           // zero this token's V row (both 64-element halves) so 0 * stale never enters PV
@@ -510,9 +624,9 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           for (int part_p = 0; part_p < 2; ++part_p)  // P = hi + lo
 #pragma unroll
             for (int kk = 0; kk < kTile / 16; ++kk)
-              mma_f16(tmem + kN, smem_desc(vt + kk * 2048, L::kHalf, 1024, kSw128),
-                      smem_desc(sm_p + part_p * L::kPBytes + kk * 512, 512, 256, kSw32), kIdescPV,
-                      part_p > 0 || kk > 0);
+              mma_f16(tmem + N, smem_desc(vt + kk * 2048, L::kHalf, 1024, kSw128),
+                      smem_desc(sm_p + part_p * L::kPBytes + kk * 512, L::kPAtom, 256, kSw32),
+                      kIdescPV, part_p > 0 || kk > 0);
           mma_commit(pv_bar);
           mma_commit(empty_bar(st));  // the stage is free once these MMAs are done
           ++pv_commits;
@@ -520,48 +634,59 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         }
         if (named_barrier_or(1, kComputeThreads, !ok || *abort_flag)) { ok = false; break; }
         tc_fence_after();
-        float ov[16];
-        tmem_ld16(tmem + t_lane + kN, ov);
+        float ov[N];
+        tmem_ld<N>(tmem + t_lane + N, ov);
 #pragma unroll
-        for (int h = 0; h < G; ++h) acc[h] = acc[h] * alpha[h] + ov[h];
+        for (int c = 0; c < NC; ++c) acc[c] = acc[c] * alpha[c] + ov[c];
         tc_fence_before();
       }
       if (!ok) break;
 
       // ---- item result: reduce the per-token sums, write output or partial
-      float lsum[G];
+      {
+        float t[NC];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float v = l_tok[h];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        lsum[h] = v;
+        for (int c = 0; c < NC; ++c) t[c] = l_tok[c];
+        const float wsum = column_reduce<NC, false>(t, lane);
+        named_barrier(1, kComputeThreads);  // `red` and `stat` of the last tile have been read
+        if (lane < NC) red[warp * N + lane] = wsum;
       }
-      named_barrier(1, kComputeThreads);  // the tile maxima in `red` have been read
-      if (lane == 0)
-#pragma unroll
-        for (int h = 0; h < G; ++h) red[warp * kN + h] = lsum[h];
       named_barrier(1, kComputeThreads);
-      const int d = tid;  // output element this thread writes, per head
-      const size_t qh0 = (size_t)s * a.num_q_heads + (size_t)kvh * G;
+      if (warp == 0 && lane < NC)
+        stat[N + lane] = (red[lane] + red[N + lane]) + (red[2 * N + lane] + red[3 * N + lane]);
+      named_barrier(1, kComputeThreads);
+      const int d = tid;  // output element this thread writes, per column
+      const int cols = GROUP ? ctx_or_members * G : G;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float L_h = red[h] + red[kN + h] + red[2 * kN + h] + red[3 * kN + h];
-        const size_t qh = qh0 + h;
-        if (ctx == 0) {
+      for (int c = 0; c < NC; ++c) {
+        if (c >= cols) break;
+        const float M = stat[c], L_c = stat[N + c];
+        const int m = GROUP ? c / G : 0, h = GROUP ? c % G : c;
+        const size_t qh = (size_t)(s + m) * a.num_q_heads + (size_t)kvh * G + h;
+        bool zero = false, direct;
+        if constexpr (GROUP) {
+          // shared partitions of the member, plus its private ones
+          const int4 pl = __ldg(a.plan + s + m);
+          const int ctx = max(0, min(__ldg(a.context_lens + s + m), a.max_context_len));
+          direct = pl.w + (ctx > pl.z ? (ctx - pl.z + PT - 1) / PT : 0) <= 1;
+        } else {
+          zero = ctx_or_members == 0;
+          direct = n_parts <= 1;
+        }
+        if (zero) {
           a.out[qh * kD + d] = 0;
-        } else if (n_parts <= 1) {
-          a.out[qh * kD + d] = Elem<T>::from_f(acc[h] / L_h);
+        } else if (direct) {
+          a.out[qh * kD + d] = Elem<T>::from_f(acc[c] / L_c);
         } else {
           const size_t wslot = qh * a.num_parts + part;
-          a.ws_acc[wslot * kD + d] = acc[h];
+          a.ws_acc[wslot * kD + d] = acc[c];
           if (d == 0) {
-            a.ws_ml[2 * wslot] = m_run[h];
-            a.ws_ml[2 * wslot + 1] = L_h;
+            a.ws_ml[2 * wslot] = M;
+            a.ws_ml[2 * wslot + 1] = L_c;
           }
         }
       }
-      named_barrier(1, kComputeThreads);  // `red` is reused by the next item
+      named_barrier(1, kComputeThreads);  // `stat` and `red` are reused by the next item
       if (lane == 0) mbar_arrive(free_bar(slot));  // its query rows have been used
     }
     if (!ok && tid == 0) *abort_flag = 1;
@@ -576,7 +701,8 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(C::kTmemCols)
                  : "memory");
   }
 }
@@ -594,11 +720,12 @@ int sm_count() {
   return count[dev];
 }
 
-template <typename T, int G>
+template <typename T, int G, bool GROUP>
 cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& tq, cudaStream_t stream, int* launches) {
-  using L = Layout<kStagesTc>;
-  auto* kern = decode_tc_kernel<T, G, kStagesTc>;
+  using C = Cfg<GROUP>;
+  using L = Layout<kStagesTc, C::kN, C::kMaxSeqs>;
+  auto* kern = decode_tc_kernel<T, G, kStagesTc, GROUP>;
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
@@ -606,19 +733,23 @@ cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUte
     configured = true;
   }
   const int sms = sm_count();
-  for (int s0 = 0; s0 < a0.num_seqs; s0 += kMaxSeqs) {
+  constexpr int kChunk = C::kMaxSeqs;
+  for (int s0 = 0; s0 < a0.num_seqs; s0 += kChunk) {
     DecodeArgs a = a0;
-    a.num_seqs = a0.num_seqs - s0 < kMaxSeqs ? a0.num_seqs - s0 : kMaxSeqs;
+    a.num_seqs = a0.num_seqs - s0 < kChunk ? a0.num_seqs - s0 : kChunk;
     a.seq_offset = s0;
     a.out = a0.out + (size_t)s0 * a0.num_q_heads * kD;
     a.block_tables = a0.block_tables + (size_t)s0 * a0.max_blocks_per_seq;
     a.context_lens = a0.context_lens + s0;
+    if (a0.plan) a.plan = a0.plan + s0;
     if (a0.ws_acc) {
       a.ws_acc = a0.ws_acc + (size_t)s0 * a0.num_q_heads * a0.num_parts * kD;
       a.ws_ml = a0.ws_ml + (size_t)s0 * a0.num_q_heads * a0.num_parts * 2;
     }
-    a.epoch = a0.epoch + (unsigned long long)(s0 / kMaxSeqs);
-    const int items0 = a.num_seqs * a.num_kv_heads;
+    a.epoch = a0.epoch + (unsigned long long)(s0 / kChunk);
+    // plain: at least one item per (sequence, kv head); shared-prefix: the
+    // number of items is only known on the device
+    const int items0 = GROUP ? sms : a.num_seqs * a.num_kv_heads;
     const int grid = items0 < sms ? items0 : sms;
     cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kThreads), L::kAlloc, stream, a, tk, tv, tq);
     if (e != cudaSuccess) return e;
@@ -627,15 +758,15 @@ cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUte
   return cudaSuccess;
 }
 
-template <typename T>
+template <typename T, bool GROUP>
 cudaError_t launch_group(const DecodeArgs& a, int G, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& tq, cudaStream_t st, int* n) {
   switch (G) {
-    case 1: return launch_typed<T, 1>(a, tk, tv, tq, st, n);
-    case 2: return launch_typed<T, 2>(a, tk, tv, tq, st, n);
-    case 4: return launch_typed<T, 4>(a, tk, tv, tq, st, n);
-    case 8: return launch_typed<T, 8>(a, tk, tv, tq, st, n);
-    case 16: return launch_typed<T, 16>(a, tk, tv, tq, st, n);
+    case 1: return launch_typed<T, 1, GROUP>(a, tk, tv, tq, st, n);
+    case 2: return launch_typed<T, 2, GROUP>(a, tk, tv, tq, st, n);
+    case 4: return launch_typed<T, 4, GROUP>(a, tk, tv, tq, st, n);
+    case 8: return launch_typed<T, 8, GROUP>(a, tk, tv, tq, st, n);
+    case 16: return launch_typed<T, 16, GROUP>(a, tk, tv, tq, st, n);
   }
   return cudaErrorInvalidValue;
 }
@@ -646,8 +777,15 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, int dtype, int group, const CU
                              const CUtensorMap& tv, const CUtensorMap& tq, cudaStream_t stream,
                              int* launches) {
   if (a.num_seqs <= 0) return cudaSuccess;
-  if (dtype == 0) return tc::launch_group<__half>(a, group, tk, tv, tq, stream, launches);
-  return tc::launch_group<__nv_bfloat16>(a, group, tk, tv, tq, stream, launches);
+  if (dtype == 0) return tc::launch_group<__half, false>(a, group, tk, tv, tq, stream, launches);
+  return tc::launch_group<__nv_bfloat16, false>(a, group, tk, tv, tq, stream, launches);
+}
+
+cudaError_t launch_decode_shared_tc(const DecodeArgs& a, int dtype, int group, const CUtensorMap& tk,
+                                    const CUtensorMap& tv, cudaStream_t stream, int* launches) {
+  if (a.num_seqs <= 0 || !a.plan) return cudaSuccess;
+  if (dtype == 0) return tc::launch_group<__half, true>(a, group, tk, tv, tk, stream, launches);
+  return tc::launch_group<__nv_bfloat16, true>(a, group, tk, tv, tk, stream, launches);
 }
 
 int decode_tc_tile_tokens() { return tc::kTile; }

@@ -24,7 +24,49 @@ struct DecodeArgs {
   unsigned long long* work_counter;  // first 8 bytes of the workspace (tensor-core path)
   unsigned long long epoch;      // tag of this call's launches (< 2^40, never 0)
   int seq_offset;                // first sequence of this launch in the whole batch
+  // Shared-prefix decode (nullptr: off): per sequence {rank in its group,
+  // members, shared tokens T, shared partitions}.  A sequence's own items
+  // then cover [T, ctx), as partitions numbered from its shared partitions.
+  const int4* plan;
+  int grid_parts;                // partitions per (sequence, kv head) of the CUDA-core grid
 };
+
+// Sequences per launch of the shared-prefix kernel; groups never cross a
+// multiple of it.
+constexpr int kSharedPrefixSeqsPerLaunch = 256;
+
+// Arguments of the plan kernel (pa_plan.cu).
+struct PlanArgs {
+  const int32_t* block_tables;   // [S][MBS]
+  const int32_t* context_lens;   // [S]
+  int4* plan;                    // [S] out
+  int num_seqs, max_blocks_per_seq, block_size, num_blocks, max_context_len;
+  int partition_tokens;
+  int max_members;               // members per group (32 / g)
+  int min_shared;                // fewer shared tokens than this: no group
+  int chunk;                     // groups stay inside [k * chunk, (k + 1) * chunk)
+};
+cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream, int* launches);
+
+// Tokens [T, ctx) of sequence s with a plan: its first own partition, the
+// workspace slot of that partition, and the sequence's partition count.
+struct SeqSplit {
+  int base, slot0, total;
+};
+__host__ __device__ inline SeqSplit seq_split(const int4* plan, int s, int ctx, int partition_tokens) {
+  int base = 0, slot0 = 0;
+  if (plan) {
+#ifdef __CUDA_ARCH__
+    const int4 pl = __ldg(plan + s);
+#else
+    const int4 pl = plan[s];
+#endif
+    base = pl.z;
+    slot0 = pl.w;
+  }
+  const int own = ctx > base ? (ctx - base + partition_tokens - 1) / partition_tokens : 0;
+  return {base, slot0, slot0 + own};
+}
 
 // Launch the partition kernel (+ the merge kernel when num_parts > 1).
 // `launches` is incremented once per kernel launched.
@@ -43,6 +85,10 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, int dtype, int group, const CU
                              const CUtensorMap& tm_v, const CUtensorMap& tm_q, cudaStream_t stream,
                              int* launches);
 int decode_tc_tile_tokens();
+// The shared-prefix kernel (a.plan set): items over the shared partitions of
+// every group, members x g query rows per tile.
+cudaError_t launch_decode_shared_tc(const DecodeArgs& a, int dtype, int group, const CUtensorMap& tm_k,
+                                    const CUtensorMap& tm_v, cudaStream_t stream, int* launches);
 
 cudaError_t launch_cache_append(const void* k, const void* v, const int32_t* slot_mapping,
                                 int num_tokens, void* k_cache, void* v_cache, long long num_slots,

@@ -1,0 +1,136 @@
+// pa_plan.cu -- which sequences of a decode batch share a prefix of physical
+// blocks, and how much of it.
+//
+// Sequences forked from one parent (beam candidates) or admitted with a common
+// prompt hold the same physical blocks at the start of their block tables
+// (zingnex.cn, "vLLM与PagedAttention深度剖析", section 3.2 item 3: blocks are
+// shared by reference count and copied only on write; jsqmd.com,
+// "vLLM-v0.11.0性能实测", section 4.2: requests with the same prefix share
+// pages).  The shared-prefix decode reads those blocks once per group of
+// sequences instead of once per sequence.  This kernel finds the groups on the
+// device, from the block tables alone:
+//
+//   - a run is a maximal range of consecutive sequences, inside one launch
+//     chunk, with context > 0 and the same first table entry;
+//   - a run is cut into groups of at most `max_members` consecutive
+//     sequences (members x g query rows fit one tile of the shared kernel);
+//   - the group shares its first T tokens, where T = block_size x (number of
+//     leading table entries equal in every member, counted only below every
+//     member's own block count), capped at the shortest member context, and
+//     rounded down to 16 tokens (one TMA box);
+//   - a group whose T is under `min_shared` tokens is not worth a second
+//     pass: its members stay alone.
+//
+// plan[s] = {rank of s in its group (0 = the leader), members, T, shared
+// partitions ceil(T / partition_tokens)}; a sequence alone gets {0, 1, 0, 0}.
+// Tokens [0, T) of every member are then computed by the group's items, and
+// [T, ctx) by the member's own items, as further split-K partitions.
+#include <cuda_runtime.h>
+
+#include <climits>
+
+#include "pa_common.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+namespace {
+
+constexpr int kPlanThreads = 128;
+
+__device__ __forceinline__ int clamp_ctx(const PlanArgs& p, int s) {
+  const int c = __ldg(p.context_lens + s);
+  return max(0, min(c, p.max_context_len));
+}
+
+// First table entry of s, or -1 when s cannot share (empty context, or an
+// entry outside the pool: the decode reports those itself).
+__device__ __forceinline__ int first_block(const PlanArgs& p, int s) {
+  if (clamp_ctx(p, s) <= 0) return -1;
+  const int b = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq);
+  return (b >= 0 && b < p.num_blocks) ? b : -1;
+}
+
+// One CTA per sequence.
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p) {
+  pdl_wait();  // the tables and lengths of this step are written
+  pdl_launch_dependents();
+  __shared__ int sh_edge, sh_min_ctx, sh_min_blocks, sh_common;
+  const int s = blockIdx.x, tid = threadIdx.x;
+  const int first = first_block(p, s);
+  int4 out = make_int4(0, 1, 0, 0);
+  if (first >= 0) {
+    const int c0 = (s / p.chunk) * p.chunk;
+    const int c1 = min(p.num_seqs, c0 + p.chunk);
+    // ---- run start: the sequence after the nearest break below s
+    int a = c0;
+    for (int base = s - 1; base >= c0; base -= kPlanThreads) {
+      if (tid == 0) sh_edge = -1;
+      __syncthreads();
+      const int sp = base - tid;
+      if (sp >= c0 && first_block(p, sp) != first) atomicMax(&sh_edge, sp);
+      __syncthreads();
+      const int e = sh_edge;
+      __syncthreads();
+      if (e >= 0) { a = e + 1; break; }
+    }
+    // ---- run end (exclusive): the nearest break above s
+    int b = c1;
+    for (int base = s + 1; base < c1; base += kPlanThreads) {
+      if (tid == 0) sh_edge = INT_MAX;
+      __syncthreads();
+      const int sp = base + tid;
+      if (sp < c1 && first_block(p, sp) != first) atomicMin(&sh_edge, sp);
+      __syncthreads();
+      const int e = sh_edge;
+      __syncthreads();
+      if (e != INT_MAX) { b = e; break; }
+    }
+    const int leader = a + ((s - a) / p.max_members) * p.max_members;
+    const int n = min(p.max_members, b - leader);
+    if (n >= 2) {
+      // ---- shortest member context and block count
+      if (tid == 0) sh_min_ctx = INT_MAX, sh_min_blocks = INT_MAX;
+      __syncthreads();
+      if (tid < n) {
+        const int c = clamp_ctx(p, leader + tid);
+        atomicMin(&sh_min_ctx, c);
+        atomicMin(&sh_min_blocks, (c + p.block_size - 1) / p.block_size);
+      }
+      __syncthreads();
+      if (tid == 0) sh_common = sh_min_blocks;
+      __syncthreads();
+      // ---- leading table entries every member has in common with the leader
+      const int32_t* lead = p.block_tables + (size_t)leader * p.max_blocks_per_seq;
+      for (int m = 1; m < n; ++m) {
+        const int32_t* row = p.block_tables + (size_t)(leader + m) * p.max_blocks_per_seq;
+        for (int j0 = 0;; j0 += kPlanThreads) {
+          const int lim = sh_common;  // the same in every thread: read between barriers
+          __syncthreads();
+          if (j0 >= lim) break;
+          const int j = j0 + tid;
+          if (j < lim && __ldg(row + j) != __ldg(lead + j)) atomicMin(&sh_common, j);
+          __syncthreads();
+        }
+      }
+      const long long t = min((long long)sh_common * p.block_size, (long long)sh_min_ctx);
+      const int shared = (int)(t & ~15LL);
+      if (shared >= p.min_shared) {
+        out = make_int4(s - leader, n, shared,
+                        (shared + p.partition_tokens - 1) / p.partition_tokens);
+      }
+    }
+  }
+  if (tid == 0) p.plan[s] = out;
+}
+
+}  // namespace
+
+cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream, int* launches) {
+  if (p.num_seqs <= 0) return cudaSuccess;
+  cudaError_t e = launch_pdl(plan_kernel, dim3(p.num_seqs), dim3(kPlanThreads), 0, stream, p);
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
+}  // namespace pa

@@ -466,6 +466,53 @@ def valid_slot_mask(block_tables: np.ndarray, context_lens: np.ndarray, num_bloc
     return valid
 
 
+def grouped_decode_case(rng: np.random.Generator, *, groups, num_q_heads: int,
+                        num_kv_heads: int, head_dim: int, block_size: int, dtype: int,
+                        poison: bool = True):
+    """A decode input whose consecutive sequences come in groups sharing a prefix.
+
+    ``groups`` is a list of ``(shared_tokens, [context of each member])``.
+    The members' tables start with the blocks of a parent that holds
+    ``shared_tokens`` tokens (its last block may be partly filled, and the
+    members then continue in it, as forks of one prompt do before they
+    diverge) and go on with private blocks; a member shorter than the shared
+    part keeps only its own prefix of it.  Blocks come from a random
+    permutation of the pool.  Returns a dict like ``random_decode_case``.
+    """
+    bs = block_size
+    ctx = [int(c) for _, members in groups for c in members]
+    need = sum(-(-int(sh) // bs) for sh, _ in groups) + sum(-(-c // bs) for c in ctx) + 2
+    NB = max(need, 4)
+    mgr = BlockManager(NB, bs, rng.permutation(NB))
+    s = 0
+    for gi, (shared, members) in enumerate(groups):
+        parent = ("parent", gi)
+        mgr.add_seq(parent, int(shared))
+        for c in members:
+            mgr.fork(parent, s)
+            if c >= shared:
+                mgr.extend(s, c - int(shared))
+            else:
+                mgr.tables[s] = mgr.tables[s][:-(-c // bs)]
+                mgr.lens[s] = c
+            s += 1
+    S = s
+    MBS = max(1, -(-max(ctx, default=0) // bs))
+    bt = mgr.table_array(list(range(S)), MBS)
+    cl = mgr.lens_array(list(range(S)))
+    q = normal_bits(rng, (S, num_q_heads, head_dim), dtype)
+    kc = normal_bits(rng, (NB, bs, num_kv_heads, head_dim), dtype)
+    vc = normal_bits(rng, (NB, bs, num_kv_heads, head_dim), dtype)
+    if poison:
+        valid = valid_slot_mask(bt, cl, NB, bs)
+        nan = np.uint16(NAN_BITS[dtype])
+        kc.reshape(NB * bs, -1)[~valid] = nan
+        vc.reshape(NB * bs, -1)[~valid] = nan
+    return dict(q=q, k_cache=kc, v_cache=vc, block_tables=bt, context_lens=cl,
+                num_blocks=NB, max_blocks_per_seq=MBS,
+                scale=float(np.float32(1.0 / math.sqrt(head_dim))))
+
+
 def random_decode_case(rng: np.random.Generator, *, num_seqs: int, num_q_heads: int,
                        num_kv_heads: int, head_dim: int, block_size: int, dtype: int,
                        context_lens, num_blocks: int | None = None, poison: bool = True,

@@ -20,6 +20,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "pa.h")
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_OOM, PA_ERR_DEVICE_CHECK = range(6)
 PA_F16, PA_BF16 = 0, 1
 PA_DECODE_AUTO, PA_DECODE_CUDA_CORES, PA_DECODE_TENSOR_CORES = 0, 1, 2
+PA_DECODE_RESOLVED_SHARED_PREFIX = 3
 PA_DEVERR_BLOCK_ID = 0x1
 PA_DEVERR_CONTEXT_LEN = 0x2
 PA_DEVERR_SLOT = 0x4
@@ -43,7 +44,7 @@ class PaError(RuntimeError):
 class pa_shape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "num_seqs", "num_q_heads", "num_kv_heads", "head_dim", "block_size", "num_blocks",
-        "max_blocks_per_seq", "partition_tokens", "dtype", "variant")]
+        "max_blocks_per_seq", "partition_tokens", "dtype", "variant", "shared_prefix")]
 
     def __repr__(self):
         return "pa_shape(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -153,9 +154,10 @@ def _stream(stream) -> int | None:
 
 
 def make_shape(*, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
-               max_blocks_per_seq, partition_tokens=0, dtype=PA_F16, variant=0) -> pa_shape:
+               max_blocks_per_seq, partition_tokens=0, dtype=PA_F16, variant=0,
+               shared_prefix=0) -> pa_shape:
     return pa_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
-                    max_blocks_per_seq, partition_tokens, dtype, variant)
+                    max_blocks_per_seq, partition_tokens, dtype, variant, shared_prefix)
 
 
 def torch_dtype(dtype: int):

@@ -18,12 +18,21 @@ def host_bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
+# Decode modes of the tests: the three values of pa_shape.variant, and
+# SHARED = automatic variant with shared_prefix on.
+SHARED = 3
+MODES = {0: "auto", 1: "cuda_cores", 2: "tensor_cores", SHARED: "shared_prefix"}
+
+
 def shape_of(dtype, q, k_cache, block_tables, partition_tokens=0, variant=0):
+    """pa_shape of host arrays; variant SHARED means automatic + shared_prefix."""
     S, Hq, D = q.shape
     NB, bs, Hkv, _ = k_cache.shape
+    shared = int(variant == SHARED)
     return pa.make_shape(num_seqs=S, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D, block_size=bs,
                          num_blocks=NB, max_blocks_per_seq=block_tables.shape[1],
-                         partition_tokens=partition_tokens, dtype=dtype, variant=variant)
+                         partition_tokens=partition_tokens, dtype=dtype,
+                         variant=0 if shared else variant, shared_prefix=shared)
 
 
 def gpu_decode(dtype, q, k_cache, v_cache, block_tables, context_lens, scale, partition_tokens=0,

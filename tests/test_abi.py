@@ -55,11 +55,29 @@ FAKE = 1 << 20  # a 16-byte-aligned non-null address; validation fails before an
     (dict(variant=2, head_dim=64), pa.PA_ERR_UNSUPPORTED),
     (dict(variant=2, partition_tokens=64), pa.PA_ERR_UNSUPPORTED),
     (dict(variant=2, partition_tokens=1024), pa.PA_ERR_UNSUPPORTED),
+    (dict(shared_prefix=2), pa.PA_ERR_INVALID_ARG),
+    (dict(shared_prefix=1, variant=1), pa.PA_ERR_UNSUPPORTED),
+    (dict(shared_prefix=1, variant=2), pa.PA_ERR_UNSUPPORTED),
+    (dict(shared_prefix=1, head_dim=64), pa.PA_ERR_UNSUPPORTED),
+    (dict(shared_prefix=1, partition_tokens=1024), pa.PA_ERR_UNSUPPORTED),
+    (dict(shared_prefix=1, partition_tokens=192), pa.PA_ERR_UNSUPPORTED),
 ])
 def test_decode_rejects_bad_shapes(lib, kw, expect):
     s = _shape(**kw)
     st = lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s), 100, FAKE, 1 << 20, None)
     assert st == expect
+
+
+def test_shared_prefix_workspace(lib):
+    """Counter, plan (16 B per sequence, 256-aligned), split-K space for P + 1 partitions."""
+    s = _shape(shared_prefix=1)
+    rows = 4 * 8 * 2                       # S * Hq * (1 partition + 1)
+    acc = rows * 128 * 4
+    assert lib.pa_decode_workspace_bytes(ctypes.byref(s), 100) == 256 + 256 + acc + rows * 8
+    s20 = _shape(shared_prefix=1, num_seqs=20, max_blocks_per_seq=64)
+    rows = 20 * 8 * 3                      # 1000 tokens: 2 partitions + 1
+    assert lib.pa_decode_workspace_bytes(ctypes.byref(s20), 1000) == 256 + 512 + rows * 128 * 4 + rows * 8
+    assert pa.pa_decode_resolved_variant(s) == pa.PA_DECODE_RESOLVED_SHARED_PREFIX
 
 
 def test_resolved_variant(lib):

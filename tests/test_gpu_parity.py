@@ -12,7 +12,7 @@ torch = pytest.importorskip("torch")
 
 from paged_kv_cache_458_b200 import gen, pa  # noqa: E402
 import golden_cases  # noqa: E402
-from gpu_util import dev, dev_i32, gpu_decode, host_bits, shape_of  # noqa: E402
+from gpu_util import MODES, SHARED, dev, dev_i32, gpu_decode, host_bits, shape_of  # noqa: E402
 from tolerance import assert_decode_close  # noqa: E402
 
 pytestmark = pytest.mark.gpu
@@ -48,7 +48,7 @@ def test_golden_block_mapping(case):
 # ---------------------------------------------------------------- full workloads
 
 
-VARIANTS = {0: "auto", 1: "cuda_cores", 2: "tensor_cores"}
+VARIANTS = MODES
 
 
 @pytest.fixture(scope="module")
@@ -108,7 +108,7 @@ def test_tiny_workload(workload_refs):
 
 
 @pytest.mark.parametrize("name", ["llama2_7b", "mistral_7b_gqa", "qwen_7b_prefix", "llama2_70b_beam"])
-@pytest.mark.parametrize("variant", [0, 1, 2], ids=lambda v: VARIANTS[v])
+@pytest.mark.parametrize("variant", [0, 1, 2, SHARED], ids=lambda v: VARIANTS[v])
 def test_full_workload(workload_refs, name, variant):
     case, s0, s1 = _run_workload(workload_refs, name, variant)
     if name == "llama2_70b_beam":
@@ -121,13 +121,13 @@ def test_full_workload(workload_refs, name, variant):
 EDGE_CTX = [0, 1, 15, 16, 17, 31, 33, 511, 512, 513, 1023, 1024, 1025, 2047, 2049]
 
 
-@pytest.mark.parametrize("variant", [1, 2], ids=lambda v: VARIANTS[v])
+@pytest.mark.parametrize("variant", [1, 2, SHARED], ids=lambda v: VARIANTS[v])
 @pytest.mark.parametrize("dtype", [gen.F16, gen.BF16], ids=["f16", "bf16"])
 @pytest.mark.parametrize("head_dim", [64, 128])
 @pytest.mark.parametrize("group", [1, 2, 4, 8, 16])
 def test_edge_contexts(orc, dtype, head_dim, group, variant):
-    if variant == 2 and head_dim != 128:
-        pytest.skip("the tensor-core variant is built for head_dim 128")
+    if variant in (2, SHARED) and head_dim != 128:
+        pytest.skip("the tensor-core kernels are built for head_dim 128")
     rng = np.random.default_rng(1000 * group + head_dim + dtype)
     Hkv = 2
     c = gen.random_decode_case(rng, num_seqs=len(EDGE_CTX), num_q_heads=Hkv * group,
@@ -141,12 +141,12 @@ def test_edge_contexts(orc, dtype, head_dim, group, variant):
     assert np.all(out[0] == 0), "an empty context must give a zero row"
 
 
-@pytest.mark.parametrize("variant", [1, 2], ids=lambda v: VARIANTS[v])
+@pytest.mark.parametrize("variant", [1, 2, SHARED], ids=lambda v: VARIANTS[v])
 @pytest.mark.parametrize("block_size", [16, 32, 256])
 @pytest.mark.parametrize("partition_tokens", [16, 48, 128, 256, 512, 2048])
 def test_block_and_partition_sizes(orc, block_size, partition_tokens, variant):
-    if variant == 2 and (partition_tokens % 128 or partition_tokens > 512):
-        pytest.skip("the tensor-core variant takes partitions of 128, 256, 384 or 512 tokens")
+    if variant in (2, SHARED) and (partition_tokens % 128 or partition_tokens > 512):
+        pytest.skip("the tensor-core kernels take partitions of 128, 256, 384 or 512 tokens")
     rng = np.random.default_rng(block_size * 7 + partition_tokens)
     ctx = [1, 47, 48, 49, 255, 256, 257, 700, 2048, 2100]
     c = gen.random_decode_case(rng, num_seqs=len(ctx), num_q_heads=8, num_kv_heads=2,
@@ -160,7 +160,7 @@ def test_block_and_partition_sizes(orc, block_size, partition_tokens, variant):
     assert_decode_close(out, ref, gen.BF16, f"bs{block_size} pt{partition_tokens}")
 
 
-@pytest.mark.parametrize("variant", [1, 2], ids=lambda v: VARIANTS[v])
+@pytest.mark.parametrize("variant", [1, 2, SHARED], ids=lambda v: VARIANTS[v])
 def test_last_physical_block_and_stale_entries(orc, variant):
     rng = np.random.default_rng(3)
     c = gen.random_decode_case(rng, num_seqs=3, num_q_heads=4, num_kv_heads=4, head_dim=128,
@@ -194,7 +194,7 @@ def test_all_contexts_empty():
     assert np.all(out == 0)
 
 
-@pytest.mark.parametrize("variant", [1, 2], ids=lambda v: VARIANTS[v])
+@pytest.mark.parametrize("variant", [1, 2, SHARED], ids=lambda v: VARIANTS[v])
 def test_permutation_invariance_and_determinism(variant):
     rng = np.random.default_rng(5)
     c = gen.random_decode_case(rng, num_seqs=6, num_q_heads=16, num_kv_heads=2, head_dim=128,

@@ -265,7 +265,15 @@ pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
   a.max_blocks_per_seq = shape->max_blocks_per_seq;
   a.partition_tokens = effective_partition(shape);
   a.num_parts = P_ws > 0 ? P_ws : 1;
-  a.grid_parts = P > 0 ? P : 1;
+  // With shared_prefix a sequence's own tokens (beam tails, private
+  // continuations of a shared prompt) are mostly short: the CUDA-core kernel
+  // takes them in partitions of its largest size, so its grid holds few empty
+  // CTAs and each sequence adds few partials.
+  a.own_tokens = shape->shared_prefix ? pa::decode_max_partition_tokens() : a.partition_tokens;
+  {
+    const int gp = (max_context_len + a.own_tokens - 1) / a.own_tokens;
+    a.grid_parts = gp > 0 ? gp : 1;
+  }
   a.max_context_len = max_context_len;
   a.err = error_word();
   if (!a.err) return cuda_failed("device error word lookup failed");

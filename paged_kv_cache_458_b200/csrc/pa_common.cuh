@@ -97,6 +97,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t phase) {
   return ok != 0;
 }
 
+// Non-blocking probe: has phase `phase` completed?  (test_wait never suspends.)
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t phase) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(phase)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }

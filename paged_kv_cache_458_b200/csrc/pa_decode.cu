@@ -140,7 +140,6 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
     if (part == 0 && kvh == 0 && threadIdx.x == 0) report(a.err, kErrContextLen);
     ctx = max(0, min(ctx, ctx_cap));
   }
-  const int PT = a.partition_tokens;
   const int q_head0 = kvh * G;
   if (ctx == 0) {
     if (part == 0) {
@@ -150,10 +149,11 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
     return;
   }
   // With a shared-prefix plan this CTA covers part of [T, ctx) only.
-  const SeqSplit split = seq_split(a.plan, s, ctx, PT);
-  const int t_begin = split.base + part * PT;
+  const int OT = a.own_tokens;
+  const SeqSplit split = seq_split(a.plan, s, ctx, OT);
+  const int t_begin = split.base + part * OT;
   if (t_begin >= ctx) return;
-  const int t_end = min(ctx, t_begin + PT);
+  const int t_end = min(ctx, t_begin + OT);
   const int n_parts_seq = split.total;
   const int n_chunks = (t_end - t_begin + kChunk - 1) / kChunk;
   const int n_mine = warp < n_chunks ? (n_chunks - warp + NW - 1) / NW : 0;
@@ -365,7 +365,7 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a) {
   const int s = pair / a.num_q_heads;
   int ctx = __ldg(a.context_lens + s);
   ctx = max(0, min(ctx, a.max_context_len));
-  const int P = seq_split(a.plan, s, ctx, a.partition_tokens).total;
+  const int P = seq_split(a.plan, s, ctx, a.own_tokens).total;
   if (P <= 1) return;
   const size_t base = (size_t)pair * a.num_parts;
   float M = -INFINITY;

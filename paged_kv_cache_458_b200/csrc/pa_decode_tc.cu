@@ -22,10 +22,15 @@
 //     share pages).
 //
 // The softmax stays in fp32 on the CUDA cores: tcgen05.ld gives thread t (of
-// 128) the N logits of token t; the per-column tile maximum is a transposed
-// warp reduction (lane c ends with column c) plus shared memory, and thread t
-// writes its row of P.  After the PV product thread d reads row d of O^T and
-// folds it into its running output (rescaled by 2^(m_old - m_new) per column).
+// 128) the N logits of token t, and thread t writes its row of P.  The
+// output accumulates in TMEM across the tiles of an item: each column keeps a
+// softmax reference m_ref that moves only when a logit exceeds it by more than
+// 8 (log2 units).  Then the tile's column maxima are found (a transposed warp
+// reduction, lane c ending with column c, plus shared memory), and thread d
+// folds row d of O^T into registers, rescaled by 2^(m_old - m_new).  On other
+// tiles nothing waits for the PV product: it is read once, at the end of the
+// item.  The products are pipelined by tile: S^T(j+1) is issued as soon as
+// every thread has read S^T(j), while tile j's softmax runs.
 // The probabilities enter the PV product as two terms of the input type, hi =
 // round(p) and lo = round(p - hi), so they carry about 16 significant bits (a
 // bf16 P alone, 8 bits, can move a short context's output by more than 2e-3);
@@ -67,8 +72,19 @@ constexpr int kTile = 128;          // tokens per MMA tile (M)
 constexpr int kD = 128;             // head_dim of this path
 constexpr int kGroupRows = 16;      // token rows per TMA box (a block is a multiple)
 constexpr int kSlots = 2;           // item slots (descriptor + query rows)
-constexpr int kComputeThreads = 128;
-constexpr int kThreads = kComputeThreads + 32;
+
+// Compute warpgroups split the NC query columns: warp w of the compute
+// warps reads TMEM lane quarter w % 4 (tokens 32 (w % 4) .. +31, output rows
+// likewise) and handles columns [(w / 4) NCW, (w / 4 + 1) NCW).  More warps
+// per scheduler hide the latency of the per-column softmax arithmetic.
+template <int NC>
+struct Warps {
+  static constexpr int kNCW = NC >= 16 ? 8 : (NC >= 8 ? 4 : NC);  // columns per warpgroup
+  static constexpr int kNWG = NC / kNCW;                           // compute warpgroups
+  static constexpr int kCompute = 128 * kNWG;                      // compute threads
+  static constexpr int kThreads = kCompute + 32;                   // + the producer warp
+  static_assert(kNCW * kNWG == NC, "columns split evenly");
+};
 
 // Per kernel kind: N columns, sequences per launch (their prefix sums live in
 // shared memory) and TMEM columns (S^T in [0, N), O^T in [N, 2N)).
@@ -95,8 +111,8 @@ struct Layout {
   static constexpr int kDesc = kStat + 2 * N * 4;              // [slots][8] int
   static constexpr int kPrefix = kDesc + kSlots * 8 * 4;       // [MAXSEQS + 1] int
   static constexpr int kBars = (kPrefix + (MAXSEQS + 1) * 4 + 7) / 8 * 8;
-  // full[NST], empty[NST], ready[slots], free[slots], qk, pv
-  static constexpr int kNumBars = 2 * NST + 2 * kSlots + 2;
+  // full[NST], empty[NST], ready[slots], free[slots], qk, pv, drain
+  static constexpr int kNumBars = 2 * NST + 2 * kSlots + 3;
   static constexpr int kMisc = kBars + kNumBars * 8;           // tmem address, abort flag
   static constexpr int kUsed = kMisc + 16;
   static constexpr int kAlloc = kUsed + 1024;                  // room to align the base
@@ -149,11 +165,26 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-// N (16 or 32) consecutive fp32 columns of this thread's TMEM lane.
-template <int N>
-__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[N]) {
-  uint32_t r[N];
-  if constexpr (N == 16) {
+// NCOL (1 .. 32) consecutive fp32 columns of this thread's TMEM lane.
+template <int NCOL>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[NCOL]) {
+  uint32_t r[NCOL];
+  if constexpr (NCOL == 1) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r[0]) : "r"(taddr));
+  } else if constexpr (NCOL == 2) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];"
+                 : "=r"(r[0]), "=r"(r[1])
+                 : "r"(taddr));
+  } else if constexpr (NCOL == 4) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+  } else if constexpr (NCOL == 8) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+  } else if constexpr (NCOL == 16) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
         "%12, %13, %14, %15}, [%16];"
@@ -162,7 +193,7 @@ __device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[N]) {
           "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
   } else {
-    static_assert(N == 32, "16 or 32 columns");
+    static_assert(NCOL == 32, "1, 2, 4, 8, 16 or 32 columns");
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
         "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
@@ -176,7 +207,7 @@ __device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[N]) {
   }
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-  for (int i = 0; i < N; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < NCOL; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int c0, int c1) {
@@ -263,12 +294,15 @@ __device__ __forceinline__ int take_item(unsigned long long* ctr, unsigned long 
 }
 
 template <typename T, int G, int NST, bool GROUP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Warps<GROUP ? Cfg<GROUP>::kN : G>::kThreads, 1)
 decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q) {
   using C = Cfg<GROUP>;
   constexpr int N = C::kN;
   constexpr int NC = GROUP ? N : G;  // columns that carry query rows
+  using W = Warps<NC>;
+  constexpr int kComputeThreads = W::kCompute, kThreads = W::kThreads, NCW = W::kNCW;
+  constexpr int kProducerWarp = kComputeThreads / 32;
   using L = Layout<NST, N, C::kMaxSeqs>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr uint32_t kIdescQK = instr_desc(kBf16 ? 1 : 0, 0, 0, kTile, N);
@@ -295,6 +329,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   auto free_bar = [&](int sl) { return bars + (2 * NST + kSlots + sl) * 8; };
   const uint32_t qk_bar = bars + (2 * NST + 2 * kSlots) * 8;
   const uint32_t pv_bar = qk_bar + 8;
+  const uint32_t drain_bar = qk_bar + 16;
   const uint32_t sm_stages = smem_addr(smem + L::kStages);
   const uint32_t sm_q = smem_addr(smem + L::kQ);
   const uint32_t sm_p = smem_addr(smem + L::kP);
@@ -313,10 +348,11 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     }
     for (int sl = 0; sl < kSlots; ++sl) {
       mbar_init(ready_bar(sl), 1);
-      mbar_init(free_bar(sl), 4);
+      mbar_init(free_bar(sl), kComputeThreads / 32);
     }
     mbar_init(qk_bar, 1);
     mbar_init(pv_bar, 1);
+    mbar_init(drain_bar, 1);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -338,7 +374,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // =====================================================================
     // producer warp: items, table entries, query rows, TMA loads
     // =====================================================================
@@ -469,15 +505,14 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         const uint32_t fb = full_bar(st);
         const uint32_t dst = sm_stages + st * L::kStageBytes;
         if (lane == 0) mbar_arrive_expect_tx(fb, ng * 4 * kGroupRows * 128);
-        for (int r = 0; r < ng; ++r) {
-          const int row = __shfl_sync(0xffffffffu, my_row, g0 + r);
-          if (lane == 0) {
-            const uint32_t o = r * kGroupRows * 128;
-            tma_load_3d(dst + o, &tm_k, fb, 0, kvh, row);
-            tma_load_3d(dst + L::kHalf + o, &tm_k, fb, 64, kvh, row);
-            tma_load_3d(dst + 2 * L::kHalf + o, &tm_v, fb, 0, kvh, row);
-            tma_load_3d(dst + 3 * L::kHalf + o, &tm_v, fb, 64, kvh, row);
-          }
+        __syncwarp();
+        {
+          // lane 4 r + k loads piece k (K or V, 64-element half) of group r
+          const int r = lane >> 2, k = lane & 3;
+          const int row = __shfl_sync(0xffffffffu, my_row, min(g0 + r, 31));
+          if (r < ng)
+            tma_load_3d(dst + k * L::kHalf + r * kGroupRows * 128, k < 2 ? &tm_k : &tm_v, fb,
+                        (k & 1) * 64, kvh, row);
         }
         ++issued;
       }
@@ -496,12 +531,39 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         mbar_wait(full_bar(k % NST), (k / NST) & 1, a.err);
   } else {
     // =====================================================================
-    // compute warps (128 threads): thread t = token row t of S^T, row d = t of O^T
+    // compute warps: thread (t, cg) = token row t of S^T and row d = t of O^T,
+    // for the columns of warpgroup cg
     // =====================================================================
-    const uint32_t t_lane = ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lane quarter
-    int n_used = 0;       // tiles consumed (stage ring position, qk/pv phases)
-    int qk_commits = 0, pv_commits = 0;  // thread 0 only
+    // Tile j of an item: S^T(j) = K(j) . Q^T was issued during tile j-1 (or at
+    // the item start); thread 0 waits for it and for O^T(j-1); every thread
+    // reads its part of its S^T row, and as soon as all are read S^T(j+1) is
+    // issued (when its stage has landed; else after O^T(j)).  The softmax
+    // writes P, and O^T(j) += V^T . P^T is issued without waiting for it.  The
+    // output stays in TMEM across tiles: each column's softmax reference m_ref
+    // only moves when a logit exceeds it by more than kRescale (log2 units),
+    // and only then is O^T folded into registers and rescaled.  Hence p <=
+    // 2^kRescale, well inside fp32 and both operand types.
+    constexpr float kRescale = 8.f;
+    const int t = tid & 127;         // token row of S^T, output row of O^T
+    const int cg = tid >> 7;         // column group
+    const int c0 = cg * NCW;         // first column of this thread
+    const int quarter = warp & 3;    // TMEM lane quarter of this warp
+    const uint32_t t_lane = ((uint32_t)(quarter * 32) << 16);
+    int n_used = 0;  // tiles consumed: the stage ring position, and the number of
+                     // each tile's qk and pv commits (one of each per tile, in order)
     bool ok = true;
+    auto issue_qk = [&](int st, uint32_t q_addr) {  // thread 0
+      tc_fence_after();
+      const uint32_t kt = sm_stages + st * L::kStageBytes;
+#pragma unroll
+      for (int kk = 0; kk < kD / 16; ++kk) {
+        const uint32_t ko = (kk / 4) * L::kHalf + (kk % 4) * 32;
+        const uint32_t qo = (kk / 4) * N * 128 + (kk % 4) * 32;
+        mma_f16(tmem, smem_desc(kt + ko, 16, 1024, kSw128), smem_desc(q_addr + qo, 16, 1024, kSw128),
+                kIdescQK, kk > 0);
+      }
+      mma_commit(qk_bar);
+    };
     for (int it = 0; ok; ++it) {
       const int slot = it % kSlots;
       if (tid == 0) ok = mbar_wait_or_abort(ready_bar(slot), (it / kSlots) & 1, a.err, abort_flag);
@@ -512,112 +574,134 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       const int s = desc[kDS], kvh = desc[kDKvh], part = desc[kDPart];
       const int t_begin = desc[kDBegin], t_end = desc[kDEnd], n_parts = desc[kDParts];
       const int ctx_or_members = desc[kDCtx];
+      const int cols = GROUP ? ctx_or_members * G : G;
       const uint32_t q_addr = sm_q + slot * L::kQBytes;
 
-      float acc[NC], l_tok[NC];
+      float acc[NCW], l_tok[NCW], m_ref[NCW];
 #pragma unroll
-      for (int c = 0; c < NC; ++c) acc[c] = 0.f, l_tok[c] = 0.f;
-      float m_col = -INFINITY;  // warp 0, lane c < NC: running max of column c
+      for (int c = 0; c < NCW; ++c) acc[c] = 0.f, l_tok[c] = 0.f, m_ref[c] = -INFINITY;
+      bool pv_acc = false;  // O^T in TMEM holds tiles not folded into acc yet
 
+      if (tid == 0 && n_tiles > 0) {
+        const int st = n_used % NST;
+        ok = mbar_wait_or_abort(full_bar(st), (n_used / NST) & 1, a.err, abort_flag);
+        if (ok) issue_qk(st, q_addr);
+      }
       for (int j = 0; j < n_tiles; ++j, ++n_used) {
         const int st = n_used % NST;
-        const uint32_t kt = sm_stages + st * L::kStageBytes;
-        const uint32_t vt = kt + 2 * L::kHalf;
+        const int st_next = (n_used + 1) % NST;
+        const bool has_next = j + 1 < n_tiles;
+        const uint32_t vt = sm_stages + st * L::kStageBytes + 2 * L::kHalf;
         const int n_valid = min(kTile, t_end - (t_begin + j * kTile));
-        // ---- S^T = K . Q^T
-        if (tid == 0) {
-          ok = mbar_wait_or_abort(full_bar(st), (n_used / NST) & 1, a.err, abort_flag);
-          if (ok) {
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint32_t ko = (kk / 4) * L::kHalf + (kk % 4) * 32;
-              const uint32_t qo = (kk / 4) * N * 128 + (kk % 4) * 32;
-              mma_f16(tmem, smem_desc(kt + ko, 16, 1024, kSw128),
-                      smem_desc(q_addr + qo, 16, 1024, kSw128), kIdescQK, kk > 0);
-            }
-            mma_commit(qk_bar);
-            ++qk_commits;
-            ok = mbar_wait_or_abort(qk_bar, n_used & 1, a.err, abort_flag);
-          }
+        // ---- S^T(j) and O^T(j-1) are complete
+        if (tid == 0 && ok) {
+          ok = mbar_wait_or_abort(qk_bar, n_used & 1, a.err, abort_flag);
+          if (ok && j > 0) ok = mbar_wait_or_abort(pv_bar, (n_used - 1) & 1, a.err, abort_flag);
         }
         if (named_barrier_or(1, kComputeThreads, !ok || *abort_flag)) { ok = false; break; }
         tc_fence_after();
-        float sv[N];
-        tmem_ld<N>(tmem + t_lane, sv);
-
-        // ---- softmax over this tile (log2 domain)
-        const bool valid = tid < n_valid;
-        {
-          float t[NC];
+        float sv[NCW];
+        tmem_ld<NCW>(tmem + t_lane + (uint32_t)c0, sv);
+        const bool valid = t < n_valid;
+        bool over = false;
 #pragma unroll
-          for (int c = 0; c < NC; ++c) {
-            sv[c] = valid ? sv[c] * a.scale_log2 : -INFINITY;
-            t[c] = sv[c];
+        for (int c = 0; c < NCW; ++c) {
+          sv[c] = valid ? sv[c] * a.scale_log2 : -INFINITY;
+          over |= (c0 + c < cols) && (sv[c] > m_ref[c] + kRescale);
+        }
+        tc_fence_before();
+        // all S^T rows are read: its columns may take S^T(j+1)
+        const bool rescale = named_barrier_or(1, kComputeThreads, over);
+        bool next_issued = false;
+        if (tid == 0 && has_next && mbar_test_wait(full_bar(st_next), ((n_used + 1) / NST) & 1)) {
+          issue_qk(st_next, q_addr);
+          next_issued = true;
+        }
+        if (rescale) {
+          // new references: this tile's column maxima where they are higher
+          {
+            float tmp[NCW];
+#pragma unroll
+            for (int c = 0; c < NCW; ++c) tmp[c] = sv[c];
+            const float wmax = column_reduce<NCW, true>(tmp, lane);
+            if (lane < NCW) red[quarter * N + c0 + lane] = wmax;
           }
-          const float wmax = column_reduce<NC, true>(t, lane);
-          if (lane < NC) red[warp * N + lane] = wmax;
-        }
-        named_barrier(1, kComputeThreads);
-        if (warp == 0 && lane < NC) {
-          const float mt = fmaxf(fmaxf(red[lane], red[N + lane]), fmaxf(red[2 * N + lane], red[3 * N + lane]));
-          const float m_new = fmaxf(m_col, mt);
-          stat[N + lane] = exp2f(m_col - m_new);  // alpha
-          stat[lane] = m_new;
-          m_col = m_new;
-        }
-        named_barrier(1, kComputeThreads);
-        float alpha[NC], p[N];
+          named_barrier(1, kComputeThreads);
+          if (tid < NC)
+            stat[tid] = fmaxf(fmaxf(red[tid], red[N + tid]), fmaxf(red[2 * N + tid], red[3 * N + tid]));
+          named_barrier(1, kComputeThreads);
+          float alpha[NCW];
 #pragma unroll
-        for (int c = 0; c < NC; ++c) {
-          alpha[c] = stat[N + c];
-          p[c] = valid ? exp2f(sv[c] - stat[c]) : 0.f;
-          l_tok[c] = l_tok[c] * alpha[c] + p[c];
-        }
+          for (int c = 0; c < NCW; ++c) {
+            const float m_new = fmaxf(m_ref[c], stat[c0 + c]);
+            alpha[c] = exp2f(m_ref[c] - m_new);  // 0 while m_ref is -inf
+            m_ref[c] = m_new;
+            l_tok[c] *= alpha[c];
+          }
+          if (pv_acc) {
+            // fold O^T (tiles before j, complete) into acc, on the new reference
+            tc_fence_after();
+            float ov[NCW];
+            tmem_ld<NCW>(tmem + t_lane + (uint32_t)(N + c0), ov);
 #pragma unroll
-        for (int c = NC; c < N; ++c) p[c] = 0.f;
+            for (int c = 0; c < NCW; ++c) acc[c] = (acc[c] + ov[c]) * alpha[c];
+          } else {
+#pragma unroll
+            for (int c = 0; c < NCW; ++c) acc[c] *= alpha[c];
+          }
+          pv_acc = false;
+        }
+        float p[NCW];
+#pragma unroll
+        for (int c = 0; c < NCW; ++c) {
+          p[c] = valid ? exp2f(sv[c] - m_ref[c]) : 0.f;
+          l_tok[c] += p[c];
+        }
         // P^T rows: per 16-column atom, a 32-byte row per token (MN-major,
         // 32-byte swizzle: 16-byte piece c of row t sits at c ^ bit 2 of t),
-        // once for hi = round(p) and once for lo = round(p - hi).
+        // once for hi = round(p) and once for lo = round(p - hi).  O^T(j-1),
+        // the last reader of P, is complete.  This thread writes columns
+        // [c0, c0 + NCW): NCW * 2 bytes inside one 16-byte piece.
         {
-          const int sw = (tid >> 2) & 1;
+          const int atom = c0 / 16, piece = (c0 % 16) / 8, within = (c0 % 8) * 2;
+          unsigned char* prow = smem + L::kP + atom * L::kPAtom + t * 32 +
+                                ((piece ^ ((t >> 2) & 1)) * 16) + within;
+          constexpr int NW2 = (NCW + 1) / 2;  // 32-bit words (an odd single column takes half of one)
+          uint32_t hi[NW2], lo[NW2];
 #pragma unroll
-          for (int at = 0; at < N / 16; ++at) {
-            const float* pa = p + at * 16;
-            uint32_t w[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) w[i] = pack2(pa[2 * i], pa[2 * i + 1], kBf16);
-            float r[16];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float2 x = Elem<T>::to_f2(w[i]);
-              r[2 * i] = pa[2 * i] - x.x;
-              r[2 * i + 1] = pa[2 * i + 1] - x.y;
-            }
-            unsigned char* prow = smem + L::kP + at * L::kPAtom + tid * 32;
-            *reinterpret_cast<uint4*>(prow + 16 * sw) = make_uint4(w[0], w[1], w[2], w[3]);
-            *reinterpret_cast<uint4*>(prow + 16 * (sw ^ 1)) = make_uint4(w[4], w[5], w[6], w[7]);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) w[i] = pack2(r[2 * i], r[2 * i + 1], kBf16);
-            *reinterpret_cast<uint4*>(prow + L::kPBytes + 16 * sw) = make_uint4(w[0], w[1], w[2], w[3]);
-            *reinterpret_cast<uint4*>(prow + L::kPBytes + 16 * (sw ^ 1)) =
-                make_uint4(w[4], w[5], w[6], w[7]);
+          for (int i = 0; i < NW2; ++i) {
+            const float x0 = p[2 * i], x1 = (2 * i + 1 < NCW) ? p[2 * i + 1] : 0.f;
+            hi[i] = pack2(x0, x1, kBf16);
+            const float2 r = Elem<T>::to_f2(hi[i]);
+            lo[i] = pack2(x0 - r.x, x1 - r.y, kBf16);
+          }
+          if constexpr (NCW == 8) {
+            *reinterpret_cast<uint4*>(prow) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(prow + L::kPBytes) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          } else if constexpr (NCW == 4) {
+            *reinterpret_cast<uint2*>(prow) = make_uint2(hi[0], hi[1]);
+            *reinterpret_cast<uint2*>(prow + L::kPBytes) = make_uint2(lo[0], lo[1]);
+          } else if constexpr (NCW == 2) {
+            *reinterpret_cast<uint32_t*>(prow) = hi[0];
+            *reinterpret_cast<uint32_t*>(prow + L::kPBytes) = lo[0];
+          } else {
+            *reinterpret_cast<uint16_t*>(prow) = (uint16_t)hi[0];
+            *reinterpret_cast<uint16_t*>(prow + L::kPBytes) = (uint16_t)lo[0];
           }
         }
         if (!valid) {
-          // zero this token's V row (both 64-element halves) so 0 * stale never enters PV
-          unsigned char* vrow = smem + L::kStages + st * L::kStageBytes + 2 * L::kHalf + tid * 128;
+          // zero this token's V row (both 64-element halves, 16 pieces shared
+          // out over the column groups) so 0 * stale never enters PV
+          unsigned char* vrow = smem + L::kStages + st * L::kStageBytes + 2 * L::kHalf + t * 128;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(vrow + L::kHalf + c * 16) = make_uint4(0, 0, 0, 0);
-          }
+          for (int i = cg; i < 16; i += W::kNWG)
+            *reinterpret_cast<uint4*>(vrow + (i >> 3) * L::kHalf + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_before();
         named_barrier(1, kComputeThreads);
 
-        // ---- O^T = V^T . P^T
+        // ---- O^T (+)= V^T . P^T, then S^T(j+1) if it is not on its way yet
         if (tid == 0) {
           tc_fence_after();
 #pragma unroll
@@ -626,49 +710,52 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
             for (int kk = 0; kk < kTile / 16; ++kk)
               mma_f16(tmem + N, smem_desc(vt + kk * 2048, L::kHalf, 1024, kSw128),
                       smem_desc(sm_p + part_p * L::kPBytes + kk * 512, L::kPAtom, 256, kSw32),
-                      kIdescPV, part_p > 0 || kk > 0);
+                      kIdescPV, pv_acc || part_p > 0 || kk > 0);
           mma_commit(pv_bar);
           mma_commit(empty_bar(st));  // the stage is free once these MMAs are done
-          ++pv_commits;
-          ok = mbar_wait_or_abort(pv_bar, n_used & 1, a.err, abort_flag);
+          if (has_next && !next_issued) {
+            ok = mbar_wait_or_abort(full_bar(st_next), ((n_used + 1) / NST) & 1, a.err, abort_flag);
+            if (ok) issue_qk(st_next, q_addr);
+          }
         }
-        if (named_barrier_or(1, kComputeThreads, !ok || *abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        float ov[N];
-        tmem_ld<N>(tmem + t_lane + N, ov);
-#pragma unroll
-        for (int c = 0; c < NC; ++c) acc[c] = acc[c] * alpha[c] + ov[c];
-        tc_fence_before();
+        pv_acc = true;
       }
       if (!ok) break;
 
-      // ---- item result: reduce the per-token sums, write output or partial
-      {
-        float t[NC];
+      // ---- item result: fold the last O^T, reduce the per-token sums, write
+      if (tid == 0 && n_tiles > 0) ok = mbar_wait_or_abort(pv_bar, (n_used - 1) & 1, a.err, abort_flag);
+      if (named_barrier_or(1, kComputeThreads, !ok || *abort_flag)) { ok = false; break; }
+      if (n_tiles > 0) {
+        tc_fence_after();
+        float ov[NCW];
+        tmem_ld<NCW>(tmem + t_lane + (uint32_t)(N + c0), ov);
 #pragma unroll
-        for (int c = 0; c < NC; ++c) t[c] = l_tok[c];
-        const float wsum = column_reduce<NC, false>(t, lane);
-        named_barrier(1, kComputeThreads);  // `red` and `stat` of the last tile have been read
-        if (lane < NC) red[warp * N + lane] = wsum;
+        for (int c = 0; c < NCW; ++c) acc[c] += ov[c];
+        tc_fence_before();
+      }
+      {
+        float tmp[NCW];
+#pragma unroll
+        for (int c = 0; c < NCW; ++c) tmp[c] = l_tok[c];
+        const float wsum = column_reduce<NCW, false>(tmp, lane);
+        if (lane < NCW) red[quarter * N + c0 + lane] = wsum;
       }
       named_barrier(1, kComputeThreads);
-      if (warp == 0 && lane < NC)
-        stat[N + lane] = (red[lane] + red[N + lane]) + (red[2 * N + lane] + red[3 * N + lane]);
+      if (tid < NC) stat[N + tid] = (red[tid] + red[N + tid]) + (red[2 * N + tid] + red[3 * N + tid]);
       named_barrier(1, kComputeThreads);
-      const int d = tid;  // output element this thread writes, per column
-      const int cols = GROUP ? ctx_or_members * G : G;
+      const int d = t;  // output element this thread writes, per column
 #pragma unroll
-      for (int c = 0; c < NC; ++c) {
-        if (c >= cols) break;
-        const float M = stat[c], L_c = stat[N + c];
-        const int m = GROUP ? c / G : 0, h = GROUP ? c % G : c;
+      for (int c = 0; c < NCW; ++c) {
+        const int col = c0 + c;
+        if (col >= cols) break;
+        const float L_c = stat[N + col];
+        const int m = GROUP ? col / G : 0, h = GROUP ? col % G : col;
         const size_t qh = (size_t)(s + m) * a.num_q_heads + (size_t)kvh * G + h;
         bool zero = false, direct;
         if constexpr (GROUP) {
-          // shared partitions of the member, plus its private ones
-          const int4 pl = __ldg(a.plan + s + m);
+          // shared partitions of the member, plus its own ones
           const int ctx = max(0, min(__ldg(a.context_lens + s + m), a.max_context_len));
-          direct = pl.w + (ctx > pl.z ? (ctx - pl.z + PT - 1) / PT : 0) <= 1;
+          direct = seq_split(a.plan, s + m, ctx, a.own_tokens).total <= 1;
         } else {
           zero = ctx_or_members == 0;
           direct = n_parts <= 1;
@@ -681,20 +768,20 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           const size_t wslot = qh * a.num_parts + part;
           a.ws_acc[wslot * kD + d] = acc[c];
           if (d == 0) {
-            a.ws_ml[2 * wslot] = M;
+            a.ws_ml[2 * wslot] = m_ref[c];
             a.ws_ml[2 * wslot + 1] = L_c;
           }
         }
       }
-      named_barrier(1, kComputeThreads);  // `stat` and `red` are reused by the next item
+      named_barrier(1, kComputeThreads);  // `red` and `stat` are reused by the next item
       if (lane == 0) mbar_arrive(free_bar(slot));  // its query rows have been used
     }
     if (!ok && tid == 0) *abort_flag = 1;
-    // MMAs issued by thread 0 complete before TMEM is freed (bounded waits;
-    // phases complete in order, so the last commit's phase covers the rest).
+    // Every MMA thread 0 issued completes before TMEM is freed: one more
+    // commit tracks all of them (bounded wait).
     if (tid == 0) {
-      if (qk_commits > 0) mbar_wait(qk_bar, (qk_commits - 1) & 1, a.err);
-      if (pv_commits > 0) mbar_wait(pv_bar, (pv_commits - 1) & 1, a.err);
+      mma_commit(drain_bar);
+      mbar_wait(drain_bar, 0, a.err);
     }
   }
   tc_fence_before();
@@ -751,7 +838,8 @@ cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUte
     // number of items is only known on the device
     const int items0 = GROUP ? sms : a.num_seqs * a.num_kv_heads;
     const int grid = items0 < sms ? items0 : sms;
-    cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kThreads), L::kAlloc, stream, a, tk, tv, tq);
+    constexpr int kBlock = Warps<GROUP ? C::kN : G>::kThreads;
+    cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kBlock), L::kAlloc, stream, a, tk, tv, tq);
     if (e != cudaSuccess) return e;
     ++*launches;
   }

@@ -28,6 +28,8 @@ struct DecodeArgs {
   // members, shared tokens T, shared partitions}.  A sequence's own items
   // then cover [T, ctx), as partitions numbered from its shared partitions.
   const int4* plan;
+  int own_tokens;                // partition size of a sequence's own tokens (partition_tokens
+                                 // without a plan)
   int grid_parts;                // partitions per (sequence, kv head) of the CUDA-core grid
 };
 
@@ -48,12 +50,13 @@ struct PlanArgs {
 };
 cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream, int* launches);
 
-// Tokens [T, ctx) of sequence s with a plan: its first own partition, the
-// workspace slot of that partition, and the sequence's partition count.
+// Tokens [T, ctx) of sequence s with a plan: its first own token, the
+// workspace slot of its first own partition (of own_tokens tokens each), and
+// the sequence's partition count.
 struct SeqSplit {
   int base, slot0, total;
 };
-__host__ __device__ inline SeqSplit seq_split(const int4* plan, int s, int ctx, int partition_tokens) {
+__host__ __device__ inline SeqSplit seq_split(const int4* plan, int s, int ctx, int own_tokens) {
   int base = 0, slot0 = 0;
   if (plan) {
 #ifdef __CUDA_ARCH__
@@ -64,7 +67,7 @@ __host__ __device__ inline SeqSplit seq_split(const int4* plan, int s, int ctx, 
     base = pl.z;
     slot0 = pl.w;
   }
-  const int own = ctx > base ? (ctx - base + partition_tokens - 1) / partition_tokens : 0;
+  const int own = ctx > base ? (ctx - base + own_tokens - 1) / own_tokens : 0;
   return {base, slot0, slot0 + own};
 }
 

@@ -62,6 +62,15 @@ def _declare(lib):
     lib.oracle_cache_append.argtypes = [c.c_longlong, c.c_longlong, c.c_int, P, P, P, P, P]
     lib.oracle_copy_blocks.restype = c.c_int
     lib.oracle_copy_blocks.argtypes = [c.c_int, c.c_longlong, c.c_int, P, P, P]
+    lib.oracle_e4m3_to_f64.restype = c.c_double
+    lib.oracle_e4m3_to_f64.argtypes = [c.c_uint8]
+    lib.oracle_e4m3_from_f32.restype = c.c_uint8
+    lib.oracle_e4m3_from_f32.argtypes = [c.c_float]
+    lib.oracle_decode_fp8.restype = c.c_int
+    lib.oracle_decode_fp8.argtypes = [c.c_int] * 8 + [P, P, P, P, P, P, P, c.c_double, P, c.c_int]
+    lib.oracle_cache_append_fp8.restype = c.c_int
+    lib.oracle_cache_append_fp8.argtypes = [c.c_int, c.c_longlong, c.c_int, c.c_int, c.c_int,
+                                            P, P, P, P, P, P, P]
     return lib
 
 
@@ -166,3 +175,53 @@ class Oracle:
                                          _ptr(v_cache))
         if rc:
             raise OracleError(f"oracle_copy_blocks refused its input (rc={rc})")
+
+    # ---- FP8 (E4M3) cache
+
+    def e4m3_to_f64(self, code: int) -> float:
+        return self.lib.oracle_e4m3_to_f64(int(code))
+
+    def e4m3_from_f32(self, y: float) -> int:
+        return int(self.lib.oracle_e4m3_from_f32(float(np.float32(y))))
+
+    def decode_fp8(self, dtype, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                   scale, num_threads: int = 0) -> np.ndarray:
+        """fp64 [S][Hq][D] attention output over an E4M3 cache (uint8 codes,
+        [NB][bs][Hkv][D]) with fp32 per-kv-head scales."""
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        kc = np.ascontiguousarray(k_cache, dtype=np.uint8)
+        vc = np.ascontiguousarray(v_cache, dtype=np.uint8)
+        ks = np.ascontiguousarray(k_scale, dtype=np.float32)
+        vs = np.ascontiguousarray(v_scale, dtype=np.float32)
+        bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+        cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+        S, Hq, D = q.shape
+        NB, bs, Hkv, D2 = kc.shape
+        assert D2 == D and vc.shape == kc.shape and ks.shape == (Hkv,) and vs.shape == (Hkv,)
+        out = np.empty((S, Hq, D), dtype=np.float64)
+        rc = self.lib.oracle_decode_fp8(int(dtype), S, Hq, Hkv, D, bs, NB, bt.shape[1], _ptr(q),
+                                        _ptr(kc), _ptr(vc), _ptr(ks), _ptr(vs), _ptr(bt), _ptr(cl),
+                                        float(scale), _ptr(out), int(num_threads))
+        if rc:
+            raise OracleError(f"oracle_decode_fp8 refused its input (rc={rc})")
+        return out
+
+    def cache_append_fp8(self, dtype, k, v, slot_mapping, k_scale, v_scale, k_cache,
+                         v_cache) -> None:
+        """In place on the uint8 code pools ``k_cache``/``v_cache`` ([NB][bs][Hkv][D]);
+        ``k``/``v`` are [T][Hkv][D] fp16/bf16 bits."""
+        assert k_cache.flags["C_CONTIGUOUS"] and v_cache.flags["C_CONTIGUOUS"]
+        assert k_cache.dtype == np.uint8 and v_cache.dtype == np.uint8
+        k = np.ascontiguousarray(k, dtype=np.uint16)
+        v = np.ascontiguousarray(v, dtype=np.uint16)
+        sm = np.ascontiguousarray(slot_mapping, dtype=np.int32)
+        ks = np.ascontiguousarray(k_scale, dtype=np.float32)
+        vs = np.ascontiguousarray(v_scale, dtype=np.float32)
+        NB, bs, Hkv, D = k_cache.shape
+        T = sm.shape[0]
+        assert k.shape == (T, Hkv, D) and v.shape == (T, Hkv, D)
+        rc = self.lib.oracle_cache_append_fp8(int(dtype), NB * bs, Hkv, D, T, _ptr(k), _ptr(v),
+                                              _ptr(sm), _ptr(ks), _ptr(vs), _ptr(k_cache),
+                                              _ptr(v_cache))
+        if rc:
+            raise OracleError(f"oracle_cache_append_fp8 refused its input (rc={rc})")

@@ -39,6 +39,19 @@
  *  - Copy-on-write: for each (src, dst) pair the whole block of K and of V is
  *    copied (zingnex.cn section 3.2 item 3).
  *
+ *  - FP8 cache (the pages name FP8 only as a quantisation format that saves
+ *    memory: zingnex.cn sections 4.1 and 6, 5688vip.com section 2.3; the
+ *    encoding below is the plain reading): K and V stored as OCP 8-bit E4M3
+ *    codes with one fp32 scale per kv head and tensor.  E4M3 is 1 sign bit,
+ *    4 exponent bits (bias 7) and 3 mantissa bits; exponent field 0 is
+ *    subnormal (mantissa * 2^-9); S.1111.111 is NaN; there is no infinity;
+ *    the largest finite value is 1.75 * 2^8 = 448.  A stored value is code * scale.  Append divides the
+ *    input (widened exactly to fp32) by the scale in fp32 and rounds the
+ *    quotient to the nearest code, ties to the even code, with magnitudes of
+ *    448 and above (infinity included) saturated to 448.  Decode widens each
+ *    code exactly and multiplies by the scale in fp64, then proceeds as
+ *    above.
+ *
  * Every function returns 0 on success and a negative value on an input it
  * refuses (bad shape, a table entry or slot outside the pool); on refusal the
  * outputs are unspecified.  Loops only: no BLAS, no SIMD intrinsics, no
@@ -80,6 +93,46 @@ double oracle_bf16_to_f64(uint16_t b)
     float f;
     memcpy(&f, &u, sizeof f);
     return (double)f;
+}
+
+/* OCP E4M3 code -> double, exact. */
+double oracle_e4m3_to_f64(uint8_t c)
+{
+    int sign = (c >> 7) & 1;
+    int e = (c >> 3) & 0xf;
+    int m = c & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);
+    else
+        v = ldexp((double)(8 + m), e - 10);
+    return sign ? -v : v;
+}
+
+/* fp32 -> nearest E4M3 code, ties to the even code, saturating at 448;
+ * NaN -> 0x7F. */
+uint8_t oracle_e4m3_from_f32(float y)
+{
+    if (isnan(y)) return 0x7f;
+    uint8_t sign = signbit(y) ? 0x80 : 0x00;
+    double a = fabs((double)y);
+    if (a >= 448.0) return sign | 0x7e;
+    if (a < ldexp(1.0, -6)) {
+        /* subnormal step 2^-9; a count of 8 is the smallest normal, code 0x08 */
+        double n = rint(ldexp(a, 9));
+        return sign | (uint8_t)n;
+    }
+    int e;
+    frexp(a, &e);            /* a = f * 2^e with f in [0.5, 1) */
+    e -= 1;                  /* a in [2^e, 2^(e+1)) */
+    double n = rint(ldexp(a, 3 - e));  /* in [8, 16] */
+    if (n == 16.0) {
+        n = 8.0;
+        e += 1;
+    }
+    return sign | (uint8_t)(((e + 7) << 3) | ((int)n - 8));
 }
 
 static double widen(int dtype, uint16_t x)
@@ -274,6 +327,102 @@ int oracle_copy_blocks(int num_blocks, long long block_bytes, int num_pairs, con
                 (size_t)block_bytes);
         memmove(v_cache + (long long)dst * block_bytes, v_cache + (long long)src * block_bytes,
                 (size_t)block_bytes);
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------
+ * FP8 (E4M3) cache.  k_cache, v_cache: uint8 codes [NB][bs][Hkv][D];
+ * k_scale, v_scale: fp32 [Hkv].  Same definition as oracle_decode with
+ * K_j[d] = e4m3(k code) * k_scale[kv head] (and V likewise), in fp64. */
+static int attend_range_fp8(int dtype, int Hkv, int D, int bs, int NB, int MBS,
+                            const uint16_t *qrow, const uint8_t *kc, const uint8_t *vc,
+                            double ks, double vs, const int32_t *tables, int s, int kvh,
+                            int L, double scale, double *x, double *acc, double *l_out)
+{
+    double m = -INFINITY;
+    for (int j = 0; j < L; ++j) {
+        long long r = token_row(tables, MBS, s, j, bs, NB, Hkv, D, kvh);
+        if (r < 0) return -2;
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d)
+            dot += widen(dtype, qrow[d]) * (oracle_e4m3_to_f64(kc[r + d]) * ks);
+        x[j] = dot * scale;
+        m = x[j] > m ? x[j] : m;
+    }
+    double l = 0.0;
+    for (int d = 0; d < D; ++d) acc[d] = 0.0;
+    for (int j = 0; j < L; ++j) {
+        double w = exp(x[j] - m);
+        l += w;
+        long long r = token_row(tables, MBS, s, j, bs, NB, Hkv, D, kvh);
+        for (int d = 0; d < D; ++d)
+            acc[d] += w * (oracle_e4m3_to_f64(vc[r + d]) * vs);
+    }
+    *l_out = l;
+    return 0;
+}
+
+/* out: double [S][Hq][D]; dtype is that of q (fp16 or bf16). */
+int oracle_decode_fp8(int dtype, int S, int Hq, int Hkv, int D, int bs, int NB, int MBS,
+                      const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                      const float *k_scale, const float *v_scale, const int32_t *block_tables,
+                      const int32_t *context_lens, double scale, double *out, int num_threads)
+{
+    if (!shape_ok(dtype, S, Hq, Hkv, D, bs, NB, MBS)) return -1;
+    for (int s = 0; s < S; ++s)
+        if (context_lens[s] < 0 || (long long)context_lens[s] > (long long)MBS * bs) return -1;
+    int g = Hq / Hkv;
+    int err = 0;
+    int nt = resolve_threads(num_threads);
+    long long total = (long long)S * Hq;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nt) reduction(| : err)
+    for (long long sh = 0; sh < total; ++sh) {
+        int s = (int)(sh / Hq), h = (int)(sh % Hq);
+        int L = context_lens[s];
+        double *o = out + sh * D;
+        if (L == 0) {
+            for (int d = 0; d < D; ++d) o[d] = 0.0;
+            continue;
+        }
+        double *x = (double *)malloc(sizeof(double) * (size_t)L);
+        double *acc = (double *)malloc(sizeof(double) * (size_t)D);
+        double lsum;
+        int kvh = h / g;
+        int rc = attend_range_fp8(dtype, Hkv, D, bs, NB, MBS, q + sh * D, k_cache, v_cache,
+                                  (double)k_scale[kvh], (double)v_scale[kvh], block_tables, s,
+                                  kvh, L, scale, x, acc, &lsum);
+        if (rc) err |= 1;
+        else
+            for (int d = 0; d < D; ++d) o[d] = acc[d] / lsum;
+        free(x);
+        free(acc);
+    }
+    return err ? -2 : 0;
+}
+
+/* Append into an FP8 cache: k, v are [num_tokens][Hkv][D] in dtype (fp16 or
+ * bf16); the codes of token t go to slot slot_mapping[t] (negative: skipped). */
+int oracle_cache_append_fp8(int dtype, long long num_slots, int Hkv, int D, int num_tokens,
+                            const uint16_t *k, const uint16_t *v, const int32_t *slot_mapping,
+                            const float *k_scale, const float *v_scale, uint8_t *k_cache,
+                            uint8_t *v_cache)
+{
+    if ((dtype != ORACLE_F16 && dtype != ORACLE_BF16) || num_slots < 0 || Hkv <= 0 || D <= 0 ||
+        num_tokens < 0)
+        return -1;
+    long long row = (long long)Hkv * D;
+    for (int t = 0; t < num_tokens; ++t) {
+        long long slot = slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot >= num_slots) return -2;
+        for (long long i = 0; i < row; ++i) {
+            int h = (int)(i / D);
+            float xk = (float)widen(dtype, k[(long long)t * row + i]);
+            float xv = (float)widen(dtype, v[(long long)t * row + i]);
+            k_cache[slot * row + i] = oracle_e4m3_from_f32(xk / k_scale[h]);
+            v_cache[slot * row + i] = oracle_e4m3_from_f32(xv / v_scale[h]);
+        }
     }
     return 0;
 }

@@ -18,7 +18,13 @@ the oracle disagrees with what the pages or the mathematics fix:
   private copies;
 * grouped queries equal full multi-head attention with repeated kv heads;
 * the partitioned (split-K) form equals the direct one;
-* append and copy-on-write equal a NumPy scatter/copy over the whole pool.
+* append and copy-on-write equal a NumPy scatter/copy over the whole pool;
+* the E4M3 cache: every code widens as PyTorch's float8_e4m3fn does, the
+  encoder rounds as PyTorch's fp32 conversion below the saturation point,
+  codes round-trip, ties go to the even code, large values saturate at 448;
+  over codes that fp16 holds exactly the FP8 decode equals the fp16 decode;
+  the scales act as factors of the logits and of the output, per kv head;
+  append encodes each element of x / scale as PyTorch does.
 
 The pins are plain functions so that tests/test_oracle_mutations.py can run
 them against oracle builds with planted mistakes.
@@ -405,6 +411,147 @@ def pin_copy_matches_block_copy(orc):
         ev[d] = ev[s]
     orc.copy_blocks(pairs, kc, vc)
     assert np.array_equal(kc, ek) and np.array_equal(vc, ev), "copy differs from a block copy"
+
+
+
+
+# ---------------------------------------------------------------- FP8 (E4M3) cache
+
+def pin_e4m3_codes_match_torch(orc):
+    """Every code widens as PyTorch's float8_e4m3fn (the OCP E4M3 format) does."""
+    import torch
+
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).double().numpy()
+    got = np.array([orc.e4m3_to_f64(c) for c in range(256)])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan) and nan.sum() == 2, "E4M3 NaN codes differ"
+    assert np.array_equal(got[~nan], ref[~nan]), "E4M3 widening differs from PyTorch"
+    assert np.signbit(got[0x80]) and got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9
+
+
+def pin_e4m3_rounding_matches_torch(orc):
+    """Below the saturation point, the encoder rounds as PyTorch's fp32 -> e4m3fn."""
+    import torch
+
+    rng = np.random.default_rng(31)
+    ys = np.concatenate([rng.uniform(-447.9, 447.9, 4000), rng.uniform(-0.02, 0.02, 4000),
+                         rng.standard_normal(4000) * 3]).astype(np.float32)
+    # exact midpoints between neighbouring codes, where ties decide
+    vals = np.array([orc.e4m3_to_f64(c) for c in range(0x7F)])
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    ys = np.concatenate([ys, mids, -mids])
+    ref = torch.from_numpy(ys).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([orc.e4m3_from_f32(float(y)) for y in ys], dtype=np.uint8)
+    assert np.array_equal(got, ref), f"{int((got != ref).sum())} roundings differ from PyTorch"
+
+
+def pin_e4m3_roundtrip_and_ties_to_even(orc):
+    vals = [orc.e4m3_to_f64(c) for c in range(256)]
+    for c in range(256):
+        if not math.isnan(vals[c]):
+            assert orc.e4m3_from_f32(vals[c]) == c, f"code {c:#x} does not round-trip"
+    for c in range(0x7E):
+        mid = (vals[c] + vals[c + 1]) / 2
+        even = c if c % 2 == 0 else c + 1
+        assert orc.e4m3_from_f32(mid) == even, f"tie between {c:#x} and {c + 1:#x}"
+        assert orc.e4m3_from_f32(np.nextafter(np.float32(mid), np.float32(1e9))) == c + 1
+        assert orc.e4m3_from_f32(np.nextafter(np.float32(mid), np.float32(-1e9))) == c
+
+
+def pin_e4m3_saturates(orc):
+    for y, code in [(448.0, 0x7E), (449.0, 0x7E), (464.0, 0x7E), (470.0, 0x7E), (479.0, 0x7E),
+                    (1e30, 0x7E),
+                    (float("inf"), 0x7E), (-1e30, 0xFE), (-449.0, 0xFE)]:
+        assert orc.e4m3_from_f32(y) == code, f"{y} should saturate to {code:#x}"
+
+
+def _exact_e4m3_case(orc, seed, dtype=gen.F16):
+    """A small paged case whose K/V values are E4M3 codes that fp16 holds exactly."""
+    rng = np.random.default_rng(seed)
+    c = _case(seed, num_seqs=3, num_q_heads=4, num_kv_heads=2, head_dim=32, block_size=16,
+              dtype=dtype, context_lens=[1, 20, 45], poison=False)
+    shape = c["k_cache"].shape
+    kcode = rng.integers(0, 256, size=shape).astype(np.uint8)
+    vcode = rng.integers(0, 256, size=shape).astype(np.uint8)
+    for a in (kcode, vcode):
+        a[(a & 0x7F) == 0x7F] = 0x38   # no NaN codes
+        a[(a & 0x78) >= 0x60] &= 0xC7  # keep |value| small enough for tame logits
+    f = np.vectorize(orc.e4m3_to_f64)
+    kf, vf = f(kcode).astype(np.float16), f(vcode).astype(np.float16)
+    assert np.array_equal(kf.astype(np.float64), f(kcode)), "values not exact in fp16"
+    return c, kcode, vcode, kf.view(np.uint16), vf.view(np.uint16)
+
+
+def pin_fp8_decode_equals_16bit_decode(orc):
+    c, kcode, vcode, kbits, vbits = _exact_e4m3_case(orc, 41)
+    ones = np.ones(2, dtype=np.float32)
+    got = orc.decode_fp8(gen.F16, c["q"], kcode, vcode, ones, ones, c["block_tables"],
+                         c["context_lens"], c["scale"])
+    ref = orc.decode(gen.F16, c["q"], kbits, vbits, c["block_tables"], c["context_lens"], c["scale"])
+    assert np.max(np.abs(got - ref)) <= 1e-13, "FP8 decode differs from the fp16 decode of the same values"
+
+
+def pin_fp8_scales(orc):
+    c, kcode, vcode, _, _ = _exact_e4m3_case(orc, 42)
+    ks = np.array([0.5, 2.0], dtype=np.float32)
+    vs = np.array([0.25, 4.0], dtype=np.float32)
+    a = orc.decode_fp8(gen.F16, c["q"], kcode, vcode, ks, vs, c["block_tables"], c["context_lens"],
+                       c["scale"])
+    b = orc.decode_fp8(gen.F16, c["q"], kcode, vcode, ks, 2 * vs, c["block_tables"],
+                       c["context_lens"], c["scale"])
+    assert np.array_equal(b, 2 * a), "the V scale must scale the output"
+    d = orc.decode_fp8(gen.F16, c["q"], kcode, vcode, 2 * ks, vs, c["block_tables"],
+                       c["context_lens"], c["scale"] / 2)
+    assert np.array_equal(d, a), "the K scale must act as a factor of the logits"
+    # kv head 1's scales must reach exactly the query heads of group 1
+    e = orc.decode_fp8(gen.F16, c["q"], kcode, vcode, ks, np.array([0.25, 8.0], np.float32),
+                       c["block_tables"], c["context_lens"], c["scale"])
+    assert np.array_equal(e[:, :2], a[:, :2]) and np.array_equal(e[:, 2:], 2 * a[:, 2:])
+
+
+def pin_fp8_large_logits_stay_finite(orc):
+    """Logits near 1000 (exp overflows fp64 without the max subtracted)."""
+    S, H, D, bs = 1, 1, 32, 16
+    q = np.full((S, H, D), gen.to_bits(np.float32(1.0), gen.F16), dtype=np.uint16)
+    kc = np.full((1, bs, H, D), 0x7D, dtype=np.uint8)   # 416
+    kc[0, 3] = 0x7E                                        # 448: the dominant key
+    vc = np.zeros((1, bs, H, D), dtype=np.uint8)
+    vc[0, 3] = 0x38                                        # 1.0
+    one = np.ones(H, dtype=np.float32)
+    scale = 1000.0 / (D * 448.0)
+    out = orc.decode_fp8(gen.F16, q, kc, vc, one, one, np.zeros((S, 1), np.int32),
+                         np.array([bs], np.int32), scale)
+    assert np.all(np.isfinite(out)), "large logits must not overflow"
+    # the dominant key's weight is 1 / (1 + 15 e^(-1000 (448 - 416) / 448))
+    w = 1.0 / (1.0 + 15.0 * math.exp(-1000.0 * 32.0 / 448.0))
+    assert abs(out[0, 0, 0] - w) < 1e-12
+
+
+def pin_fp8_append_encodes_each_element(orc):
+    import torch
+
+    rng = np.random.default_rng(43)
+    NB, bs, Hkv, D, T = 6, 16, 2, 32, 9
+    for dtype in (gen.F16, gen.BF16):
+        kc = rng.integers(0, 256, size=(NB, bs, Hkv, D), dtype=np.uint8)
+        vc = kc.copy()
+        ek, ev = kc.copy(), vc.copy()
+        slots = rng.choice(NB * bs, size=T, replace=False).astype(np.int32)
+        slots[4] = -1
+        k = gen.normal_bits(rng, (T, Hkv, D), dtype)
+        v = gen.normal_bits(rng, (T, Hkv, D), dtype)
+        ks = np.array([0.012, 0.02], dtype=np.float32)
+        vs = np.array([0.03, 0.015], dtype=np.float32)
+        orc.cache_append_fp8(dtype, k, v, slots, ks, vs, kc, vc)
+        for src, scales, exp in ((k, ks, ek), (v, vs, ev)):
+            y = gen.bits_to_f32(src, dtype) / scales[None, :, None]   # fp32 division
+            assert np.abs(y).max() < 448
+            codes = torch.from_numpy(np.ascontiguousarray(y)).to(torch.float8_e4m3fn)
+            codes = codes.view(torch.uint8).numpy()
+            keep = slots >= 0
+            exp.reshape(NB * bs, Hkv, D)[slots[keep]] = codes[keep]
+        assert np.array_equal(kc, ek) and np.array_equal(vc, ev), "FP8 append differs"
 
 
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

@@ -49,6 +49,19 @@ MUTANTS = {
     "copy_direction_swapped": (
         "memmove(k_cache + (long long)dst * block_bytes, k_cache + (long long)src * block_bytes,",
         "memmove(k_cache + (long long)src * block_bytes, k_cache + (long long)dst * block_bytes,"),
+    "e4m3_exponent_bias": ("v = ldexp((double)(8 + m), e - 10);", "v = ldexp((double)(8 + m), e - 11);"),
+    "e4m3_subnormal_step": ("v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
+    "e4m3_no_saturation": ("if (a >= 448.0) return sign | 0x7e;", "if (a >= 480.0) return sign | 0x7e;"),
+    "e4m3_ties_away": ("double n = rint(ldexp(a, 3 - e));", "double n = floor(ldexp(a, 3 - e) + 0.5);"),
+    "fp8_v_scale_dropped": ("acc[d] += w * (oracle_e4m3_to_f64(vc[r + d]) * vs);",
+                            "acc[d] += w * oracle_e4m3_to_f64(vc[r + d]);"),
+    "fp8_max_not_subtracted": ("double w = exp(x[j] - m);", "double w = exp(x[j]);"),
+    "fp8_normalisation_dropped": ("o[d] = acc[d] / lsum;", "o[d] = acc[d];"),
+    "fp8_k_scale_from_v": ("(double)k_scale[kvh], (double)v_scale[kvh], block_tables, s,",
+                           "(double)v_scale[kvh], (double)v_scale[kvh], block_tables, s,"),
+    "fp8_append_multiplies": ("oracle_e4m3_from_f32(xk / k_scale[h]);",
+                              "oracle_e4m3_from_f32(xk * k_scale[h]);"),
+    "fp8_append_head_index": ("int h = (int)(i / D);", "int h = (int)(i % Hkv);"),
     "v_copy_skipped": (
         "memmove(v_cache + (long long)dst * block_bytes, v_cache + (long long)src * block_bytes,\n"
         "                (size_t)block_bytes);",

@@ -56,6 +56,9 @@ def parse_args(argv=None):
     p.add_argument("--partition-tokens", type=int, default=0)
     p.add_argument("--variant", default="auto", choices=sorted(VARIANTS),
                    help="decode kernel: auto, cuda_cores or tensor_cores")
+    p.add_argument("--kv-cache", default="dtype", choices=["dtype", "fp8"],
+                   help="K/V cache elements: the workload's 16-bit dtype, or E4M3 codes with "
+                        "per-kv-head scales (halves the K/V bytes)")
     p.add_argument("--shared-prefix", default="auto", choices=["auto", "on", "off"],
                    help="read blocks shared by consecutive sequences once per group; auto: on "
                         "when the workload's tables share their first block")
@@ -114,11 +117,13 @@ def sum_over_ranks(x: float, dist, device=None) -> float:
 # byte and flop accounting (per decode)
 
 
-def decode_bytes(ctx: np.ndarray, num_q_heads, num_kv_heads, head_dim, block_size, elem=2) -> int:
-    """Algorithmic bytes of one decode: K+V rows, q+out, table entries, lengths."""
+def decode_bytes(ctx: np.ndarray, num_q_heads, num_kv_heads, head_dim, block_size, elem=2,
+                 kv_elem=None) -> int:
+    """Algorithmic bytes of one decode: K+V rows (kv_elem bytes per element,
+    default elem), q+out, table entries, lengths."""
     ctx = np.asarray(ctx, dtype=np.int64)
     S = ctx.shape[0]
-    kv = int(2 * ctx.sum() * num_kv_heads * head_dim * elem)
+    kv = int(2 * ctx.sum() * num_kv_heads * head_dim * (elem if kv_elem is None else kv_elem))
     qo = 2 * S * num_q_heads * head_dim * elem
     tables = int(4 * np.ceil(ctx / block_size).sum())
     return kv + qo + tables + 4 * S
@@ -242,7 +247,7 @@ class DeviceWorkload:
     """The pool and a cycle of precomputed steps, resident on the device."""
 
     def __init__(self, case, torch, pa, partition_tokens: int, variant: int = 0,
-                 shared_prefix: int = 0):
+                 shared_prefix: int = 0, fp8: bool = False):
         self.case = case
         self.torch, self.pa = torch, pa
         dt = pa.torch_dtype(case.dtype)
@@ -255,6 +260,7 @@ class DeviceWorkload:
             return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
 
         self.k_cache, self.v_cache = dev16(case.k_cache), dev16(case.v_cache)
+        self.fp8 = fp8
         self.steps = []
         for st in case.steps:
             self.steps.append(dict(
@@ -267,7 +273,23 @@ class DeviceWorkload:
             num_seqs=case.num_seqs, num_q_heads=case.num_q_heads, num_kv_heads=case.num_kv_heads,
             head_dim=case.head_dim, block_size=case.block_size, num_blocks=case.num_blocks,
             max_blocks_per_seq=case.max_blocks_per_seq, partition_tokens=partition_tokens,
-            dtype=case.dtype, variant=variant, shared_prefix=shared_prefix)
+            dtype=case.dtype, variant=variant, shared_prefix=shared_prefix,
+            cache_format=pa.PA_CACHE_FP8_E4M3 if fp8 else pa.PA_CACHE_AS_DTYPE)
+        if fp8:
+            # E4M3 pools encoded from the 16-bit ones by the library's own
+            # append over every slot, with per-kv-head scales amax / 448
+            NB, bs, Hkv, D = case.k_cache.shape
+            k16, v16 = self.k_cache, self.v_cache
+            amax = lambda t: t.float().abs().reshape(-1, Hkv, D).amax(dim=(0, 2))  # noqa: E731
+            self.k_scale = (amax(k16) / 448.0).clamp_min(1e-12).contiguous()
+            self.v_scale = (amax(v16) / 448.0).clamp_min(1e-12).contiguous()
+            self.k_cache = torch.empty((NB, bs, Hkv, D), dtype=torch.uint8, device="cuda")
+            self.v_cache = torch.empty_like(self.k_cache)
+            slots = torch.arange(NB * bs, dtype=torch.int32, device="cuda")
+            pa.pa_cache_append_fp8(k16, v16, slots, NB * bs, self.k_cache, self.v_cache,
+                                   self.k_scale, self.v_scale, self.shape)
+            torch.cuda.synchronize()
+            del k16, v16
         self.ws_bytes = pa.pa_decode_workspace_bytes(self.shape, self.max_len)
         self.ws = torch.empty(max(16, self.ws_bytes), dtype=torch.uint8, device="cuda")
         self.out = torch.empty((case.num_seqs, case.num_q_heads, case.head_dim), dtype=dt,
@@ -284,13 +306,23 @@ class DeviceWorkload:
         if st["n_pairs"]:
             pa.pa_copy_blocks(st["pairs"], st["n_pairs"], self.k_cache, self.v_cache, self.shape,
                               stream.cuda_stream)
-        pa.pa_cache_append(st["k_new"], st["v_new"], st["slots"], self.case.num_seqs,
-                           self.k_cache, self.v_cache, self.shape, stream.cuda_stream)
+        if self.fp8:
+            pa.pa_cache_append_fp8(st["k_new"], st["v_new"], st["slots"], self.case.num_seqs,
+                                   self.k_cache, self.v_cache, self.k_scale, self.v_scale,
+                                   self.shape, stream.cuda_stream)
+        else:
+            pa.pa_cache_append(st["k_new"], st["v_new"], st["slots"], self.case.num_seqs,
+                               self.k_cache, self.v_cache, self.shape, stream.cuda_stream)
         if ev:
             ev[1].record(stream)
-        pa.pa_decode(st["q"], self.k_cache, self.v_cache, st["tables"], st["lens"],
-                     self.case.scale, self.out, self.shape, st["max_len"], self.ws, self.ws_bytes,
-                     stream.cuda_stream)
+        if self.fp8:
+            pa.pa_decode_fp8(st["q"], self.k_cache, self.v_cache, self.k_scale, self.v_scale,
+                             st["tables"], st["lens"], self.case.scale, self.out, self.shape,
+                             st["max_len"], self.ws, self.ws_bytes, stream.cuda_stream)
+        else:
+            pa.pa_decode(st["q"], self.k_cache, self.v_cache, st["tables"], st["lens"],
+                         self.case.scale, self.out, self.shape, st["max_len"], self.ws,
+                         self.ws_bytes, stream.cuda_stream)
         if ev:
             ev[2].record(stream)
 
@@ -307,13 +339,15 @@ def run_ours(args, rank, world, local, dist):
                          seed=gen.SEED_BASE + gen.WORKLOADS[args.workload].number + 1000 * rank)
     shared = {"on": 1, "off": 0}.get(args.shared_prefix)
     if shared is None:
-        shared = int(args.variant == "auto" and
+        shared = int(args.variant == "auto" and args.kv_cache != "fp8" and
                      tables_share_blocks(case.steps[0].block_tables, case.steps[0].context_lens))
-    w = DeviceWorkload(case, torch, pa, args.partition_tokens, VARIANTS[args.variant], shared)
+    fp8 = args.kv_cache == "fp8"
+    w = DeviceWorkload(case, torch, pa, args.partition_tokens, VARIANTS[args.variant], shared, fp8)
+    kv_elem = 1 if fp8 else 2
     bytes_per = [decode_bytes(s.context_lens, case.num_q_heads, case.num_kv_heads, case.head_dim,
-                              case.block_size) for s in case.steps]
-    pool_bytes = 2 * case.k_cache.nbytes
-    kv_step0 = 2 * int(case.steps[0].context_lens.sum()) * case.num_kv_heads * case.head_dim * 2
+                              case.block_size, kv_elem=kv_elem) for s in case.steps]
+    pool_bytes = 2 * case.k_cache.nbytes * kv_elem // 2
+    kv_step0 = 2 * int(case.steps[0].context_lens.sum()) * case.num_kv_heads * case.head_dim * kv_elem
 
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
@@ -353,7 +387,7 @@ def run_ours(args, rank, world, local, dist):
     achieved = step_bytes / (dec_total_ms * 1e-3) / 1e9
     resolved = {1: "cuda_cores", 2: "tensor_cores",
                 3: "shared_prefix"}[pa.pa_decode_resolved_variant(w.shape)]
-    traffic = profiled_traffic(args.workload, resolved, step_bytes / args.steps)
+    traffic = (None if fp8 else profiled_traffic(args.workload, resolved, step_bytes / args.steps))
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -368,6 +402,7 @@ def run_ours(args, rank, world, local, dist):
             "partition_tokens": args.partition_tokens or 512,
             "decode_variant": f"{args.variant} -> {resolved}",
             "shared_prefix": bool(shared),
+            "kv_cache": "e4m3 codes + per-kv-head fp32 scales" if fp8 else gen.DTYPE_NAMES[case.dtype],
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "steps_cycle": n_cycle,
             "l2": (f"inputs larger than L2: {kv_step0 / 1e6:.0f} MB of K/V read per decode, "

@@ -95,7 +95,22 @@ typedef struct {
   int32_t variant; /* pa_decode_variant (pa_decode only; 0 = automatic) */
   int32_t shared_prefix; /* pa_decode only: 1 = read blocks shared by consecutive
                             sequences once per group (see pa_decode); 0 = off */
+  int32_t cache_format;  /* pa_cache_format: what k_cache / v_cache hold */
 } pa_shape;
+
+/* Element format of k_cache / v_cache.
+ *  PA_CACHE_AS_DTYPE   2-byte elements of shape->dtype (pa_decode,
+ *                      pa_cache_append).
+ *  PA_CACHE_FP8_E4M3   1-byte OCP E4M3 codes (1 sign, 4 exponent bits with
+ *                      bias 7, 3 mantissa bits, no infinity, S.1111.111 =
+ *                      NaN, largest finite 448) with one fp32 scale per kv
+ *                      head for K and one for V: stored value = code * scale.
+ *                      Read by pa_decode_fp8, written by pa_cache_append_fp8;
+ *                      q and out stay in shape->dtype.  The pages name FP8
+ *                      only as a quantisation format that saves memory
+ *                      (zingnex.cn sections 4.1 and 6; 5688vip.com section
+ *                      2.3); this encoding is the library's reading. */
+typedef enum { PA_CACHE_AS_DTYPE = 0, PA_CACHE_FP8_E4M3 = 1 } pa_cache_format;
 
 /* How pa_decode computes QK^T and PV.  Both variants read K/V with tiled TMA
  * loads through the block table and keep the softmax in fp32.
@@ -173,6 +188,8 @@ size_t pa_decode_workspace_bytes(const pa_shape *shape, int32_t max_context_len)
  * workspace: device, at least pa_decode_workspace_bytes(shape, max_context_len)
  *   bytes, 16-byte aligned, never NULL.  It must not be shared with a decode
  *   that runs concurrently.
+ * An E4M3 cache (cache_format PA_CACHE_FP8_E4M3) needs pa_decode_fp8 and its
+ * scales: pa_decode refuses it with PA_ERR_INVALID_ARG.
  */
 pa_status pa_decode(const void *q, const void *k_cache, const void *v_cache,
                     const int32_t *block_tables, const int32_t *context_lens, float scale,
@@ -216,7 +233,8 @@ pa_status pa_decode_noalloc(const void *q, const void *k_cache, const void *v_ca
                             pa_stream_t stream);
 
 /*
- * Append one new token per entry into the cache (the "update KV cache" step of
+ * Append one new token per entry into a 16-bit cache (cache_format
+ * PA_CACHE_AS_DTYPE, else PA_ERR_INVALID_ARG; the "update KV cache" step of
  * each decode iteration, 5688vip.com section 2.1): for t < num_tokens with
  * slot = slot_mapping[t] >= 0,
  *   k_cache viewed as [num_blocks * block_size][num_kv_heads][head_dim] gets
@@ -231,9 +249,40 @@ pa_status pa_cache_append(const void *k, const void *v, const int32_t *slot_mapp
                           const pa_shape *shape, pa_stream_t stream);
 
 /*
+ * Append into an E4M3 cache (shape->cache_format == PA_CACHE_FP8_E4M3, else
+ * PA_ERR_INVALID_ARG): as pa_cache_append, but each element x of k[t] (fp16
+ * or bf16, shape->dtype, widened exactly to fp32) of kv head h is stored as
+ * the E4M3 code nearest to x / k_scale[h], the division in fp32 rounded to
+ * nearest, ties to the even code, magnitudes of 448 and above saturated to
+ * 448 (and v likewise with v_scale).  k_scale, v_scale: device fp32
+ * [num_kv_heads], finite and > 0 (not checked).
+ */
+pa_status pa_cache_append_fp8(const void *k, const void *v, const int32_t *slot_mapping,
+                              int32_t num_tokens, void *k_cache, void *v_cache,
+                              const float *k_scale, const float *v_scale,
+                              const pa_shape *shape, pa_stream_t stream);
+
+/*
+ * Decode attention over an E4M3 cache (shape->cache_format ==
+ * PA_CACHE_FP8_E4M3, else PA_ERR_INVALID_ARG): pa_decode's result with
+ * K_j = code * k_scale[h / g] and V_j = code * v_scale[h / g].  Runs the
+ * CUDA-core kernel (variant PA_DECODE_TENSOR_CORES or shared_prefix give
+ * PA_ERR_UNSUPPORTED); the K scale is folded into the query and the V scale
+ * into the output.  Same workspace as pa_decode.  k_scale, v_scale: device
+ * fp32 [num_kv_heads].
+ */
+pa_status pa_decode_fp8(const void *q, const void *k_cache, const void *v_cache,
+                        const float *k_scale, const float *v_scale,
+                        const int32_t *block_tables, const int32_t *context_lens, float scale,
+                        void *out, const pa_shape *shape, int32_t max_context_len,
+                        void *workspace, size_t workspace_bytes, pa_stream_t stream);
+
+/*
  * Copy-on-write of whole blocks (zingnex.cn section 3.2 item 3): for each
  * pair i, block src_dst_pairs[2i+1] of k_cache and of v_cache becomes a
- * byte copy of block src_dst_pairs[2i].  Destinations must be distinct and no
+ * byte copy of block src_dst_pairs[2i] (either cache format: a block is
+ * block_size * num_kv_heads * head_dim elements of 2 or 1 bytes).
+ * Destinations must be distinct and no
  * destination may also be a source in the same call.
  * src_dst_pairs: device int32 [num_pairs][2].  num_pairs == 0 launches nothing.
  */
@@ -249,7 +298,7 @@ pa_status pa_last_device_error(pa_stream_t stream, uint32_t *bits_out);
 const char *pa_status_string(pa_status status);
 
 /* Text of the CUDA error behind the calling thread's most recent
- * PA_ERR_CUDA from pa_decode, pa_cache_append, pa_copy_blocks or
+ * PA_ERR_CUDA from pa_decode(_fp8), pa_cache_append(_fp8), pa_copy_blocks or
  * pa_last_device_error ("no CUDA error" before the first one).  The string is
  * static; the caller does not free it.  Not part of the method: a diagnostic
  * of this library. */

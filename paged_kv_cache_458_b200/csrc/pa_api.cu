@@ -63,6 +63,8 @@ pa_status check_pool_shape(const pa_shape* s) {
   if (s->num_kv_heads <= 0 || s->head_dim <= 0 || s->block_size <= 0 || s->num_blocks < 0)
     return PA_ERR_INVALID_ARG;
   if (s->dtype != PA_F16 && s->dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (s->cache_format != PA_CACHE_AS_DTYPE && s->cache_format != PA_CACHE_FP8_E4M3)
+    return PA_ERR_UNSUPPORTED;
   if (s->head_dim != 64 && s->head_dim != 128) return PA_ERR_UNSUPPORTED;
   if (s->block_size % 16 != 0) return PA_ERR_UNSUPPORTED;
   if ((long long)s->num_blocks * s->block_size >= (1LL << 31)) return PA_ERR_UNSUPPORTED;
@@ -85,6 +87,9 @@ pa_status check_decode_shape(const pa_shape* s, int32_t max_context_len) {
       (s->head_dim != 128 || pt % pa::decode_tc_tile_tokens() != 0 || pt > 512))
     return PA_ERR_UNSUPPORTED;
   if (s->shared_prefix != 0 && s->shared_prefix != 1) return PA_ERR_INVALID_ARG;
+  // an E4M3 cache is read by the CUDA-core kernel only
+  if (s->cache_format == PA_CACHE_FP8_E4M3 && (s->variant == PA_DECODE_TENSOR_CORES || s->shared_prefix))
+    return PA_ERR_UNSUPPORTED;
   if (s->shared_prefix &&
       (s->variant != PA_DECODE_AUTO || s->head_dim != 128 || pt % pa::decode_tc_tile_tokens() != 0 ||
        pt > 512))
@@ -96,7 +101,11 @@ pa_status check_decode_shape(const pa_shape* s, int32_t max_context_len) {
 }
 
 // Whether pa_decode runs the tensor-core variant for this (valid) shape.
+// Bytes of one cached element.
+int cache_elem_bytes(const pa_shape* s) { return s->cache_format == PA_CACHE_FP8_E4M3 ? 1 : 2; }
+
 bool use_tensor_cores(const pa_shape* s) {
+  if (s->cache_format == PA_CACHE_FP8_E4M3) return false;
   if (s->variant == PA_DECODE_TENSOR_CORES) return true;
   if (s->variant == PA_DECODE_CUDA_CORES) return false;
   const int pt = effective_partition(s);
@@ -166,13 +175,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 bool make_pool_map(CUtensorMap* map, const void* pool, const pa_shape* s, int rows) {
   auto fn = encode_fn();
   if (!fn) return false;
+  const int eb = cache_elem_bytes(s);
   const cuuint64_t dims[3] = {(cuuint64_t)s->head_dim, (cuuint64_t)s->num_kv_heads,
                               (cuuint64_t)s->num_blocks * s->block_size};
-  const cuuint64_t strides[2] = {(cuuint64_t)s->head_dim * 2,
-                                 (cuuint64_t)s->num_kv_heads * s->head_dim * 2};
+  const cuuint64_t strides[2] = {(cuuint64_t)s->head_dim * eb,
+                                 (cuuint64_t)s->num_kv_heads * s->head_dim * eb};
   const cuuint32_t box[3] = {(cuuint32_t)s->head_dim, 1, (cuuint32_t)rows};
   const cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(pool), dims, strides,
+  CUresult r = fn(map, eb == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 3,
+                  const_cast<void*>(pool), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -219,13 +230,24 @@ size_t pa_decode_workspace_bytes(const pa_shape* shape, int32_t max_context_len)
   return (size_t)(head + round256(acc) + ml);
 }
 
-pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
-                    const int32_t* block_tables, const int32_t* context_lens, float scale,
-                    void* out, const pa_shape* shape, int32_t max_context_len, void* workspace,
-                    size_t workspace_bytes, pa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// pa_decode and pa_decode_fp8 (scales set iff the cache holds E4M3 codes).
+pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
+                      const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                      const int32_t* context_lens, float scale, void* out, const pa_shape* shape,
+                      int32_t max_context_len, void* workspace, size_t workspace_bytes,
+                      pa_stream_t stream) {
   pa_status st = check_decode_shape(shape, max_context_len);
   if (st != PA_OK) return st;
+  const bool fp8 = shape->cache_format == PA_CACHE_FP8_E4M3;
+  if (fp8 != (k_scale != nullptr)) return PA_ERR_INVALID_ARG;  // the entry point must match
   if (shape->num_seqs == 0) return PA_OK;
+  if (fp8 && (!v_scale || (reinterpret_cast<uintptr_t>(k_scale) & 3u) ||
+              (reinterpret_cast<uintptr_t>(v_scale) & 3u)))
+    return PA_ERR_INVALID_ARG;
   if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out) return PA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
     return PA_ERR_INVALID_ARG;
@@ -257,6 +279,8 @@ pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
     a.ws_ml = reinterpret_cast<float*>(ws + round256(rows * shape->head_dim * 4));
   }
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
   a.num_seqs = shape->num_seqs;
   a.num_q_heads = shape->num_q_heads;
   a.num_kv_heads = shape->num_kv_heads;
@@ -329,10 +353,32 @@ pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
       memset(&tk, 0, sizeof tk);
       memset(&tv, 0, sizeof tv);
     }
-    e = pa::launch_decode(a, shape->dtype, shape->head_dim, group, tk, tv, cs, &launched);
+    e = pa::launch_decode(a, shape->dtype, shape->head_dim, group, tk, tv, cs, &launched, fp8);
   }
   count_launches(launched);
   return e == cudaSuccess ? PA_OK : cuda_failed(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, const int32_t* context_lens, float scale,
+                    void* out, const pa_shape* shape, int32_t max_context_len, void* workspace,
+                    size_t workspace_bytes, pa_stream_t stream) {
+  return decode_impl(q, k_cache, v_cache, nullptr, nullptr, block_tables, context_lens, scale, out,
+                     shape, max_context_len, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache,
+                        const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                        const int32_t* context_lens, float scale, void* out, const pa_shape* shape,
+                        int32_t max_context_len, void* workspace, size_t workspace_bytes,
+                        pa_stream_t stream) {
+  if (!k_scale) return PA_ERR_INVALID_ARG;
+  return decode_impl(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale, out,
+                     shape, max_context_len, workspace, workspace_bytes, stream);
 }
 
 pa_status pa_cache_append(const void* k, const void* v, const int32_t* slot_mapping,
@@ -342,6 +388,7 @@ pa_status pa_cache_append(const void* k, const void* v, const int32_t* slot_mapp
   if (st != PA_OK) return st;
   if (num_tokens < 0) return PA_ERR_INVALID_ARG;
   if (num_tokens == 0) return PA_OK;
+  if (shape->cache_format != PA_CACHE_AS_DTYPE) return PA_ERR_INVALID_ARG;  // pa_cache_append_fp8
   if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PA_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
       (reinterpret_cast<uintptr_t>(slot_mapping) & 3u))
@@ -358,6 +405,32 @@ pa_status pa_cache_append(const void* k, const void* v, const int32_t* slot_mapp
   return e == cudaSuccess ? PA_OK : cuda_failed(e);
 }
 
+pa_status pa_cache_append_fp8(const void* k, const void* v, const int32_t* slot_mapping,
+                              int32_t num_tokens, void* k_cache, void* v_cache,
+                              const float* k_scale, const float* v_scale, const pa_shape* shape,
+                              pa_stream_t stream) {
+  pa_status st = check_pool_shape(shape);
+  if (st != PA_OK) return st;
+  if (shape->cache_format != PA_CACHE_FP8_E4M3) return PA_ERR_INVALID_ARG;
+  if (num_tokens < 0) return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !slot_mapping || !k_cache || !v_cache || !k_scale || !v_scale)
+    return PA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (reinterpret_cast<uintptr_t>(slot_mapping) & 3u) ||
+      (reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u))
+    return PA_ERR_INVALID_ARG;
+  unsigned int* err = error_word();
+  if (!err) return cuda_failed("device error word lookup failed");
+  int launched = 0;
+  cudaError_t e = pa::launch_cache_append_fp8(
+      k, v, slot_mapping, num_tokens, k_cache, v_cache,
+      (long long)shape->num_blocks * shape->block_size, shape->dtype, shape->num_kv_heads,
+      shape->head_dim, k_scale, v_scale, err, reinterpret_cast<cudaStream_t>(stream), &launched);
+  count_launches(launched);
+  return e == cudaSuccess ? PA_OK : cuda_failed(e);
+}
+
 pa_status pa_copy_blocks(const int32_t* src_dst_pairs, int32_t num_pairs, void* k_cache,
                          void* v_cache, const pa_shape* shape, pa_stream_t stream) {
   pa_status st = check_pool_shape(shape);
@@ -368,8 +441,8 @@ pa_status pa_copy_blocks(const int32_t* src_dst_pairs, int32_t num_pairs, void* 
   if (!src_dst_pairs || !k_cache || !v_cache) return PA_ERR_INVALID_ARG;
   if (!aligned16(k_cache) || !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(src_dst_pairs) & 3u))
     return PA_ERR_INVALID_ARG;
-  const long long block_bytes =
-      (long long)shape->block_size * shape->num_kv_heads * shape->head_dim * 2;
+  const long long block_bytes = (long long)shape->block_size * shape->num_kv_heads *
+                                shape->head_dim * cache_elem_bytes(shape);
   unsigned int* err = error_word();
   if (!err) return cuda_failed("device error word lookup failed");
   int launched = 0;

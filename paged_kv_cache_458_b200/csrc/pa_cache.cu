@@ -42,6 +42,60 @@ cache_append_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
   }
 }
 
+// Append into an E4M3 cache.  One CTA per token; each thread converts 8
+// consecutive elements (16 bytes in, 8 bytes out) per step: x / scale[head]
+// in fp32 (IEEE division, round to nearest), then the nearest E4M3 code,
+// ties to even, saturating at 448.
+template <typename T>
+__global__ void __launch_bounds__(256)
+cache_append_fp8_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                        const int32_t* __restrict__ slot_mapping, uint2* __restrict__ k_cache,
+                        uint2* __restrict__ v_cache, long long num_slots, int head_dim,
+                        int row_vecs, const float* __restrict__ k_scale,
+                        const float* __restrict__ v_scale, unsigned int* err) {
+  pdl_wait();  // a copy-on-write of this slot's block must land first
+  pdl_launch_dependents();
+  const int t = blockIdx.x;
+  const long long slot = __ldg(slot_mapping + t);
+  if (slot < 0) return;
+  if (slot >= num_slots) {
+    if (threadIdx.x == 0) report(err, kErrSlot);
+    return;
+  }
+  for (int i = threadIdx.x; i < row_vecs; i += blockDim.x) {
+    const int h = (i * 8) / head_dim;  // 8 elements never straddle two heads
+    const float ks = __ldg(k_scale + h), vs = __ldg(v_scale + h);
+    const uint4 xk = __ldg(k + (size_t)t * row_vecs + i), xv = __ldg(v + (size_t)t * row_vecs + i);
+    uint2 ok, ov;
+    uint32_t* pk = &ok.x;
+    uint32_t* pv = &ov.x;
+    const uint32_t wk[4] = {xk.x, xk.y, xk.z, xk.w}, wv[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+    for (int w = 0; w < 4; w += 2) {
+      const float2 k0 = Elem<T>::to_f2(wk[w]), k1 = Elem<T>::to_f2(wk[w + 1]);
+      const float2 v0 = Elem<T>::to_f2(wv[w]), v1 = Elem<T>::to_f2(wv[w + 1]);
+      const uint32_t ck = (uint32_t)__nv_cvt_float2_to_fp8x2(
+                              make_float2(__fdiv_rn(k0.x, ks), __fdiv_rn(k0.y, ks)), __NV_SATFINITE,
+                              __NV_E4M3) |
+                          ((uint32_t)__nv_cvt_float2_to_fp8x2(
+                               make_float2(__fdiv_rn(k1.x, ks), __fdiv_rn(k1.y, ks)), __NV_SATFINITE,
+                               __NV_E4M3)
+                           << 16);
+      const uint32_t cv = (uint32_t)__nv_cvt_float2_to_fp8x2(
+                              make_float2(__fdiv_rn(v0.x, vs), __fdiv_rn(v0.y, vs)), __NV_SATFINITE,
+                              __NV_E4M3) |
+                          ((uint32_t)__nv_cvt_float2_to_fp8x2(
+                               make_float2(__fdiv_rn(v1.x, vs), __fdiv_rn(v1.y, vs)), __NV_SATFINITE,
+                               __NV_E4M3)
+                           << 16);
+      pk[w / 2] = ck;
+      pv[w / 2] = cv;
+    }
+    k_cache[slot * row_vecs + i] = ok;
+    v_cache[slot * row_vecs + i] = ov;
+  }
+}
+
 // grid.x = pieces of a block, grid.y = pair.  Each CTA copies kPiece vectors
 // of the K block and of the V block.
 constexpr int kCopyThreads = 256;
@@ -89,6 +143,23 @@ cudaError_t launch_cache_append(const void* k, const void* v, const int32_t* slo
                              static_cast<const uint4*>(k), static_cast<const uint4*>(v),
                              slot_mapping, static_cast<uint4*>(k_cache),
                              static_cast<uint4*>(v_cache), num_slots, row_vecs, err);
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
+cudaError_t launch_cache_append_fp8(const void* k, const void* v, const int32_t* slot_mapping,
+                                    int num_tokens, void* k_cache, void* v_cache,
+                                    long long num_slots, int dtype, int num_kv_heads, int head_dim,
+                                    const float* k_scale, const float* v_scale, unsigned int* err,
+                                    cudaStream_t stream, int* launches) {
+  if (num_tokens == 0) return cudaSuccess;
+  const int row_vecs = num_kv_heads * head_dim / 8;  // 8 elements per step
+  const int threads = row_vecs >= 256 ? 256 : ((row_vecs + 31) / 32) * 32;
+  auto* kern = dtype == 0 ? cache_append_fp8_kernel<__half> : cache_append_fp8_kernel<__nv_bfloat16>;
+  cudaError_t e = launch_pdl(kern, dim3(num_tokens), dim3(threads), 0, stream,
+                             static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
+                             static_cast<uint2*>(k_cache), static_cast<uint2*>(v_cache), num_slots,
+                             head_dim, row_vecs, k_scale, v_scale, err);
   if (e == cudaSuccess) ++*launches;
   return e;
 }

@@ -10,6 +10,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 namespace pa {
@@ -54,6 +55,16 @@ template <> struct Elem<__nv_bfloat16> {
     return *reinterpret_cast<uint16_t*>(&b);
   }
 };
+
+// 8-bit E4M3 cache codes (one byte per element) and their widening.
+struct Fp8E4M3 {};
+
+// Two E4M3 codes (low byte first) -> two floats, exact (via the hardware
+// E4M3 -> f16 conversion, which every E4M3 value survives unchanged).
+__device__ __forceinline__ float2 e4m3x2_to_f2(uint16_t u) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(u), __NV_E4M3);
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
 
 // ---------------------------------------------------------------------------
 // time and shared-memory addressing

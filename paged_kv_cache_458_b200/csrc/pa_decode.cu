@@ -35,6 +35,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "pa_common.cuh"
 #include "pa_internal.h"
 
@@ -42,16 +44,17 @@ namespace pa {
 
 constexpr int kChunk = 16;  // tokens per TMA box (a block is a multiple of this)
 
-template <int D, int G, int NW, int NST>
+template <int D, int G, int NW, int NST, int EB = 2>  // EB: bytes per cached element
 struct DecodeSmem {
-  static constexpr int kRowBytes = D * 2;
+  static constexpr int kRowBytes = D * EB;
   static constexpr int kStageBytes = 2 * kChunk * kRowBytes;  // K box then V box
   static constexpr int kStagesBytes = NW * NST * kStageBytes;
   static constexpr int kPBytes = NW * (kChunk * G + G) * 4;   // p[16][G] + alpha[G] per warp
   static constexpr int kBarBytes = NW * NST * 8;
   static constexpr int kMergeBytes = NW * (G * D + 2 * G) * 4;
-  static_assert(kMergeBytes <= kStagesBytes, "merge area reuses the stage buffers");
-  static constexpr int kTotal = kStagesBytes + kPBytes + kBarBytes;
+  // the warps' final merge reuses the stage buffers (grown if they are smaller)
+  static constexpr int kStageArea = kMergeBytes > kStagesBytes ? kMergeBytes : kStagesBytes;
+  static constexpr int kTotal = kStageArea + kPBytes + kBarBytes;
 };
 
 __device__ __forceinline__ float warp_max_xor(float v, int lo, int hi) {
@@ -112,11 +115,32 @@ __device__ __forceinline__ void load_row_slice(const unsigned char* row, int lan
   }
 }
 
-template <typename T, int D, int G, int NW, int NST>
+// This lane's D/32 elements of a cached row, widened: 16-bit elements as
+// load_row_slice, E4M3 codes exactly (the head's scale is applied elsewhere).
+template <typename KV, typename T, int D>
+__device__ __forceinline__ void load_kv_slice(const unsigned char* row, int lane, float* out) {
+  if constexpr (std::is_same<KV, Fp8E4M3>::value) {
+    if constexpr (D == 128) {
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(row + lane * 4);
+      const float2 a = e4m3x2_to_f2((uint16_t)(u & 0xffffu)), b = e4m3x2_to_f2((uint16_t)(u >> 16));
+      out[0] = a.x; out[1] = a.y; out[2] = b.x; out[3] = b.y;
+    } else {
+      const float2 a = e4m3x2_to_f2(*reinterpret_cast<const uint16_t*>(row + lane * 2));
+      out[0] = a.x; out[1] = a.y;
+    }
+  } else {
+    load_row_slice<T, D>(row, lane, out);
+  }
+}
+
+// KV: T (fp16/bf16 cache) or Fp8E4M3 (one-byte codes, per-kv-head scales:
+// the K scale is folded into the query, the V scale into the output).
+template <typename T, typename KV, int D, int G, int NW, int NST>
 __global__ void __launch_bounds__(NW * 32)
 decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v) {
-  using L = DecodeSmem<D, G, NW, NST>;
+  constexpr bool kFp8 = std::is_same<KV, Fp8E4M3>::value;
+  using L = DecodeSmem<D, G, NW, NST, kFp8 ? 1 : 2>;
   constexpr int VEC = D / 32;
   constexpr int TPP = (G == 1) ? 16 : 32 / G;  // tokens per reduce-scatter pass
   constexpr int NPASS = kChunk / TPP;          // passes per chunk
@@ -159,10 +183,10 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
   const int n_mine = warp < n_chunks ? (n_chunks - warp + NW - 1) / NW : 0;
 
   unsigned char* stages = smem;
-  float* p_all = reinterpret_cast<float*>(smem + L::kStagesBytes);
+  float* p_all = reinterpret_cast<float*>(smem + L::kStageArea);
   float* p_sm = p_all + warp * (kChunk * G + G);  // [16][G]
   float* alpha_sm = p_sm + kChunk * G;             // [G]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kStagesBytes + L::kPBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kStageArea + L::kPBytes);
   const uint32_t bar0 = smem_addr(bars + warp * NST);
   const uint32_t stage0 = smem_addr(stages + warp * NST * L::kStageBytes);
 
@@ -201,7 +225,10 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
     }
   };
 
-  // Query group in registers, pre-scaled into the log2 domain.
+  // Query group in registers, pre-scaled into the log2 domain (and by the K
+  // scale of an E4M3 cache).
+  float qscale = a.scale_log2;
+  if constexpr (kFp8) qscale *= __ldg(a.k_scale + kvh);
   float qr[G][VEC];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
@@ -209,7 +236,7 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
         a.q + ((size_t)s * a.num_q_heads + q_head0 + h) * D);
     load_row_slice<T, D>(qrow, lane, qr[h]);
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) qr[h][v] *= a.scale_log2;
+    for (int v = 0; v < VEC; ++v) qr[h][v] *= qscale;
   }
 
   float acc[G][VEC];
@@ -242,7 +269,7 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
 #pragma unroll
       for (int jj = 0; jj < TPP; ++jj) {
         float kf[VEC];
-        load_row_slice<T, D>(Ks + (ps * TPP + jj) * L::kRowBytes, lane, kf);
+        load_kv_slice<KV, T, D>(Ks + (ps * TPP + jj) * L::kRowBytes, lane, kf);
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           float d = 0.f;
@@ -286,7 +313,7 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
     }
     for (int j = 0; j < n_valid; ++j) {
       float vf[VEC];
-      load_row_slice<T, D>(Vs + j * L::kRowBytes, lane, vf);
+      load_kv_slice<KV, T, D>(Vs + j * L::kRowBytes, lane, vf);
       float pj[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) pj[h] = p_sm[j * G + h];
@@ -337,6 +364,7 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
       num = fmaf(wt, mg_acc[(w * G + h) * D + d], num);
       den = fmaf(wt, mg_l[w * G + h], den);
     }
+    if constexpr (kFp8) num *= __ldg(a.v_scale + kvh);
     if (any_failed) num = __int_as_float(0x7fc00000), den = 1.f;
     const size_t qh = (size_t)s * a.num_q_heads + q_head0 + h;
     if (direct) {
@@ -409,11 +437,11 @@ namespace {
 constexpr int kWarps = PA_DECODE_WARPS;
 constexpr int kStages = PA_DECODE_STAGES;
 
-template <typename T, int D, int G>
+template <typename T, typename KV, int D, int G>
 cudaError_t launch_typed(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
                          int grid, cudaStream_t stream, int* launches) {
-  using L = DecodeSmem<D, G, kWarps, kStages>;
-  auto* kern = decode_partition_kernel<T, D, G, kWarps, kStages>;
+  using L = DecodeSmem<D, G, kWarps, kStages, std::is_same<KV, Fp8E4M3>::value ? 1 : 2>;
+  auto* kern = decode_partition_kernel<T, KV, D, G, kWarps, kStages>;
   static bool configured = false;  // per instantiation; idempotent if raced
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
@@ -430,33 +458,42 @@ cudaError_t launch_typed(const DecodeArgs& a, const CUtensorMap& tk, const CUten
   return e;
 }
 
-template <typename T, int D>
+template <typename T, typename KV, int D>
 cudaError_t launch_group(const DecodeArgs& a, int G, const CUtensorMap& tk, const CUtensorMap& tv,
                          int grid, cudaStream_t st, int* n) {
   switch (G) {
-    case 1: return launch_typed<T, D, 1>(a, tk, tv, grid, st, n);
-    case 2: return launch_typed<T, D, 2>(a, tk, tv, grid, st, n);
-    case 4: return launch_typed<T, D, 4>(a, tk, tv, grid, st, n);
-    case 8: return launch_typed<T, D, 8>(a, tk, tv, grid, st, n);
-    case 16: return launch_typed<T, D, 16>(a, tk, tv, grid, st, n);
+    case 1: return launch_typed<T, KV, D, 1>(a, tk, tv, grid, st, n);
+    case 2: return launch_typed<T, KV, D, 2>(a, tk, tv, grid, st, n);
+    case 4: return launch_typed<T, KV, D, 4>(a, tk, tv, grid, st, n);
+    case 8: return launch_typed<T, KV, D, 8>(a, tk, tv, grid, st, n);
+    case 16: return launch_typed<T, KV, D, 16>(a, tk, tv, grid, st, n);
   }
   return cudaErrorInvalidValue;
+}
+
+template <typename T, typename KV>
+cudaError_t launch_dims(const DecodeArgs& a, int head_dim, int group, const CUtensorMap& tk,
+                        const CUtensorMap& tv, int grid, cudaStream_t stream, int* launches) {
+  if (head_dim == 128) return launch_group<T, KV, 128>(a, group, tk, tv, grid, stream, launches);
+  return launch_group<T, KV, 64>(a, group, tk, tv, grid, stream, launches);
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const DecodeArgs& a, int dtype, int head_dim, int group,
                           const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream,
-                          int* launches) {
+                          int* launches, bool fp8_cache) {
   const long long grid = (long long)a.grid_parts * a.num_seqs * a.num_kv_heads;
   if (grid <= 0) return cudaSuccess;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  if (dtype == 0) {
-    if (head_dim == 128) return launch_group<__half, 128>(a, group, tk, tv, (int)grid, stream, launches);
-    return launch_group<__half, 64>(a, group, tk, tv, (int)grid, stream, launches);
-  }
-  if (head_dim == 128) return launch_group<__nv_bfloat16, 128>(a, group, tk, tv, (int)grid, stream, launches);
-  return launch_group<__nv_bfloat16, 64>(a, group, tk, tv, (int)grid, stream, launches);
+  const int g = (int)grid;
+  if (dtype == 0)
+    return fp8_cache ? launch_dims<__half, Fp8E4M3>(a, head_dim, group, tk, tv, g, stream, launches)
+                     : launch_dims<__half, __half>(a, head_dim, group, tk, tv, g, stream, launches);
+  return fp8_cache
+             ? launch_dims<__nv_bfloat16, Fp8E4M3>(a, head_dim, group, tk, tv, g, stream, launches)
+             : launch_dims<__nv_bfloat16, __nv_bfloat16>(a, head_dim, group, tk, tv, g, stream,
+                                                         launches);
 }
 
 cudaError_t launch_decode_merge(const DecodeArgs& a, int dtype, int head_dim, cudaStream_t stream,

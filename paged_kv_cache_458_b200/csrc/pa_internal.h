@@ -27,6 +27,8 @@ struct DecodeArgs {
   // Shared-prefix decode (nullptr: off): per sequence {rank in its group,
   // members, shared tokens T, shared partitions}.  A sequence's own items
   // then cover [T, ctx), as partitions numbered from its shared partitions.
+  const float* k_scale;          // [Hkv] with an E4M3 cache (stored value = code * scale)
+  const float* v_scale;          // [Hkv]
   const int4* plan;
   int own_tokens;                // partition size of a sequence's own tokens (partition_tokens
                                  // without a plan)
@@ -72,10 +74,11 @@ __host__ __device__ inline SeqSplit seq_split(const int4* plan, int s, int ctx, 
 }
 
 // Launch the partition kernel (+ the merge kernel when num_parts > 1).
-// `launches` is incremented once per kernel launched.
+// `launches` is incremented once per kernel launched.  fp8_cache: K/V hold
+// E4M3 codes (a.k_scale / a.v_scale set).
 cudaError_t launch_decode(const DecodeArgs& a, int dtype, int head_dim, int group,
                           const CUtensorMap& tm_k, const CUtensorMap& tm_v, cudaStream_t stream,
-                          int* launches);
+                          int* launches, bool fp8_cache = false);
 int decode_chunk_tokens();
 int decode_max_partition_tokens();
 // The split-K merge alone (after a partition kernel that wrote partials).
@@ -97,6 +100,14 @@ cudaError_t launch_cache_append(const void* k, const void* v, const int32_t* slo
                                 int num_tokens, void* k_cache, void* v_cache, long long num_slots,
                                 int row_bytes, unsigned int* err, cudaStream_t stream,
                                 int* launches);
+// Append into an E4M3 cache: k, v rows of Hkv * D fp16/bf16 elements (dtype
+// 0 / 1) are divided by their head's scale and rounded to E4M3 (nearest,
+// ties to even, saturating at 448).
+cudaError_t launch_cache_append_fp8(const void* k, const void* v, const int32_t* slot_mapping,
+                                    int num_tokens, void* k_cache, void* v_cache,
+                                    long long num_slots, int dtype, int num_kv_heads, int head_dim,
+                                    const float* k_scale, const float* v_scale, unsigned int* err,
+                                    cudaStream_t stream, int* launches);
 cudaError_t launch_copy_blocks(const int32_t* pairs, int num_pairs, void* k_cache, void* v_cache,
                                int num_blocks, long long block_bytes, unsigned int* err,
                                cudaStream_t stream, int* launches);

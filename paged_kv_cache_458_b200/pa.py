@@ -21,6 +21,7 @@ PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_OOM, PA_ERR_D
 PA_F16, PA_BF16 = 0, 1
 PA_DECODE_AUTO, PA_DECODE_CUDA_CORES, PA_DECODE_TENSOR_CORES = 0, 1, 2
 PA_DECODE_RESOLVED_SHARED_PREFIX = 3
+PA_CACHE_AS_DTYPE, PA_CACHE_FP8_E4M3 = 0, 1
 PA_DEVERR_BLOCK_ID = 0x1
 PA_DEVERR_CONTEXT_LEN = 0x2
 PA_DEVERR_SLOT = 0x4
@@ -44,7 +45,8 @@ class PaError(RuntimeError):
 class pa_shape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "num_seqs", "num_q_heads", "num_kv_heads", "head_dim", "block_size", "num_blocks",
-        "max_blocks_per_seq", "partition_tokens", "dtype", "variant", "shared_prefix")]
+        "max_blocks_per_seq", "partition_tokens", "dtype", "variant", "shared_prefix",
+        "cache_format")]
 
     def __repr__(self):
         return "pa_shape(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -66,6 +68,10 @@ def _declare(lib):
     lib.pa_decode_noalloc.argtypes = [P, P, P, P, P, c.c_float, P, SP, I32, P]
     lib.pa_cache_append.restype = c.c_int
     lib.pa_cache_append.argtypes = [P, P, P, I32, P, P, SP, P]
+    lib.pa_cache_append_fp8.restype = c.c_int
+    lib.pa_cache_append_fp8.argtypes = [P, P, P, I32, P, P, P, P, SP, P]
+    lib.pa_decode_fp8.restype = c.c_int
+    lib.pa_decode_fp8.argtypes = [P, P, P, P, P, P, P, c.c_float, P, SP, I32, P, SZ, P]
     lib.pa_copy_blocks.restype = c.c_int
     lib.pa_copy_blocks.argtypes = [P, I32, P, P, SP, P]
     lib.pa_last_device_error.restype = c.c_int
@@ -155,9 +161,10 @@ def _stream(stream) -> int | None:
 
 def make_shape(*, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
                max_blocks_per_seq, partition_tokens=0, dtype=PA_F16, variant=0,
-               shared_prefix=0) -> pa_shape:
+               shared_prefix=0, cache_format=PA_CACHE_AS_DTYPE) -> pa_shape:
     return pa_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
-                    max_blocks_per_seq, partition_tokens, dtype, variant, shared_prefix)
+                    max_blocks_per_seq, partition_tokens, dtype, variant, shared_prefix,
+                    cache_format)
 
 
 def torch_dtype(dtype: int):
@@ -202,6 +209,24 @@ def pa_cache_append(k, v, slot_mapping, num_tokens: int, k_cache, v_cache, shape
     _check("pa_cache_append", lib().pa_cache_append(
         _ptr(k), _ptr(v), _ptr(slot_mapping), int(num_tokens), _ptr(k_cache), _ptr(v_cache),
         ctypes.byref(shape), _stream(stream)))
+
+
+def pa_cache_append_fp8(k, v, slot_mapping, num_tokens: int, k_cache, v_cache, k_scale, v_scale,
+                        shape: pa_shape, stream=None) -> None:
+    _check("pa_cache_append_fp8", lib().pa_cache_append_fp8(
+        _ptr(k), _ptr(v), _ptr(slot_mapping), int(num_tokens), _ptr(k_cache), _ptr(v_cache),
+        _ptr(k_scale), _ptr(v_scale), ctypes.byref(shape), _stream(stream)))
+
+
+def pa_decode_fp8(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale: float,
+                  out, shape: pa_shape, max_context_len: int, workspace=None,
+                  workspace_bytes: int | None = None, stream=None) -> None:
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("pa_decode_fp8", lib().pa_decode_fp8(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+        _ptr(context_lens), float(scale), _ptr(out), ctypes.byref(shape), int(max_context_len),
+        _ptr(workspace), int(workspace_bytes), _stream(stream)))
 
 
 def pa_copy_blocks(src_dst_pairs, num_pairs: int, k_cache, v_cache, shape: pa_shape,

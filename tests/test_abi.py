@@ -80,6 +80,41 @@ def test_shared_prefix_workspace(lib):
     assert pa.pa_decode_resolved_variant(s) == pa.PA_DECODE_RESOLVED_SHARED_PREFIX
 
 
+def test_fp8_cache_validation(lib):
+    s8 = _shape(cache_format=pa.PA_CACHE_FP8_E4M3)
+    s16 = _shape()
+    args = (FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE)
+    # each entry point takes its own cache format
+    assert lib.pa_decode(*args, ctypes.byref(s8), 100, FAKE, 1 << 20, None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_decode_fp8(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s16),
+                             100, FAKE, 1 << 20, None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_decode_fp8(FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s8),
+                             100, FAKE, 1 << 20, None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_decode_fp8(FAKE, FAKE, FAKE, FAKE + 2, FAKE, FAKE, FAKE, 0.1, FAKE,
+                             ctypes.byref(s8), 100, FAKE, 1 << 20, None) == pa.PA_ERR_INVALID_ARG
+    for bad, st in ((dict(cache_format=2), pa.PA_ERR_UNSUPPORTED),
+                    (dict(cache_format=pa.PA_CACHE_FP8_E4M3, variant=2), pa.PA_ERR_UNSUPPORTED),
+                    (dict(cache_format=pa.PA_CACHE_FP8_E4M3, shared_prefix=1),
+                     pa.PA_ERR_UNSUPPORTED)):
+        s = _shape(**bad)
+        assert lib.pa_decode_fp8(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE,
+                                 ctypes.byref(s), 100, FAKE, 1 << 20, None) == st
+    assert pa.pa_decode_resolved_variant(_shape(cache_format=1, num_q_heads=16)) == \
+        pa.PA_DECODE_CUDA_CORES
+    # appends
+    assert lib.pa_cache_append(FAKE, FAKE, FAKE, 3, FAKE, FAKE, ctypes.byref(s8), None) == \
+        pa.PA_ERR_INVALID_ARG
+    assert lib.pa_cache_append_fp8(FAKE, FAKE, FAKE, 3, FAKE, FAKE, FAKE, FAKE, ctypes.byref(s16),
+                                   None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_cache_append_fp8(FAKE, FAKE, FAKE, 3, FAKE, FAKE, None, FAKE, ctypes.byref(s8),
+                                   None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_cache_append_fp8(FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, ctypes.byref(s8),
+                                   None) == pa.PA_OK
+    # the workspace does not depend on the cache format
+    assert lib.pa_decode_workspace_bytes(ctypes.byref(s8), 1000) == \
+        lib.pa_decode_workspace_bytes(ctypes.byref(s16), 1000)
+
+
 def test_resolved_variant(lib):
     assert pa.pa_decode_resolved_variant(_shape()) == pa.PA_DECODE_CUDA_CORES          # group 4
     assert pa.pa_decode_resolved_variant(_shape(num_q_heads=16)) == pa.PA_DECODE_TENSOR_CORES

@@ -7,6 +7,12 @@ half a unit in the last place, and fp32 arithmetic near a rounding boundary
 can move the result by one more half unit.  Where one ulp of the output type
 exceeds 2e-3 (bf16 at |o| >= 0.5, fp16 at |o| >= 4) the per-element bound is
 one ulp of that type at the exact value instead.  The number of elements that used that branch is reported.
+
+The mean bound likewise counts only what the kernel adds to the rounding of
+the output: mean |err| <= 2e-4 + mean |round(ref) - ref|, where round(ref)
+is the exact result rounded to the output type.  Rounding alone averages a
+quarter ulp, 4.9e-4 for bf16 outputs in [0.25, 0.5), so without this term no
+implementation could meet the bound on short contexts.
 """
 import numpy as np
 
@@ -25,12 +31,21 @@ def ulp(ref: np.ndarray, dtype: int) -> np.ndarray:
     return np.exp2(e - _MANTISSA[dtype])
 
 
+def rounding_floor(ref: np.ndarray, dtype: int) -> float:
+    """Mean |round(ref) - ref| with round() to the output type."""
+    if ref.size == 0:
+        return 0.0
+    r = gen.bits_to_f32(gen.to_bits(ref.astype(np.float32), dtype), dtype).astype(np.float64)
+    return float(np.mean(np.abs(r - ref)))
+
+
 def decode_errors(out_bits: np.ndarray, ref: np.ndarray, dtype: int) -> dict:
     got = gen.bits_to_f32(out_bits, dtype).astype(np.float64).reshape(ref.shape)
     err = np.abs(got - ref)
     allowed = np.maximum(MAX_ABS, ulp(ref, dtype))
     return dict(max_abs=float(np.nanmax(err)) if err.size else 0.0,
                 mean_abs=float(np.mean(err)) if err.size else 0.0,
+                mean_floor=rounding_floor(ref, dtype),
                 n_nan=int(np.isnan(got).sum()),
                 n_over=int((err > allowed).sum()),
                 n_ulp_branch=int((ulp(ref, dtype) > MAX_ABS).sum()),
@@ -41,5 +56,6 @@ def assert_decode_close(out_bits, ref, dtype, what=""):
     st = decode_errors(out_bits, ref, dtype)
     assert st["n_nan"] == 0, f"{what}: {st['n_nan']} NaN outputs"
     assert st["n_over"] == 0, f"{what}: {st['n_over']} elements above the bound (max {st['max_abs']:.3e})"
-    assert st["mean_abs"] <= MEAN_ABS, f"{what}: mean abs error {st['mean_abs']:.3e}"
+    assert st["mean_abs"] <= MEAN_ABS + st["mean_floor"], \
+        f"{what}: mean abs error {st['mean_abs']:.3e} (rounding alone {st['mean_floor']:.3e})"
     return st

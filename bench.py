@@ -343,7 +343,8 @@ def run_ours(args, rank, world, local, dist):
         shared = int(args.variant == "auto" and args.kv_cache != "fp8" and
                      tables_share_blocks(case.steps[0].block_tables, case.steps[0].context_lens))
     fp8 = args.kv_cache == "fp8"
-    w = DeviceWorkload(case, torch, pa, args.partition_tokens, VARIANTS[args.variant], shared, fp8)
+    partition = args.partition_tokens or case.workload.partition_tokens
+    w = DeviceWorkload(case, torch, pa, partition, VARIANTS[args.variant], shared, fp8)
     kv_elem = 1 if fp8 else 2
     bytes_per = [decode_bytes(s.context_lens, case.num_q_heads, case.num_kv_heads, case.head_dim,
                               case.block_size, kv_elem=kv_elem) for s in case.steps]
@@ -400,7 +401,7 @@ def run_ours(args, rank, world, local, dist):
             "num_seqs": case.num_seqs, "num_q_heads": case.num_q_heads,
             "num_kv_heads": case.num_kv_heads, "head_dim": case.head_dim,
             "block_size": case.block_size, "storage_dtype": gen.DTYPE_NAMES[case.dtype],
-            "partition_tokens": args.partition_tokens or 512,
+            "partition_tokens": pa.pa_decode_partition_tokens(w.shape),
             "decode_variant": f"{args.variant} -> {resolved}",
             "shared_prefix": bool(shared),
             "kv_cache": "e4m3 codes + per-kv-head fp32 scales" if fp8 else gen.DTYPE_NAMES[case.dtype],

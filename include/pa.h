@@ -80,7 +80,8 @@ typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
  * Built values: head_dim in {64, 128}; num_q_heads / num_kv_heads in
  * {1, 2, 4, 8, 16}; block_size a multiple of 16 (16 and 256 are the measured
  * ones); num_blocks * block_size < 2^31; partition_tokens a multiple of 16 in
- * [16, 2048], or 0 for the default 512.
+ * [16, 2048], or 0 for the default: 512 for the tensor-core kernels and
+ * with shared_prefix (their largest item), 1024 for the CUDA-core kernel.
  */
 typedef struct {
   int32_t num_seqs;
@@ -125,6 +126,11 @@ typedef enum { PA_CACHE_AS_DTYPE = 0, PA_CACHE_FP8_E4M3 = 1 } pa_cache_format;
  *                          and partition_tokens a multiple of 128 (else
  *                          PA_ERR_UNSUPPORTED). */
 typedef enum { PA_DECODE_AUTO = 0, PA_DECODE_CUDA_CORES = 1, PA_DECODE_TENSOR_CORES = 2 } pa_decode_variant;
+
+/* The split-K partition pa_decode() uses for `shape` (partition_tokens, or
+ * its default when 0), or minus the status pa_decode() would refuse the
+ * shape with.  Host only. */
+int pa_decode_partition_tokens(const pa_shape *shape);
 
 /* The kernel pa_decode() runs for `shape`: PA_DECODE_CUDA_CORES or
  * PA_DECODE_TENSOR_CORES (PA_DECODE_AUTO resolved), or

@@ -53,8 +53,16 @@ void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Whether the tensor-core kernels run, with partition_tokens == 0 read as
+// "their default"; defined below.
+bool tensor_core_kernel(const pa_shape* s, int pt);
+
+// partition_tokens, or its default: 512 for the tensor-core kernels (their
+// largest item), 1024 for the CUDA-core kernel, where fewer partials measured
+// faster than 512 (llama2_7b 6025 vs 5697 GB/s, mistral_7b_gqa 4993 vs 4889).
 int effective_partition(const pa_shape* s) {
-  return s->partition_tokens == 0 ? 512 : s->partition_tokens;
+  if (s->partition_tokens != 0) return s->partition_tokens;
+  return (s->shared_prefix || tensor_core_kernel(s, 512)) ? 512 : 1024;
 }
 
 // Shape checks common to every call that touches the pool.
@@ -104,16 +112,17 @@ pa_status check_decode_shape(const pa_shape* s, int32_t max_context_len) {
 // Bytes of one cached element.
 int cache_elem_bytes(const pa_shape* s) { return s->cache_format == PA_CACHE_FP8_E4M3 ? 1 : 2; }
 
-bool use_tensor_cores(const pa_shape* s) {
+bool tensor_core_kernel(const pa_shape* s, int pt) {
   if (s->cache_format == PA_CACHE_FP8_E4M3) return false;
   if (s->variant == PA_DECODE_TENSOR_CORES) return true;
   if (s->variant == PA_DECODE_CUDA_CORES) return false;
-  const int pt = effective_partition(s);
   // measured: tensor cores win from group 8 up; at group 4 the CUDA-core
   // kernel still keeps up with HBM
   return s->head_dim == 128 && s->num_q_heads / s->num_kv_heads >= 8 &&
          pt % pa::decode_tc_tile_tokens() == 0 && pt <= 512;
 }
+
+bool use_tensor_cores(const pa_shape* s) { return tensor_core_kernel(s, effective_partition(s)); }
 
 // Workspace: the work counter (8 bytes used of 256); with shared_prefix the
 // plan, int4 [S] (rounded up to 256 bytes); then, for split-K, partial
@@ -451,6 +460,12 @@ pa_status pa_copy_blocks(const int32_t* src_dst_pairs, int32_t num_pairs, void* 
                                          reinterpret_cast<cudaStream_t>(stream), &launched);
   count_launches(launched);
   return e == cudaSuccess ? PA_OK : cuda_failed(e);
+}
+
+int pa_decode_partition_tokens(const pa_shape* shape) {
+  const pa_status st = check_decode_shape(shape, 0);
+  if (st != PA_OK) return -(int)st;
+  return effective_partition(shape);
 }
 
 int pa_decode_resolved_variant(const pa_shape* shape) {

@@ -57,6 +57,7 @@ class Workload:
     block_size: int
     dtype: int
     description: str
+    partition_tokens: int = 0   # split-K partition the workload states (0: the library's default)
 
 
 WORKLOADS = {
@@ -70,7 +71,7 @@ WORKLOADS = {
                  "shuffled pool 1.25x need, +1 token per seq per step"),
         Workload("mistral_7b_gqa", 3, 128, 32, 8, 128, 16, BF16,
                  "batch 128, 32/8 heads (group 4), D 128, bs 16, bf16, "
-                 "ctx U[1024,4096], shuffled pool 1.25x need, 512-token partitions"),
+                 "ctx U[1024,4096], shuffled pool 1.25x need, 512-token partitions", 512),
         Workload("qwen_7b_prefix", 4, 64, 32, 32, 128, 256, F16,
                  "batch 64, 32/32 heads, D 128, bs 256, fp16, all tables share 2 "
                  "prefix blocks (512 tokens) + private U[1,512] tokens"),
@@ -389,7 +390,7 @@ def make_case(name: str, n_steps: int = 1, poison: bool = True, seed: int | None
         if w.name == "llama2_70b_beam":
             assert num_seqs % 4 == 0
         w = Workload(w.name, w.number, num_seqs, w.num_q_heads, w.num_kv_heads,
-                     w.head_dim, w.block_size, w.dtype, w.description)
+                     w.head_dim, w.block_size, w.dtype, w.description, w.partition_tokens)
     seed = SEED_BASE + w.number if seed is None else int(seed)
     rs = _rng(seed, _STREAM_STRUCT)
     ctx0, info = _context_lengths(w, rs)

@@ -82,6 +82,8 @@ def _declare(lib):
     lib.pa_kernel_launches.argtypes = []
     lib.pa_build_info.restype = c.c_char_p
     lib.pa_build_info.argtypes = []
+    lib.pa_decode_partition_tokens.restype = c.c_int
+    lib.pa_decode_partition_tokens.argtypes = [SP]
     lib.pa_decode_resolved_variant.restype = c.c_int
     lib.pa_decode_resolved_variant.argtypes = [SP]
     lib.pa_last_cuda_error.restype = c.c_char_p
@@ -245,6 +247,13 @@ def pa_last_device_error(stream=None) -> tuple[int, int]:
 
 def pa_kernel_launches() -> int:
     return int(lib().pa_kernel_launches())
+
+
+def pa_decode_partition_tokens(shape: pa_shape) -> int:
+    v = lib().pa_decode_partition_tokens(ctypes.byref(shape))
+    if v < 0:
+        raise PaError("pa_decode_partition_tokens", -v)
+    return v
 
 
 def pa_decode_resolved_variant(shape: pa_shape) -> int:

@@ -115,6 +115,14 @@ def test_fp8_cache_validation(lib):
         lib.pa_decode_workspace_bytes(ctypes.byref(s16), 1000)
 
 
+def test_default_partition(lib):
+    assert pa.pa_decode_partition_tokens(_shape()) == 1024                     # CUDA cores
+    assert pa.pa_decode_partition_tokens(_shape(num_q_heads=16)) == 512        # tensor cores
+    assert pa.pa_decode_partition_tokens(_shape(shared_prefix=1)) == 512
+    assert pa.pa_decode_partition_tokens(_shape(partition_tokens=48)) == 48
+    assert pa.pa_decode_partition_tokens(_shape(num_q_heads=16, variant=1)) == 1024
+
+
 def test_resolved_variant(lib):
     assert pa.pa_decode_resolved_variant(_shape()) == pa.PA_DECODE_CUDA_CORES          # group 4
     assert pa.pa_decode_resolved_variant(_shape(num_q_heads=16)) == pa.PA_DECODE_TENSOR_CORES
@@ -137,18 +145,23 @@ def test_decode_rejects_bad_pointers_and_sizes(lib):
     assert call(scale=float("nan")) == pa.PA_ERR_INVALID_ARG
     assert call(maxlen=8 * 16 + 1) == pa.PA_ERR_INVALID_ARG     # beyond max_blocks_per_seq * bs
     assert call(maxlen=-1) == pa.PA_ERR_INVALID_ARG
-    # 100 tokens fit one 512-token partition: only the work counter ...
+    # 100 tokens fit one partition: only the work counter ...
     assert lib.pa_decode_workspace_bytes(ctypes.byref(s), 100) == 256
     st = lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s), 100, None, 0, None)
     assert st == pa.PA_ERR_INVALID_ARG
-    # ... 1000 tokens need two partitions and split-K space
-    s2 = _shape(max_blocks_per_seq=64)
-    need = lib.pa_decode_workspace_bytes(ctypes.byref(s2), 1000)
-    assert need >= 256 + 4 * 8 * 2 * (128 + 2) * 4
-    st = lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s2), 1000, FAKE, need - 1, None)
+    # ... 2000 tokens need two default (1024-token, CUDA-core) partitions and split-K space
+    s2 = _shape(max_blocks_per_seq=128)
+    assert lib.pa_decode_workspace_bytes(ctypes.byref(s2), 1024) == 256
+    need = lib.pa_decode_workspace_bytes(ctypes.byref(s2), 2000)
+    rows = 4 * 8 * 2
+    assert need == 256 + rows * 128 * 4 + rows * 2 * 4
+    st = lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s2), 2000, FAKE, need - 1, None)
     assert st == pa.PA_ERR_INVALID_ARG
-    st = lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s2), 1000, None, 0, None)
+    st = lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s2), 2000, None, 0, None)
     assert st == pa.PA_ERR_INVALID_ARG
+    # the tensor-core kernel's default partition is 512 tokens
+    s3 = _shape(num_q_heads=16, max_blocks_per_seq=128)
+    assert lib.pa_decode_workspace_bytes(ctypes.byref(s3), 1000) == 256 + 4 * 16 * 2 * 130 * 4
 
 
 def test_empty_batches_launch_nothing(lib):

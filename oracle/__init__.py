@@ -62,6 +62,8 @@ def _declare(lib):
     lib.oracle_cache_append.argtypes = [c.c_longlong, c.c_longlong, c.c_int, P, P, P, P, P]
     lib.oracle_copy_blocks.restype = c.c_int
     lib.oracle_copy_blocks.argtypes = [c.c_int, c.c_longlong, c.c_int, P, P, P]
+    lib.oracle_decode_multi.restype = c.c_int
+    lib.oracle_decode_multi.argtypes = [c.c_int] * 9 + [P, P, P, P, P, c.c_double, P, c.c_int]
     lib.oracle_e4m3_to_f64.restype = c.c_double
     lib.oracle_e4m3_to_f64.argtypes = [c.c_uint8]
     lib.oracle_e4m3_from_f32.restype = c.c_uint8
@@ -175,6 +177,23 @@ class Oracle:
                                          _ptr(v_cache))
         if rc:
             raise OracleError(f"oracle_copy_blocks refused its input (rc={rc})")
+
+    def decode_multi(self, dtype, q, k_cache, v_cache, block_tables, context_lens, scale,
+                     num_threads: int = 0) -> np.ndarray:
+        """fp64 [S][Tq][Hq][D]: Tq query tokens per sequence (q [S][Tq][Hq][D]),
+        query t attending to tokens 0 .. ctx - Tq + t."""
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        S, Tq, Hq, D = q.shape
+        arrs, dims = self._decode_args(dtype, q.reshape(S, Tq * Hq, D), k_cache, v_cache,
+                                       block_tables, context_lens)
+        _, _, _, Hkv, _, bs, NB, MBS = dims
+        out = np.empty((S, Tq, Hq, D), dtype=np.float64)
+        rc = self.lib.oracle_decode_multi(int(dtype), S, Tq, Hq, Hkv, D, bs, NB, MBS,
+                                          *(_ptr(a) for a in arrs), float(scale), _ptr(out),
+                                          int(num_threads))
+        if rc:
+            raise OracleError(f"oracle_decode_multi refused its input (rc={rc})")
+        return out
 
     # ---- FP8 (E4M3) cache
 

@@ -39,6 +39,15 @@
  *  - Copy-on-write: for each (src, dst) pair the whole block of K and of V is
  *    copied (zingnex.cn section 3.2 item 3).
  *
+ *  - Several query tokens per sequence (the scope table's multi-token
+ *    queries: speculative verification and chunked prefill under continuous
+ *    batching, 5688vip.com section 2.2): context_lens[s] counts the
+ *    sequence's Tq new tokens,
+ *    already appended, and query token t (0 <= t < Tq) attends causally to
+ *    tokens 0 .. ctx_s - Tq + t, i.e. to every cached token before the new
+ *    ones plus the new ones up to itself.  A query whose range is empty
+ *    (ctx_s - Tq + t < 0) gives a zero row.
+ *
  *  - FP8 cache (the pages name FP8 only as a quantisation format that saves
  *    memory: zingnex.cn sections 4.1 and 6, 5688vip.com section 2.3; the
  *    encoding below is the plain reading): K and V stored as OCP 8-bit E4M3
@@ -425,4 +434,48 @@ int oracle_cache_append_fp8(int dtype, long long num_slots, int Hkv, int D, int 
         }
     }
     return 0;
+}
+
+/* ---------------------------------------------------------------------
+ * Tq query tokens per sequence, causal over the new tokens.
+ * q: [S][Tq][Hq][D]; out: double [S][Tq][Hq][D]. */
+int oracle_decode_multi(int dtype, int S, int Tq, int Hq, int Hkv, int D, int bs, int NB,
+                        int MBS, const uint16_t *q, const uint16_t *k_cache,
+                        const uint16_t *v_cache, const int32_t *block_tables,
+                        const int32_t *context_lens, double scale, double *out, int num_threads)
+{
+    if (!shape_ok(dtype, S, Hq, Hkv, D, bs, NB, MBS) || Tq <= 0) return -1;
+    for (int s = 0; s < S; ++s)
+        if (context_lens[s] < 0 || (long long)context_lens[s] > (long long)MBS * bs) return -1;
+    int g = Hq / Hkv;
+    int err = 0;
+    int nt = resolve_threads(num_threads);
+    long long total = (long long)S * Tq * Hq;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nt) reduction(| : err)
+    for (long long row = 0; row < total; ++row) {
+        int h = (int)(row % Hq);
+        long long st = row / Hq;
+        int t = (int)(st % Tq), s = (int)(st / Tq);
+        int last = context_lens[s] - Tq + t;   /* last token this query sees */
+        double *o = out + row * D;
+        if (last < 0) {
+            for (int d = 0; d < D; ++d) o[d] = 0.0;
+            continue;
+        }
+        int L = last + 1;
+        double *x = (double *)malloc(sizeof(double) * (size_t)L);
+        double *acc = (double *)malloc(sizeof(double) * (size_t)D);
+        double m, l;
+        int kv_head = h / g;
+        int rc = attend_range(dtype, Hkv, D, bs, NB, MBS, q + row * D, k_cache, v_cache,
+                              block_tables, s, kv_head, 0, L, scale, x, &m, &l, acc);
+        if (rc) err |= 1;
+        else {
+            double inv = 1.0 / l;
+            for (int d = 0; d < D; ++d) o[d] = acc[d] * inv;
+        }
+        free(x);
+        free(acc);
+    }
+    return err ? -2 : 0;
 }

@@ -554,4 +554,55 @@ def pin_fp8_append_encodes_each_element(orc):
         assert np.array_equal(kc, ek) and np.array_equal(vc, ev), "FP8 append differs"
 
 
+# ---------------------------------------------------------------- several query tokens per sequence
+
+def _multi_case(seed, Tq, dtype=gen.BF16, ctx=(40, 5, 3, 70)):
+    rng = np.random.default_rng(seed)
+    c = _case(seed, num_seqs=len(ctx), num_q_heads=4, num_kv_heads=2, head_dim=32, block_size=16,
+              dtype=dtype, context_lens=list(ctx))
+    q = gen.normal_bits(rng, (len(ctx), Tq, 4, 32), dtype)
+    return c, q
+
+
+def pin_multi_one_token_is_decode(orc):
+    c, q = _multi_case(51, 1)
+    got = orc.decode_multi(gen.BF16, q, c["k_cache"], c["v_cache"], c["block_tables"],
+                           c["context_lens"], c["scale"])
+    ref = orc.decode(gen.BF16, q[:, 0], c["k_cache"], c["v_cache"], c["block_tables"],
+                     c["context_lens"], c["scale"])
+    assert np.max(np.abs(got[:, 0] - ref)) <= 1e-14
+
+
+def pin_multi_token_t_is_decode_over_its_prefix(orc):
+    """Query t of Tq equals a one-token decode whose context ends at its own token."""
+    Tq = 4
+    c, q = _multi_case(52, Tq)
+    got = orc.decode_multi(gen.BF16, q, c["k_cache"], c["v_cache"], c["block_tables"],
+                           c["context_lens"], c["scale"])
+    for t in range(Tq):
+        lens = np.maximum(c["context_lens"] - Tq + t + 1, 0).astype(np.int32)
+        ref = orc.decode(gen.BF16, q[:, t], c["k_cache"], c["v_cache"], c["block_tables"], lens,
+                         c["scale"])
+        assert np.max(np.abs(got[:, t] - ref)) <= 1e-14, f"query token {t}"
+    # a context shorter than Tq leaves the first queries without tokens: zero rows
+    assert np.all(got[2, 0] == 0) and np.any(got[2, 3] != 0)
+
+
+def pin_multi_is_causal(orc):
+    """Tokens after a query's own position never reach it (they are NaN here)."""
+    Tq = 3
+    c, q = _multi_case(53, Tq, ctx=(33, 20))
+    kc, vc = c["k_cache"].copy(), c["v_cache"].copy()
+    nan = np.uint16(gen.NAN_BITS[gen.BF16])
+    bs = 16
+    for s, L in enumerate(c["context_lens"]):
+        j = L - 1   # the last new token: only query Tq - 1 may see it
+        slot = int(c["block_tables"][s, j // bs]) * bs + j % bs
+        kc.reshape(-1, 2, 32)[slot] = nan
+        vc.reshape(-1, 2, 32)[slot] = nan
+    got = orc.decode_multi(gen.BF16, q, kc, vc, c["block_tables"], c["context_lens"], c["scale"])
+    assert np.all(np.isfinite(got[:, :Tq - 1])), "an earlier query read a later token"
+    assert np.all(np.isnan(got[:, Tq - 1])), "the last query must read every token"
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

@@ -62,6 +62,10 @@ MUTANTS = {
     "fp8_append_multiplies": ("oracle_e4m3_from_f32(xk / k_scale[h]);",
                               "oracle_e4m3_from_f32(xk * k_scale[h]);"),
     "fp8_append_head_index": ("int h = (int)(i / D);", "int h = (int)(i % Hkv);"),
+    "multi_sees_next_token": ("int last = context_lens[s] - Tq + t;", "int last = context_lens[s] - Tq + t + 1;"),
+    "multi_gqa_interleaved": ("int kv_head = h / g;", "int kv_head = h % Hkv;"),
+    "multi_query_index_dropped": ("int t = (int)(st % Tq), s = (int)(st / Tq);",
+                                  "int t = 0, s = (int)(st / Tq);"),
     "v_copy_skipped": (
         "memmove(v_cache + (long long)dst * block_bytes, v_cache + (long long)src * block_bytes,\n"
         "                (size_t)block_bytes);",

@@ -56,6 +56,9 @@ def parse_args(argv=None):
     p.add_argument("--partition-tokens", type=int, default=0)
     p.add_argument("--variant", default="auto", choices=sorted(VARIANTS),
                    help="decode kernel: auto, cuda_cores or tensor_cores")
+    p.add_argument("--query-tokens", type=int, default=1,
+                   help="query tokens per sequence (pa_decode_multi when > 1): the last ones "
+                        "of each context, causal among themselves")
     p.add_argument("--kv-cache", default="dtype", choices=["dtype", "fp8"],
                    help="K/V cache elements: the workload's 16-bit dtype, or E4M3 codes with "
                         "per-kv-head scales (halves the K/V bytes)")
@@ -118,13 +121,14 @@ def sum_over_ranks(x: float, dist, device=None) -> float:
 
 
 def decode_bytes(ctx: np.ndarray, num_q_heads, num_kv_heads, head_dim, block_size, elem=2,
-                 kv_elem=None) -> int:
+                 kv_elem=None, query_tokens=1) -> int:
     """Algorithmic bytes of one decode: K+V rows (kv_elem bytes per element,
-    default elem), q+out, table entries, lengths."""
+    default elem) once per sequence, q+out for each query token, table
+    entries, lengths."""
     ctx = np.asarray(ctx, dtype=np.int64)
     S = ctx.shape[0]
     kv = int(2 * ctx.sum() * num_kv_heads * head_dim * (elem if kv_elem is None else kv_elem))
-    qo = 2 * S * num_q_heads * head_dim * elem
+    qo = 2 * S * query_tokens * num_q_heads * head_dim * elem
     tables = int(4 * np.ceil(ctx / block_size).sum())
     return kv + qo + tables + 4 * S
 
@@ -247,7 +251,7 @@ class DeviceWorkload:
     """The pool and a cycle of precomputed steps, resident on the device."""
 
     def __init__(self, case, torch, pa, partition_tokens: int, variant: int = 0,
-                 shared_prefix: int = 0, fp8: bool = False):
+                 shared_prefix: int = 0, fp8: bool = False, query_tokens: int = 1):
         self.case = case
         self.torch, self.pa = torch, pa
         dt = pa.torch_dtype(case.dtype)
@@ -261,12 +265,16 @@ class DeviceWorkload:
 
         self.k_cache, self.v_cache = dev16(case.k_cache), dev16(case.v_cache)
         self.fp8 = fp8
+        self.tq = query_tokens
+        qrng = np.random.default_rng(case.seed + 77)
         self.steps = []
         for st in case.steps:
+            q = st.q if query_tokens == 1 else gen.normal_bits(
+                qrng, (case.num_seqs, query_tokens, case.num_q_heads, case.head_dim), case.dtype)
             self.steps.append(dict(
                 pairs=dev32(st.pairs.reshape(-1, 2)) if len(st.pairs) else None,
                 n_pairs=len(st.pairs), slots=dev32(st.slot_mapping), k_new=dev16(st.k_new),
-                v_new=dev16(st.v_new), q=dev16(st.q), tables=dev32(st.block_tables),
+                v_new=dev16(st.v_new), q=dev16(q), tables=dev32(st.block_tables),
                 lens=dev32(st.context_lens), max_len=int(st.context_lens.max())))
         self.max_len = max(s["max_len"] for s in self.steps)
         self.shape = pa.make_shape(
@@ -290,9 +298,12 @@ class DeviceWorkload:
                                    self.k_scale, self.v_scale, self.shape)
             torch.cuda.synchronize()
             del k16, v16
-        self.ws_bytes = pa.pa_decode_workspace_bytes(self.shape, self.max_len)
+        self.ws_bytes = (pa.pa_decode_workspace_bytes(self.shape, self.max_len) if self.tq == 1 else
+                         pa.pa_decode_multi_workspace_bytes(self.shape, self.tq, self.max_len))
         self.ws = torch.empty(max(16, self.ws_bytes), dtype=torch.uint8, device="cuda")
-        self.out = torch.empty((case.num_seqs, case.num_q_heads, case.head_dim), dtype=dt,
+        self.out = torch.empty((case.num_seqs, query_tokens, case.num_q_heads, case.head_dim)
+                               if query_tokens > 1 else
+                               (case.num_seqs, case.num_q_heads, case.head_dim), dtype=dt,
                                device="cuda")
 
     def step(self, i: int, stream, ev=None):
@@ -320,6 +331,10 @@ class DeviceWorkload:
             pa.pa_decode_fp8(st["q"], self.k_cache, self.v_cache, self.k_scale, self.v_scale,
                              st["tables"], st["lens"], self.case.scale, out, self.shape,
                              st["max_len"], self.ws, self.ws_bytes, stream.cuda_stream)
+        elif self.tq > 1:
+            pa.pa_decode_multi(st["q"], self.k_cache, self.v_cache, st["tables"], st["lens"],
+                               self.case.scale, out, self.shape, self.tq, st["max_len"], self.ws,
+                               self.ws_bytes, stream.cuda_stream)
         else:
             pa.pa_decode(st["q"], self.k_cache, self.v_cache, st["tables"], st["lens"],
                          self.case.scale, out, self.shape, st["max_len"], self.ws,
@@ -344,10 +359,14 @@ def run_ours(args, rank, world, local, dist):
                      tables_share_blocks(case.steps[0].block_tables, case.steps[0].context_lens))
     fp8 = args.kv_cache == "fp8"
     partition = args.partition_tokens or case.workload.partition_tokens
-    w = DeviceWorkload(case, torch, pa, partition, VARIANTS[args.variant], shared, fp8)
+    if args.query_tokens > 1 and fp8:
+        raise SystemExit("--query-tokens > 1 reads a 16-bit cache")
+    w = DeviceWorkload(case, torch, pa, partition, VARIANTS[args.variant], shared, fp8,
+                       args.query_tokens)
     kv_elem = 1 if fp8 else 2
     bytes_per = [decode_bytes(s.context_lens, case.num_q_heads, case.num_kv_heads, case.head_dim,
-                              case.block_size, kv_elem=kv_elem) for s in case.steps]
+                              case.block_size, kv_elem=kv_elem, query_tokens=args.query_tokens)
+                 for s in case.steps]
     pool_bytes = 2 * case.k_cache.nbytes * kv_elem // 2
     kv_step0 = 2 * int(case.steps[0].context_lens.sum()) * case.num_kv_heads * case.head_dim * kv_elem
 
@@ -389,7 +408,10 @@ def run_ours(args, rank, world, local, dist):
     achieved = step_bytes / (dec_total_ms * 1e-3) / 1e9
     resolved = {1: "cuda_cores", 2: "tensor_cores",
                 3: "shared_prefix"}[pa.pa_decode_resolved_variant(w.shape)]
-    traffic = (None if fp8 else profiled_traffic(args.workload, resolved, step_bytes / args.steps))
+    if args.query_tokens > 1:
+        resolved = "multi_query"
+    traffic = (None if fp8 or args.query_tokens > 1 else
+               profiled_traffic(args.workload, resolved, step_bytes / args.steps))
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -404,13 +426,15 @@ def run_ours(args, rank, world, local, dist):
             "partition_tokens": pa.pa_decode_partition_tokens(w.shape),
             "decode_variant": f"{args.variant} -> {resolved}",
             "shared_prefix": bool(shared),
+            "query_tokens": args.query_tokens,
             "kv_cache": "e4m3 codes + per-kv-head fp32 scales" if fp8 else gen.DTYPE_NAMES[case.dtype],
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "steps_cycle": n_cycle,
             "l2": (f"inputs larger than L2: {kv_step0 / 1e6:.0f} MB of K/V read per decode, "
                    f"{pool_bytes / 1e6:.0f} MB pool, L2 126 MB; no flush"),
         },
-        "tokens_per_s_per_layer": round(case.num_seqs * args.steps * world / (max_ms * 1e-3), 1),
+        "tokens_per_s_per_layer": round(case.num_seqs * args.query_tokens * args.steps * world /
+                                        (max_ms * 1e-3), 1),
         "decode_ms_per_step": round(dec_total_ms / args.steps, 5),
         "decode_bytes_per_step": int(step_bytes / args.steps),
         "pct_of_8tbps": round(100 * value / 8000.0, 2),
@@ -451,7 +475,7 @@ def run_e2e(args, w, stream, bytes_per, n_cycle, dist):
 
     case = w.case
     host = []
-    for st in case.steps:
+    for i, st in enumerate(case.steps):
         def pin16(a):
             return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(w.dt).pin_memory()
 
@@ -460,7 +484,8 @@ def run_e2e(args, w, stream, bytes_per, n_cycle, dist):
 
         host.append(dict(pairs=pin32(st.pairs.reshape(-1, 2)) if len(st.pairs) else None,
                          n_pairs=len(st.pairs), slots=pin32(st.slot_mapping), k_new=pin16(st.k_new),
-                         v_new=pin16(st.v_new), q=pin16(st.q), tables=pin32(st.block_tables),
+                         v_new=pin16(st.v_new), q=w.steps[i]["q"].cpu().pin_memory(),
+                         tables=pin32(st.block_tables),
                          lens=pin32(st.context_lens), max_len=int(st.context_lens.max())))
     outs = [w.out, torch.empty_like(w.out)]
     out_host = [torch.empty(w.out.shape, dtype=w.dt).pin_memory() for _ in range(2)]

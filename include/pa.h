@@ -203,6 +203,33 @@ pa_status pa_decode(const void *q, const void *k_cache, const void *v_cache,
                     void *workspace, size_t workspace_bytes, pa_stream_t stream);
 
 /*
+ * Several query tokens per sequence (the scope table's multi-token queries:
+ * verifying speculated tokens, chunked prefill under continuous batching,
+ * 5688vip.com section 2.2).  q, out: [num_seqs][num_query_tokens][Hq][D]
+ * (shape->num_seqs real sequences).  context_lens[s] counts the sequence's
+ * num_query_tokens (Tq) new tokens, whose K/V are already appended; query
+ * token t attends causally to tokens 0 .. ctx_s - Tq + t.  A query whose
+ * range is empty (ctx_s < Tq - t) gives a zero row.
+ *
+ * Query t of s is a one-token decode of a virtual sequence with the same
+ * block table and context ctx_s - Tq + t + 1.  A first kernel writes the
+ * virtual tables and contexts into the workspace.  The virtual sequences of
+ * one sequence are consecutive and start with the same blocks, so when the
+ * shape allows the shared-prefix kernel (head_dim 128, variant
+ * PA_DECODE_AUTO, a 16-bit cache, partition_tokens 0 or a multiple of 128
+ * up to 512), the tokens they have in common are read once for all of them.
+ * Otherwise each is decoded on its own.  Tq == 1 is pa_decode.
+ * workspace: pa_decode_multi_workspace_bytes(shape, Tq, max_context_len).
+ */
+size_t pa_decode_multi_workspace_bytes(const pa_shape *shape, int32_t num_query_tokens,
+                                       int32_t max_context_len);
+pa_status pa_decode_multi(const void *q, const void *k_cache, const void *v_cache,
+                          const int32_t *block_tables, const int32_t *context_lens, float scale,
+                          void *out, const pa_shape *shape, int32_t num_query_tokens,
+                          int32_t max_context_len, void *workspace, size_t workspace_bytes,
+                          pa_stream_t stream);
+
+/*
  * pa_decode for callers that cannot allocate device memory.
  *
  * The paper has no counterpart to this call (it is not part of the method);

@@ -380,6 +380,89 @@ pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
                      shape, max_context_len, workspace, workspace_bytes, stream);
 }
 
+}  // extern "C"
+
+namespace {
+
+// The one-token batch pa_decode_multi runs: S * Tq virtual sequences, grouped
+// by shared prefix whenever the shape allows the shared-prefix kernel.
+pa_shape multi_shape(const pa_shape* s, int num_query_tokens) {
+  pa_shape e = *s;
+  e.num_seqs = s->num_seqs * num_query_tokens;
+  const int pt = s->partition_tokens;
+  e.shared_prefix = s->head_dim == 128 && s->variant == PA_DECODE_AUTO &&
+                    s->cache_format == PA_CACHE_AS_DTYPE &&
+                    (pt == 0 || (pt % pa::decode_tc_tile_tokens() == 0 && pt <= 512));
+  return e;
+}
+
+// Virtual block tables [S * Tq][MBS] and contexts [S * Tq], each 256-aligned.
+long long multi_tables_bytes(const pa_shape* s, int num_query_tokens) {
+  return round256(4LL * s->num_seqs * num_query_tokens * s->max_blocks_per_seq);
+}
+long long multi_head_bytes(const pa_shape* s, int num_query_tokens) {
+  return multi_tables_bytes(s, num_query_tokens) + round256(4LL * s->num_seqs * num_query_tokens);
+}
+
+bool multi_args_ok(const pa_shape* s, int num_query_tokens) {
+  return s && num_query_tokens >= 1 && s->num_seqs >= 0 &&
+         (long long)s->num_seqs * num_query_tokens <= (1LL << 30);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t pa_decode_multi_workspace_bytes(const pa_shape* shape, int32_t num_query_tokens,
+                                       int32_t max_context_len) {
+  if (!multi_args_ok(shape, num_query_tokens)) return 0;
+  if (num_query_tokens == 1) return pa_decode_workspace_bytes(shape, max_context_len);
+  const pa_shape e = multi_shape(shape, num_query_tokens);
+  const size_t inner = pa_decode_workspace_bytes(&e, max_context_len);
+  if (inner == 0) return 0;
+  return (size_t)multi_head_bytes(shape, num_query_tokens) + inner;
+}
+
+pa_status pa_decode_multi(const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* block_tables, const int32_t* context_lens, float scale,
+                          void* out, const pa_shape* shape, int32_t num_query_tokens,
+                          int32_t max_context_len, void* workspace, size_t workspace_bytes,
+                          pa_stream_t stream) {
+  if (!multi_args_ok(shape, num_query_tokens)) return PA_ERR_INVALID_ARG;
+  if (num_query_tokens == 1)
+    return pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, shape,
+                     max_context_len, workspace, workspace_bytes, stream);
+  pa_status st = check_decode_shape(shape, max_context_len);
+  if (st != PA_OK) return st;
+  if (shape->cache_format != PA_CACHE_AS_DTYPE) return PA_ERR_INVALID_ARG;
+  const pa_shape e = multi_shape(shape, num_query_tokens);
+  st = check_decode_shape(&e, max_context_len);
+  if (st != PA_OK) return st;
+  if (shape->num_seqs == 0) return PA_OK;
+  if (!block_tables || !context_lens || (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+      (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+    return PA_ERR_INVALID_ARG;
+  const size_t need = pa_decode_multi_workspace_bytes(shape, num_query_tokens, max_context_len);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_INVALID_ARG;
+  if (max_context_len > (long long)shape->max_blocks_per_seq * shape->block_size)
+    return PA_ERR_INVALID_ARG;
+  unsigned int* err = error_word();
+  if (!err) return cuda_failed("device error word lookup failed");
+  char* ws = static_cast<char*>(workspace);
+  int32_t* tables_v = reinterpret_cast<int32_t*>(ws);
+  int32_t* ctx_v = reinterpret_cast<int32_t*>(ws + multi_tables_bytes(shape, num_query_tokens));
+  const long long head = multi_head_bytes(shape, num_query_tokens);
+  int launched = 0;
+  cudaError_t ce = pa::launch_expand_queries(block_tables, context_lens, shape->num_seqs,
+                                             num_query_tokens, shape->max_blocks_per_seq,
+                                             shape->block_size, max_context_len, tables_v, ctx_v,
+                                             err, reinterpret_cast<cudaStream_t>(stream), &launched);
+  count_launches(launched);
+  if (ce != cudaSuccess) return cuda_failed(ce);
+  return decode_impl(q, k_cache, v_cache, nullptr, nullptr, tables_v, ctx_v, scale, out, &e,
+                     max_context_len, ws + head, workspace_bytes - (size_t)head, stream);
+}
+
 pa_status pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache,
                         const float* k_scale, const float* v_scale, const int32_t* block_tables,
                         const int32_t* context_lens, float scale, void* out, const pa_shape* shape,

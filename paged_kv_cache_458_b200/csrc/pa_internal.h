@@ -51,6 +51,11 @@ struct PlanArgs {
   int chunk;                     // groups stay inside [k * chunk, (k + 1) * chunk)
 };
 cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream, int* launches);
+// Virtual one-token sequences for Tq query tokens per sequence (pa_plan.cu).
+cudaError_t launch_expand_queries(const int32_t* tables, const int32_t* ctx, int num_seqs,
+                                  int num_query_tokens, int max_blocks_per_seq, int block_size,
+                                  int max_context_len, int32_t* tables_out, int32_t* ctx_out,
+                                  unsigned int* err, cudaStream_t stream, int* launches);
 
 // Tokens [T, ctx) of sequence s with a plan: its first own token, the
 // workspace slot of its first own partition (of own_tokens tokens each), and

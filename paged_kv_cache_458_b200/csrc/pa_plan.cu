@@ -134,3 +134,54 @@ cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream, int* launches) {
 }
 
 }  // namespace pa
+
+// ---------------------------------------------------------------------------
+// Several query tokens per sequence.  Query token t of sequence s attends to
+// tokens 0 .. ctx_s - Tq + t, so it is a one-token decode of a "virtual"
+// sequence v = s * Tq + t with the same block table and context
+// ctx_s - Tq + t + 1: the Tq virtual sequences of s are consecutive and start
+// with the same blocks, so the shared-prefix plan groups them and their
+// common tokens are read once.  This kernel writes the virtual tables and
+// contexts (one CTA per virtual sequence; only the entries a context uses).
+
+namespace pa {
+namespace {
+
+__global__ void __launch_bounds__(128)
+expand_queries_kernel(const int32_t* __restrict__ tables, const int32_t* __restrict__ ctx,
+                      int num_query_tokens, int max_blocks_per_seq, int block_size,
+                      int max_context_len, int32_t* __restrict__ tables_out,
+                      int32_t* __restrict__ ctx_out, unsigned int* err) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int v = blockIdx.x;
+  const int s = v / num_query_tokens, t = v % num_query_tokens;
+  int c = __ldg(ctx + s);
+  if (c < 0 || c > max_context_len) {
+    if (t == 0 && threadIdx.x == 0) report(err, kErrContextLen);
+    c = max(0, min(c, max_context_len));
+  }
+  const int cv = max(0, c - num_query_tokens + t + 1);
+  const int nb = (cv + block_size - 1) / block_size;
+  const int32_t* src = tables + (size_t)s * max_blocks_per_seq;
+  int32_t* dst = tables_out + (size_t)v * max_blocks_per_seq;
+  for (int j = threadIdx.x; j < nb; j += blockDim.x) dst[j] = __ldg(src + j);
+  if (threadIdx.x == 0) ctx_out[v] = cv;
+}
+
+}  // namespace
+
+cudaError_t launch_expand_queries(const int32_t* tables, const int32_t* ctx, int num_seqs,
+                                  int num_query_tokens, int max_blocks_per_seq, int block_size,
+                                  int max_context_len, int32_t* tables_out, int32_t* ctx_out,
+                                  unsigned int* err, cudaStream_t stream, int* launches) {
+  const long long n = (long long)num_seqs * num_query_tokens;
+  if (n <= 0) return cudaSuccess;
+  cudaError_t e = launch_pdl(expand_queries_kernel, dim3((unsigned)n), dim3(128), 0, stream, tables,
+                             ctx, num_query_tokens, max_blocks_per_seq, block_size,
+                             max_context_len, tables_out, ctx_out, err);
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
+}  // namespace pa

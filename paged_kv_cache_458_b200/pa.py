@@ -82,6 +82,10 @@ def _declare(lib):
     lib.pa_kernel_launches.argtypes = []
     lib.pa_build_info.restype = c.c_char_p
     lib.pa_build_info.argtypes = []
+    lib.pa_decode_multi_workspace_bytes.restype = SZ
+    lib.pa_decode_multi_workspace_bytes.argtypes = [SP, I32, I32]
+    lib.pa_decode_multi.restype = c.c_int
+    lib.pa_decode_multi.argtypes = [P, P, P, P, P, c.c_float, P, SP, I32, I32, P, SZ, P]
     lib.pa_decode_partition_tokens.restype = c.c_int
     lib.pa_decode_partition_tokens.argtypes = [SP]
     lib.pa_decode_resolved_variant.restype = c.c_int
@@ -192,6 +196,24 @@ def pa_decode(q, k_cache, v_cache, block_tables, context_lens, scale: float, out
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
         float(scale), _ptr(out), ctypes.byref(shape), int(max_context_len), _ptr(workspace),
         int(workspace_bytes), _stream(stream)))
+
+
+def pa_decode_multi_workspace_bytes(shape: pa_shape, num_query_tokens: int,
+                                    max_context_len: int) -> int:
+    return int(lib().pa_decode_multi_workspace_bytes(ctypes.byref(shape), int(num_query_tokens),
+                                                     int(max_context_len)))
+
+
+def pa_decode_multi(q, k_cache, v_cache, block_tables, context_lens, scale: float, out,
+                    shape: pa_shape, num_query_tokens: int, max_context_len: int, workspace=None,
+                    workspace_bytes: int | None = None, stream=None) -> None:
+    """Tq query tokens per sequence, causal over the new tokens (see pa.h)."""
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("pa_decode_multi", lib().pa_decode_multi(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+        float(scale), _ptr(out), ctypes.byref(shape), int(num_query_tokens), int(max_context_len),
+        _ptr(workspace), int(workspace_bytes), _stream(stream)))
 
 
 def pa_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale: float, out,

@@ -115,6 +115,28 @@ def test_fp8_cache_validation(lib):
         lib.pa_decode_workspace_bytes(ctypes.byref(s16), 1000)
 
 
+def test_multi_query_workspace_and_validation(lib):
+    s = _shape(max_blocks_per_seq=64)
+    one = lib.pa_decode_workspace_bytes(ctypes.byref(s), 700)
+    assert lib.pa_decode_multi_workspace_bytes(ctypes.byref(s), 1, 700) == one
+    assert lib.pa_decode_multi_workspace_bytes(ctypes.byref(s), 0, 700) == 0
+    w4 = lib.pa_decode_multi_workspace_bytes(ctypes.byref(s), 4, 700)
+    # virtual tables and contexts, then a shared-prefix decode of 16 virtual sequences
+    # (16 * 8 heads * (2 + 1) partitions of (128 + 2) floats, plan 256 bytes, counter 256)
+    rows = 16 * 8 * 3
+    assert w4 == 4 * 16 * 64 + 256 + 256 + 256 + rows * 128 * 4 + rows * 8
+    st = lib.pa_decode_multi(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s), 0, 700, FAKE,
+                             1 << 24, None)
+    assert st == pa.PA_ERR_INVALID_ARG
+    st = lib.pa_decode_multi(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s), 4, 700, FAKE,
+                             w4 - 1, None)
+    assert st == pa.PA_ERR_INVALID_ARG
+    s8 = _shape(max_blocks_per_seq=64, cache_format=pa.PA_CACHE_FP8_E4M3)
+    st = lib.pa_decode_multi(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s8), 4, 700,
+                             FAKE, 1 << 24, None)
+    assert st == pa.PA_ERR_INVALID_ARG
+
+
 def test_default_partition(lib):
     assert pa.pa_decode_partition_tokens(_shape()) == 1024                     # CUDA cores
     assert pa.pa_decode_partition_tokens(_shape(num_q_heads=16)) == 512        # tensor cores

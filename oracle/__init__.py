@@ -62,6 +62,8 @@ def _declare(lib):
     lib.oracle_cache_append.argtypes = [c.c_longlong, c.c_longlong, c.c_int, P, P, P, P, P]
     lib.oracle_copy_blocks.restype = c.c_int
     lib.oracle_copy_blocks.argtypes = [c.c_int, c.c_longlong, c.c_int, P, P, P]
+    lib.oracle_swap_blocks.restype = c.c_int
+    lib.oracle_swap_blocks.argtypes = [c.c_int, c.c_int, c.c_longlong, c.c_int, P, P, P, P, P]
     lib.oracle_decode_multi.restype = c.c_int
     lib.oracle_decode_multi.argtypes = [c.c_int] * 9 + [P, P, P, P, P, c.c_double, P, c.c_int]
     lib.oracle_e4m3_to_f64.restype = c.c_double
@@ -177,6 +179,20 @@ class Oracle:
                                          _ptr(v_cache))
         if rc:
             raise OracleError(f"oracle_copy_blocks refused its input (rc={rc})")
+
+    def swap_blocks(self, pairs, src_k, src_v, dst_k, dst_v) -> None:
+        """In place on ``dst_k``/``dst_v``: dst block p[1] = src block p[0] per pair."""
+        for a in (dst_k, dst_v):
+            assert a.flags["C_CONTIGUOUS"]
+        src_k = np.ascontiguousarray(src_k)
+        src_v = np.ascontiguousarray(src_v)
+        pr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
+        bb = src_k.nbytes // src_k.shape[0] if src_k.shape[0] else 1
+        assert dst_k.nbytes // max(1, dst_k.shape[0]) == bb
+        rc = self.lib.oracle_swap_blocks(src_k.shape[0], dst_k.shape[0], bb, pr.shape[0], _ptr(pr),
+                                         _ptr(src_k), _ptr(src_v), _ptr(dst_k), _ptr(dst_v))
+        if rc:
+            raise OracleError(f"oracle_swap_blocks refused its input (rc={rc})")
 
     def decode_multi(self, dtype, q, k_cache, v_cache, block_tables, context_lens, scale,
                      num_threads: int = 0) -> np.ndarray:

@@ -39,6 +39,11 @@
  *  - Copy-on-write: for each (src, dst) pair the whole block of K and of V is
  *    copied (zingnex.cn section 3.2 item 3).
  *
+ *  - Swap: whole blocks copied between two pools, for instance a device
+ *    pool and a pool in host memory (zingnex.cn section 5, tuning advice:
+ *    CPU offload through swap space): block src of the source pools
+ *    becomes block dst of the destination pools.
+ *
  *  - Several query tokens per sequence (the scope table's multi-token
  *    queries: speculative verification and chunked prefill under continuous
  *    batching, 5688vip.com section 2.2): context_lens[s] counts the
@@ -478,4 +483,23 @@ int oracle_decode_multi(int dtype, int S, int Tq, int Hq, int Hkv, int D, int bs
         free(acc);
     }
     return err ? -2 : 0;
+}
+
+/* Swap: for each pair, dst block pairs[2i+1] of (dst_k, dst_v) becomes a copy
+ * of src block pairs[2i] of (src_k, src_v).  The pools are distinct; blocks
+ * hold block_bytes bytes. */
+int oracle_swap_blocks(int src_blocks, int dst_blocks, long long block_bytes, int num_pairs,
+                       const int32_t *pairs, const uint8_t *src_k, const uint8_t *src_v,
+                       uint8_t *dst_k, uint8_t *dst_v)
+{
+    if (src_blocks < 0 || dst_blocks < 0 || block_bytes <= 0 || num_pairs < 0) return -1;
+    for (int i = 0; i < num_pairs; ++i) {
+        int from = pairs[2 * i], to = pairs[2 * i + 1];
+        if (from < 0 || from >= src_blocks || to < 0 || to >= dst_blocks) return -2;
+        memcpy(dst_k + (long long)to * block_bytes, src_k + (long long)from * block_bytes,
+               (size_t)block_bytes);
+        memcpy(dst_v + (long long)to * block_bytes, src_v + (long long)from * block_bytes,
+               (size_t)block_bytes);
+    }
+    return 0;
 }

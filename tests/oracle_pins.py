@@ -18,7 +18,9 @@ the oracle disagrees with what the pages or the mathematics fix:
   private copies;
 * grouped queries equal full multi-head attention with repeated kv heads;
 * the partitioned (split-K) form equals the direct one;
-* append and copy-on-write equal a NumPy scatter/copy over the whole pool;
+* append and copy-on-write equal a NumPy scatter/copy over the whole pool, and
+  a swap between two pools equals a block copy; a pool of 16-token blocks
+  read as twice as many 8-token blocks gives the same output;
 * the E4M3 cache: every code widens as PyTorch's float8_e4m3fn does, the
   encoder rounds as PyTorch's fp32 conversion below the saturation point,
   codes round-trip, ties go to the even code, large values saturate at 448;
@@ -603,6 +605,44 @@ def pin_multi_is_causal(orc):
     got = orc.decode_multi(gen.BF16, q, kc, vc, c["block_tables"], c["context_lens"], c["scale"])
     assert np.all(np.isfinite(got[:, :Tq - 1])), "an earlier query read a later token"
     assert np.all(np.isnan(got[:, Tq - 1])), "the last query must read every token"
+
+# ---------------------------------------------------------------- block size 8, swap
+
+def pin_block_size_8_equals_16(orc):
+    """A pool of 16-token blocks read as twice as many 8-token blocks gives the same output."""
+    c = _case(61, num_seqs=4, num_q_heads=4, num_kv_heads=2, head_dim=32, block_size=16,
+              dtype=gen.F16, context_lens=[1, 9, 24, 47])
+    NB = c["num_blocks"]
+    k8 = c["k_cache"].reshape(NB * 2, 8, 2, 32)
+    v8 = c["v_cache"].reshape(NB * 2, 8, 2, 32)
+    t16 = c["block_tables"]
+    t8 = np.empty((t16.shape[0], 2 * t16.shape[1]), dtype=np.int32)
+    t8[:, 0::2] = np.where(t16 >= 0, 2 * t16, -1)
+    t8[:, 1::2] = np.where(t16 >= 0, 2 * t16 + 1, -1)
+    a = _decode(orc, gen.F16, c)
+    b = orc.decode(gen.F16, c["q"], k8, v8, t8, c["context_lens"], c["scale"])
+    assert np.array_equal(a, b), "8-token blocks must read the same tokens"
+
+
+def pin_swap_matches_block_copy(orc):
+    rng = np.random.default_rng(62)
+    bs, Hkv, D = 16, 2, 32
+    dev_k = rng.integers(0, 1 << 16, size=(10, bs, Hkv, D), dtype=np.uint16)
+    dev_v = rng.integers(0, 1 << 16, size=(10, bs, Hkv, D), dtype=np.uint16)
+    host_k = rng.integers(0, 1 << 16, size=(6, bs, Hkv, D), dtype=np.uint16)
+    host_v = rng.integers(0, 1 << 16, size=(6, bs, Hkv, D), dtype=np.uint16)
+    pairs = np.array([[7, 0], [2, 5], [9, 3]], dtype=np.int32)
+    ek, ev = host_k.copy(), host_v.copy()
+    for s, d in pairs:
+        ek[d], ev[d] = dev_k[s], dev_v[s]
+    orc.swap_blocks(pairs, dev_k, dev_v, host_k, host_v)
+    assert np.array_equal(host_k, ek) and np.array_equal(host_v, ev), "swap differs from a block copy"
+    try:
+        orc.swap_blocks(np.array([[10, 0]], np.int32), dev_k, dev_v, host_k, host_v)
+    except Exception:
+        pass
+    else:
+        raise AssertionError("a source block outside the pool must be refused")
 
 
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

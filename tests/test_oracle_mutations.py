@@ -66,6 +66,8 @@ MUTANTS = {
     "multi_gqa_interleaved": ("int kv_head = h / g;", "int kv_head = h % Hkv;"),
     "multi_query_index_dropped": ("int t = (int)(st % Tq), s = (int)(st / Tq);",
                                   "int t = 0, s = (int)(st / Tq);"),
+    "swap_direction": ("memcpy(dst_k + (long long)to * block_bytes, src_k + (long long)from * block_bytes,",
+                       "memcpy(dst_k + (long long)from * block_bytes, src_k + (long long)to * block_bytes,"),
     "v_copy_skipped": (
         "memmove(v_cache + (long long)dst * block_bytes, v_cache + (long long)src * block_bytes,\n"
         "                (size_t)block_bytes);",

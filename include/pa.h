@@ -78,8 +78,10 @@ typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
  * heads are contiguous.
  *
  * Built values: head_dim in {64, 128}; num_q_heads / num_kv_heads in
- * {1, 2, 4, 8, 16}; block_size a multiple of 16 (16 and 256 are the measured
- * ones); num_blocks * block_size < 2^31; partition_tokens a multiple of 16 in
+ * {1, 2, 4, 8, 16}; block_size a multiple of 8 (8, 16 and 256 are the measured
+ * ones; with a multiple of 8 that is not one of 16, every 16-token TMA box is
+ * loaded as two 8-token boxes, zingnex.cn section 5: block_size 8 for short
+ * sequences); num_blocks * block_size < 2^31; partition_tokens a multiple of 16 in
  * [16, 2048], or 0 for the default: 512 for the tensor-core kernels and
  * with shared_prefix (their largest item), 1024 for the CUDA-core kernel.
  */
@@ -321,6 +323,26 @@ pa_status pa_decode_fp8(const void *q, const void *k_cache, const void *v_cache,
  */
 pa_status pa_copy_blocks(const int32_t *src_dst_pairs, int32_t num_pairs, void *k_cache,
                          void *v_cache, const pa_shape *shape, pa_stream_t stream);
+
+/*
+ * Swap whole blocks between two pools (zingnex.cn section 5, tuning advice:
+ * CPU offload through swap space): for each pair i, block src_dst_pairs[2i+1]
+ * of (dst_k, dst_v) becomes a byte copy of block src_dst_pairs[2i] of
+ * (src_k, src_v).  Either pool may be host memory the device can address
+ * (pinned and mapped, e.g. cudaHostAlloc'd under unified addressing), so
+ * swapping a preempted sequence out to the host and back in is two calls.
+ * Pageable host memory, or pinned memory the device cannot address at the
+ * same pointer, is refused (PA_ERR_INVALID_ARG, checked with
+ * cudaPointerGetAttributes before any launch).
+ * The two pools of each tensor must not overlap (else PA_ERR_INVALID_ARG);
+ * src_num_blocks / dst_num_blocks size them; an entry outside either is
+ * reported (PA_DEVERR_PAIR) and skipped.  shape gives the block geometry
+ * and cache format (shape->num_blocks is not used).
+ * src_dst_pairs: device int32 [num_pairs][2].  num_pairs == 0 launches nothing.
+ */
+pa_status pa_swap_blocks(const int32_t *src_dst_pairs, int32_t num_pairs, const void *src_k,
+                         const void *src_v, int32_t src_num_blocks, void *dst_k, void *dst_v,
+                         int32_t dst_num_blocks, const pa_shape *shape, pa_stream_t stream);
 
 /* Synchronises `stream`, then reads and clears this device's error word.
  * Returns PA_OK when it was zero, PA_ERR_DEVICE_CHECK otherwise (bits in

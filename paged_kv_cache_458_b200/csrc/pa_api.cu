@@ -74,7 +74,7 @@ pa_status check_pool_shape(const pa_shape* s) {
   if (s->cache_format != PA_CACHE_AS_DTYPE && s->cache_format != PA_CACHE_FP8_E4M3)
     return PA_ERR_UNSUPPORTED;
   if (s->head_dim != 64 && s->head_dim != 128) return PA_ERR_UNSUPPORTED;
-  if (s->block_size % 16 != 0) return PA_ERR_UNSUPPORTED;
+  if (s->block_size % 8 != 0) return PA_ERR_UNSUPPORTED;
   if ((long long)s->num_blocks * s->block_size >= (1LL << 31)) return PA_ERR_UNSUPPORTED;
   return PA_OK;
 }
@@ -201,13 +201,17 @@ bool make_pool_map(CUtensorMap* map, const void* pool, const pa_shape* s, int ro
 // Maps of the tensor-core variant: pools viewed as [NB * bs][Hkv][128] with
 // 128B-swizzled boxes of 64 elements x 16 token rows; q viewed as
 // [S * Hq][128] with 128B-swizzled boxes of 64 elements x `group` rows.
+// TMA box rows over the pool: 16 (one box per 16-token group), or 8 when
+// blocks hold a multiple of 8 but not of 16 tokens (two boxes per group).
+int box_rows(const pa_shape* s) { return s->block_size % 16 == 0 ? 16 : 8; }
+
 bool make_tc_maps(CUtensorMap* tk, CUtensorMap* tv, CUtensorMap* tq, const void* k, const void* v,
                   const void* q, const pa_shape* s) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {128, (cuuint64_t)s->num_kv_heads, (cuuint64_t)s->num_blocks * s->block_size};
   const cuuint64_t strides[2] = {256, (cuuint64_t)s->num_kv_heads * 256};
-  const cuuint32_t box[3] = {64, 1, 16};
+  const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows(s)};
   const cuuint32_t estr[3] = {1, 1, 1};
   for (int i = 0; i < 2; ++i) {
     CUresult r = fn(i ? tv : tk, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(i ? v : k), dims,
@@ -307,6 +311,7 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
     const int gp = (max_context_len + a.own_tokens - 1) / a.own_tokens;
     a.grid_parts = gp > 0 ? gp : 1;
   }
+  a.half_boxes = box_rows(shape) == 8;
   a.max_context_len = max_context_len;
   a.err = error_word();
   if (!a.err) return cuda_failed("device error word lookup failed");
@@ -321,8 +326,8 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
     // sequence's own tokens on CUDA cores, then the merge
     CUtensorMap tk, tv, tq, pk, pv;
     if (!make_tc_maps(&tk, &tv, &tq, k_cache, v_cache, q, shape) ||
-        !make_pool_map(&pk, k_cache, shape, pa::decode_chunk_tokens()) ||
-        !make_pool_map(&pv, v_cache, shape, pa::decode_chunk_tokens()))
+        !make_pool_map(&pk, k_cache, shape, box_rows(shape)) ||
+        !make_pool_map(&pv, v_cache, shape, box_rows(shape)))
       return cuda_failed("cuTensorMapEncodeTiled failed");
     pa::PlanArgs pl{};
     pl.block_tables = block_tables;
@@ -354,8 +359,8 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
   } else {
     CUtensorMap tk, tv;
     if (shape->num_blocks > 0) {
-      if (!make_pool_map(&tk, k_cache, shape, pa::decode_chunk_tokens()) ||
-          !make_pool_map(&tv, v_cache, shape, pa::decode_chunk_tokens()))
+      if (!make_pool_map(&tk, k_cache, shape, box_rows(shape)) ||
+          !make_pool_map(&tv, v_cache, shape, box_rows(shape)))
         return cuda_failed("cuTensorMapEncodeTiled failed");
     } else {
       // An empty pool can only serve empty contexts; the kernels issue no load.
@@ -539,7 +544,52 @@ pa_status pa_copy_blocks(const int32_t* src_dst_pairs, int32_t num_pairs, void* 
   if (!err) return cuda_failed("device error word lookup failed");
   int launched = 0;
   cudaError_t e = pa::launch_copy_blocks(src_dst_pairs, num_pairs, k_cache, v_cache,
-                                         shape->num_blocks, block_bytes, err,
+                                         shape->num_blocks, k_cache, v_cache, shape->num_blocks,
+                                         block_bytes, err, reinterpret_cast<cudaStream_t>(stream),
+                                         &launched);
+  count_launches(launched);
+  return e == cudaSuccess ? PA_OK : cuda_failed(e);
+}
+
+pa_status pa_swap_blocks(const int32_t* src_dst_pairs, int32_t num_pairs, const void* src_k,
+                         const void* src_v, int32_t src_num_blocks, void* dst_k, void* dst_v,
+                         int32_t dst_num_blocks, const pa_shape* shape, pa_stream_t stream) {
+  pa_status st = check_pool_shape(shape);
+  if (st != PA_OK) return st;
+  if (num_pairs < 0 || src_num_blocks < 0 || dst_num_blocks < 0) return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PA_OK;
+  if (num_pairs > 65535) return PA_ERR_UNSUPPORTED;
+  if (!src_dst_pairs || !src_k || !src_v || !dst_k || !dst_v) return PA_ERR_INVALID_ARG;
+  if (!aligned16(src_k) || !aligned16(src_v) || !aligned16(dst_k) || !aligned16(dst_v) ||
+      (reinterpret_cast<uintptr_t>(src_dst_pairs) & 3u))
+    return PA_ERR_INVALID_ARG;
+  // the pools must not overlap: a swap moves blocks between two pools
+  const long long block_bytes = (long long)shape->block_size * shape->num_kv_heads *
+                                shape->head_dim * cache_elem_bytes(shape);
+  auto disjoint = [&](const void* a, long long na, const void* b, long long nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x + (uintptr_t)(na * block_bytes) <= y || y + (uintptr_t)(nb * block_bytes) <= x;
+  };
+  if (!disjoint(src_k, src_num_blocks, dst_k, dst_num_blocks) ||
+      !disjoint(src_v, src_num_blocks, dst_v, dst_num_blocks))
+    return PA_ERR_INVALID_ARG;
+  // every pool must be memory the device can address at the same pointer:
+  // device memory, managed memory, or pinned host memory mapped under
+  // unified addressing (never pageable host memory)
+  for (const void* p : {src_k, src_v, static_cast<const void*>(dst_k), static_cast<const void*>(dst_v)}) {
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+      cudaGetLastError();
+      return PA_ERR_INVALID_ARG;
+    }
+    if (attr.type == cudaMemoryTypeUnregistered) return PA_ERR_INVALID_ARG;
+    if (attr.type == cudaMemoryTypeHost && attr.devicePointer != p) return PA_ERR_INVALID_ARG;
+  }
+  unsigned int* err = error_word();
+  if (!err) return cuda_failed("device error word lookup failed");
+  int launched = 0;
+  cudaError_t e = pa::launch_copy_blocks(src_dst_pairs, num_pairs, src_k, src_v, src_num_blocks,
+                                         dst_k, dst_v, dst_num_blocks, block_bytes, err,
                                          reinterpret_cast<cudaStream_t>(stream), &launched);
   count_launches(launched);
   return e == cudaSuccess ? PA_OK : cuda_failed(e);

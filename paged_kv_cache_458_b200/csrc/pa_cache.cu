@@ -97,28 +97,31 @@ cache_append_fp8_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v
 }
 
 // grid.x = pieces of a block, grid.y = pair.  Each CTA copies kPiece vectors
-// of the K block and of the V block.
+// of block src of the source K pool and of the V pool into block dst of the
+// destination pools.  Copy-on-write passes the same pool as source and
+// destination; swap passes a device pool and a host pool the device can
+// address (pinned and mapped), in either order.
 constexpr int kCopyThreads = 256;
 constexpr int kCopyUnroll = 4;
 constexpr int kPiece = kCopyThreads * kCopyUnroll;
 
 __global__ void __launch_bounds__(kCopyThreads)
-copy_blocks_kernel(const int32_t* __restrict__ pairs, uint4* __restrict__ k_cache,
-                   uint4* __restrict__ v_cache, int num_blocks, long long block_vecs,
+copy_blocks_kernel(const int32_t* __restrict__ pairs, const uint4* src_k, const uint4* src_v,
+                   int src_blocks, uint4* dst_k, uint4* dst_v, int dst_blocks, long long block_vecs,
                    unsigned int* err) {
   pdl_wait();
   pdl_launch_dependents();
   const int i = blockIdx.y;
   const int src = __ldg(pairs + 2 * i), dst = __ldg(pairs + 2 * i + 1);
-  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+  if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
     if (blockIdx.x == 0 && threadIdx.x == 0) report(err, kErrPair);
     return;
   }
   const long long base = (long long)blockIdx.x * kPiece;
-  const uint4* ks = k_cache + src * block_vecs;
-  const uint4* vs = v_cache + src * block_vecs;
-  uint4* kd = k_cache + dst * block_vecs;
-  uint4* vd = v_cache + dst * block_vecs;
+  const uint4* ks = src_k + src * block_vecs;
+  const uint4* vs = src_v + src * block_vecs;
+  uint4* kd = dst_k + dst * block_vecs;
+  uint4* vd = dst_v + dst * block_vecs;
   uint4 rk[kCopyUnroll], rv[kCopyUnroll];
 #pragma unroll
   for (int u = 0; u < kCopyUnroll; ++u) {
@@ -164,8 +167,9 @@ cudaError_t launch_cache_append_fp8(const void* k, const void* v, const int32_t*
   return e;
 }
 
-cudaError_t launch_copy_blocks(const int32_t* pairs, int num_pairs, void* k_cache, void* v_cache,
-                               int num_blocks, long long block_bytes, unsigned int* err,
+cudaError_t launch_copy_blocks(const int32_t* pairs, int num_pairs, const void* src_k,
+                               const void* src_v, int src_blocks, void* dst_k, void* dst_v,
+                               int dst_blocks, long long block_bytes, unsigned int* err,
                                cudaStream_t stream, int* launches) {
   if (num_pairs == 0) return cudaSuccess;
   const long long block_vecs = block_bytes / 16;
@@ -173,8 +177,9 @@ cudaError_t launch_copy_blocks(const int32_t* pairs, int num_pairs, void* k_cach
   if (num_pairs > 65535 || pieces > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   dim3 grid((unsigned)pieces, (unsigned)num_pairs);
   cudaError_t e = launch_pdl(copy_blocks_kernel, grid, dim3(kCopyThreads), 0, stream, pairs,
-                             static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
-                             num_blocks, block_vecs, err);
+                             static_cast<const uint4*>(src_k), static_cast<const uint4*>(src_v),
+                             src_blocks, static_cast<uint4*>(dst_k), static_cast<uint4*>(dst_v),
+                             dst_blocks, block_vecs, err);
   if (e == cudaSuccess) ++*launches;
   return e;
 }

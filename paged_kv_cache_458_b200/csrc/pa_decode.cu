@@ -201,27 +201,43 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
 
   // Lane k resolves the physical row of this warp's k-th chunk through the
   // block table (one read per chunk, all issued up front).
-  int my_row = 0;
-  if (lane < n_mine) {
-    const int tok = t_begin + (warp + lane * NW) * kChunk;
-    const int blk = __ldg(a.block_tables + (size_t)s * a.max_blocks_per_seq + tok / a.block_size);
+  // With 8-token blocks (half_boxes) the chunk's rows 8..15 have an entry of
+  // their own; past the end of the range they re-read rows of the first
+  // block instead (masked), so no entry beyond the context is read.
+  const int32_t* table = a.block_tables + (size_t)s * a.max_blocks_per_seq;
+  auto resolve = [&](int tok) {
+    const int blk = __ldg(table + tok / a.block_size);
     if (blk < 0 || blk >= a.num_blocks) {
       report(a.err, kErrBlockId);
-      my_row = a.num_blocks * a.block_size;  // outside the map: TMA fills zeros
-    } else {
-      my_row = blk * a.block_size + tok % a.block_size;
+      return a.num_blocks * a.block_size;  // outside the map: TMA fills zeros
     }
+    return blk * a.block_size + tok % a.block_size;
+  };
+  int my_row = 0, my_row2 = 0;
+  if (lane < n_mine) {
+    const int tok = t_begin + (warp + lane * NW) * kChunk;
+    my_row = resolve(tok);
+    if (a.half_boxes) my_row2 = tok + kChunk / 2 < t_end ? resolve(tok + kChunk / 2) : my_row;
   }
 
   auto issue = [&](int k) {
     const int row = __shfl_sync(0xffffffffu, my_row, k);
+    const int row2 = __shfl_sync(0xffffffffu, my_row2, k);
     if (lane == 0) {
       const int st = k % NST;
       const uint32_t bar = bar0 + st * 8;
       const uint32_t dst = stage0 + st * L::kStageBytes;
       mbar_arrive_expect_tx(bar, L::kStageBytes);
-      tma_load_3d(dst, &tm_k, bar, 0, kvh, row);
-      tma_load_3d(dst + kChunk * L::kRowBytes, &tm_v, bar, 0, kvh, row);
+      if (a.half_boxes) {
+        constexpr uint32_t kHalfBox = (kChunk / 2) * L::kRowBytes;
+        tma_load_3d(dst, &tm_k, bar, 0, kvh, row);
+        tma_load_3d(dst + kHalfBox, &tm_k, bar, 0, kvh, row2);
+        tma_load_3d(dst + kChunk * L::kRowBytes, &tm_v, bar, 0, kvh, row);
+        tma_load_3d(dst + kChunk * L::kRowBytes + kHalfBox, &tm_v, bar, 0, kvh, row2);
+      } else {
+        tma_load_3d(dst, &tm_k, bar, 0, kvh, row);
+        tma_load_3d(dst + kChunk * L::kRowBytes, &tm_v, bar, 0, kvh, row);
+      }
     }
   };
 

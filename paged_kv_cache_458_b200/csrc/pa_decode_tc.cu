@@ -445,16 +445,23 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       const int n_tok = max(0, t_end - t_begin);
       const int n_tiles = (n_tok + kTile - 1) / kTile;
       const int n_groups = (n_tok + kGroupRows - 1) / kGroupRows;  // <= 32
-      int my_row = 0;
-      if (lane < n_groups) {
-        const int tok = t_begin + lane * kGroupRows;
-        const int blk = __ldg(a.block_tables + (size_t)s * a.max_blocks_per_seq + tok / a.block_size);
+      // With 8-token blocks (half_boxes) rows 8..15 of a group have their own
+      // entry; past the end of the item they re-read the first block (masked).
+      const int32_t* table = a.block_tables + (size_t)s * a.max_blocks_per_seq;
+      auto resolve = [&](int tok) {
+        const int blk = __ldg(table + tok / a.block_size);
         if (blk < 0 || blk >= a.num_blocks) {
           report(a.err, kErrBlockId);
-          my_row = a.num_blocks * a.block_size;  // outside the map: TMA fills zeros
-        } else {
-          my_row = blk * a.block_size + tok % a.block_size;
+          return a.num_blocks * a.block_size;  // outside the map: TMA fills zeros
         }
+        return blk * a.block_size + tok % a.block_size;
+      };
+      int my_row = 0, my_row2 = 0;
+      if (lane < n_groups) {
+        const int tok = t_begin + lane * kGroupRows;
+        my_row = resolve(tok);
+        if (a.half_boxes)
+          my_row2 = tok + kGroupRows / 2 < t_end ? resolve(tok + kGroupRows / 2) : my_row;
       }
       if constexpr (GROUP) {
         // members x g query rows, 16-byte pieces stored in the 128B-swizzled
@@ -510,9 +517,13 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           // lane 4 r + k loads piece k (K or V, 64-element half) of group r
           const int r = lane >> 2, k = lane & 3;
           const int row = __shfl_sync(0xffffffffu, my_row, min(g0 + r, 31));
-          if (r < ng)
-            tma_load_3d(dst + k * L::kHalf + r * kGroupRows * 128, k < 2 ? &tm_k : &tm_v, fb,
-                        (k & 1) * 64, kvh, row);
+          const int row2 = __shfl_sync(0xffffffffu, my_row2, min(g0 + r, 31));
+          if (r < ng) {
+            const uint32_t d = dst + k * L::kHalf + r * kGroupRows * 128;
+            const void* map = k < 2 ? &tm_k : &tm_v;
+            tma_load_3d(d, map, fb, (k & 1) * 64, kvh, row);
+            if (a.half_boxes) tma_load_3d(d + (kGroupRows / 2) * 128, map, fb, (k & 1) * 64, kvh, row2);
+          }
         }
         ++issued;
       }

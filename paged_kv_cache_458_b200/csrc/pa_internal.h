@@ -33,6 +33,9 @@ struct DecodeArgs {
   int own_tokens;                // partition size of a sequence's own tokens (partition_tokens
                                  // without a plan)
   int grid_parts;                // partitions per (sequence, kv head) of the CUDA-core grid
+  int half_boxes;                // block_size is a multiple of 8 but not of 16: each
+                                 // 16-token TMA box is loaded as two 8-token boxes, which
+                                 // may come from two blocks
 };
 
 // Sequences per launch of the shared-prefix kernel; groups never cross a
@@ -113,8 +116,11 @@ cudaError_t launch_cache_append_fp8(const void* k, const void* v, const int32_t*
                                     long long num_slots, int dtype, int num_kv_heads, int head_dim,
                                     const float* k_scale, const float* v_scale, unsigned int* err,
                                     cudaStream_t stream, int* launches);
-cudaError_t launch_copy_blocks(const int32_t* pairs, int num_pairs, void* k_cache, void* v_cache,
-                               int num_blocks, long long block_bytes, unsigned int* err,
+// Copy-on-write within one pool (src == dst pools) and swap between two
+// pools, either of which may be host memory the device can address.
+cudaError_t launch_copy_blocks(const int32_t* pairs, int num_pairs, const void* src_k,
+                               const void* src_v, int src_blocks, void* dst_k, void* dst_v,
+                               int dst_blocks, long long block_bytes, unsigned int* err,
                                cudaStream_t stream, int* launches);
 
 }  // namespace pa

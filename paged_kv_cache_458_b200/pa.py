@@ -74,6 +74,8 @@ def _declare(lib):
     lib.pa_decode_fp8.argtypes = [P, P, P, P, P, P, P, c.c_float, P, SP, I32, P, SZ, P]
     lib.pa_copy_blocks.restype = c.c_int
     lib.pa_copy_blocks.argtypes = [P, I32, P, P, SP, P]
+    lib.pa_swap_blocks.restype = c.c_int
+    lib.pa_swap_blocks.argtypes = [P, I32, P, P, I32, P, P, I32, SP, P]
     lib.pa_last_device_error.restype = c.c_int
     lib.pa_last_device_error.argtypes = [P, c.POINTER(c.c_uint32)]
     lib.pa_status_string.restype = c.c_char_p
@@ -258,6 +260,14 @@ def pa_copy_blocks(src_dst_pairs, num_pairs: int, k_cache, v_cache, shape: pa_sh
     _check("pa_copy_blocks", lib().pa_copy_blocks(
         _ptr(src_dst_pairs), int(num_pairs), _ptr(k_cache), _ptr(v_cache), ctypes.byref(shape),
         _stream(stream)))
+
+
+def pa_swap_blocks(src_dst_pairs, num_pairs: int, src_k, src_v, src_num_blocks: int, dst_k, dst_v,
+                   dst_num_blocks: int, shape: pa_shape, stream=None) -> None:
+    """Copy whole blocks between two pools (device and/or pinned host memory)."""
+    _check("pa_swap_blocks", lib().pa_swap_blocks(
+        _ptr(src_dst_pairs), int(num_pairs), _ptr(src_k), _ptr(src_v), int(src_num_blocks),
+        _ptr(dst_k), _ptr(dst_v), int(dst_num_blocks), ctypes.byref(shape), _stream(stream)))
 
 
 def pa_last_device_error(stream=None) -> tuple[int, int]:

@@ -45,7 +45,7 @@ FAKE = 1 << 20  # a 16-byte-aligned non-null address; validation fails before an
     (dict(head_dim=0), pa.PA_ERR_INVALID_ARG),
     (dict(num_q_heads=8, num_kv_heads=3), pa.PA_ERR_INVALID_ARG),
     (dict(num_q_heads=64, num_kv_heads=2), pa.PA_ERR_UNSUPPORTED),  # group 32
-    (dict(block_size=8), pa.PA_ERR_UNSUPPORTED),
+    (dict(block_size=12), pa.PA_ERR_UNSUPPORTED),       # blocks are multiples of 8 tokens
     (dict(dtype=7), pa.PA_ERR_UNSUPPORTED),
     (dict(partition_tokens=24), pa.PA_ERR_UNSUPPORTED),
     (dict(partition_tokens=4096), pa.PA_ERR_UNSUPPORTED),
@@ -135,6 +135,24 @@ def test_multi_query_workspace_and_validation(lib):
     st = lib.pa_decode_multi(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s8), 4, 700,
                              FAKE, 1 << 24, None)
     assert st == pa.PA_ERR_INVALID_ARG
+
+
+def test_swap_validation(lib):
+    s = _shape()
+    call = lambda pairs=FAKE, n=2, sk=FAKE, sv=FAKE + (1 << 24), snb=8, dk=FAKE + (2 << 24), \
+        dv=FAKE + (3 << 24), dnb=8: lib.pa_swap_blocks(pairs, n, sk, sv, snb, dk, dv, dnb,  # noqa: E731
+                                                      ctypes.byref(s), None)
+    n0 = pa.pa_kernel_launches()
+    assert call(n=0) == pa.PA_OK
+    assert call(n=-1) == pa.PA_ERR_INVALID_ARG
+    assert call(pairs=None) == pa.PA_ERR_INVALID_ARG
+    assert call(dk=None) == pa.PA_ERR_INVALID_ARG
+    assert call(sk=FAKE + 8) == pa.PA_ERR_INVALID_ARG            # misaligned
+    assert call(dk=FAKE + 4096) == pa.PA_ERR_INVALID_ARG         # pools overlap
+    assert call(n=70000) == pa.PA_ERR_UNSUPPORTED
+    # FAKE addresses are no memory the device knows: refused before any launch
+    assert call() == pa.PA_ERR_INVALID_ARG
+    assert pa.pa_kernel_launches() == n0
 
 
 def test_default_partition(lib):

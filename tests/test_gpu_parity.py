@@ -142,7 +142,7 @@ def test_edge_contexts(orc, dtype, head_dim, group, variant):
 
 
 @pytest.mark.parametrize("variant", [1, 2, SHARED], ids=lambda v: VARIANTS[v])
-@pytest.mark.parametrize("block_size", [16, 32, 256])
+@pytest.mark.parametrize("block_size", [8, 16, 32, 256])
 @pytest.mark.parametrize("partition_tokens", [16, 48, 128, 256, 512, 2048])
 def test_block_and_partition_sizes(orc, block_size, partition_tokens, variant):
     if variant in (2, SHARED) and (partition_tokens % 128 or partition_tokens > 512):

@@ -116,7 +116,7 @@ def groups_for(rng, group):
 
 @pytest.mark.parametrize("dtype", [gen.F16, gen.BF16], ids=["f16", "bf16"])
 @pytest.mark.parametrize("group", [1, 2, 4, 8, 16])
-@pytest.mark.parametrize("block_size", [16, 256])
+@pytest.mark.parametrize("block_size", [8, 16, 256])
 def test_shared_prefix_groups(orc, dtype, group, block_size):
     rng = np.random.default_rng(9000 + 10 * group + block_size + dtype)
     c = gen.grouped_decode_case(rng, groups=groups_for(rng, group), num_q_heads=2 * group,

@@ -56,6 +56,11 @@ def parse_args(argv=None):
     p.add_argument("--partition-tokens", type=int, default=0)
     p.add_argument("--variant", default="auto", choices=sorted(VARIANTS),
                    help="decode kernel: auto, cuda_cores or tensor_cores")
+    p.add_argument("--block-size", type=int, default=0,
+                   help="re-block the workload's pool into blocks of this many tokens "
+                        "(a divisor of its block size, e.g. 8); every token keeps its slot")
+    p.add_argument("--swap", action="store_true",
+                   help="also time pa_swap_blocks between the pool and pinned host memory")
     p.add_argument("--query-tokens", type=int, default=1,
                    help="query tokens per sequence (pa_decode_multi when > 1): the last ones "
                         "of each context, causal among themselves")
@@ -343,6 +348,62 @@ class DeviceWorkload:
             ev[2].record(stream)
 
 
+def split_blocks(case, factor: int):
+    """The same case over blocks `factor` times smaller: each block b becomes
+    blocks factor*b .. factor*b + factor-1, so every token keeps its slot."""
+    import dataclasses
+
+    if factor == 1:
+        return case
+    NB, bs, Hkv, D = case.k_cache.shape
+    nbs = bs // factor
+
+    def tables(t):
+        out = np.full((t.shape[0], t.shape[1] * factor), -1, dtype=np.int32)
+        for i in range(factor):
+            out[:, i::factor] = np.where(t >= 0, factor * t + i, -1)
+        return out
+
+    def pairs(p):
+        p = np.asarray(p, dtype=np.int32).reshape(-1, 2)
+        return np.concatenate([factor * p + i for i in range(factor)]) if len(p) else p
+
+    steps = [dataclasses.replace(st, block_tables=tables(st.block_tables), pairs=pairs(st.pairs))
+             for st in case.steps]
+    return dataclasses.replace(
+        case, block_size=nbs, num_blocks=NB * factor, max_blocks_per_seq=case.max_blocks_per_seq * factor,
+        k_cache=case.k_cache.reshape(NB * factor, nbs, Hkv, D),
+        v_cache=case.v_cache.reshape(NB * factor, nbs, Hkv, D),
+        block_tables=tables(case.block_tables), steps=steps)
+
+
+def swap_bandwidth(w, torch, pa, n_blocks: int = 256, reps: int = 5):
+    """pa_swap_blocks out to pinned host memory and back in, GB/s each way."""
+    NB = w.case.num_blocks
+    n = min(n_blocks, NB)
+    hk = torch.empty((n,) + tuple(w.k_cache.shape[1:]), dtype=w.k_cache.dtype).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    out_pairs = torch.tensor([[b, i] for i, b in enumerate(range(NB - n, NB))], dtype=torch.int32,
+                             device="cuda")
+    in_pairs = out_pairs.flip(1).contiguous()
+    nbytes = 2 * hk.numel() * hk.element_size()
+    res = {}
+    for name, args in (("out", (out_pairs, n, w.k_cache, w.v_cache, NB, hk, hv, n)),
+                       ("in", (in_pairs, n, hk, hv, n, w.k_cache, w.v_cache, NB))):
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            pa.pa_swap_blocks(*args, w.shape)
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        res[f"{name}_gbs"] = round(nbytes / (sorted(ts)[len(ts) // 2] * 1e-3) / 1e9, 2)
+    res["blocks"] = n
+    res["bytes_each_way"] = nbytes
+    return res
+
+
 def run_ours(args, rank, world, local, dist):
     import torch
 
@@ -353,6 +414,10 @@ def run_ours(args, rank, world, local, dist):
     n_cycle = max(1, min(args.cycle, args.steps + args.warmup))
     case = gen.make_case(args.workload, n_steps=n_cycle, poison=False,
                          seed=gen.SEED_BASE + gen.WORKLOADS[args.workload].number + 1000 * rank)
+    if args.block_size:
+        if case.block_size % args.block_size:
+            raise SystemExit(f"--block-size must divide the workload's {case.block_size}")
+        case = split_blocks(case, case.block_size // args.block_size)
     shared = {"on": 1, "off": 0}.get(args.shared_prefix)
     if shared is None:
         shared = int(args.variant == "auto" and args.kv_cache != "fp8" and
@@ -458,6 +523,8 @@ def run_ours(args, rank, world, local, dist):
         # the same decode counted in distinct K/V slots (shared blocks once)
         result["unique_kv_gbs_step0_est"] = round(
             result["unique_kv_bytes_step0"] / (dec_total_ms / args.steps * 1e-3) / 1e9, 2)
+    if args.swap:
+        result["swap"] = swap_bandwidth(w, torch, pa)
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, w, stream, bytes_per, n_cycle, dist)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

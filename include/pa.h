@@ -219,8 +219,9 @@ pa_status pa_decode(const void *q, const void *k_cache, const void *v_cache,
  * one sequence are consecutive and start with the same blocks, so when the
  * shape allows the shared-prefix kernel (head_dim 128, variant
  * PA_DECODE_AUTO, a 16-bit cache, partition_tokens 0 or a multiple of 128
- * up to 512), the tokens they have in common are read once for all of them.
- * Otherwise each is decoded on its own.  Tq == 1 is pa_decode.
+ * up to 512) and Tq * g >= 8, the tokens they have in common are read once
+ * for all of them.  Otherwise each is decoded on its own (the common tokens
+ * then come mostly from L2).  Tq == 1 is pa_decode.
  * workspace: pa_decode_multi_workspace_bytes(shape, Tq, max_context_len).
  */
 size_t pa_decode_multi_workspace_bytes(const pa_shape *shape, int32_t num_query_tokens,

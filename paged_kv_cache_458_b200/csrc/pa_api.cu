@@ -390,13 +390,19 @@ pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
 namespace {
 
 // The one-token batch pa_decode_multi runs: S * Tq virtual sequences, grouped
-// by shared prefix whenever the shape allows the shared-prefix kernel.
+// by shared prefix when the shape allows the shared-prefix kernel and a
+// sequence's Tq x g query rows fill at least 8 of its 32 columns.  Below that
+// the CUDA-core kernel over the virtual sequences (which re-read their common
+// tokens, mostly from L2) measured faster: llama2_7b with Tq = 2 took 0.141
+// vs 0.251 ms, with Tq = 4 0.255 vs 0.293 ms; with Tq x g = 16 or 32 the
+// shared path wins (mistral_7b_gqa, Tq = 4: 0.572 vs 0.955 ms).
 pa_shape multi_shape(const pa_shape* s, int num_query_tokens) {
   pa_shape e = *s;
   e.num_seqs = s->num_seqs * num_query_tokens;
   const int pt = s->partition_tokens;
+  const int rows = num_query_tokens * (s->num_q_heads / s->num_kv_heads);
   e.shared_prefix = s->head_dim == 128 && s->variant == PA_DECODE_AUTO &&
-                    s->cache_format == PA_CACHE_AS_DTYPE &&
+                    s->cache_format == PA_CACHE_AS_DTYPE && rows >= 8 &&
                     (pt == 0 || (pt % pa::decode_tc_tile_tokens() == 0 && pt <= 512));
   return e;
 }

@@ -121,10 +121,15 @@ def test_multi_query_workspace_and_validation(lib):
     assert lib.pa_decode_multi_workspace_bytes(ctypes.byref(s), 1, 700) == one
     assert lib.pa_decode_multi_workspace_bytes(ctypes.byref(s), 0, 700) == 0
     w4 = lib.pa_decode_multi_workspace_bytes(ctypes.byref(s), 4, 700)
-    # virtual tables and contexts, then a shared-prefix decode of 16 virtual sequences
-    # (16 * 8 heads * (2 + 1) partitions of (128 + 2) floats, plan 256 bytes, counter 256)
+    # virtual tables and contexts, then a shared-prefix decode of 16 virtual
+    # sequences (4 tokens x g 4 = 16 rows >= 8): 16 * 8 heads * (2 + 1)
+    # partitions of (128 + 2) floats, plan 256 bytes, counter 256
     rows = 16 * 8 * 3
     assert w4 == 4 * 16 * 64 + 256 + 256 + 256 + rows * 128 * 4 + rows * 8
+    # 1 query head per kv head, 2 tokens: 2 rows < 8, plain decode of 8 virtual
+    # sequences (one 1024-token partition: the counter only)
+    s1 = _shape(num_q_heads=2, max_blocks_per_seq=64)
+    assert lib.pa_decode_multi_workspace_bytes(ctypes.byref(s1), 2, 700) == 4 * 8 * 64 + 256 + 256
     st = lib.pa_decode_multi(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s), 0, 700, FAKE,
                              1 << 24, None)
     assert st == pa.PA_ERR_INVALID_ARG

@@ -46,17 +46,20 @@
 // 16-token group of an item through the block table and issues per 128-token
 // tile 32 tiled TMA loads (8 groups x {K, V} x two 64-element halves,
 // 128B-swizzled) into one of NST stages, plus the item's query rows into an
-// item slot.  Four compute warps consume tiles in order; thread 0 issues the
-// MMAs and commits them to mbarriers.  Tokens at or past the end of the item
-// are masked in P and their V rows are zeroed in shared memory before the PV
-// product, so stale or NaN rows never reach the result.
+// item slot.  A dedicated MMA warp issues every MMA and commits it to an
+// mbarrier, so issuing them never holds up the softmax; the compute warps
+// consume tiles in order and tell it through two more mbarriers when S^T(g)
+// has been read and when P(g) has been written.  Tokens at or past the end of
+// the item are masked in P and their V rows are zeroed in shared memory before
+// the PV product, so stale or NaN rows never reach the result.
 //
 // Split-K partials and the merge kernel are shared with the CUDA-core path.
 //
-// Every wait is bounded; a compute-side wait is made by thread 0 and its
-// outcome shared through an OR-reduced named barrier, so the four compute
-// warps always agree whether to go on.  On the way out the producer waits for
-// its TMA copies, thread 0 for its MMAs, and warp 0 frees the TMEM columns.
+// Every wait is bounded.  The compute warps wait per warp, and an OR-reduced
+// named barrier then makes them all take the same way out when any wait
+// failed (every decision before a named barrier comes from a barrier result).
+// On the way out the producer waits for its TMA copies, the MMA warp commits
+// once more and waits for all its MMAs, and warp 0 frees the TMEM columns.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -82,7 +85,7 @@ struct Warps {
   static constexpr int kNCW = NC >= 16 ? 8 : (NC >= 8 ? 4 : NC);  // columns per warpgroup
   static constexpr int kNWG = NC / kNCW;                           // compute warpgroups
   static constexpr int kCompute = 128 * kNWG;                      // compute threads
-  static constexpr int kThreads = kCompute + 32;                   // + the producer warp
+  static constexpr int kThreads = kCompute + 64;                   // + MMA warp + producer warp
   static_assert(kNCW * kNWG == NC, "columns split evenly");
 };
 
@@ -111,9 +114,10 @@ struct Layout {
   static constexpr int kDesc = kStat + 2 * N * 4;              // [slots][8] int
   static constexpr int kPrefix = kDesc + kSlots * 8 * 4;       // [MAXSEQS + 1] int
   static constexpr int kBars = (kPrefix + (MAXSEQS + 1) * 4 + 7) / 8 * 8;
-  // full[NST], empty[NST], ready[slots], free[slots], qk, pv, drain
-  static constexpr int kNumBars = 2 * NST + 2 * kSlots + 3;
-  static constexpr int kMisc = kBars + kNumBars * 8;           // tmem address, abort flag
+  // full[NST], empty[NST], ready[slots], free[slots], qk, pv, drain, s_free, p_ready
+  static constexpr int kNumBars = 2 * NST + 2 * kSlots + 5;
+  static constexpr int kMisc = kBars + kNumBars * 8;           // tmem address, abort flag,
+                                                               // accumulate flags [2]
   static constexpr int kUsed = kMisc + 16;
   static constexpr int kAlloc = kUsed + 1024;                  // room to align the base
   static_assert(kQ % 1024 == 0 && kQBytes % 1024 == 0 && kP % 256 == 0, "swizzle atoms");
@@ -302,7 +306,8 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   constexpr int NC = GROUP ? N : G;  // columns that carry query rows
   using W = Warps<NC>;
   constexpr int kComputeThreads = W::kCompute, kThreads = W::kThreads, NCW = W::kNCW;
-  constexpr int kProducerWarp = kComputeThreads / 32;
+  constexpr int kComputeWarps = kComputeThreads / 32;
+  constexpr int kMmaWarp = kComputeWarps, kProducerWarp = kComputeWarps + 1;
   using L = Layout<NST, N, C::kMaxSeqs>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr uint32_t kIdescQK = instr_desc(kBf16 ? 1 : 0, 0, 0, kTile, N);
@@ -330,6 +335,9 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   const uint32_t qk_bar = bars + (2 * NST + 2 * kSlots) * 8;
   const uint32_t pv_bar = qk_bar + 8;
   const uint32_t drain_bar = qk_bar + 16;
+  const uint32_t s_free_bar = qk_bar + 24;   // compute warps have read S^T(g)
+  const uint32_t p_ready_bar = qk_bar + 32;  // compute warps have written P(g)
+  volatile int* acc_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);  // [2]
   const uint32_t sm_stages = smem_addr(smem + L::kStages);
   const uint32_t sm_q = smem_addr(smem + L::kQ);
   const uint32_t sm_p = smem_addr(smem + L::kP);
@@ -348,11 +356,13 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     }
     for (int sl = 0; sl < kSlots; ++sl) {
       mbar_init(ready_bar(sl), 1);
-      mbar_init(free_bar(sl), kComputeThreads / 32);
+      mbar_init(free_bar(sl), kComputeWarps);
     }
     mbar_init(qk_bar, 1);
     mbar_init(pv_bar, 1);
     mbar_init(drain_bar, 1);
+    mbar_init(s_free_bar, kComputeWarps);
+    mbar_init(p_ready_bar, kComputeWarps);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -481,6 +491,17 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
       }
+      // shared-prefix item: bit m set when member m's result is this
+      // partition alone (written directly, not as a split-K partial)
+      int direct_mask = 0;
+      if constexpr (GROUP) {
+        bool dm = false;
+        if (lane < ctx_or_members) {
+          const int ctx = max(0, min(__ldg(a.context_lens + s + lane), a.max_context_len));
+          dm = seq_split(a.plan, s + lane, ctx, a.own_tokens).total <= 1;
+        }
+        direct_mask = (int)__ballot_sync(0xffffffffu, dm);
+      }
       if (lane == 0) {
         desc[kDS] = s;
         desc[kDKvh] = kvh;
@@ -488,7 +509,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         desc[kDBegin] = t_begin;
         desc[kDEnd] = t_end;
         desc[kDTiles] = n_tiles;
-        desc[kDParts] = GROUP ? 0 : (ctx_or_members + PT - 1) / PT;
+        desc[kDParts] = GROUP ? direct_mask : (ctx_or_members + PT - 1) / PT;
         desc[kDCtx] = ctx_or_members;
         const uint32_t rb = ready_bar(slot);
         if constexpr (GROUP) {
@@ -540,30 +561,18 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     if (lane == 0)
       for (int k = max(0, issued - NST); k < issued; ++k)
         mbar_wait(full_bar(k % NST), (k / NST) & 1, a.err);
-  } else {
+  } else if (warp == kMmaWarp) {
     // =====================================================================
-    // compute warps: thread (t, cg) = token row t of S^T and row d = t of O^T,
-    // for the columns of warpgroup cg
+    // MMA warp (lane 0): every tcgen05.mma of the CTA, so that issuing them
+    // never holds up the compute warps.  Per tile g (numbered across items):
+    //   S^T(g) = K(g) . Q^T   once stage g has landed and S^T(g-1) was read;
+    //   O^T (+)= V^T . P^T(g) once the compute warps have written P(g).
+    // Each of qk, pv, s_free and p_ready completes once per tile, in order,
+    // so tile g waits on phase parity g & 1.
     // =====================================================================
-    // Tile j of an item: S^T(j) = K(j) . Q^T was issued during tile j-1 (or at
-    // the item start); thread 0 waits for it and for O^T(j-1); every thread
-    // reads its part of its S^T row, and as soon as all are read S^T(j+1) is
-    // issued (when its stage has landed; else after O^T(j)).  The softmax
-    // writes P, and O^T(j) += V^T . P^T is issued without waiting for it.  The
-    // output stays in TMEM across tiles: each column's softmax reference m_ref
-    // only moves when a logit exceeds it by more than kRescale (log2 units),
-    // and only then is O^T folded into registers and rescaled.  Hence p <=
-    // 2^kRescale, well inside fp32 and both operand types.
-    constexpr float kRescale = 8.f;
-    const int t = tid & 127;         // token row of S^T, output row of O^T
-    const int cg = tid >> 7;         // column group
-    const int c0 = cg * NCW;         // first column of this thread
-    const int quarter = warp & 3;    // TMEM lane quarter of this warp
-    const uint32_t t_lane = ((uint32_t)(quarter * 32) << 16);
-    int n_used = 0;  // tiles consumed: the stage ring position, and the number of
-                     // each tile's qk and pv commits (one of each per tile, in order)
     bool ok = true;
-    auto issue_qk = [&](int st, uint32_t q_addr) {  // thread 0
+    int g = 0;  // tiles issued so far
+    auto issue_qk = [&](int st, uint32_t q_addr) {
       tc_fence_after();
       const uint32_t kt = sm_stages + st * L::kStageBytes;
 #pragma unroll
@@ -574,6 +583,77 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                 kIdescQK, kk > 0);
       }
       mma_commit(qk_bar);
+    };
+    if (lane == 0) {
+      for (int it = 0; ok; ++it) {
+        const int slot = it % kSlots;
+        ok = mbar_wait_or_abort(ready_bar(slot), (it / kSlots) & 1, a.err, abort_flag);
+        if (!ok) break;
+        const int n_tiles = desc_all[slot * 8 + kDTiles];
+        if (n_tiles < 0) break;  // end of work
+        const uint32_t q_addr = sm_q + slot * L::kQBytes;
+        // S^T(h) needs its stage landed and S^T(h-1) read by the compute warps
+        auto qk_for = [&](int h) {
+          bool w = mbar_wait_or_abort(full_bar(h % NST), (h / NST) & 1, a.err, abort_flag);
+          if (w && h > 0) w = mbar_wait_or_abort(s_free_bar, (h - 1) & 1, a.err, abort_flag);
+          if (w) issue_qk(h % NST, q_addr);
+          return w;
+        };
+        if (n_tiles > 0) ok = qk_for(g);
+        for (int j = 0; j < n_tiles && ok; ++j, ++g) {
+          const int st = g % NST;
+          // S^T(g+1) as soon as S^T(g) has been read: it runs during tile g's
+          // softmax; then, once P(g) is written, O^T(g)
+          if (j + 1 < n_tiles) {
+            ok = qk_for(g + 1);
+            if (!ok) break;
+          }
+          ok = mbar_wait_or_abort(p_ready_bar, g & 1, a.err, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t vt = sm_stages + st * L::kStageBytes + 2 * L::kHalf;
+          const uint32_t acc0 = (uint32_t)acc_flag[g & 1];
+#pragma unroll
+          for (int part_p = 0; part_p < 2; ++part_p)  // P = hi + lo
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk)
+              mma_f16(tmem + N, smem_desc(vt + kk * 2048, L::kHalf, 1024, kSw128),
+                      smem_desc(sm_p + part_p * L::kPBytes + kk * 512, L::kPAtom, 256, kSw32),
+                      kIdescPV, acc0 | (uint32_t)(part_p > 0 || kk > 0));
+          mma_commit(pv_bar);
+          mma_commit(empty_bar(st));  // the stage is free once these MMAs are done
+        }
+      }
+      if (!ok) *abort_flag = 1;
+      // every MMA issued here completes before TMEM is freed (bounded wait)
+      mma_commit(drain_bar);
+      mbar_wait(drain_bar, 0, a.err);
+    }
+    __syncwarp();
+  } else {
+    // =====================================================================
+    // compute warps: thread (t, cg) = token row t of S^T and row d = t of O^T,
+    // for the columns of warpgroup cg.  Per tile g: wait for S^T(g), read it
+    // and release it (s_free) so the MMA warp can issue S^T(g+1); the softmax
+    // writes P(g) after O^T(g-1), its last reader, completed; then p_ready.
+    // The output stays in TMEM across tiles: each column's softmax reference
+    // m_ref only moves when a logit exceeds it by more than kRescale (log2
+    // units), and only then is O^T folded into registers and rescaled (and
+    // the next PV overwrites instead of accumulating).  Hence p <= 2^kRescale.
+    // =====================================================================
+    constexpr float kRescale = 8.f;
+    const int t = tid & 127;         // token row of S^T, output row of O^T
+    const int cg = tid >> 7;         // column group
+    const int c0 = cg * NCW;         // first column of this thread
+    const int quarter = warp & 3;    // TMEM lane quarter of this warp
+    const uint32_t t_lane = ((uint32_t)(quarter * 32) << 16);
+    int g = 0;  // tiles consumed, numbered across items
+    bool ok = true;
+    // one lane per warp waits on an mbarrier, the warp follows
+    auto warp_wait = [&](uint32_t bar, uint32_t parity) {
+      bool w = true;
+      if (lane == 0) w = mbar_wait_or_abort(bar, parity, a.err, abort_flag);
+      return __shfl_sync(0xffffffffu, (int)w, 0) != 0;
     };
     for (int it = 0; ok; ++it) {
       const int slot = it % kSlots;
@@ -586,33 +666,29 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       const int t_begin = desc[kDBegin], t_end = desc[kDEnd], n_parts = desc[kDParts];
       const int ctx_or_members = desc[kDCtx];
       const int cols = GROUP ? ctx_or_members * G : G;
-      const uint32_t q_addr = sm_q + slot * L::kQBytes;
 
       float acc[NCW], l_tok[NCW], m_ref[NCW];
 #pragma unroll
       for (int c = 0; c < NCW; ++c) acc[c] = 0.f, l_tok[c] = 0.f, m_ref[c] = -INFINITY;
       bool pv_acc = false;  // O^T in TMEM holds tiles not folded into acc yet
 
-      if (tid == 0 && n_tiles > 0) {
-        const int st = n_used % NST;
-        ok = mbar_wait_or_abort(full_bar(st), (n_used / NST) & 1, a.err, abort_flag);
-        if (ok) issue_qk(st, q_addr);
-      }
-      for (int j = 0; j < n_tiles; ++j, ++n_used) {
-        const int st = n_used % NST;
-        const int st_next = (n_used + 1) % NST;
-        const bool has_next = j + 1 < n_tiles;
-        const uint32_t vt = sm_stages + st * L::kStageBytes + 2 * L::kHalf;
+      for (int j = 0; j < n_tiles; ++j, ++g) {
+        const int st = g % NST;
         const int n_valid = min(kTile, t_end - (t_begin + j * kTile));
-        // ---- S^T(j) and O^T(j-1) are complete
-        if (tid == 0 && ok) {
-          ok = mbar_wait_or_abort(qk_bar, n_used & 1, a.err, abort_flag);
-          if (ok && j > 0) ok = mbar_wait_or_abort(pv_bar, (n_used - 1) & 1, a.err, abort_flag);
-        }
-        if (named_barrier_or(1, kComputeThreads, !ok || *abort_flag)) { ok = false; break; }
-        tc_fence_after();
+        // ---- S^T(g); and O^T(g-1), the last reader of P and the last writer
+        // of O^T, is done.  Each warp waits on its own; the OR-barrier then
+        // makes every compute thread take the same way out if any wait failed.
         float sv[NCW];
-        tmem_ld<NCW>(tmem + t_lane + (uint32_t)c0, sv);
+        bool ok_w = warp_wait(qk_bar, g & 1);
+        if (ok_w) {
+          tc_fence_after();
+          tmem_ld<NCW>(tmem + t_lane + (uint32_t)c0, sv);
+          tc_fence_before();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free_bar);  // S^T(g) read: the MMA warp may reuse it
+        if (ok_w && j > 0) ok_w = warp_wait(pv_bar, (g - 1) & 1);
+        if (named_barrier_or(1, kComputeThreads, !ok_w || *abort_flag)) { ok = false; break; }
         const bool valid = t < n_valid;
         bool over = false;
 #pragma unroll
@@ -620,14 +696,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           sv[c] = valid ? sv[c] * a.scale_log2 : -INFINITY;
           over |= (c0 + c < cols) && (sv[c] > m_ref[c] + kRescale);
         }
-        tc_fence_before();
-        // all S^T rows are read: its columns may take S^T(j+1)
         const bool rescale = named_barrier_or(1, kComputeThreads, over);
-        bool next_issued = false;
-        if (tid == 0 && has_next && mbar_test_wait(full_bar(st_next), ((n_used + 1) / NST) & 1)) {
-          issue_qk(st_next, q_addr);
-          next_issued = true;
-        }
         if (rescale) {
           // new references: this tile's column maxima where they are higher
           {
@@ -650,7 +719,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
             l_tok[c] *= alpha[c];
           }
           if (pv_acc) {
-            // fold O^T (tiles before j, complete) into acc, on the new reference
+            // fold O^T (tiles before g, complete) into acc, on the new reference
             tc_fence_after();
             float ov[NCW];
             tmem_ld<NCW>(tmem + t_lane + (uint32_t)(N + c0), ov);
@@ -670,9 +739,9 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         }
         // P^T rows: per 16-column atom, a 32-byte row per token (MN-major,
         // 32-byte swizzle: 16-byte piece c of row t sits at c ^ bit 2 of t),
-        // once for hi = round(p) and once for lo = round(p - hi).  O^T(j-1),
-        // the last reader of P, is complete.  This thread writes columns
-        // [c0, c0 + NCW): NCW * 2 bytes inside one 16-byte piece.
+        // once for hi = round(p) and once for lo = round(p - hi).  This
+        // thread writes columns [c0, c0 + NCW): NCW * 2 bytes inside one
+        // 16-byte piece.
         {
           const int atom = c0 / 16, piece = (c0 % 16) / 8, within = (c0 % 8) * 2;
           unsigned char* prow = smem + L::kP + atom * L::kPAtom + t * 32 +
@@ -708,33 +777,17 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           for (int i = cg; i < 16; i += W::kNWG)
             *reinterpret_cast<uint4*>(vrow + (i >> 3) * L::kHalf + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
         }
+        if (tid == 0) acc_flag[g & 1] = pv_acc ? 1 : 0;  // does O^T(g) accumulate?
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_before();
-        named_barrier(1, kComputeThreads);
-
-        // ---- O^T (+)= V^T . P^T, then S^T(j+1) if it is not on its way yet
-        if (tid == 0) {
-          tc_fence_after();
-#pragma unroll
-          for (int part_p = 0; part_p < 2; ++part_p)  // P = hi + lo
-#pragma unroll
-            for (int kk = 0; kk < kTile / 16; ++kk)
-              mma_f16(tmem + N, smem_desc(vt + kk * 2048, L::kHalf, 1024, kSw128),
-                      smem_desc(sm_p + part_p * L::kPBytes + kk * 512, L::kPAtom, 256, kSw32),
-                      kIdescPV, pv_acc || part_p > 0 || kk > 0);
-          mma_commit(pv_bar);
-          mma_commit(empty_bar(st));  // the stage is free once these MMAs are done
-          if (has_next && !next_issued) {
-            ok = mbar_wait_or_abort(full_bar(st_next), ((n_used + 1) / NST) & 1, a.err, abort_flag);
-            if (ok) issue_qk(st_next, q_addr);
-          }
-        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_ready_bar);  // P(g) written: the MMA warp issues O^T(g)
         pv_acc = true;
       }
       if (!ok) break;
 
       // ---- item result: fold the last O^T, reduce the per-token sums, write
-      if (tid == 0 && n_tiles > 0) ok = mbar_wait_or_abort(pv_bar, (n_used - 1) & 1, a.err, abort_flag);
+      if (tid == 0 && n_tiles > 0) ok = mbar_wait_or_abort(pv_bar, (g - 1) & 1, a.err, abort_flag);
       if (named_barrier_or(1, kComputeThreads, !ok || *abort_flag)) { ok = false; break; }
       if (n_tiles > 0) {
         tc_fence_after();
@@ -764,9 +817,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         const size_t qh = (size_t)(s + m) * a.num_q_heads + (size_t)kvh * G + h;
         bool zero = false, direct;
         if constexpr (GROUP) {
-          // shared partitions of the member, plus its own ones
-          const int ctx = max(0, min(__ldg(a.context_lens + s + m), a.max_context_len));
-          direct = seq_split(a.plan, s + m, ctx, a.own_tokens).total <= 1;
+          direct = (n_parts >> m) & 1;  // from the producer: this partition is the member's result
         } else {
           zero = ctx_or_members == 0;
           direct = n_parts <= 1;
@@ -787,13 +838,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       named_barrier(1, kComputeThreads);  // `red` and `stat` are reused by the next item
       if (lane == 0) mbar_arrive(free_bar(slot));  // its query rows have been used
     }
-    if (!ok && tid == 0) *abort_flag = 1;
-    // Every MMA thread 0 issued completes before TMEM is freed: one more
-    // commit tracks all of them (bounded wait).
-    if (tid == 0) {
-      mma_commit(drain_bar);
-      mbar_wait(drain_bar, 0, a.err);
-    }
+    if (!ok) *abort_flag = 1;
   }
   tc_fence_before();
   __syncthreads();

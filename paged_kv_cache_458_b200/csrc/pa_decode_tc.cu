@@ -30,11 +30,13 @@
 // folds row d of O^T into registers, rescaled by 2^(m_old - m_new).  On other
 // tiles nothing waits for the PV product: it is read once, at the end of the
 // item.  The products are pipelined by tile: S^T(j+1) is issued as soon as
-// every thread has read S^T(j), while tile j's softmax runs.
+// every thread has read S^T(j), while tile j's softmax runs, and the softmax
+// of tile j waits for O^T(j-1) only to store P(j) (or to fold O^T).
 // The probabilities enter the PV product as two terms of the input type, hi =
 // round(p) and lo = round(p - hi), so they carry about 16 significant bits (a
-// bf16 P alone, 8 bits, can move a short context's output by more than 2e-3);
-// the tensor cores have ample room for the second set of MMAs.
+// bf16 P alone, 8 bits, can move a short context's output by more than 2e-3).
+// The two terms sit side by side as 2N columns of one PV product, so each V
+// slice is read once for both, into O^T hi and O^T lo, summed when O^T is read.
 //
 // Work, plain kernel: items (sequence, kv head, partition of partition_tokens
 // tokens, a multiple of 128) are numbered as in the CUDA-core kernel (partition
@@ -90,12 +92,13 @@ struct Warps {
 };
 
 // Per kernel kind: N columns, sequences per launch (their prefix sums live in
-// shared memory) and TMEM columns (S^T in [0, N), O^T in [N, 2N)).
+// shared memory) and TMEM columns (S^T in [0, N); O^T in [N, 3N), its hi part
+// in [N, 2N) and its lo part in [2N, 3N), rounded up to a power of two).
 template <bool GROUP>
 struct Cfg {
   static constexpr int kN = GROUP ? 32 : 16;
   static constexpr int kMaxSeqs = GROUP ? kSharedPrefixSeqsPerLaunch : 512;
-  static constexpr uint32_t kTmemCols = GROUP ? 64 : 32;
+  static constexpr uint32_t kTmemCols = GROUP ? 128 : 64;
 };
 
 template <int NST, int N, int MAXSEQS>
@@ -311,7 +314,9 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   using L = Layout<NST, N, C::kMaxSeqs>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr uint32_t kIdescQK = instr_desc(kBf16 ? 1 : 0, 0, 0, kTile, N);
-  constexpr uint32_t kIdescPV = instr_desc(kBf16 ? 1 : 0, 1, 1, kTile, N);
+  // PV has 2N columns: P hi and P lo sit in consecutive 16-column atoms, so one
+  // MMA reads each V slice once for both and writes O^T hi and O^T lo side by side
+  constexpr uint32_t kIdescPV = instr_desc(kBf16 ? 1 : 0, 1, 1, kTile, 2 * N);
   static_assert(GROUP || G <= N, "query heads per tile");
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -614,12 +619,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           const uint32_t vt = sm_stages + st * L::kStageBytes + 2 * L::kHalf;
           const uint32_t acc0 = (uint32_t)acc_flag[g & 1];
 #pragma unroll
-          for (int part_p = 0; part_p < 2; ++part_p)  // P = hi + lo
-#pragma unroll
-            for (int kk = 0; kk < kTile / 16; ++kk)
-              mma_f16(tmem + N, smem_desc(vt + kk * 2048, L::kHalf, 1024, kSw128),
-                      smem_desc(sm_p + part_p * L::kPBytes + kk * 512, L::kPAtom, 256, kSw32),
-                      kIdescPV, acc0 | (uint32_t)(part_p > 0 || kk > 0));
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_f16(tmem + N, smem_desc(vt + kk * 2048, L::kHalf, 1024, kSw128),
+                    smem_desc(sm_p + kk * 512, L::kPAtom, 256, kSw32), kIdescPV,
+                    acc0 | (uint32_t)(kk > 0));
           mma_commit(pv_bar);
           mma_commit(empty_bar(st));  // the stage is free once these MMAs are done
         }
@@ -671,15 +674,16 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
       for (int c = 0; c < NCW; ++c) acc[c] = 0.f, l_tok[c] = 0.f, m_ref[c] = -INFINITY;
       bool pv_acc = false;  // O^T in TMEM holds tiles not folded into acc yet
+      bool ok_w = true;     // every wait of this warp so far succeeded
 
       for (int j = 0; j < n_tiles; ++j, ++g) {
         const int st = g % NST;
         const int n_valid = min(kTile, t_end - (t_begin + j * kTile));
-        // ---- S^T(g); and O^T(g-1), the last reader of P and the last writer
-        // of O^T, is done.  Each warp waits on its own; the OR-barrier then
-        // makes every compute thread take the same way out if any wait failed.
+        // ---- S^T(g).  Each warp waits on its own; the OR-barrier then makes
+        // every compute thread take the same way out if this or an earlier
+        // wait of its warp failed.
         float sv[NCW];
-        bool ok_w = warp_wait(qk_bar, g & 1);
+        if (ok_w) ok_w = warp_wait(qk_bar, g & 1);
         if (ok_w) {
           tc_fence_after();
           tmem_ld<NCW>(tmem + t_lane + (uint32_t)c0, sv);
@@ -687,8 +691,11 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free_bar);  // S^T(g) read: the MMA warp may reuse it
-        if (ok_w && j > 0) ok_w = warp_wait(pv_bar, (g - 1) & 1);
         if (named_barrier_or(1, kComputeThreads, !ok_w || *abort_flag)) { ok = false; break; }
+        // O^T(g-1), the last reader of P and the last writer of O^T, is
+        // waited for only where this tile needs it: before O^T is folded and
+        // before P(g) is written
+        bool pv_done = j == 0;
         const bool valid = t < n_valid;
         bool over = false;
 #pragma unroll
@@ -719,12 +726,14 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
             l_tok[c] *= alpha[c];
           }
           if (pv_acc) {
-            // fold O^T (tiles before g, complete) into acc, on the new reference
+            // fold O^T (tiles before g) into acc, on the new reference
+            if (!pv_done) ok_w = warp_wait(pv_bar, (g - 1) & 1), pv_done = true;
             tc_fence_after();
-            float ov[NCW];
+            float ov[NCW], ow[NCW];
             tmem_ld<NCW>(tmem + t_lane + (uint32_t)(N + c0), ov);
+            tmem_ld<NCW>(tmem + t_lane + (uint32_t)(2 * N + c0), ow);
 #pragma unroll
-            for (int c = 0; c < NCW; ++c) acc[c] = (acc[c] + ov[c]) * alpha[c];
+            for (int c = 0; c < NCW; ++c) acc[c] = (acc[c] + (ov[c] + ow[c])) * alpha[c];
           } else {
 #pragma unroll
             for (int c = 0; c < NCW; ++c) acc[c] *= alpha[c];
@@ -755,6 +764,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
             const float2 r = Elem<T>::to_f2(hi[i]);
             lo[i] = pack2(x0 - r.x, x1 - r.y, kBf16);
           }
+          // P is free once O^T(g-1) is done; a failed wait is acted on at the
+          // next OR-barrier (the stores below then only race with an MMA whose
+          // result is discarded)
+          if (!pv_done) ok_w = warp_wait(pv_bar, (g - 1) & 1), pv_done = true;
           if constexpr (NCW == 8) {
             *reinterpret_cast<uint4*>(prow) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
             *reinterpret_cast<uint4*>(prow + L::kPBytes) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
@@ -788,13 +801,14 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
 
       // ---- item result: fold the last O^T, reduce the per-token sums, write
       if (tid == 0 && n_tiles > 0) ok = mbar_wait_or_abort(pv_bar, (g - 1) & 1, a.err, abort_flag);
-      if (named_barrier_or(1, kComputeThreads, !ok || *abort_flag)) { ok = false; break; }
+      if (named_barrier_or(1, kComputeThreads, !ok || !ok_w || *abort_flag)) { ok = false; break; }
       if (n_tiles > 0) {
         tc_fence_after();
-        float ov[NCW];
+        float ov[NCW], ow[NCW];
         tmem_ld<NCW>(tmem + t_lane + (uint32_t)(N + c0), ov);
+        tmem_ld<NCW>(tmem + t_lane + (uint32_t)(2 * N + c0), ow);
 #pragma unroll
-        for (int c = 0; c < NCW; ++c) acc[c] += ov[c];
+        for (int c = 0; c < NCW; ++c) acc[c] += ov[c] + ow[c];
         tc_fence_before();
       }
       {

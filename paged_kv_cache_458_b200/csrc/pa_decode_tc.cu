@@ -43,12 +43,13 @@
 // 0 of every (sequence, kv head) first, then the further partitions of longer
 // sequences).  Shared-prefix kernel: items (group leader, kv head, partition of
 // the shared tokens), numbered over the leaders of the launch.  One persistent
-// CTA per SM: a producer warp takes items (its first one by number, then from a
-// counter in the workspace whose value carries the call's epoch), resolves each
-// 16-token group of an item through the block table and issues per 128-token
-// tile 32 tiled TMA loads (8 groups x {K, V} x two 64-element halves,
-// 128B-swizzled) into one of NST stages, plus the item's query rows into an
-// item slot.  A dedicated MMA warp issues every MMA and commits it to an
+// CTA per SM: a scheduler warp takes items (its first one by number, then from
+// a counter in the workspace whose value carries the call's epoch), resolves
+// each 16-token group of an item through the block table and fills one of two
+// item slots (descriptor, pool rows, query rows), up to two items ahead; a
+// producer warp then only issues, per 128-token tile, 32 tiled TMA loads
+// (8 groups x {K, V} x two 64-element halves, 128B-swizzled) into one of NST
+// stages, the per-SM rate of which bounds the kernel.  A dedicated MMA warp issues every MMA and commits it to an
 // mbarrier, so issuing them never holds up the softmax; the compute warps
 // consume tiles in order and tell it through two more mbarriers when S^T(g)
 // has been read and when P(g) has been written.  Tokens at or past the end of
@@ -65,6 +66,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <type_traits>
 
 #include "pa_common.cuh"
@@ -87,7 +89,7 @@ struct Warps {
   static constexpr int kNCW = NC >= 16 ? 8 : (NC >= 8 ? 4 : NC);  // columns per warpgroup
   static constexpr int kNWG = NC / kNCW;                           // compute warpgroups
   static constexpr int kCompute = 128 * kNWG;                      // compute threads
-  static constexpr int kThreads = kCompute + 64;                   // + MMA warp + producer warp
+  static constexpr int kThreads = kCompute + 96;                   // + MMA, producer, scheduler warps
   static_assert(kNCW * kNWG == NC, "columns split evenly");
 };
 
@@ -101,7 +103,7 @@ struct Cfg {
   static constexpr uint32_t kTmemCols = GROUP ? 128 : 64;
 };
 
-template <int NST, int N, int MAXSEQS>
+template <int NST, int N>
 struct Layout {
   // offsets from a 1024-byte aligned base
   static constexpr int kStageBytes = 2 * kTile * kD * 2;      // K tile then V tile (64 KB)
@@ -115,10 +117,12 @@ struct Layout {
   static constexpr int kRed = kP + 2 * kPBytes;                // [4 warps][N] f32
   static constexpr int kStat = kRed + 4 * N * 4;               // m[N], then alpha[N] or l[N], f32
   static constexpr int kDesc = kStat + 2 * N * 4;              // [slots][8] int
-  static constexpr int kPrefix = kDesc + kSlots * 8 * 4;       // [MAXSEQS + 1] int
-  static constexpr int kBars = (kPrefix + (MAXSEQS + 1) * 4 + 7) / 8 * 8;
-  // full[NST], empty[NST], ready[slots], free[slots], qk, pv, drain, s_free, p_ready
-  static constexpr int kNumBars = 2 * NST + 2 * kSlots + 5;
+  static constexpr int kRows = kDesc + kSlots * 8 * 4;         // [slots][2][32] int: pool rows of
+                                                               // the item's 16-token groups
+  static constexpr int kBars = kRows + kSlots * 2 * 32 * 4;
+  // full[NST], empty[NST], ready[slots], free[slots], meta[slots], qk, pv, drain,
+  // s_free, p_ready
+  static constexpr int kNumBars = 2 * NST + 3 * kSlots + 5;
   static constexpr int kMisc = kBars + kNumBars * 8;           // tmem address, abort flag,
                                                                // accumulate flags [2]
   static constexpr int kUsed = kMisc + 16;
@@ -265,9 +269,12 @@ __device__ __forceinline__ float column_reduce(float (&v)[NC], int lane) {
 // Item number -> (sequence, kv head, partition); see the file comment.  The
 // first n_first numbers are partition 0 of every (sequence, kv head); the
 // rest are counted by prefix[] (prefix[s] = items of sequences before s, per
-// kv head), numbered from `part0` within a sequence.
-__device__ __forceinline__ void locate(int f, int n_first, int Hkv, int S, const int* prefix, int part0,
-                                       int& s, int& kvh, int& part) {
+// kv head, non-decreasing), numbered from `part0` within a sequence.  The
+// warp holds prefix[] in registers: lane l has prefix[32 k + l] in pre[k]
+// (INT_MAX past prefix[S]).  Called by all 32 lanes.
+template <int PPL>
+__device__ __forceinline__ void locate(int f, int n_first, int Hkv, const int (&pre)[PPL], int part0,
+                                       int lane, int& s, int& kvh, int& part) {
   if (f < n_first) {
     s = f / Hkv;
     kvh = f % Hkv;
@@ -277,13 +284,16 @@ __device__ __forceinline__ void locate(int f, int n_first, int Hkv, int S, const
   const int g = f - n_first;
   kvh = g % Hkv;
   const int r = g / Hkv;
-  int lo = 0, hi = S;  // largest s with prefix[s] <= r
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (prefix[mid] <= r) lo = mid; else hi = mid;
-  }
-  s = lo;
-  part = part0 + r - prefix[lo];
+  // largest s with prefix[s] <= r: the number of such entries, less one
+  int cnt = 0;
+#pragma unroll
+  for (int k = 0; k < PPL; ++k) cnt += pre[k] <= r ? 1 : 0;
+  s = __reduce_add_sync(0xffffffffu, cnt) - 1;
+  int mine = 0;
+#pragma unroll
+  for (int k = 0; k < PPL; ++k)
+    if (k == (s >> 5)) mine = pre[k];
+  part = part0 + r - __shfl_sync(0xffffffffu, mine, s & 31);
 }
 
 // Work counter tagged with the call's epoch in bits 24..63 (see pa_decode.cu).
@@ -310,8 +320,9 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   using W = Warps<NC>;
   constexpr int kComputeThreads = W::kCompute, kThreads = W::kThreads, NCW = W::kNCW;
   constexpr int kComputeWarps = kComputeThreads / 32;
-  constexpr int kMmaWarp = kComputeWarps, kProducerWarp = kComputeWarps + 1;
-  using L = Layout<NST, N, C::kMaxSeqs>;
+  constexpr int kMmaWarp = kComputeWarps, kProducerWarp = kComputeWarps + 1,
+                kSchedWarp = kComputeWarps + 2;
+  using L = Layout<NST, N>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr uint32_t kIdescQK = instr_desc(kBf16 ? 1 : 0, 0, 0, kTile, N);
   // PV has 2N columns: P hi and P lo sit in consecutive 16-column atoms, so one
@@ -327,7 +338,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = a.num_seqs, Hkv = a.num_kv_heads, PT = a.partition_tokens;
   int* desc_all = reinterpret_cast<int*>(smem + L::kDesc);
-  int* prefix = reinterpret_cast<int*>(smem + L::kPrefix);
+  int* rows_all = reinterpret_cast<int*>(smem + L::kRows);
   float* red = reinterpret_cast<float*>(smem + L::kRed);
   float* stat = reinterpret_cast<float*>(smem + L::kStat);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
@@ -337,7 +348,8 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   auto empty_bar = [&](int st) { return bars + (NST + st) * 8; };
   auto ready_bar = [&](int sl) { return bars + (2 * NST + sl) * 8; };
   auto free_bar = [&](int sl) { return bars + (2 * NST + kSlots + sl) * 8; };
-  const uint32_t qk_bar = bars + (2 * NST + 2 * kSlots) * 8;
+  auto meta_bar = [&](int sl) { return bars + (2 * NST + 2 * kSlots + sl) * 8; };
+  const uint32_t qk_bar = bars + (2 * NST + 3 * kSlots) * 8;
   const uint32_t pv_bar = qk_bar + 8;
   const uint32_t drain_bar = qk_bar + 16;
   const uint32_t s_free_bar = qk_bar + 24;   // compute warps have read S^T(g)
@@ -362,6 +374,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     for (int sl = 0; sl < kSlots; ++sl) {
       mbar_init(ready_bar(sl), 1);
       mbar_init(free_bar(sl), kComputeWarps);
+      mbar_init(meta_bar(sl), 1);
     }
     mbar_init(qk_bar, 1);
     mbar_init(pv_bar, 1);
@@ -389,16 +402,22 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == kProducerWarp) {
+  if (warp == kSchedWarp) {
     // =====================================================================
-    // producer warp: items, table entries, query rows, TMA loads
+    // scheduler warp: takes items, resolves them (sequence, kv head, token
+    // range, the pool row of each 16-token group) and fills an item slot:
+    // descriptor and rows (meta, for the producer), query rows (ready, for
+    // the MMA and compute warps).  It runs up to two items ahead of the
+    // compute warps, so none of its global round trips holds up the loads.
     // =====================================================================
     // Per sequence, the items numbered through prefix[]: further partitions
     // (plain) or the shared partitions of a group leader (shared-prefix).
+    constexpr int PPL = C::kMaxSeqs / 32 + 1;  // prefix[0..S] over the lanes
+    int pre[PPL];
     int carry = 0;
-    if (lane == 0) prefix[0] = 0;
-    for (int base = 0; base < S; base += 32) {
-      const int s = base + lane;
+#pragma unroll
+    for (int k = 0; k < PPL; ++k) {
+      const int s = k * 32 + lane;  // this lane's entry prefix[s] = carry + counts before s
       int cnt = 0;
       if (s < S) {
         if constexpr (GROUP) {
@@ -419,33 +438,36 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         const int t = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += t;
       }
-      if (s < S) prefix[s + 1] = carry + incl;
+      pre[k] = s <= S ? carry + incl - cnt : INT_MAX;
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    __syncwarp();
     const int n_first = GROUP ? 0 : S * Hkv;
     const int total = n_first + Hkv * carry;
 
-    int issued = 0;  // tiles armed so far (stage ring position)
     bool ok = true;
+    int it = 0;
     int f = blockIdx.x;
-    for (int it = 0;; ++it) {
+    for (;; ++it) {
       const int slot = it % kSlots;
-      if (it >= kSlots &&
-          !mbar_wait_or_abort(free_bar(slot), ((it / kSlots) - 1) & 1, a.err, abort_flag)) {
-        ok = false;
-        break;
+      if (it >= kSlots) {
+        bool w = true;
+        if (lane == 0) w = mbar_wait_or_abort(free_bar(slot), ((it / kSlots) - 1) & 1, a.err, abort_flag);
+        if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
+          ok = false;
+          break;
+        }
       }
       int* desc = desc_all + slot * 8;
       if (f >= total) {
         if (lane == 0) {
           desc[kDTiles] = -1;  // end of work
+          mbar_arrive(meta_bar(slot));
           mbar_arrive(ready_bar(slot));
         }
         break;
       }
       int s, kvh, part;
-      locate(f, n_first, Hkv, S, prefix, GROUP ? 0 : 1, s, kvh, part);
+      locate(f, n_first, Hkv, pre, GROUP ? 0 : 1, lane, s, kvh, part);
       int t_end, ctx_or_members;
       const int t_begin = part * PT;
       if constexpr (GROUP) {
@@ -471,12 +493,12 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         }
         return blk * a.block_size + tok % a.block_size;
       };
-      int my_row = 0, my_row2 = 0;
       if (lane < n_groups) {
         const int tok = t_begin + lane * kGroupRows;
-        my_row = resolve(tok);
-        if (a.half_boxes)
-          my_row2 = tok + kGroupRows / 2 < t_end ? resolve(tok + kGroupRows / 2) : my_row;
+        const int row = resolve(tok);
+        int* rows = rows_all + slot * 64;
+        rows[lane] = row;
+        if (a.half_boxes) rows[32 + lane] = tok + kGroupRows / 2 < t_end ? resolve(tok + kGroupRows / 2) : row;
       }
       if constexpr (GROUP) {
         // members x g query rows, 16-byte pieces stored in the 128B-swizzled
@@ -494,7 +516,6 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                        : "memory");
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
       }
       // shared-prefix item: bit m set when member m's result is this
       // partition alone (written directly, not as a split-K partial)
@@ -507,6 +528,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         }
         direct_mask = (int)__ballot_sync(0xffffffffu, dm);
       }
+      __syncwarp();  // every lane's rows (and query rows) before the arrivals
       if (lane == 0) {
         desc[kDS] = s;
         desc[kDKvh] = kvh;
@@ -516,6 +538,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         desc[kDTiles] = n_tiles;
         desc[kDParts] = GROUP ? direct_mask : (ctx_or_members + PT - 1) / PT;
         desc[kDCtx] = ctx_or_members;
+        mbar_arrive(meta_bar(slot));
         const uint32_t rb = ready_bar(slot);
         if constexpr (GROUP) {
           mbar_arrive(rb);
@@ -526,6 +549,46 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           tma_load_2d(sm_q + slot * L::kQBytes + N * 128, &tm_q, rb, 64, qrow);
         }
       }
+      int nf = 0;
+      if (lane == 0) {
+        const int t = take_item(a.work_counter, a.epoch, a.err);
+        nf = t < 0 ? total : (int)gridDim.x + t;
+      }
+      f = __shfl_sync(0xffffffffu, nf, 0);
+    }
+    if (!ok) *abort_flag = 1;
+    // The query rows this warp loaded by TMA land before the CTA leaves
+    // (bounded waits).  Items it-2 and it-1 may still be in flight, unless the
+    // end-of-work mark went into item it-2's slot: that needed the slot freed,
+    // so its rows had landed, and its phase parity now names a later phase.
+    if (!GROUP && lane == 0)
+      for (int k = max(0, it - (ok ? 1 : kSlots)); k < it; ++k)
+        mbar_wait(ready_bar(k % kSlots), (k / kSlots) & 1, a.err);
+  } else if (warp == kProducerWarp) {
+    // =====================================================================
+    // producer warp: the K/V tiles of each item, from the rows the scheduler
+    // resolved, by TMA into the stage ring
+    // =====================================================================
+    int issued = 0;  // tiles armed so far (stage ring position)
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+      const int slot = it % kSlots;
+      {
+        bool w = true;
+        if (lane == 0) w = mbar_wait_or_abort(meta_bar(slot), (it / kSlots) & 1, a.err, abort_flag);
+        if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
+          ok = false;
+          break;
+        }
+        __syncwarp();  // lane 0's acquire orders the other lanes' reads below
+      }
+      const int* desc = desc_all + slot * 8;
+      const int n_tiles = desc[kDTiles];
+      if (n_tiles < 0) break;  // end of work
+      const int kvh = desc[kDKvh];
+      const int n_groups = (desc[kDEnd] - desc[kDBegin] + kGroupRows - 1) / kGroupRows;
+      const int my_row = rows_all[slot * 64 + lane];
+      const int my_row2 = a.half_boxes ? rows_all[slot * 64 + 32 + lane] : 0;
       for (int j = 0; j < n_tiles && ok; ++j) {
         const int st = issued % NST;
         if (issued >= NST &&
@@ -553,13 +616,6 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         }
         ++issued;
       }
-      if (!ok) break;
-      int nf = 0;
-      if (lane == 0) {
-        const int t = take_item(a.work_counter, a.epoch, a.err);
-        nf = t < 0 ? total : (int)gridDim.x + t;
-      }
-      f = __shfl_sync(0xffffffffu, nf, 0);
     }
     if (!ok) *abort_flag = 1;
     // Every TMA copy armed by this warp lands before the CTA leaves.
@@ -881,7 +937,7 @@ template <typename T, int G, bool GROUP>
 cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& tq, cudaStream_t stream, int* launches) {
   using C = Cfg<GROUP>;
-  using L = Layout<kStagesTc, C::kN, C::kMaxSeqs>;
+  using L = Layout<kStagesTc, C::kN>;
   auto* kern = decode_tc_kernel<T, G, kStagesTc, GROUP>;
   static bool configured = false;
   if (!configured) {

@@ -118,15 +118,17 @@ typedef enum { PA_CACHE_AS_DTYPE = 0, PA_CACHE_FP8_E4M3 = 1 } pa_cache_format;
 /* How pa_decode computes QK^T and PV.  Both variants read K/V with tiled TMA
  * loads through the block table and keep the softmax in fp32.
  *  PA_DECODE_AUTO          tensor cores when head_dim == 128, the group
- *                          g = Hq / Hkv is at least 8 and partition_tokens is
- *                          a multiple of 128 up to 512; CUDA cores otherwise.
+ *                          g = Hq / Hkv is at least 8 (at least 4 when
+ *                          block_size is a multiple of 16) and
+ *                          partition_tokens is a multiple of 128 up to 512;
+ *                          CUDA cores otherwise.
  *  PA_DECODE_CUDA_CORES    fp32 FMA on the CUDA cores (any built shape).
  *  PA_DECODE_TENSOR_CORES  tcgen05 MMA with the g heads padded to 16: fp16/bf16
- *                          operands (the probabilities are rounded to the
- *                          input type before the PV product), fp32
- *                          accumulators in tensor memory.  Needs head_dim 128
- *                          and partition_tokens a multiple of 128 (else
- *                          PA_ERR_UNSUPPORTED). */
+ *                          operands (the probabilities enter the PV product as
+ *                          two terms of the input type, hi + lo, about 16
+ *                          significant bits), fp32 accumulators in tensor
+ *                          memory.  Needs head_dim 128 and partition_tokens a
+ *                          multiple of 128 up to 512 (else PA_ERR_UNSUPPORTED). */
 typedef enum { PA_DECODE_AUTO = 0, PA_DECODE_CUDA_CORES = 1, PA_DECODE_TENSOR_CORES = 2 } pa_decode_variant;
 
 /* The split-K partition pa_decode() uses for `shape` (partition_tokens, or

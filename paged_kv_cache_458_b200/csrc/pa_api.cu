@@ -56,6 +56,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // Whether the tensor-core kernels run, with partition_tokens == 0 read as
 // "their default"; defined below.
 bool tensor_core_kernel(const pa_shape* s, int pt);
+int box_rows(const pa_shape* s);
 
 // partition_tokens, or its default: 512 for the tensor-core kernels (their
 // largest item), 1024 for the CUDA-core kernel, where fewer partials measured
@@ -116,9 +117,12 @@ bool tensor_core_kernel(const pa_shape* s, int pt) {
   if (s->cache_format == PA_CACHE_FP8_E4M3) return false;
   if (s->variant == PA_DECODE_TENSOR_CORES) return true;
   if (s->variant == PA_DECODE_CUDA_CORES) return false;
-  // measured: tensor cores win from group 8 up; at group 4 the CUDA-core
-  // kernel still keeps up with HBM
-  return s->head_dim == 128 && s->num_q_heads / s->num_kv_heads >= 8 &&
+  // measured: tensor cores win from group 8 up, and at group 4 with 16-token
+  // TMA boxes (mistral_7b_gqa: 5187 vs 4977 GB/s).  With 8-token blocks the
+  // tensor-core kernel issues twice as many half-size boxes, and at group 4
+  // that costs more than the MMAs save (3602 vs 4890 GB/s).
+  const int g = s->num_q_heads / s->num_kv_heads;
+  return s->head_dim == 128 && (g >= 8 || (g >= 4 && box_rows(s) == 16)) &&
          pt % pa::decode_tc_tile_tokens() == 0 && pt <= 512;
 }
 

@@ -110,9 +110,10 @@ def test_fp8_cache_validation(lib):
                                    None) == pa.PA_ERR_INVALID_ARG
     assert lib.pa_cache_append_fp8(FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, ctypes.byref(s8),
                                    None) == pa.PA_OK
-    # the workspace does not depend on the cache format
+    # the workspace depends on the cache format only through the default
+    # partition (an E4M3 pool always takes the CUDA-core kernel)
     assert lib.pa_decode_workspace_bytes(ctypes.byref(s8), 1000) == \
-        lib.pa_decode_workspace_bytes(ctypes.byref(s16), 1000)
+        lib.pa_decode_workspace_bytes(ctypes.byref(_shape(variant=1)), 1000)
 
 
 def test_multi_query_workspace_and_validation(lib):
@@ -161,7 +162,8 @@ def test_swap_validation(lib):
 
 
 def test_default_partition(lib):
-    assert pa.pa_decode_partition_tokens(_shape()) == 1024                     # CUDA cores
+    assert pa.pa_decode_partition_tokens(_shape()) == 512                      # tensor cores (group 4)
+    assert pa.pa_decode_partition_tokens(_shape(num_q_heads=4)) == 1024        # CUDA cores (group 2)
     assert pa.pa_decode_partition_tokens(_shape(num_q_heads=16)) == 512        # tensor cores
     assert pa.pa_decode_partition_tokens(_shape(shared_prefix=1)) == 512
     assert pa.pa_decode_partition_tokens(_shape(partition_tokens=48)) == 48
@@ -169,7 +171,11 @@ def test_default_partition(lib):
 
 
 def test_resolved_variant(lib):
-    assert pa.pa_decode_resolved_variant(_shape()) == pa.PA_DECODE_CUDA_CORES          # group 4
+    assert pa.pa_decode_resolved_variant(_shape()) == pa.PA_DECODE_TENSOR_CORES        # group 4
+    assert pa.pa_decode_resolved_variant(_shape(num_q_heads=4)) == pa.PA_DECODE_CUDA_CORES  # group 2
+    # 8-token blocks: tensor cores from group 8 only
+    assert pa.pa_decode_resolved_variant(_shape(block_size=8)) == pa.PA_DECODE_CUDA_CORES
+    assert pa.pa_decode_resolved_variant(_shape(block_size=8, num_q_heads=16)) == pa.PA_DECODE_TENSOR_CORES
     assert pa.pa_decode_resolved_variant(_shape(num_q_heads=16)) == pa.PA_DECODE_TENSOR_CORES
     assert pa.pa_decode_resolved_variant(_shape(num_q_heads=16, head_dim=64)) == pa.PA_DECODE_CUDA_CORES
     assert pa.pa_decode_resolved_variant(_shape(num_q_heads=16, partition_tokens=1024)) == pa.PA_DECODE_CUDA_CORES
@@ -195,10 +201,10 @@ def test_decode_rejects_bad_pointers_and_sizes(lib):
     st = lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s), 100, None, 0, None)
     assert st == pa.PA_ERR_INVALID_ARG
     # ... 2000 tokens need two default (1024-token, CUDA-core) partitions and split-K space
-    s2 = _shape(max_blocks_per_seq=128)
+    s2 = _shape(max_blocks_per_seq=128, num_q_heads=4)  # group 2
     assert lib.pa_decode_workspace_bytes(ctypes.byref(s2), 1024) == 256
     need = lib.pa_decode_workspace_bytes(ctypes.byref(s2), 2000)
-    rows = 4 * 8 * 2
+    rows = 4 * 4 * 2
     assert need == 256 + rows * 128 * 4 + rows * 2 * 4
     st = lib.pa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s2), 2000, FAKE, need - 1, None)
     assert st == pa.PA_ERR_INVALID_ARG

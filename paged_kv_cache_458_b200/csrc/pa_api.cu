@@ -207,15 +207,24 @@ bool make_pool_map(CUtensorMap* map, const void* pool, const pa_shape* s, int ro
 // [S * Hq][128] with 128B-swizzled boxes of 64 elements x `group` rows.
 // TMA box rows over the pool: 16 (one box per 16-token group), or 8 when
 // blocks hold a multiple of 8 but not of 16 tokens (two boxes per group).
+// With `pair` (items of two kv heads) the pools are viewed with the head as
+// the outer dimension, [Hkv][NB * bs][128] by strides, so that one box holds
+// 16 rows of one head and then the same rows of the next (4 KB instead of
+// 2 KB: the per-SM box rate bounds this kernel), and a q box holds 2 x group
+// rows.
 int box_rows(const pa_shape* s) { return s->block_size % 16 == 0 ? 16 : 8; }
 
 bool make_tc_maps(CUtensorMap* tk, CUtensorMap* tv, CUtensorMap* tq, const void* k, const void* v,
-                  const void* q, const pa_shape* s) {
+                  const void* q, const pa_shape* s, bool pair) {
   auto fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[3] = {128, (cuuint64_t)s->num_kv_heads, (cuuint64_t)s->num_blocks * s->block_size};
-  const cuuint64_t strides[2] = {256, (cuuint64_t)s->num_kv_heads * 256};
-  const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows(s)};
+  const cuuint64_t rows = (cuuint64_t)s->num_blocks * s->block_size, Hkv = (cuuint64_t)s->num_kv_heads;
+  const cuuint64_t dims_h[3] = {128, Hkv, rows}, dims_p[3] = {128, rows, Hkv};
+  const cuuint64_t strides_h[2] = {256, Hkv * 256}, strides_p[2] = {Hkv * 256, 256};
+  const cuuint32_t box_h[3] = {64, 1, (cuuint32_t)box_rows(s)}, box_p[3] = {64, 16, 2};
+  const cuuint64_t* dims = pair ? dims_p : dims_h;
+  const cuuint64_t* strides = pair ? strides_p : strides_h;
+  const cuuint32_t* box = pair ? box_p : box_h;
   const cuuint32_t estr[3] = {1, 1, 1};
   for (int i = 0; i < 2; ++i) {
     CUresult r = fn(i ? tv : tk, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(i ? v : k), dims,
@@ -225,7 +234,7 @@ bool make_tc_maps(CUtensorMap* tk, CUtensorMap* tv, CUtensorMap* tq, const void*
   }
   const cuuint64_t qdims[2] = {128, (cuuint64_t)s->num_seqs * s->num_q_heads};
   const cuuint64_t qstrides[1] = {256};
-  const cuuint32_t qbox[2] = {64, (cuuint32_t)(s->num_q_heads / s->num_kv_heads)};
+  const cuuint32_t qbox[2] = {64, (cuuint32_t)((pair ? 2 : 1) * (s->num_q_heads / s->num_kv_heads))};
   const cuuint32_t qestr[2] = {1, 1};
   return fn(tq, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(q), qdims, qstrides, qbox, qestr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -329,7 +338,7 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
     // plan the groups, then their shared tokens on tensor cores, then every
     // sequence's own tokens on CUDA cores, then the merge
     CUtensorMap tk, tv, tq, pk, pv;
-    if (!make_tc_maps(&tk, &tv, &tq, k_cache, v_cache, q, shape) ||
+    if (!make_tc_maps(&tk, &tv, &tq, k_cache, v_cache, q, shape, false) ||
         !make_pool_map(&pk, k_cache, shape, box_rows(shape)) ||
         !make_pool_map(&pv, v_cache, shape, box_rows(shape)))
       return cuda_failed("cuTensorMapEncodeTiled failed");
@@ -354,11 +363,14 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
     if (e == cudaSuccess)
       e = pa::launch_decode(a, shape->dtype, shape->head_dim, group, pk, pv, cs, &launched);
   } else if (use_tensor_cores(shape) && shape->num_blocks > 0) {
+    // items of two kv heads (4 KB boxes) where the heads pair up, the group
+    // fits 16 columns twice and blocks give 16-row boxes
+    const bool pair = shape->num_kv_heads % 2 == 0 && group <= 8 && !a.half_boxes;
     CUtensorMap tk, tv, tq;
-    if (!make_tc_maps(&tk, &tv, &tq, k_cache, v_cache, q, shape))
+    if (!make_tc_maps(&tk, &tv, &tq, k_cache, v_cache, q, shape, pair))
       return cuda_failed("cuTensorMapEncodeTiled failed");
     a.epoch = next_epochs((shape->num_seqs + 511) / 512);
-    e = pa::launch_decode_tc(a, shape->dtype, group, tk, tv, tq, cs, &launched);
+    e = pa::launch_decode_tc(a, shape->dtype, group, tk, tv, tq, cs, &launched, pair);
     if (e == cudaSuccess) e = pa::launch_decode_merge(a, shape->dtype, shape->head_dim, cs, &launched);
   } else {
     CUtensorMap tk, tv;

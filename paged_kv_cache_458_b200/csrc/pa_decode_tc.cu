@@ -12,6 +12,13 @@
 // with fp16/bf16 operands and fp32 accumulators in tensor memory (TMEM).  The
 // N columns are query rows:
 //   - one sequence (the plain kernel): its g query heads, padded to N = 16;
+//     or, where the kv heads pair up and 2g <= 16, the 2g query heads of two
+//     kv heads.  Then a tile is 64 tokens of both heads as the 128 MMA rows
+//     (16-row groups of head 2e and of head 2e+1 alternate), so that one TMA
+//     box carries 4 KB (16 rows of both heads) instead of 2 KB: the rate at
+//     which one SM issues boxes bounds this kernel.  A row's logits against
+//     the other head's queries are computed and discarded (p = 0), which the
+//     tensor cores can afford;
 //   - a group of sequences whose block tables begin with the same physical
 //     blocks (the shared-prefix kernel): members x g query rows, N = 32.  The
 //     blocks every member reads are then read once for all of them, which is
@@ -310,13 +317,23 @@ __device__ __forceinline__ int take_item(unsigned long long* ctr, unsigned long 
   return -1;
 }
 
-template <typename T, int G, int NST, bool GROUP>
-__global__ void __launch_bounds__(Warps<GROUP ? Cfg<GROUP>::kN : G>::kThreads, 1)
+// Query columns of a kernel kind: members x g (shared-prefix), 2g (an item of
+// two kv heads), g.
+template <int G, bool GROUP, bool PAIR>
+__host__ __device__ constexpr int columns() { return GROUP ? Cfg<GROUP>::kN : (PAIR ? 2 * G : G); }
+
+template <typename T, int G, int NST, bool GROUP, bool PAIR>
+__global__ void __launch_bounds__(Warps<columns<G, GROUP, PAIR>()>::kThreads, 1)
 decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q) {
   using C = Cfg<GROUP>;
   constexpr int N = C::kN;
-  constexpr int NC = GROUP ? N : G;  // columns that carry query rows
+  constexpr int NC = columns<G, GROUP, PAIR>();  // columns that carry query rows
+  // An item covers kHeads kv heads; a tile is kTok tokens of each, as kTile
+  // MMA rows (with two heads, 16-row groups of head 2e and head 2e+1 alternate)
+  constexpr int kHeads = PAIR ? 2 : 1;
+  constexpr int kTok = kTile / kHeads;
+  static_assert(!(GROUP && PAIR), "a shared-prefix item covers one kv head");
   using W = Warps<NC>;
   constexpr int kComputeThreads = W::kCompute, kThreads = W::kThreads, NCW = W::kNCW;
   constexpr int kComputeWarps = kComputeThreads / 32;
@@ -328,7 +345,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   // PV has 2N columns: P hi and P lo sit in consecutive 16-column atoms, so one
   // MMA reads each V slice once for both and writes O^T hi and O^T lo side by side
   constexpr uint32_t kIdescPV = instr_desc(kBf16 ? 1 : 0, 1, 1, kTile, 2 * N);
-  static_assert(GROUP || G <= N, "query heads per tile");
+  static_assert(GROUP || kHeads * G <= N, "query heads per tile");
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -386,7 +403,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   }
   // Query rows that no item fills stay zero (padded heads); a shared-prefix
   // item fills members x g rows, so the slots start all zero.
-  constexpr int kRow0 = GROUP ? 0 : G;
+  constexpr int kRow0 = GROUP ? 0 : kHeads * G;
   constexpr int kPad = N - kRow0;
   if constexpr (kPad > 0) {
     for (int i = tid; i < kSlots * 2 * kPad * 8; i += kThreads) {
@@ -441,8 +458,9 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       pre[k] = s <= S ? carry + incl - cnt : INT_MAX;
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    const int n_first = GROUP ? 0 : S * Hkv;
-    const int total = n_first + Hkv * carry;
+    const int Hitem = Hkv / kHeads;  // kv-head units of the item numbering
+    const int n_first = GROUP ? 0 : S * Hitem;
+    const int total = n_first + Hitem * carry;
 
     bool ok = true;
     int it = 0;
@@ -467,7 +485,8 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         break;
       }
       int s, kvh, part;
-      locate(f, n_first, Hkv, pre, GROUP ? 0 : 1, lane, s, kvh, part);
+      locate(f, n_first, Hitem, pre, GROUP ? 0 : 1, lane, s, kvh, part);
+      kvh *= kHeads;  // the item's first kv head
       int t_end, ctx_or_members;
       const int t_begin = part * PT;
       if constexpr (GROUP) {
@@ -480,7 +499,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         ctx_or_members = ctx;
       }
       const int n_tok = max(0, t_end - t_begin);
-      const int n_tiles = (n_tok + kTile - 1) / kTile;
+      const int n_tiles = (n_tok + kTok - 1) / kTok;
       const int n_groups = (n_tok + kGroupRows - 1) / kGroupRows;  // <= 32
       // With 8-token blocks (half_boxes) rows 8..15 of a group have their own
       // entry; past the end of the item they re-read the first block (masked).
@@ -543,7 +562,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         if constexpr (GROUP) {
           mbar_arrive(rb);
         } else {
-          mbar_arrive_expect_tx(rb, 2 * G * 128);
+          mbar_arrive_expect_tx(rb, 2 * kHeads * G * 128);
           const int qrow = (a.seq_offset + s) * a.num_q_heads + kvh * G;
           tma_load_2d(sm_q + slot * L::kQBytes, &tm_q, rb, 0, qrow);
           tma_load_2d(sm_q + slot * L::kQBytes + N * 128, &tm_q, rb, 64, qrow);
@@ -596,11 +615,12 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           ok = false;
           break;
         }
-        const int g0 = j * (kTile / kGroupRows);
-        const int ng = min(kTile / kGroupRows, n_groups - g0);
+        const int g0 = j * (kTok / kGroupRows);
+        const int ng = min(kTok / kGroupRows, n_groups - g0);
         const uint32_t fb = full_bar(st);
         const uint32_t dst = sm_stages + st * L::kStageBytes;
-        if (lane == 0) mbar_arrive_expect_tx(fb, ng * 4 * kGroupRows * 128);
+        constexpr int kBoxBytes = kHeads * kGroupRows * 128;  // one box: a group of kHeads heads
+        if (lane == 0) mbar_arrive_expect_tx(fb, ng * 4 * kBoxBytes);
         __syncwarp();
         {
           // lane 4 r + k loads piece k (K or V, 64-element half) of group r
@@ -608,10 +628,16 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           const int row = __shfl_sync(0xffffffffu, my_row, min(g0 + r, 31));
           const int row2 = __shfl_sync(0xffffffffu, my_row2, min(g0 + r, 31));
           if (r < ng) {
-            const uint32_t d = dst + k * L::kHalf + r * kGroupRows * 128;
+            const uint32_t d = dst + k * L::kHalf + r * kBoxBytes;
             const void* map = k < 2 ? &tm_k : &tm_v;
-            tma_load_3d(d, map, fb, (k & 1) * 64, kvh, row);
-            if (a.half_boxes) tma_load_3d(d + (kGroupRows / 2) * 128, map, fb, (k & 1) * 64, kvh, row2);
+            if constexpr (PAIR) {
+              // maps of this kind are [rows][head] with the head innermost
+              // after the dims: a box is 16 rows of head kvh, then of kvh + 1
+              tma_load_3d(d, map, fb, (k & 1) * 64, row, kvh);
+            } else {
+              tma_load_3d(d, map, fb, (k & 1) * 64, kvh, row);
+              if (a.half_boxes) tma_load_3d(d + (kGroupRows / 2) * 128, map, fb, (k & 1) * 64, kvh, row2);
+            }
           }
         }
         ++issued;
@@ -706,6 +732,13 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     const int c0 = cg * NCW;         // first column of this thread
     const int quarter = warp & 3;    // TMEM lane quarter of this warp
     const uint32_t t_lane = ((uint32_t)(quarter * 32) << 16);
+    // MMA row t: kv head e_row of the item, token tok_row of the tile; with
+    // two heads only the columns of head e_row are this row's logits
+    const int e_row = PAIR ? (t >> 4) & 1 : 0;
+    const int tok_row = PAIR ? ((t >> 5) << 4) + (t & 15) : t;
+    bool col_ok[NCW];
+#pragma unroll
+    for (int c = 0; c < NCW; ++c) col_ok[c] = !PAIR || (c0 + c) / G == e_row;
     int g = 0;  // tiles consumed, numbered across items
     bool ok = true;
     // one lane per warp waits on an mbarrier, the warp follows
@@ -724,7 +757,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       const int s = desc[kDS], kvh = desc[kDKvh], part = desc[kDPart];
       const int t_begin = desc[kDBegin], t_end = desc[kDEnd], n_parts = desc[kDParts];
       const int ctx_or_members = desc[kDCtx];
-      const int cols = GROUP ? ctx_or_members * G : G;
+      const int cols = GROUP ? ctx_or_members * G : kHeads * G;
 
       float acc[NCW], l_tok[NCW], m_ref[NCW];
 #pragma unroll
@@ -734,7 +767,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
 
       for (int j = 0; j < n_tiles; ++j, ++g) {
         const int st = g % NST;
-        const int n_valid = min(kTile, t_end - (t_begin + j * kTile));
+        const int n_valid = min(kTok, t_end - (t_begin + j * kTok));
         // ---- S^T(g).  Each warp waits on its own; the OR-barrier then makes
         // every compute thread take the same way out if this or an earlier
         // wait of its warp failed.
@@ -752,11 +785,11 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         // waited for only where this tile needs it: before O^T is folded and
         // before P(g) is written
         bool pv_done = j == 0;
-        const bool valid = t < n_valid;
+        const bool valid = tok_row < n_valid;
         bool over = false;
 #pragma unroll
         for (int c = 0; c < NCW; ++c) {
-          sv[c] = valid ? sv[c] * a.scale_log2 : -INFINITY;
+          sv[c] = valid && col_ok[c] ? sv[c] * a.scale_log2 : -INFINITY;
           over |= (c0 + c < cols) && (sv[c] > m_ref[c] + kRescale);
         }
         const bool rescale = named_barrier_or(1, kComputeThreads, over);
@@ -799,7 +832,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         float p[NCW];
 #pragma unroll
         for (int c = 0; c < NCW; ++c) {
-          p[c] = valid ? exp2f(sv[c] - m_ref[c]) : 0.f;
+          p[c] = valid && col_ok[c] ? exp2f(sv[c] - m_ref[c]) : 0.f;
           l_tok[c] += p[c];
         }
         // P^T rows: per 16-column atom, a 32-byte row per token (MN-major,
@@ -933,12 +966,12 @@ int sm_count() {
   return count[dev];
 }
 
-template <typename T, int G, bool GROUP>
+template <typename T, int G, bool GROUP, bool PAIR>
 cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& tq, cudaStream_t stream, int* launches) {
   using C = Cfg<GROUP>;
   using L = Layout<kStagesTc, C::kN>;
-  auto* kern = decode_tc_kernel<T, G, kStagesTc, GROUP>;
+  auto* kern = decode_tc_kernel<T, G, kStagesTc, GROUP, PAIR>;
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
@@ -962,9 +995,9 @@ cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUte
     a.epoch = a0.epoch + (unsigned long long)(s0 / kChunk);
     // plain: at least one item per (sequence, kv head); shared-prefix: the
     // number of items is only known on the device
-    const int items0 = GROUP ? sms : a.num_seqs * a.num_kv_heads;
+    const int items0 = GROUP ? sms : a.num_seqs * (a.num_kv_heads / (PAIR ? 2 : 1));
     const int grid = items0 < sms ? items0 : sms;
-    constexpr int kBlock = Warps<GROUP ? C::kN : G>::kThreads;
+    constexpr int kBlock = Warps<columns<G, GROUP, PAIR>()>::kThreads;
     cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kBlock), L::kAlloc, stream, a, tk, tv, tq);
     if (e != cudaSuccess) return e;
     ++*launches;
@@ -972,15 +1005,16 @@ cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUte
   return cudaSuccess;
 }
 
-template <typename T, bool GROUP>
+template <typename T, bool GROUP, bool PAIR>
 cudaError_t launch_group(const DecodeArgs& a, int G, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& tq, cudaStream_t st, int* n) {
   switch (G) {
-    case 1: return launch_typed<T, 1, GROUP>(a, tk, tv, tq, st, n);
-    case 2: return launch_typed<T, 2, GROUP>(a, tk, tv, tq, st, n);
-    case 4: return launch_typed<T, 4, GROUP>(a, tk, tv, tq, st, n);
-    case 8: return launch_typed<T, 8, GROUP>(a, tk, tv, tq, st, n);
-    case 16: return launch_typed<T, 16, GROUP>(a, tk, tv, tq, st, n);
+    case 1: return launch_typed<T, 1, GROUP, PAIR>(a, tk, tv, tq, st, n);
+    case 2: return launch_typed<T, 2, GROUP, PAIR>(a, tk, tv, tq, st, n);
+    case 4: return launch_typed<T, 4, GROUP, PAIR>(a, tk, tv, tq, st, n);
+    case 8: return launch_typed<T, 8, GROUP, PAIR>(a, tk, tv, tq, st, n);
+    case 16:
+      if constexpr (!PAIR) return launch_typed<T, 16, GROUP, false>(a, tk, tv, tq, st, n);
   }
   return cudaErrorInvalidValue;
 }
@@ -989,17 +1023,21 @@ cudaError_t launch_group(const DecodeArgs& a, int G, const CUtensorMap& tk, cons
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, int dtype, int group, const CUtensorMap& tk,
                              const CUtensorMap& tv, const CUtensorMap& tq, cudaStream_t stream,
-                             int* launches) {
+                             int* launches, bool pair) {
   if (a.num_seqs <= 0) return cudaSuccess;
-  if (dtype == 0) return tc::launch_group<__half, false>(a, group, tk, tv, tq, stream, launches);
-  return tc::launch_group<__nv_bfloat16, false>(a, group, tk, tv, tq, stream, launches);
+  if (pair) {
+    if (dtype == 0) return tc::launch_group<__half, false, true>(a, group, tk, tv, tq, stream, launches);
+    return tc::launch_group<__nv_bfloat16, false, true>(a, group, tk, tv, tq, stream, launches);
+  }
+  if (dtype == 0) return tc::launch_group<__half, false, false>(a, group, tk, tv, tq, stream, launches);
+  return tc::launch_group<__nv_bfloat16, false, false>(a, group, tk, tv, tq, stream, launches);
 }
 
 cudaError_t launch_decode_shared_tc(const DecodeArgs& a, int dtype, int group, const CUtensorMap& tk,
                                     const CUtensorMap& tv, cudaStream_t stream, int* launches) {
   if (a.num_seqs <= 0 || !a.plan) return cudaSuccess;
-  if (dtype == 0) return tc::launch_group<__half, true>(a, group, tk, tv, tk, stream, launches);
-  return tc::launch_group<__nv_bfloat16, true>(a, group, tk, tv, tk, stream, launches);
+  if (dtype == 0) return tc::launch_group<__half, true, false>(a, group, tk, tv, tk, stream, launches);
+  return tc::launch_group<__nv_bfloat16, true, false>(a, group, tk, tv, tk, stream, launches);
 }
 
 int decode_tc_tile_tokens() { return tc::kTile; }

@@ -95,9 +95,11 @@ cudaError_t launch_decode_merge(const DecodeArgs& a, int dtype, int head_dim, cu
 
 // The tensor-core path (head_dim 128): maps are 128B-swizzled, boxes of 64
 // elements; tq views q as [S * Hq][128] with boxes of (64 x group) elements.
+// With `pair`, items cover two kv heads: the pool maps are [Hkv][rows][128] by
+// strides with boxes of 64 x 16 rows x 2 heads, and q boxes hold 2 x group rows.
 cudaError_t launch_decode_tc(const DecodeArgs& a, int dtype, int group, const CUtensorMap& tm_k,
                              const CUtensorMap& tm_v, const CUtensorMap& tm_q, cudaStream_t stream,
-                             int* launches);
+                             int* launches, bool pair);
 int decode_tc_tile_tokens();
 // The shared-prefix kernel (a.plan set): items over the shared partitions of
 // every group, members x g query rows per tile.

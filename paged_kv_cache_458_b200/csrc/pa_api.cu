@@ -118,7 +118,7 @@ bool tensor_core_kernel(const pa_shape* s, int pt) {
   if (s->variant == PA_DECODE_TENSOR_CORES) return true;
   if (s->variant == PA_DECODE_CUDA_CORES) return false;
   // measured: tensor cores win from group 8 up, and at group 4 with 16-token
-  // TMA boxes (mistral_7b_gqa: 5187 vs 4977 GB/s).  With 8-token blocks the
+  // TMA boxes (mistral_7b_gqa: 5564 vs 4977 GB/s).  With 8-token blocks the
   // tensor-core kernel issues twice as many half-size boxes, and at group 4
   // that costs more than the MMAs save (3602 vs 4890 GB/s).
   const int g = s->num_q_heads / s->num_kv_heads;

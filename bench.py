@@ -230,6 +230,16 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def source_digest(path: str) -> str:
+    """First 16 hex digits of the SHA-256 of a kernel source without its
+    blank lines and whole-line // comments: a comment edit keeps the digest,
+    any change to code (trailing comments included) changes it."""
+    with open(path, "rb") as f:
+        lines = f.read().split(b"\n")
+    kept = [ln for ln in lines if ln.strip() and not ln.strip().startswith(b"//")]
+    return hashlib.sha256(b"\n".join(kept)).hexdigest()[:16]
+
+
 def profiled_traffic(workload: str, variant: str, step_bytes: float):
     """DRAM bytes per decode launch from the committed ncu summary of this
     workload, if it was taken on the kernel that runs (same variant, same
@@ -239,8 +249,7 @@ def profiled_traffic(workload: str, variant: str, step_bytes: float):
     try:
         with open(path) as f:
             prof = json.load(f)
-        with open(os.path.join(ROOT, prof["source"]), "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()[:16]
+        digest = source_digest(os.path.join(ROOT, prof["source"]))
     except (OSError, ValueError, KeyError):
         return None
     if prof.get("variant") != variant or prof.get("source_sha256_16") != digest:

@@ -45,19 +45,21 @@
 // The two terms sit side by side as 2N columns of one PV product, so each V
 // slice is read once for both, into O^T hi and O^T lo, summed when O^T is read.
 //
-// Work, plain kernel: items (sequence, kv head, partition of partition_tokens
-// tokens, a multiple of 128) are numbered as in the CUDA-core kernel (partition
-// 0 of every (sequence, kv head) first, then the further partitions of longer
-// sequences).  Shared-prefix kernel: items (group leader, kv head, partition of
-// the shared tokens), numbered over the leaders of the launch.  One persistent
-// CTA per SM: a scheduler warp takes items (its first one by number, then from
-// a counter in the workspace whose value carries the call's epoch), resolves
-// each 16-token group of an item through the block table and fills one of two
-// item slots (descriptor, pool rows, query rows), up to two items ahead; a
-// producer warp then only issues, per 128-token tile, 32 tiled TMA loads
-// (8 groups x {K, V} x two 64-element halves, 128B-swizzled) into one of NST
-// stages, the per-SM rate of which bounds the kernel.  A dedicated MMA warp issues every MMA and commits it to an
-// mbarrier, so issuing them never holds up the softmax; the compute warps
+// Work, plain kernel: items (sequence, kv head or pair of kv heads, partition
+// of partition_tokens tokens, a multiple of 128) are numbered as in the
+// CUDA-core kernel (partition 0 of every (sequence, kv head) first, then the
+// further partitions of longer sequences).  Shared-prefix kernel: items
+// (group leader, kv head, partition of the shared tokens), numbered over the
+// leaders of the launch.  One persistent CTA per SM: a scheduler warp takes
+// items (its first one by number, then from a counter in the workspace whose
+// value carries the call's epoch), resolves each 16-token group of an item
+// through the block table and fills one of two item slots (descriptor, pool
+// rows, query rows), up to two items ahead; a producer warp then only issues
+// the tiles' tiled TMA loads, one box per lane (per tile: 8 groups of one
+// head or 4 groups of two heads, x {K, V} x two 64-element halves,
+// 128B-swizzled), into one of NST stages.  A dedicated MMA warp issues every
+// MMA and commits it to an mbarrier, so issuing them never holds up the
+// softmax; the compute warps
 // consume tiles in order and tell it through two more mbarriers when S^T(g)
 // has been read and when P(g) has been written.  Tokens at or past the end of
 // the item are masked in P and their V rows are zeroed in shared memory before

@@ -200,6 +200,11 @@ size_t pa_decode_workspace_bytes(const pa_shape *shape, int32_t max_context_len)
  *   that runs concurrently.
  * An E4M3 cache (cache_format PA_CACHE_FP8_E4M3) needs pa_decode_fp8 and its
  * scales: pa_decode refuses it with PA_ERR_INVALID_ARG.
+ * CUDA graphs: the call may be captured (stream capture) once the same shape
+ * has run eagerly on that device, and the graph replayed any number of
+ * times.  A captured call that uses the tensor-core kernels adds a memset
+ * of the workspace's work counter to the graph, which resets it before each
+ * replay.  The same holds for pa_decode_fp8 and pa_decode_multi.
  */
 pa_status pa_decode(const void *q, const void *k_cache, const void *v_cache,
                     const int32_t *block_tables, const int32_t *context_lens, float scale,

@@ -334,6 +334,20 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   int launched = 0;
   cudaError_t e;
+  // The tensor-core kernels take items from the work counter, tagged with a
+  // per-call epoch.  Inside a CUDA graph that epoch is fixed at capture, so a
+  // replay would find the count its previous replay left under the same
+  // epoch and skip those items.  A captured call therefore zeroes the counter
+  // first: the memset becomes a node of the graph and runs before each
+  // replay's kernels (a zero word carries a foreign epoch, or the right one
+  // with a count of zero).  Eager calls keep relying on the epoch alone.
+  if (shape->num_blocks > 0 && (shape->shared_prefix || use_tensor_cores(shape))) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(cs, &cap) != cudaSuccess) return cuda_failed("cudaStreamIsCapturing failed");
+    if (cap == cudaStreamCaptureStatusActive &&
+        cudaMemsetAsync(a.work_counter, 0, sizeof(unsigned long long), cs) != cudaSuccess)
+      return cuda_failed("cudaMemsetAsync of the work counter failed");
+  }
   if (shape->shared_prefix && shape->num_blocks > 0) {
     // plan the groups, then their shared tokens on tensor cores, then every
     // sequence's own tokens on CUDA cores, then the merge

@@ -102,8 +102,8 @@ struct Warps {
   static_assert(kNCW * kNWG == NC, "columns split evenly");
 };
 
-// Per kernel kind: N columns, sequences per launch (their prefix sums live in
-// shared memory) and TMEM columns (S^T in [0, N); O^T in [N, 3N), its hi part
+// Per kernel kind: N columns, sequences per launch (the scheduler warp holds
+// their prefix counts in registers) and TMEM columns (S^T in [0, N); O^T in [N, 3N), its hi part
 // in [N, 2N) and its lo part in [2N, 3N), rounded up to a power of two).
 template <bool GROUP>
 struct Cfg {

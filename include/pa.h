@@ -26,9 +26,10 @@
  *    the access is skipped (a K/V row outside the pool reads as zeros), a bit
  *    is recorded in a per-device error word, and pa_last_device_error()
  *    returns PA_ERR_DEVICE_CHECK until it is read.
- *  - No kernel waits on anything but its own TMA copies, and every such wait
- *    has a wall-clock limit (2 s) after which the kernel records
- *    PA_DEVERR_WAIT_TIMEOUT and returns.
+ *  - No kernel waits on anything outside its own CTA: its TMA copies, its
+ *    tensor-core products and its own warps' hand-offs.  Every such wait has
+ *    a wall-clock limit (2 s) after which the kernel records
+ *    PA_DEVERR_WAIT_TIMEOUT, lets its copies and products land, and returns.
  */
 #ifndef PA_H_
 #define PA_H_

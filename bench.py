@@ -10,8 +10,10 @@ resident in HBM before the timed region starts.
 The reported metric is the decode's K/V-read bandwidth: algorithmic bytes of
 the decode (K and V rows of every context, q, out, block-table entries and
 context lengths) divided by the device time of the whole step, plus decode
-tokens/s per layer.  The `roofline` object is the decode kernels alone,
-timed with CUDA events on their stream.
+tokens/s per layer.  The K timed steps run between one pair of CUDA events
+with nothing else on the stream.  The `roofline` object is the decode
+kernels alone, timed with CUDA events around each step's decode in a second
+pass over the same steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--impl ours|reference]

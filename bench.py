@@ -46,6 +46,8 @@ METRIC = ("paged decode-attn KV-read GB/s (% of B200 HBM peak); decode tokens/s 
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 VARIANTS = {"auto": 0, "cuda_cores": 1, "tensor_cores": 2}
+# Timed beside the main workload, decode only, in the same run.
+OTHER_WORKLOADS = ("llama2_7b", "qwen_7b_prefix", "llama2_70b_beam")
 
 
 def parse_args(argv=None):
@@ -53,7 +55,7 @@ def parse_args(argv=None):
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=3000)
     p.add_argument("--warmup", type=int, default=20)
-    p.add_argument("--workload", default="llama2_7b", choices=sorted(gen.WORKLOADS))
+    p.add_argument("--workload", default="mistral_7b_gqa", choices=sorted(gen.WORKLOADS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--partition-tokens", type=int, default=0)
     p.add_argument("--variant", default="auto", choices=sorted(VARIANTS),
@@ -78,6 +80,10 @@ def parse_args(argv=None):
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
+    p.add_argument("--per-workload", default=",".join(OTHER_WORKLOADS),
+                   help="further workloads whose decode is timed beside the main line "
+                        "(comma list; empty for none)")
+    p.add_argument("--per-workload-steps", type=int, default=300)
     return p.parse_args(argv)
 
 
@@ -150,14 +156,17 @@ def tables_share_blocks(tables: np.ndarray, ctx: np.ndarray) -> bool:
 def unique_kv_bytes(tables: np.ndarray, ctx: np.ndarray, block_size, num_kv_heads, head_dim,
                     elem=2) -> int:
     """K+V bytes of the distinct slots a decode reads (shared blocks once)."""
-    slots = set()
+    slots = []
+    ar = np.arange(block_size, dtype=np.int64)
     for s in range(len(ctx)):
         L = int(ctx[s])
+        if L <= 0:
+            continue
         nb = -(-L // block_size)
-        for i in range(nb):
-            n = min(block_size, L - i * block_size)
-            slots.update(int(tables[s, i]) * block_size + j for j in range(n))
-    return 2 * len(slots) * num_kv_heads * head_dim * elem
+        rows = (np.asarray(tables[s, :nb], dtype=np.int64)[:, None] * block_size + ar).reshape(-1)
+        slots.append(rows[:L])
+    n = len(np.unique(np.concatenate(slots))) if slots else 0
+    return 2 * n * num_kv_heads * head_dim * elem
 
 
 # ---------------------------------------------------------------------------
@@ -415,6 +424,78 @@ def swap_bandwidth(w, torch, pa, n_blocks: int = 256, reps: int = 5):
     return res
 
 
+def time_other_workload(name, args, rank, torch, pa, stream, peak):
+    """Decode of another workload in the same run: automatic variant (shared
+    prefixes on where the tables share blocks), W warm-up steps, then K steps
+    timed as one stretch and again with events around each decode.  Returns
+    the decode GB/s and its roofline fraction; for workloads whose tables
+    share blocks, also the GB/s of the distinct K/V slots read."""
+    steps = max(1, args.per_workload_steps)
+    warm = max(3, args.warmup)
+    n_cycle = max(1, min(args.cycle, steps + warm))
+    case = gen.make_case(name, n_steps=n_cycle, poison=False,
+                         seed=gen.SEED_BASE + gen.WORKLOADS[name].number + 1000 * rank)
+    shared = int(tables_share_blocks(case.steps[0].block_tables, case.steps[0].context_lens))
+    w = DeviceWorkload(case, torch, pa, case.workload.partition_tokens, 0, shared)
+    bytes_per = [decode_bytes(s.context_lens, case.num_q_heads, case.num_kv_heads, case.head_dim,
+                              case.block_size) for s in case.steps]
+    with torch.cuda.stream(stream):
+        for i in range(warm):
+            w.step(i, stream)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(device_uuid(torch)) as clocks:
+            t0.record(stream)
+            for i in range(steps):
+                w.step(warm + i, stream)
+            t1.record(stream)
+            torch.cuda.synchronize()
+        evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(steps)]
+        for i in range(steps):
+            w.step(warm + i, stream, evs[i])
+        torch.cuda.synchronize()
+    status, bits = pa.pa_last_device_error(stream.cuda_stream)
+    if status != pa.PA_OK:
+        raise RuntimeError(f"device check in {name}: {bits:#x}")
+    step_bytes = sum(bytes_per[(warm + i) % n_cycle] for i in range(steps))
+    dec_ms = sum(evs[i][1].elapsed_time(evs[i][2]) for i in range(steps))
+    dec_gbs = step_bytes / (dec_ms * 1e-3) / 1e9
+    resolved = {1: "cuda_cores", 2: "tensor_cores",
+                3: "shared_prefix"}[pa.pa_decode_resolved_variant(w.shape)]
+    res = {
+        "decode_variant": resolved,
+        "steps": steps, "warmup": warm,
+        "step_gbs": round(step_bytes / (t0.elapsed_time(t1) * 1e-3) / 1e9, 2),
+        "decode_gbs": round(dec_gbs, 2),
+        "decode_ms_per_step": round(dec_ms / steps, 5),
+        "decode_bytes_per_step": int(step_bytes / steps),
+        "frac": round(dec_gbs / peak, 4),
+        "traffic": profiled_traffic(name, resolved, step_bytes / steps),
+        "tokens_per_s_per_layer": round(case.num_seqs * steps / (dec_ms * 1e-3), 1),
+        "clocks": clocks.summary(),
+    }
+    if shared:
+        # unique bytes of the timed steps: distinct K/V slots (shared blocks
+        # once) plus the same q, out, table and length bytes
+        per_cycle = {}
+        uniq = 0
+        for i in range(steps):
+            j = (warm + i) % n_cycle
+            if j not in per_cycle:
+                st = case.steps[j]
+                kv_logical = 2 * int(st.context_lens.sum()) * case.num_kv_heads * case.head_dim * 2
+                per_cycle[j] = bytes_per[j] - kv_logical + unique_kv_bytes(
+                    st.block_tables, st.context_lens, case.block_size, case.num_kv_heads,
+                    case.head_dim)
+            uniq += per_cycle[j]
+        res["unique_bytes_per_step"] = int(uniq / steps)
+        res["unique_gbs"] = round(uniq / (dec_ms * 1e-3) / 1e9, 2)
+        res["unique_frac"] = round(res["unique_gbs"] / peak, 4)
+    del w
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, rank, world, local, dist):
     import torch
 
@@ -502,7 +583,8 @@ def run_ours(args, rank, world, local, dist):
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(max_ms / args.steps, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3" if fp8 else gen.DTYPE_NAMES[case.dtype], "accum_dtype": "f32",
         "data": "synthetic (seeded N(0,1) values, shapes and block structure of the workload)",
         "config": {
             "workload": f"{args.workload}: {case.workload.description}",
@@ -548,6 +630,15 @@ def run_ours(args, rank, world, local, dist):
         result["swap"] = swap_bandwidth(w, torch, pa)
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, w, stream, bytes_per, n_cycle, dist)
+    others = [n for n in args.per_workload.split(",") if n and n != args.workload]
+    unknown = [n for n in others if n not in gen.WORKLOADS]
+    if unknown:
+        raise SystemExit(f"--per-workload: unknown workloads {unknown}")
+    if others:
+        del w
+        torch.cuda.empty_cache()
+        result["per_workload"] = {n: time_other_workload(n, args, rank, torch, pa, stream, peak)
+                                  for n in others}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(case, args.cpu_seconds, case.steps[0])
     return result
@@ -648,14 +739,10 @@ def _oracle_sample(case, st, n_seqs, orc, threads):
     return dt, nbytes
 
 
-def cpu_baseline(case, seconds: float, st):
-    """The fp64 oracle on the host cores, on the first sequences of the batch
-    (sized to about `seconds` of work); reported as GB/s of algorithmic bytes."""
-    import oracle
-
-    orc = oracle.load()
-    cores = len(os.sched_getaffinity(0))
-    threads = orc.num_threads(cores)
+def _timed_oracle(case, st, orc, threads, seconds):
+    """Decode the first sequences of the batch, as many as about `seconds`
+    of work on `threads` threads (the whole batch again while under half of
+    it); returns (seconds, algorithmic bytes, sequences, repetitions)."""
     dt1, _ = _oracle_sample(case, st, 1, orc, threads)
     n = int(max(1, min(case.num_seqs, seconds / max(dt1, 1e-6))))
     dt, nbytes = _oracle_sample(case, st, n, orc, threads)
@@ -663,11 +750,30 @@ def cpu_baseline(case, seconds: float, st):
     while dt < 0.5 * seconds:  # the whole batch took less: decode it again
         d, b = _oracle_sample(case, st, n, orc, threads)
         dt, nbytes, reps = dt + d, nbytes + b, reps + 1
+    return dt, nbytes, n, reps
+
+
+def cpu_baseline(case, seconds: float, st):
+    """The fp64 oracle on the host cores, on the first sequences of the batch
+    (sized to about `seconds` of work on all cores, and a third of that on one
+    thread); reported as GB/s of algorithmic bytes."""
+    import oracle
+
+    orc = oracle.load()
+    cores = len(os.sched_getaffinity(0))
+    threads = orc.num_threads(cores)
+    dt, nbytes, n, reps = _timed_oracle(case, st, orc, threads, seconds)
+    dt_1, nbytes_1, n_1, reps_1 = _timed_oracle(case, st, orc, 1, seconds / 3)
     return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": threads,
             "kind": "oracle",
             "sample": f"fp64 C oracle, decode of the first {n} of {case.num_seqs} sequences of step 0, "
                       f"{reps} time(s) ({nbytes / 1e6:.1f} MB algorithmic), {dt:.2f} s wall, "
-                      f"{threads} threads"}
+                      f"{threads} threads",
+            "single_thread": {
+                "value": round(nbytes_1 / dt_1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                "sample": f"the first {n_1} sequences, {reps_1} time(s) "
+                          f"({nbytes_1 / 1e6:.1f} MB), {dt_1:.2f} s wall, 1 thread"},
+            "affinity_cores": cores}
 
 
 def run_reference(args, rank, world):

@@ -263,7 +263,10 @@ pa_status pa_decode_multi(const void *q, const void *k_cache, const void *v_cach
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) and caches it; make that first call before any
  *    stream capture on that device.  It returns PA_ERR_CUDA if the lookup
- *    fails.
+ *    fails.  The cached address belongs to the device's context at that
+ *    time: after cudaDeviceReset(), or anything else that destroys the
+ *    primary context, it is stale, so do not call pa_decode_noalloc on that
+ *    device again in the same process.
  *  - Every call on a device shares the one array and finds the previous
  *    call's contents in it; nothing in it has to start at zero, because each
  *    call writes every scratch slot it later reads.  Calls whose kernels can

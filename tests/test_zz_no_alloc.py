@@ -4,12 +4,19 @@ Some callers of this library cannot allocate the split-K workspace that
 pa_decode needs -- a plug-in inside a host runtime that owns all device memory
 and offers no allocator, or a decode loop that must not call cudaMalloc while
 it runs.  pa_decode_noalloc takes that scratch from a fixed array inside the
-library instead.  This file checks, through the C ABI, that two calls in a
-row give the same output as pa_decode with a caller-owned workspace (within
-the tests' decode tolerance), that the second call is not disturbed by what
-the first left in the shared array, and that a request larger than the
-array is refused.  It is named to be collected last and needs nothing from
-the other test files, so it also runs alone in a fresh process.
+library instead.  This file checks, through the C ABI:
+
+- two calls in a row, of different shapes, each against the fp64 oracle
+  (the decode tolerance) and bit for bit against pa_decode with a
+  caller-owned workspace (the same kernels write the same partials into
+  fixed slots and merge them in a fixed order, so anything the first call
+  left in the shared array that leaked into the second would show);
+- the same with shared_prefix = 1, whose group plan and work counter also
+  live in the shared array, with two different groupings in a row;
+- that a request larger than the array is refused with nothing launched.
+
+It is named to be collected last and needs nothing from the other test files,
+so it also runs alone in a fresh process.
 """
 import numpy as np
 import pytest
@@ -17,7 +24,7 @@ import pytest
 torch = pytest.importorskip("torch")
 
 from paged_kv_cache_458_b200 import gen, pa  # noqa: E402
-from gpu_util import dev, dev_i32, host_bits, shape_of  # noqa: E402
+from gpu_util import SHARED, dev, dev_i32, host_bits, shape_of  # noqa: E402
 from tolerance import assert_decode_close  # noqa: E402
 
 pytestmark = pytest.mark.gpu
@@ -34,47 +41,73 @@ def _cuda():
     yield
 
 
-def _inputs(seed, ctx, group=4, dtype=gen.BF16):
-    c = gen.random_decode_case(np.random.default_rng(seed), num_seqs=len(ctx),
-                               num_q_heads=2 * group, num_kv_heads=2, head_dim=128,
-                               block_size=16, dtype=dtype, context_lens=ctx)
-    shape = shape_of(dtype, c["q"], c["k_cache"], c["block_tables"])
+def _on_device(c, dtype, variant=0):
+    shape = shape_of(dtype, c["q"], c["k_cache"], c["block_tables"], variant=variant)
     d = dict(q=dev(c["q"], dtype), k=dev(c["k_cache"], dtype), v=dev(c["v_cache"], dtype),
              bt=dev_i32(c["block_tables"]), cl=dev_i32(c["context_lens"]))
-    return c, shape, d, int(max(ctx))
+    return shape, d, int(np.max(c["context_lens"], initial=0))
 
 
 def _with_workspace(c, shape, d, maxlen, dtype):
-    out = torch.empty(c["q"].shape, dtype=pa.torch_dtype(dtype), device="cuda")
+    out = torch.full(c["q"].shape, float("nan"), dtype=pa.torch_dtype(dtype), device="cuda")
     wsb = pa.pa_decode_workspace_bytes(shape, maxlen)
-    ws = torch.empty(max(16, wsb), dtype=torch.uint8, device="cuda")
+    # arbitrary bytes: the workspace needs no initial contents
+    ws = torch.randint(0, 256, (max(16, wsb),), dtype=torch.uint8, device="cuda")
     pa.pa_decode(d["q"], d["k"], d["v"], d["bt"], d["cl"], c["scale"], out, shape, maxlen, ws, wsb)
-    return out
+    return host_bits(out)
 
 
 def _no_alloc(c, shape, d, maxlen, dtype):
     out = torch.full(c["q"].shape, float("nan"), dtype=pa.torch_dtype(dtype), device="cuda")
     pa.pa_decode_noalloc(d["q"], d["k"], d["v"], d["bt"], d["cl"], c["scale"], out, shape, maxlen)
-    return out
+    return host_bits(out)
 
 
-def test_two_calls_in_a_row_match_pa_decode():
-    dtype = gen.BF16
-    # first call: long contexts, many partitions (fills much of the scratch)
-    c1, s1, d1, m1 = _inputs(31, [3000, 1, 2049, 700, 4096, 513], group=4)
-    assert pa.pa_decode_workspace_bytes(s1, m1) > 0
-    # second call: other shapes and contexts, so stale scratch from call 1 would show
-    c2, s2, d2, m2 = _inputs(32, [1500, 600, 33, 2500], group=8)
-    ref1 = _with_workspace(c1, s1, d1, m1, dtype)
-    ref2 = _with_workspace(c2, s2, d2, m2, dtype)
-    got1 = _no_alloc(c1, s1, d1, m1, dtype)
-    got2 = _no_alloc(c2, s2, d2, m2, dtype)
+def _check_pair(orc, cases, dtype, variant):
+    """Both calls through pa_decode_noalloc in a row, then each against the
+    oracle and against pa_decode with its own workspace."""
+    dev_cases = [(c,) + _on_device(c, dtype, variant) for c in cases]
+    for _, shape, _, maxlen in dev_cases:
+        assert 0 < pa.pa_decode_workspace_bytes(shape, maxlen) <= pa.PA_NOALLOC_SCRATCH_BYTES
+    got = [_no_alloc(c, s, d, m, dtype) for c, s, d, m in dev_cases]
     status, bits = pa.pa_last_device_error()
     assert status == pa.PA_OK, f"device check fired: {bits:#x}"
-    for got, ref, what in ((got1, ref1, "first call"), (got2, ref2, "second call")):
-        r = host_bits(ref).astype(np.uint16)
-        ref64 = gen.bits_to_f32(r, dtype).astype(np.float64).reshape(ref.shape)
-        assert_decode_close(host_bits(got), ref64, dtype, what)
+    ref = [_with_workspace(c, s, d, m, dtype) for c, s, d, m in dev_cases]
+    for i, (c, g, r) in enumerate(zip(cases, got, ref)):
+        exact = orc.decode(dtype, c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
+                           c["context_lens"], c["scale"])
+        assert_decode_close(g, exact, dtype, f"call {i + 1} vs the oracle")
+        assert np.array_equal(g, r), f"call {i + 1}: differs from pa_decode with a workspace"
+
+
+def test_two_calls_in_a_row(orc):
+    dtype = gen.BF16
+    rng = np.random.default_rng(31)
+    # first call: long contexts, many partitions (fills much of the scratch);
+    # second: other shapes and contexts, so stale scratch from call 1 would show
+    c1 = gen.random_decode_case(rng, num_seqs=6, num_q_heads=8, num_kv_heads=2, head_dim=128,
+                                block_size=16, dtype=dtype,
+                                context_lens=[3000, 1, 2049, 700, 4096, 513])
+    c2 = gen.random_decode_case(rng, num_seqs=4, num_q_heads=16, num_kv_heads=2, head_dim=128,
+                                block_size=16, dtype=dtype, context_lens=[1500, 600, 33, 2500])
+    _check_pair(orc, [c1, c2], dtype, variant=0)
+
+
+def test_two_shared_prefix_calls_in_a_row(orc):
+    """The plan and the tagged work counter sit in the shared array too."""
+    dtype = gen.F16
+    rng = np.random.default_rng(32)
+    c1 = gen.grouped_decode_case(rng, groups=[(700, [710, 730, 760, 705]), (300, [310, 305]),
+                                              (0, [37])],
+                                 num_q_heads=16, num_kv_heads=2, head_dim=128, block_size=16,
+                                 dtype=dtype)
+    # different groupings in the same sequence positions: stale plan entries
+    # from call 1 would put members in the wrong groups
+    c2 = gen.grouped_decode_case(rng, groups=[(0, [50]), (1200, [1210, 1300, 1250]),
+                                              (260, [270, 300, 290, 280])],
+                                 num_q_heads=16, num_kv_heads=2, head_dim=128, block_size=16,
+                                 dtype=dtype)
+    _check_pair(orc, [c1, c2], dtype, variant=SHARED)
 
 
 def test_request_larger_than_the_scratch_is_refused():

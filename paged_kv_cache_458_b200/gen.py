@@ -130,111 +130,76 @@ def bits_to_f32(bits: np.ndarray, dtype: int) -> np.ndarray:
 # block manager (input construction)
 
 
-class BlockManager:
-    """Free list + reference counts + per-sequence block tables.
+class PoolAllocator:
+    """The library's host block allocator (the C ABI's pa_alloc_*: free list,
+    reference counts, block tables) behind the calls the workload builders
+    make, plus the peak number of blocks in use.
 
-    The free list is a stack: it starts as ``order`` with ``order[0]`` on top,
-    and a block whose reference count drops to zero is pushed back on top, so
-    the next allocation reuses it (the pool reuse of zingnex.cn section 3.2,
-    item 4).  ``append_slot`` allocates only when a token crosses into a new
-    block (item 1) and copies a shared last block before writing to it
-    (item 3, copy-on-write).
+    The free list is a stack that starts as ``order`` with ``order[0]`` on
+    top; a block whose reference count drops to zero goes back on top, so the
+    next allocation reuses it (the pool reuse of zingnex.cn section 3.2, item
+    4).  ``append_slots`` allocates only when a token crosses into a new block
+    (item 1) and copies a shared last block before writing to it (item 3,
+    copy-on-write), returning the copy pairs.
     """
 
     def __init__(self, num_blocks: int, block_size: int, order=None):
+        from . import build, pa
+
+        try:
+            pa.lib()
+        except pa.LibraryMissing:
+            build.build()  # host code only: the allocator needs no GPU
         self.num_blocks = int(num_blocks)
         self.block_size = int(block_size)
-        order = np.arange(num_blocks) if order is None else np.asarray(order)
-        assert sorted(order.tolist()) == list(range(num_blocks))
-        self.free = [int(b) for b in order[::-1]]
-        self.ref = np.zeros(num_blocks, dtype=np.int64)
-        self.tables: dict[int, list[int]] = {}
-        self.lens: dict[int, int] = {}
+        self._a = pa.Allocator(self.num_blocks, self.block_size, order)
+        self.lens: dict[int, int] = {}  # tokens per live sequence
         self.peak_used = 0
 
-    # -- primitives
-    def used(self) -> int:
-        return self.num_blocks - len(self.free)
-
-    def alloc(self) -> int:
-        if not self.free:
-            raise MemoryError("block pool exhausted")
-        b = self.free.pop()
-        assert self.ref[b] == 0
-        self.ref[b] = 1
+    def _track(self):
         self.peak_used = max(self.peak_used, self.used())
-        return b
 
-    def release(self, b: int) -> None:
-        assert self.ref[b] > 0
-        self.ref[b] -= 1
-        if self.ref[b] == 0:
-            self.free.append(b)
+    def used(self) -> int:
+        return self.num_blocks - self._a.num_free()
 
-    # -- sequence operations
     def add_seq(self, seq: int, n_tokens: int) -> None:
-        assert seq not in self.tables
-        self.tables[seq] = []
-        self.lens[seq] = 0
-        self.extend(seq, n_tokens)
+        self._a.add_seq(seq, n_tokens)
+        self.lens[seq] = int(n_tokens)
+        self._track()
 
     def extend(self, seq: int, n_tokens: int) -> None:
-        """Grow a sequence by ``n_tokens`` (prefill): blocks on demand, no CoW."""
-        tab = self.tables[seq]
-        L = self.lens[seq] + n_tokens
-        while len(tab) * self.block_size < L:
-            tab.append(self.alloc())
-        self.lens[seq] = L
+        """Grow a sequence by ``n_tokens`` (prefill): blocks on demand, no copy."""
+        self._a.extend(seq, n_tokens)
+        self.lens[seq] += int(n_tokens)
+        self._track()
 
     def fork(self, parent: int, child: int) -> None:
-        """``child`` shares every block of ``parent`` (refcount + 1 each)."""
-        assert child not in self.tables
-        tab = list(self.tables[parent])
-        for b in tab:
-            self.ref[b] += 1
-        self.tables[child] = tab
+        """``child`` shares every block of ``parent`` (reference count + 1 each)."""
+        self._a.fork(parent, child)
         self.lens[child] = self.lens[parent]
 
     def free_seq(self, seq: int) -> None:
-        # last block first, so the sequence's first block ends on top of the stack
-        for b in reversed(self.tables.pop(seq)):
-            self.release(b)
+        self._a.free_seq(seq)
         del self.lens[seq]
 
-    def append_slot(self, seq: int):
-        """Reserve the slot of the next token of ``seq``.
-
-        Returns ``(slot, pair)`` where ``pair`` is ``(src, dst)`` when the last
-        block was shared and had to be copied first, else ``None``.
-        """
-        tab = self.tables[seq]
-        L = self.lens[seq]
-        off = L % self.block_size
-        pair = None
-        if off == 0:
-            b = self.alloc()
-            tab.append(b)
-        else:
-            b = tab[-1]
-            if self.ref[b] > 1:
-                nb = self.alloc()
-                pair = (b, nb)
-                self.release(b)
-                tab[-1] = nb
-                b = nb
-        self.lens[seq] = L + 1
-        return b * self.block_size + off, pair
+    def append_slots(self, seqs):
+        """Slots of the next token of each of ``seqs`` (in order) and the
+        copy-on-write pairs (src, dst), int32 [n][2]."""
+        slots, pairs = self._a.append_slots(seqs)
+        for s in seqs:
+            self.lens[int(s)] += 1
+        self._track()
+        return slots, pairs
 
     def table_array(self, seqs, max_blocks: int) -> np.ndarray:
-        t = np.full((len(seqs), max_blocks), -1, dtype=np.int32)
-        for i, s in enumerate(seqs):
-            tab = self.tables[s]
-            assert len(tab) <= max_blocks
-            t[i, :len(tab)] = tab
-        return t
+        """Block tables [len(seqs)][max_blocks], padded with -1."""
+        return self._a.block_tables(list(seqs), max_blocks)[0]
 
     def lens_array(self, seqs) -> np.ndarray:
-        return np.array([self.lens[s] for s in seqs], dtype=np.int32)
+        return np.array([self.lens[int(s)] for s in seqs], dtype=np.int32)
+
+    def close(self) -> None:
+        self._a.close()
 
 
 # ----------------------------------------------------------------------------
@@ -320,7 +285,7 @@ def _context_lengths(w: Workload, rng: np.random.Generator):
     return ctx.astype(np.int64), info
 
 
-def _build_initial(w: Workload, mgr: BlockManager, ctx: np.ndarray, info: dict) -> None:
+def _build_initial(w: Workload, mgr: PoolAllocator, ctx: np.ndarray, info: dict) -> None:
     S, bs = w.num_seqs, w.block_size
     if w.name == "qwen_7b_prefix":
         P = info["prefix_tokens"]
@@ -344,8 +309,9 @@ def _build_initial(w: Workload, mgr: BlockManager, ctx: np.ndarray, info: dict) 
             mgr.add_seq(s, int(ctx[s]))
 
 
-def _run_steps(w: Workload, mgr: BlockManager, n_steps: int):
-    """Host block operations of each step: beam re-fork, then append slots."""
+def _run_steps(w: Workload, mgr: PoolAllocator, n_steps: int):
+    """Host block operations of each step: beam re-fork, then one appended
+    slot per sequence (with the copy-on-write pairs the allocator returns)."""
     S = w.num_seqs
     out = []
     for _ in range(n_steps):
@@ -355,23 +321,18 @@ def _run_steps(w: Workload, mgr: BlockManager, n_steps: int):
                 for k in range(1, 4):
                     mgr.free_seq(4 * g + k)
                     mgr.fork(4 * g, 4 * g + k)
-        slots = np.empty(S, dtype=np.int32)
-        pairs = []
-        for s in range(S):
-            slot, pair = mgr.append_slot(s)
-            slots[s] = slot
-            if pair is not None:
-                pairs.append(pair)
-        out.append((slots, np.array(pairs, dtype=np.int32).reshape(-1, 2)))
+        slots, pairs = mgr.append_slots(list(range(S)))
+        out.append((slots, np.asarray(pairs, dtype=np.int32).reshape(-1, 2)))
     return out
 
 
 def _pool_blocks(w: Workload, ctx, info, n_steps: int) -> int:
     if w.name == "tiny":
         return 32
-    probe = BlockManager(1 << 22, w.block_size)
+    probe = PoolAllocator(1 << 22, w.block_size)
     _build_initial(w, probe, ctx, info)
     _run_steps(w, probe, n_steps)
+    probe.close()
     return int(math.ceil(1.25 * probe.peak_used))
 
 
@@ -398,7 +359,7 @@ def make_case(name: str, n_steps: int = 1, poison: bool = True, seed: int | None
         ctx0 = ctx0[:num_seqs]
     NB = _pool_blocks(w, ctx0, info, n_steps)
     order = rs.permutation(NB)
-    mgr = BlockManager(NB, w.block_size, order)
+    mgr = PoolAllocator(NB, w.block_size, order)
     _build_initial(w, mgr, ctx0, info)
     seqs = list(range(w.num_seqs))
     max_len = int(ctx0.max()) + n_steps
@@ -409,7 +370,7 @@ def make_case(name: str, n_steps: int = 1, poison: bool = True, seed: int | None
 
     # Replay the operations to record the per-step tables (cheap; keeps the
     # structure pass above free of per-step bookkeeping).
-    mgr2 = BlockManager(NB, w.block_size, order)
+    mgr2 = PoolAllocator(NB, w.block_size, order)
     _build_initial(w, mgr2, ctx0, info)
     steps_tables = []
     for _ in range(n_steps):
@@ -484,19 +445,26 @@ def grouped_decode_case(rng: np.random.Generator, *, groups, num_q_heads: int,
     ctx = [int(c) for _, members in groups for c in members]
     need = sum(-(-int(sh) // bs) for sh, _ in groups) + sum(-(-c // bs) for c in ctx) + 2
     NB = max(need, 4)
-    mgr = BlockManager(NB, bs, rng.permutation(NB))
+    mgr = PoolAllocator(NB, bs, rng.permutation(NB))
     s = 0
     for gi, (shared, members) in enumerate(groups):
-        parent = ("parent", gi)
-        mgr.add_seq(parent, int(shared))
-        for c in members:
-            mgr.fork(parent, s)
+        # The parent grows to the shared length; a member shorter than that
+        # forks when the parent holds exactly its tokens, the others fork at
+        # the shared length and then grow on their own.
+        parent = -1 - gi
+        mgr.add_seq(parent, 0)
+        ids = list(range(s, s + len(members)))
+        for L in sorted({int(c) for c in members if c < shared}):
+            mgr.extend(parent, L - mgr.lens[parent])
+            for sid, c in zip(ids, members):
+                if c == L:
+                    mgr.fork(parent, sid)
+        mgr.extend(parent, int(shared) - mgr.lens[parent])
+        for sid, c in zip(ids, members):
             if c >= shared:
-                mgr.extend(s, c - int(shared))
-            else:
-                mgr.tables[s] = mgr.tables[s][:-(-c // bs)]
-                mgr.lens[s] = c
-            s += 1
+                mgr.fork(parent, sid)
+                mgr.extend(sid, int(c) - int(shared))
+        s += len(members)
     S = s
     MBS = max(1, -(-max(ctx, default=0) // bs))
     bt = mgr.table_array(list(range(S)), MBS)
@@ -530,7 +498,7 @@ def random_decode_case(rng: np.random.Generator, *, num_seqs: int, num_q_heads: 
     need = int(sum(-(-int(L) // block_size) for L in ctx)) + 1
     NB = max(need + 2, 4) if num_blocks is None else int(num_blocks)
     order = rng.permutation(NB)
-    mgr = BlockManager(NB, block_size, order)
+    mgr = PoolAllocator(NB, block_size, order)
     if shared_prefix_blocks:
         P = shared_prefix_blocks * block_size
         mgr.add_seq(-1, P)

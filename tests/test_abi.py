@@ -4,6 +4,7 @@ import ctypes
 import numpy as np
 import pytest
 
+import block_manager_twin
 from paged_kv_cache_458_b200 import gen, pa
 
 
@@ -69,14 +70,17 @@ def test_decode_rejects_bad_shapes(lib, kw, expect):
 
 
 def test_shared_prefix_workspace(lib):
-    """Counter, plan (16 B per sequence, 256-aligned), split-K space for P + 1 partitions."""
+    """Counter, two plan records (16 B per sequence each, 256-aligned), split-K
+    space for P + 2 partitions (a member's shared tokens and its own run may
+    each end in a partial partition and start the next one part-way)."""
     s = _shape(shared_prefix=1)
-    rows = 4 * 8 * 2                       # S * Hq * (1 partition + 1)
+    rows = 4 * 8 * 3                       # S * Hq * (1 partition + 2)
     acc = rows * 128 * 4
-    assert lib.pa_decode_workspace_bytes(ctypes.byref(s), 100) == 256 + 256 + acc + rows * 8
+    assert lib.pa_decode_workspace_bytes(ctypes.byref(s), 100) == 256 + 2 * 256 + acc + rows * 8
     s20 = _shape(shared_prefix=1, num_seqs=20, max_blocks_per_seq=64)
-    rows = 20 * 8 * 3                      # 1000 tokens: 2 partitions + 1
-    assert lib.pa_decode_workspace_bytes(ctypes.byref(s20), 1000) == 256 + 512 + rows * 128 * 4 + rows * 8
+    rows = 20 * 8 * 4                      # 1000 tokens: 2 partitions + 2
+    assert lib.pa_decode_workspace_bytes(ctypes.byref(s20), 1000) == \
+        256 + 2 * 512 + rows * 128 * 4 + rows * 8
     assert pa.pa_decode_resolved_variant(s) == pa.PA_DECODE_RESOLVED_SHARED_PREFIX
 
 
@@ -122,15 +126,23 @@ def test_multi_query_workspace_and_validation(lib):
     assert lib.pa_decode_multi_workspace_bytes(ctypes.byref(s), 1, 700) == one
     assert lib.pa_decode_multi_workspace_bytes(ctypes.byref(s), 0, 700) == 0
     w4 = lib.pa_decode_multi_workspace_bytes(ctypes.byref(s), 4, 700)
-    # virtual tables and contexts, then a shared-prefix decode of 16 virtual
-    # sequences (4 tokens x g 4 = 16 rows >= 8): 16 * 8 heads * (2 + 1)
-    # partitions of (128 + 2) floats, plan 256 bytes, counter 256
-    rows = 16 * 8 * 3
-    assert w4 == 4 * 16 * 64 + 256 + 256 + 256 + rows * 128 * 4 + rows * 8
-    # 1 query head per kv head, 2 tokens: 2 rows < 8, plain decode of 8 virtual
-    # sequences (one 1024-token partition: the counter only)
+    # 4 tokens x g 4 = 16 columns: one tensor-core item per (sequence, kv
+    # head, partition) for all four queries, 512-token partitions: counter,
+    # then 4 sequences x 4 queries x 8 heads x 2 partitions of (128 + 2) floats
+    rows = 4 * 4 * 8 * 2
+    assert w4 == 256 + rows * 128 * 4 + rows * 8
+    # 1 query head per kv head, 2 tokens: the same path, 2 partitions
     s1 = _shape(num_q_heads=2, max_blocks_per_seq=64)
-    assert lib.pa_decode_multi_workspace_bytes(ctypes.byref(s1), 2, 700) == 4 * 8 * 64 + 256 + 256
+    rows = 4 * 2 * 2 * 2
+    assert lib.pa_decode_multi_workspace_bytes(ctypes.byref(s1), 2, 700) == \
+        256 + rows * 128 * 4 + rows * 8
+    # forced onto CUDA cores: virtual tables and contexts, then a one-token
+    # decode of 8 virtual sequences (one 1024-token partition: the counter only)
+    s1c = _shape(num_q_heads=2, max_blocks_per_seq=64, variant=1)
+    assert lib.pa_decode_multi_workspace_bytes(ctypes.byref(s1c), 2, 700) == 4 * 8 * 64 + 256 + 256
+    # 8 tokens x g 8 = 64 columns > 32: the virtual sequences, grouped
+    s88 = _shape(num_q_heads=16, max_blocks_per_seq=64)
+    assert lib.pa_decode_multi_workspace_bytes(ctypes.byref(s88), 8, 700) > 4 * 8 * 16 * 2 * 520
     st = lib.pa_decode_multi(FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, ctypes.byref(s), 0, 700, FAKE,
                              1 << 24, None)
     assert st == pa.PA_ERR_INVALID_ARG
@@ -273,11 +285,11 @@ def _apply(ops, mgr_py, mgr_c, max_blocks):
             assert mgr_c.refcount(b) == mgr_py.ref[b]
 
 
-def test_allocator_matches_generator_block_manager(lib):
+def test_allocator_matches_python_twin(lib):
     rng = np.random.default_rng(7)
     NB, bs = 96, 16
     order = rng.permutation(NB)
-    py = gen.BlockManager(NB, bs, order)
+    py = block_manager_twin.BlockManager(NB, bs, order)
     c = pa.Allocator(NB, bs, order)
     ops, live, nxt = [], [], 0
     for _ in range(300):
@@ -304,34 +316,43 @@ def test_allocator_matches_generator_block_manager(lib):
     c.close()
 
 
-def test_allocator_beam_workload_matches_generator(lib):
-    """The beam workload's per-step host operations through the C allocator."""
+def test_beam_workload_copies_come_from_the_allocator(lib):
+    """The beam workload's per-step tables, slots and copy-on-write pairs are
+    the C allocator's: replay the same host operations on the Python twin and
+    check the recorded case against it, and against the copy rule itself."""
     case = gen.make_case("llama2_70b_beam", n_steps=3, with_pool=False, num_seqs=32)
-    c = pa.Allocator(case.num_blocks, case.block_size, case.structure["pool_order"])
+    py = block_manager_twin.BlockManager(case.num_blocks, case.block_size,
+                                         case.structure["pool_order"])
     ctx = case.structure["initial_context_lens"]
     bs = case.block_size
     for g in range(8):
         L = int(ctx[4 * g])
         shared = ((L - 1) // bs) * bs
-        c.add_seq(4 * g, shared)
+        py.add_seq(4 * g, shared)
         for k in range(1, 4):
-            c.fork(4 * g, 4 * g + k)
+            py.fork(4 * g, 4 * g + k)
         for k in range(4):
-            c.extend(4 * g + k, L - shared)
+            py.extend(4 * g + k, L - shared)
     seqs = list(range(32))
-    t, lens = c.block_tables(seqs, case.max_blocks_per_seq)
-    assert np.array_equal(t, case.block_tables) and np.array_equal(lens, case.context_lens)
+    assert np.array_equal(py.table_array(seqs, case.max_blocks_per_seq), case.block_tables)
     for st in case.steps:
         for g in range(8):
             for k in range(1, 4):
-                c.free_seq(4 * g + k)
-                c.fork(4 * g, 4 * g + k)
-        slots, pairs = c.append_slots(seqs)
-        assert np.array_equal(slots, st.slot_mapping)
-        assert np.array_equal(pairs, st.pairs)
-        t, lens = c.block_tables(seqs, case.max_blocks_per_seq)
-        assert np.array_equal(t, st.block_tables) and np.array_equal(lens, st.context_lens)
-    c.close()
+                py.free_seq(4 * g + k)
+                py.fork(4 * g, 4 * g + k)
+        before = py.table_array(seqs, case.max_blocks_per_seq)
+        lens = [py.lens[s] for s in seqs]
+        res = [py.append_slot(s) for s in seqs]
+        assert np.array_equal(st.slot_mapping, [r[0] for r in res])
+        assert [tuple(p) for p in st.pairs.tolist()] == [r[1] for r in res if r[1] is not None]
+        assert np.array_equal(py.table_array(seqs, case.max_blocks_per_seq), st.block_tables)
+        # the rule: a pair exactly where a sequence appends into a partly
+        # filled last block that another sequence still holds
+        for s, (slot, pair) in zip(seqs, res):
+            last = int(before[s, (lens[s] - 1) // bs]) if lens[s] else -1
+            partial = lens[s] % bs != 0
+            if pair is not None:
+                assert partial and pair[0] == last and slot // bs == pair[1]
 
 
 def test_allocator_out_of_blocks_changes_nothing(lib):

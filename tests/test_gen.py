@@ -2,7 +2,8 @@
 import numpy as np
 import pytest
 
-from paged_kv_cache_458_b200 import gen
+import block_manager_twin
+from paged_kv_cache_458_b200 import gen, pa
 
 
 def test_tiny_workload_matches_its_statement():
@@ -98,35 +99,108 @@ def test_beam_workload_shares_all_but_last_block():
         assert not np.isin(dst, st.pairs[:, 0]).any()
 
 
-def test_block_manager_reuses_freed_blocks_lifo():
-    m = gen.BlockManager(8, 16, order=[5, 2, 7, 0, 1, 3, 4, 6])
-    m.add_seq(0, 40)
-    assert m.tables[0] == [5, 2, 7]
-    m.add_seq(1, 1)
-    assert m.tables[1] == [0]
-    m.free_seq(0)
+# The allocator's behaviour, derived by hand from its rules, on the library's
+# C allocator (through gen.PoolAllocator) and on the tests' Python twin.
+
+
+class _Twin:
+    def __init__(self, nb, bs, order=None):
+        self.m = block_manager_twin.BlockManager(nb, bs, order)
+
+    def add(self, s, n):
+        self.m.add_seq(s, n)
+
+    def fork(self, p, c):
+        self.m.fork(p, c)
+
+    def free(self, s):
+        self.m.free_seq(s)
+
+    def table(self, s):
+        return list(self.m.tables[s])
+
+    def append(self, seqs):
+        out = [self.m.append_slot(s) for s in seqs]
+        return [o[0] for o in out], [o[1] for o in out if o[1] is not None]
+
+    def ref(self, b):
+        return int(self.m.ref[b])
+
+    def used(self):
+        return self.m.used()
+
+
+class _C:
+    def __init__(self, nb, bs, order=None):
+        self.m = gen.PoolAllocator(nb, bs, order)
+
+    def add(self, s, n):
+        self.m.add_seq(s, n)
+
+    def fork(self, p, c):
+        self.m.fork(p, c)
+
+    def free(self, s):
+        self.m.free_seq(s)
+
+    def table(self, s):
+        t = self.m.table_array([s], self.m.num_blocks)[0]
+        return [int(b) for b in t if b >= 0]
+
+    def append(self, seqs):
+        slots, pairs = self.m.append_slots(seqs)
+        return slots.tolist(), [tuple(p) for p in pairs.tolist()]
+
+    def ref(self, b):
+        return self.m._a.refcount(b)
+
+    def used(self):
+        return self.m.used()
+
+
+IMPLS = pytest.mark.parametrize("impl", [_C, _Twin], ids=["c_allocator", "python_twin"])
+
+
+@IMPLS
+def test_allocator_reuses_freed_blocks_lifo(impl):
+    m = impl(8, 16, order=[5, 2, 7, 0, 1, 3, 4, 6])
+    m.add(0, 40)
+    assert m.table(0) == [5, 2, 7]
+    m.add(1, 1)
+    assert m.table(1) == [0]
+    m.free(0)
     assert m.used() == 1
-    m.add_seq(2, 20)
-    assert m.tables[2] == [5, 2], "most recently freed blocks are reused first"
+    m.add(2, 20)
+    assert m.table(2) == [5, 2], "most recently freed blocks are reused first"
 
 
-def test_block_manager_cow_and_refcounts():
-    m = gen.BlockManager(6, 4)
-    m.add_seq(0, 6)                  # blocks 0, 1 (second block half full)
+@IMPLS
+def test_allocator_cow_and_refcounts(impl):
+    m = impl(6, 4)
+    m.add(0, 6)                      # blocks 0, 1 (second block half full)
     m.fork(0, 1)
-    assert m.ref.tolist()[:2] == [2, 2]
-    slot, pair = m.append_slot(1)    # shared partially-filled block -> copy
-    assert pair == (1, 2) and slot == 2 * 4 + 2
-    assert m.ref.tolist()[:3] == [2, 1, 1]
-    slot, pair = m.append_slot(0)    # now private again -> in place
-    assert pair is None and slot == 1 * 4 + 2
-    m.free_seq(0)
-    m.free_seq(1)
-    assert m.used() == 0 and np.all(m.ref == 0)
+    assert [m.ref(b) for b in range(2)] == [2, 2]
+    slots, pairs = m.append([1])     # shared partially-filled block -> copy
+    assert pairs == [(1, 2)] and slots == [2 * 4 + 2]
+    assert [m.ref(b) for b in range(3)] == [2, 1, 1]
+    slots, pairs = m.append([0])     # now private again -> in place
+    assert pairs == [] and slots == [1 * 4 + 2]
+    slots, pairs = m.append([0, 1])  # both fill their blocks: no allocation
+    assert slots == [1 * 4 + 3, 2 * 4 + 3] and pairs == []
+    slots, pairs = m.append([1])     # block full: a fresh block, no copy
+    assert slots == [3 * 4 + 0] and pairs == []
+    m.free(0)
+    m.free(1)
+    assert m.used() == 0 and all(m.ref(b) == 0 for b in range(6))
 
 
-def test_block_manager_out_of_blocks():
-    m = gen.BlockManager(2, 16)
+def test_allocator_out_of_blocks():
+    m = block_manager_twin.BlockManager(2, 16)
     m.add_seq(0, 32)
     with pytest.raises(MemoryError):
         m.append_slot(0)
+    c = gen.PoolAllocator(2, 16)
+    c.add_seq(0, 32)
+    with pytest.raises(pa.PaError):
+        c.append_slots([0])
+

@@ -14,9 +14,16 @@ is the exact result rounded to the output type.  Rounding alone averages a
 quarter ulp, 4.9e-4 for bf16 outputs in [0.25, 0.5), so without this term no
 implementation could meet the bound on short contexts.
 """
+import json
+import os
+
 import numpy as np
 
 from paged_kv_cache_458_b200 import gen
+
+# With PA_TOLERANCE_LOG set to a file path, every check appends one JSON line:
+# the case, its error statistics and how much of each bound they use.
+_LOG = os.environ.get("PA_TOLERANCE_LOG")
 
 MAX_ABS = 2e-3
 MEAN_ABS = 2e-4
@@ -52,8 +59,20 @@ def decode_errors(out_bits: np.ndarray, ref: np.ndarray, dtype: int) -> dict:
                 n=int(err.size))
 
 
+def _log(st, dtype, what):
+    if not _LOG:
+        return
+    rec = dict(st, what=what, dtype=gen.DTYPE_NAMES[dtype],
+               test=os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0],
+               max_used=st["max_abs"] / MAX_ABS,
+               mean_over_floor=st["mean_abs"] - st["mean_floor"])
+    with open(_LOG, "a") as f:
+        f.write(json.dumps(rec) + "\n")
+
+
 def assert_decode_close(out_bits, ref, dtype, what=""):
     st = decode_errors(out_bits, ref, dtype)
+    _log(st, dtype, what)
     assert st["n_nan"] == 0, f"{what}: {st['n_nan']} NaN outputs"
     assert st["n_over"] == 0, f"{what}: {st['n_over']} elements above the bound (max {st['max_abs']:.3e})"
     assert st["mean_abs"] <= MEAN_ABS + st["mean_floor"], \

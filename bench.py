@@ -512,7 +512,7 @@ def run_ours(args, rank, world, local, dist):
         case = split_blocks(case, case.block_size // args.block_size)
     shared = {"on": 1, "off": 0}.get(args.shared_prefix)
     if shared is None:
-        shared = int(args.variant == "auto" and args.kv_cache != "fp8" and
+        shared = int(args.variant == "auto" and
                      tables_share_blocks(case.steps[0].block_tables, case.steps[0].context_lens))
     fp8 = args.kv_cache == "fp8"
     partition = args.partition_tokens or case.workload.partition_tokens
@@ -577,7 +577,7 @@ def run_ours(args, rank, world, local, dist):
                 3: "shared_prefix"}[pa.pa_decode_resolved_variant(w.shape)]
     if args.query_tokens > 1:
         resolved = "multi_query"
-    traffic = (None if fp8 or args.query_tokens > 1 else
+    traffic = (None if fp8 or args.query_tokens > 1 or args.block_size else
                profiled_traffic(args.workload, resolved, step_bytes / args.steps))
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -610,7 +610,7 @@ def run_ours(args, rank, world, local, dist):
             "bound": "hbm",
             "kernel": (f"pa_decode ({resolved} partition kernel + split-K merge kernel)"
                        if resolved != "shared_prefix" else
-                       "pa_decode (plan + shared-prefix tensor-core kernel + CUDA-core kernel "
+                       "pa_decode (plan + tensor-core kernel over every group's row list "
                        "+ split-K merge)"),
             "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
             "frac": round(achieved / peak, 4),
@@ -622,7 +622,8 @@ def run_ours(args, rank, world, local, dist):
     if case.workload.name in ("qwen_7b_prefix", "llama2_70b_beam"):
         st = case.steps[0]
         result["unique_kv_bytes_step0"] = unique_kv_bytes(
-            st.block_tables, st.context_lens, case.block_size, case.num_kv_heads, case.head_dim)
+            st.block_tables, st.context_lens, case.block_size, case.num_kv_heads, case.head_dim,
+            elem=kv_elem)
         # the same decode counted in distinct K/V slots (shared blocks once)
         result["unique_kv_gbs_step0_est"] = round(
             result["unique_kv_bytes_step0"] / (dec_total_ms / args.steps * 1e-3) / 1e9, 2)

@@ -96,9 +96,6 @@ pa_status check_decode_shape(const pa_shape* s, int32_t max_context_len) {
       (s->head_dim != 128 || pt % pa::decode_tc_tile_tokens() != 0 || pt > 512))
     return PA_ERR_UNSUPPORTED;
   if (s->shared_prefix != 0 && s->shared_prefix != 1) return PA_ERR_INVALID_ARG;
-  // an E4M3 cache is read by the CUDA-core kernel only
-  if (s->cache_format == PA_CACHE_FP8_E4M3 && (s->variant == PA_DECODE_TENSOR_CORES || s->shared_prefix))
-    return PA_ERR_UNSUPPORTED;
   if (s->shared_prefix &&
       (s->variant != PA_DECODE_AUTO || s->head_dim != 128 || pt % pa::decode_tc_tile_tokens() != 0 ||
        pt > 512))
@@ -114,7 +111,6 @@ pa_status check_decode_shape(const pa_shape* s, int32_t max_context_len) {
 int cache_elem_bytes(const pa_shape* s) { return s->cache_format == PA_CACHE_FP8_E4M3 ? 1 : 2; }
 
 bool tensor_core_kernel(const pa_shape* s, int pt) {
-  if (s->cache_format == PA_CACHE_FP8_E4M3) return false;
   if (s->variant == PA_DECODE_TENSOR_CORES) return true;
   if (s->variant == PA_DECODE_CUDA_CORES) return false;
   // measured: tensor cores win from group 8 up, and at group 4 with 16-token
@@ -129,23 +125,26 @@ bool tensor_core_kernel(const pa_shape* s, int pt) {
 bool use_tensor_cores(const pa_shape* s) { return tensor_core_kernel(s, effective_partition(s)); }
 
 // Workspace: the work counter (8 bytes used of 256); with shared_prefix the
-// plan, int4 [S] (rounded up to 256 bytes); then, for split-K, partial
-// outputs [S][Hq][P][D] and (max, sum) pairs [S][Hq][P][2] in fp32.  P is
-// ceil(max_context_len / partition_tokens), plus one with shared_prefix (a
-// sequence's shared tokens and its own ones may each end in a partial
-// partition).
+// two plan records, int4 [S] each (each rounded up to 256 bytes); then, for
+// split-K, partial outputs [S][Hq][P][D] and (max, sum) pairs [S][Hq][P][2]
+// in fp32.  P is ceil(max_context_len / partition_tokens), plus two with
+// shared_prefix: a member's rows in its group's row list are its shared
+// tokens and its own run, which may each end in a partial partition and
+// start the next one part-way.
 constexpr long long kCounterBytes = 256;
 
 long long round256(long long x) { return (x + 255) / 256 * 256; }
 
 int num_partitions(const pa_shape* s, int32_t max_context_len);
 
-long long plan_bytes(const pa_shape* s) { return s->shared_prefix ? round256(16LL * s->num_seqs) : 0; }
+long long plan_bytes(const pa_shape* s) {
+  return s->shared_prefix ? 2 * round256(16LL * s->num_seqs) : 0;
+}
 
 // Partitions per (sequence, query head) in the workspace (0: no split-K space).
 long long workspace_parts(const pa_shape* s, int32_t max_context_len) {
   const long long P = num_partitions(s, max_context_len);
-  if (s->shared_prefix) return P + 1;
+  if (s->shared_prefix) return P + 2;
   return P > 1 ? P : 0;
 }
 
@@ -215,28 +214,38 @@ bool make_pool_map(CUtensorMap* map, const void* pool, const pa_shape* s, int ro
 int box_rows(const pa_shape* s) { return s->block_size % 16 == 0 ? 16 : 8; }
 
 bool make_tc_maps(CUtensorMap* tk, CUtensorMap* tv, CUtensorMap* tq, const void* k, const void* v,
-                  const void* q, const pa_shape* s, bool pair) {
+                  const void* q, const pa_shape* s, bool pair, int query_tokens, bool grouped) {
   auto fn = encode_fn();
   if (!fn) return false;
+  // a box row is 128 bytes: 64 two-byte elements, or (E4M3 cache) all 128
+  // one-byte elements of a head's row
+  const bool fp8 = s->cache_format == PA_CACHE_FP8_E4M3;
+  const cuuint64_t eb = fp8 ? 1 : 2, inner = 128 / eb;
   const cuuint64_t rows = (cuuint64_t)s->num_blocks * s->block_size, Hkv = (cuuint64_t)s->num_kv_heads;
   const cuuint64_t dims_h[3] = {128, Hkv, rows}, dims_p[3] = {128, rows, Hkv};
-  const cuuint64_t strides_h[2] = {256, Hkv * 256}, strides_p[2] = {Hkv * 256, 256};
-  const cuuint32_t box_h[3] = {64, 1, (cuuint32_t)box_rows(s)}, box_p[3] = {64, 16, 2};
+  const cuuint64_t strides_h[2] = {128 * eb, Hkv * 128 * eb}, strides_p[2] = {Hkv * 128 * eb, 128 * eb};
+  const cuuint32_t box_h[3] = {(cuuint32_t)inner, 1, (cuuint32_t)box_rows(s)},
+                   box_p[3] = {(cuuint32_t)inner, 16, 2};
   const cuuint64_t* dims = pair ? dims_p : dims_h;
   const cuuint64_t* strides = pair ? strides_p : strides_h;
   const cuuint32_t* box = pair ? box_p : box_h;
   const cuuint32_t estr[3] = {1, 1, 1};
   for (int i = 0; i < 2; ++i) {
-    CUresult r = fn(i ? tv : tk, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(i ? v : k), dims,
+    CUresult r = fn(i ? tv : tk, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16,
+                    3, const_cast<void*>(i ? v : k), dims,
                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return false;
   }
-  const cuuint64_t qdims[2] = {128, (cuuint64_t)s->num_seqs * s->num_q_heads};
-  const cuuint64_t qstrides[1] = {256};
-  const cuuint32_t qbox[2] = {64, (cuuint32_t)((pair ? 2 : 1) * (s->num_q_heads / s->num_kv_heads))};
-  const cuuint32_t qestr[2] = {1, 1};
-  return fn(tq, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(q), qdims, qstrides, qbox, qestr,
+  // q viewed as [S * Tq][Hq][128]: one box is the query rows of an item,
+  // [rows][heads][64] (rows past the batch read as zeros)
+  const int g = s->num_q_heads / s->num_kv_heads;
+  const pa::TcQueryBox qb = pa::tc_query_box(g, query_tokens, pair, grouped);
+  const cuuint64_t qdims[3] = {128, (cuuint64_t)s->num_q_heads,
+                               (cuuint64_t)s->num_seqs * (cuuint64_t)query_tokens};
+  const cuuint64_t qstrides[2] = {256, (cuuint64_t)s->num_q_heads * 256};
+  const cuuint32_t qbox[3] = {64, (cuuint32_t)qb.heads, (cuuint32_t)qb.rows};
+  return fn(tq, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(q), qdims, qstrides, qbox, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -260,12 +269,14 @@ size_t pa_decode_workspace_bytes(const pa_shape* shape, int32_t max_context_len)
 
 namespace {
 
-// pa_decode and pa_decode_fp8 (scales set iff the cache holds E4M3 codes).
+// pa_decode and pa_decode_fp8 (scales set iff the cache holds E4M3 codes),
+// and pa_decode_multi on the tensor-core kernels (query_tokens > 1: q and out
+// are [S][Tq][Hq][D]; the caller has checked that the shape takes that path).
 pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
                       const float* k_scale, const float* v_scale, const int32_t* block_tables,
                       const int32_t* context_lens, float scale, void* out, const pa_shape* shape,
                       int32_t max_context_len, void* workspace, size_t workspace_bytes,
-                      pa_stream_t stream) {
+                      pa_stream_t stream, int query_tokens = 1) {
   pa_status st = check_decode_shape(shape, max_context_len);
   if (st != PA_OK) return st;
   const bool fp8 = shape->cache_format == PA_CACHE_FP8_E4M3;
@@ -280,13 +291,16 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
   if ((reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u))
     return PA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
-  const size_t need = pa_decode_workspace_bytes(shape, max_context_len);
+  // the split-K rows of query_tokens queries per sequence
+  pa_shape ws_shape = *shape;
+  ws_shape.num_seqs = shape->num_seqs * query_tokens;
+  const size_t need = pa_decode_workspace_bytes(&ws_shape, max_context_len);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_INVALID_ARG;
   if (max_context_len > (long long)shape->max_blocks_per_seq * shape->block_size)
     return PA_ERR_INVALID_ARG;
 
-  const int P = num_partitions(shape, max_context_len);
   const int P_ws = (int)workspace_parts(shape, max_context_len);
+  const int group = shape->num_q_heads / shape->num_kv_heads;
   pa::DecodeArgs a{};
   a.q = static_cast<const uint16_t*>(q);
   a.block_tables = block_tables;
@@ -295,12 +309,14 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
   a.work_counter = static_cast<unsigned long long*>(workspace);
   char* ws = static_cast<char*>(workspace) + kCounterBytes;
   int4* plan = nullptr;
+  int4* plan2 = nullptr;
   if (shape->shared_prefix) {
     plan = reinterpret_cast<int4*>(ws);
+    plan2 = reinterpret_cast<int4*>(ws + plan_bytes(shape) / 2);
     ws += plan_bytes(shape);
   }
   if (P_ws > 0) {
-    const long long rows = (long long)shape->num_seqs * shape->num_q_heads * P_ws;
+    const long long rows = (long long)ws_shape.num_seqs * shape->num_q_heads * P_ws;
     a.ws_acc = reinterpret_cast<float*>(ws);
     a.ws_ml = reinterpret_cast<float*>(ws + round256(rows * shape->head_dim * 4));
   }
@@ -315,25 +331,23 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
   a.max_blocks_per_seq = shape->max_blocks_per_seq;
   a.partition_tokens = effective_partition(shape);
   a.num_parts = P_ws > 0 ? P_ws : 1;
-  // With shared_prefix a sequence's own tokens (beam tails, private
-  // continuations of a shared prompt) are mostly short: the CUDA-core kernel
-  // takes them in partitions of its largest size, so its grid holds few empty
-  // CTAs and each sequence adds few partials.
-  a.own_tokens = shape->shared_prefix ? pa::decode_max_partition_tokens() : a.partition_tokens;
+  a.own_tokens = a.partition_tokens;
   {
     const int gp = (max_context_len + a.own_tokens - 1) / a.own_tokens;
     a.grid_parts = gp > 0 ? gp : 1;
   }
+  a.query_tokens = query_tokens;
+  a.group = group;
   a.half_boxes = box_rows(shape) == 8;
   a.max_context_len = max_context_len;
   a.err = error_word();
   if (!a.err) return cuda_failed("device error word lookup failed");
 
   if (shape->num_blocks == 0 && max_context_len > 0) return PA_ERR_INVALID_ARG;
-  const int group = shape->num_q_heads / shape->num_kv_heads;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   int launched = 0;
   cudaError_t e;
+  const bool tc_path = shape->num_blocks > 0 && (shape->shared_prefix || use_tensor_cores(shape));
   // The tensor-core kernels take items from the work counter, tagged with a
   // per-call epoch.  Inside a CUDA graph that epoch is fixed at capture, so a
   // replay would find the count its previous replay left under the same
@@ -341,52 +355,53 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
   // first: the memset becomes a node of the graph and runs before each
   // replay's kernels (a zero word carries a foreign epoch, or the right one
   // with a count of zero).  Eager calls keep relying on the epoch alone.
-  if (shape->num_blocks > 0 && (shape->shared_prefix || use_tensor_cores(shape))) {
+  if (tc_path) {
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(cs, &cap) != cudaSuccess) return cuda_failed("cudaStreamIsCapturing failed");
     if (cap == cudaStreamCaptureStatusActive &&
         cudaMemsetAsync(a.work_counter, 0, sizeof(unsigned long long), cs) != cudaSuccess)
       return cuda_failed("cudaMemsetAsync of the work counter failed");
   }
-  if (shape->shared_prefix && shape->num_blocks > 0) {
-    // plan the groups, then their shared tokens on tensor cores, then every
-    // sequence's own tokens on CUDA cores, then the merge
-    CUtensorMap tk, tv, tq, pk, pv;
-    if (!make_tc_maps(&tk, &tv, &tq, k_cache, v_cache, q, shape, false) ||
-        !make_pool_map(&pk, k_cache, shape, box_rows(shape)) ||
-        !make_pool_map(&pv, v_cache, shape, box_rows(shape)))
-      return cuda_failed("cuTensorMapEncodeTiled failed");
-    pa::PlanArgs pl{};
-    pl.block_tables = block_tables;
-    pl.context_lens = context_lens;
-    pl.plan = plan;
-    pl.num_seqs = shape->num_seqs;
-    pl.max_blocks_per_seq = shape->max_blocks_per_seq;
-    pl.block_size = shape->block_size;
-    pl.num_blocks = shape->num_blocks;
-    pl.max_context_len = max_context_len;
-    pl.partition_tokens = a.partition_tokens;
-    pl.max_members = 32 / group;
-    pl.min_shared = pa::decode_tc_tile_tokens();
-    pl.chunk = pa::kSharedPrefixSeqsPerLaunch;
-    a.plan = plan;
-    a.epoch = next_epochs((shape->num_seqs + pa::kSharedPrefixSeqsPerLaunch - 1) /
-                          pa::kSharedPrefixSeqsPerLaunch);
-    e = pa::launch_plan(pl, cs, &launched);
-    if (e == cudaSuccess) e = pa::launch_decode_shared_tc(a, shape->dtype, group, tk, tv, cs, &launched);
-    if (e == cudaSuccess)
-      e = pa::launch_decode(a, shape->dtype, shape->head_dim, group, pk, pv, cs, &launched);
-  } else if (use_tensor_cores(shape) && shape->num_blocks > 0) {
-    // items of two kv heads (4 KB boxes) where the heads pair up, the group
-    // fits 16 columns twice and blocks give 16-row boxes
-    const bool pair = shape->num_kv_heads % 2 == 0 && group <= 8 && !a.half_boxes;
+  if (tc_path) {
+    // items of two kv heads (4 KB boxes) where the heads pair up, their query
+    // columns fit 16 and blocks give 16-row boxes; shared-prefix groups keep
+    // one head per item
+    const bool pair = !shape->shared_prefix && shape->num_kv_heads % 2 == 0 && !a.half_boxes &&
+                      2 * group * query_tokens <= 16;
     CUtensorMap tk, tv, tq;
-    if (!make_tc_maps(&tk, &tv, &tq, k_cache, v_cache, q, shape, pair))
+    if (!make_tc_maps(&tk, &tv, &tq, k_cache, v_cache, q, shape, pair, query_tokens,
+                      shape->shared_prefix != 0))
       return cuda_failed("cuTensorMapEncodeTiled failed");
-    a.epoch = next_epochs((shape->num_seqs + 511) / 512);
-    e = pa::launch_decode_tc(a, shape->dtype, group, tk, tv, tq, cs, &launched, pair);
+    e = cudaSuccess;
+    if (shape->shared_prefix) {
+      // plan the groups, then every group's row list on tensor cores
+      pa::PlanArgs pl{};
+      pl.block_tables = block_tables;
+      pl.context_lens = context_lens;
+      pl.plan = plan;
+      pl.plan2 = plan2;
+      pl.num_seqs = shape->num_seqs;
+      pl.max_blocks_per_seq = shape->max_blocks_per_seq;
+      pl.block_size = shape->block_size;
+      pl.num_blocks = shape->num_blocks;
+      pl.max_context_len = max_context_len;
+      pl.partition_tokens = a.partition_tokens;
+      pl.max_members = pa::kTcMaxColumns / group;
+      pl.min_shared = pa::decode_tc_tile_tokens();
+      pl.chunk = pa::kSharedPrefixSeqsPerLaunch;
+      a.plan = plan;
+      a.plan2 = plan2;
+      a.epoch = next_epochs((shape->num_seqs + pa::kSharedPrefixSeqsPerLaunch - 1) /
+                            pa::kSharedPrefixSeqsPerLaunch);
+      e = pa::launch_plan(pl, cs, &launched);
+    } else {
+      a.epoch = next_epochs((shape->num_seqs + 511) / 512);
+    }
+    if (e == cudaSuccess)
+      e = pa::launch_decode_tc(a, shape->dtype, tk, tv, tq, cs, &launched, pair, fp8);
     if (e == cudaSuccess) e = pa::launch_decode_merge(a, shape->dtype, shape->head_dim, cs, &launched);
   } else {
+    if (query_tokens != 1) return PA_ERR_UNSUPPORTED;  // the caller expands the queries
     CUtensorMap tk, tv;
     if (shape->num_blocks > 0) {
       if (!make_pool_map(&tk, k_cache, shape, box_rows(shape)) ||
@@ -419,20 +434,34 @@ pa_status pa_decode(const void* q, const void* k_cache, const void* v_cache,
 
 namespace {
 
-// The one-token batch pa_decode_multi runs: S * Tq virtual sequences, grouped
-// by shared prefix when the shape allows the shared-prefix kernel and a
-// sequence's Tq x g query rows fill at least 8 of its 32 columns.  Below that
-// the CUDA-core kernel over the virtual sequences (which re-read their common
-// tokens, mostly from L2) measured faster: llama2_7b with Tq = 2 took 0.141
-// vs 0.251 ms, with Tq = 4 0.255 vs 0.293 ms; with Tq x g = 16 or 32 the
-// shared path wins (mistral_7b_gqa, Tq = 4: 0.572 vs 0.955 ms).
+// pa_decode_multi reads each sequence's K/V once for all its Tq query tokens
+// on the tensor-core kernel when the shape allows it (head_dim 128, a 16-bit
+// cache, the variant not forced to CUDA cores, partition_tokens 0 or a
+// multiple of 128 up to 512) and Tq x g <= 32: the Tq x g query rows are the
+// columns of one item, each query masked at its own causal limit.  The shape
+// it runs (tensor-core variant, 512-token partitions by default):
+bool multi_direct(const pa_shape* s, int num_query_tokens) {
+  const int pt = s->partition_tokens;
+  return s->num_kv_heads > 0 && s->head_dim == 128 && s->variant != PA_DECODE_CUDA_CORES &&
+         s->cache_format == PA_CACHE_AS_DTYPE &&
+         (long long)num_query_tokens * (s->num_q_heads / s->num_kv_heads) <= pa::kTcMaxColumns &&
+         (pt == 0 || (pt % pa::decode_tc_tile_tokens() == 0 && pt <= 512));
+}
+pa_shape multi_direct_shape(const pa_shape* s) {
+  pa_shape e = *s;
+  e.variant = PA_DECODE_TENSOR_CORES;
+  e.shared_prefix = 0;
+  if (e.partition_tokens == 0) e.partition_tokens = 512;
+  return e;
+}
+// Otherwise it runs a one-token batch of S * Tq virtual sequences, grouped by
+// shared prefix when the shape allows the shared-prefix kernel.
 pa_shape multi_shape(const pa_shape* s, int num_query_tokens) {
   pa_shape e = *s;
   e.num_seqs = s->num_seqs * num_query_tokens;
   const int pt = s->partition_tokens;
-  const int rows = num_query_tokens * (s->num_q_heads / s->num_kv_heads);
   e.shared_prefix = s->head_dim == 128 && s->variant == PA_DECODE_AUTO &&
-                    s->cache_format == PA_CACHE_AS_DTYPE && rows >= 8 &&
+                    s->cache_format == PA_CACHE_AS_DTYPE &&
                     (pt == 0 || (pt % pa::decode_tc_tile_tokens() == 0 && pt <= 512));
   return e;
 }
@@ -458,6 +487,12 @@ size_t pa_decode_multi_workspace_bytes(const pa_shape* shape, int32_t num_query_
                                        int32_t max_context_len) {
   if (!multi_args_ok(shape, num_query_tokens)) return 0;
   if (num_query_tokens == 1) return pa_decode_workspace_bytes(shape, max_context_len);
+  if (multi_direct(shape, num_query_tokens)) {
+    pa_shape e = multi_direct_shape(shape);
+    if (check_decode_shape(&e, max_context_len) != PA_OK) return 0;
+    e.num_seqs = shape->num_seqs * num_query_tokens;  // split-K rows
+    return pa_decode_workspace_bytes(&e, max_context_len);
+  }
   const pa_shape e = multi_shape(shape, num_query_tokens);
   const size_t inner = pa_decode_workspace_bytes(&e, max_context_len);
   if (inner == 0) return 0;
@@ -476,6 +511,12 @@ pa_status pa_decode_multi(const void* q, const void* k_cache, const void* v_cach
   pa_status st = check_decode_shape(shape, max_context_len);
   if (st != PA_OK) return st;
   if (shape->cache_format != PA_CACHE_AS_DTYPE) return PA_ERR_INVALID_ARG;
+  if (multi_direct(shape, num_query_tokens)) {
+    const pa_shape d = multi_direct_shape(shape);
+    return decode_impl(q, k_cache, v_cache, nullptr, nullptr, block_tables, context_lens, scale,
+                       out, &d, max_context_len, workspace, workspace_bytes, stream,
+                       num_query_tokens);
+  }
   const pa_shape e = multi_shape(shape, num_query_tokens);
   st = check_decode_shape(&e, max_context_len);
   if (st != PA_OK) return st;

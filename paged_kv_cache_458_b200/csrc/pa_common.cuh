@@ -22,6 +22,7 @@ enum DeviceErrorBits : unsigned int {
   kErrSlot = 1u << 2,         // an append slot is outside the pool
   kErrPair = 1u << 3,         // a copy pair names a block outside the pool
   kErrWaitTimeout = 1u << 4,  // an mbarrier wait ran past its time limit
+  kErrConfig = 1u << 5,       // a kernel could not lay out its shared memory (did nothing)
 };
 
 // Kernels receive the address of the per-device error word (read and
@@ -93,6 +94,13 @@ __device__ __forceinline__ void mbar_init_fence() {
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+// Raise the transaction count of the current phase without arriving: the
+// phase then completes once its arrivals are in and those bytes have landed.
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
 

@@ -172,13 +172,11 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
     }
     return;
   }
-  // With a shared-prefix plan this CTA covers part of [T, ctx) only.
-  const int OT = a.own_tokens;
-  const SeqSplit split = seq_split(a.plan, s, ctx, OT);
-  const int t_begin = split.base + part * OT;
+  const int PT = a.own_tokens;
+  const int t_begin = part * PT;
   if (t_begin >= ctx) return;
-  const int t_end = min(ctx, t_begin + OT);
-  const int n_parts_seq = split.total;
+  const int t_end = min(ctx, t_begin + PT);
+  const int n_parts_seq = (ctx + PT - 1) / PT;
   const int n_chunks = (t_end - t_begin + kChunk - 1) / kChunk;
   const int n_mine = warp < n_chunks ? (n_chunks - warp + NW - 1) / NW : 0;
 
@@ -386,7 +384,7 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
     if (direct) {
       a.out[qh * D + d] = Elem<T>::from_f(num / den);
     } else {
-      const size_t slot = qh * a.num_parts + split.slot0 + part;
+      const size_t slot = qh * a.num_parts + part;
       a.ws_acc[slot * D + d] = num;
       if (d == 0) {
         a.ws_ml[2 * slot] = M;
@@ -398,6 +396,9 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
 
 // Merge of the partitions of every (sequence, query head) that has more than
 // one.  One warp per (sequence, query head); lane l owns dims [l*VEC, l*VEC+VEC).
+// Rows are [num_seqs * query_tokens][Hq]: query t of sequence s attends to
+// ctx_s - query_tokens + t + 1 tokens.  With a shared-prefix plan a sequence's
+// partial count is in the plan (its partials are slots 0 .. count - 1).
 template <typename T, int D>
 __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a) {
   constexpr int VEC = D / 32;
@@ -405,30 +406,64 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a) {
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int pair = blockIdx.x * 4 + (threadIdx.x >> 5);
-  if (pair >= a.num_seqs * a.num_q_heads) return;
-  const int s = pair / a.num_q_heads;
-  int ctx = __ldg(a.context_lens + s);
-  ctx = max(0, min(ctx, a.max_context_len));
-  const int P = seq_split(a.plan, s, ctx, a.own_tokens).total;
+  const int Tq = a.query_tokens;
+  if (pair >= a.num_seqs * Tq * a.num_q_heads) return;
+  const int v = pair / a.num_q_heads;  // virtual sequence: query v % Tq of sequence v / Tq
+  int P;
+  if (a.plan2) {
+    P = __ldg(a.plan2 + v).y;
+  } else {
+    int ctx = __ldg(a.context_lens + v / Tq);
+    ctx = max(0, min(ctx, a.max_context_len)) - Tq + 1 + v % Tq;
+    P = ctx > 0 ? (ctx + a.own_tokens - 1) / a.own_tokens : 0;
+  }
   if (P <= 1) return;
   const size_t base = (size_t)pair * a.num_parts;
+  // (m, l) of partial p in lane p % 32: the reference M and each partial's
+  // weight 2^(m_p - M) come from warp reductions, not a loop of round trips
   float M = -INFINITY;
-  for (int p = 0; p < P; ++p) M = fmaxf(M, a.ws_ml[2 * (base + p)]);
+  for (int p0 = 0; p0 < P; p0 += 32) {
+    float m = p0 + lane < P ? a.ws_ml[2 * (base + p0 + lane)] : -INFINITY;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    M = fmaxf(M, m);
+  }
   float num[VEC];
 #pragma unroll
   for (int v = 0; v < VEC; ++v) num[v] = 0.f;
   float den = 0.f;
-  for (int p = 0; p < P; ++p) {
-    const float wt = exp2f(a.ws_ml[2 * (base + p)] - M);
-    den = fmaf(wt, a.ws_ml[2 * (base + p) + 1], den);
-    const float* row = a.ws_acc + (base + p) * D + lane * VEC;
-    if constexpr (VEC == 4) {
-      const float4 r = *reinterpret_cast<const float4*>(row);
-      num[0] = fmaf(wt, r.x, num[0]); num[1] = fmaf(wt, r.y, num[1]);
-      num[2] = fmaf(wt, r.z, num[2]); num[3] = fmaf(wt, r.w, num[3]);
-    } else {
-      const float2 r = *reinterpret_cast<const float2*>(row);
-      num[0] = fmaf(wt, r.x, num[0]); num[1] = fmaf(wt, r.y, num[1]);
+  for (int p0 = 0; p0 < P; p0 += 32) {
+    float wt = 0.f, lw = 0.f;
+    if (p0 + lane < P) {
+      wt = exp2f(a.ws_ml[2 * (base + p0 + lane)] - M);
+      lw = wt * a.ws_ml[2 * (base + p0 + lane) + 1];
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+    den += lw;
+    // partial rows four at a time: their loads are in flight together
+    const int n = min(32, P - p0);
+    for (int i = 0; i < n; i += 4) {
+      float r[4][VEC];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int p = min(i + u, n - 1);  // past the end: re-read the last row, weight 0
+        const float* row = a.ws_acc + (base + p0 + p) * D + lane * VEC;
+        if constexpr (VEC == 4) {
+          const float4 x = *reinterpret_cast<const float4*>(row);
+          r[u][0] = x.x; r[u][1] = x.y; r[u][2] = x.z; r[u][3] = x.w;
+        } else {
+          const float2 x = *reinterpret_cast<const float2*>(row);
+          r[u][0] = x.x; r[u][1] = x.y;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float w = __shfl_sync(0xffffffffu, wt, (i + u) & 31);
+        const float wu = i + u < n ? w : 0.f;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) num[v] = fmaf(wu, r[u][v], num[v]);
+      }
     }
   }
   const float inv = 1.f / den;
@@ -468,7 +503,7 @@ cudaError_t launch_typed(const DecodeArgs& a, const CUtensorMap& tk, const CUten
   if (e != cudaSuccess) return e;
   ++*launches;
   if (a.num_parts <= 1) return cudaSuccess;
-  const int pairs = a.num_seqs * a.num_q_heads;
+  const int pairs = a.num_seqs * a.query_tokens * a.num_q_heads;
   e = launch_pdl(decode_merge_kernel<T, D>, dim3((pairs + 3) / 4), dim3(128), 0, stream, a);
   if (e == cudaSuccess) ++*launches;
   return e;
@@ -515,7 +550,7 @@ cudaError_t launch_decode(const DecodeArgs& a, int dtype, int head_dim, int grou
 cudaError_t launch_decode_merge(const DecodeArgs& a, int dtype, int head_dim, cudaStream_t stream,
                                 int* launches) {
   if (a.num_parts <= 1 || a.num_seqs <= 0) return cudaSuccess;
-  const int pairs = a.num_seqs * a.num_q_heads;
+  const int pairs = a.num_seqs * a.query_tokens * a.num_q_heads;
   const dim3 grid((pairs + 3) / 4), block(128);
   cudaError_t e;
   if (dtype == 0) {

@@ -6,64 +6,68 @@
 // that costs CUDA cores about as much time as the HBM read once g >= 4.  This
 // kernel moves both products onto tcgen05.mma and keeps the read on TMA:
 //
-//   S^T[128 tok x N]  = K_tile[128 tok x 128 d] . Q^T[128 d x N]     (A K-major, B K-major)
-//   O^T[128 d x N]    = V_tile^T[128 d x 128 tok] . P^T[128 tok x N] (A MN-major, B MN-major)
+//   S^T[128 rows x N]  = K_tile[128 rows x 128 d] . Q^T[128 d x N]     (A K-major, B K-major)
+//   O^T[128 d x N]     = V_tile^T[128 d x 128 rows] . P^T[128 rows x N] (A MN-major, B MN-major)
 //
-// with fp16/bf16 operands and fp32 accumulators in tensor memory (TMEM).  The
-// N columns are query rows:
-//   - one sequence (the plain kernel): its g query heads, padded to N = 16;
-//     or, where the kv heads pair up and 2g <= 16, the 2g query heads of two
-//     kv heads.  Then a tile is 64 tokens of both heads as the 128 MMA rows
-//     (16-row groups of head 2e and of head 2e+1 alternate), so that one TMA
-//     box carries 4 KB (16 rows of both heads) instead of 2 KB: the rate at
-//     which one SM issues boxes bounds this kernel.  A row's logits against
-//     the other head's queries are computed and discarded (p = 0), which the
-//     tensor cores can afford;
+// with fp16/bf16 operands and fp32 accumulators in tensor memory (TMEM).
+//
+// Items.  An item is one partition (partition_tokens rows) of a row list of
+// one kv head (or of two), read for a set of query columns (N = 16 or 32):
+//   - a sequence: its tokens, for its g query heads; with several query
+//     tokens per sequence (verifying speculated tokens, chunked prefill:
+//     5688vip.com vLLM notes, section 2.2) for Tq x g columns, query t seeing
+//     tokens below ctx - Tq + t + 1, so that every K/V tile is read once for
+//     all of them;
+//   - where kv heads pair up, two heads at once: a tile is then 64 tokens of
+//     both heads as the 128 MMA rows (16-row groups of head 2e and of head
+//     2e+1 alternate), so that one TMA box carries 4 KB (16 rows of both heads)
+//     instead of 2 KB: the rate at which one SM issues boxes bounds this
+//     kernel.  A row's logits against the other head's queries are computed
+//     and discarded (p = 0), which the tensor cores can afford;
 //   - a group of sequences whose block tables begin with the same physical
-//     blocks (the shared-prefix kernel): members x g query rows, N = 32.  The
-//     blocks every member reads are then read once for all of them, which is
-//     what sharing blocks between sequences (a common prompt prefix, beam
-//     candidates forked from one parent) is for (zingnex.cn,
-//     "vLLM与PagedAttention深度剖析", section 3.2 item 3; jsqmd.com,
-//     "vLLM-v0.11.0性能实测", section 4.2: requests with the same prefix
-//     share pages).
+//     blocks (shared_prefix), for members x g columns: the row list is the
+//     T shared tokens, read once for every member (zingnex.cn,
+//     "vLLM与PagedAttention深度剖析", section 3.2 item 3: beam candidates share
+//     blocks; jsqmd.com, "vLLM-v0.11.0性能实测", section 4.2: requests with the
+//     same prefix share pages), then each member's own tokens, each run
+//     rounded up to 16 rows and seen by that member's columns only.  A
+//     sequence alone is a group of one with no shared tokens.
+// Every 16-row group of an item carries its owner (a member, or every member)
+// and its first token; every member its token limit and where its result
+// goes: the output itself (a single partial), a split-K slot, or nowhere (no
+// row of this partition is its).
 //
 // The softmax stays in fp32 on the CUDA cores: tcgen05.ld gives thread t (of
-// 128) the N logits of token t, and thread t writes its row of P.  The
-// output accumulates in TMEM across the tiles of an item: each column keeps a
+// 128) the logits of MMA row t, and thread t writes its row of P.  The output
+// accumulates in TMEM across the tiles of an item: each column keeps a
 // softmax reference m_ref that moves only when a logit exceeds it by more than
 // 8 (log2 units).  Then the tile's column maxima are found (a transposed warp
-// reduction, lane c ending with column c, plus shared memory), and thread d
-// folds row d of O^T into registers, rescaled by 2^(m_old - m_new).  On other
-// tiles nothing waits for the PV product: it is read once, at the end of the
-// item.  The products are pipelined by tile: S^T(j+1) is issued as soon as
-// every thread has read S^T(j), while tile j's softmax runs, and the softmax
-// of tile j waits for O^T(j-1) only to store P(j) (or to fold O^T).
-// The probabilities enter the PV product as two terms of the input type, hi =
-// round(p) and lo = round(p - hi), so they carry about 16 significant bits (a
-// bf16 P alone, 8 bits, can move a short context's output by more than 2e-3).
-// The two terms sit side by side as 2N columns of one PV product, so each V
-// slice is read once for both, into O^T hi and O^T lo, summed when O^T is read.
+// reduction plus shared memory), and thread d folds row d of O^T into
+// registers, rescaled by 2^(m_old - m_new).  On other tiles nothing waits for
+// the PV product: it is read once, at the end of the item.  The products are
+// pipelined by tile: S^T(j+1) is issued as soon as every thread has read
+// S^T(j), while tile j's softmax runs, and the softmax of tile j waits for
+// O^T(j-1) only to store P(j) (or to fold O^T).  The probabilities enter the
+// PV product as two terms of the input type, hi = round(p) and lo = round(p -
+// hi), so they carry about 16 significant bits (a bf16 P alone, 8 bits, can
+// move a short context's output by more than 2e-3); the two terms sit side by
+// side as 2N columns of one PV product, so each V slice is read once for both.
 //
-// Work, plain kernel: items (sequence, kv head or pair of kv heads, partition
-// of partition_tokens tokens, a multiple of 128) are numbered as in the
-// CUDA-core kernel (partition 0 of every (sequence, kv head) first, then the
-// further partitions of longer sequences).  Shared-prefix kernel: items
-// (group leader, kv head, partition of the shared tokens), numbered over the
-// leaders of the launch.  One persistent CTA per SM: a scheduler warp takes
-// items (its first one by number, then from a counter in the workspace whose
-// value carries the call's epoch), resolves each 16-token group of an item
-// through the block table and fills one of two item slots (descriptor, pool
-// rows, query rows), up to two items ahead; a producer warp then only issues
-// the tiles' tiled TMA loads, one box per lane (per tile: 8 groups of one
-// head or 4 groups of two heads, x {K, V} x two 64-element halves,
-// 128B-swizzled), into one of NST stages.  A dedicated MMA warp issues every
-// MMA and commits it to an mbarrier, so issuing them never holds up the
-// softmax; the compute warps
-// consume tiles in order and tell it through two more mbarriers when S^T(g)
-// has been read and when P(g) has been written.  Tokens at or past the end of
-// the item are masked in P and their V rows are zeroed in shared memory before
-// the PV product, so stale or NaN rows never reach the result.
+// Warps.  One persistent CTA per SM.  A scheduler warp takes items (its first
+// one by number, then from a counter in the workspace whose value carries the
+// call's epoch), resolves each 16-row group through its block table and fills
+// one of two item slots (descriptor, pool rows, group and member tables, and
+// the query rows by one TMA box), up to two items ahead; a producer warp
+// issues the tiles' tiled TMA loads, one box per lane (per tile: 8 groups of
+// one head or 4 groups of two heads, x {K, V} x two 64-element halves,
+// 128B-swizzled), into one of three stages; a dedicated MMA warp issues every
+// MMA and commits it to an mbarrier; the compute warps consume tiles in order
+// and tell it through two more mbarriers when S^T(g) has been read and when
+// P(g) has been written.  Items are numbered full partitions first and the
+// shorter last partitions after them, so the CTAs finish close together.
+// Rows that are no token of any column are masked in P and their V rows are
+// zeroed in shared memory before the PV product, so stale or NaN rows never
+// reach the result.
 //
 // Split-K partials and the merge kernel are shared with the CUDA-core path.
 //
@@ -84,13 +88,18 @@
 namespace pa {
 namespace tc {
 
-constexpr int kTile = 128;          // tokens per MMA tile (M)
+constexpr int kTile = 128;          // MMA rows per tile (M)
 constexpr int kD = 128;             // head_dim of this path
-constexpr int kGroupRows = 16;      // token rows per TMA box (a block is a multiple)
-constexpr int kSlots = 2;           // item slots (descriptor + query rows)
+constexpr int kGroupRows = 16;      // rows per TMA box (a block is a multiple)
+constexpr int kSlots = 2;           // item slots
+constexpr int kStages = 3;          // K/V stages of 64 KB
+constexpr int kMaxGroups = 32;      // 16-row groups per item (partition_tokens <= 512)
+constexpr int kMaxUnits = 512;      // sequences (or group leaders) per launch
+// Where a member's result for an item goes (codes >= 0 are split-K slots).
+constexpr int kSkip = -1, kDirect = -2, kZero = -3;
 
 // Compute warpgroups split the NC query columns: warp w of the compute
-// warps reads TMEM lane quarter w % 4 (tokens 32 (w % 4) .. +31, output rows
+// warps reads TMEM lane quarter w % 4 (MMA rows 32 (w % 4) .. +31, output rows
 // likewise) and handles columns [(w / 4) NCW, (w / 4 + 1) NCW).  More warps
 // per scheduler hide the latency of the per-column softmax arithmetic.
 template <int NC>
@@ -102,47 +111,49 @@ struct Warps {
   static_assert(kNCW * kNWG == NC, "columns split evenly");
 };
 
-// Per kernel kind: N columns, sequences per launch (the scheduler warp holds
-// their prefix counts in registers) and TMEM columns (S^T in [0, N); O^T in [N, 3N), its hi part
-// in [N, 2N) and its lo part in [2N, 3N), rounded up to a power of two).
-template <bool GROUP>
-struct Cfg {
-  static constexpr int kN = GROUP ? 32 : 16;
-  static constexpr int kMaxSeqs = GROUP ? kSharedPrefixSeqsPerLaunch : 512;
-  static constexpr uint32_t kTmemCols = GROUP ? 128 : 64;
-};
-
-template <int NST, int N>
+// Shared memory.  A small region at the start of the dynamic allocation
+// (barriers and per-item tables), then, from the next 1024-byte boundary, the
+// stages, the query slots and P, whose swizzled layouts need that alignment.
+// TMEM: S^T in [0, N); O^T hi in [N, 2N), O^T lo in [2N, 3N).
+// With an E4M3 cache (KV8) the stages only land the 8-bit tiles (32 KB); the
+// compute warps widen each one into a 16-bit K tile (one buffer) and a 16-bit
+// V tile (two buffers, alternating by tile), which the MMAs read.
+template <int N, bool KV8>
 struct Layout {
-  // offsets from a 1024-byte aligned base
-  static constexpr int kStageBytes = 2 * kTile * kD * 2;      // K tile then V tile (64 KB)
-  static constexpr int kHalf = kTile * 128;                    // one 64-element half of a tile (16 KB)
-  static constexpr int kStages = 0;
-  static constexpr int kQ = kStages + NST * kStageBytes;       // [slots][2 halves][N rows][128 B]
+  // small region (byte offsets from the dynamic base)
+  // barriers: full[3], empty[3], ready[2], free[2], meta[2], qk, pv, drain, s_free, p_ready, conv
+  static constexpr int kNumBars = 2 * kStages + 3 * kSlots + 6;
+  static constexpr int kBars = 0;
+  static constexpr int kMisc = kBars + kNumBars * 8;        // tmem address, abort flag, accumulate flags [2]
+  static constexpr int kDesc = kMisc + 16;                  // [slots][16] int
+  static constexpr int kRows = kDesc + kSlots * 16 * 4;     // [slots][2][32] int: pool rows of the groups
+  static constexpr int kGTok = kRows + kSlots * 64 * 4;     // [slots][32] int: first token of each group
+  static constexpr int kGMeta = kGTok + kSlots * 32 * 4;    // [slots][32] int: owner + 1 | valid rows << 8
+  static constexpr int kMLim = kGMeta + kSlots * 32 * 4;    // [slots][32] int: token limit of each member
+  static constexpr int kMCode = kMLim + kSlots * 32 * 4;    // [slots][32] int: destination of each member
+  static constexpr int kRed = kMCode + kSlots * 32 * 4;     // [4 warps][N] f32
+  static constexpr int kStat = kRed + 4 * N * 4;            // m[N], then l[N], f32
+  static constexpr int kSmall = kStat + 2 * N * 4;
+  // big region (byte offsets from the first 1024-byte boundary after the small one)
+  static constexpr int kHalf = kTile * 128;  // a 64-element half of a 16-bit tile, or an 8-bit tile (16 KB)
+  static constexpr int kStageBytes = KV8 ? 2 * kHalf : 4 * kHalf;  // K tile then V tile
+  static constexpr int kStages0 = 0;
+  static constexpr int kK16 = kStages0 + kStages * kStageBytes;   // KV8: widened K [2 halves]
+  static constexpr int kV16 = kK16 + (KV8 ? 2 * kHalf : 0);       // KV8: widened V [2][2 halves]
+  static constexpr int kQ = kV16 + (KV8 ? 4 * kHalf : 0);         // [slots][2 halves][N rows][128 B]
   static constexpr int kQBytes = 2 * N * 128;
-  static constexpr int kP = kQ + kSlots * kQBytes;             // P hi, then P lo
-  static constexpr int kPBytes = kTile * N * 2;                // [N/16 atoms][128 tok][32 B]
-  static constexpr int kPAtom = kTile * 32;                    // bytes of one 16-column atom
-  static constexpr int kRed = kP + 2 * kPBytes;                // [4 warps][N] f32
-  static constexpr int kStat = kRed + 4 * N * 4;               // m[N], then alpha[N] or l[N], f32
-  static constexpr int kDesc = kStat + 2 * N * 4;              // [slots][8] int
-  static constexpr int kRows = kDesc + kSlots * 8 * 4;         // [slots][2][32] int: pool rows of
-                                                               // the item's 16-token groups
-  static constexpr int kBars = kRows + kSlots * 2 * 32 * 4;
-  // full[NST], empty[NST], ready[slots], free[slots], meta[slots], qk, pv, drain,
-  // s_free, p_ready
-  static constexpr int kNumBars = 2 * NST + 3 * kSlots + 5;
-  static constexpr int kMisc = kBars + kNumBars * 8;           // tmem address, abort flag,
-                                                               // accumulate flags [2]
-  static constexpr int kUsed = kMisc + 16;
-  static constexpr int kAlloc = kUsed + 1024;                  // room to align the base
+  static constexpr int kP = kQ + kSlots * kQBytes;          // P hi, then P lo
+  static constexpr int kPBytes = kTile * N * 2;             // [N/16 atoms][128 rows][32 B]
+  static constexpr int kPAtom = kTile * 32;                 // bytes of one 16-column atom
+  static constexpr int kBig = kP + 2 * kPBytes;
+  // the allocation when the dynamic base is 1024-aligned (the kernel checks)
+  static constexpr int kAlloc = (kSmall + 1023) / 1024 * 1024 + kBig;
   static_assert(kQ % 1024 == 0 && kQBytes % 1024 == 0 && kP % 256 == 0, "swizzle atoms");
   static_assert(kAlloc <= 232448, "shared memory per CTA");
 };
 
-// Item descriptor fields (kDCtx: the context of a plain item, the number of
-// member sequences of a shared-prefix item).
-enum { kDS = 0, kDKvh, kDPart, kDBegin, kDEnd, kDTiles, kDParts, kDCtx };
+// Item descriptor fields.
+enum { kDS = 0, kDKvh, kDPart, kDBegin, kDEnd, kDTiles, kDMembers, kDVbase, kDNumFields };
 
 // ---------------------------------------------------------------------------
 // tcgen05 / descriptor helpers
@@ -275,40 +286,57 @@ __device__ __forceinline__ float column_reduce(float (&v)[NC], int lane) {
   return v[0];
 }
 
-// Item number -> (sequence, kv head, partition); see the file comment.  The
-// first n_first numbers are partition 0 of every (sequence, kv head); the
-// rest are counted by prefix[] (prefix[s] = items of sequences before s, per
-// kv head, non-decreasing), numbered from `part0` within a sequence.  The
-// warp holds prefix[] in registers: lane l has prefix[32 k + l] in pre[k]
-// (INT_MAX past prefix[S]).  Called by all 32 lanes.
+// Entry k >> 5 of a per-lane register array, then lane k & 31's copy of it.
 template <int PPL>
-__device__ __forceinline__ void locate(int f, int n_first, int Hkv, const int (&pre)[PPL], int part0,
-                                       int lane, int& s, int& kvh, int& part) {
-  if (f < n_first) {
-    s = f / Hkv;
-    kvh = f % Hkv;
-    part = 0;
-    return;
-  }
-  const int g = f - n_first;
-  kvh = g % Hkv;
-  const int r = g / Hkv;
-  // largest s with prefix[s] <= r: the number of such entries, less one
+__device__ __forceinline__ int lane_entry(const int (&v)[PPL], int k) {
+  int mine = 0;
+#pragma unroll
+  for (int i = 0; i < PPL; ++i)
+    if (i == (k >> 5)) mine = v[i];
+  return __shfl_sync(0xffffffffu, mine, k & 31);
+}
+
+// Largest unit u with pre[u] <= r (pre non-decreasing, INT_MAX past the end).
+template <int PPL>
+__device__ __forceinline__ int last_at_most(const int (&pre)[PPL], int r) {
   int cnt = 0;
 #pragma unroll
   for (int k = 0; k < PPL; ++k) cnt += pre[k] <= r ? 1 : 0;
-  s = __reduce_add_sync(0xffffffffu, cnt) - 1;
-  int mine = 0;
-#pragma unroll
-  for (int k = 0; k < PPL; ++k)
-    if (k == (s >> 5)) mine = pre[k];
-  part = part0 + r - __shfl_sync(0xffffffffu, mine, s & 31);
+  return __reduce_add_sync(0xffffffffu, cnt) - 1;
 }
 
-// Work counter tagged with the call's epoch in bits 24..63 (see pa_decode.cu).
-__device__ __forceinline__ int take_item(unsigned long long* ctr, unsigned long long epoch,
-                                         unsigned int* err) {
-  const unsigned long long old = atomicAdd(ctr, 1ull);
+// Item number -> (unit, kv unit, partition).  A unit (a sequence, or a group
+// leader) whose row list holds R rows has R / PT full partitions and, when PT
+// does not divide R (or R == 0), one last shorter one.  Items 0 .. Hu F - 1
+// are the full partitions of every unit (F in all), the rest the last ones;
+// the kv unit varies fastest.  pre_f / pre_p: exclusive prefix counts of full
+// / last partitions over the units, lane l holding entries l, l + 32, ...
+// Called by all 32 lanes.
+template <int PPL>
+__device__ __forceinline__ void locate(int f, int Hu, int F, const int (&pre_f)[PPL],
+                                       const int (&pre_p)[PPL], int& u, int& kvu, int& part) {
+  if (f < Hu * F) {
+    kvu = f % Hu;
+    const int r = f / Hu;
+    u = last_at_most(pre_f, r);
+    part = r - lane_entry(pre_f, u);
+  } else {
+    const int g = f - Hu * F;
+    kvu = g % Hu;
+    u = last_at_most(pre_p, g / Hu);
+    part = lane_entry(pre_f, u + 1) - lane_entry(pre_f, u);
+  }
+}
+
+// Work counter tagged with the call's epoch in bits 24..63 (see pa_decode.cu):
+// take_begin issues the increment, take_end (later, so that the round trip
+// overlaps other work) reads its result, installing this call's epoch if the
+// word still carries another one.
+__device__ __forceinline__ unsigned long long take_begin(unsigned long long* ctr) {
+  return atomicAdd(ctr, 1ull);
+}
+__device__ __forceinline__ int take_end(unsigned long long* ctr, unsigned long long old,
+                                        unsigned long long epoch, unsigned int* err) {
   if ((old >> 24) == epoch) return (int)(old & 0xffffffull);
   for (int round = 0; round < (1 << 20); ++round) {
     const unsigned long long cur = atomicAdd(ctr, 0ull);
@@ -319,76 +347,122 @@ __device__ __forceinline__ int take_item(unsigned long long* ctr, unsigned long 
   return -1;
 }
 
-// Query columns of a kernel kind: members x g (shared-prefix), 2g (an item of
-// two kv heads), g.
-template <int G, bool GROUP, bool PAIR>
-__host__ __device__ constexpr int columns() { return GROUP ? Cfg<GROUP>::kN : (PAIR ? 2 * G : G); }
+// Columns an item of this launch fills at most: members x g with shared
+// prefixes (32), else query tokens x heads per item x g.
+__host__ __device__ inline int tc_columns(int group, int query_tokens, bool pair, bool grouped) {
+  return grouped ? kTcMaxColumns : query_tokens * (pair ? 2 : 1) * group;
+}
 
-template <typename T, int G, int NST, bool GROUP, bool PAIR>
-__global__ void __launch_bounds__(Warps<columns<G, GROUP, PAIR>()>::kThreads, 1)
+// Sixteen E4M3 codes (one 16-byte piece of a row, first element in the lowest
+// byte) -> sixteen 16-bit values of T, two per word, first element in the low
+// half.  Exact: every E4M3 value is an f16 (the hardware conversion) and a bf16.
+template <typename T>
+__device__ __forceinline__ void widen16(const uint4 x, uint32_t (&w)[8]) {
+  const uint32_t in[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int hw = 0; hw < 2; ++hw) {
+      const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(
+          static_cast<__nv_fp8x2_storage_t>((in[i] >> (16 * hw)) & 0xffffu), __NV_E4M3);
+      uint32_t r;
+      if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        const __nv_bfloat162 b = __float22bfloat162_rn(__half22float2(*reinterpret_cast<const __half2*>(&h)));
+        r = *reinterpret_cast<const uint32_t*>(&b);
+      } else {
+        r = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      w[2 * i + hw] = r;
+    }
+}
+
+template <typename T, int NC, bool PAIR, bool KV8>
+__global__ void __launch_bounds__(Warps<NC>::kThreads, 1)
 decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q) {
-  using C = Cfg<GROUP>;
-  constexpr int N = C::kN;
-  constexpr int NC = columns<G, GROUP, PAIR>();  // columns that carry query rows
-  // An item covers kHeads kv heads; a tile is kTok tokens of each, as kTile
-  // MMA rows (with two heads, 16-row groups of head 2e and head 2e+1 alternate)
+  constexpr int N = NC <= 16 ? 16 : 32;          // MMA columns
+  constexpr uint32_t kTmemCols = N == 16 ? 64 : 128;
+  // A tile is kTok tokens of each of the item's kHeads kv heads, as kTile MMA
+  // rows (with two heads, 16-row groups of head 2e and head 2e+1 alternate)
   constexpr int kHeads = PAIR ? 2 : 1;
   constexpr int kTok = kTile / kHeads;
-  static_assert(!(GROUP && PAIR), "a shared-prefix item covers one kv head");
+  constexpr int kGroupsPerTile = kTok / kGroupRows;
   using W = Warps<NC>;
   constexpr int kComputeThreads = W::kCompute, kThreads = W::kThreads, NCW = W::kNCW;
   constexpr int kComputeWarps = kComputeThreads / 32;
   constexpr int kMmaWarp = kComputeWarps, kProducerWarp = kComputeWarps + 1,
                 kSchedWarp = kComputeWarps + 2;
-  using L = Layout<NST, N>;
+  using L = Layout<N, KV8>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr uint32_t kIdescQK = instr_desc(kBf16 ? 1 : 0, 0, 0, kTile, N);
   // PV has 2N columns: P hi and P lo sit in consecutive 16-column atoms, so one
   // MMA reads each V slice once for both and writes O^T hi and O^T lo side by side
   constexpr uint32_t kIdescPV = instr_desc(kBf16 ? 1 : 0, 1, 1, kTile, 2 * N);
-  static_assert(GROUP || kHeads * G <= N, "query heads per tile");
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(16) unsigned char smem_raw[];
 
-  pdl_wait();  // the kernels before this decode (append, plan) must have landed
-  pdl_launch_dependents();
+  // Until pdl_wait() below, this CTA touches only its own shared and tensor
+  // memory: that part overlaps the end of the kernel before it on the stream.
+  // The big region starts at the first 1024-byte boundary after the small one;
+  // the allocation assumes a 1024-aligned base.  Any other base that leaves
+  // too little room is reported, and the CTA does nothing.
+  unsigned char* smem;
+  {
+    uint32_t dyn;
+    asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t off = ((raw + L::kSmall + 1023u) & ~1023u) - raw;
+    if (off + (uint32_t)L::kBig > dyn) {
+      pdl_wait();
+      if (threadIdx.x == 0) report(a.err, kErrConfig);
+      return;
+    }
+    smem = smem_raw + off;
+  }
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int S = a.num_seqs, Hkv = a.num_kv_heads, PT = a.partition_tokens;
-  int* desc_all = reinterpret_cast<int*>(smem + L::kDesc);
-  int* rows_all = reinterpret_cast<int*>(smem + L::kRows);
-  float* red = reinterpret_cast<float*>(smem + L::kRed);
-  float* stat = reinterpret_cast<float*>(smem + L::kStat);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-  const uint32_t bars = smem_addr(smem + L::kBars);
+  const int Hkv = a.num_kv_heads, PT = a.partition_tokens, G = a.group, Tq = a.query_tokens;
+  const bool grouped = a.plan != nullptr;
+  int* desc_all = reinterpret_cast<int*>(smem_raw + L::kDesc);
+  int* rows_all = reinterpret_cast<int*>(smem_raw + L::kRows);
+  int* gtok_all = reinterpret_cast<int*>(smem_raw + L::kGTok);
+  int* gmeta_all = reinterpret_cast<int*>(smem_raw + L::kGMeta);
+  int* mlim_all = reinterpret_cast<int*>(smem_raw + L::kMLim);
+  int* mcode_all = reinterpret_cast<int*>(smem_raw + L::kMCode);
+  float* red = reinterpret_cast<float*>(smem_raw + L::kRed);
+  float* stat = reinterpret_cast<float*>(smem_raw + L::kStat);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem_raw + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + L::kMisc + 4);
+  volatile int* acc_flag = reinterpret_cast<volatile int*>(smem_raw + L::kMisc + 8);  // [2]
+  const uint32_t bars = smem_addr(smem_raw + L::kBars);
   auto full_bar = [&](int st) { return bars + st * 8; };
-  auto empty_bar = [&](int st) { return bars + (NST + st) * 8; };
-  auto ready_bar = [&](int sl) { return bars + (2 * NST + sl) * 8; };
-  auto free_bar = [&](int sl) { return bars + (2 * NST + kSlots + sl) * 8; };
-  auto meta_bar = [&](int sl) { return bars + (2 * NST + 2 * kSlots + sl) * 8; };
-  const uint32_t qk_bar = bars + (2 * NST + 3 * kSlots) * 8;
+  auto empty_bar = [&](int st) { return bars + (kStages + st) * 8; };
+  auto ready_bar = [&](int sl) { return bars + (2 * kStages + sl) * 8; };
+  auto free_bar = [&](int sl) { return bars + (2 * kStages + kSlots + sl) * 8; };
+  auto meta_bar = [&](int sl) { return bars + (2 * kStages + 2 * kSlots + sl) * 8; };
+  const uint32_t qk_bar = bars + (2 * kStages + 3 * kSlots) * 8;
   const uint32_t pv_bar = qk_bar + 8;
   const uint32_t drain_bar = qk_bar + 16;
   const uint32_t s_free_bar = qk_bar + 24;   // compute warps have read S^T(g)
   const uint32_t p_ready_bar = qk_bar + 32;  // compute warps have written P(g)
-  volatile int* acc_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);  // [2]
-  const uint32_t sm_stages = smem_addr(smem + L::kStages);
+  const uint32_t conv_bar = qk_bar + 40;     // KV8: compute warps have widened tile g
+  const uint32_t sm_stages = smem_addr(smem + L::kStages0);
   const uint32_t sm_q = smem_addr(smem + L::kQ);
   const uint32_t sm_p = smem_addr(smem + L::kP);
+  // query rows one item's TMA box fills (the rest of the N rows stay zero)
+  const int q_rows = grouped ? kTcMaxColumns : Tq * kHeads * G;
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(tmem_holder)),
-                 "r"(C::kTmemCols)
+                 "r"(kTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (tid == 0) {
-    for (int st = 0; st < NST; ++st) {
+    for (int st = 0; st < kStages; ++st) {
       mbar_init(full_bar(st), 1);
-      mbar_init(empty_bar(st), 1);
+      // a stage is released by the MMA warp's commit, or with an 8-bit cache
+      // by every compute warp once it has widened the tile
+      mbar_init(empty_bar(st), KV8 ? kComputeWarps : 1);
     }
     for (int sl = 0; sl < kSlots; ++sl) {
       mbar_init(ready_bar(sl), 1);
@@ -400,69 +474,73 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     mbar_init(drain_bar, 1);
     mbar_init(s_free_bar, kComputeWarps);
     mbar_init(p_ready_bar, kComputeWarps);
+    mbar_init(conv_bar, kComputeWarps);
     *abort_flag = 0;
     mbar_init_fence();
   }
-  // Query rows that no item fills stay zero (padded heads); a shared-prefix
-  // item fills members x g rows, so the slots start all zero.
-  constexpr int kRow0 = GROUP ? 0 : kHeads * G;
-  constexpr int kPad = N - kRow0;
-  if constexpr (kPad > 0) {
-    for (int i = tid; i < kSlots * 2 * kPad * 8; i += kThreads) {
-      const int chunk = i % 8, row = kRow0 + (i / 8) % kPad, half = (i / 8 / kPad) % 2,
-                slot = i / 8 / kPad / 2;
-      *reinterpret_cast<uint4*>(smem + L::kQ + slot * L::kQBytes + half * N * 128 + row * 128 +
-                                chunk * 16) = make_uint4(0, 0, 0, 0);
-    }
+  // Query rows past the item's box stay zero (padded columns).
+  for (int i = tid; i < kSlots * 2 * N * 8; i += kThreads) {
+    const int row = (i / 8) % N;
+    if (row >= q_rows)
+      *reinterpret_cast<uint4*>(smem + L::kQ + (i / 8 / N) * N * 128 + row * 128 + (i % 8) * 16) =
+          make_uint4(0, 0, 0, 0);
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  pdl_wait();  // the kernels before this decode (append, plan, expansion) have landed
+  pdl_launch_dependents();
 
   if (warp == kSchedWarp) {
     // =====================================================================
-    // scheduler warp: takes items, resolves them (sequence, kv head, token
-    // range, the pool row of each 16-token group) and fills an item slot:
+    // scheduler warp: takes items, resolves them (unit, kv head, row range,
+    // the pool row, owner and first token of each 16-row group, each
+    // member's token limit and destination) and fills an item slot:
     // descriptor and rows (meta, for the producer), query rows (ready, for
     // the MMA and compute warps).  It runs up to two items ahead of the
     // compute warps, so none of its global round trips holds up the loads.
     // =====================================================================
-    // Per sequence, the items numbered through prefix[]: further partitions
-    // (plain) or the shared partitions of a group leader (shared-prefix).
-    constexpr int PPL = C::kMaxSeqs / 32 + 1;  // prefix[0..S] over the lanes
-    int pre[PPL];
-    int carry = 0;
+    const int S = a.num_seqs;
+    constexpr int PPL = kMaxUnits / 32 + 1;  // prefix[0..S] over the lanes
+    int pre_f[PPL], pre_p[PPL];
+    int carry_f = 0, carry_p = 0;
 #pragma unroll
     for (int k = 0; k < PPL; ++k) {
-      const int s = k * 32 + lane;  // this lane's entry prefix[s] = carry + counts before s
-      int cnt = 0;
+      const int s = k * 32 + lane;  // this lane's unit
+      int full = 0, last = 0;
       if (s < S) {
-        if constexpr (GROUP) {
-          const int4 pl = __ldg(a.plan + s);
-          cnt = (pl.x == 0 && pl.y >= 2) ? pl.w : 0;
+        int rows = -1;  // rows of the unit's list; -1: not a unit
+        if (grouped) {
+          if (__ldg(a.plan + s).x == 0) rows = __ldg(a.plan2 + s).w;
         } else {
           int ctx = __ldg(a.context_lens + s);
           if (ctx < 0 || ctx > a.max_context_len) {
             if (blockIdx.x == 0) report(a.err, kErrContextLen);
             ctx = max(0, min(ctx, a.max_context_len));
           }
-          cnt = max((ctx + PT - 1) / PT - 1, 0);
+          rows = ctx;
+        }
+        if (rows >= 0) {
+          full = rows / PT;
+          last = (rows % PT != 0 || rows == 0) ? 1 : 0;
         }
       }
-      int incl = cnt;
+      int inc_f = full, inc_p = last;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
+        const int tf = __shfl_up_sync(0xffffffffu, inc_f, o);
+        const int tp = __shfl_up_sync(0xffffffffu, inc_p, o);
+        if (lane >= o) inc_f += tf, inc_p += tp;
       }
-      pre[k] = s <= S ? carry + incl - cnt : INT_MAX;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
+      pre_f[k] = s <= S ? carry_f + inc_f - full : INT_MAX;
+      pre_p[k] = s <= S ? carry_p + inc_p - last : INT_MAX;
+      carry_f += __shfl_sync(0xffffffffu, inc_f, 31);
+      carry_p += __shfl_sync(0xffffffffu, inc_p, 31);
     }
-    const int Hitem = Hkv / kHeads;  // kv-head units of the item numbering
-    const int n_first = GROUP ? 0 : S * Hitem;
-    const int total = n_first + Hitem * carry;
+    const int Hu = Hkv / kHeads;  // kv units of the item numbering
+    const int total = Hu * (carry_f + carry_p);
 
     bool ok = true;
     int it = 0;
@@ -477,7 +555,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           break;
         }
       }
-      int* desc = desc_all + slot * 8;
+      int* desc = desc_all + slot * 16;
       if (f >= total) {
         if (lane == 0) {
           desc[kDTiles] = -1;  // end of work
@@ -486,93 +564,128 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         }
         break;
       }
-      int s, kvh, part;
-      locate(f, n_first, Hitem, pre, GROUP ? 0 : 1, lane, s, kvh, part);
-      kvh *= kHeads;  // the item's first kv head
-      int t_end, ctx_or_members;
-      const int t_begin = part * PT;
-      if constexpr (GROUP) {
+      // the next item's number, fetched while this one is resolved
+      unsigned long long ticket = 0;
+      if (lane == 0) ticket = take_begin(a.work_counter);
+      int s, kvu, part;
+      locate(f, Hu, carry_f, pre_f, pre_p, s, kvu, part);
+      const int kvh = kvu * kHeads;  // the item's first kv head
+      // query rows: one TMA box per 64-element half, [members][heads][64]
+      const uint32_t rb = ready_bar(slot);
+      if (lane == 0) {
+        const int qrow = grouped ? a.seq_offset + s : (a.seq_offset + s) * Tq;
+        mbar_expect_tx(rb, 2 * q_rows * 128);  // the phase also needs the arrival below
+        tma_load_3d(sm_q + slot * L::kQBytes, &tm_q, rb, 0, kvh * G, qrow);
+        tma_load_3d(sm_q + slot * L::kQBytes + N * 128, &tm_q, rb, 64, kvh * G, qrow);
+      }
+      // ---- members (lane m): token limit, destination of the result; the
+      // row list of the item
+      int members, T, n_list, vbase;  // shared rows, rows in the unit's list
+      int m_ctx = 0, m_off = 0, m_code = kSkip;
+      const int p0 = part * PT;
+      if (grouped) {
         const int4 pl = __ldg(a.plan + s);
-        t_end = min(pl.z, t_begin + PT);
-        ctx_or_members = pl.y;
+        members = pl.y;
+        T = pl.z;
+        const int p_sh = pl.w;
+        vbase = s;
+        int m_slots = 0;
+        if (lane < members) {
+          const int4 p2 = __ldg(a.plan2 + s + lane);
+          m_off = p2.x;
+          m_slots = p2.y;
+          m_ctx = max(0, min(__ldg(a.context_lens + s + lane), a.max_context_len));
+        }
+        n_list = __shfl_sync(0xffffffffu, __ldg(a.plan2 + s).w, 0);
+        if (lane < members) {
+          const int own = m_ctx - T;
+          const int first_own = max(m_off / PT, p_sh);
+          const bool mine = part < p_sh || (own > 0 && part >= m_off / PT && part <= (m_off + own - 1) / PT);
+          if (m_ctx == 0) m_code = part == 0 ? kZero : kSkip;
+          else if (!mine) m_code = kSkip;
+          else if (m_slots == 1) m_code = kDirect;
+          else m_code = part < p_sh ? part : p_sh + part - first_own;
+        }
       } else {
         const int ctx = max(0, min(__ldg(a.context_lens + s), a.max_context_len));
-        t_end = min(ctx, t_begin + PT);
-        ctx_or_members = ctx;
-      }
-      const int n_tok = max(0, t_end - t_begin);
-      const int n_tiles = (n_tok + kTok - 1) / kTok;
-      const int n_groups = (n_tok + kGroupRows - 1) / kGroupRows;  // <= 32
-      // With 8-token blocks (half_boxes) rows 8..15 of a group have their own
-      // entry; past the end of the item they re-read the first block (masked).
-      const int32_t* table = a.block_tables + (size_t)s * a.max_blocks_per_seq;
-      auto resolve = [&](int tok) {
-        const int blk = __ldg(table + tok / a.block_size);
-        if (blk < 0 || blk >= a.num_blocks) {
-          report(a.err, kErrBlockId);
-          return a.num_blocks * a.block_size;  // outside the map: TMA fills zeros
+        members = Tq;
+        T = ctx;  // every row is every query's, up to its limit
+        n_list = ctx;
+        vbase = s * Tq;
+        if (lane < Tq) {
+          m_ctx = ctx - Tq + 1 + lane;  // causal limit of query token `lane`
+          const int P_t = m_ctx > 0 ? (m_ctx + PT - 1) / PT : 0;
+          if (m_ctx <= 0) m_code = part == 0 ? kZero : kSkip;
+          else if (part >= P_t) m_code = kSkip;
+          else if (P_t == 1) m_code = kDirect;
+          else m_code = part;
         }
-        return blk * a.block_size + tok % a.block_size;
-      };
+      }
+      const int t_end = min(n_list, p0 + PT);
+      const int n_rows = max(0, t_end - p0);
+      const int n_tiles = (n_rows + kTok - 1) / kTok;
+      const int n_groups = (n_rows + kGroupRows - 1) / kGroupRows;  // <= 32
+      // ---- 16-row groups (lane i): owner, first token, valid rows, pool rows
+      int g_own = -1, g_tok = 0, g_valid = 0, g_row = 0, g_row2 = 0;
+      const int r0 = p0 + lane * kGroupRows;
+      // own rows: the member whose run holds r0 (runs are in member order,
+      // offsets non-decreasing; an empty run holds nothing)
+      int own = 0;
+      for (int m = 1; m < members; ++m)
+        if (__shfl_sync(0xffffffffu, m_off, m) <= r0) own = m;
+      const int own_off = __shfl_sync(0xffffffffu, m_off, own);
+      const int own_ctx = __shfl_sync(0xffffffffu, m_ctx, own);
       if (lane < n_groups) {
-        const int tok = t_begin + lane * kGroupRows;
-        const int row = resolve(tok);
+        int seq = s, lim;
+        if (r0 < T) {
+          g_tok = r0;
+          lim = T;
+        } else {
+          g_own = own;
+          g_tok = T + r0 - own_off;
+          lim = own_ctx;
+          seq = s + own;
+        }
+        g_valid = min(kGroupRows, lim - g_tok);
+        // With 8-token blocks (half_boxes) rows 8..15 of a group have their own
+        // entry; past the group's valid rows they re-read the first block (masked).
+        const int32_t* table = a.block_tables + (size_t)seq * a.max_blocks_per_seq;
+        auto resolve = [&](int tok) {
+          const int blk = __ldg(table + tok / a.block_size);
+          if (blk < 0 || blk >= a.num_blocks) {
+            report(a.err, kErrBlockId);
+            return a.num_blocks * a.block_size;  // outside the map: TMA fills zeros
+          }
+          return blk * a.block_size + tok % a.block_size;
+        };
+        g_row = resolve(g_tok);
+        if (a.half_boxes) g_row2 = g_valid > kGroupRows / 2 ? resolve(g_tok + kGroupRows / 2) : g_row;
+      }
+      {
         int* rows = rows_all + slot * 64;
-        rows[lane] = row;
-        if (a.half_boxes) rows[32 + lane] = tok + kGroupRows / 2 < t_end ? resolve(tok + kGroupRows / 2) : row;
+        rows[lane] = g_row;
+        rows[32 + lane] = g_row2;
+        gtok_all[slot * 32 + lane] = g_tok;
+        gmeta_all[slot * 32 + lane] = (g_own + 1) | (max(g_valid, 0) << 8);
+        mlim_all[slot * 32 + lane] = lane < members ? m_ctx : -1;
+        mcode_all[slot * 32 + lane] = lane < members ? m_code : kSkip;
       }
-      if constexpr (GROUP) {
-        // members x g query rows, 16-byte pieces stored in the 128B-swizzled
-        // K-major layout the QK descriptor reads (piece c of row r at c ^ (r & 7))
-        const int rows = ctx_or_members * G;
-        const uint32_t qs = sm_q + slot * L::kQBytes;
-        for (int i = lane; i < rows * 16; i += 32) {
-          const int r = i >> 4, cc = i & 15;
-          const int m = r / G, h = r % G;
-          const size_t qrow = (size_t)(a.seq_offset + s + m) * a.num_q_heads + kvh * G + h;
-          const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.q + qrow * kD) + cc);
-          const uint32_t dst = qs + (cc >> 3) * N * 128 + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y),
-                       "r"(v.z), "r"(v.w)
-                       : "memory");
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      }
-      // shared-prefix item: bit m set when member m's result is this
-      // partition alone (written directly, not as a split-K partial)
-      int direct_mask = 0;
-      if constexpr (GROUP) {
-        bool dm = false;
-        if (lane < ctx_or_members) {
-          const int ctx = max(0, min(__ldg(a.context_lens + s + lane), a.max_context_len));
-          dm = seq_split(a.plan, s + lane, ctx, a.own_tokens).total <= 1;
-        }
-        direct_mask = (int)__ballot_sync(0xffffffffu, dm);
-      }
-      __syncwarp();  // every lane's rows (and query rows) before the arrivals
+      __syncwarp();  // every lane's tables before the arrivals
       if (lane == 0) {
         desc[kDS] = s;
         desc[kDKvh] = kvh;
         desc[kDPart] = part;
-        desc[kDBegin] = t_begin;
+        desc[kDBegin] = p0;
         desc[kDEnd] = t_end;
         desc[kDTiles] = n_tiles;
-        desc[kDParts] = GROUP ? direct_mask : (ctx_or_members + PT - 1) / PT;
-        desc[kDCtx] = ctx_or_members;
+        desc[kDMembers] = members;
+        desc[kDVbase] = vbase;
         mbar_arrive(meta_bar(slot));
-        const uint32_t rb = ready_bar(slot);
-        if constexpr (GROUP) {
-          mbar_arrive(rb);
-        } else {
-          mbar_arrive_expect_tx(rb, 2 * kHeads * G * 128);
-          const int qrow = (a.seq_offset + s) * a.num_q_heads + kvh * G;
-          tma_load_2d(sm_q + slot * L::kQBytes, &tm_q, rb, 0, qrow);
-          tma_load_2d(sm_q + slot * L::kQBytes + N * 128, &tm_q, rb, 64, qrow);
-        }
+        mbar_arrive(rb);  // with the query rows' bytes, completes the ready phase
       }
       int nf = 0;
       if (lane == 0) {
-        const int t = take_item(a.work_counter, a.epoch, a.err);
+        const int t = take_end(a.work_counter, ticket, a.epoch, a.err);
         nf = t < 0 ? total : (int)gridDim.x + t;
       }
       f = __shfl_sync(0xffffffffu, nf, 0);
@@ -582,7 +695,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     // (bounded waits).  Items it-2 and it-1 may still be in flight, unless the
     // end-of-work mark went into item it-2's slot: that needed the slot freed,
     // so its rows had landed, and its phase parity now names a later phase.
-    if (!GROUP && lane == 0)
+    if (lane == 0)
       for (int k = max(0, it - (ok ? 1 : kSlots)); k < it; ++k)
         mbar_wait(ready_bar(k % kSlots), (k / kSlots) & 1, a.err);
   } else if (warp == kProducerWarp) {
@@ -603,28 +716,44 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         }
         __syncwarp();  // lane 0's acquire orders the other lanes' reads below
       }
-      const int* desc = desc_all + slot * 8;
+      const int* desc = desc_all + slot * 16;
       const int n_tiles = desc[kDTiles];
       if (n_tiles < 0) break;  // end of work
       const int kvh = desc[kDKvh];
       const int n_groups = (desc[kDEnd] - desc[kDBegin] + kGroupRows - 1) / kGroupRows;
       const int my_row = rows_all[slot * 64 + lane];
-      const int my_row2 = a.half_boxes ? rows_all[slot * 64 + 32 + lane] : 0;
+      const int my_row2 = rows_all[slot * 64 + 32 + lane];
       for (int j = 0; j < n_tiles && ok; ++j) {
-        const int st = issued % NST;
-        if (issued >= NST &&
-            !mbar_wait_or_abort(empty_bar(st), ((issued / NST) - 1) & 1, a.err, abort_flag)) {
+        const int st = issued % kStages;
+        if (issued >= kStages &&
+            !mbar_wait_or_abort(empty_bar(st), ((issued / kStages) - 1) & 1, a.err, abort_flag)) {
           ok = false;
           break;
         }
-        const int g0 = j * (kTok / kGroupRows);
-        const int ng = min(kTok / kGroupRows, n_groups - g0);
+        const int g0 = j * kGroupsPerTile;
+        const int ng = min(kGroupsPerTile, n_groups - g0);
         const uint32_t fb = full_bar(st);
         const uint32_t dst = sm_stages + st * L::kStageBytes;
         constexpr int kBoxBytes = kHeads * kGroupRows * 128;  // one box: a group of kHeads heads
-        if (lane == 0) mbar_arrive_expect_tx(fb, ng * 4 * kBoxBytes);
+        if (lane == 0) mbar_arrive_expect_tx(fb, ng * (KV8 ? 2 : 4) * kBoxBytes);
         __syncwarp();
-        {
+        if constexpr (KV8) {
+          // lane 2 r + k loads K (k = 0) or V (k = 1) of group r: 128 one-byte
+          // elements x 16 rows (x 2 heads), the whole head_dim in one box
+          const int r = lane >> 1, k = lane & 1;
+          const int row = __shfl_sync(0xffffffffu, my_row, min(g0 + r, 31));
+          const int row2 = __shfl_sync(0xffffffffu, my_row2, min(g0 + r, 31));
+          if (r < ng) {
+            const uint32_t d = dst + k * L::kHalf + r * kBoxBytes;
+            const void* map = k == 0 ? &tm_k : &tm_v;
+            if constexpr (PAIR) {
+              tma_load_3d(d, map, fb, 0, row, kvh);
+            } else {
+              tma_load_3d(d, map, fb, 0, kvh, row);
+              if (a.half_boxes) tma_load_3d(d + (kGroupRows / 2) * 128, map, fb, 0, kvh, row2);
+            }
+          }
+        } else {
           // lane 4 r + k loads piece k (K or V, 64-element half) of group r
           const int r = lane >> 2, k = lane & 3;
           const int row = __shfl_sync(0xffffffffu, my_row, min(g0 + r, 31));
@@ -648,8 +777,8 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     if (!ok) *abort_flag = 1;
     // Every TMA copy armed by this warp lands before the CTA leaves.
     if (lane == 0)
-      for (int k = max(0, issued - NST); k < issued; ++k)
-        mbar_wait(full_bar(k % NST), (k / NST) & 1, a.err);
+      for (int k = max(0, issued - kStages); k < issued; ++k)
+        mbar_wait(full_bar(k % kStages), (k / kStages) & 1, a.err);
   } else if (warp == kMmaWarp) {
     // =====================================================================
     // MMA warp (lane 0): every tcgen05.mma of the CTA, so that issuing them
@@ -663,7 +792,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     int g = 0;  // tiles issued so far
     auto issue_qk = [&](int st, uint32_t q_addr) {
       tc_fence_after();
-      const uint32_t kt = sm_stages + st * L::kStageBytes;
+      const uint32_t kt = KV8 ? smem_addr(smem + L::kK16) : sm_stages + st * L::kStageBytes;
 #pragma unroll
       for (int kk = 0; kk < kD / 16; ++kk) {
         const uint32_t ko = (kk / 4) * L::kHalf + (kk % 4) * 32;
@@ -678,19 +807,21 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         const int slot = it % kSlots;
         ok = mbar_wait_or_abort(ready_bar(slot), (it / kSlots) & 1, a.err, abort_flag);
         if (!ok) break;
-        const int n_tiles = desc_all[slot * 8 + kDTiles];
+        const int n_tiles = desc_all[slot * 16 + kDTiles];
         if (n_tiles < 0) break;  // end of work
         const uint32_t q_addr = sm_q + slot * L::kQBytes;
-        // S^T(h) needs its stage landed and S^T(h-1) read by the compute warps
+        // S^T(h) needs its stage landed (with an 8-bit cache: widened) and
+        // S^T(h-1) read by the compute warps
         auto qk_for = [&](int h) {
-          bool w = mbar_wait_or_abort(full_bar(h % NST), (h / NST) & 1, a.err, abort_flag);
+          bool w = KV8 ? mbar_wait_or_abort(conv_bar, h & 1, a.err, abort_flag)
+                       : mbar_wait_or_abort(full_bar(h % kStages), (h / kStages) & 1, a.err, abort_flag);
           if (w && h > 0) w = mbar_wait_or_abort(s_free_bar, (h - 1) & 1, a.err, abort_flag);
-          if (w) issue_qk(h % NST, q_addr);
+          if (w) issue_qk(h % kStages, q_addr);
           return w;
         };
         if (n_tiles > 0) ok = qk_for(g);
         for (int j = 0; j < n_tiles && ok; ++j, ++g) {
-          const int st = g % NST;
+          const int st = g % kStages;
           // S^T(g+1) as soon as S^T(g) has been read: it runs during tile g's
           // softmax; then, once P(g) is written, O^T(g)
           if (j + 1 < n_tiles) {
@@ -700,7 +831,8 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           ok = mbar_wait_or_abort(p_ready_bar, g & 1, a.err, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t vt = sm_stages + st * L::kStageBytes + 2 * L::kHalf;
+          const uint32_t vt = KV8 ? smem_addr(smem + L::kV16) + (g & 1) * 2 * L::kHalf
+                                  : sm_stages + st * L::kStageBytes + 2 * L::kHalf;
           const uint32_t acc0 = (uint32_t)acc_flag[g & 1];
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
@@ -708,7 +840,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                     smem_desc(sm_p + kk * 512, L::kPAtom, 256, kSw32), kIdescPV,
                     acc0 | (uint32_t)(kk > 0));
           mma_commit(pv_bar);
-          mma_commit(empty_bar(st));  // the stage is free once these MMAs are done
+          if constexpr (!KV8) mma_commit(empty_bar(st));  // the stage is free once these MMAs are done
         }
       }
       if (!ok) *abort_flag = 1;
@@ -719,7 +851,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     __syncwarp();
   } else {
     // =====================================================================
-    // compute warps: thread (t, cg) = token row t of S^T and row d = t of O^T,
+    // compute warps: thread (t, cg) = MMA row t of S^T and row d = t of O^T,
     // for the columns of warpgroup cg.  Per tile g: wait for S^T(g), read it
     // and release it (s_free) so the MMA warp can issue S^T(g+1); the softmax
     // writes P(g) after O^T(g-1), its last reader, completed; then p_ready.
@@ -729,18 +861,25 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     // the next PV overwrites instead of accumulating).  Hence p <= 2^kRescale.
     // =====================================================================
     constexpr float kRescale = 8.f;
-    const int t = tid & 127;         // token row of S^T, output row of O^T
+    const int t = tid & 127;         // MMA row of S^T, output row of O^T
     const int cg = tid >> 7;         // column group
     const int c0 = cg * NCW;         // first column of this thread
     const int quarter = warp & 3;    // TMEM lane quarter of this warp
     const uint32_t t_lane = ((uint32_t)(quarter * 32) << 16);
-    // MMA row t: kv head e_row of the item, token tok_row of the tile; with
-    // two heads only the columns of head e_row are this row's logits
+    // MMA row t: kv head e_row of the item, 16-row group t / 16 of the tile
+    // (with two heads: token group t / 32)
     const int e_row = PAIR ? (t >> 4) & 1 : 0;
-    const int tok_row = PAIR ? ((t >> 5) << 4) + (t & 15) : t;
-    bool col_ok[NCW];
+    const int grp_in_tile = PAIR ? (t >> 5) : (t >> 4);
+    // column c: member m_c (query token, or group member), kv head e_c of the
+    // item, query head h_c of that kv head
+    int m_c[NCW], e_c[NCW], h_c[NCW];
 #pragma unroll
-    for (int c = 0; c < NCW; ++c) col_ok[c] = !PAIR || (c0 + c) / G == e_row;
+    for (int c = 0; c < NCW; ++c) {
+      const int col = c0 + c;
+      m_c[c] = col / (kHeads * G);
+      e_c[c] = (col / G) % kHeads;
+      h_c[c] = col % G;
+    }
     int g = 0;  // tiles consumed, numbered across items
     bool ok = true;
     // one lane per warp waits on an mbarrier, the warp follows
@@ -749,17 +888,72 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       if (lane == 0) w = mbar_wait_or_abort(bar, parity, a.err, abort_flag);
       return __shfl_sync(0xffffffffu, (int)w, 0) != 0;
     };
+    // KV8: widen the 8-bit tile gt (tile jt of the item whose group table is
+    // gmeta_s) into the 16-bit K buffer and V buffer gt & 1.  Thread t takes
+    // row t, warpgroup cg the 16-byte pieces cg, cg + NWG, ... (both layouts
+    // 128B-swizzled: piece c of row t at c ^ (t & 7), so a warp's accesses
+    // spread over every bank); a row that is no token gets a zero V row.
+    // Then the stage goes back to the producer and the MMA warp may issue
+    // S^T(gt).  K's buffer is free (S^T(gt - 1) has been read) and so is V's
+    // (O^T(gt - 2) has completed): the callers make sure.
+    auto widen = [&](int gt, int jt, const int* gmeta_s) {
+      const int st = gt % kStages;
+      const bool w = warp_wait(full_bar(st), (gt / kStages) & 1);
+      if (w) {
+        const bool rok = (t & 15) < (gmeta_s[jt * kGroupsPerTile + grp_in_tile] >> 8);
+        const unsigned char* kin = smem + L::kStages0 + st * L::kStageBytes + t * 128;
+        const unsigned char* vin = kin + L::kHalf;
+        unsigned char* kout = smem + L::kK16 + t * 128;
+        unsigned char* vout = smem + L::kV16 + (gt & 1) * 2 * L::kHalf + t * 128;
+        const int sw = t & 7;
+#pragma unroll
+        for (int i = 0; i < 8 / W::kNWG; ++i) {
+          const int jc = cg + i * W::kNWG;  // elements 16 jc .. 16 jc + 15 of the row
+          const uint4 kx = *reinterpret_cast<const uint4*>(kin + ((jc ^ sw) << 4));
+          const uint4 vx = *reinterpret_cast<const uint4*>(vin + ((jc ^ sw) << 4));
+          uint32_t kw[8], vw[8];
+          widen16<T>(kx, kw);
+          widen16<T>(vx, vw);
+          if (!rok) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) vw[e] = 0u;
+          }
+          const int h = jc >> 2, c = 2 * (jc & 3);  // half, first 16-byte piece of it
+          unsigned char* ko = kout + h * L::kHalf;
+          unsigned char* vo = vout + h * L::kHalf;
+          *reinterpret_cast<uint4*>(ko + ((c ^ sw) << 4)) = make_uint4(kw[0], kw[1], kw[2], kw[3]);
+          *reinterpret_cast<uint4*>(ko + (((c + 1) ^ sw) << 4)) = make_uint4(kw[4], kw[5], kw[6], kw[7]);
+          *reinterpret_cast<uint4*>(vo + ((c ^ sw) << 4)) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
+          *reinterpret_cast<uint4*>(vo + (((c + 1) ^ sw) << 4)) = make_uint4(vw[4], vw[5], vw[6], vw[7]);
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(empty_bar(st));
+        mbar_arrive(conv_bar);
+      }
+      return w;
+    };
     for (int it = 0; ok; ++it) {
       const int slot = it % kSlots;
       if (tid == 0) ok = mbar_wait_or_abort(ready_bar(slot), (it / kSlots) & 1, a.err, abort_flag);
       if (named_barrier_or(1, kComputeThreads, !ok || *abort_flag)) { ok = false; break; }
-      const int* desc = desc_all + slot * 8;
+      const int* desc = desc_all + slot * 16;
       const int n_tiles = desc[kDTiles];
       if (n_tiles < 0) break;  // end of work
-      const int s = desc[kDS], kvh = desc[kDKvh], part = desc[kDPart];
-      const int t_begin = desc[kDBegin], t_end = desc[kDEnd], n_parts = desc[kDParts];
-      const int ctx_or_members = desc[kDCtx];
-      const int cols = GROUP ? ctx_or_members * G : kHeads * G;
+      const int kvh = desc[kDKvh], vbase = desc[kDVbase];
+      const int* gtok = gtok_all + slot * 32;
+      const int* gmeta = gmeta_all + slot * 32;
+      // token limit of each column's member (-1: a column no member fills)
+      int lim_c[NCW];
+#pragma unroll
+      for (int c = 0; c < NCW; ++c) lim_c[c] = mlim_all[slot * 32 + min(m_c[c], 31)];
+      // logits in log2 units; an 8-bit cache folds each kv head's K scale in
+      float kfac[NCW];
+#pragma unroll
+      for (int c = 0; c < NCW; ++c)
+        kfac[c] = KV8 ? a.scale_log2 * __ldg(a.k_scale + min(kvh + e_c[c], Hkv - 1)) : a.scale_log2;
 
       float acc[NCW], l_tok[NCW], m_ref[NCW];
 #pragma unroll
@@ -768,8 +962,21 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       bool ok_w = true;     // every wait of this warp so far succeeded
 
       for (int j = 0; j < n_tiles; ++j, ++g) {
-        const int st = g % NST;
-        const int n_valid = min(kTok, t_end - (t_begin + j * kTok));
+        const int st = g % kStages;
+        // this row's group: owner (-1: every member), first token, valid rows
+        const int grp = j * kGroupsPerTile + grp_in_tile;
+        const int gm = gmeta[grp];
+        const int own = (gm & 0xff) - 1;
+        const int tok = gtok[grp] + (t & 15);
+        const bool row_ok = (t & 15) < (gm >> 8);
+        bool valid[NCW];
+#pragma unroll
+        for (int c = 0; c < NCW; ++c)
+          valid[c] = row_ok && (own < 0 || own == m_c[c]) && (!PAIR || e_c[c] == e_row) &&
+                     tok < lim_c[c];
+        if constexpr (KV8) {
+          if (j == 0 && ok_w) ok_w = widen(g, 0, gmeta);  // an item's first tile
+        }
         // ---- S^T(g).  Each warp waits on its own; the OR-barrier then makes
         // every compute thread take the same way out if this or an earlier
         // wait of its warp failed.
@@ -787,12 +994,19 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         // waited for only where this tile needs it: before O^T is folded and
         // before P(g) is written
         bool pv_done = j == 0;
-        const bool valid = tok_row < n_valid;
+        if constexpr (KV8) {
+          // the next tile of the item is widened now, so that S^T(g+1) runs
+          // during this tile's softmax; its V buffer was O^T(g-1)'s
+          if (j + 1 < n_tiles) {
+            if (!pv_done && ok_w) ok_w = warp_wait(pv_bar, (g - 1) & 1), pv_done = true;
+            if (ok_w) ok_w = widen(g + 1, j + 1, gmeta);
+          }
+        }
         bool over = false;
 #pragma unroll
         for (int c = 0; c < NCW; ++c) {
-          sv[c] = valid && col_ok[c] ? sv[c] * a.scale_log2 : -INFINITY;
-          over |= (c0 + c < cols) && (sv[c] > m_ref[c] + kRescale);
+          sv[c] = valid[c] ? sv[c] * kfac[c] : -INFINITY;
+          over |= sv[c] > m_ref[c] + kRescale;
         }
         const bool rescale = named_barrier_or(1, kComputeThreads, over);
         if (rescale) {
@@ -812,7 +1026,8 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
           for (int c = 0; c < NCW; ++c) {
             const float m_new = fmaxf(m_ref[c], stat[c0 + c]);
-            alpha[c] = exp2f(m_ref[c] - m_new);  // 0 while m_ref is -inf
+            // 0 while m_ref is -inf; 1 while the column has seen no valid row
+            alpha[c] = m_new == -INFINITY ? 1.f : exp2f(m_ref[c] - m_new);
             m_ref[c] = m_new;
             l_tok[c] *= alpha[c];
           }
@@ -834,10 +1049,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         float p[NCW];
 #pragma unroll
         for (int c = 0; c < NCW; ++c) {
-          p[c] = valid && col_ok[c] ? exp2f(sv[c] - m_ref[c]) : 0.f;
+          p[c] = valid[c] ? exp2f(sv[c] - m_ref[c]) : 0.f;
           l_tok[c] += p[c];
         }
-        // P^T rows: per 16-column atom, a 32-byte row per token (MN-major,
+        // P^T rows: per 16-column atom, a 32-byte row per MMA row (MN-major,
         // 32-byte swizzle: 16-byte piece c of row t sits at c ^ bit 2 of t),
         // once for hi = round(p) and once for lo = round(p - hi).  This
         // thread writes columns [c0, c0 + NCW): NCW * 2 bytes inside one
@@ -873,10 +1088,11 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
             *reinterpret_cast<uint16_t*>(prow + L::kPBytes) = (uint16_t)lo[0];
           }
         }
-        if (!valid) {
-          // zero this token's V row (both 64-element halves, 16 pieces shared
-          // out over the column groups) so 0 * stale never enters PV
-          unsigned char* vrow = smem + L::kStages + st * L::kStageBytes + 2 * L::kHalf + t * 128;
+        if (!KV8 && !row_ok) {
+          // this row is no token: zero its V row (both 64-element halves, 16
+          // pieces shared out over the column groups) so 0 * stale never
+          // enters PV
+          unsigned char* vrow = smem + L::kStages0 + st * L::kStageBytes + 2 * L::kHalf + t * 128;
 #pragma unroll
           for (int i = cg; i < 16; i += W::kNWG)
             *reinterpret_cast<uint4*>(vrow + (i >> 3) * L::kHalf + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
@@ -890,7 +1106,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       }
       if (!ok) break;
 
-      // ---- item result: fold the last O^T, reduce the per-token sums, write
+      // ---- item result: fold the last O^T, reduce the per-row sums, write
       if (tid == 0 && n_tiles > 0) ok = mbar_wait_or_abort(pv_bar, (g - 1) & 1, a.err, abort_flag);
       if (named_barrier_or(1, kComputeThreads, !ok || !ok_w || *abort_flag)) { ok = false; break; }
       if (n_tiles > 0) {
@@ -915,28 +1131,22 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       const int d = t;  // output element this thread writes, per column
 #pragma unroll
       for (int c = 0; c < NCW; ++c) {
-        const int col = c0 + c;
-        if (col >= cols) break;
-        const float L_c = stat[N + col];
-        const int m = GROUP ? col / G : 0, h = GROUP ? col % G : col;
-        const size_t qh = (size_t)(s + m) * a.num_q_heads + (size_t)kvh * G + h;
-        bool zero = false, direct;
-        if constexpr (GROUP) {
-          direct = (n_parts >> m) & 1;  // from the producer: this partition is the member's result
-        } else {
-          zero = ctx_or_members == 0;
-          direct = n_parts <= 1;
-        }
-        if (zero) {
+        if (m_c[c] >= desc[kDMembers]) continue;  // a padded column
+        const int code = mcode_all[slot * 32 + m_c[c]];
+        if (code == kSkip) continue;
+        const size_t qh = (size_t)(vbase + m_c[c]) * a.num_q_heads + (size_t)(kvh + e_c[c]) * G + h_c[c];
+        // an 8-bit cache applies its V scale here (the merge is linear in it)
+        const float o = KV8 ? acc[c] * __ldg(a.v_scale + kvh + e_c[c]) : acc[c];
+        if (code == kZero) {
           a.out[qh * kD + d] = 0;
-        } else if (direct) {
-          a.out[qh * kD + d] = Elem<T>::from_f(acc[c] / L_c);
+        } else if (code == kDirect) {
+          a.out[qh * kD + d] = Elem<T>::from_f(o / stat[N + c0 + c]);
         } else {
-          const size_t wslot = qh * a.num_parts + part;
-          a.ws_acc[wslot * kD + d] = acc[c];
+          const size_t wslot = qh * a.num_parts + code;
+          a.ws_acc[wslot * kD + d] = o;
           if (d == 0) {
             a.ws_ml[2 * wslot] = m_ref[c];
-            a.ws_ml[2 * wslot + 1] = L_c;
+            a.ws_ml[2 * wslot + 1] = stat[N + c0 + c];
           }
         }
       }
@@ -950,15 +1160,13 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   if (warp == 0) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(C::kTmemCols)
+                 "r"(kTmemCols)
                  : "memory");
   }
 }
 
 // ---------------------------------------------------------------------------
 // host side
-
-constexpr int kStagesTc = 3;
 
 int sm_count() {
   static int count[64] = {};
@@ -968,12 +1176,11 @@ int sm_count() {
   return count[dev];
 }
 
-template <typename T, int G, bool GROUP, bool PAIR>
+template <typename T, int NC, bool PAIR, bool KV8>
 cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& tq, cudaStream_t stream, int* launches) {
-  using C = Cfg<GROUP>;
-  using L = Layout<kStagesTc, C::kN>;
-  auto* kern = decode_tc_kernel<T, G, kStagesTc, GROUP, PAIR>;
+  using L = Layout<(NC <= 16 ? 16 : 32), KV8>;
+  auto* kern = decode_tc_kernel<T, NC, PAIR, KV8>;
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
@@ -981,25 +1188,32 @@ cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUte
     configured = true;
   }
   const int sms = sm_count();
-  constexpr int kChunk = C::kMaxSeqs;
-  for (int s0 = 0; s0 < a0.num_seqs; s0 += kChunk) {
+  const bool grouped = a0.plan != nullptr;
+  // groups never cross a multiple of the shared-prefix window
+  const int chunk = grouped ? kSharedPrefixSeqsPerLaunch : kMaxUnits;
+  const int Tq = a0.query_tokens;
+  for (int s0 = 0; s0 < a0.num_seqs; s0 += chunk) {
     DecodeArgs a = a0;
-    a.num_seqs = a0.num_seqs - s0 < kChunk ? a0.num_seqs - s0 : kChunk;
+    a.num_seqs = a0.num_seqs - s0 < chunk ? a0.num_seqs - s0 : chunk;
     a.seq_offset = s0;
-    a.out = a0.out + (size_t)s0 * a0.num_q_heads * kD;
+    const size_t rows0 = (size_t)s0 * Tq * a0.num_q_heads;  // first output row of the launch
+    a.out = a0.out + rows0 * kD;
     a.block_tables = a0.block_tables + (size_t)s0 * a0.max_blocks_per_seq;
     a.context_lens = a0.context_lens + s0;
-    if (a0.plan) a.plan = a0.plan + s0;
-    if (a0.ws_acc) {
-      a.ws_acc = a0.ws_acc + (size_t)s0 * a0.num_q_heads * a0.num_parts * kD;
-      a.ws_ml = a0.ws_ml + (size_t)s0 * a0.num_q_heads * a0.num_parts * 2;
+    if (grouped) {
+      a.plan = a0.plan + s0;
+      a.plan2 = a0.plan2 + s0;
     }
-    a.epoch = a0.epoch + (unsigned long long)(s0 / kChunk);
-    // plain: at least one item per (sequence, kv head); shared-prefix: the
+    if (a0.ws_acc) {
+      a.ws_acc = a0.ws_acc + rows0 * a0.num_parts * kD;
+      a.ws_ml = a0.ws_ml + rows0 * a0.num_parts * 2;
+    }
+    a.epoch = a0.epoch + (unsigned long long)(s0 / chunk);
+    // at least one item per (unit, kv unit) without a plan; with one, the
     // number of items is only known on the device
-    const int items0 = GROUP ? sms : a.num_seqs * (a.num_kv_heads / (PAIR ? 2 : 1));
+    const int items0 = grouped ? sms : a.num_seqs * (a.num_kv_heads / (PAIR ? 2 : 1));
     const int grid = items0 < sms ? items0 : sms;
-    constexpr int kBlock = Warps<columns<G, GROUP, PAIR>()>::kThreads;
+    constexpr int kBlock = Warps<NC>::kThreads;
     cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kBlock), L::kAlloc, stream, a, tk, tv, tq);
     if (e != cudaSuccess) return e;
     ++*launches;
@@ -1007,39 +1221,52 @@ cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUte
   return cudaSuccess;
 }
 
-template <typename T, bool GROUP, bool PAIR>
-cudaError_t launch_group(const DecodeArgs& a, int G, const CUtensorMap& tk, const CUtensorMap& tv,
-                         const CUtensorMap& tq, cudaStream_t st, int* n) {
-  switch (G) {
-    case 1: return launch_typed<T, 1, GROUP, PAIR>(a, tk, tv, tq, st, n);
-    case 2: return launch_typed<T, 2, GROUP, PAIR>(a, tk, tv, tq, st, n);
-    case 4: return launch_typed<T, 4, GROUP, PAIR>(a, tk, tv, tq, st, n);
-    case 8: return launch_typed<T, 8, GROUP, PAIR>(a, tk, tv, tq, st, n);
-    case 16:
-      if constexpr (!PAIR) return launch_typed<T, 16, GROUP, false>(a, tk, tv, tq, st, n);
+template <typename T, bool PAIR, bool KV8>
+cudaError_t launch_cols(const DecodeArgs& a, int nc, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const CUtensorMap& tq, cudaStream_t st, int* n) {
+  switch (nc) {
+    case 1:
+      if constexpr (!PAIR) return launch_typed<T, 1, false, KV8>(a, tk, tv, tq, st, n);
+      break;
+    case 2: return launch_typed<T, 2, PAIR, KV8>(a, tk, tv, tq, st, n);
+    case 4: return launch_typed<T, 4, PAIR, KV8>(a, tk, tv, tq, st, n);
+    case 8: return launch_typed<T, 8, PAIR, KV8>(a, tk, tv, tq, st, n);
+    case 16: return launch_typed<T, 16, PAIR, KV8>(a, tk, tv, tq, st, n);
+    case 32:  // two-head items take at most 16 columns
+      if constexpr (!PAIR) return launch_typed<T, 32, false, KV8>(a, tk, tv, tq, st, n);
+      break;
   }
   return cudaErrorInvalidValue;
 }
 
-}  // namespace tc
-
-cudaError_t launch_decode_tc(const DecodeArgs& a, int dtype, int group, const CUtensorMap& tk,
-                             const CUtensorMap& tv, const CUtensorMap& tq, cudaStream_t stream,
-                             int* launches, bool pair) {
-  if (a.num_seqs <= 0) return cudaSuccess;
-  if (pair) {
-    if (dtype == 0) return tc::launch_group<__half, false, true>(a, group, tk, tv, tq, stream, launches);
-    return tc::launch_group<__nv_bfloat16, false, true>(a, group, tk, tv, tq, stream, launches);
-  }
-  if (dtype == 0) return tc::launch_group<__half, false, false>(a, group, tk, tv, tq, stream, launches);
-  return tc::launch_group<__nv_bfloat16, false, false>(a, group, tk, tv, tq, stream, launches);
+template <typename T, bool KV8>
+cudaError_t launch_kind(const DecodeArgs& a, int nc, bool pair, const CUtensorMap& tk,
+                        const CUtensorMap& tv, const CUtensorMap& tq, cudaStream_t st, int* n) {
+  return pair ? launch_cols<T, true, KV8>(a, nc, tk, tv, tq, st, n)
+              : launch_cols<T, false, KV8>(a, nc, tk, tv, tq, st, n);
 }
 
-cudaError_t launch_decode_shared_tc(const DecodeArgs& a, int dtype, int group, const CUtensorMap& tk,
-                                    const CUtensorMap& tv, cudaStream_t stream, int* launches) {
-  if (a.num_seqs <= 0 || !a.plan) return cudaSuccess;
-  if (dtype == 0) return tc::launch_group<__half, true, false>(a, group, tk, tv, tk, stream, launches);
-  return tc::launch_group<__nv_bfloat16, true, false>(a, group, tk, tv, tk, stream, launches);
+}  // namespace tc
+
+TcQueryBox tc_query_box(int group, int query_tokens, bool pair, bool grouped) {
+  if (grouped) return {group, kTcMaxColumns / group};
+  return {(pair ? 2 : 1) * group, query_tokens};
+}
+
+cudaError_t launch_decode_tc(const DecodeArgs& a, int dtype, const CUtensorMap& tk,
+                             const CUtensorMap& tv, const CUtensorMap& tq, cudaStream_t stream,
+                             int* launches, bool pair, bool fp8_cache) {
+  if (a.num_seqs <= 0) return cudaSuccess;
+  const int cols = tc::tc_columns(a.group, a.query_tokens, pair, a.plan != nullptr);
+  if (cols < 1 || cols > kTcMaxColumns) return cudaErrorInvalidValue;
+  int nc = 1;
+  while (nc < cols) nc *= 2;
+  if (fp8_cache) {
+    if (dtype == 0) return tc::launch_kind<__half, true>(a, nc, pair, tk, tv, tq, stream, launches);
+    return tc::launch_kind<__nv_bfloat16, true>(a, nc, pair, tk, tv, tq, stream, launches);
+  }
+  if (dtype == 0) return tc::launch_kind<__half, false>(a, nc, pair, tk, tv, tq, stream, launches);
+  return tc::launch_kind<__nv_bfloat16, false>(a, nc, pair, tk, tv, tq, stream, launches);
 }
 
 int decode_tc_tile_tokens() { return tc::kTile; }

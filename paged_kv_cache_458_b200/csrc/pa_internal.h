@@ -30,9 +30,16 @@ struct DecodeArgs {
   const float* k_scale;          // [Hkv] with an E4M3 cache (stored value = code * scale)
   const float* v_scale;          // [Hkv]
   const int4* plan;
-  int own_tokens;                // partition size of a sequence's own tokens (partition_tokens
-                                 // without a plan)
+  // With a plan, per sequence {row offset of its own tokens in its group's
+  // row list, number of partials it gets (1: written directly), partitions
+  // of the group's row list, rows in that list}.
+  const int4* plan2;
+  int own_tokens;                // partition size of the CUDA-core kernel
   int grid_parts;                // partitions per (sequence, kv head) of the CUDA-core grid
+  int query_tokens;              // query tokens per sequence (pa_decode_multi on the
+                                 // tensor-core kernels; 1 otherwise): q, out and the
+                                 // split-K rows are [num_seqs * query_tokens][Hq]
+  int group;                     // g = Hq / Hkv
   int half_boxes;                // block_size is a multiple of 8 but not of 16: each
                                  // 16-token TMA box is loaded as two 8-token boxes, which
                                  // may come from two blocks
@@ -47,6 +54,7 @@ struct PlanArgs {
   const int32_t* block_tables;   // [S][MBS]
   const int32_t* context_lens;   // [S]
   int4* plan;                    // [S] out
+  int4* plan2;                   // [S] out
   int num_seqs, max_blocks_per_seq, block_size, num_blocks, max_context_len;
   int partition_tokens;
   int max_members;               // members per group (32 / g)
@@ -60,26 +68,6 @@ cudaError_t launch_expand_queries(const int32_t* tables, const int32_t* ctx, int
                                   int max_context_len, int32_t* tables_out, int32_t* ctx_out,
                                   unsigned int* err, cudaStream_t stream, int* launches);
 
-// Tokens [T, ctx) of sequence s with a plan: its first own token, the
-// workspace slot of its first own partition (of own_tokens tokens each), and
-// the sequence's partition count.
-struct SeqSplit {
-  int base, slot0, total;
-};
-__host__ __device__ inline SeqSplit seq_split(const int4* plan, int s, int ctx, int own_tokens) {
-  int base = 0, slot0 = 0;
-  if (plan) {
-#ifdef __CUDA_ARCH__
-    const int4 pl = __ldg(plan + s);
-#else
-    const int4 pl = plan[s];
-#endif
-    base = pl.z;
-    slot0 = pl.w;
-  }
-  const int own = ctx > base ? (ctx - base + own_tokens - 1) / own_tokens : 0;
-  return {base, slot0, slot0 + own};
-}
 
 // Launch the partition kernel (+ the merge kernel when num_parts > 1).
 // `launches` is incremented once per kernel launched.  fp8_cache: K/V hold
@@ -93,18 +81,29 @@ int decode_max_partition_tokens();
 cudaError_t launch_decode_merge(const DecodeArgs& a, int dtype, int head_dim, cudaStream_t stream,
                                 int* launches);
 
-// The tensor-core path (head_dim 128): maps are 128B-swizzled, boxes of 64
-// elements; tq views q as [S * Hq][128] with boxes of (64 x group) elements.
-// With `pair`, items cover two kv heads: the pool maps are [Hkv][rows][128] by
-// strides with boxes of 64 x 16 rows x 2 heads, and q boxes hold 2 x group rows.
-cudaError_t launch_decode_tc(const DecodeArgs& a, int dtype, int group, const CUtensorMap& tm_k,
+// The tensor-core path (head_dim 128): pool maps are 128B-swizzled, boxes of
+// 64 elements x 16 (or 8) token rows of one kv head; with `pair`, items cover
+// two kv heads and the pool maps are [Hkv][rows][128] by strides with boxes
+// of 64 x 16 rows x 2 heads.  tm_q views q as [rows][Hq][128] (rows =
+// num_seqs * query_tokens) with 128B-swizzled boxes of 64 elements x
+// heads_per_box x rows_per_box; see tc_query_box().
+// Without a plan, items are (sequence, kv head or pair, partition) with the
+// sequence's query_tokens x heads query rows as columns; with a plan
+// (a.plan, a.plan2), items are (group leader, kv head, partition of the
+// group's row list) with members x g columns.
+// fp8_cache: the pools hold E4M3 codes (8-bit maps with boxes of 128
+// one-byte elements; a.k_scale / a.v_scale set).
+cudaError_t launch_decode_tc(const DecodeArgs& a, int dtype, const CUtensorMap& tm_k,
                              const CUtensorMap& tm_v, const CUtensorMap& tm_q, cudaStream_t stream,
-                             int* launches, bool pair);
+                             int* launches, bool pair, bool fp8_cache);
 int decode_tc_tile_tokens();
-// The shared-prefix kernel (a.plan set): items over the shared partitions of
-// every group, members x g query rows per tile.
-cudaError_t launch_decode_shared_tc(const DecodeArgs& a, int dtype, int group, const CUtensorMap& tm_k,
-                                    const CUtensorMap& tm_v, cudaStream_t stream, int* launches);
+// Query columns one tensor-core item holds at most.
+constexpr int kTcMaxColumns = 32;
+// The q box of the tensor-core kernel for a launch: {heads, rows} per box.
+struct TcQueryBox {
+  int heads, rows;
+};
+TcQueryBox tc_query_box(int group, int query_tokens, bool pair, bool grouped);
 
 cudaError_t launch_cache_append(const void* k, const void* v, const int32_t* slot_mapping,
                                 int num_tokens, void* k_cache, void* v_cache, long long num_slots,

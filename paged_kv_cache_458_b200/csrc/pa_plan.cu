@@ -23,8 +23,14 @@
 //
 // plan[s] = {rank of s in its group (0 = the leader), members, T, shared
 // partitions ceil(T / partition_tokens)}; a sequence alone gets {0, 1, 0, 0}.
-// Tokens [0, T) of every member are then computed by the group's items, and
-// [T, ctx) by the member's own items, as further split-K partitions.
+//
+// The decode then reads each group through one row list: the T shared tokens,
+// followed by each member's own tokens [T, ctx) in member order, each member's
+// run rounded up to 16 rows so that a 16-row box never mixes members.  A
+// sequence alone is a group of one with T = 0.  plan2[s] = {offset of s's own
+// rows in its group's list, number of partials s gets (the partitions of the
+// list holding its shared or own rows; 1: its result is written directly, 0:
+// empty context), partitions of the list (at least 1), rows in the list}.
 #include <cuda_runtime.h>
 
 #include <climits>
@@ -56,9 +62,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p) {
   pdl_wait();  // the tables and lengths of this step are written
   pdl_launch_dependents();
   __shared__ int sh_edge, sh_min_ctx, sh_min_blocks, sh_common;
+  __shared__ int sh_rows[32];  // own rows of each member, rounded up to 16
   const int s = blockIdx.x, tid = threadIdx.x;
   const int first = first_block(p, s);
-  int4 out = make_int4(0, 1, 0, 0);
+  int leader = s, n = 1, shared = 0;
   if (first >= 0) {
     const int c0 = (s / p.chunk) * p.chunk;
     const int c1 = min(p.num_seqs, c0 + p.chunk);
@@ -86,42 +93,63 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p) {
       __syncthreads();
       if (e != INT_MAX) { b = e; break; }
     }
-    const int leader = a + ((s - a) / p.max_members) * p.max_members;
-    const int n = min(p.max_members, b - leader);
-    if (n >= 2) {
+    const int lead = a + ((s - a) / p.max_members) * p.max_members;
+    const int nm = min(p.max_members, b - lead);
+    if (nm >= 2) {
       // ---- shortest member context and block count
       if (tid == 0) sh_min_ctx = INT_MAX, sh_min_blocks = INT_MAX;
       __syncthreads();
-      if (tid < n) {
-        const int c = clamp_ctx(p, leader + tid);
+      if (tid < nm) {
+        const int c = clamp_ctx(p, lead + tid);
         atomicMin(&sh_min_ctx, c);
         atomicMin(&sh_min_blocks, (c + p.block_size - 1) / p.block_size);
       }
       __syncthreads();
       if (tid == 0) sh_common = sh_min_blocks;
       __syncthreads();
-      // ---- leading table entries every member has in common with the leader
-      const int32_t* lead = p.block_tables + (size_t)leader * p.max_blocks_per_seq;
-      for (int m = 1; m < n; ++m) {
-        const int32_t* row = p.block_tables + (size_t)(leader + m) * p.max_blocks_per_seq;
-        for (int j0 = 0;; j0 += kPlanThreads) {
-          const int lim = sh_common;  // the same in every thread: read between barriers
-          __syncthreads();
-          if (j0 >= lim) break;
-          const int j = j0 + tid;
-          if (j < lim && __ldg(row + j) != __ldg(lead + j)) atomicMin(&sh_common, j);
-          __syncthreads();
-        }
+      // ---- leading table entries every member has in common with the leader:
+      // each round compares J entries of every other member at once
+      const int32_t* lead_row = p.block_tables + (size_t)lead * p.max_blocks_per_seq;
+      const int J = max(1, kPlanThreads / (nm - 1));
+      const int m = 1 + tid / J;
+      const int32_t* row = p.block_tables + (size_t)(lead + min(m, nm - 1)) * p.max_blocks_per_seq;
+      for (int j0 = 0;; j0 += J) {
+        const int lim = sh_common;  // the same in every thread: read between barriers
+        __syncthreads();
+        if (j0 >= lim) break;
+        const int j = j0 + tid % J;
+        if (m < nm && j < lim && __ldg(row + j) != __ldg(lead_row + j)) atomicMin(&sh_common, j);
+        __syncthreads();
       }
       const long long t = min((long long)sh_common * p.block_size, (long long)sh_min_ctx);
-      const int shared = (int)(t & ~15LL);
-      if (shared >= p.min_shared) {
-        out = make_int4(s - leader, n, shared,
-                        (shared + p.partition_tokens - 1) / p.partition_tokens);
-      }
+      const int sh = (int)(t & ~15LL);
+      if (sh >= p.min_shared) leader = lead, n = nm, shared = sh;
     }
   }
-  if (tid == 0) p.plan[s] = out;
+  // ---- this sequence's place in its group's row list
+  if (tid < n) {
+    const int own = clamp_ctx(p, leader + tid) - shared;
+    sh_rows[tid] = (own + 15) / 16 * 16;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    const int PT = p.partition_tokens;
+    int off = shared, my_off = 0;
+    for (int m = 0; m < n; ++m) {
+      if (leader + m == s) my_off = off;
+      off += sh_rows[m];
+    }
+    const int rows = off;
+    const int p_shared = (shared + PT - 1) / PT;
+    const int own = clamp_ctx(p, s) - shared;
+    int n_slots = p_shared;
+    if (own > 0) {
+      const int first_p = max(my_off / PT, p_shared), last_p = (my_off + own - 1) / PT;
+      if (last_p >= first_p) n_slots += last_p - first_p + 1;
+    }
+    p.plan[s] = n >= 2 ? make_int4(s - leader, n, shared, p_shared) : make_int4(0, 1, 0, 0);
+    p.plan2[s] = make_int4(my_off, n_slots, max(1, (rows + PT - 1) / PT), rows);
+  }
 }
 
 }  // namespace

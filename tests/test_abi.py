@@ -97,14 +97,20 @@ def test_fp8_cache_validation(lib):
     assert lib.pa_decode_fp8(FAKE, FAKE, FAKE, FAKE + 2, FAKE, FAKE, FAKE, 0.1, FAKE,
                              ctypes.byref(s8), 100, FAKE, 1 << 20, None) == pa.PA_ERR_INVALID_ARG
     for bad, st in ((dict(cache_format=2), pa.PA_ERR_UNSUPPORTED),
-                    (dict(cache_format=pa.PA_CACHE_FP8_E4M3, variant=2), pa.PA_ERR_UNSUPPORTED),
-                    (dict(cache_format=pa.PA_CACHE_FP8_E4M3, shared_prefix=1),
+                    (dict(cache_format=pa.PA_CACHE_FP8_E4M3, variant=2, head_dim=64),
+                     pa.PA_ERR_UNSUPPORTED),
+                    (dict(cache_format=pa.PA_CACHE_FP8_E4M3, shared_prefix=1, variant=1),
                      pa.PA_ERR_UNSUPPORTED)):
         s = _shape(**bad)
         assert lib.pa_decode_fp8(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.1, FAKE,
                                  ctypes.byref(s), 100, FAKE, 1 << 20, None) == st
+    # an E4M3 cache takes the tensor-core kernels by the same rule as a 16-bit one
     assert pa.pa_decode_resolved_variant(_shape(cache_format=1, num_q_heads=16)) == \
+        pa.PA_DECODE_TENSOR_CORES
+    assert pa.pa_decode_resolved_variant(_shape(cache_format=1, num_q_heads=4)) == \
         pa.PA_DECODE_CUDA_CORES
+    assert pa.pa_decode_resolved_variant(_shape(cache_format=1, shared_prefix=1)) == \
+        pa.PA_DECODE_RESOLVED_SHARED_PREFIX
     # appends
     assert lib.pa_cache_append(FAKE, FAKE, FAKE, 3, FAKE, FAKE, ctypes.byref(s8), None) == \
         pa.PA_ERR_INVALID_ARG
@@ -114,10 +120,10 @@ def test_fp8_cache_validation(lib):
                                    None) == pa.PA_ERR_INVALID_ARG
     assert lib.pa_cache_append_fp8(FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, ctypes.byref(s8),
                                    None) == pa.PA_OK
-    # the workspace depends on the cache format only through the default
-    # partition (an E4M3 pool always takes the CUDA-core kernel)
-    assert lib.pa_decode_workspace_bytes(ctypes.byref(s8), 1000) == \
-        lib.pa_decode_workspace_bytes(ctypes.byref(_shape(variant=1)), 1000)
+    # the workspace does not depend on the cache format
+    for kw in (dict(), dict(variant=1), dict(num_q_heads=4), dict(shared_prefix=1)):
+        assert lib.pa_decode_workspace_bytes(ctypes.byref(_shape(cache_format=1, **kw)), 1000) == \
+            lib.pa_decode_workspace_bytes(ctypes.byref(_shape(**kw)), 1000)
 
 
 def test_multi_query_workspace_and_validation(lib):

@@ -56,18 +56,28 @@ def _quantised_case(orc, rng, dtype, Hq, Hkv, D, bs, ctx):
     c = gen.random_decode_case(rng, num_seqs=len(ctx), num_q_heads=Hq, num_kv_heads=Hkv,
                                head_dim=D, block_size=bs, dtype=dtype, context_lens=ctx,
                                poison=False)
-    NB = c["num_blocks"]
+    return _quantise(orc, rng, c, dtype)
+
+
+def _quantise(orc, rng, c, dtype):
+    """The case with both pools encoded to E4M3 by the oracle (per-head scales)."""
+    NB, bs, Hkv, D = c["k_cache"].shape
     ks, vs = _scales(rng, Hkv)
     kc = np.zeros((NB, bs, Hkv, D), dtype=np.uint8)
     vc = np.zeros_like(kc)
     slots = np.arange(NB * bs, dtype=np.int32)
     orc.cache_append_fp8(dtype, c["k_cache"].reshape(NB * bs, Hkv, D),
                          c["v_cache"].reshape(NB * bs, Hkv, D), slots, ks, vs, kc, vc)
+    # slots no sequence holds get the E4M3 NaN code: a read past a context shows
+    valid = gen.valid_slot_mask(c["block_tables"], c["context_lens"], NB, bs)
+    kc.reshape(NB * bs, -1)[~valid] = 0x7F
+    vc.reshape(NB * bs, -1)[~valid] = 0x7F
     return dict(c, k_cache=kc, v_cache=vc, k_scale=ks, v_scale=vs)
 
 
-def _gpu_decode_fp8(c, dtype, Hq, partition_tokens=0):
-    shape = _shape(c, dtype, Hq, partition_tokens)
+def _gpu_decode_fp8(c, dtype, Hq, partition_tokens=0, variant=0, shared_prefix=0):
+    shape = _shape(c, dtype, Hq, partition_tokens, variant)
+    shape.shared_prefix = shared_prefix
     maxlen = int(np.max(c["context_lens"], initial=0))
     wsb = pa.pa_decode_workspace_bytes(shape, maxlen)
     ws = torch.empty(max(16, wsb), dtype=torch.uint8, device="cuda")
@@ -168,6 +178,43 @@ def test_fp8_decode_partitions_and_blocks(orc, partition_tokens, block_size):
     ref = orc.decode_fp8(gen.BF16, c["q"], c["k_cache"], c["v_cache"], c["k_scale"], c["v_scale"],
                          c["block_tables"], c["context_lens"], c["scale"])
     assert_decode_close(out, ref, gen.BF16, f"fp8 bs{block_size} pt{partition_tokens}")
+
+
+@pytest.mark.parametrize("dtype", [gen.F16, gen.BF16], ids=["f16", "bf16"])
+@pytest.mark.parametrize("group", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("block_size", [8, 16])
+@pytest.mark.parametrize("variant", [1, 2], ids=["cuda_cores", "tensor_cores"])
+def test_fp8_decode_variants(orc, dtype, group, block_size, variant):
+    """Both kernels on an E4M3 cache: the tensor-core one widens each tile to
+    16 bits in shared memory (one head per item, or two)."""
+    rng = np.random.default_rng(1200 + 11 * group + block_size + 3 * variant + dtype)
+    for Hkv in (2, 3):
+        c = _quantised_case(orc, rng, dtype, Hkv * group, Hkv, 128, block_size, EDGE_CTX)
+        for pt in (0, 128):
+            out = _gpu_decode_fp8(c, dtype, Hkv * group, pt, variant)
+            ref = orc.decode_fp8(dtype, c["q"], c["k_cache"], c["v_cache"], c["k_scale"],
+                                 c["v_scale"], c["block_tables"], c["context_lens"], c["scale"])
+            assert_decode_close(out, ref, dtype,
+                                f"fp8 v{variant} g{group} bs{block_size} Hkv{Hkv} pt{pt}")
+            assert np.all(out[0] == 0)
+
+
+@pytest.mark.parametrize("dtype", [gen.F16, gen.BF16], ids=["f16", "bf16"])
+@pytest.mark.parametrize("group", [1, 4, 8])
+def test_fp8_shared_prefix(orc, dtype, group):
+    """Shared prefixes on an E4M3 cache: groups read once, own tokens after."""
+    rng = np.random.default_rng(1300 + group + dtype)
+    mm = 32 // group
+    groups = [(700, [700 + int(x) for x in rng.integers(1, 40, size=mm + 2)]),
+              (256, [256, 261]), (100, [110, 120]), (0, [0]), (1000, [1030, 500]),
+              (300, [310, 305, 301, 300][:max(2, min(4, mm))]), (0, [37])]
+    c = gen.grouped_decode_case(rng, groups=groups, num_q_heads=2 * group, num_kv_heads=2,
+                                head_dim=128, block_size=16, dtype=dtype, poison=False)
+    c = _quantise(orc, rng, c, dtype)
+    out = _gpu_decode_fp8(c, dtype, 2 * group, shared_prefix=1)
+    ref = orc.decode_fp8(dtype, c["q"], c["k_cache"], c["v_cache"], c["k_scale"], c["v_scale"],
+                         c["block_tables"], c["context_lens"], c["scale"])
+    assert_decode_close(out, ref, dtype, f"fp8 shared g{group}")
 
 
 def test_fp8_step_append_copy_decode(orc):

@@ -28,9 +28,8 @@ def _cuda():
     torch.cuda.empty_cache()
 
 
-def _case(seed, Tq, ctx, group, head_dim, dtype, block_size=16, shared_prefix_blocks=0):
+def _case(seed, Tq, ctx, group, head_dim, dtype, block_size=16, shared_prefix_blocks=0, Hkv=2):
     rng = np.random.default_rng(seed)
-    Hkv = 2
     c = gen.random_decode_case(rng, num_seqs=len(ctx), num_q_heads=Hkv * group, num_kv_heads=Hkv,
                                head_dim=head_dim, block_size=block_size, dtype=dtype,
                                context_lens=ctx, shared_prefix_blocks=shared_prefix_blocks)
@@ -126,9 +125,32 @@ def test_multi_verification_step(orc):
     pa.pa_decode_multi(dev(q, gen.BF16), kc, vc, dev_i32(bt), dev_i32(ctx), c["scale"], out, shape,
                        Tq, maxlen, ws, wsb)
     assert pa.pa_last_device_error()[0] == pa.PA_OK
-    # expand + plan + shared-prefix kernel + CUDA-core kernel + merge
-    assert pa.pa_kernel_launches() - n0 == 5
+    # Tq x g = 16 columns: one tensor-core kernel reads every K/V tile once
+    # for all four queries (contexts under 512 tokens: no merge)
+    assert pa.pa_kernel_launches() - n0 == 1
     hk, hv = c["k_cache"].copy(), c["v_cache"].copy()
     orc.cache_append(k_new, v_new, slots, hk, hv)
     ref = orc.decode_multi(gen.BF16, q, hk, hv, bt, ctx, c["scale"])
     assert_decode_close(host_bits(out), ref, gen.BF16, "verification step")
+
+
+@pytest.mark.parametrize("Tq,group,Hkv,block_size", [
+    (3, 2, 3, 16),    # odd kv heads: one head per item, 6 of 8 columns
+    (4, 1, 2, 8),     # 8-token blocks: one head per item, two 8-row boxes per group
+    (5, 4, 2, 16),    # 20 of 32 columns
+    (2, 16, 2, 16),   # 32 columns of one head
+    (8, 1, 4, 16),    # two heads per item, 16 columns
+    (7, 2, 2, 256),   # two heads per item, 14 of 16 columns, 256-token blocks
+])
+def test_multi_one_read_for_all_queries(orc, Tq, group, Hkv, block_size):
+    """The tensor-core path that reads each tile once for all Tq queries, with
+    the causal limit of every query falling inside, at and across partition
+    and tile boundaries."""
+    ctx = [1, Tq - 1 if Tq > 1 else 1, Tq, 63 + Tq, 64 + Tq, 127 + Tq, 512, 513, 515, 1030, 1540]
+    c = _case(1600 + 13 * Tq + group + Hkv + block_size, Tq, ctx, group, 128, gen.BF16,
+              block_size=block_size, Hkv=Hkv)
+    for pt in (0, 128):
+        out = _gpu_multi(c, gen.BF16, Tq, partition_tokens=pt)
+        ref = orc.decode_multi(gen.BF16, c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
+                               c["context_lens"], c["scale"])
+        assert_decode_close(out, ref, gen.BF16, f"Tq{Tq} g{group} Hkv{Hkv} bs{block_size} pt{pt}")

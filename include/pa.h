@@ -62,6 +62,7 @@ typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
 #define PA_DEVERR_SLOT 0x4u         /* append slot >= num_blocks * block_size */
 #define PA_DEVERR_PAIR 0x8u         /* copy pair names a block outside [0, num_blocks) */
 #define PA_DEVERR_WAIT_TIMEOUT 0x10u
+#define PA_DEVERR_CONFIG 0x20u      /* a kernel found less shared memory than it laid out; it did nothing */
 
 /*
  * Shape of one paged KV cache and of the batch that reads it.
@@ -122,7 +123,8 @@ typedef enum { PA_CACHE_AS_DTYPE = 0, PA_CACHE_FP8_E4M3 = 1 } pa_cache_format;
  *                          g = Hq / Hkv is at least 8 (at least 4 when
  *                          block_size is a multiple of 16) and
  *                          partition_tokens is a multiple of 128 up to 512;
- *                          CUDA cores otherwise.
+ *                          CUDA cores otherwise.  The same rule holds for an
+ *                          E4M3 cache (pa_decode_fp8).
  *  PA_DECODE_CUDA_CORES    fp32 FMA on the CUDA cores (any built shape).
  *  PA_DECODE_TENSOR_CORES  tcgen05 MMA with the g heads padded to 16: fp16/bf16
  *                          operands (the probabilities enter the PV product as
@@ -139,20 +141,21 @@ int pa_decode_partition_tokens(const pa_shape *shape);
 
 /* The kernel pa_decode() runs for `shape`: PA_DECODE_CUDA_CORES or
  * PA_DECODE_TENSOR_CORES (PA_DECODE_AUTO resolved), or
- * PA_DECODE_RESOLVED_SHARED_PREFIX with shape->shared_prefix (tensor cores for
- * the shared tokens, CUDA cores for the rest), or minus the status pa_decode()
- * would refuse the shape with.  Host only; launches nothing. */
+ * PA_DECODE_RESOLVED_SHARED_PREFIX with shape->shared_prefix (a plan kernel,
+ * then the tensor-core kernel over every group's row list), or minus the
+ * status pa_decode() would refuse the shape with.  Host only; launches
+ * nothing. */
 #define PA_DECODE_RESOLVED_SHARED_PREFIX 3
 int pa_decode_resolved_variant(const pa_shape *shape);
 
 /* Bytes of device workspace pa_decode() needs for `shape` when no context is
  * longer than `max_context_len` tokens: 256 bytes for the work counter the
  * tensor-core variant's persistent CTAs take items from; with shared_prefix,
- * 16 bytes per sequence (rounded up to 256) for the group plan; plus, when a
- * context spans more than one partition (always with shared_prefix), per
- * (sequence, query head, partition) the running max, the softmax sum and the
- * unnormalised output row in fp32, for ceil(max_context_len /
- * partition_tokens) partitions, one more with shared_prefix.  The
+ * two records of 16 bytes per sequence (each rounded up to 256) for the group
+ * plan; plus, when a context spans more than one partition (always with
+ * shared_prefix), per (sequence, query head, partition) the running max, the
+ * softmax sum and the unnormalised output row in fp32, for ceil(max_context_len
+ * / partition_tokens) partitions, two more with shared_prefix.  The
  * workspace needs no initialisation (the counter carries a per-call tag, so a
  * value left by an earlier call is recognised and replaced) and is dead after
  * the call's kernels finish.  Returns 0 for an invalid shape. */
@@ -186,12 +189,15 @@ size_t pa_decode_workspace_bytes(const pa_shape *shape, int32_t max_context_len)
  * into groups of at most 32 / g members; a group shares its first T tokens,
  * where T counts the leading table entries equal in all members (below each
  * member's own block count), capped at the shortest member context and
- * rounded down to a multiple of 16; groups with T < 128 are dropped.  A
- * tensor-core kernel computes every group's shared tokens for all members x g
- * query rows at once, the CUDA-core kernel each sequence's remaining tokens,
- * and the merge kernel combines the two (log-sum-exp rule).  The result is the
- * same attention, up to fp32 rounding order; only the order in which the sums
- * are formed differs.
+ * rounded down to a multiple of 16; groups with T < 128 are dropped (their
+ * members, and every sequence in no group, are groups of one with T = 0).
+ * Each group is then read as one row list: its T shared tokens, followed by
+ * each member's own tokens [T, ctx) rounded up to 16 rows; the tensor-core
+ * kernel reads each partition of that list once, for all members x g query
+ * rows (a member's columns see the shared rows and its own), and the merge
+ * kernel combines a member's partitions (log-sum-exp rule).  The result is
+ * the same attention, up to fp32 rounding order; only the order in which the
+ * sums are formed differs.
  *
  * q, k_cache, v_cache, block_tables, context_lens, out: device, layouts above.
  * max_context_len: host-side upper bound on every context_lens[s]; it sizes the
@@ -221,15 +227,17 @@ pa_status pa_decode(const void *q, const void *k_cache, const void *v_cache,
  * token t attends causally to tokens 0 .. ctx_s - Tq + t.  A query whose
  * range is empty (ctx_s < Tq - t) gives a zero row.
  *
- * Query t of s is a one-token decode of a virtual sequence with the same
- * block table and context ctx_s - Tq + t + 1.  A first kernel writes the
- * virtual tables and contexts into the workspace.  The virtual sequences of
- * one sequence are consecutive and start with the same blocks, so when the
- * shape allows the shared-prefix kernel (head_dim 128, variant
- * PA_DECODE_AUTO, a 16-bit cache, partition_tokens 0 or a multiple of 128
- * up to 512) and Tq * g >= 8, the tokens they have in common are read once
- * for all of them.  Otherwise each is decoded on its own (the common tokens
- * then come mostly from L2).  Tq == 1 is pa_decode.
+ * Where the shape allows the tensor-core kernel (head_dim 128, a 16-bit
+ * cache, variant not PA_DECODE_CUDA_CORES, partition_tokens 0 (then 512) or
+ * a multiple of 128 up to 512) and Tq * g <= 32, the Tq x g query rows of a
+ * sequence are the columns of one item per (sequence, kv head, partition),
+ * each masked at its own causal limit: every K/V tile is read once for all
+ * Tq queries.  Otherwise query t of s is decoded as a one-token virtual
+ * sequence with the same block table and context ctx_s - Tq + t + 1: a first
+ * kernel writes the virtual tables and contexts into the workspace, and the
+ * virtual sequences of one sequence, which start with the same blocks, are
+ * grouped as shared prefixes when the shape allows it (variant
+ * PA_DECODE_AUTO).  Tq == 1 is pa_decode.
  * workspace: pa_decode_multi_workspace_bytes(shape, Tq, max_context_len).
  */
 size_t pa_decode_multi_workspace_bytes(const pa_shape *shape, int32_t num_query_tokens,
@@ -312,11 +320,13 @@ pa_status pa_cache_append_fp8(const void *k, const void *v, const int32_t *slot_
 /*
  * Decode attention over an E4M3 cache (shape->cache_format ==
  * PA_CACHE_FP8_E4M3, else PA_ERR_INVALID_ARG): pa_decode's result with
- * K_j = code * k_scale[h / g] and V_j = code * v_scale[h / g].  Runs the
- * CUDA-core kernel (variant PA_DECODE_TENSOR_CORES or shared_prefix give
- * PA_ERR_UNSUPPORTED); the K scale is folded into the query and the V scale
- * into the output.  Same workspace as pa_decode.  k_scale, v_scale: device
- * fp32 [num_kv_heads].
+ * K_j = code * k_scale[h / g] and V_j = code * v_scale[h / g].  The variant
+ * and shared_prefix work as in pa_decode.  The CUDA-core kernel widens each
+ * lane's codes as it reads them; the tensor-core kernels land the 8-bit tiles
+ * by TMA and widen them exactly to 16 bits in shared memory before the
+ * products.  The K scale is folded into the logits and the V scale into the
+ * output.  Same workspace as pa_decode.  k_scale, v_scale: device fp32
+ * [num_kv_heads].
  */
 pa_status pa_decode_fp8(const void *q, const void *k_cache, const void *v_cache,
                         const float *k_scale, const float *v_scale,

@@ -8,11 +8,13 @@ can move the result by one more half unit.  Where one ulp of the output type
 exceeds 2e-3 (bf16 at |o| >= 0.5, fp16 at |o| >= 4) the per-element bound is
 one ulp of that type at the exact value instead.  The number of elements that used that branch is reported.
 
-The mean bound likewise counts only what the kernel adds to the rounding of
-the output: mean |err| <= 2e-4 + mean |round(ref) - ref|, where round(ref)
-is the exact result rounded to the output type.  Rounding alone averages a
-quarter ulp, 4.9e-4 for bf16 outputs in [0.25, 0.5), so without this term no
-implementation could meet the bound on short contexts.
+The mean bound is mean |err| <= max(2e-4, mean |round(ref) - ref| + 5e-5),
+where round(ref) is the exact result rounded to the output type.  Rounding
+alone averages a quarter ulp, 4.9e-4 for bf16 outputs in [0.25, 0.5), so a
+plain 2e-4 could not be met by any implementation on short contexts; above
+that floor a kernel may add at most 5e-5.  (Measured over every parity case
+of the GPU suite, the kernels' mean error exceeds the rounding floor by at
+most 1.1e-9: they round as well as a correctly rounded result.)
 """
 import json
 import os
@@ -27,6 +29,7 @@ _LOG = os.environ.get("PA_TOLERANCE_LOG")
 
 MAX_ABS = 2e-3
 MEAN_ABS = 2e-4
+MEAN_OVER_FLOOR = 5e-5  # what a kernel may add to the output's own rounding, on average
 _MANTISSA = {gen.F16: 10, gen.BF16: 7}
 _MIN_EXP = {gen.F16: -14, gen.BF16: -126}
 
@@ -75,6 +78,6 @@ def assert_decode_close(out_bits, ref, dtype, what=""):
     _log(st, dtype, what)
     assert st["n_nan"] == 0, f"{what}: {st['n_nan']} NaN outputs"
     assert st["n_over"] == 0, f"{what}: {st['n_over']} elements above the bound (max {st['max_abs']:.3e})"
-    assert st["mean_abs"] <= MEAN_ABS + st["mean_floor"], \
+    assert st["mean_abs"] <= max(MEAN_ABS, st["mean_floor"] + MEAN_OVER_FLOOR), \
         f"{what}: mean abs error {st['mean_abs']:.3e} (rounding alone {st['mean_floor']:.3e})"
     return st

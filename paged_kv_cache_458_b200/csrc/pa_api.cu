@@ -366,15 +366,19 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
     // items of two kv heads (4 KB boxes) where the heads pair up, their query
     // columns fit 16 and blocks give 16-row boxes; shared-prefix groups keep
     // one head per item
-    const bool pair = !shape->shared_prefix && shape->num_kv_heads % 2 == 0 && !a.half_boxes &&
-                      2 * group * query_tokens <= 16;
+    const bool pair = shape->num_kv_heads % 2 == 0 && !a.half_boxes && 2 * group * query_tokens <= 16;
     CUtensorMap tk, tv, tq;
-    if (!make_tc_maps(&tk, &tv, &tq, k_cache, v_cache, q, shape, pair, query_tokens,
-                      shape->shared_prefix != 0))
+    if (!make_tc_maps(&tk, &tv, &tq, k_cache, v_cache, q, shape, pair, query_tokens, false))
       return cuda_failed("cuTensorMapEncodeTiled failed");
     e = cudaSuccess;
     if (shape->shared_prefix) {
-      // plan the groups, then every group's row list on tensor cores
+      // plan the groups; then every group's row list (shared tokens, and the
+      // members' own tokens where they are few) on the tensor-core kernel
+      // with members x g columns; then, per sequence, the own tokens that are
+      // in no list
+      CUtensorMap gk, gv, gq;
+      if (!make_tc_maps(&gk, &gv, &gq, k_cache, v_cache, q, shape, false, 1, true))
+        return cuda_failed("cuTensorMapEncodeTiled failed");
       pa::PlanArgs pl{};
       pl.block_tables = block_tables;
       pl.context_lens = context_lens;
@@ -391,9 +395,13 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
       pl.chunk = pa::kSharedPrefixSeqsPerLaunch;
       a.plan = plan;
       a.plan2 = plan2;
-      a.epoch = next_epochs((shape->num_seqs + pa::kSharedPrefixSeqsPerLaunch - 1) /
-                            pa::kSharedPrefixSeqsPerLaunch);
+      const int chunks = (shape->num_seqs + pa::kSharedPrefixSeqsPerLaunch - 1) /
+                         pa::kSharedPrefixSeqsPerLaunch;
+      a.epoch = next_epochs(chunks);
       e = pa::launch_plan(pl, cs, &launched);
+      if (e == cudaSuccess) e = pa::launch_decode_tc(a, shape->dtype, gk, gv, gq, cs, &launched, false, fp8);
+      a.own_pass = 1;
+      a.epoch = next_epochs((shape->num_seqs + 511) / 512);
     } else {
       a.epoch = next_epochs((shape->num_seqs + 511) / 512);
     }

@@ -63,8 +63,11 @@
 // 128B-swizzled), into one of three stages; a dedicated MMA warp issues every
 // MMA and commits it to an mbarrier; the compute warps consume tiles in order
 // and tell it through two more mbarriers when S^T(g) has been read and when
-// P(g) has been written.  Items are numbered full partitions first and the
-// shorter last partitions after them, so the CTAs finish close together.
+// P(g) has been written.  Per-sequence items are numbered partition 0 of every
+// sequence first, then each sequence's further partitions (measured 2 % faster
+// on mistral_7b_gqa than full partitions first and the shorter last ones
+// after them); a group's items, full partitions first and the shorter last
+// ones after them.
 // Rows that are no token of any column are masked in P and their V rows are
 // zeroed in shared memory before the PV product, so stale or NaN rows never
 // reach the result.
@@ -121,8 +124,9 @@ struct Warps {
 template <int N, bool KV8>
 struct Layout {
   // small region (byte offsets from the dynamic base)
-  // barriers: full[3], empty[3], ready[2], free[2], meta[2], qk, pv, drain, s_free, p_ready, conv
-  static constexpr int kNumBars = 2 * kStages + 3 * kSlots + 6;
+  // barriers: full[3], empty[3], ready[2], free[2], meta[2], qk, pv, drain, s_free, p_ready,
+  // conv, qconv
+  static constexpr int kNumBars = 2 * kStages + 3 * kSlots + 7;
   static constexpr int kBars = 0;
   static constexpr int kMisc = kBars + kNumBars * 8;        // tmem address, abort flag, accumulate flags [2]
   static constexpr int kDesc = kMisc + 16;                  // [slots][16] int
@@ -133,7 +137,8 @@ struct Layout {
   static constexpr int kMCode = kMLim + kSlots * 32 * 4;    // [slots][32] int: destination of each member
   static constexpr int kRed = kMCode + kSlots * 32 * 4;     // [4 warps][N] f32
   static constexpr int kStat = kRed + 4 * N * 4;            // m[N], then l[N], f32
-  static constexpr int kSmall = kStat + 2 * N * 4;
+  static constexpr int kQScale = kStat + 2 * N * 4;        // KV8: [slots][32] f32, query row scales
+  static constexpr int kSmall = kQScale + kSlots * 32 * 4;
   // big region (byte offsets from the first 1024-byte boundary after the small one)
   static constexpr int kHalf = kTile * 128;  // a 64-element half of a 16-bit tile, or an 8-bit tile (16 KB)
   static constexpr int kStageBytes = KV8 ? 2 * kHalf : 4 * kHalf;  // K tile then V tile
@@ -241,6 +246,26 @@ __device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[NCOL]) {
   for (int i = 0; i < NCOL; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Zero NCOL (1 .. 8) consecutive fp32 columns of this thread's TMEM lane.
+template <int NCOL>
+__device__ __forceinline__ void tmem_zero(uint32_t taddr) {
+  const uint32_t z = 0u;
+  if constexpr (NCOL == 1) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(z) : "memory");
+  } else if constexpr (NCOL == 2) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %1};" ::"r"(taddr), "r"(z) : "memory");
+  } else if constexpr (NCOL == 4) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %1, %1, %1};" ::"r"(taddr), "r"(z)
+                 : "memory");
+  } else {
+    static_assert(NCOL == 8, "1, 2, 4 or 8 columns");
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(
+                     taddr),
+                 "r"(z)
+                 : "memory");
+  }
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int c0, int c1) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
@@ -305,13 +330,14 @@ __device__ __forceinline__ int last_at_most(const int (&pre)[PPL], int r) {
   return __reduce_add_sync(0xffffffffu, cnt) - 1;
 }
 
-// Item number -> (unit, kv unit, partition).  A unit (a sequence, or a group
-// leader) whose row list holds R rows has R / PT full partitions and, when PT
-// does not divide R (or R == 0), one last shorter one.  Items 0 .. Hu F - 1
-// are the full partitions of every unit (F in all), the rest the last ones;
-// the kv unit varies fastest.  pre_f / pre_p: exclusive prefix counts of full
-// / last partitions over the units, lane l holding entries l, l + 32, ...
-// Called by all 32 lanes.
+// Item number -> (unit, kv unit, partition).  A unit whose row list holds R
+// rows has R / PT full partitions and, when PT does not divide R (or R == 0),
+// one last shorter one.  Items 0 .. Hu F - 1 are the full partitions of every
+// unit (F in all), the rest the last ones; the kv unit varies fastest.
+// pre_f / pre_p: exclusive prefix counts of full / last partitions over the
+// units, lane l holding entries l, l + 32, ...  (Per-sequence items number
+// partition 0 of every sequence first and locate the rest with pre_f
+// counting further partitions and pre_p zero.)  Called by all 32 lanes.
 template <int PPL>
 __device__ __forceinline__ void locate(int f, int Hu, int F, const int (&pre_f)[PPL],
                                        const int (&pre_p)[PPL], int& u, int& kvu, int& part) {
@@ -394,10 +420,16 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                 kSchedWarp = kComputeWarps + 2;
   using L = Layout<N, KV8>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
-  constexpr uint32_t kIdescQK = instr_desc(kBf16 ? 1 : 0, 0, 0, kTile, N);
+  // An 8-bit cache is widened to f16 (one conversion per pair) and the
+  // products run in f16 whatever the query type: bf16 query rows are
+  // converted to f16 at the start of each item (kQToF16).
+  constexpr bool kQToF16 = KV8 && kBf16;
+  using MT = typename std::conditional<KV8, __half, T>::type;  // operand type of the products
+  constexpr bool kMmaBf16 = std::is_same<MT, __nv_bfloat16>::value;
+  constexpr uint32_t kIdescQK = instr_desc(kMmaBf16 ? 1 : 0, 0, 0, kTile, N);
   // PV has 2N columns: P hi and P lo sit in consecutive 16-column atoms, so one
   // MMA reads each V slice once for both and writes O^T hi and O^T lo side by side
-  constexpr uint32_t kIdescPV = instr_desc(kBf16 ? 1 : 0, 1, 1, kTile, 2 * N);
+  constexpr uint32_t kIdescPV = instr_desc(kMmaBf16 ? 1 : 0, 1, 1, kTile, 2 * N);
   extern __shared__ __align__(16) unsigned char smem_raw[];
 
   // Until pdl_wait() below, this CTA touches only its own shared and tensor
@@ -420,7 +452,9 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   }
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int Hkv = a.num_kv_heads, PT = a.partition_tokens, G = a.group, Tq = a.query_tokens;
-  const bool grouped = a.plan != nullptr;
+  // row lists of shared-prefix groups; else per-sequence items (with a plan:
+  // the own tokens of the sequences whose own tokens are in no list)
+  const bool grouped = a.plan != nullptr && !a.own_pass;
   int* desc_all = reinterpret_cast<int*>(smem_raw + L::kDesc);
   int* rows_all = reinterpret_cast<int*>(smem_raw + L::kRows);
   int* gtok_all = reinterpret_cast<int*>(smem_raw + L::kGTok);
@@ -444,6 +478,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   const uint32_t s_free_bar = qk_bar + 24;   // compute warps have read S^T(g)
   const uint32_t p_ready_bar = qk_bar + 32;  // compute warps have written P(g)
   const uint32_t conv_bar = qk_bar + 40;     // KV8: compute warps have widened tile g
+  const uint32_t qconv_bar = qk_bar + 48;    // the item's query rows are f16 (kQToF16)
   const uint32_t sm_stages = smem_addr(smem + L::kStages0);
   const uint32_t sm_q = smem_addr(smem + L::kQ);
   const uint32_t sm_p = smem_addr(smem + L::kP);
@@ -475,6 +510,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     mbar_init(s_free_bar, kComputeWarps);
     mbar_init(p_ready_bar, kComputeWarps);
     mbar_init(conv_bar, kComputeWarps);
+    mbar_init(qconv_bar, W::kNWG);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -513,7 +549,8 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       if (s < S) {
         int rows = -1;  // rows of the unit's list; -1: not a unit
         if (grouped) {
-          if (__ldg(a.plan + s).x == 0) rows = __ldg(a.plan2 + s).w;
+          const int4 pl = __ldg(a.plan + s);
+          if (pl.x == 0 && pl.y >= 2) rows = __ldg(a.plan2 + s).w;
         } else {
           int ctx = __ldg(a.context_lens + s);
           if (ctx < 0 || ctx > a.max_context_len) {
@@ -521,10 +558,21 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
             ctx = max(0, min(ctx, a.max_context_len));
           }
           rows = ctx;
+          if (a.plan) {
+            // own tokens read on their own: a sequence in no group (even an
+            // empty one, whose item writes zeros), or a member with own tokens
+            const int4 pl = __ldg(a.plan + s);
+            const bool alone = __ldg(a.plan2 + s).x < 0 && (pl.y == 1 || ctx > pl.z);
+            rows = alone ? ctx - pl.z : -1;
+          }
         }
         if (rows >= 0) {
           full = rows / PT;
           last = (rows % PT != 0 || rows == 0) ? 1 : 0;
+          if (!grouped) {
+            full = full + last - 1;  // further partitions after partition 0
+            last = 0;
+          }
         }
       }
       int inc_f = full, inc_p = last;
@@ -540,7 +588,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       carry_p += __shfl_sync(0xffffffffu, inc_p, 31);
     }
     const int Hu = Hkv / kHeads;  // kv units of the item numbering
-    const int total = Hu * (carry_f + carry_p);
+    const int total = Hu * (carry_f + carry_p) + (grouped ? 0 : S * Hu);
 
     bool ok = true;
     int it = 0;
@@ -568,7 +616,17 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       unsigned long long ticket = 0;
       if (lane == 0) ticket = take_begin(a.work_counter);
       int s, kvu, part;
-      locate(f, Hu, carry_f, pre_f, pre_p, s, kvu, part);
+      if (!grouped) {
+        // partition 0 of every sequence, then further partitions by sequence
+        if (f < S * Hu) {
+          s = f / Hu, kvu = f % Hu, part = 0;
+        } else {
+          locate(f - S * Hu, Hu, carry_f, pre_f, pre_p, s, kvu, part);
+          part += 1;
+        }
+      } else {
+        locate(f, Hu, carry_f, pre_f, pre_p, s, kvu, part);
+      }
       const int kvh = kvu * kHeads;  // the item's first kv head
       // query rows: one TMA box per 64-element half, [members][heads][64]
       const uint32_t rb = ready_bar(slot);
@@ -581,6 +639,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       // ---- members (lane m): token limit, destination of the result; the
       // row list of the item
       int members, T, n_list, vbase;  // shared rows, rows in the unit's list
+      int tok_base = 0;               // token of the list's first row (own-token pass)
       int m_ctx = 0, m_off = 0, m_code = kSkip;
       const int p0 = part * PT;
       if (grouped) {
@@ -600,7 +659,8 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         if (lane < members) {
           const int own = m_ctx - T;
           const int first_own = max(m_off / PT, p_sh);
-          const bool mine = part < p_sh || (own > 0 && part >= m_off / PT && part <= (m_off + own - 1) / PT);
+          const bool mine = part < p_sh || (m_off >= 0 && own > 0 && part >= m_off / PT &&
+                                            part <= (m_off + own - 1) / PT);
           if (m_ctx == 0) m_code = part == 0 ? kZero : kSkip;
           else if (!mine) m_code = kSkip;
           else if (m_slots == 1) m_code = kDirect;
@@ -610,12 +670,22 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         const int ctx = max(0, min(__ldg(a.context_lens + s), a.max_context_len));
         members = Tq;
         T = ctx;  // every row is every query's, up to its limit
-        n_list = ctx;
         vbase = s * Tq;
+        // with a plan, the own tokens [base, ctx) after the partials of the
+        // sequence's shared tokens
+        int slot0 = 0, n_slots = 0;
+        if (a.plan) {
+          const int4 pl = __ldg(a.plan + s);
+          tok_base = pl.z;
+          slot0 = pl.w;
+          n_slots = __ldg(a.plan2 + s).y;
+        }
+        n_list = ctx - tok_base;
         if (lane < Tq) {
           m_ctx = ctx - Tq + 1 + lane;  // causal limit of query token `lane`
           const int P_t = m_ctx > 0 ? (m_ctx + PT - 1) / PT : 0;
           if (m_ctx <= 0) m_code = part == 0 ? kZero : kSkip;
+          else if (a.plan) m_code = n_slots == 1 ? kDirect : slot0 + part;
           else if (part >= P_t) m_code = kSkip;
           else if (P_t == 1) m_code = kDirect;
           else m_code = part;
@@ -637,8 +707,8 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       const int own_ctx = __shfl_sync(0xffffffffu, m_ctx, own);
       if (lane < n_groups) {
         int seq = s, lim;
-        if (r0 < T) {
-          g_tok = r0;
+        if (tok_base + r0 < T) {
+          g_tok = tok_base + r0;
           lim = T;
         } else {
           g_own = own;
@@ -809,6 +879,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         if (!ok) break;
         const int n_tiles = desc_all[slot * 16 + kDTiles];
         if (n_tiles < 0) break;  // end of work
+        if constexpr (kQToF16) {
+          ok = mbar_wait_or_abort(qconv_bar, it & 1, a.err, abort_flag);
+          if (!ok) break;
+        }
         const uint32_t q_addr = sm_q + slot * L::kQBytes;
         // S^T(h) needs its stage landed (with an 8-bit cache: widened) and
         // S^T(h-1) read by the compute warps
@@ -888,57 +962,51 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       if (lane == 0) w = mbar_wait_or_abort(bar, parity, a.err, abort_flag);
       return __shfl_sync(0xffffffffu, (int)w, 0) != 0;
     };
-    // KV8: widen the 8-bit tile gt (tile jt of the item whose group table is
-    // gmeta_s) into the 16-bit K buffer and V buffer gt & 1.  Thread t takes
-    // row t, warpgroup cg the 16-byte pieces cg, cg + NWG, ... (both layouts
-    // 128B-swizzled: piece c of row t at c ^ (t & 7), so a warp's accesses
-    // spread over every bank); a row that is no token gets a zero V row.
-    // Then the stage goes back to the producer and the MMA warp may issue
-    // S^T(gt).  K's buffer is free (S^T(gt - 1) has been read) and so is V's
-    // (O^T(gt - 2) has completed): the callers make sure.
-    auto widen = [&](int gt, int jt, const int* gmeta_s) {
+    // KV8: widen the K (or V) half of the 8-bit tile gt (tile jt of the item
+    // whose group table is gmeta_s) into the 16-bit K buffer (V buffer gt & 1).
+    // Thread t takes row t, warpgroup cg the 16-byte pieces cg, cg + NWG, ...
+    // (both layouts 128B-swizzled: piece c of row t at c ^ (t & 7), so a
+    // warp's accesses spread over every bank); a row that is no token gets a
+    // zero V row.  After K the MMA warp may issue S^T(gt) (conv); after V the
+    // stage goes back to the producer.  The callers make sure the buffer is
+    // free: K's once S^T(gt - 1) has been read, V's once O^T(gt - 2) is done.
+    auto widen = [&](int gt, int jt, const int* gmeta_s, bool is_v) {
       const int st = gt % kStages;
       const bool w = warp_wait(full_bar(st), (gt / kStages) & 1);
       if (w) {
-        const bool rok = (t & 15) < (gmeta_s[jt * kGroupsPerTile + grp_in_tile] >> 8);
-        const unsigned char* kin = smem + L::kStages0 + st * L::kStageBytes + t * 128;
-        const unsigned char* vin = kin + L::kHalf;
-        unsigned char* kout = smem + L::kK16 + t * 128;
-        unsigned char* vout = smem + L::kV16 + (gt & 1) * 2 * L::kHalf + t * 128;
+        const bool zero = is_v && (t & 15) >= (gmeta_s[jt * kGroupsPerTile + grp_in_tile] >> 8);
+        const unsigned char* in = smem + L::kStages0 + st * L::kStageBytes + (is_v ? L::kHalf : 0) + t * 128;
+        unsigned char* out = smem + (is_v ? L::kV16 + (gt & 1) * 2 * L::kHalf : L::kK16) + t * 128;
         const int sw = t & 7;
 #pragma unroll
         for (int i = 0; i < 8 / W::kNWG; ++i) {
           const int jc = cg + i * W::kNWG;  // elements 16 jc .. 16 jc + 15 of the row
-          const uint4 kx = *reinterpret_cast<const uint4*>(kin + ((jc ^ sw) << 4));
-          const uint4 vx = *reinterpret_cast<const uint4*>(vin + ((jc ^ sw) << 4));
-          uint32_t kw[8], vw[8];
-          widen16<T>(kx, kw);
-          widen16<T>(vx, vw);
-          if (!rok) {
+          const uint4 x = *reinterpret_cast<const uint4*>(in + ((jc ^ sw) << 4));
+          uint32_t wd[8];
+          widen16<MT>(x, wd);
+          if (zero) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) vw[e] = 0u;
+            for (int e = 0; e < 8; ++e) wd[e] = 0u;
           }
           const int h = jc >> 2, c = 2 * (jc & 3);  // half, first 16-byte piece of it
-          unsigned char* ko = kout + h * L::kHalf;
-          unsigned char* vo = vout + h * L::kHalf;
-          *reinterpret_cast<uint4*>(ko + ((c ^ sw) << 4)) = make_uint4(kw[0], kw[1], kw[2], kw[3]);
-          *reinterpret_cast<uint4*>(ko + (((c + 1) ^ sw) << 4)) = make_uint4(kw[4], kw[5], kw[6], kw[7]);
-          *reinterpret_cast<uint4*>(vo + ((c ^ sw) << 4)) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
-          *reinterpret_cast<uint4*>(vo + (((c + 1) ^ sw) << 4)) = make_uint4(vw[4], vw[5], vw[6], vw[7]);
+          unsigned char* o = out + h * L::kHalf;
+          *reinterpret_cast<uint4*>(o + ((c ^ sw) << 4)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+          *reinterpret_cast<uint4*>(o + (((c + 1) ^ sw) << 4)) = make_uint4(wd[4], wd[5], wd[6], wd[7]);
         }
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(empty_bar(st));
-        mbar_arrive(conv_bar);
-      }
+      if (lane == 0) mbar_arrive(is_v ? empty_bar(st) : conv_bar);
       return w;
     };
+    // Each warpgroup owns its columns: its rescale decisions, column
+    // reductions and the agreement on a failed wait take a named barrier of
+    // its own 128 threads (id 2 + cg), never one of all compute warps.
+    const int wg_bar = 2 + cg;
     for (int it = 0; ok; ++it) {
       const int slot = it % kSlots;
-      if (tid == 0) ok = mbar_wait_or_abort(ready_bar(slot), (it / kSlots) & 1, a.err, abort_flag);
-      if (named_barrier_or(1, kComputeThreads, !ok || *abort_flag)) { ok = false; break; }
+      if (t == 0) ok = mbar_wait_or_abort(ready_bar(slot), (it / kSlots) & 1, a.err, abort_flag);
+      if (named_barrier_or(wg_bar, 128, !ok || *abort_flag)) { ok = false; break; }
       const int* desc = desc_all + slot * 16;
       const int n_tiles = desc[kDTiles];
       if (n_tiles < 0) break;  // end of work
@@ -949,16 +1017,58 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       int lim_c[NCW];
 #pragma unroll
       for (int c = 0; c < NCW; ++c) lim_c[c] = mlim_all[slot * 32 + min(m_c[c], 31)];
+      float* qscale = reinterpret_cast<float*>(smem_raw + L::kQScale) + slot * 32;
+      if constexpr (kQToF16) {
+        // this warpgroup's query rows (its columns c0 .. c0 + NCW - 1),
+        // bf16 -> f16 in place, 16 threads per row (a 16-byte piece each); a
+        // row whose largest magnitude would overflow f16 is scaled down by a
+        // power of two, which its logits take back (f16 keeps every bf16
+        // significand)
+        const int rl = t >> 4, k = t & 15;
+        const int r = c0 + rl;
+        const bool act = rl < NCW && r < q_rows;
+        unsigned char* piece = smem + L::kQ + slot * L::kQBytes + (k >> 3) * N * 128 +
+                               min(r, N - 1) * 128 + (((k & 7) ^ (r & 7)) << 4);
+        const uint4 v = act ? *reinterpret_cast<const uint4*>(piece) : make_uint4(0, 0, 0, 0);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        float mx = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = Elem<__nv_bfloat16>::to_f2(w[e]);
+          mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        int ex = 0;
+        frexpf(mx, &ex);                  // mx < 2^ex
+        const int sh = max(0, ex - 15);   // mx * 2^-sh < 2^15
+        const float down = ldexpf(1.f, -sh);
+        if (act) {
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = Elem<__nv_bfloat16>::to_f2(w[e]);
+            o[e] = pack2(f.x * down, f.y * down, false);
+          }
+          *reinterpret_cast<uint4*>(piece) = make_uint4(o[0], o[1], o[2], o[3]);
+          if (k == 0) qscale[r] = ldexpf(1.f, sh);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        named_barrier(wg_bar, 128);
+        if (t == 0) mbar_arrive(qconv_bar);  // one arrival per warpgroup
+      }
       // logits in log2 units; an 8-bit cache folds each kv head's K scale in
+      // (and, with f16 query rows, each row's scale)
       float kfac[NCW];
 #pragma unroll
-      for (int c = 0; c < NCW; ++c)
+      for (int c = 0; c < NCW; ++c) {
         kfac[c] = KV8 ? a.scale_log2 * __ldg(a.k_scale + min(kvh + e_c[c], Hkv - 1)) : a.scale_log2;
+        if constexpr (kQToF16) kfac[c] *= c0 + c < q_rows ? qscale[c0 + c] : 1.f;
+      }
 
       float acc[NCW], l_tok[NCW], m_ref[NCW];
 #pragma unroll
       for (int c = 0; c < NCW; ++c) acc[c] = 0.f, l_tok[c] = 0.f, m_ref[c] = -INFINITY;
-      bool pv_acc = false;  // O^T in TMEM holds tiles not folded into acc yet
       bool ok_w = true;     // every wait of this warp so far succeeded
 
       for (int j = 0; j < n_tiles; ++j, ++g) {
@@ -975,7 +1085,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           valid[c] = row_ok && (own < 0 || own == m_c[c]) && (!PAIR || e_c[c] == e_row) &&
                      tok < lim_c[c];
         if constexpr (KV8) {
-          if (j == 0 && ok_w) ok_w = widen(g, 0, gmeta);  // an item's first tile
+          // an item's first tile: its V buffer was O^T(g-2)'s, done when the
+          // item before ended
+          if (j == 0 && ok_w) ok_w = widen(g, 0, gmeta, false);
+          if (j == 0 && ok_w) ok_w = widen(g, 0, gmeta, true);
         }
         // ---- S^T(g).  Each warp waits on its own; the OR-barrier then makes
         // every compute thread take the same way out if this or an earlier
@@ -989,18 +1102,14 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free_bar);  // S^T(g) read: the MMA warp may reuse it
-        if (named_barrier_or(1, kComputeThreads, !ok_w || *abort_flag)) { ok = false; break; }
         // O^T(g-1), the last reader of P and the last writer of O^T, is
         // waited for only where this tile needs it: before O^T is folded and
         // before P(g) is written
         bool pv_done = j == 0;
         if constexpr (KV8) {
-          // the next tile of the item is widened now, so that S^T(g+1) runs
-          // during this tile's softmax; its V buffer was O^T(g-1)'s
-          if (j + 1 < n_tiles) {
-            if (!pv_done && ok_w) ok_w = warp_wait(pv_bar, (g - 1) & 1), pv_done = true;
-            if (ok_w) ok_w = widen(g + 1, j + 1, gmeta);
-          }
+          // the next tile's K now, so that S^T(g+1) runs during this tile's
+          // softmax (its V after P(g), below)
+          if (j + 1 < n_tiles && ok_w) ok_w = widen(g + 1, j + 1, gmeta, false);
         }
         bool over = false;
 #pragma unroll
@@ -1008,8 +1117,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           sv[c] = valid[c] ? sv[c] * kfac[c] : -INFINITY;
           over |= sv[c] > m_ref[c] + kRescale;
         }
-        const bool rescale = named_barrier_or(1, kComputeThreads, over);
-        if (rescale) {
+        // one barrier for the common case (no failure, no new maximum); the
+        // rare true answer is told apart by a second one
+        if (named_barrier_or(wg_bar, 128, !ok_w || *abort_flag || over)) {
+          if (named_barrier_or(wg_bar, 128, !ok_w || *abort_flag)) { ok = false; break; }
           // new references: this tile's column maxima where they are higher
           {
             float tmp[NCW];
@@ -1018,10 +1129,12 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
             const float wmax = column_reduce<NCW, true>(tmp, lane);
             if (lane < NCW) red[quarter * N + c0 + lane] = wmax;
           }
-          named_barrier(1, kComputeThreads);
-          if (tid < NC)
-            stat[tid] = fmaxf(fmaxf(red[tid], red[N + tid]), fmaxf(red[2 * N + tid], red[3 * N + tid]));
-          named_barrier(1, kComputeThreads);
+          named_barrier(wg_bar, 128);
+          if (t < NCW) {
+            const int col = c0 + t;
+            stat[col] = fmaxf(fmaxf(red[col], red[N + col]), fmaxf(red[2 * N + col], red[3 * N + col]));
+          }
+          named_barrier(wg_bar, 128);
           float alpha[NCW];
 #pragma unroll
           for (int c = 0; c < NCW; ++c) {
@@ -1031,8 +1144,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
             m_ref[c] = m_new;
             l_tok[c] *= alpha[c];
           }
-          if (pv_acc) {
-            // fold O^T (tiles before g) into acc, on the new reference
+          if (j > 0) {
+            // fold O^T (this item's tiles before g) into acc, on the new
+            // reference, and zero these columns of O^T: the next products
+            // accumulate onto them (they do for every warpgroup)
             if (!pv_done) ok_w = warp_wait(pv_bar, (g - 1) & 1), pv_done = true;
             tc_fence_after();
             float ov[NCW], ow[NCW];
@@ -1040,11 +1155,13 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
             tmem_ld<NCW>(tmem + t_lane + (uint32_t)(2 * N + c0), ow);
 #pragma unroll
             for (int c = 0; c < NCW; ++c) acc[c] = (acc[c] + (ov[c] + ow[c])) * alpha[c];
+            tmem_zero<NCW>(tmem + t_lane + (uint32_t)(N + c0));
+            tmem_zero<NCW>(tmem + t_lane + (uint32_t)(2 * N + c0));
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
           } else {
 #pragma unroll
             for (int c = 0; c < NCW; ++c) acc[c] *= alpha[c];
           }
-          pv_acc = false;
         }
         float p[NCW];
 #pragma unroll
@@ -1066,9 +1183,9 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
           for (int i = 0; i < NW2; ++i) {
             const float x0 = p[2 * i], x1 = (2 * i + 1 < NCW) ? p[2 * i + 1] : 0.f;
-            hi[i] = pack2(x0, x1, kBf16);
-            const float2 r = Elem<T>::to_f2(hi[i]);
-            lo[i] = pack2(x0 - r.x, x1 - r.y, kBf16);
+            hi[i] = pack2(x0, x1, kMmaBf16);
+            const float2 r = Elem<MT>::to_f2(hi[i]);
+            lo[i] = pack2(x0 - r.x, x1 - r.y, kMmaBf16);
           }
           // P is free once O^T(g-1) is done; a failed wait is acted on at the
           // next OR-barrier (the stores below then only race with an MMA whose
@@ -1097,18 +1214,22 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           for (int i = cg; i < 16; i += W::kNWG)
             *reinterpret_cast<uint4*>(vrow + (i >> 3) * L::kHalf + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
         }
-        if (tid == 0) acc_flag[g & 1] = pv_acc ? 1 : 0;  // does O^T(g) accumulate?
+        // O^T(g) overwrites at an item's first tile and accumulates after it
+        if (tid == 0) acc_flag[g & 1] = j > 0 ? 1 : 0;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_ready_bar);  // P(g) written: the MMA warp issues O^T(g)
-        pv_acc = true;
+        if constexpr (KV8) {
+          // the next tile's V: its buffer was O^T(g-1)'s, waited for above
+          if (j + 1 < n_tiles && ok_w) ok_w = widen(g + 1, j + 1, gmeta, true);
+        }
       }
       if (!ok) break;
 
       // ---- item result: fold the last O^T, reduce the per-row sums, write
-      if (tid == 0 && n_tiles > 0) ok = mbar_wait_or_abort(pv_bar, (g - 1) & 1, a.err, abort_flag);
-      if (named_barrier_or(1, kComputeThreads, !ok || !ok_w || *abort_flag)) { ok = false; break; }
+      if (t == 0 && n_tiles > 0) ok = mbar_wait_or_abort(pv_bar, (g - 1) & 1, a.err, abort_flag);
+      if (named_barrier_or(wg_bar, 128, !ok || !ok_w || *abort_flag)) { ok = false; break; }
       if (n_tiles > 0) {
         tc_fence_after();
         float ov[NCW], ow[NCW];
@@ -1125,9 +1246,12 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         const float wsum = column_reduce<NCW, false>(tmp, lane);
         if (lane < NCW) red[quarter * N + c0 + lane] = wsum;
       }
-      named_barrier(1, kComputeThreads);
-      if (tid < NC) stat[N + tid] = (red[tid] + red[N + tid]) + (red[2 * N + tid] + red[3 * N + tid]);
-      named_barrier(1, kComputeThreads);
+      named_barrier(wg_bar, 128);
+      if (t < NCW) {
+        const int col = c0 + t;
+        stat[N + col] = (red[col] + red[N + col]) + (red[2 * N + col] + red[3 * N + col]);
+      }
+      named_barrier(wg_bar, 128);
       const int d = t;  // output element this thread writes, per column
 #pragma unroll
       for (int c = 0; c < NCW; ++c) {
@@ -1150,7 +1274,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           }
         }
       }
-      named_barrier(1, kComputeThreads);  // `red` and `stat` are reused by the next item
+      named_barrier(wg_bar, 128);  // this warpgroup's `red` and `stat` are reused next item
       if (lane == 0) mbar_arrive(free_bar(slot));  // its query rows have been used
     }
     if (!ok) *abort_flag = 1;
@@ -1188,7 +1312,7 @@ cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUte
     configured = true;
   }
   const int sms = sm_count();
-  const bool grouped = a0.plan != nullptr;
+  const bool grouped = a0.plan != nullptr && !a0.own_pass;
   // groups never cross a multiple of the shared-prefix window
   const int chunk = grouped ? kSharedPrefixSeqsPerLaunch : kMaxUnits;
   const int Tq = a0.query_tokens;
@@ -1200,7 +1324,7 @@ cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUte
     a.out = a0.out + rows0 * kD;
     a.block_tables = a0.block_tables + (size_t)s0 * a0.max_blocks_per_seq;
     a.context_lens = a0.context_lens + s0;
-    if (grouped) {
+    if (a0.plan) {
       a.plan = a0.plan + s0;
       a.plan2 = a0.plan2 + s0;
     }
@@ -1257,7 +1381,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, int dtype, const CUtensorMap& 
                              const CUtensorMap& tv, const CUtensorMap& tq, cudaStream_t stream,
                              int* launches, bool pair, bool fp8_cache) {
   if (a.num_seqs <= 0) return cudaSuccess;
-  const int cols = tc::tc_columns(a.group, a.query_tokens, pair, a.plan != nullptr);
+  const int cols = tc::tc_columns(a.group, a.query_tokens, pair, a.plan != nullptr && !a.own_pass);
   if (cols < 1 || cols > kTcMaxColumns) return cudaErrorInvalidValue;
   int nc = 1;
   while (nc < cols) nc *= 2;

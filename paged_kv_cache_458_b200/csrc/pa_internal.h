@@ -40,6 +40,8 @@ struct DecodeArgs {
                                  // tensor-core kernels; 1 otherwise): q, out and the
                                  // split-K rows are [num_seqs * query_tokens][Hq]
   int group;                     // g = Hq / Hkv
+  int own_pass;                  // with a plan: 1 = items over the own tokens [T, ctx) of the
+                                 // sequences whose own tokens are in no row list
   int half_boxes;                // block_size is a multiple of 8 but not of 16: each
                                  // 16-token TMA box is loaded as two 8-token boxes, which
                                  // may come from two blocks

@@ -24,13 +24,18 @@
 // plan[s] = {rank of s in its group (0 = the leader), members, T, shared
 // partitions ceil(T / partition_tokens)}; a sequence alone gets {0, 1, 0, 0}.
 //
-// The decode then reads each group through one row list: the T shared tokens,
-// followed by each member's own tokens [T, ctx) in member order, each member's
-// run rounded up to 16 rows so that a 16-row box never mixes members.  A
-// sequence alone is a group of one with T = 0.  plan2[s] = {offset of s's own
-// rows in its group's list, number of partials s gets (the partitions of the
-// list holding its shared or own rows; 1: its result is written directly, 0:
-// empty context), partitions of the list (at least 1), rows in the list}.
+// The decode then reads each group (of two or more) through one row list: the
+// T shared tokens and, when the members' own tokens [T, ctx) are few (in all
+// at most max(T, 64 x members) rows once each member's run is rounded up to
+// 16 rows, as for beam candidates), those runs in member order after them, so
+// that a 16-row box never mixes members.  Own tokens not folded into a list
+// (a long private continuation of a shared prompt, and every sequence in no
+// group, whose T is 0) are read by per-sequence items of their own.
+// plan2[s] = {offset of s's own rows in its group's list, or -1 when they are
+// read on their own; number of partials s gets (the partitions of the list
+// holding its rows, then those of its own tokens; 1: its result is written
+// directly, 0: empty context); partitions of the list (0 for a sequence in no
+// group); rows in the list}.
 #include <cuda_runtime.h>
 
 #include <climits>
@@ -139,16 +144,21 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p) {
       if (leader + m == s) my_off = off;
       off += sh_rows[m];
     }
-    const int rows = off;
+    const bool fold = n >= 2 && off - shared <= max(shared, 64 * n);
+    const int rows = fold ? off : shared;
     const int p_shared = (shared + PT - 1) / PT;
     const int own = clamp_ctx(p, s) - shared;
     int n_slots = p_shared;
     if (own > 0) {
-      const int first_p = max(my_off / PT, p_shared), last_p = (my_off + own - 1) / PT;
-      if (last_p >= first_p) n_slots += last_p - first_p + 1;
+      if (fold) {
+        const int first_p = max(my_off / PT, p_shared), last_p = (my_off + own - 1) / PT;
+        if (last_p >= first_p) n_slots += last_p - first_p + 1;
+      } else {
+        n_slots += (own + PT - 1) / PT;
+      }
     }
     p.plan[s] = n >= 2 ? make_int4(s - leader, n, shared, p_shared) : make_int4(0, 1, 0, 0);
-    p.plan2[s] = make_int4(my_off, n_slots, max(1, (rows + PT - 1) / PT), rows);
+    p.plan2[s] = make_int4(fold ? my_off : -1, n_slots, n >= 2 ? (rows + PT - 1) / PT : 0, rows);
   }
 }
 

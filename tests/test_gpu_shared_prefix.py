@@ -75,6 +75,41 @@ def expected_plan(bt, cl, block_size, group, partition_tokens):
     return plan
 
 
+def expected_plan2(plan, cl, partition_tokens):
+    """Second plan record: {own-row offset in the group's row list (-1: read
+    on their own), partial count, list partitions (0 alone), list rows}.  A
+    group folds its members' own tokens into its list when, each run rounded
+    up to 16 rows, they total at most max(T, 64 x members) rows."""
+    PT = partition_tokens
+    S = len(cl)
+    out = np.zeros((S, 4), dtype=np.int32)
+    s = 0
+    while s < S:
+        rank, n, T, p_sh = (int(x) for x in plan[s])
+        assert rank == 0
+        members = list(range(s, s + n))
+        runs = [-(-(int(cl[m]) - T) // 16) * 16 for m in members]
+        fold = n >= 2 and sum(runs) <= max(T, 64 * n)
+        off = T
+        offs = []
+        for r in runs:
+            offs.append(off)
+            off += r
+        rows = off if fold else T
+        for i, m in enumerate(members):
+            own = int(cl[m]) - T
+            slots = p_sh
+            if own > 0:
+                if fold:
+                    first, last = max(offs[i] // PT, p_sh), (offs[i] + own - 1) // PT
+                    slots += max(0, last - first + 1)
+                else:
+                    slots += -(-own // PT)
+            out[m] = (offs[i] if fold else -1, slots, -(-rows // PT) if n >= 2 else 0, rows)
+        s += n
+    return out
+
+
 def run_shared(c, dtype, partition_tokens=0, poison_ws=True):
     """pa_decode with shared_prefix; returns (out bits, plan left in the workspace)."""
     shape = shape_of(dtype, c["q"], c["k_cache"], c["block_tables"], partition_tokens, SHARED)
@@ -93,7 +128,12 @@ def run_shared(c, dtype, partition_tokens=0, poison_ws=True):
     status, bits = pa.pa_last_device_error()
     assert status == pa.PA_OK, f"device check fired: {bits:#x}"
     S = c["q"].shape[0]
+    rec = -(-16 * S // 256) * 256
     plan = ws[256:256 + 16 * S].cpu().numpy().view(np.int32).reshape(S, 4)
+    plan2 = ws[256 + rec:256 + rec + 16 * S].cpu().numpy().view(np.int32).reshape(S, 4)
+    pt = pa.pa_decode_partition_tokens(shape)
+    exp2 = expected_plan2(plan, c["context_lens"], pt)
+    assert np.array_equal(plan2, exp2), f"second plan record differs:\n{plan2}\nexpected\n{exp2}"
     return host_bits(out), plan
 
 
@@ -111,6 +151,8 @@ def groups_for(rng, group):
     g.append((2049, [2100, 2060]))             # several shared partitions
     g.append((0, [37]))                        # alone
     g.append((300, [310, 305, 301, 300][:max(2, min(4, mm))]))  # beam-like
+    g.append((200, [800, 700]))                # long own tokens: read on their own
+    g.append((512, [1000, 600, 530][:max(2, min(3, mm))]))  # a long shared prompt, long continuations
     return g
 
 
@@ -208,10 +250,11 @@ def test_shared_prefix_bad_block_ids_reported():
 
 
 def test_shared_prefix_launches():
-    """plan + one tensor-core kernel for the shared and the own tokens + merge."""
+    """plan + the row lists of the groups + the own tokens read on their own
+    (here none) + merge."""
     rng = np.random.default_rng(9600)
     c = gen.grouped_decode_case(rng, groups=[(300, [310, 320])], num_q_heads=8, num_kv_heads=1,
                                 head_dim=128, block_size=16, dtype=gen.BF16)
     before = pa.pa_kernel_launches()
     run_shared(c, gen.BF16)
-    assert pa.pa_kernel_launches() - before == 3
+    assert pa.pa_kernel_launches() - before == 4

@@ -276,7 +276,7 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
                       const float* k_scale, const float* v_scale, const int32_t* block_tables,
                       const int32_t* context_lens, float scale, void* out, const pa_shape* shape,
                       int32_t max_context_len, void* workspace, size_t workspace_bytes,
-                      pa_stream_t stream, int query_tokens = 1) {
+                      pa_stream_t stream, int query_tokens = 1, bool tables_just_written = false) {
   pa_status st = check_decode_shape(shape, max_context_len);
   if (st != PA_OK) return st;
   const bool fp8 = shape->cache_format == PA_CACHE_FP8_E4M3;
@@ -393,6 +393,7 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
       pl.max_members = pa::kTcMaxColumns / group;
       pl.min_shared = pa::decode_tc_tile_tokens();
       pl.chunk = pa::kSharedPrefixSeqsPerLaunch;
+      pl.inputs_written_before = tables_just_written ? 1 : 0;
       a.plan = plan;
       a.plan2 = plan2;
       const int chunks = (shape->num_seqs + pa::kSharedPrefixSeqsPerLaunch - 1) /
@@ -550,7 +551,7 @@ pa_status pa_decode_multi(const void* q, const void* k_cache, const void* v_cach
   count_launches(launched);
   if (ce != cudaSuccess) return cuda_failed(ce);
   return decode_impl(q, k_cache, v_cache, nullptr, nullptr, tables_v, ctx_v, scale, out, &e,
-                     max_context_len, ws + head, workspace_bytes - (size_t)head, stream);
+                     max_context_len, ws + head, workspace_bytes - (size_t)head, stream, 1, true);
 }
 
 pa_status pa_decode_fp8(const void* q, const void* k_cache, const void* v_cache,

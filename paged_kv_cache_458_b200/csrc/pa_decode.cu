@@ -405,19 +405,21 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a) {
   pdl_wait();  // every partition's partial is written
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
-  const int pair = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int Tq = a.query_tokens;
-  if (pair >= a.num_seqs * Tq * a.num_q_heads) return;
-  const int v = pair / a.num_q_heads;  // virtual sequence: query v % Tq of sequence v / Tq
+  const int n_pairs = a.num_seqs * Tq * a.num_q_heads;
+  // a fixed grid strides over the pairs: most pairs of a batch whose
+  // sequences were written directly need no merge and cost one load here
+  for (int pair = blockIdx.x * 4 + (threadIdx.x >> 5); pair < n_pairs; pair += gridDim.x * 4) {
+  const int vs = pair / a.num_q_heads;  // virtual sequence: query vs % Tq of sequence vs / Tq
   int P;
   if (a.plan2) {
-    P = __ldg(a.plan2 + v).y;
+    P = __ldg(a.plan2 + vs).y;
   } else {
-    int ctx = __ldg(a.context_lens + v / Tq);
-    ctx = max(0, min(ctx, a.max_context_len)) - Tq + 1 + v % Tq;
+    int ctx = __ldg(a.context_lens + vs / Tq);
+    ctx = max(0, min(ctx, a.max_context_len)) - Tq + 1 + vs % Tq;
     P = ctx > 0 ? (ctx + a.own_tokens - 1) / a.own_tokens : 0;
   }
-  if (P <= 1) return;
+  if (P <= 1) continue;
   const size_t base = (size_t)pair * a.num_parts;
   // (m, l) of partial p in lane p % 32: the reference M and each partial's
   // weight 2^(m_p - M) come from warp reductions, not a loop of round trips
@@ -470,6 +472,20 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a) {
   uint16_t* o = a.out + (size_t)pair * D + lane * VEC;
 #pragma unroll
   for (int v = 0; v < VEC; ++v) o[v] = Elem<T>::from_f(num[v] * inv);
+  }
+}
+
+// Grid of the merge kernel: one warp per pair up to 8 CTAs of 4 warps per SM.
+inline unsigned merge_grid(int pairs) {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+      sms = 148;
+  }
+  const long long want = (pairs + 3) / 4, cap = 8LL * sms;
+  return (unsigned)(want < cap ? want : cap);
 }
 
 // ---------------------------------------------------------------------------
@@ -504,7 +520,7 @@ cudaError_t launch_typed(const DecodeArgs& a, const CUtensorMap& tk, const CUten
   ++*launches;
   if (a.num_parts <= 1) return cudaSuccess;
   const int pairs = a.num_seqs * a.query_tokens * a.num_q_heads;
-  e = launch_pdl(decode_merge_kernel<T, D>, dim3((pairs + 3) / 4), dim3(128), 0, stream, a);
+  e = launch_pdl(decode_merge_kernel<T, D>, dim3(merge_grid(pairs)), dim3(128), 0, stream, a);
   if (e == cudaSuccess) ++*launches;
   return e;
 }
@@ -551,7 +567,7 @@ cudaError_t launch_decode_merge(const DecodeArgs& a, int dtype, int head_dim, cu
                                 int* launches) {
   if (a.num_parts <= 1 || a.num_seqs <= 0) return cudaSuccess;
   const int pairs = a.num_seqs * a.query_tokens * a.num_q_heads;
-  const dim3 grid((pairs + 3) / 4), block(128);
+  const dim3 grid(merge_grid(pairs)), block(128);
   cudaError_t e;
   if (dtype == 0) {
     e = head_dim == 128 ? launch_pdl(decode_merge_kernel<__half, 128>, grid, block, 0, stream, a)

@@ -63,11 +63,11 @@
 // 128B-swizzled), into one of three stages; a dedicated MMA warp issues every
 // MMA and commits it to an mbarrier; the compute warps consume tiles in order
 // and tell it through two more mbarriers when S^T(g) has been read and when
-// P(g) has been written.  Per-sequence items are numbered partition 0 of every
-// sequence first, then each sequence's further partitions (measured 2 % faster
-// on mistral_7b_gqa than full partitions first and the shorter last ones
-// after them); a group's items, full partitions first and the shorter last
-// ones after them.
+// P(g) has been written.  Without a plan, items are numbered partition 0 of
+// every sequence first, then each sequence's further partitions (measured 2 %
+// faster on mistral_7b_gqa than full partitions first and the shorter last
+// ones after them); with one (only some sequences are units), full partitions
+// first and the shorter last ones after them.
 // Rows that are no token of any column are masked in P and their V rows are
 // zeroed in shared memory before the PV product, so stale or NaN rows never
 // reach the result.
@@ -539,6 +539,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     // compute warps, so none of its global round trips holds up the loads.
     // =====================================================================
     const int S = a.num_seqs;
+    // partition 0 of every sequence first when every sequence is a unit (no
+    // plan); with a plan (groups, or own tokens read on their own) only some
+    // sequences are units: full partitions first, then the last ones
+    const bool p0_first = a.plan == nullptr;
     constexpr int PPL = kMaxUnits / 32 + 1;  // prefix[0..S] over the lanes
     int pre_f[PPL], pre_p[PPL];
     int carry_f = 0, carry_p = 0;
@@ -569,7 +573,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         if (rows >= 0) {
           full = rows / PT;
           last = (rows % PT != 0 || rows == 0) ? 1 : 0;
-          if (!grouped) {
+          if (p0_first) {
             full = full + last - 1;  // further partitions after partition 0
             last = 0;
           }
@@ -588,7 +592,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       carry_p += __shfl_sync(0xffffffffu, inc_p, 31);
     }
     const int Hu = Hkv / kHeads;  // kv units of the item numbering
-    const int total = Hu * (carry_f + carry_p) + (grouped ? 0 : S * Hu);
+    const int total = Hu * (carry_f + carry_p) + (p0_first ? S * Hu : 0);
 
     bool ok = true;
     int it = 0;
@@ -616,7 +620,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       unsigned long long ticket = 0;
       if (lane == 0) ticket = take_begin(a.work_counter);
       int s, kvu, part;
-      if (!grouped) {
+      if (p0_first) {
         // partition 0 of every sequence, then further partitions by sequence
         if (f < S * Hu) {
           s = f / Hu, kvu = f % Hu, part = 0;

@@ -62,6 +62,8 @@ struct PlanArgs {
   int max_members;               // members per group (32 / g)
   int min_shared;                // fewer shared tokens than this: no group
   int chunk;                     // groups stay inside [k * chunk, (k + 1) * chunk)
+  int inputs_written_before;     // 1: the kernel just before wrote the tables or lengths (the
+                                 // plan then reads them only after waiting for it)
 };
 cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream, int* launches);
 // Virtual one-token sequences for Tq query tokens per sequence (pa_plan.cu).

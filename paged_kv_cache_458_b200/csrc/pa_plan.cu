@@ -62,9 +62,14 @@ __device__ __forceinline__ int first_block(const PlanArgs& p, int s) {
   return (b >= 0 && b < p.num_blocks) ? b : -1;
 }
 
-// One CTA per sequence.
+// One CTA per sequence.  The tables and lengths are inputs no kernel of this
+// library writes (except the query expansion of pa_decode_multi, after which
+// inputs_written_before is set): the search runs before waiting for the
+// kernel before this one, overlapping it, and only the plan's writes wait
+// (the decode and merge of an earlier call may still be reading the plan
+// until then).
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p) {
-  pdl_wait();  // the tables and lengths of this step are written
+  if (p.inputs_written_before) pdl_wait();
   pdl_launch_dependents();
   __shared__ int sh_edge, sh_min_ctx, sh_min_blocks, sh_common;
   __shared__ int sh_rows[32];  // own rows of each member, rounded up to 16
@@ -157,6 +162,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p) {
         n_slots += (own + PT - 1) / PT;
       }
     }
+    pdl_wait();
     p.plan[s] = n >= 2 ? make_int4(s - leader, n, shared, p_shared) : make_int4(0, 1, 0, 0);
     p.plan2[s] = make_int4(fold ? my_off : -1, n_slots, n >= 2 ? (rows + PT - 1) / PT : 0, rows);
   }

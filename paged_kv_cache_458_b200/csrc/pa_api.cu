@@ -367,6 +367,7 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
     // columns fit 16 and blocks give 16-row boxes; shared-prefix groups keep
     // one head per item
     const bool pair = shape->num_kv_heads % 2 == 0 && !a.half_boxes && 2 * group * query_tokens <= 16;
+    bool own_tc = true;
     CUtensorMap tk, tv, tq;
     if (!make_tc_maps(&tk, &tv, &tq, k_cache, v_cache, q, shape, pair, query_tokens, false))
       return cuda_failed("cuTensorMapEncodeTiled failed");
@@ -394,6 +395,11 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
       pl.min_shared = pa::decode_tc_tile_tokens();
       pl.chunk = pa::kSharedPrefixSeqsPerLaunch;
       pl.inputs_written_before = tables_just_written ? 1 : 0;
+      // own tokens read on their own go to the kernel this shape would get
+      // without shared prefixes: tensor cores at larger groups, else CUDA
+      // cores (in their largest partitions: few partials)
+      own_tc = use_tensor_cores(shape);
+      pl.own_partition_tokens = own_tc ? a.partition_tokens : pa::decode_max_partition_tokens();
       a.plan = plan;
       a.plan2 = plan2;
       const int chunks = (shape->num_seqs + pa::kSharedPrefixSeqsPerLaunch - 1) /
@@ -403,6 +409,19 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
       if (e == cudaSuccess) e = pa::launch_decode_tc(a, shape->dtype, gk, gv, gq, cs, &launched, false, fp8);
       a.own_pass = 1;
       a.epoch = next_epochs((shape->num_seqs + 511) / 512);
+      if (!own_tc && e == cudaSuccess) {
+        // the CUDA-core kernel (it launches the merge itself)
+        CUtensorMap pk, pv;
+        if (!make_pool_map(&pk, k_cache, shape, box_rows(shape)) ||
+            !make_pool_map(&pv, v_cache, shape, box_rows(shape)))
+          return cuda_failed("cuTensorMapEncodeTiled failed");
+        a.own_tokens = pa::decode_max_partition_tokens();
+        a.grid_parts = (max_context_len + a.own_tokens - 1) / a.own_tokens;
+        if (a.grid_parts < 1) a.grid_parts = 1;
+        e = pa::launch_decode(a, shape->dtype, shape->head_dim, group, pk, pv, cs, &launched, fp8);
+        count_launches(launched);
+        return e == cudaSuccess ? PA_OK : cuda_failed(e);
+      }
     } else {
       a.epoch = next_epochs((shape->num_seqs + 511) / 512);
     }

@@ -165,6 +165,18 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
     ctx = max(0, min(ctx, ctx_cap));
   }
   const int q_head0 = kvh * G;
+  // With a shared-prefix plan this kernel reads the own tokens [T, ctx) of
+  // the sequences whose own tokens are in no group's row list (every
+  // sequence in no group, T = 0), as partials after its shared ones.
+  int base = 0, slot0 = 0, n_parts_seq = -1;
+  if (a.plan) {
+    const int4 pl = __ldg(a.plan + s);
+    const int4 p2 = __ldg(a.plan2 + s);
+    if (!(p2.x < 0 && (pl.y == 1 || ctx > pl.z))) return;
+    base = pl.z;
+    slot0 = pl.w;
+    n_parts_seq = p2.y;
+  }
   if (ctx == 0) {
     if (part == 0) {
       uint16_t* o = a.out + ((size_t)s * a.num_q_heads + q_head0) * D;
@@ -173,10 +185,10 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
     return;
   }
   const int PT = a.own_tokens;
-  const int t_begin = part * PT;
+  const int t_begin = base + part * PT;
   if (t_begin >= ctx) return;
   const int t_end = min(ctx, t_begin + PT);
-  const int n_parts_seq = (ctx + PT - 1) / PT;
+  if (n_parts_seq < 0) n_parts_seq = (ctx + PT - 1) / PT;
   const int n_chunks = (t_end - t_begin + kChunk - 1) / kChunk;
   const int n_mine = warp < n_chunks ? (n_chunks - warp + NW - 1) / NW : 0;
 
@@ -384,7 +396,7 @@ decode_partition_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap 
     if (direct) {
       a.out[qh * D + d] = Elem<T>::from_f(num / den);
     } else {
-      const size_t slot = qh * a.num_parts + part;
+      const size_t slot = qh * a.num_parts + slot0 + part;
       a.ws_acc[slot * D + d] = num;
       if (d == 0) {
         a.ws_ml[2 * slot] = M;
@@ -484,8 +496,10 @@ inline unsigned merge_grid(int pairs) {
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
       sms = 148;
   }
-  const long long want = (pairs + 3) / 4, cap = 8LL * sms;
-  return (unsigned)(want < cap ? want : cap);
+  // one warp per pair: a merge is a few dependent round trips, which a warp
+  // striding over several pairs would pay one after another
+  (void)sms;
+  return (unsigned)((pairs + 3) / 4);
 }
 
 // ---------------------------------------------------------------------------

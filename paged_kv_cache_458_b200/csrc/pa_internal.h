@@ -34,7 +34,8 @@ struct DecodeArgs {
   // row list, number of partials it gets (1: written directly), partitions
   // of the group's row list, rows in that list}.
   const int4* plan2;
-  int own_tokens;                // partition size of the CUDA-core kernel
+  int own_tokens;                // partition size of the CUDA-core kernel (with a plan: of the
+                                 // own tokens it reads)
   int grid_parts;                // partitions per (sequence, kv head) of the CUDA-core grid
   int query_tokens;              // query tokens per sequence (pa_decode_multi on the
                                  // tensor-core kernels; 1 otherwise): q, out and the
@@ -59,6 +60,7 @@ struct PlanArgs {
   int4* plan2;                   // [S] out
   int num_seqs, max_blocks_per_seq, block_size, num_blocks, max_context_len;
   int partition_tokens;
+  int own_partition_tokens;      // partition of the own tokens read on their own
   int max_members;               // members per group (32 / g)
   int min_shared;                // fewer shared tokens than this: no group
   int chunk;                     // groups stay inside [k * chunk, (k + 1) * chunk)

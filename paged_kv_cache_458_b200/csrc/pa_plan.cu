@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p) {
         const int first_p = max(my_off / PT, p_shared), last_p = (my_off + own - 1) / PT;
         if (last_p >= first_p) n_slots += last_p - first_p + 1;
       } else {
-        n_slots += (own + PT - 1) / PT;
+        n_slots += (own + p.own_partition_tokens - 1) / p.own_partition_tokens;
       }
     }
     pdl_wait();

@@ -75,7 +75,7 @@ def expected_plan(bt, cl, block_size, group, partition_tokens):
     return plan
 
 
-def expected_plan2(plan, cl, partition_tokens):
+def expected_plan2(plan, cl, partition_tokens, own_partition_tokens):
     """Second plan record: {own-row offset in the group's row list (-1: read
     on their own), partial count, list partitions (0 alone), list rows}.  A
     group folds its members' own tokens into its list when, each run rounded
@@ -104,7 +104,7 @@ def expected_plan2(plan, cl, partition_tokens):
                     first, last = max(offs[i] // PT, p_sh), (offs[i] + own - 1) // PT
                     slots += max(0, last - first + 1)
                 else:
-                    slots += -(-own // PT)
+                    slots += -(-own // own_partition_tokens)
             out[m] = (offs[i] if fold else -1, slots, -(-rows // PT) if n >= 2 else 0, rows)
         s += n
     return out
@@ -132,7 +132,12 @@ def run_shared(c, dtype, partition_tokens=0, poison_ws=True):
     plan = ws[256:256 + 16 * S].cpu().numpy().view(np.int32).reshape(S, 4)
     plan2 = ws[256 + rec:256 + rec + 16 * S].cpu().numpy().view(np.int32).reshape(S, 4)
     pt = pa.pa_decode_partition_tokens(shape)
-    exp2 = expected_plan2(plan, c["context_lens"], pt)
+    # own tokens read on their own: the kernel the shape gets without shared
+    # prefixes, the tensor-core one in partitions of pt, the CUDA-core one in
+    # its largest partitions (2048 tokens)
+    plain = shape_of(dtype, c["q"], c["k_cache"], c["block_tables"], partition_tokens)
+    own_pt = pt if pa.pa_decode_resolved_variant(plain) == pa.PA_DECODE_TENSOR_CORES else 2048
+    exp2 = expected_plan2(plan, c["context_lens"], pt, own_pt)
     assert np.array_equal(plan2, exp2), f"second plan record differs:\n{plan2}\nexpected\n{exp2}"
     return host_bits(out), plan
 

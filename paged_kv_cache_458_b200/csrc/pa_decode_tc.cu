@@ -545,18 +545,24 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     const bool p0_first = a.plan == nullptr;
     constexpr int PPL = kMaxUnits / 32 + 1;  // prefix[0..S] over the lanes
     int pre_f[PPL], pre_p[PPL];
-    int carry_f = 0, carry_p = 0;
+    // First every unit's counts (full partitions in pre_f, the last one in
+    // pre_p), all loads independent of one another so that they are in
+    // flight together; then the scans, in place.
 #pragma unroll
     for (int k = 0; k < PPL; ++k) {
       const int s = k * 32 + lane;  // this lane's unit
       int full = 0, last = 0;
       if (s < S) {
+        int ctx = __ldg(a.context_lens + s);
+        int4 pl = make_int4(0, 1, 0, 0), p2 = make_int4(0, 0, 0, 0);
+        if (a.plan) {
+          pl = __ldg(a.plan + s);
+          p2 = __ldg(a.plan2 + s);
+        }
         int rows = -1;  // rows of the unit's list; -1: not a unit
         if (grouped) {
-          const int4 pl = __ldg(a.plan + s);
-          if (pl.x == 0 && pl.y >= 2) rows = __ldg(a.plan2 + s).w;
+          if (pl.x == 0 && pl.y >= 2) rows = p2.w;
         } else {
-          int ctx = __ldg(a.context_lens + s);
           if (ctx < 0 || ctx > a.max_context_len) {
             if (blockIdx.x == 0) report(a.err, kErrContextLen);
             ctx = max(0, min(ctx, a.max_context_len));
@@ -565,8 +571,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           if (a.plan) {
             // own tokens read on their own: a sequence in no group (even an
             // empty one, whose item writes zeros), or a member with own tokens
-            const int4 pl = __ldg(a.plan + s);
-            const bool alone = __ldg(a.plan2 + s).x < 0 && (pl.y == 1 || ctx > pl.z);
+            const bool alone = p2.x < 0 && (pl.y == 1 || ctx > pl.z);
             rows = alone ? ctx - pl.z : -1;
           }
         }
@@ -579,6 +584,14 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           }
         }
       }
+      pre_f[k] = full;
+      pre_p[k] = last;
+    }
+    int carry_f = 0, carry_p = 0;
+#pragma unroll
+    for (int k = 0; k < PPL; ++k) {
+      const int s = k * 32 + lane;
+      const int full = pre_f[k], last = pre_p[k];
       int inc_f = full, inc_p = last;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {

@@ -408,7 +408,7 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
       e = pa::launch_plan(pl, cs, &launched);
       if (e == cudaSuccess) e = pa::launch_decode_tc(a, shape->dtype, gk, gv, gq, cs, &launched, false, fp8);
       a.own_pass = 1;
-      a.epoch = next_epochs((shape->num_seqs + 511) / 512);
+      a.epoch = next_epochs((shape->num_seqs + pa::kSharedPrefixSeqsPerLaunch - 1) / pa::kSharedPrefixSeqsPerLaunch);
       if (!own_tc && e == cudaSuccess) {
         // the CUDA-core kernel (it launches the merge itself)
         CUtensorMap pk, pv;
@@ -423,7 +423,7 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
         return e == cudaSuccess ? PA_OK : cuda_failed(e);
       }
     } else {
-      a.epoch = next_epochs((shape->num_seqs + 511) / 512);
+      a.epoch = next_epochs((shape->num_seqs + pa::kSharedPrefixSeqsPerLaunch - 1) / pa::kSharedPrefixSeqsPerLaunch);
     }
     if (e == cudaSuccess)
       e = pa::launch_decode_tc(a, shape->dtype, tk, tv, tq, cs, &launched, pair, fp8);

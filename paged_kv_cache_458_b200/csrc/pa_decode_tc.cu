@@ -97,7 +97,7 @@ constexpr int kGroupRows = 16;      // rows per TMA box (a block is a multiple)
 constexpr int kSlots = 2;           // item slots
 constexpr int kStages = 3;          // K/V stages of 64 KB
 constexpr int kMaxGroups = 32;      // 16-row groups per item (partition_tokens <= 512)
-constexpr int kMaxUnits = 512;      // sequences (or group leaders) per launch
+constexpr int kMaxUnits = kSharedPrefixSeqsPerLaunch;  // sequences per launch (256)
 // Where a member's result for an item goes (codes >= 0 are split-K slots).
 constexpr int kSkip = -1, kDirect = -2, kZero = -3;
 
@@ -379,6 +379,73 @@ __host__ __device__ inline int tc_columns(int group, int query_tokens, bool pair
   return grouped ? kTcMaxColumns : query_tokens * (pair ? 2 : 1) * group;
 }
 
+// Every unit's partition counts and their exclusive prefix over the units of
+// the launch (see locate).  Called by all 32 lanes of the scheduler warp.  The
+// loads never branch (indices clamped to the batch), so all of them are in
+// flight together.  Units: without a plan, every sequence (rows = its
+// context; p0_first: pre_f counts the partitions after partition 0);
+// grouped, the leaders of groups of two or more (rows = the list's); own
+// pass, the sequences whose own tokens are in no list (rows = ctx - T).
+template <int PPL>
+__device__ __forceinline__ void unit_prefix(const DecodeArgs& a, bool grouped, bool p0_first, int PT,
+                                            int lane, int (&pre_f)[PPL], int (&pre_p)[PPL],
+                                            int& carry_f, int& carry_p) {
+  const int S = a.num_seqs;
+#pragma unroll
+  for (int k = 0; k < PPL; ++k) {
+    const int s = k * 32 + lane;  // this lane's unit
+    const int sc = min(s, S - 1);
+    int ctx = __ldg(a.context_lens + sc);
+    int4 pl = make_int4(0, 1, 0, 0), p2 = make_int4(0, 0, 0, 0);
+    if (a.plan) {
+      pl = __ldg(a.plan + sc);
+      p2 = __ldg(a.plan2 + sc);
+    }
+    int rows = -1;  // rows of the unit's list; -1: not a unit
+    if (grouped) {
+      if (pl.x == 0 && pl.y >= 2) rows = p2.w;
+    } else {
+      if (s < S && (ctx < 0 || ctx > a.max_context_len) && blockIdx.x == 0) report(a.err, kErrContextLen);
+      ctx = max(0, min(ctx, a.max_context_len));
+      rows = ctx;
+      if (a.plan) {
+        // own tokens read on their own: a sequence in no group (even an empty
+        // one, whose item writes zeros), or a member with own tokens
+        const bool alone = p2.x < 0 && (pl.y == 1 || ctx > pl.z);
+        rows = alone ? ctx - pl.z : -1;
+      }
+    }
+    int full = 0, last = 0;
+    if (s < S && rows >= 0) {
+      full = rows / PT;
+      last = (rows % PT != 0 || rows == 0) ? 1 : 0;
+      if (p0_first) {
+        full = full + last - 1;  // further partitions after partition 0
+        last = 0;
+      }
+    }
+    pre_f[k] = full;
+    pre_p[k] = last;
+  }
+  carry_f = 0, carry_p = 0;
+#pragma unroll
+  for (int k = 0; k < PPL; ++k) {
+    const int s = k * 32 + lane;
+    const int full = pre_f[k], last = pre_p[k];
+    int inc_f = full, inc_p = last;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int tf = __shfl_up_sync(0xffffffffu, inc_f, o);
+      const int tp = __shfl_up_sync(0xffffffffu, inc_p, o);
+      if (lane >= o) inc_f += tf, inc_p += tp;
+    }
+    pre_f[k] = s <= S ? carry_f + inc_f - full : INT_MAX;
+    pre_p[k] = s <= S ? carry_p + inc_p - last : INT_MAX;
+    carry_f += __shfl_sync(0xffffffffu, inc_f, 31);
+    carry_p += __shfl_sync(0xffffffffu, inc_p, 31);
+  }
+}
+
 // Sixteen E4M3 codes (one 16-byte piece of a row, first element in the lowest
 // byte) -> sixteen 16-bit values of T, two per word, first element in the low
 // half.  Exact: every E4M3 value is an f16 (the hardware conversion) and a bf16.
@@ -540,72 +607,19 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     // =====================================================================
     const int S = a.num_seqs;
     // partition 0 of every sequence first when every sequence is a unit (no
-    // plan); with a plan (groups, or own tokens read on their own) only some
-    // sequences are units: full partitions first, then the last ones
+    // plan): the first item of every CTA is then known without the prefix
+    // counts, which are computed while its tiles load; with a plan (groups, or
+    // own tokens read on their own) only some sequences are units: full
+    // partitions first, then the last ones, counted before the first item
     const bool p0_first = a.plan == nullptr;
+    const int Hu = Hkv / kHeads;  // kv units of the item numbering
     constexpr int PPL = kMaxUnits / 32 + 1;  // prefix[0..S] over the lanes
     int pre_f[PPL], pre_p[PPL];
-    // First every unit's counts (full partitions in pre_f, the last one in
-    // pre_p), all loads independent of one another so that they are in
-    // flight together; then the scans, in place.
-#pragma unroll
-    for (int k = 0; k < PPL; ++k) {
-      const int s = k * 32 + lane;  // this lane's unit
-      int full = 0, last = 0;
-      if (s < S) {
-        int ctx = __ldg(a.context_lens + s);
-        int4 pl = make_int4(0, 1, 0, 0), p2 = make_int4(0, 0, 0, 0);
-        if (a.plan) {
-          pl = __ldg(a.plan + s);
-          p2 = __ldg(a.plan2 + s);
-        }
-        int rows = -1;  // rows of the unit's list; -1: not a unit
-        if (grouped) {
-          if (pl.x == 0 && pl.y >= 2) rows = p2.w;
-        } else {
-          if (ctx < 0 || ctx > a.max_context_len) {
-            if (blockIdx.x == 0) report(a.err, kErrContextLen);
-            ctx = max(0, min(ctx, a.max_context_len));
-          }
-          rows = ctx;
-          if (a.plan) {
-            // own tokens read on their own: a sequence in no group (even an
-            // empty one, whose item writes zeros), or a member with own tokens
-            const bool alone = p2.x < 0 && (pl.y == 1 || ctx > pl.z);
-            rows = alone ? ctx - pl.z : -1;
-          }
-        }
-        if (rows >= 0) {
-          full = rows / PT;
-          last = (rows % PT != 0 || rows == 0) ? 1 : 0;
-          if (p0_first) {
-            full = full + last - 1;  // further partitions after partition 0
-            last = 0;
-          }
-        }
-      }
-      pre_f[k] = full;
-      pre_p[k] = last;
-    }
     int carry_f = 0, carry_p = 0;
-#pragma unroll
-    for (int k = 0; k < PPL; ++k) {
-      const int s = k * 32 + lane;
-      const int full = pre_f[k], last = pre_p[k];
-      int inc_f = full, inc_p = last;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int tf = __shfl_up_sync(0xffffffffu, inc_f, o);
-        const int tp = __shfl_up_sync(0xffffffffu, inc_p, o);
-        if (lane >= o) inc_f += tf, inc_p += tp;
-      }
-      pre_f[k] = s <= S ? carry_f + inc_f - full : INT_MAX;
-      pre_p[k] = s <= S ? carry_p + inc_p - last : INT_MAX;
-      carry_f += __shfl_sync(0xffffffffu, inc_f, 31);
-      carry_p += __shfl_sync(0xffffffffu, inc_p, 31);
-    }
-    const int Hu = Hkv / kHeads;  // kv units of the item numbering
-    const int total = Hu * (carry_f + carry_p) + (p0_first ? S * Hu : 0);
+    if (!p0_first) unit_prefix(a, grouped, p0_first, PT, lane, pre_f, pre_p, carry_f, carry_p);
+    // items known so far (without a plan, the partition-0 items until the
+    // prefix is in)
+    int total = p0_first ? S * Hu : Hu * (carry_f + carry_p);
 
     bool ok = true;
     int it = 0;
@@ -629,9 +643,6 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         }
         break;
       }
-      // the next item's number, fetched while this one is resolved
-      unsigned long long ticket = 0;
-      if (lane == 0) ticket = take_begin(a.work_counter);
       int s, kvu, part;
       if (p0_first) {
         // partition 0 of every sequence, then further partitions by sequence
@@ -659,35 +670,44 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       int tok_base = 0;               // token of the list's first row (own-token pass)
       int m_ctx = 0, m_off = 0, m_code = kSkip;
       const int p0 = part * PT;
+      const int r0 = p0 + lane * kGroupRows;  // this lane's 16-row group of the list
+      // without a plan a lane's group is the sequence's tokens r0 .. r0 + 15:
+      // its table entries are read at once, with the context (entries below
+      // max_context_len lie inside the table; only a group below the context
+      // uses its entry)
+      int spec_blk = -1, spec_blk2 = -1;
+      const int32_t* stable = a.block_tables + (size_t)s * a.max_blocks_per_seq;
+      if (!a.plan) {
+        if (r0 < a.max_context_len) spec_blk = __ldg(stable + r0 / a.block_size);
+        if (a.half_boxes && r0 + kGroupRows / 2 < a.max_context_len)
+          spec_blk2 = __ldg(stable + (r0 + kGroupRows / 2) / a.block_size);
+      }
       if (grouped) {
+        // the group's plan and every member's record and context in one round
+        // trip (lanes past the group read a neighbour, unused)
+        const int sl = min(s + lane, S - 1);
         const int4 pl = __ldg(a.plan + s);
+        const int4 p2 = __ldg(a.plan2 + sl);
+        const int cx = __ldg(a.context_lens + sl);
         members = pl.y;
         T = pl.z;
         const int p_sh = pl.w;
         vbase = s;
-        int m_slots = 0;
+        n_list = __shfl_sync(0xffffffffu, p2.w, 0);
         if (lane < members) {
-          const int4 p2 = __ldg(a.plan2 + s + lane);
           m_off = p2.x;
-          m_slots = p2.y;
-          m_ctx = max(0, min(__ldg(a.context_lens + s + lane), a.max_context_len));
-        }
-        n_list = __shfl_sync(0xffffffffu, __ldg(a.plan2 + s).w, 0);
-        if (lane < members) {
+          m_ctx = max(0, min(cx, a.max_context_len));
           const int own = m_ctx - T;
           const int first_own = max(m_off / PT, p_sh);
           const bool mine = part < p_sh || (m_off >= 0 && own > 0 && part >= m_off / PT &&
                                             part <= (m_off + own - 1) / PT);
           if (m_ctx == 0) m_code = part == 0 ? kZero : kSkip;
           else if (!mine) m_code = kSkip;
-          else if (m_slots == 1) m_code = kDirect;
+          else if (p2.y == 1) m_code = kDirect;
           else m_code = part < p_sh ? part : p_sh + part - first_own;
         }
       } else {
-        const int ctx = max(0, min(__ldg(a.context_lens + s), a.max_context_len));
-        members = Tq;
-        T = ctx;  // every row is every query's, up to its limit
-        vbase = s * Tq;
+        int ctx = __ldg(a.context_lens + s);
         // with a plan, the own tokens [base, ctx) after the partials of the
         // sequence's shared tokens
         int slot0 = 0, n_slots = 0;
@@ -697,6 +717,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
           slot0 = pl.w;
           n_slots = __ldg(a.plan2 + s).y;
         }
+        ctx = max(0, min(ctx, a.max_context_len));
+        members = Tq;
+        T = ctx;  // every row is every query's, up to its limit
+        vbase = s * Tq;
         n_list = ctx - tok_base;
         if (lane < Tq) {
           m_ctx = ctx - Tq + 1 + lane;  // causal limit of query token `lane`
@@ -714,12 +738,17 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       const int n_groups = (n_rows + kGroupRows - 1) / kGroupRows;  // <= 32
       // ---- 16-row groups (lane i): owner, first token, valid rows, pool rows
       int g_own = -1, g_tok = 0, g_valid = 0, g_row = 0, g_row2 = 0;
-      const int r0 = p0 + lane * kGroupRows;
       // own rows: the member whose run holds r0 (runs are in member order,
-      // offsets non-decreasing; an empty run holds nothing)
+      // offsets non-decreasing; an empty run holds nothing): a binary search
       int own = 0;
-      for (int m = 1; m < members; ++m)
-        if (__shfl_sync(0xffffffffu, m_off, m) <= r0) own = m;
+      if (grouped) {
+#pragma unroll
+        for (int step = 16; step >= 1; step >>= 1) {
+          const int cand = own + step;
+          const int o = __shfl_sync(0xffffffffu, m_off, cand & 31);
+          if (cand < members && o <= r0) own = cand;
+        }
+      }
       const int own_off = __shfl_sync(0xffffffffu, m_off, own);
       const int own_ctx = __shfl_sync(0xffffffffu, m_ctx, own);
       if (lane < n_groups) {
@@ -737,16 +766,20 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         // With 8-token blocks (half_boxes) rows 8..15 of a group have their own
         // entry; past the group's valid rows they re-read the first block (masked).
         const int32_t* table = a.block_tables + (size_t)seq * a.max_blocks_per_seq;
-        auto resolve = [&](int tok) {
-          const int blk = __ldg(table + tok / a.block_size);
+        auto resolve = [&](int tok, int blk) {
           if (blk < 0 || blk >= a.num_blocks) {
             report(a.err, kErrBlockId);
             return a.num_blocks * a.block_size;  // outside the map: TMA fills zeros
           }
           return blk * a.block_size + tok % a.block_size;
         };
-        g_row = resolve(g_tok);
-        if (a.half_boxes) g_row2 = g_valid > kGroupRows / 2 ? resolve(g_tok + kGroupRows / 2) : g_row;
+        g_row = resolve(g_tok, a.plan ? __ldg(table + g_tok / a.block_size) : spec_blk);
+        if (a.half_boxes) {
+          const int t2 = g_tok + kGroupRows / 2;
+          g_row2 = g_valid > kGroupRows / 2
+                       ? resolve(t2, a.plan ? __ldg(table + t2 / a.block_size) : spec_blk2)
+                       : g_row;
+        }
       }
       {
         int* rows = rows_all + slot * 64;
@@ -770,9 +803,16 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         mbar_arrive(meta_bar(slot));
         mbar_arrive(rb);  // with the query rows' bytes, completes the ready phase
       }
-      int nf = 0;
-      if (lane == 0) {
-        const int t = take_end(a.work_counter, ticket, a.epoch, a.err);
+      if (p0_first && it == 0) {
+        // the counts of the further partitions, while this item's tiles load
+        unit_prefix(a, grouped, p0_first, PT, lane, pre_f, pre_p, carry_f, carry_p);
+        total = Hu * carry_f + S * Hu;
+      }
+      // the next item: a launch with no more items than CTAs takes none
+      // (every CTA had its one item); else from the work counter
+      int nf = total;
+      if (lane == 0 && total > (int)gridDim.x) {
+        const int t = take_end(a.work_counter, take_begin(a.work_counter), a.epoch, a.err);
         nf = t < 0 ? total : (int)gridDim.x + t;
       }
       f = __shfl_sync(0xffffffffu, nf, 0);
@@ -1331,7 +1371,7 @@ cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUte
   const int sms = sm_count();
   const bool grouped = a0.plan != nullptr && !a0.own_pass;
   // groups never cross a multiple of the shared-prefix window
-  const int chunk = grouped ? kSharedPrefixSeqsPerLaunch : kMaxUnits;
+  const int chunk = kMaxUnits;
   const int Tq = a0.query_tokens;
   for (int s0 = 0; s0 < a0.num_seqs; s0 += chunk) {
     DecodeArgs a = a0;

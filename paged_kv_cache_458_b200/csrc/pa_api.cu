@@ -100,7 +100,8 @@ pa_status check_decode_shape(const pa_shape* s, int32_t max_context_len) {
       (s->variant != PA_DECODE_AUTO || s->head_dim != 128 || pt % pa::decode_tc_tile_tokens() != 0 ||
        pt > 512))
     return PA_ERR_UNSUPPORTED;
-  // work items of one launch (<= 512 sequences) must fit the 24-bit counter
+  // work items of one launch (256 sequences; the bound takes 512) must fit the
+  // 24-bit counter
   const long long parts = ((long long)max_context_len + pt - 1) / pt;
   if (512LL * s->num_kv_heads * (parts > 0 ? parts : 1) >= (1LL << 23)) return PA_ERR_UNSUPPORTED;
   return PA_OK;

@@ -380,40 +380,32 @@ __host__ __device__ inline int tc_columns(int group, int query_tokens, bool pair
 }
 
 // Every unit's partition counts and their exclusive prefix over the units of
-// the launch (see locate).  Called by all 32 lanes of the scheduler warp.  The
-// loads never branch (indices clamped to the batch), so all of them are in
-// flight together.  Units: without a plan, every sequence (rows = its
-// context; p0_first: pre_f counts the partitions after partition 0);
-// grouped, the leaders of groups of two or more (rows = the list's); own
-// pass, the sequences whose own tokens are in no list (rows = ctx - T).
+// the launch (see locate).  Called by all 32 lanes of the scheduler warp.  A
+// unit's rows come from one load per sequence, all of them issued before any
+// is used (indices clamped to the batch), so they are in flight together:
+// without a plan every sequence is a unit (rows = its context; p0_first:
+// pre_f counts the partitions after partition 0); grouped, the leaders of
+// groups of two or more (rows = their list's, the plan's fourth field);
+// own pass, the sequences whose own tokens are in no list (rows = ctx - T,
+// the plan's third field).  -1: no unit.
 template <int PPL>
 __device__ __forceinline__ void unit_prefix(const DecodeArgs& a, bool grouped, bool p0_first, int PT,
                                             int lane, int (&pre_f)[PPL], int (&pre_p)[PPL],
                                             int& carry_f, int& carry_p) {
   const int S = a.num_seqs;
+  int rows_k[PPL];
+#pragma unroll
+  for (int k = 0; k < PPL; ++k) {
+    const int sc = min(k * 32 + lane, S - 1);
+    rows_k[k] = grouped ? __ldg(&a.plan2[sc].w) : a.plan ? __ldg(&a.plan2[sc].z) : __ldg(a.context_lens + sc);
+  }
 #pragma unroll
   for (int k = 0; k < PPL; ++k) {
     const int s = k * 32 + lane;  // this lane's unit
-    const int sc = min(s, S - 1);
-    int ctx = __ldg(a.context_lens + sc);
-    int4 pl = make_int4(0, 1, 0, 0), p2 = make_int4(0, 0, 0, 0);
-    if (a.plan) {
-      pl = __ldg(a.plan + sc);
-      p2 = __ldg(a.plan2 + sc);
-    }
-    int rows = -1;  // rows of the unit's list; -1: not a unit
-    if (grouped) {
-      if (pl.x == 0 && pl.y >= 2) rows = p2.w;
-    } else {
-      if (s < S && (ctx < 0 || ctx > a.max_context_len) && blockIdx.x == 0) report(a.err, kErrContextLen);
-      ctx = max(0, min(ctx, a.max_context_len));
-      rows = ctx;
-      if (a.plan) {
-        // own tokens read on their own: a sequence in no group (even an empty
-        // one, whose item writes zeros), or a member with own tokens
-        const bool alone = p2.x < 0 && (pl.y == 1 || ctx > pl.z);
-        rows = alone ? ctx - pl.z : -1;
-      }
+    int rows = rows_k[k];
+    if (!a.plan) {
+      if (s < S && (rows < 0 || rows > a.max_context_len) && blockIdx.x == 0) report(a.err, kErrContextLen);
+      rows = max(0, min(rows, a.max_context_len));
     }
     int full = 0, last = 0;
     if (s < S && rows >= 0) {

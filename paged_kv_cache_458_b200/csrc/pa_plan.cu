@@ -34,8 +34,10 @@
 // plan2[s] = {offset of s's own rows in its group's list, or -1 when they are
 // read on their own; number of partials s gets (the partitions of the list
 // holding its rows, then those of its own tokens; 1: its result is written
-// directly, 0: empty context); partitions of the list (0 for a sequence in no
-// group); rows in the list}.
+// directly, 0: empty context); rows s's own tokens are read in on their own
+// (ctx - T), or -1 when they are not (in a list, or none); rows in the list
+// of the group s leads, or -1 when s leads no group of two or more}.  The last
+// two are what the decode's item numbering counts per sequence: one load each.
 #include <cuda_runtime.h>
 
 #include <climits>
@@ -164,7 +166,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p) {
     }
     pdl_wait();
     p.plan[s] = n >= 2 ? make_int4(s - leader, n, shared, p_shared) : make_int4(0, 1, 0, 0);
-    p.plan2[s] = make_int4(fold ? my_off : -1, n_slots, n >= 2 ? (rows + PT - 1) / PT : 0, rows);
+    const int own_rows = !fold && (n == 1 || own > 0) ? own : -1;
+    p.plan2[s] = make_int4(fold ? my_off : -1, n_slots, own_rows, n >= 2 && s == leader ? rows : -1);
   }
 }
 

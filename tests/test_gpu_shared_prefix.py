@@ -77,9 +77,11 @@ def expected_plan(bt, cl, block_size, group, partition_tokens):
 
 def expected_plan2(plan, cl, partition_tokens, own_partition_tokens):
     """Second plan record: {own-row offset in the group's row list (-1: read
-    on their own), partial count, list partitions (0 alone), list rows}.  A
-    group folds its members' own tokens into its list when, each run rounded
-    up to 16 rows, they total at most max(T, 64 x members) rows."""
+    on their own), partial count, rows of the own tokens read on their own
+    (-1: none, or in the list), rows of the list the sequence leads (-1: it
+    leads no group of two or more)}.  A group folds its members' own tokens
+    into its list when, each run rounded up to 16 rows, they total at most
+    max(T, 64 x members) rows."""
     PT = partition_tokens
     S = len(cl)
     out = np.zeros((S, 4), dtype=np.int32)
@@ -105,7 +107,8 @@ def expected_plan2(plan, cl, partition_tokens, own_partition_tokens):
                     slots += max(0, last - first + 1)
                 else:
                     slots += -(-own // own_partition_tokens)
-            out[m] = (offs[i] if fold else -1, slots, -(-rows // PT) if n >= 2 else 0, rows)
+            own_rows = own if not fold and (n == 1 or own > 0) else -1
+            out[m] = (offs[i] if fold else -1, slots, own_rows, rows if i == 0 and n >= 2 else -1)
         s += n
     return out
 

@@ -95,7 +95,7 @@ constexpr int kTile = 128;          // MMA rows per tile (M)
 constexpr int kD = 128;             // head_dim of this path
 constexpr int kGroupRows = 16;      // rows per TMA box (a block is a multiple)
 constexpr int kSlots = 2;           // item slots
-constexpr int kStages = 3;          // K/V stages of 64 KB
+constexpr int kStages = 3;          // K/V stages of 64 KB (K and V halves filled and freed apart)
 constexpr int kMaxGroups = 32;      // 16-row groups per item (partition_tokens <= 512)
 constexpr int kMaxUnits = kSharedPrefixSeqsPerLaunch;  // sequences per launch (256)
 // Where a member's result for an item goes (codes >= 0 are split-K slots).
@@ -110,7 +110,7 @@ struct Warps {
   static constexpr int kNCW = NC >= 16 ? 8 : (NC >= 8 ? 4 : NC);  // columns per warpgroup
   static constexpr int kNWG = NC / kNCW;                           // compute warpgroups
   static constexpr int kCompute = 128 * kNWG;                      // compute threads
-  static constexpr int kThreads = kCompute + 96;                   // + MMA, producer, scheduler warps
+  static constexpr int kThreads = kCompute + 128;  // + MMA, K producer, scheduler, V producer warps
   static_assert(kNCW * kNWG == NC, "columns split evenly");
 };
 
@@ -124,9 +124,9 @@ struct Warps {
 template <int N, bool KV8>
 struct Layout {
   // small region (byte offsets from the dynamic base)
-  // barriers: full[3], empty[3], ready[2], free[2], meta[2], qk, pv, drain, s_free, p_ready,
-  // conv, qconv
-  static constexpr int kNumBars = 2 * kStages + 3 * kSlots + 7;
+  // barriers: K full[3], K empty[3], ready[2], free[2], meta[2], qk, pv, drain, s_free,
+  // p_ready, conv, qconv, V full[3], V empty[3]
+  static constexpr int kNumBars = 4 * kStages + 3 * kSlots + 7;
   static constexpr int kBars = 0;
   static constexpr int kMisc = kBars + kNumBars * 8;        // tmem address, abort flag, accumulate flags [2]
   static constexpr int kDesc = kMisc + 16;                  // [slots][16] int
@@ -476,7 +476,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   constexpr int kComputeThreads = W::kCompute, kThreads = W::kThreads, NCW = W::kNCW;
   constexpr int kComputeWarps = kComputeThreads / 32;
   constexpr int kMmaWarp = kComputeWarps, kProducerWarp = kComputeWarps + 1,
-                kSchedWarp = kComputeWarps + 2;
+                kSchedWarp = kComputeWarps + 2, kProducerVWarp = kComputeWarps + 3;
   using L = Layout<N, KV8>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   // An 8-bit cache is widened to f16 (one conversion per pair) and the
@@ -526,8 +526,11 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + L::kMisc + 4);
   volatile int* acc_flag = reinterpret_cast<volatile int*>(smem_raw + L::kMisc + 8);  // [2]
   const uint32_t bars = smem_addr(smem_raw + L::kBars);
+  // stage st's K half and V half: landed (full), and free again (empty)
   auto full_bar = [&](int st) { return bars + st * 8; };
   auto empty_bar = [&](int st) { return bars + (kStages + st) * 8; };
+  auto vfull_bar = [&](int st) { return bars + (2 * kStages + 3 * kSlots + 7 + st) * 8; };
+  auto vempty_bar = [&](int st) { return bars + (3 * kStages + 3 * kSlots + 7 + st) * 8; };
   auto ready_bar = [&](int sl) { return bars + (2 * kStages + sl) * 8; };
   auto free_bar = [&](int sl) { return bars + (2 * kStages + kSlots + sl) * 8; };
   auto meta_bar = [&](int sl) { return bars + (2 * kStages + 2 * kSlots + sl) * 8; };
@@ -554,9 +557,11 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   if (tid == 0) {
     for (int st = 0; st < kStages; ++st) {
       mbar_init(full_bar(st), 1);
-      // a stage is released by the MMA warp's commit, or with an 8-bit cache
-      // by every compute warp once it has widened the tile
+      mbar_init(vfull_bar(st), 1);
+      // a half is released by the MMA warp's commit after its products, or
+      // with an 8-bit cache by every compute warp once it has widened it
       mbar_init(empty_bar(st), KV8 ? kComputeWarps : 1);
+      mbar_init(vempty_bar(st), KV8 ? kComputeWarps : 1);
     }
     for (int sl = 0; sl < kSlots; ++sl) {
       mbar_init(ready_bar(sl), 1);
@@ -817,11 +822,14 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     if (lane == 0)
       for (int k = max(0, it - (ok ? 1 : kSlots)); k < it; ++k)
         mbar_wait(ready_bar(k % kSlots), (k / kSlots) & 1, a.err);
-  } else if (warp == kProducerWarp) {
+  } else if (warp == kProducerWarp || warp == kProducerVWarp) {
     // =====================================================================
-    // producer warp: the K/V tiles of each item, from the rows the scheduler
-    // resolved, by TMA into the stage ring
+    // producer warps: one loads the K half of each tile, the other the V
+    // half, by TMA from the rows the scheduler resolved.  Each half of a
+    // stage is freed on its own (K once S^T is computed, V once O^T is), so
+    // the K loads run up to a tile further ahead than the V loads.
     // =====================================================================
+    const bool is_v = warp == kProducerVWarp;
     int issued = 0;  // tiles armed so far (stage ring position)
     bool ok = true;
     for (int it = 0; ok; ++it) {
@@ -842,29 +850,31 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       const int n_groups = (desc[kDEnd] - desc[kDBegin] + kGroupRows - 1) / kGroupRows;
       const int my_row = rows_all[slot * 64 + lane];
       const int my_row2 = rows_all[slot * 64 + 32 + lane];
+      const void* map = is_v ? &tm_v : &tm_k;
       for (int j = 0; j < n_tiles && ok; ++j) {
         const int st = issued % kStages;
         if (issued >= kStages &&
-            !mbar_wait_or_abort(empty_bar(st), ((issued / kStages) - 1) & 1, a.err, abort_flag)) {
+            !mbar_wait_or_abort(is_v ? vempty_bar(st) : empty_bar(st), ((issued / kStages) - 1) & 1, a.err,
+                                abort_flag)) {
           ok = false;
           break;
         }
         const int g0 = j * kGroupsPerTile;
         const int ng = min(kGroupsPerTile, n_groups - g0);
-        const uint32_t fb = full_bar(st);
-        const uint32_t dst = sm_stages + st * L::kStageBytes;
+        const uint32_t fb = is_v ? vfull_bar(st) : full_bar(st);
+        // this warp's half of the stage: K at its start, V after it
+        const uint32_t dst = sm_stages + st * L::kStageBytes + (is_v ? L::kStageBytes / 2 : 0);
         constexpr int kBoxBytes = kHeads * kGroupRows * 128;  // one box: a group of kHeads heads
-        if (lane == 0) mbar_arrive_expect_tx(fb, ng * (KV8 ? 2 : 4) * kBoxBytes);
+        if (lane == 0) mbar_arrive_expect_tx(fb, ng * (KV8 ? 1 : 2) * kBoxBytes);
         __syncwarp();
         if constexpr (KV8) {
-          // lane 2 r + k loads K (k = 0) or V (k = 1) of group r: 128 one-byte
-          // elements x 16 rows (x 2 heads), the whole head_dim in one box
-          const int r = lane >> 1, k = lane & 1;
+          // lane r loads group r: 128 one-byte elements x 16 rows (x 2 heads),
+          // the whole head_dim in one box
+          const int r = lane;
           const int row = __shfl_sync(0xffffffffu, my_row, min(g0 + r, 31));
           const int row2 = __shfl_sync(0xffffffffu, my_row2, min(g0 + r, 31));
           if (r < ng) {
-            const uint32_t d = dst + k * L::kHalf + r * kBoxBytes;
-            const void* map = k == 0 ? &tm_k : &tm_v;
+            const uint32_t d = dst + r * kBoxBytes;
             if constexpr (PAIR) {
               tma_load_3d(d, map, fb, 0, row, kvh);
             } else {
@@ -873,20 +883,19 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
             }
           }
         } else {
-          // lane 4 r + k loads piece k (K or V, 64-element half) of group r
-          const int r = lane >> 2, k = lane & 3;
+          // lane 2 r + k loads the 64-element half k of group r
+          const int r = lane >> 1, k = lane & 1;
           const int row = __shfl_sync(0xffffffffu, my_row, min(g0 + r, 31));
           const int row2 = __shfl_sync(0xffffffffu, my_row2, min(g0 + r, 31));
           if (r < ng) {
             const uint32_t d = dst + k * L::kHalf + r * kBoxBytes;
-            const void* map = k < 2 ? &tm_k : &tm_v;
             if constexpr (PAIR) {
               // maps of this kind are [rows][head] with the head innermost
               // after the dims: a box is 16 rows of head kvh, then of kvh + 1
-              tma_load_3d(d, map, fb, (k & 1) * 64, row, kvh);
+              tma_load_3d(d, map, fb, k * 64, row, kvh);
             } else {
-              tma_load_3d(d, map, fb, (k & 1) * 64, kvh, row);
-              if (a.half_boxes) tma_load_3d(d + (kGroupRows / 2) * 128, map, fb, (k & 1) * 64, kvh, row2);
+              tma_load_3d(d, map, fb, k * 64, kvh, row);
+              if (a.half_boxes) tma_load_3d(d + (kGroupRows / 2) * 128, map, fb, k * 64, kvh, row2);
             }
           }
         }
@@ -897,7 +906,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     // Every TMA copy armed by this warp lands before the CTA leaves.
     if (lane == 0)
       for (int k = max(0, issued - kStages); k < issued; ++k)
-        mbar_wait(full_bar(k % kStages), (k / kStages) & 1, a.err);
+        mbar_wait(is_v ? vfull_bar(k % kStages) : full_bar(k % kStages), (k / kStages) & 1, a.err);
   } else if (warp == kMmaWarp) {
     // =====================================================================
     // MMA warp (lane 0): every tcgen05.mma of the CTA, so that issuing them
@@ -920,6 +929,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                 kIdescQK, kk > 0);
       }
       mma_commit(qk_bar);
+      if constexpr (!KV8) mma_commit(empty_bar(st));  // the K half is free once S^T is done
     };
     if (lane == 0) {
       for (int it = 0; ok; ++it) {
@@ -952,6 +962,8 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
             if (!ok) break;
           }
           ok = mbar_wait_or_abort(p_ready_bar, g & 1, a.err, abort_flag);
+          // the V half has landed (with an 8-bit cache the compute warps widened it)
+          if (ok && !KV8) ok = mbar_wait_or_abort(vfull_bar(st), (g / kStages) & 1, a.err, abort_flag);
           if (!ok) break;
           tc_fence_after();
           const uint32_t vt = KV8 ? smem_addr(smem + L::kV16) + (g & 1) * 2 * L::kHalf
@@ -963,7 +975,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                     smem_desc(sm_p + kk * 512, L::kPAtom, 256, kSw32), kIdescPV,
                     acc0 | (uint32_t)(kk > 0));
           mma_commit(pv_bar);
-          if constexpr (!KV8) mma_commit(empty_bar(st));  // the stage is free once these MMAs are done
+          if constexpr (!KV8) mma_commit(vempty_bar(st));  // the V half is free once these MMAs are done
         }
       }
       if (!ok) *abort_flag = 1;
@@ -1016,12 +1028,13 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     // Thread t takes row t, warpgroup cg the 16-byte pieces cg, cg + NWG, ...
     // (both layouts 128B-swizzled: piece c of row t at c ^ (t & 7), so a
     // warp's accesses spread over every bank); a row that is no token gets a
-    // zero V row.  After K the MMA warp may issue S^T(gt) (conv); after V the
-    // stage goes back to the producer.  The callers make sure the buffer is
-    // free: K's once S^T(gt - 1) has been read, V's once O^T(gt - 2) is done.
+    // zero V row.  After K the MMA warp may issue S^T(gt) (conv); each half of
+    // the stage goes back to its producer once widened.  The callers make sure
+    // the buffer is free: K's once S^T(gt - 1) has been read, V's once
+    // O^T(gt - 2) is done.
     auto widen = [&](int gt, int jt, const int* gmeta_s, bool is_v) {
       const int st = gt % kStages;
-      const bool w = warp_wait(full_bar(st), (gt / kStages) & 1);
+      const bool w = warp_wait(is_v ? vfull_bar(st) : full_bar(st), (gt / kStages) & 1);
       if (w) {
         const bool zero = is_v && (t & 15) >= (gmeta_s[jt * kGroupsPerTile + grp_in_tile] >> 8);
         const unsigned char* in = smem + L::kStages0 + st * L::kStageBytes + (is_v ? L::kHalf : 0) + t * 128;
@@ -1045,7 +1058,14 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
-      if (lane == 0) mbar_arrive(is_v ? empty_bar(st) : conv_bar);
+      if (lane == 0) {
+        if (is_v) {
+          mbar_arrive(vempty_bar(st));
+        } else {
+          mbar_arrive(empty_bar(st));
+          mbar_arrive(conv_bar);
+        }
+      }
       return w;
     };
     // Each warpgroup owns its columns: its rescale decisions, column
@@ -1254,6 +1274,12 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
             *reinterpret_cast<uint16_t*>(prow + L::kPBytes) = (uint16_t)lo[0];
           }
         }
+        if constexpr (!KV8) {
+          // the V half lands apart from the K half: it is waited for before a
+          // row of it is zeroed (this is a warp-wide wait, taken by the warps
+          // that have such a row)
+          if (__any_sync(0xffffffffu, !row_ok) && ok_w) ok_w = warp_wait(vfull_bar(st), (g / kStages) & 1);
+        }
         if (!KV8 && !row_ok) {
           // this row is no token: zero its V row (both 64-element halves, 16
           // pieces shared out over the column groups) so 0 * stale never
@@ -1302,10 +1328,21 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       }
       named_barrier(wg_bar, 128);
       const int d = t;  // output element this thread writes, per column
+      // the shared-memory reads first, then the stores: the compiler keeps a
+      // read through these pointers after a global store that came before it
+      int code_c[NCW];
+      float sum_c[NCW];
+      {
+        const int members = desc[kDMembers];
+#pragma unroll
+        for (int c = 0; c < NCW; ++c) {
+          code_c[c] = m_c[c] < members ? mcode_all[slot * 32 + m_c[c]] : kSkip;  // padded: none
+          sum_c[c] = stat[N + c0 + c];
+        }
+      }
 #pragma unroll
       for (int c = 0; c < NCW; ++c) {
-        if (m_c[c] >= desc[kDMembers]) continue;  // a padded column
-        const int code = mcode_all[slot * 32 + m_c[c]];
+        const int code = code_c[c];
         if (code == kSkip) continue;
         const size_t qh = (size_t)(vbase + m_c[c]) * a.num_q_heads + (size_t)(kvh + e_c[c]) * G + h_c[c];
         // an 8-bit cache applies its V scale here (the merge is linear in it)
@@ -1313,13 +1350,13 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         if (code == kZero) {
           a.out[qh * kD + d] = 0;
         } else if (code == kDirect) {
-          a.out[qh * kD + d] = Elem<T>::from_f(o / stat[N + c0 + c]);
+          a.out[qh * kD + d] = Elem<T>::from_f(o / sum_c[c]);
         } else {
           const size_t wslot = qh * a.num_parts + code;
           a.ws_acc[wslot * kD + d] = o;
           if (d == 0) {
             a.ws_ml[2 * wslot] = m_ref[c];
-            a.ws_ml[2 * wslot + 1] = stat[N + c0 + c];
+            a.ws_ml[2 * wslot + 1] = sum_c[c];
           }
         }
       }

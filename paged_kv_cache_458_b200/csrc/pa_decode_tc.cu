@@ -105,12 +105,17 @@ constexpr int kSkip = -1, kDirect = -2, kZero = -3;
 // warps reads TMEM lane quarter w % 4 (MMA rows 32 (w % 4) .. +31, output rows
 // likewise) and handles columns [(w / 4) NCW, (w / 4 + 1) NCW).  More warps
 // per scheduler hide the latency of the per-column softmax arithmetic.
-template <int NC>
+template <int NC, bool KV8>
 struct Warps {
   static constexpr int kNCW = NC >= 16 ? 8 : (NC >= 8 ? 4 : NC);  // columns per warpgroup
   static constexpr int kNWG = NC / kNCW;                           // compute warpgroups
   static constexpr int kCompute = 128 * kNWG;                      // compute threads
-  static constexpr int kThreads = kCompute + 128;  // + MMA, K producer, scheduler, V producer warps
+  // + MMA, K producer, scheduler, V producer warps; with an E4M3 cache the
+  // converter warps: one or two warpgroups (each row of a tile taken by one or
+  // two threads: K into TMEM, V into shared memory).  Two, unless the four
+  // compute warpgroups need the registers.
+  static constexpr int kConvWarps = KV8 ? (kNWG == 4 ? 4 : 8) : 0;
+  static constexpr int kThreads = kCompute + 128 + 32 * kConvWarps;
   static_assert(kNCW * kNWG == NC, "columns split evenly");
 };
 
@@ -119,14 +124,16 @@ struct Warps {
 // stages, the query slots and P, whose swizzled layouts need that alignment.
 // TMEM: S^T in [0, N); O^T hi in [N, 2N), O^T lo in [2N, 3N).
 // With an E4M3 cache (KV8) the stages only land the 8-bit tiles (32 KB); the
-// compute warps widen each one into a 16-bit K tile (one buffer) and a 16-bit
-// V tile (two buffers, alternating by tile), which the MMAs read.
+// converter warps widen each K tile into TMEM (two buffers of 64 columns,
+// alternating by tile: S^T's A operand) and each V tile into a 16-bit V tile
+// in shared memory (two buffers, alternating by tile).
 template <int N, bool KV8>
 struct Layout {
   // small region (byte offsets from the dynamic base)
   // barriers: K full[3], K empty[3], ready[2], free[2], meta[2], qk, pv, drain, s_free,
-  // p_ready, conv, qconv, V full[3], V empty[3]
-  static constexpr int kNumBars = 4 * kStages + 3 * kSlots + 7;
+  // p_ready, conv, qconv, V full[3], V empty[3], then (KV8) per widened V buffer: widened[2],
+  // free[2], and per widened K buffer: widened[2], free[2]
+  static constexpr int kNumBars = 4 * kStages + 3 * kSlots + 7 + (KV8 ? 8 : 0);
   static constexpr int kBars = 0;
   static constexpr int kMisc = kBars + kNumBars * 8;        // tmem address, abort flag, accumulate flags [2]
   static constexpr int kDesc = kMisc + 16;                  // [slots][16] int
@@ -143,8 +150,7 @@ struct Layout {
   static constexpr int kHalf = kTile * 128;  // a 64-element half of a 16-bit tile, or an 8-bit tile (16 KB)
   static constexpr int kStageBytes = KV8 ? 2 * kHalf : 4 * kHalf;  // K tile then V tile
   static constexpr int kStages0 = 0;
-  static constexpr int kK16 = kStages0 + kStages * kStageBytes;   // KV8: widened K [2 halves]
-  static constexpr int kV16 = kK16 + (KV8 ? 2 * kHalf : 0);       // KV8: widened V [2][2 halves]
+  static constexpr int kV16 = kStages0 + kStages * kStageBytes;  // KV8: widened V [2][2 halves]
   static constexpr int kQ = kV16 + (KV8 ? 4 * kHalf : 0);         // [slots][2 halves][N rows][128 B]
   static constexpr int kQBytes = 2 * N * 128;
   static constexpr int kP = kQ + kSlots * kQBytes;          // P hi, then P lo
@@ -189,6 +195,16 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b,
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// As mma_f16, with A read from TMEM (rows in lanes, two 16-bit elements per column).
+__device__ __forceinline__ void mma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -247,6 +263,16 @@ __device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[NCOL]) {
 }
 
 // Zero NCOL (1 .. 8) consecutive fp32 columns of this thread's TMEM lane.
+// Store 16 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+      "%13, %14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
 template <int NCOL>
 __device__ __forceinline__ void tmem_zero(uint32_t taddr) {
   const uint32_t z = 0u;
@@ -462,21 +488,24 @@ __device__ __forceinline__ void widen16(const uint4 x, uint32_t (&w)[8]) {
 }
 
 template <typename T, int NC, bool PAIR, bool KV8>
-__global__ void __launch_bounds__(Warps<NC>::kThreads, 1)
+__global__ void __launch_bounds__(Warps<NC, KV8>::kThreads, 1)
 decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q) {
   constexpr int N = NC <= 16 ? 16 : 32;          // MMA columns
-  constexpr uint32_t kTmemCols = N == 16 ? 64 : 128;
+  // S^T, O^T hi and lo, and with an 8-bit cache two widened K tiles (A operands)
+  constexpr uint32_t kACol = 3 * N;  // KV8: K buffer b at kACol + 64 b (two f16 per column)
+  constexpr uint32_t kTmemCols = KV8 ? 256 : (N == 16 ? 64 : 128);
   // A tile is kTok tokens of each of the item's kHeads kv heads, as kTile MMA
   // rows (with two heads, 16-row groups of head 2e and head 2e+1 alternate)
   constexpr int kHeads = PAIR ? 2 : 1;
   constexpr int kTok = kTile / kHeads;
   constexpr int kGroupsPerTile = kTok / kGroupRows;
-  using W = Warps<NC>;
+  using W = Warps<NC, KV8>;
   constexpr int kComputeThreads = W::kCompute, kThreads = W::kThreads, NCW = W::kNCW;
   constexpr int kComputeWarps = kComputeThreads / 32;
   constexpr int kMmaWarp = kComputeWarps, kProducerWarp = kComputeWarps + 1,
-                kSchedWarp = kComputeWarps + 2, kProducerVWarp = kComputeWarps + 3;
+                kSchedWarp = kComputeWarps + 2, kProducerVWarp = kComputeWarps + 3,
+                kConvWarp0 = kComputeWarps + 4;  // KV8: K converters, then V converters
   using L = Layout<N, KV8>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   // An 8-bit cache is widened to f16 (one conversion per pair) and the
@@ -531,6 +560,12 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   auto empty_bar = [&](int st) { return bars + (kStages + st) * 8; };
   auto vfull_bar = [&](int st) { return bars + (2 * kStages + 3 * kSlots + 7 + st) * 8; };
   auto vempty_bar = [&](int st) { return bars + (3 * kStages + 3 * kSlots + 7 + st) * 8; };
+  // KV8, 16-bit V buffer b: widened for its tile, and free again (O^T done)
+  auto vconv_bar = [&](int b) { return bars + (4 * kStages + 3 * kSlots + 7 + b) * 8; };
+  auto vfree_bar = [&](int b) { return bars + (4 * kStages + 3 * kSlots + 9 + b) * 8; };
+  // KV8, TMEM K buffer b: widened for its tile, and free again (S^T done)
+  auto aconv_bar = [&](int b) { return bars + (4 * kStages + 3 * kSlots + 11 + b) * 8; };
+  auto afree_bar = [&](int b) { return bars + (4 * kStages + 3 * kSlots + 13 + b) * 8; };
   auto ready_bar = [&](int sl) { return bars + (2 * kStages + sl) * 8; };
   auto free_bar = [&](int sl) { return bars + (2 * kStages + kSlots + sl) * 8; };
   auto meta_bar = [&](int sl) { return bars + (2 * kStages + 2 * kSlots + sl) * 8; };
@@ -539,7 +574,6 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
   const uint32_t drain_bar = qk_bar + 16;
   const uint32_t s_free_bar = qk_bar + 24;   // compute warps have read S^T(g)
   const uint32_t p_ready_bar = qk_bar + 32;  // compute warps have written P(g)
-  const uint32_t conv_bar = qk_bar + 40;     // KV8: compute warps have widened tile g
   const uint32_t qconv_bar = qk_bar + 48;    // the item's query rows are f16 (kQToF16)
   const uint32_t sm_stages = smem_addr(smem + L::kStages0);
   const uint32_t sm_q = smem_addr(smem + L::kQ);
@@ -560,8 +594,16 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       mbar_init(vfull_bar(st), 1);
       // a half is released by the MMA warp's commit after its products, or
       // with an 8-bit cache by every compute warp once it has widened it
-      mbar_init(empty_bar(st), KV8 ? kComputeWarps : 1);
-      mbar_init(vempty_bar(st), KV8 ? kComputeWarps : 1);
+      mbar_init(empty_bar(st), KV8 ? W::kConvWarps : 1);
+      mbar_init(vempty_bar(st), KV8 ? W::kConvWarps : 1);
+    }
+    if constexpr (KV8) {
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(vconv_bar(b), W::kConvWarps);
+        mbar_init(vfree_bar(b), 1);
+        mbar_init(aconv_bar(b), W::kConvWarps);
+        mbar_init(afree_bar(b), 1);
+      }
     }
     for (int sl = 0; sl < kSlots; ++sl) {
       mbar_init(ready_bar(sl), 1);
@@ -573,7 +615,6 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     mbar_init(drain_bar, 1);
     mbar_init(s_free_bar, kComputeWarps);
     mbar_init(p_ready_bar, kComputeWarps);
-    mbar_init(conv_bar, kComputeWarps);
     mbar_init(qconv_bar, W::kNWG);
     *abort_flag = 0;
     mbar_init_fence();
@@ -918,18 +959,27 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     // =====================================================================
     bool ok = true;
     int g = 0;  // tiles issued so far
-    auto issue_qk = [&](int st, uint32_t q_addr) {
+    auto issue_qk = [&](int h, uint32_t q_addr) {
       tc_fence_after();
-      const uint32_t kt = KV8 ? smem_addr(smem + L::kK16) : sm_stages + st * L::kStageBytes;
+      const int st = h % kStages;
+      const uint32_t kt = sm_stages + st * L::kStageBytes;
 #pragma unroll
       for (int kk = 0; kk < kD / 16; ++kk) {
-        const uint32_t ko = (kk / 4) * L::kHalf + (kk % 4) * 32;
         const uint32_t qo = (kk / 4) * N * 128 + (kk % 4) * 32;
-        mma_f16(tmem, smem_desc(kt + ko, 16, 1024, kSw128), smem_desc(q_addr + qo, 16, 1024, kSw128),
-                kIdescQK, kk > 0);
+        if constexpr (KV8) {
+          // A = the widened K tile in TMEM: row r in lane r, dims 16 kk .. 16 kk + 15
+          // in columns 8 kk .. 8 kk + 7
+          mma_f16_ta(tmem, tmem + kACol + 64 * (h & 1) + 8 * kk, smem_desc(q_addr + qo, 16, 1024, kSw128),
+                     kIdescQK, kk > 0);
+        } else {
+          const uint32_t ko = (kk / 4) * L::kHalf + (kk % 4) * 32;
+          mma_f16(tmem, smem_desc(kt + ko, 16, 1024, kSw128), smem_desc(q_addr + qo, 16, 1024, kSw128),
+                  kIdescQK, kk > 0);
+        }
       }
       mma_commit(qk_bar);
       if constexpr (!KV8) mma_commit(empty_bar(st));  // the K half is free once S^T is done
+      if constexpr (KV8) mma_commit(afree_bar(h & 1));  // the TMEM K buffer too
     };
     if (lane == 0) {
       for (int it = 0; ok; ++it) {
@@ -946,10 +996,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         // S^T(h) needs its stage landed (with an 8-bit cache: widened) and
         // S^T(h-1) read by the compute warps
         auto qk_for = [&](int h) {
-          bool w = KV8 ? mbar_wait_or_abort(conv_bar, h & 1, a.err, abort_flag)
+          bool w = KV8 ? mbar_wait_or_abort(aconv_bar(h & 1), (h >> 1) & 1, a.err, abort_flag)
                        : mbar_wait_or_abort(full_bar(h % kStages), (h / kStages) & 1, a.err, abort_flag);
           if (w && h > 0) w = mbar_wait_or_abort(s_free_bar, (h - 1) & 1, a.err, abort_flag);
-          if (w) issue_qk(h % kStages, q_addr);
+          if (w) issue_qk(h, q_addr);
           return w;
         };
         if (n_tiles > 0) ok = qk_for(g);
@@ -962,8 +1012,9 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
             if (!ok) break;
           }
           ok = mbar_wait_or_abort(p_ready_bar, g & 1, a.err, abort_flag);
-          // the V half has landed (with an 8-bit cache the compute warps widened it)
+          // the V half has landed (with an 8-bit cache: has been widened)
           if (ok && !KV8) ok = mbar_wait_or_abort(vfull_bar(st), (g / kStages) & 1, a.err, abort_flag);
+          if (ok && KV8) ok = mbar_wait_or_abort(vconv_bar(g & 1), (g >> 1) & 1, a.err, abort_flag);
           if (!ok) break;
           tc_fence_after();
           const uint32_t vt = KV8 ? smem_addr(smem + L::kV16) + (g & 1) * 2 * L::kHalf
@@ -976,6 +1027,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                     acc0 | (uint32_t)(kk > 0));
           mma_commit(pv_bar);
           if constexpr (!KV8) mma_commit(vempty_bar(st));  // the V half is free once these MMAs are done
+          if constexpr (KV8) mma_commit(vfree_bar(g & 1));    // the 16-bit V buffer too
         }
       }
       if (!ok) *abort_flag = 1;
@@ -984,6 +1036,114 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       mbar_wait(drain_bar, 0, a.err);
     }
     __syncwarp();
+  } else if (KV8 && warp >= kConvWarp0) {
+    // =====================================================================
+    // converter warps (E4M3 cache): row t of every tile (TMEM lane t) is taken
+    // by the threads of lane t % 32 in the warps of lane quarter t / 32, each
+    // widening a share of its 16-byte pieces.  Per tile g: the 8-bit K row
+    // widened into TMEM K buffer g & 1 once S^T(g-2) is done with it; then the
+    // 8-bit V row widened into shared V buffer g & 1 once O^T(g-2) is done
+    // with it.  A row that is no token of
+    // its tile gets a zero V row, so a stale NaN never meets p = 0.  The 8-bit
+    // tiles and the 16-bit V tiles are 128B-swizzled: 16-byte piece c of row
+    // t sits at c ^ (t & 7).  The buffers let the widening run up to two
+    // tiles ahead of the products.
+    // =====================================================================
+    const int quarter = warp & 3;
+    const int t = quarter * 32 + lane;
+    const uint32_t t_lane = (uint32_t)(quarter * 32) << 16;
+    const int sw = t & 7;
+    constexpr int kShares = W::kConvWarps >= 8 ? 2 : 1;  // threads per row
+    constexpr int kPieces = 8 / kShares;            // 16-byte 8-bit pieces per thread
+    const int p0 = ((warp - kConvWarp0) >> 2) * kPieces;  // this thread's first piece
+    bool ok = true;
+    int g = 0;  // tiles widened so far, numbered across items
+    auto conv_wait = [&](uint32_t bar, uint32_t parity) {
+      bool r = true;
+      if (lane == 0) r = mbar_wait_or_abort(bar, parity, a.err, abort_flag);
+      return __shfl_sync(0xffffffffu, (int)r, 0) != 0;
+    };
+    for (int it = 0; ok; ++it) {
+      const int slot = it % kSlots;
+      if (!conv_wait(meta_bar(slot), (it / kSlots) & 1)) {
+        ok = false;
+        break;
+      }
+      __syncwarp();  // lane 0's acquire orders the other lanes' reads below
+      const int* desc = desc_all + slot * 16;
+      const int n_tiles = desc[kDTiles];
+      if (n_tiles < 0) break;  // end of work
+      const int* gmeta = gmeta_all + slot * 32;
+      for (int j = 0; j < n_tiles; ++j, ++g) {  // tile j of the item
+        const int st = g % kStages;
+        // ---- K: row t into TMEM K buffer g & 1
+        bool wt = g < 2 || conv_wait(afree_bar(g & 1), ((g >> 1) - 1) & 1);
+        if (wt) wt = conv_wait(full_bar(st), (g / kStages) & 1);
+        if (!wt) {
+          ok = false;
+          break;
+        }
+        {
+          const unsigned char* in = smem + L::kStages0 + st * L::kStageBytes + t * 128;
+          const uint32_t dst = tmem + t_lane + kACol + 64 * (g & 1);
+#pragma unroll
+          for (int hq = p0 / 2; hq < (p0 + kPieces) / 2; ++hq) {  // dims 32 hq .. 32 hq + 31: 16 columns
+            uint32_t wd[16];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int jc = 2 * hq + u;
+              const uint4 x = *reinterpret_cast<const uint4*>(in + ((jc ^ sw) << 4));
+              uint32_t w8[8];
+              widen16<MT>(x, w8);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) wd[8 * u + e] = w8[e];
+            }
+            tmem_st16(dst + 16 * hq, wd);
+          }
+          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(empty_bar(st));      // the 8-bit K half back to its producer
+          mbar_arrive(aconv_bar(g & 1));   // the MMA warp may issue S^T(g)
+        }
+        // ---- V: row t into shared V buffer g & 1
+        wt = g < 2 || conv_wait(vfree_bar(g & 1), ((g >> 1) - 1) & 1);
+        if (wt) wt = conv_wait(vfull_bar(st), (g / kStages) & 1);
+        if (!wt) {
+          ok = false;
+          break;
+        }
+        {
+          const int grp = j * kGroupsPerTile + (PAIR ? (t >> 5) : (t >> 4));
+          const bool zero = (t & 15) >= (gmeta[grp] >> 8);
+          const unsigned char* in = smem + L::kStages0 + st * L::kStageBytes + L::kHalf + t * 128;
+          unsigned char* out = smem + L::kV16 + (g & 1) * 2 * L::kHalf + t * 128;
+#pragma unroll
+          for (int jc = p0; jc < p0 + kPieces; ++jc) {  // elements 16 jc .. 16 jc + 15 of the row
+            const uint4 x = *reinterpret_cast<const uint4*>(in + ((jc ^ sw) << 4));
+            uint32_t wd[8];
+            widen16<MT>(x, wd);
+            if (zero) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) wd[e] = 0u;
+            }
+            const int h = jc >> 2, c = 2 * (jc & 3);  // half, first 16-byte piece of it
+            unsigned char* o = out + h * L::kHalf;
+            *reinterpret_cast<uint4*>(o + ((c ^ sw) << 4)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+            *reinterpret_cast<uint4*>(o + (((c + 1) ^ sw) << 4)) = make_uint4(wd[4], wd[5], wd[6], wd[7]);
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(vempty_bar(st));     // the 8-bit V half back to its producer
+          mbar_arrive(vconv_bar(g & 1));   // the MMA warp may issue O^T(g)
+        }
+      }
+    }
+    if (!ok) *abort_flag = 1;
   } else {
     // =====================================================================
     // compute warps: thread (t, cg) = MMA row t of S^T and row d = t of O^T,
@@ -1022,51 +1182,6 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       bool w = true;
       if (lane == 0) w = mbar_wait_or_abort(bar, parity, a.err, abort_flag);
       return __shfl_sync(0xffffffffu, (int)w, 0) != 0;
-    };
-    // KV8: widen the K (or V) half of the 8-bit tile gt (tile jt of the item
-    // whose group table is gmeta_s) into the 16-bit K buffer (V buffer gt & 1).
-    // Thread t takes row t, warpgroup cg the 16-byte pieces cg, cg + NWG, ...
-    // (both layouts 128B-swizzled: piece c of row t at c ^ (t & 7), so a
-    // warp's accesses spread over every bank); a row that is no token gets a
-    // zero V row.  After K the MMA warp may issue S^T(gt) (conv); each half of
-    // the stage goes back to its producer once widened.  The callers make sure
-    // the buffer is free: K's once S^T(gt - 1) has been read, V's once
-    // O^T(gt - 2) is done.
-    auto widen = [&](int gt, int jt, const int* gmeta_s, bool is_v) {
-      const int st = gt % kStages;
-      const bool w = warp_wait(is_v ? vfull_bar(st) : full_bar(st), (gt / kStages) & 1);
-      if (w) {
-        const bool zero = is_v && (t & 15) >= (gmeta_s[jt * kGroupsPerTile + grp_in_tile] >> 8);
-        const unsigned char* in = smem + L::kStages0 + st * L::kStageBytes + (is_v ? L::kHalf : 0) + t * 128;
-        unsigned char* out = smem + (is_v ? L::kV16 + (gt & 1) * 2 * L::kHalf : L::kK16) + t * 128;
-        const int sw = t & 7;
-#pragma unroll
-        for (int i = 0; i < 8 / W::kNWG; ++i) {
-          const int jc = cg + i * W::kNWG;  // elements 16 jc .. 16 jc + 15 of the row
-          const uint4 x = *reinterpret_cast<const uint4*>(in + ((jc ^ sw) << 4));
-          uint32_t wd[8];
-          widen16<MT>(x, wd);
-          if (zero) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) wd[e] = 0u;
-          }
-          const int h = jc >> 2, c = 2 * (jc & 3);  // half, first 16-byte piece of it
-          unsigned char* o = out + h * L::kHalf;
-          *reinterpret_cast<uint4*>(o + ((c ^ sw) << 4)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-          *reinterpret_cast<uint4*>(o + (((c + 1) ^ sw) << 4)) = make_uint4(wd[4], wd[5], wd[6], wd[7]);
-        }
-      }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncwarp();
-      if (lane == 0) {
-        if (is_v) {
-          mbar_arrive(vempty_bar(st));
-        } else {
-          mbar_arrive(empty_bar(st));
-          mbar_arrive(conv_bar);
-        }
-      }
-      return w;
     };
     // Each warpgroup owns its columns: its rescale decisions, column
     // reductions and the agreement on a failed wait take a named barrier of
@@ -1153,12 +1268,6 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         for (int c = 0; c < NCW; ++c)
           valid[c] = row_ok && (own < 0 || own == m_c[c]) && (!PAIR || e_c[c] == e_row) &&
                      tok < lim_c[c];
-        if constexpr (KV8) {
-          // an item's first tile: its V buffer was O^T(g-2)'s, done when the
-          // item before ended
-          if (j == 0 && ok_w) ok_w = widen(g, 0, gmeta, false);
-          if (j == 0 && ok_w) ok_w = widen(g, 0, gmeta, true);
-        }
         // ---- S^T(g).  Each warp waits on its own; the OR-barrier then makes
         // every compute thread take the same way out if this or an earlier
         // wait of its warp failed.
@@ -1175,11 +1284,6 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         // waited for only where this tile needs it: before O^T is folded and
         // before P(g) is written
         bool pv_done = j == 0;
-        if constexpr (KV8) {
-          // the next tile's K now, so that S^T(g+1) runs during this tile's
-          // softmax (its V after P(g), below)
-          if (j + 1 < n_tiles && ok_w) ok_w = widen(g + 1, j + 1, gmeta, false);
-        }
         bool over = false;
 #pragma unroll
         for (int c = 0; c < NCW; ++c) {
@@ -1295,10 +1399,6 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_ready_bar);  // P(g) written: the MMA warp issues O^T(g)
-        if constexpr (KV8) {
-          // the next tile's V: its buffer was O^T(g-1)'s, waited for above
-          if (j + 1 < n_tiles && ok_w) ok_w = widen(g + 1, j + 1, gmeta, true);
-        }
       }
       if (!ok) break;
 
@@ -1423,7 +1523,7 @@ cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUte
     // number of items is only known on the device
     const int items0 = grouped ? sms : a.num_seqs * (a.num_kv_heads / (PAIR ? 2 : 1));
     const int grid = items0 < sms ? items0 : sms;
-    constexpr int kBlock = Warps<NC>::kThreads;
+    constexpr int kBlock = Warps<NC, KV8>::kThreads;
     cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kBlock), L::kAlloc, stream, a, tk, tv, tq);
     if (e != cudaSuccess) return e;
     ++*launches;

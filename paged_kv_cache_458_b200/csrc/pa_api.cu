@@ -407,8 +407,12 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
                          pa::kSharedPrefixSeqsPerLaunch;
       a.epoch = next_epochs(chunks);
       e = pa::launch_plan(pl, cs, &launched);
+      // own tokens for the tensor cores go into the same launch as the row
+      // lists, after them: no launch of its own for what is often little work
+      a.own_in_lists = own_tc ? 1 : 0;
       if (e == cudaSuccess) e = pa::launch_decode_tc(a, shape->dtype, gk, gv, gq, cs, &launched, false, fp8);
       a.own_pass = 1;
+      a.own_in_lists = 0;
       a.epoch = next_epochs((shape->num_seqs + pa::kSharedPrefixSeqsPerLaunch - 1) / pa::kSharedPrefixSeqsPerLaunch);
       if (!own_tc && e == cudaSuccess) {
         // the CUDA-core kernel (it launches the merge itself)
@@ -423,6 +427,9 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
         count_launches(launched);
         return e == cudaSuccess ? PA_OK : cuda_failed(e);
       }
+      if (e == cudaSuccess) e = pa::launch_decode_merge(a, shape->dtype, shape->head_dim, cs, &launched);
+      count_launches(launched);
+      return e == cudaSuccess ? PA_OK : cuda_failed(e);
     } else {
       a.epoch = next_epochs((shape->num_seqs + pa::kSharedPrefixSeqsPerLaunch - 1) / pa::kSharedPrefixSeqsPerLaunch);
     }

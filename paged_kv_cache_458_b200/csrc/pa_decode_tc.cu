@@ -413,17 +413,23 @@ __host__ __device__ inline int tc_columns(int group, int query_tokens, bool pair
 // pre_f counts the partitions after partition 0); grouped, the leaders of
 // groups of two or more (rows = their list's, the plan's fourth field);
 // own pass, the sequences whose own tokens are in no list (rows = ctx - T,
-// the plan's third field).  -1: no unit.
+// the plan's third field).  -1: no unit.  With both (a list launch that also
+// takes the own tokens) units 0 .. S - 1 are the lists' and S .. 2 S - 1 the
+// own tokens'.
 template <int PPL>
-__device__ __forceinline__ void unit_prefix(const DecodeArgs& a, bool grouped, bool p0_first, int PT,
-                                            int lane, int (&pre_f)[PPL], int (&pre_p)[PPL],
+__device__ __forceinline__ void unit_prefix(const DecodeArgs& a, bool grouped, bool both, bool p0_first,
+                                            int PT, int lane, int (&pre_f)[PPL], int (&pre_p)[PPL],
                                             int& carry_f, int& carry_p) {
-  const int S = a.num_seqs;
+  const int S = both ? 2 * a.num_seqs : a.num_seqs;  // units
   int rows_k[PPL];
 #pragma unroll
   for (int k = 0; k < PPL; ++k) {
-    const int sc = min(k * 32 + lane, S - 1);
-    rows_k[k] = grouped ? __ldg(&a.plan2[sc].w) : a.plan ? __ldg(&a.plan2[sc].z) : __ldg(a.context_lens + sc);
+    const int u = min(k * 32 + lane, S - 1);
+    const bool own = both && u >= a.num_seqs;
+    const int sc = own ? u - a.num_seqs : u;
+    rows_k[k] = grouped && !own ? __ldg(&a.plan2[sc].w)
+                : a.plan        ? __ldg(&a.plan2[sc].z)
+                                : __ldg(a.context_lens + sc);
   }
 #pragma unroll
   for (int k = 0; k < PPL; ++k) {
@@ -487,7 +493,8 @@ __device__ __forceinline__ void widen16(const uint4 x, uint32_t (&w)[8]) {
     }
 }
 
-template <typename T, int NC, bool PAIR, bool KV8>
+// WIDE: a row-list launch that also takes the own-token items (2 x 256 units).
+template <typename T, int NC, bool PAIR, bool KV8, bool WIDE>
 __global__ void __launch_bounds__(Warps<NC, KV8>::kThreads, 1)
 decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q) {
@@ -650,11 +657,14 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
     // own tokens read on their own) only some sequences are units: full
     // partitions first, then the last ones, counted before the first item
     const bool p0_first = a.plan == nullptr;
+    // a list launch that also takes the own tokens read on their own: units
+    // S .. 2 S - 1 are those sequences' own tokens, as per-sequence items
+    const bool both = WIDE && grouped && a.own_in_lists != 0;
     const int Hu = Hkv / kHeads;  // kv units of the item numbering
-    constexpr int PPL = kMaxUnits / 32 + 1;  // prefix[0..S] over the lanes
+    constexpr int PPL = (WIDE ? 2 : 1) * kMaxUnits / 32 + 1;  // prefix[0..units] over the lanes
     int pre_f[PPL], pre_p[PPL];
     int carry_f = 0, carry_p = 0;
-    if (!p0_first) unit_prefix(a, grouped, p0_first, PT, lane, pre_f, pre_p, carry_f, carry_p);
+    if (!p0_first) unit_prefix(a, grouped, both, p0_first, PT, lane, pre_f, pre_p, carry_f, carry_p);
     // items known so far (without a plan, the partition-0 items until the
     // prefix is in)
     int total = p0_first ? S * Hu : Hu * (carry_f + carry_p);
@@ -693,11 +703,16 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       } else {
         locate(f, Hu, carry_f, pre_f, pre_p, s, kvu, part);
       }
+      bool g_item = grouped;  // this item reads a group's row list
+      if (both && s >= S) {
+        s -= S;
+        g_item = false;
+      }
       const int kvh = kvu * kHeads;  // the item's first kv head
       // query rows: one TMA box per 64-element half, [members][heads][64]
       const uint32_t rb = ready_bar(slot);
       if (lane == 0) {
-        const int qrow = grouped ? a.seq_offset + s : (a.seq_offset + s) * Tq;
+        const int qrow = g_item || grouped ? a.seq_offset + s : (a.seq_offset + s) * Tq;
         mbar_expect_tx(rb, 2 * q_rows * 128);  // the phase also needs the arrival below
         tma_load_3d(sm_q + slot * L::kQBytes, &tm_q, rb, 0, kvh * G, qrow);
         tma_load_3d(sm_q + slot * L::kQBytes + N * 128, &tm_q, rb, 64, kvh * G, qrow);
@@ -720,7 +735,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         if (a.half_boxes && r0 + kGroupRows / 2 < a.max_context_len)
           spec_blk2 = __ldg(stable + (r0 + kGroupRows / 2) / a.block_size);
       }
-      if (grouped) {
+      if (g_item) {
         // the group's plan and every member's record and context in one round
         // trip (lanes past the group read a neighbour, unused)
         const int sl = min(s + lane, S - 1);
@@ -779,7 +794,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       // own rows: the member whose run holds r0 (runs are in member order,
       // offsets non-decreasing; an empty run holds nothing): a binary search
       int own = 0;
-      if (grouped) {
+      if (g_item) {
 #pragma unroll
         for (int step = 16; step >= 1; step >>= 1) {
           const int cand = own + step;
@@ -843,7 +858,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
       }
       if (p0_first && it == 0) {
         // the counts of the further partitions, while this item's tiles load
-        unit_prefix(a, grouped, p0_first, PT, lane, pre_f, pre_p, carry_f, carry_p);
+        unit_prefix(a, grouped, both, p0_first, PT, lane, pre_f, pre_p, carry_f, carry_p);
         total = Hu * carry_f + S * Hu;
       }
       // the next item: a launch with no more items than CTAs takes none
@@ -1450,7 +1465,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tm_k,
         if (code == kZero) {
           a.out[qh * kD + d] = 0;
         } else if (code == kDirect) {
-          a.out[qh * kD + d] = Elem<T>::from_f(o / sum_c[c]);
+          a.out[qh * kD + d] = Elem<T>::from_f(__fdividef(o, sum_c[c]));
         } else {
           const size_t wslot = qh * a.num_parts + code;
           a.ws_acc[wslot * kD + d] = o;
@@ -1486,11 +1501,11 @@ int sm_count() {
   return count[dev];
 }
 
-template <typename T, int NC, bool PAIR, bool KV8>
+template <typename T, int NC, bool PAIR, bool KV8, bool WIDE = false>
 cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& tq, cudaStream_t stream, int* launches) {
   using L = Layout<(NC <= 16 ? 16 : 32), KV8>;
-  auto* kern = decode_tc_kernel<T, NC, PAIR, KV8>;
+  auto* kern = decode_tc_kernel<T, NC, PAIR, KV8, WIDE>;
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
@@ -1500,7 +1515,7 @@ cudaError_t launch_typed(const DecodeArgs& a0, const CUtensorMap& tk, const CUte
   const int sms = sm_count();
   const bool grouped = a0.plan != nullptr && !a0.own_pass;
   // groups never cross a multiple of the shared-prefix window
-  const int chunk = kMaxUnits;
+  const int chunk = kSharedPrefixSeqsPerLaunch;
   const int Tq = a0.query_tokens;
   for (int s0 = 0; s0 < a0.num_seqs; s0 += chunk) {
     DecodeArgs a = a0;
@@ -1543,7 +1558,10 @@ cudaError_t launch_cols(const DecodeArgs& a, int nc, const CUtensorMap& tk, cons
     case 8: return launch_typed<T, 8, PAIR, KV8>(a, tk, tv, tq, st, n);
     case 16: return launch_typed<T, 16, PAIR, KV8>(a, tk, tv, tq, st, n);
     case 32:  // two-head items take at most 16 columns
-      if constexpr (!PAIR) return launch_typed<T, 32, false, KV8>(a, tk, tv, tq, st, n);
+      if constexpr (!PAIR) {
+        if (a.own_in_lists) return launch_typed<T, 32, false, KV8, true>(a, tk, tv, tq, st, n);
+        return launch_typed<T, 32, false, KV8>(a, tk, tv, tq, st, n);
+      }
       break;
   }
   return cudaErrorInvalidValue;

@@ -43,6 +43,8 @@ struct DecodeArgs {
   int group;                     // g = Hq / Hkv
   int own_pass;                  // with a plan: 1 = items over the own tokens [T, ctx) of the
                                  // sequences whose own tokens are in no row list
+  int own_in_lists;              // with a plan and own_pass 0: the row-list launch also takes
+                                 // those own-token items (after the lists' items)
   int half_boxes;                // block_size is a multiple of 8 but not of 16: each
                                  // 16-token TMA box is loaded as two 8-token boxes, which
                                  // may come from two blocks

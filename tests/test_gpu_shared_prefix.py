@@ -257,12 +257,15 @@ def test_shared_prefix_bad_block_ids_reported():
     assert status == pa.PA_ERR_DEVICE_CHECK and bits & 0x1
 
 
-def test_shared_prefix_launches():
-    """plan + the row lists of the groups + the own tokens read on their own
-    (here none) + merge."""
+@pytest.mark.parametrize("group,launches", [(8, 3), (1, 4)])
+def test_shared_prefix_launches(group, launches):
+    """plan + the row lists of the groups + merge; where the own tokens read
+    on their own go to the tensor cores (group 8) they are items of the list
+    launch, else (group 1) the CUDA-core kernel reads them in a launch of its
+    own."""
     rng = np.random.default_rng(9600)
-    c = gen.grouped_decode_case(rng, groups=[(300, [310, 320])], num_q_heads=8, num_kv_heads=1,
-                                head_dim=128, block_size=16, dtype=gen.BF16)
+    c = gen.grouped_decode_case(rng, groups=[(300, [310, 320]), (0, [45])], num_q_heads=group,
+                                num_kv_heads=1, head_dim=128, block_size=16, dtype=gen.BF16)
     before = pa.pa_kernel_launches()
-    run_shared(c, gen.BF16)
-    assert pa.pa_kernel_launches() - before == 4
+    out, _ = run_shared(c, gen.BF16)
+    assert pa.pa_kernel_launches() - before == launches

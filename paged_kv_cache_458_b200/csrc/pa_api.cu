@@ -136,6 +136,33 @@ constexpr long long kCounterBytes = 256;
 
 long long round256(long long x) { return (x + 255) / 256 * 256; }
 
+// A second stream per device, and two events, for the shared-prefix decode
+// whose own tokens go to the CUDA-core kernel: that kernel runs beside the
+// row-list launch, which often leaves most SMs idle.  Created on first use;
+// the fork and join are enqueued under a lock, so that calls from several
+// host threads never wait on each other's event records.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t forked = nullptr, done = nullptr;
+};
+std::mutex g_side_lock;
+SideStream g_side[64];
+
+bool side_stream(int dev, SideStream* out) {
+  if (dev < 0 || dev >= 64) return false;
+  SideStream& s = g_side[dev];
+  if (!s.stream) {
+    SideStream n;
+    if (cudaEventCreateWithFlags(&n.forked, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&n.done, cudaEventDisableTiming) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&n.stream, cudaStreamNonBlocking) != cudaSuccess)
+      return false;
+    s = n;
+  }
+  *out = s;
+  return true;
+}
+
 int num_partitions(const pa_shape* s, int32_t max_context_len);
 
 long long plan_bytes(const pa_shape* s) {
@@ -407,25 +434,38 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
                          pa::kSharedPrefixSeqsPerLaunch;
       a.epoch = next_epochs(chunks);
       e = pa::launch_plan(pl, cs, &launched);
-      // own tokens for the tensor cores go into the same launch as the row
-      // lists, after them: no launch of its own for what is often little work
-      a.own_in_lists = own_tc ? 1 : 0;
-      if (e == cudaSuccess) e = pa::launch_decode_tc(a, shape->dtype, gk, gv, gq, cs, &launched, false, fp8);
-      a.own_pass = 1;
-      a.own_in_lists = 0;
-      a.epoch = next_epochs((shape->num_seqs + pa::kSharedPrefixSeqsPerLaunch - 1) / pa::kSharedPrefixSeqsPerLaunch);
-      if (!own_tc && e == cudaSuccess) {
-        // the CUDA-core kernel (it launches the merge itself)
+      if (own_tc) {
+        // own tokens for the tensor cores go into the same launch as the
+        // row lists, after them: no launch of their own for what is often
+        // little work
+        a.own_in_lists = 1;
+        if (e == cudaSuccess) e = pa::launch_decode_tc(a, shape->dtype, gk, gv, gq, cs, &launched, false, fp8);
+        a.own_in_lists = 0;
+      } else if (e == cudaSuccess) {
+        // own tokens on the CUDA-core kernel, on a second stream forked after
+        // the plan, beside the row-list launch; both join before the merge
         CUtensorMap pk, pv;
         if (!make_pool_map(&pk, k_cache, shape, box_rows(shape)) ||
             !make_pool_map(&pv, v_cache, shape, box_rows(shape)))
           return cuda_failed("cuTensorMapEncodeTiled failed");
-        a.own_tokens = pa::decode_max_partition_tokens();
-        a.grid_parts = (max_context_len + a.own_tokens - 1) / a.own_tokens;
-        if (a.grid_parts < 1) a.grid_parts = 1;
-        e = pa::launch_decode(a, shape->dtype, shape->head_dim, group, pk, pv, cs, &launched, fp8);
-        count_launches(launched);
-        return e == cudaSuccess ? PA_OK : cuda_failed(e);
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return cuda_failed("cudaGetDevice failed");
+        std::lock_guard<std::mutex> lock(g_side_lock);
+        SideStream side;
+        if (!side_stream(dev, &side)) return cuda_failed("creating the second stream failed");
+        pa::DecodeArgs own = a;
+        own.own_pass = 1;
+        own.own_tokens = pa::decode_max_partition_tokens();
+        own.grid_parts = (max_context_len + own.own_tokens - 1) / own.own_tokens;
+        if (own.grid_parts < 1) own.grid_parts = 1;
+        e = cudaEventRecord(side.forked, cs);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(side.stream, side.forked, 0);
+        if (e == cudaSuccess)
+          e = pa::launch_decode(own, shape->dtype, shape->head_dim, group, pk, pv, side.stream, &launched, fp8,
+                                false);
+        if (e == cudaSuccess) e = cudaEventRecord(side.done, side.stream);
+        if (e == cudaSuccess) e = pa::launch_decode_tc(a, shape->dtype, gk, gv, gq, cs, &launched, false, fp8);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, side.done, 0);
       }
       if (e == cudaSuccess) e = pa::launch_decode_merge(a, shape->dtype, shape->head_dim, cs, &launched);
       count_launches(launched);

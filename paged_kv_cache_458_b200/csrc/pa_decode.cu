@@ -532,7 +532,7 @@ cudaError_t launch_typed(const DecodeArgs& a, const CUtensorMap& tk, const CUten
   cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kWarps * 32), L::kTotal, stream, a, tk, tv);
   if (e != cudaSuccess) return e;
   ++*launches;
-  if (a.num_parts <= 1) return cudaSuccess;
+  if (a.num_parts <= 1 || a.skip_merge) return cudaSuccess;
   const int pairs = a.num_seqs * a.query_tokens * a.num_q_heads;
   e = launch_pdl(decode_merge_kernel<T, D>, dim3(merge_grid(pairs)), dim3(128), 0, stream, a);
   if (e == cudaSuccess) ++*launches;
@@ -561,13 +561,15 @@ cudaError_t launch_dims(const DecodeArgs& a, int head_dim, int group, const CUte
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeArgs& a, int dtype, int head_dim, int group,
+cudaError_t launch_decode(const DecodeArgs& a0, int dtype, int head_dim, int group,
                           const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t stream,
-                          int* launches, bool fp8_cache) {
-  const long long grid = (long long)a.grid_parts * a.num_seqs * a.num_kv_heads;
+                          int* launches, bool fp8_cache, bool with_merge) {
+  const long long grid = (long long)a0.grid_parts * a0.num_seqs * a0.num_kv_heads;
   if (grid <= 0) return cudaSuccess;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const int g = (int)grid;
+  DecodeArgs a = a0;
+  if (!with_merge) a.skip_merge = 1;
   if (dtype == 0)
     return fp8_cache ? launch_dims<__half, Fp8E4M3>(a, head_dim, group, tk, tv, g, stream, launches)
                      : launch_dims<__half, __half>(a, head_dim, group, tk, tv, g, stream, launches);

@@ -45,6 +45,7 @@ struct DecodeArgs {
                                  // sequences whose own tokens are in no row list
   int own_in_lists;              // with a plan and own_pass 0: the row-list launch also takes
                                  // those own-token items (after the lists' items)
+  int skip_merge;                // host side: 1 = the CUDA-core launch leaves the merge to its caller
   int half_boxes;                // block_size is a multiple of 8 but not of 16: each
                                  // 16-token TMA box is loaded as two 8-token boxes, which
                                  // may come from two blocks
@@ -77,12 +78,12 @@ cudaError_t launch_expand_queries(const int32_t* tables, const int32_t* ctx, int
                                   unsigned int* err, cudaStream_t stream, int* launches);
 
 
-// Launch the partition kernel (+ the merge kernel when num_parts > 1).
-// `launches` is incremented once per kernel launched.  fp8_cache: K/V hold
-// E4M3 codes (a.k_scale / a.v_scale set).
+// Launch the partition kernel (+ the merge kernel when num_parts > 1 and
+// with_merge).  `launches` is incremented once per kernel launched.
+// fp8_cache: K/V hold E4M3 codes (a.k_scale / a.v_scale set).
 cudaError_t launch_decode(const DecodeArgs& a, int dtype, int head_dim, int group,
                           const CUtensorMap& tm_k, const CUtensorMap& tm_v, cudaStream_t stream,
-                          int* launches, bool fp8_cache = false);
+                          int* launches, bool fp8_cache = false, bool with_merge = true);
 int decode_chunk_tokens();
 int decode_max_partition_tokens();
 // The split-K merge alone (after a partition kernel that wrote partials).

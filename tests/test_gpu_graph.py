@@ -3,7 +3,9 @@
 The tensor-core kernels take their items from a counter in the workspace,
 tagged with a per-call epoch that a graph fixes at capture; a captured call
 must still cover every item on every replay.  The output is NaN-filled before
-each replay, so a skipped item shows up.
+each replay, so a skipped item shows up.  With shared prefixes at group 1 the
+call forks the own-token pass onto a second stream and joins it again; the
+capture takes both branches.
 """
 import numpy as np
 import pytest
@@ -32,8 +34,10 @@ def _cuda():
 CTX = [5, 300, 1100, 2050, 700, 129, 1, 513]
 
 
-@pytest.mark.parametrize("variant,shared,group", [(1, 0, 4), (2, 0, 4), (2, 0, 8), (2, 0, 16), (0, 1, 8)],
-                         ids=["cuda_cores", "tc_pairs_g4", "tc_pairs_g8", "tc_g16", "shared_prefix"])
+@pytest.mark.parametrize("variant,shared,group",
+                         [(1, 0, 4), (2, 0, 4), (2, 0, 8), (2, 0, 16), (0, 1, 8), (0, 1, 1)],
+                         ids=["cuda_cores", "tc_pairs_g4", "tc_pairs_g8", "tc_g16", "shared_prefix",
+                              "shared_prefix_second_stream"])
 def test_decode_graph_replays(orc, variant, shared, group):
     rng = np.random.default_rng(1700 + 10 * variant + shared + group)
     Hkv, dtype = 2, gen.BF16

@@ -51,96 +51,99 @@ namespace {
 
 constexpr int kPlanThreads = 128;
 
-__device__ __forceinline__ int clamp_ctx(const PlanArgs& p, int s) {
-  const int c = __ldg(p.context_lens + s);
-  return max(0, min(c, p.max_context_len));
-}
-
-// First table entry of s, or -1 when s cannot share (empty context, or an
-// entry outside the pool: the decode reports those itself).
-__device__ __forceinline__ int first_block(const PlanArgs& p, int s) {
-  if (clamp_ctx(p, s) <= 0) return -1;
-  const int b = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq);
-  return (b >= 0 && b < p.num_blocks) ? b : -1;
-}
-
 // One CTA per sequence.  The tables and lengths are inputs no kernel of this
 // library writes (except the query expansion of pa_decode_multi, after which
 // inputs_written_before is set): the search runs before waiting for the
 // kernel before this one, overlapping it, and only the plan's writes wait
 // (the decode and merge of an earlier call may still be reading the plan
-// until then).
+// until then).  The search takes two rounds of independent loads: every
+// sequence's context and first table entry in the chunk (the runs are found
+// in shared memory), then the table entries the group's members compare.
+constexpr int kPlanMaxChunk = 256;  // sequences of a chunk (groups never cross one)
+constexpr int kPlanPer = kPlanMaxChunk / kPlanThreads;
+
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p) {
   if (p.inputs_written_before) pdl_wait();
   pdl_launch_dependents();
-  __shared__ int sh_edge, sh_min_ctx, sh_min_blocks, sh_common;
+  __shared__ int sh_ctx[kPlanMaxChunk], sh_first[kPlanMaxChunk];
+  __shared__ int sh_lo, sh_hi, sh_common;
   __shared__ int sh_rows[32];  // own rows of each member, rounded up to 16
   const int s = blockIdx.x, tid = threadIdx.x;
-  const int first = first_block(p, s);
+  const int c0 = (s / p.chunk) * p.chunk;
+  const int c1 = min(p.num_seqs, c0 + p.chunk);
+  const int i_s = s - c0;  // s within the chunk
+  // ---- every sequence's context and first entry (-1: it cannot share: an
+  // empty context, or an entry outside the pool, which the decode reports)
+  {
+    int c[kPlanPer], b[kPlanPer];
+#pragma unroll
+    for (int k = 0; k < kPlanPer; ++k) {
+      const int q = min(c0 + tid + k * kPlanThreads, c1 - 1);
+      c[k] = __ldg(p.context_lens + q);
+      // (a batch with no table entries has only empty contexts: nothing to read)
+      b[k] = p.max_blocks_per_seq > 0 ? __ldg(p.block_tables + (size_t)q * p.max_blocks_per_seq) : -1;
+    }
+#pragma unroll
+    for (int k = 0; k < kPlanPer; ++k) {
+      const int i = tid + k * kPlanThreads;
+      if (c0 + i < c1) {
+        const int cc = max(0, min(c[k], p.max_context_len));
+        sh_ctx[i] = cc;
+        sh_first[i] = (cc > 0 && b[k] >= 0 && b[k] < p.num_blocks) ? b[k] : -1;
+      }
+    }
+    if (tid == 0) sh_lo = -1, sh_hi = c1 - c0, sh_common = INT_MAX;
+  }
+  __syncthreads();
+  const int first = sh_first[i_s];
   int leader = s, n = 1, shared = 0;
   if (first >= 0) {
-    const int c0 = (s / p.chunk) * p.chunk;
-    const int c1 = min(p.num_seqs, c0 + p.chunk);
-    // ---- run start: the sequence after the nearest break below s
-    int a = c0;
-    for (int base = s - 1; base >= c0; base -= kPlanThreads) {
-      if (tid == 0) sh_edge = -1;
-      __syncthreads();
-      const int sp = base - tid;
-      if (sp >= c0 && first_block(p, sp) != first) atomicMax(&sh_edge, sp);
-      __syncthreads();
-      const int e = sh_edge;
-      __syncthreads();
-      if (e >= 0) { a = e + 1; break; }
+    // ---- the run: the nearest breaks below and above s
+#pragma unroll
+    for (int k = 0; k < kPlanPer; ++k) {
+      const int i = tid + k * kPlanThreads;
+      if (c0 + i < c1 && sh_first[i] != first) {
+        if (i < i_s) atomicMax(&sh_lo, i);
+        if (i > i_s) atomicMin(&sh_hi, i);
+      }
     }
-    // ---- run end (exclusive): the nearest break above s
-    int b = c1;
-    for (int base = s + 1; base < c1; base += kPlanThreads) {
-      if (tid == 0) sh_edge = INT_MAX;
-      __syncthreads();
-      const int sp = base + tid;
-      if (sp < c1 && first_block(p, sp) != first) atomicMin(&sh_edge, sp);
-      __syncthreads();
-      const int e = sh_edge;
-      __syncthreads();
-      if (e != INT_MAX) { b = e; break; }
-    }
-    const int lead = a + ((s - a) / p.max_members) * p.max_members;
+    __syncthreads();
+    const int a = sh_lo + 1, b = sh_hi;  // the run [a, b) within the chunk
+    const int lead = a + ((i_s - a) / p.max_members) * p.max_members;
     const int nm = min(p.max_members, b - lead);
     if (nm >= 2) {
       // ---- shortest member context and block count
-      if (tid == 0) sh_min_ctx = INT_MAX, sh_min_blocks = INT_MAX;
-      __syncthreads();
-      if (tid < nm) {
-        const int c = clamp_ctx(p, lead + tid);
-        atomicMin(&sh_min_ctx, c);
-        atomicMin(&sh_min_blocks, (c + p.block_size - 1) / p.block_size);
+      int min_ctx = INT_MAX;
+      for (int m = 0; m < nm; ++m) min_ctx = min(min_ctx, sh_ctx[lead + m]);
+      const int lim = (min_ctx + p.block_size - 1) / p.block_size;
+      // ---- leading table entries every member has in common with the
+      // leader: the first entry below lim where some member differs
+      const int32_t* lead_row = p.block_tables + (size_t)(c0 + lead) * p.max_blocks_per_seq;
+      const int pairs = (nm - 1) * lim;
+      for (int x0 = 0; x0 < pairs; x0 += 4 * kPlanThreads) {
+        int mine[4], theirs[4], jj[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int x = min(x0 + u * kPlanThreads + tid, pairs - 1);
+          const int m = 1 + x / lim, j = x % lim;
+          jj[u] = x0 + u * kPlanThreads + tid < pairs ? j : INT_MAX;
+          mine[u] = __ldg(p.block_tables + (size_t)(c0 + lead + m) * p.max_blocks_per_seq + j);
+          theirs[u] = __ldg(lead_row + j);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (jj[u] != INT_MAX && mine[u] != theirs[u]) atomicMin(&sh_common, jj[u]);
       }
       __syncthreads();
-      if (tid == 0) sh_common = sh_min_blocks;
-      __syncthreads();
-      // ---- leading table entries every member has in common with the leader:
-      // each round compares J entries of every other member at once
-      const int32_t* lead_row = p.block_tables + (size_t)lead * p.max_blocks_per_seq;
-      const int J = max(1, kPlanThreads / (nm - 1));
-      const int m = 1 + tid / J;
-      const int32_t* row = p.block_tables + (size_t)(lead + min(m, nm - 1)) * p.max_blocks_per_seq;
-      for (int j0 = 0;; j0 += J) {
-        const int lim = sh_common;  // the same in every thread: read between barriers
-        __syncthreads();
-        if (j0 >= lim) break;
-        const int j = j0 + tid % J;
-        if (m < nm && j < lim && __ldg(row + j) != __ldg(lead_row + j)) atomicMin(&sh_common, j);
-        __syncthreads();
-      }
-      const long long t = min((long long)sh_common * p.block_size, (long long)sh_min_ctx);
+      const int common = min(sh_common, lim);
+      const long long t = min((long long)common * p.block_size, (long long)min_ctx);
       const int sh = (int)(t & ~15LL);
-      if (sh >= p.min_shared) leader = lead, n = nm, shared = sh;
+      if (sh >= p.min_shared) leader = c0 + lead, n = nm, shared = sh;
     }
   }
   // ---- this sequence's place in its group's row list
   if (tid < n) {
-    const int own = clamp_ctx(p, leader + tid) - shared;
+    const int own = sh_ctx[leader - c0 + tid] - shared;
     sh_rows[tid] = (own + 15) / 16 * 16;
   }
   __syncthreads();
@@ -154,7 +157,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p) {
     const bool fold = n >= 2 && off - shared <= max(shared, 64 * n);
     const int rows = fold ? off : shared;
     const int p_shared = (shared + PT - 1) / PT;
-    const int own = clamp_ctx(p, s) - shared;
+    const int own = sh_ctx[i_s] - shared;
     int n_slots = p_shared;
     if (own > 0) {
       if (fold) {
@@ -175,6 +178,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p) {
 
 cudaError_t launch_plan(const PlanArgs& p, cudaStream_t stream, int* launches) {
   if (p.num_seqs <= 0) return cudaSuccess;
+  if (p.chunk <= 0 || p.chunk > kPlanMaxChunk || p.max_members > 32) return cudaErrorInvalidValue;
   cudaError_t e = launch_pdl(plan_kernel, dim3(p.num_seqs), dim3(kPlanThreads), 0, stream, p);
   if (e == cudaSuccess) ++*launches;
   return e;

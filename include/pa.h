@@ -17,7 +17,13 @@
  *    nothing per call and keeps no pointer after the call returns.
  *  - All device work is enqueued asynchronously on `stream` (a cudaStream_t;
  *    NULL is the legacy default stream).  No call reads device memory on the
- *    host or synchronises, except pa_last_device_error().
+ *    host or synchronises, except pa_last_device_error().  One call forks:
+ *    a shared-prefix decode whose own tokens go to the CUDA-core kernel (see
+ *    pa_decode) enqueues that pass on a second stream of the library's (one
+ *    per device, created on first use), ordered after the call's earlier
+ *    work on `stream` by an event, and makes `stream` wait for it before the
+ *    merge: every kernel of the call is still ordered before `stream`'s next
+ *    work.
  *  - Shapes and host-side arguments are validated before anything is
  *    launched; a refusal returns PA_ERR_INVALID_ARG or PA_ERR_UNSUPPORTED and
  *    launches nothing.  A failed launch returns PA_ERR_CUDA.
@@ -197,7 +203,12 @@ size_t pa_decode_workspace_bytes(const pa_shape *shape, int32_t max_context_len)
  * rows (a member's columns see the shared rows and its own), and the merge
  * kernel combines a member's partitions (log-sum-exp rule).  The result is
  * the same attention, up to fp32 rounding order; only the order in which the
- * sums are formed differs.
+ * sums are formed differs.  Own tokens not in a list (a long private
+ * continuation, or a sequence in no group) are read per sequence: at group
+ * sizes where the plain decode runs on the tensor cores, as further items of
+ * the same launch as the lists; else on the CUDA-core kernel, on the
+ * library's second stream (see the conventions above), beside the lists'
+ * launch.
  *
  * q, k_cache, v_cache, block_tables, context_lens, out: device, layouts above.
  * max_context_len: host-side upper bound on every context_lens[s]; it sizes the

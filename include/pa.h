@@ -23,7 +23,9 @@
  *    per device, created on first use), ordered after the call's earlier
  *    work on `stream` by an event, and makes `stream` wait for it before the
  *    merge: every kernel of the call is still ordered before `stream`'s next
- *    work.
+ *    work.  Make the first such call on a device before any stream capture
+ *    on it (creating a stream is not allowed inside a capture); after a
+ *    context reset the stream and events are made again.
  *  - Shapes and host-side arguments are validated before anything is
  *    launched; a refusal returns PA_ERR_INVALID_ARG or PA_ERR_UNSUPPORTED and
  *    launches nothing.  A failed launch returns PA_ERR_CUDA.

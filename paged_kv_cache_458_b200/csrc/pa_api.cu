@@ -459,6 +459,13 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
         own.grid_parts = (max_context_len + own.own_tokens - 1) / own.own_tokens;
         if (own.grid_parts < 1) own.grid_parts = 1;
         e = cudaEventRecord(side.forked, cs);
+        if (e == cudaErrorInvalidResourceHandle) {
+          // a context reset since the stream and events were made: make them again
+          (void)cudaGetLastError();
+          g_side[dev] = SideStream{};
+          if (!side_stream(dev, &side)) return cuda_failed("creating the second stream failed");
+          e = cudaEventRecord(side.forked, cs);
+        }
         if (e == cudaSuccess) e = cudaStreamWaitEvent(side.stream, side.forked, 0);
         if (e == cudaSuccess)
           e = pa::launch_decode(own, shape->dtype, shape->head_dim, group, pk, pv, side.stream, &launched, fp8,

@@ -57,13 +57,17 @@
 // one by number, then from a counter in the workspace whose value carries the
 // call's epoch), resolves each 16-row group through its block table and fills
 // one of two item slots (descriptor, pool rows, group and member tables, and
-// the query rows by one TMA box), up to two items ahead; a producer warp
-// issues the tiles' tiled TMA loads, one box per lane (per tile: 8 groups of
-// one head or 4 groups of two heads, x {K, V} x two 64-element halves,
-// 128B-swizzled), into one of three stages; a dedicated MMA warp issues every
-// MMA and commits it to an mbarrier; the compute warps consume tiles in order
-// and tell it through two more mbarriers when S^T(g) has been read and when
-// P(g) has been written.  Without a plan, items are numbered partition 0 of
+// the query rows by one TMA box), up to two items ahead; two producer warps
+// issue the tiles' tiled TMA loads, one the K half and one the V half of each
+// stage, one box per lane (per tile and half: 8 groups of one head or 4 groups
+// of two heads, x two 64-element halves, 128B-swizzled), into one of three
+// stages whose halves are freed apart (K once S^T is computed, V once O^T
+// is); a dedicated MMA warp issues every MMA and commits it to an mbarrier;
+// the compute warps consume tiles in order and tell it through two more
+// mbarriers when S^T(g) has been read and when P(g) has been written.  With
+// an E4M3 cache, converter warps widen K into TMEM and V into shared memory
+// (see Layout).  A launch over shared-prefix row lists may also take the
+// per-sequence items of the own tokens no list holds (WIDE).  Without a plan, items are numbered partition 0 of
 // every sequence first, then each sequence's further partitions (measured 2 %
 // faster on mistral_7b_gqa than full partitions first and the shorter last
 // ones after them); with one (only some sequences are units), full partitions

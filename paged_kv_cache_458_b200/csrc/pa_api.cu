@@ -467,12 +467,18 @@ pa_status decode_impl(const void* q, const void* k_cache, const void* v_cache,
           e = cudaEventRecord(side.forked, cs);
         }
         if (e == cudaSuccess) e = cudaStreamWaitEvent(side.stream, side.forked, 0);
+        const bool forked = e == cudaSuccess;
         if (e == cudaSuccess)
           e = pa::launch_decode(own, shape->dtype, shape->head_dim, group, pk, pv, side.stream, &launched, fp8,
                                 false);
-        if (e == cudaSuccess) e = cudaEventRecord(side.done, side.stream);
         if (e == cudaSuccess) e = pa::launch_decode_tc(a, shape->dtype, gk, gv, gq, cs, &launched, false, fp8);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, side.done, 0);
+        if (forked) {
+          // join whatever went onto the second stream, even after a failed
+          // launch (a stream capture must not end with it unjoined)
+          cudaError_t j = cudaEventRecord(side.done, side.stream);
+          if (j == cudaSuccess) j = cudaStreamWaitEvent(cs, side.done, 0);
+          if (e == cudaSuccess) e = j;
+        }
       }
       if (e == cudaSuccess) e = pa::launch_decode_merge(a, shape->dtype, shape->head_dim, cs, &launched);
       count_launches(launched);

@@ -269,3 +269,29 @@ def test_shared_prefix_launches(group, launches):
     before = pa.pa_kernel_launches()
     out, _ = run_shared(c, gen.BF16)
     assert pa.pa_kernel_launches() - before == launches
+
+
+@pytest.mark.parametrize("group", [1, 8])
+def test_shared_prefix_tables_without_entries(group):
+    """A batch of empty contexts whose tables hold no entries at all
+    (max_blocks_per_seq = 0; the table pointer is valid but names nothing):
+    the plan reads no table entry, every output row is zero, and no device
+    check fires."""
+    rng = np.random.default_rng(9700 + group)
+    S, Hkv, D, bs, NB = 5, 1, 128, 16, 4
+    dtype = gen.BF16
+    q = gen.normal_bits(rng, (S, Hkv * group, D), dtype)
+    k = gen.normal_bits(rng, (NB, bs, Hkv, D), dtype)
+    v = gen.normal_bits(rng, (NB, bs, Hkv, D), dtype)
+    shape = pa.make_shape(num_seqs=S, num_q_heads=Hkv * group, num_kv_heads=Hkv, head_dim=D,
+                          block_size=bs, num_blocks=NB, max_blocks_per_seq=0, dtype=dtype,
+                          shared_prefix=1)
+    wsb = pa.pa_decode_workspace_bytes(shape, 0)
+    ws = torch.randint(0, 256, (max(16, wsb),), dtype=torch.uint8, device="cuda")
+    out = torch.full(q.shape, float("nan"), dtype=pa.torch_dtype(dtype), device="cuda")
+    no_entries = dev_i32(np.zeros(4, dtype=np.int32))  # a valid pointer, nothing in it is read
+    pa.pa_decode(dev(q, dtype), dev(k, dtype), dev(v, dtype), no_entries,
+                 dev_i32(np.zeros(S, dtype=np.int32)), 0.088, out, shape, 0, ws, wsb)
+    status, bits = pa.pa_last_device_error()
+    assert status == pa.PA_OK, f"device check fired: {bits:#x}"
+    assert np.all(host_bits(out) == 0)

@@ -587,16 +587,10 @@ def run_ours(args, rank, world, local, dist):
         "dtype": "e4m3" if fp8 else gen.DTYPE_NAMES[case.dtype], "accum_dtype": "f32",
         "data": "synthetic (seeded N(0,1) values, shapes and block structure of the workload)",
         "config": {
-            "workload": f"{args.workload}: {case.workload.description}",
-            "num_seqs": case.num_seqs, "num_q_heads": case.num_q_heads,
-            "num_kv_heads": case.num_kv_heads, "head_dim": case.head_dim,
-            "block_size": case.block_size, "storage_dtype": gen.DTYPE_NAMES[case.dtype],
+            **workload_config(args, case, world, fp8),
             "partition_tokens": pa.pa_decode_partition_tokens(w.shape),
             "decode_variant": f"{args.variant} -> {resolved}",
             "shared_prefix": bool(shared),
-            "query_tokens": args.query_tokens,
-            "kv_cache": "e4m3 codes + per-kv-head fp32 scales" if fp8 else gen.DTYPE_NAMES[case.dtype],
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "steps_cycle": n_cycle,
             "l2": (f"inputs larger than L2: {kv_step0 / 1e6:.0f} MB of K/V read per decode, "
                    f"{pool_bytes / 1e6:.0f} MB pool, L2 126 MB; no flush"),
@@ -777,6 +771,19 @@ def cpu_baseline(case, seconds: float, st):
             "affinity_cores": cores}
 
 
+def workload_config(args, case, world, fp8):
+    """The keys of a result's config that name the workload (both arms)."""
+    return {
+        "workload": f"{args.workload}: {case.workload.description}",
+        "num_seqs": case.num_seqs, "num_q_heads": case.num_q_heads,
+        "num_kv_heads": case.num_kv_heads, "head_dim": case.head_dim,
+        "block_size": case.block_size, "storage_dtype": gen.DTYPE_NAMES[case.dtype],
+        "query_tokens": args.query_tokens,
+        "kv_cache": "e4m3 codes + per-kv-head fp32 scales" if fp8 else gen.DTYPE_NAMES[case.dtype],
+        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+    }
+
+
 def run_reference(args, rank, world):
     """The oracle as the reference arm: each step decodes a bounded sample."""
     import oracle
@@ -803,7 +810,7 @@ def run_reference(args, rank, world):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1e3 * tot_t / args.steps, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{args.workload}: {case.workload.description}"},
+            "config": workload_config(args, case, world, False),
             "impl": "reference",
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
                              "kind": "oracle", "sample": sample},
